@@ -1,0 +1,725 @@
+/*
+ * kvc_oracle.c — plain, slow CPU oracle of the FastKVComp-style KV-cache codec.
+ *
+ * TEST INFRASTRUCTURE: only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg use this file. It shares no code with the CUDA library.
+ *
+ * Each function states the passage or reading it follows. The pages used:
+ *   [P2] "Beyond Compression Ratio: High-Throughput KV Compression for
+ *        Disaggregated LLM Serving" (arxivlens), Abstract and Methodology:
+ *        distribution transformation and low-bit quantization fused, no
+ *        intermediate tensor; LC-style lossless backend built from composable
+ *        primitives.
+ *   [P3] "FastKVComp: checking whether high-throughput KV compression pays
+ *        off" (podcast), episode notes: the pipeline is a randomized Hadamard
+ *        transform, low-bit quantization and a lossless codec; only the
+ *        quantization loses information; the cache crosses a link to a decode
+ *        GPU, so a decoder inverts the pipeline.
+ * The stage list comes from the pages; the exact rules are readings R1..R12
+ * (named at each function) chosen as the plainest definitions the pages admit.
+ *
+ * Build: gcc -std=c11 -O2 -ffp-contract=off -fno-fast-math (no FMA fusion, no
+ * excess precision: x86-64 SSE evaluates float in float).
+ */
+#include "kvc_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ========================================================================== */
+/* Sign generator. Reading R3: one +-1 diagonal over head_dim for the whole   */
+/* tensor ("randomized" Hadamard, [P3]). Its bits are the outputs of          */
+/* SplitMix64 (Steele, Lea, Flood, "Fast splittable pseudorandom number       */
+/* generators", OOPSLA 2014) started from state = sign_seed; channel c is     */
+/* negated iff bit (c mod 64) of output number floor(c/64) is 1.              */
+/* ========================================================================== */
+uint64_t orc_splitmix64_next(uint64_t *state) {
+  uint64_t z;
+  *state += 0x9E3779B97F4A7C15ull; /* golden-ratio increment */
+  z = *state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+void orc_sign_words(uint64_t seed, int d, uint64_t *words) {
+  uint64_t state = seed;
+  int i;
+  for (i = 0; i < (d + 63) / 64; i++) words[i] = orc_splitmix64_next(&state);
+}
+
+static int sign_bit(const uint64_t *words, int c) {
+  return (int)((words[c / 64] >> (c % 64)) & 1u);
+}
+
+/* ========================================================================== */
+/* Walsh-Hadamard transform ([P3] "randomized Hadamard transform").           */
+/* Reading R1: unnormalized, y = H_d x with the Sylvester matrix H_d.         */
+/* Reading R2: the butterfly order is normative because fp32 sums round:      */
+/* strides h = 1, 2, 4, ..., d/2 in ascending order; within a stride every    */
+/* pair (i, i+h) with (i & h) == 0 becomes (a+b, a-b), one rounding each.     */
+/* ========================================================================== */
+void orc_fwht(float *y, int d) {
+  int h, i;
+  for (h = 1; h < d; h *= 2) {
+    for (i = 0; i < d; i++) {
+      if ((i & h) == 0) {
+        float a = y[i];
+        float b = y[i + h];
+        y[i] = a + b;
+        y[i + h] = a - b;
+      }
+    }
+  }
+}
+
+/* Reading R4: the meta is stored divided by 2^k, k = floor(log2(d)/2), so that
+ * it sits in the range of the orthonormal transform (|H x| ~ sqrt(d)|x|). */
+int orc_meta_shift(int d) {
+  int l = 0;
+  while ((1 << l) < d) l++;
+  return l / 2;
+}
+
+/* ========================================================================== */
+/* Number formats.                                                            */
+/* ========================================================================== */
+float orc_bf16_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16; /* bf16 is the top half of an fp32 */
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* fp32 -> bf16, round to nearest, ties to even (decoded output, reading R9). */
+uint16_t orc_f32_to_bf16_rne(float x) {
+  uint32_t u;
+  memcpy(&u, &x, 4);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x0040u);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+/* fp16 (IEEE binary16) -> fp32, exact. */
+float orc_f16_to_f32(uint16_t h) {
+  int s = h >> 15, e = (h >> 10) & 31, m = h & 1023;
+  double v;
+  if (e == 31) {
+    if (m) return NAN;
+    return s ? -INFINITY : INFINITY;
+  }
+  if (e == 0)
+    v = ldexp((double)m, -24);
+  else
+    v = ldexp((double)(1024 + m), e - 25);
+  return (float)(s ? -v : v);
+}
+
+/* Encodes a non-negative value that already lies on the binary16 grid. */
+static uint16_t f16_bits_of_grid_value(double r) {
+  int e2;
+  if (r < ldexp(1.0, -14)) return (uint16_t)ldexp(r, 24); /* subnormal */
+  frexp(r, &e2);                                           /* r in [2^(e2-1), 2^e2) */
+  return (uint16_t)(((e2 - 1 + 15) << 10) |
+                    (int)ldexp(ldexp(r, -(e2 - 1)) - 1.0, 10));
+}
+
+/* fp32 -> fp16 with a directed rounding. The exact value of x is taken in
+ * double, scaled by the quantum of its binary16 binade (exact), rounded to an
+ * integer toward or away from zero, and scaled back. toward_neg = 1 rounds
+ * toward -inf (RD), 0 toward +inf (RU). */
+static uint16_t f32_to_f16_directed(float x, int toward_neg) {
+  int neg, away, e, E, qexp;
+  double a, q, n, r;
+  uint16_t sgn;
+  if (isnan(x)) return 0x7E00;
+  neg = signbit(x) ? 1 : 0;
+  sgn = (uint16_t)(neg << 15);
+  if (isinf(x)) return (uint16_t)(sgn | 0x7C00);
+  a = fabs((double)x);
+  if (a == 0.0) return sgn;
+  away = toward_neg ? neg : !neg; /* magnitude grows for RD<0 and RU>0 */
+  frexp(a, &e);
+  E = e - 1;                              /* a in [2^E, 2^(E+1)) */
+  qexp = (E < -14) ? -24 : E - 10;        /* spacing of the binade */
+  q = ldexp(a, -qexp);
+  n = away ? ceil(q) : floor(q);
+  r = ldexp(n, qexp);
+  if (r > 65504.0) return (uint16_t)(sgn | (away ? 0x7C00 : 0x7BFF));
+  if (r == 0.0) return sgn;
+  return (uint16_t)(sgn | f16_bits_of_grid_value(r));
+}
+
+uint16_t orc_f32_to_f16_rd(float x) { return f32_to_f16_directed(x, 1); }
+uint16_t orc_f32_to_f16_ru(float x) { return f32_to_f16_directed(x, 0); }
+
+static int f16_is_inf(uint16_t h) { return (h & 0x7FFFu) == 0x7C00u; }
+
+/* ========================================================================== */
+/* Code packing. Reading R6: codes of one vector in channel order, LSB first: */
+/* 4-bit: byte j = q[2j] | q[2j+1] << 4;                                      */
+/* 2-bit: byte j = q[4j] | q[4j+1] << 2 | q[4j+2] << 4 | q[4j+3] << 6.        */
+/* ========================================================================== */
+void orc_pack_codes(const uint8_t *q, int d, int bits, uint8_t *packed) {
+  int per = 8 / bits, j, i;
+  for (j = 0; j < d / per; j++) {
+    uint8_t b = 0;
+    for (i = 0; i < per; i++) b = (uint8_t)(b | (q[j * per + i] << (i * bits)));
+    packed[j] = b;
+  }
+}
+
+void orc_unpack_codes(const uint8_t *packed, int d, int bits, uint8_t *q) {
+  int per = 8 / bits, c;
+  uint8_t mask = (uint8_t)((1 << bits) - 1);
+  for (c = 0; c < d; c++)
+    q[c] = (uint8_t)((packed[c / per] >> ((c % per) * bits)) & mask);
+}
+
+/* ========================================================================== */
+/* Quantization of one vector ([P2] Methodology: distribution transformation  */
+/* then low-bit quantization; [P3]: only this step loses information).        */
+/* Reading R5 (asymmetric min/max group quantization with fp16 meta):         */
+/*   groups are g consecutive channels of the transformed vector y;           */
+/*   mn, mx = group min and max, then mn+0, mx+0 (so -0 becomes +0);          */
+/*   z_h = RD16(mn * 2^-k),  zf = f32(z_h) * 2^k;                             */
+/*   s32 = (mx - zf) / (2^b - 1),  s_h = RU16(s32 * 2^-k), sf = f32(s_h)*2^k; */
+/*   r = 0 if s_h == 0 else 1/sf;                                             */
+/*   q = clamp(RNE((y - zf) * r), 0, 2^b - 1).                                */
+/* Directed rounding makes the grid zf + q*sf cover [mn, mx]. A non-finite y  */
+/* gives NONFINITE; an infinite z_h or s_h gives RANGE (reading R8). The meta */
+/* of group j is 4 bytes: s_h then z_h, little-endian.                        */
+/* ========================================================================== */
+int orc_quantize_vector(const uint16_t *x, int d, int bits, int g,
+                        const uint64_t *sign_words, uint8_t *codes,
+                        uint8_t *meta) {
+  float y[ORC_MAX_D];
+  uint8_t q[ORC_MAX_D];
+  int k = orc_meta_shift(d);
+  float up = ldexpf(1.0f, k), down = ldexpf(1.0f, -k);
+  int qmax = (1 << bits) - 1;
+  int status = ORC_OK;
+  int c, j;
+
+  for (c = 0; c < d; c++) {
+    y[c] = orc_bf16_to_f32(x[c]);
+    if (sign_bit(sign_words, c)) y[c] = -y[c];
+  }
+  orc_fwht(y, d);
+
+  for (j = 0; j < d / g; j++) {
+    const float *yg = y + j * g;
+    float mn = yg[0], mx = yg[0], zf, s32, sf, r;
+    uint16_t zh, sh;
+    int finite = 1;
+    for (c = 0; c < g; c++) {
+      if (!isfinite(yg[c])) finite = 0;
+      if (yg[c] < mn) mn = yg[c];
+      if (yg[c] > mx) mx = yg[c];
+    }
+    if (!finite) {
+      status = ORC_ERR_NONFINITE;
+      for (c = 0; c < g; c++) q[j * g + c] = 0;
+      memset(meta + 4 * j, 0, 4);
+      continue;
+    }
+    mn = mn + 0.0f;
+    mx = mx + 0.0f;
+    zh = orc_f32_to_f16_rd(mn * down);
+    zf = orc_f16_to_f32(zh) * up;
+    s32 = (mx - zf) / (float)qmax;
+    sh = orc_f32_to_f16_ru(s32 * down);
+    sf = orc_f16_to_f32(sh) * up;
+    if (f16_is_inf(zh) || f16_is_inf(sh)) {
+      if (status == ORC_OK) status = ORC_ERR_RANGE;
+      for (c = 0; c < g; c++) q[j * g + c] = 0;
+    } else {
+      r = ((sh & 0x7FFFu) == 0) ? 0.0f : 1.0f / sf;
+      for (c = 0; c < g; c++) {
+        float t = (yg[c] - zf) * r;
+        float n = nearbyintf(t); /* default mode: nearest, ties to even */
+        if (n < 0.0f) n = 0.0f;
+        if (n > (float)qmax) n = (float)qmax;
+        q[j * g + c] = (uint8_t)n;
+      }
+    }
+    meta[4 * j + 0] = (uint8_t)(sh & 0xFF);
+    meta[4 * j + 1] = (uint8_t)(sh >> 8);
+    meta[4 * j + 2] = (uint8_t)(zh & 0xFF);
+    meta[4 * j + 3] = (uint8_t)(zh >> 8);
+  }
+  orc_pack_codes(q, d, bits, codes);
+  return status;
+}
+
+/* Decode of one vector, the inverse path of [P3]. Reading R9:
+ *   y^ = zf + q*sf (the product rounded, then the sum rounded);
+ *   the same butterfly as the encoder (H_d H_d = d I);
+ *   x^ = bf16_RNE(sign_c * (u * 2^-log2(d))). */
+void orc_dequantize_vector(const uint8_t *codes, const uint8_t *meta, int d,
+                           int bits, int g, const uint64_t *sign_words,
+                           uint16_t *xhat) {
+  float y[ORC_MAX_D];
+  uint8_t q[ORC_MAX_D];
+  int k = orc_meta_shift(d), l2d = 0, c, j;
+  float up = ldexpf(1.0f, k), inv_d;
+  while ((1 << l2d) < d) l2d++;
+  inv_d = ldexpf(1.0f, -l2d);
+  orc_unpack_codes(codes, d, bits, q);
+  for (j = 0; j < d / g; j++) {
+    uint16_t sh = (uint16_t)(meta[4 * j] | (meta[4 * j + 1] << 8));
+    uint16_t zh = (uint16_t)(meta[4 * j + 2] | (meta[4 * j + 3] << 8));
+    float sf = orc_f16_to_f32(sh) * up;
+    float zf = orc_f16_to_f32(zh) * up;
+    for (c = j * g; c < (j + 1) * g; c++) {
+      float p = (float)q[c] * sf;
+      y[c] = zf + p;
+    }
+  }
+  orc_fwht(y, d);
+  for (c = 0; c < d; c++) {
+    float u = y[c] * inv_d;
+    if (sign_bit(sign_words, c)) u = -u;
+    xhat[c] = orc_f32_to_bf16_rne(u);
+  }
+}
+
+/* ========================================================================== */
+/* Lossless stage on one 16 KB chunk ([P2]: LC-style backend composed of      */
+/* primitives). The components are a bit-plane shuffle, zero-byte            */
+/* elimination with a bitmap, and a prefix sum over chunk sizes.              */
+/* Reading R10: the chunk is 4096 little-endian u32 words w[j]; plane p       */
+/* (p = 0..31, LSB first) is 512 bytes; bit (j mod 8) of byte p*512 + j/8 of  */
+/* the output is bit p of w[j]. Only full 16 KB chunks are shuffled.          */
+/* ========================================================================== */
+static uint32_t word_at(const uint8_t *b, int j) {
+  return (uint32_t)b[4 * j] | ((uint32_t)b[4 * j + 1] << 8) |
+         ((uint32_t)b[4 * j + 2] << 16) | ((uint32_t)b[4 * j + 3] << 24);
+}
+
+void orc_bitplane_shuffle(const uint8_t *in, uint8_t *out) {
+  int p, j;
+  memset(out, 0, ORC_CHUNK);
+  for (j = 0; j < ORC_CHUNK / 4; j++) {
+    uint32_t w = word_at(in, j);
+    for (p = 0; p < 32; p++)
+      if ((w >> p) & 1u) out[p * 512 + j / 8] |= (uint8_t)(1u << (j % 8));
+  }
+}
+
+void orc_bitplane_unshuffle(const uint8_t *in, uint8_t *out) {
+  int p, j;
+  for (j = 0; j < ORC_CHUNK / 4; j++) {
+    uint32_t w = 0;
+    for (p = 0; p < 32; p++)
+      if ((in[p * 512 + j / 8] >> (j % 8)) & 1u) w |= 1u << p;
+    out[4 * j] = (uint8_t)w;
+    out[4 * j + 1] = (uint8_t)(w >> 8);
+    out[4 * j + 2] = (uint8_t)(w >> 16);
+    out[4 * j + 3] = (uint8_t)(w >> 24);
+  }
+}
+
+/* Reading R11: zero-byte elimination writes a 2048-byte bitmap (bit i, LSB
+ * first, says shuffled byte i is nonzero) followed by the nonzero bytes in
+ * order. It is used only if strictly shorter than the chunk; otherwise the
+ * chunk is stored raw, as the original unshuffled bytes. A short chunk (the
+ * tail of a region) is always raw. The decoder tells the two apart by size:
+ * size == chunk length means raw. Returns the encoded size. */
+uint32_t orc_lossless_encode_chunk(const uint8_t *in, uint32_t len,
+                                   uint8_t *out) {
+  uint8_t s[ORC_CHUNK];
+  uint32_t nnz = 0, i;
+  if (len < ORC_CHUNK) {
+    memcpy(out, in, len);
+    return len;
+  }
+  orc_bitplane_shuffle(in, s);
+  for (i = 0; i < ORC_CHUNK; i++)
+    if (s[i]) nnz++;
+  if (ORC_BITMAP + nnz >= ORC_CHUNK) {
+    memcpy(out, in, ORC_CHUNK);
+    return ORC_CHUNK;
+  }
+  memset(out, 0, ORC_BITMAP);
+  nnz = 0;
+  for (i = 0; i < ORC_CHUNK; i++) {
+    if (s[i]) {
+      out[i / 8] |= (uint8_t)(1u << (i % 8));
+      out[ORC_BITMAP + nnz] = s[i];
+      nnz++;
+    }
+  }
+  return ORC_BITMAP + nnz;
+}
+
+int orc_lossless_decode_chunk(const uint8_t *in, uint32_t size, uint32_t len,
+                              uint8_t *out) {
+  uint8_t s[ORC_CHUNK];
+  uint32_t i, pos = 0;
+  if (size == len) {
+    memcpy(out, in, len);
+    return ORC_OK;
+  }
+  if (len != ORC_CHUNK || size < ORC_BITMAP || size >= ORC_CHUNK)
+    return ORC_ERR_CORRUPT;
+  for (i = 0; i < ORC_CHUNK; i++) {
+    if ((in[i / 8] >> (i % 8)) & 1u) {
+      if (ORC_BITMAP + pos >= size) return ORC_ERR_CORRUPT;
+      s[i] = in[ORC_BITMAP + pos];
+      pos++;
+    } else {
+      s[i] = 0;
+    }
+  }
+  if (ORC_BITMAP + pos != size) return ORC_ERR_CORRUPT;
+  orc_bitplane_unshuffle(s, out);
+  return ORC_OK;
+}
+
+/* ========================================================================== */
+/* Stream layout. Reading R12 (self-describing stream, little-endian):        */
+/*   [0,64)    header: u32 magic "KVC1", u16 version 1, u16 header bytes 64,  */
+/*             u8 bits, u8 k, u8 origin (0 dense, 1 paged), u8 0, u32 group,  */
+/*             u32 layers, u32 kv (=2), u32 kv_heads, u32 head_dim,           */
+/*             u64 tokens (sum over requests), u64 sign_seed,                 */
+/*             u32 n_requests, u32 n_chunks, u64 stream_bytes;                */
+/*   then      u64 chunk table [n_chunks]: bits 0..15 = unpadded size,        */
+/*             bits 16..63 = offset from the data base in 16-byte units;      */
+/*   then      u32 token lengths [n_requests];                                */
+/*   then      zeros up to a 16-byte boundary = data base;                    */
+/*   then      the chunks, each zero-padded to 16 bytes, at their offsets.    */
+/* The codes region (packed codes of all vectors in logical order) and the    */
+/* meta region (4 bytes per group) are cut into 16 KB chunks separately. A    */
+/* meta chunk covers R = g*b/32 code chunks; stream order is segment by       */
+/* segment: the R code chunks of a segment, then its meta chunk. Chunk        */
+/* offsets are the exclusive prefix sum of the padded chunk sizes.            */
+/* ========================================================================== */
+static uint64_t round16(uint64_t x) { return (x + 15u) & ~(uint64_t)15u; }
+
+int orc_check_desc(const orc_desc *d) {
+  int r;
+  if (!d) return ORC_ERR_INVALID_ARG;
+  if (d->bits != 2 && d->bits != 4) return ORC_ERR_UNSUPPORTED;
+  if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256)
+    return ORC_ERR_UNSUPPORTED;
+  if (d->group != 32 && d->group != 64 && d->group != 128)
+    return ORC_ERR_UNSUPPORTED;
+  if (d->group > d->head_dim) return ORC_ERR_UNSUPPORTED;
+  if (d->layers < 0 || d->kv_heads < 0 || d->n_requests < 0)
+    return ORC_ERR_INVALID_ARG;
+  if (d->n_requests > 0 && !d->token_lens) return ORC_ERR_INVALID_ARG;
+  for (r = 0; r < d->n_requests; r++)
+    if (d->token_lens[r] > 0x7FFFFFFFu) return ORC_ERR_INVALID_ARG;
+  return ORC_OK;
+}
+
+int orc_layout_of(const orc_desc *d, orc_layout *lay) {
+  uint64_t T = 0, i;
+  int st = orc_check_desc(d), r;
+  if (st != ORC_OK) return st;
+  for (r = 0; r < d->n_requests; r++) T += d->token_lens[r];
+  lay->V = (uint64_t)d->layers * 2u * (uint64_t)d->kv_heads * T;
+  lay->code_bytes = (uint32_t)(d->head_dim * d->bits / 8);
+  lay->meta_bytes = (uint32_t)((d->head_dim / d->group) * 4);
+  lay->vec_per_code = ORC_CHUNK / lay->code_bytes;
+  lay->code_per_seg = (uint32_t)(d->group * d->bits / 32);
+  lay->n_code = (lay->V + lay->vec_per_code - 1) / lay->vec_per_code;
+  lay->n_seg = (lay->n_code + lay->code_per_seg - 1) / lay->code_per_seg;
+  lay->n_meta = lay->n_seg;
+  lay->n_chunks = lay->n_code + lay->n_meta;
+  lay->data_base =
+      round16(ORC_HEADER + 8u * lay->n_chunks + 4u * (uint64_t)d->n_requests);
+  lay->max_bytes = lay->data_base;
+  /* every chunk at its raw length, padded */
+  for (i = 0; i < lay->n_code; i++) {
+    uint64_t v0 = i * lay->vec_per_code;
+    uint64_t nv = lay->V - v0 < lay->vec_per_code ? lay->V - v0 : lay->vec_per_code;
+    lay->max_bytes += round16(nv * lay->code_bytes);
+  }
+  for (i = 0; i < lay->n_meta; i++) {
+    uint64_t vm = (uint64_t)lay->vec_per_code * lay->code_per_seg;
+    uint64_t v0 = i * vm;
+    uint64_t nv = lay->V - v0 < vm ? lay->V - v0 : vm;
+    lay->max_bytes += round16(nv * lay->meta_bytes);
+  }
+  return ORC_OK;
+}
+
+uint64_t orc_max_compressed_bytes(const orc_desc *d) {
+  orc_layout lay;
+  if (orc_layout_of(d, &lay) != ORC_OK) return 0;
+  return lay.max_bytes;
+}
+
+uint64_t orc_code_chunk_index(const orc_layout *lay, uint64_t c) {
+  return c + c / lay->code_per_seg;
+}
+
+uint64_t orc_meta_chunk_index(const orc_layout *lay, uint64_t s) {
+  uint64_t end = (s + 1) * lay->code_per_seg;
+  if (end > lay->n_code) end = lay->n_code;
+  return end + s;
+}
+
+static void put16(uint8_t *p, uint16_t v) {
+  p[0] = (uint8_t)v;
+  p[1] = (uint8_t)(v >> 8);
+}
+static void put32(uint8_t *p, uint32_t v) {
+  int i;
+  for (i = 0; i < 4; i++) p[i] = (uint8_t)(v >> (8 * i));
+}
+static void put64(uint8_t *p, uint64_t v) {
+  int i;
+  for (i = 0; i < 8; i++) p[i] = (uint8_t)(v >> (8 * i));
+}
+static uint16_t get16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+static uint32_t get32(const uint8_t *p) {
+  return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) |
+         ((uint32_t)p[3] << 24);
+}
+static uint64_t get64(const uint8_t *p) {
+  return (uint64_t)get32(p) | ((uint64_t)get32(p + 4) << 32);
+}
+
+int orc_encode_segment(const orc_desc *d, uint64_t s, const uint16_t *vectors,
+                       uint8_t *chunks, uint32_t *sizes, uint32_t *n_out) {
+  orc_layout lay;
+  uint64_t vm, v0, nv, v, c0, c1, c;
+  uint8_t *codes, *meta;
+  uint64_t sw[4];
+  uint32_t pos = 0;
+  int st = orc_layout_of(d, &lay), vst;
+  if (st != ORC_OK) return st;
+  if (s >= lay.n_seg) return ORC_ERR_INVALID_ARG;
+  vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
+  v0 = s * vm;
+  nv = lay.V - v0 < vm ? lay.V - v0 : vm;
+  orc_sign_words(d->sign_seed, d->head_dim, sw);
+  codes = (uint8_t *)malloc((size_t)(nv * lay.code_bytes));
+  meta = (uint8_t *)malloc((size_t)(nv * lay.meta_bytes));
+  for (v = 0; v < nv; v++) {
+    vst = orc_quantize_vector(vectors + v * d->head_dim, d->head_dim, d->bits,
+                              d->group, sw, codes + v * lay.code_bytes,
+                              meta + v * lay.meta_bytes);
+    if (vst != ORC_OK && st == ORC_OK) st = vst;
+  }
+  c0 = s * lay.code_per_seg;
+  c1 = c0 + lay.code_per_seg < lay.n_code ? c0 + lay.code_per_seg : lay.n_code;
+  *n_out = 0;
+  for (c = c0; c < c1; c++) {
+    uint64_t a = (c - c0) * lay.vec_per_code;
+    uint64_t b = a + lay.vec_per_code < nv ? a + lay.vec_per_code : nv;
+    uint32_t sz = orc_lossless_encode_chunk(
+        codes + a * lay.code_bytes, (uint32_t)((b - a) * lay.code_bytes),
+        chunks + pos);
+    sizes[(*n_out)++] = sz;
+    pos += sz;
+  }
+  sizes[(*n_out)++] =
+      orc_lossless_encode_chunk(meta, (uint32_t)(nv * lay.meta_bytes), chunks + pos);
+  free(codes);
+  free(meta);
+  return st;
+}
+
+int orc_decode_segment(const orc_desc *d, uint64_t s, const uint8_t *chunks,
+                       const uint32_t *sizes, uint16_t *vectors) {
+  orc_layout lay;
+  uint64_t vm, v0, nv, v, c0, c1, c, i = 0;
+  uint8_t *codes, *meta;
+  uint64_t sw[4];
+  uint32_t pos = 0;
+  int st = orc_layout_of(d, &lay);
+  if (st != ORC_OK) return st;
+  if (s >= lay.n_seg) return ORC_ERR_INVALID_ARG;
+  vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
+  v0 = s * vm;
+  nv = lay.V - v0 < vm ? lay.V - v0 : vm;
+  orc_sign_words(d->sign_seed, d->head_dim, sw);
+  codes = (uint8_t *)malloc((size_t)(nv * lay.code_bytes));
+  meta = (uint8_t *)malloc((size_t)(nv * lay.meta_bytes));
+  c0 = s * lay.code_per_seg;
+  c1 = c0 + lay.code_per_seg < lay.n_code ? c0 + lay.code_per_seg : lay.n_code;
+  for (c = c0; c < c1 && st == ORC_OK; c++, i++) {
+    uint64_t a = (c - c0) * lay.vec_per_code;
+    uint64_t b = a + lay.vec_per_code < nv ? a + lay.vec_per_code : nv;
+    st = orc_lossless_decode_chunk(chunks + pos, sizes[i],
+                                   (uint32_t)((b - a) * lay.code_bytes),
+                                   codes + a * lay.code_bytes);
+    pos += sizes[i];
+  }
+  if (st == ORC_OK)
+    st = orc_lossless_decode_chunk(chunks + pos, sizes[i],
+                                   (uint32_t)(nv * lay.meta_bytes), meta);
+  if (st == ORC_OK)
+    for (v = 0; v < nv; v++)
+      orc_dequantize_vector(codes + v * lay.code_bytes, meta + v * lay.meta_bytes,
+                            d->head_dim, d->bits, d->group, sw,
+                            vectors + v * d->head_dim);
+  free(codes);
+  free(meta);
+  return st;
+}
+
+int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
+                 uint64_t capacity, uint64_t *out_bytes) {
+  orc_layout lay;
+  uint64_t s, off = 0, T = 0, vm;
+  uint8_t *seg;
+  uint32_t sizes[17], n, i;
+  int st = orc_layout_of(d, &lay), sst, r;
+  if (st != ORC_OK) return st;
+  if (capacity < lay.max_bytes) return ORC_ERR_CAPACITY;
+  for (r = 0; r < d->n_requests; r++) T += d->token_lens[r];
+  memset(out, 0, (size_t)lay.data_base);
+  put32(out + 0, ORC_MAGIC);
+  put16(out + 4, 1);
+  put16(out + 6, ORC_HEADER);
+  out[8] = (uint8_t)d->bits;
+  out[9] = (uint8_t)orc_meta_shift(d->head_dim);
+  out[10] = (uint8_t)d->origin;
+  out[11] = 0;
+  put32(out + 12, (uint32_t)d->group);
+  put32(out + 16, (uint32_t)d->layers);
+  put32(out + 20, 2);
+  put32(out + 24, (uint32_t)d->kv_heads);
+  put32(out + 28, (uint32_t)d->head_dim);
+  put64(out + 32, T);
+  put64(out + 40, d->sign_seed);
+  put32(out + 48, (uint32_t)d->n_requests);
+  put32(out + 52, (uint32_t)lay.n_chunks);
+  for (r = 0; r < d->n_requests; r++)
+    put32(out + ORC_HEADER + 8 * lay.n_chunks + 4 * r, d->token_lens[r]);
+  vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
+  seg = (uint8_t *)malloc((size_t)(lay.code_per_seg + 1) * ORC_CHUNK);
+  for (s = 0; s < lay.n_seg; s++) {
+    uint64_t first = orc_code_chunk_index(&lay, s * lay.code_per_seg);
+    uint32_t pos = 0;
+    sst = orc_encode_segment(d, s, vectors + s * vm * d->head_dim, seg, sizes, &n);
+    if (sst != ORC_OK && st == ORC_OK) st = sst;
+    for (i = 0; i < n; i++) {
+      uint64_t padded = round16(sizes[i]);
+      put64(out + ORC_HEADER + 8 * (first + i), ((off / 16) << 16) | sizes[i]);
+      memset(out + lay.data_base + off, 0, (size_t)padded);
+      memcpy(out + lay.data_base + off, seg + pos, sizes[i]);
+      pos += sizes[i];
+      off += padded;
+    }
+  }
+  free(seg);
+  put64(out + 56, lay.data_base + off);
+  *out_bytes = lay.data_base + off;
+  return st;
+}
+
+int orc_decompress(const uint8_t *stream, uint64_t stream_bytes,
+                   const orc_desc *expect, uint16_t *vectors) {
+  orc_layout lay;
+  uint64_t s, T = 0, vm, expect_off = 0, total;
+  uint8_t *seg;
+  uint32_t sizes[17];
+  int st = orc_layout_of(expect, &lay), r;
+  if (st != ORC_OK) return st;
+  if (stream_bytes < ORC_HEADER) return ORC_ERR_CORRUPT;
+  for (r = 0; r < expect->n_requests; r++) T += expect->token_lens[r];
+  if (get32(stream) != ORC_MAGIC || get16(stream + 4) != 1 ||
+      get16(stream + 6) != ORC_HEADER || stream[8] != expect->bits ||
+      stream[9] != orc_meta_shift(expect->head_dim) ||
+      get32(stream + 12) != (uint32_t)expect->group ||
+      get32(stream + 16) != (uint32_t)expect->layers || get32(stream + 20) != 2 ||
+      get32(stream + 24) != (uint32_t)expect->kv_heads ||
+      get32(stream + 28) != (uint32_t)expect->head_dim || get64(stream + 32) != T ||
+      get64(stream + 40) != expect->sign_seed ||
+      get32(stream + 48) != (uint32_t)expect->n_requests ||
+      get32(stream + 52) != lay.n_chunks)
+    return ORC_ERR_CORRUPT;
+  total = get64(stream + 56);
+  if (total > stream_bytes || total < lay.data_base) return ORC_ERR_CORRUPT;
+  for (r = 0; r < expect->n_requests; r++)
+    if (get32(stream + ORC_HEADER + 8 * lay.n_chunks + 4 * r) !=
+        expect->token_lens[r])
+      return ORC_ERR_CORRUPT;
+  vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
+  seg = (uint8_t *)malloc((size_t)(lay.code_per_seg + 1) * ORC_CHUNK);
+  for (s = 0; s < lay.n_seg && st == ORC_OK; s++) {
+    uint64_t first = orc_code_chunk_index(&lay, s * lay.code_per_seg);
+    uint64_t last = orc_meta_chunk_index(&lay, s);
+    uint64_t i;
+    uint32_t pos = 0;
+    for (i = first; i <= last; i++) {
+      uint64_t e = get64(stream + ORC_HEADER + 8 * i);
+      uint32_t sz = (uint32_t)(e & 0xFFFFu);
+      uint64_t off = (e >> 16) * 16;
+      if (off != expect_off || sz > ORC_CHUNK ||
+          lay.data_base + off + round16(sz) > total) {
+        st = ORC_ERR_CORRUPT;
+        break;
+      }
+      memcpy(seg + pos, stream + lay.data_base + off, sz);
+      sizes[i - first] = sz;
+      pos += sz;
+      expect_off = off + round16(sz);
+    }
+    if (st == ORC_OK)
+      st = orc_decode_segment(expect, s, seg, sizes,
+                              vectors + s * vm * expect->head_dim);
+  }
+  free(seg);
+  if (st == ORC_OK && lay.data_base + expect_off != total) st = ORC_ERR_CORRUPT;
+  return st;
+}
+
+/* ========================================================================== */
+/* Logical vector order [layer][kv][head][request][token]; requests are       */
+/* concatenated along tokens. Dense input: one request of `tokens` tokens.   */
+/* Strides are in elements; head_dim is contiguous.                           */
+/* ========================================================================== */
+void orc_gather_dense(const uint16_t *base, int layers, int kv_heads,
+                      int64_t tokens, int d, int64_t s_layer, int64_t s_kv,
+                      int64_t s_head, int64_t s_token, uint64_t v_begin,
+                      uint64_t v_end, uint16_t *out) {
+  uint64_t v;
+  (void)layers;
+  for (v = v_begin; v < v_end; v++) {
+    int64_t t = (int64_t)(v % (uint64_t)tokens);
+    uint64_t lkh = v / (uint64_t)tokens;
+    int64_t h = (int64_t)(lkh % (uint64_t)kv_heads);
+    int64_t kv = (int64_t)((lkh / (uint64_t)kv_heads) % 2u);
+    int64_t l = (int64_t)(lkh / (uint64_t)kv_heads / 2u);
+    const uint16_t *src = base + l * s_layer + kv * s_kv + h * s_head + t * s_token;
+    memcpy(out + (v - v_begin) * (uint64_t)d, src, (size_t)d * 2u);
+  }
+}
+
+void orc_gather_paged(const uint16_t *pool, int layers, int kv_heads, int d,
+                      int64_t s_layer, int64_t s_page, int64_t s_kv,
+                      int64_t s_head, int64_t s_slot, int page_tokens,
+                      int n_requests, const uint32_t *seq_lens,
+                      const int32_t *page_table, int64_t pt_stride,
+                      uint64_t v_begin, uint64_t v_end, uint16_t *out) {
+  uint64_t v, T = 0;
+  int r;
+  (void)layers;
+  for (r = 0; r < n_requests; r++) T += seq_lens[r];
+  for (v = v_begin; v < v_end; v++) {
+    uint64_t u = v % T, lkh = v / T;
+    int64_t h = (int64_t)(lkh % (uint64_t)kv_heads);
+    int64_t kv = (int64_t)((lkh / (uint64_t)kv_heads) % 2u);
+    int64_t l = (int64_t)(lkh / (uint64_t)kv_heads / 2u);
+    int64_t t, page;
+    const uint16_t *src;
+    r = 0;
+    while (u >= seq_lens[r]) {
+      u -= seq_lens[r];
+      r++;
+    }
+    t = (int64_t)u;
+    page = page_table[(int64_t)r * pt_stride + t / page_tokens];
+    src = pool + l * s_layer + page * s_page + kv * s_kv + h * s_head +
+          (t % page_tokens) * s_slot;
+    memcpy(out + (v - v_begin) * (uint64_t)d, src, (size_t)d * 2u);
+  }
+}

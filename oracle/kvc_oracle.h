@@ -1,0 +1,136 @@
+/*
+ * kvc_oracle.h — plain, slow CPU oracle of the FastKVComp-style KV-cache codec.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package entry's smoke check and
+ * the benchmark's CPU-baseline leg may call, link or execute this code. The
+ * product path (the CUDA library) never uses it, and the two share no code:
+ * every definition below is written independently of the CUDA sources.
+ *
+ * What it computes (sources: "Beyond Compression Ratio: High-Throughput KV
+ * Compression for Disaggregated LLM Serving", Abstract and Methodology; the
+ * podcast page "FastKVComp: checking whether high-throughput KV compression
+ * pays off", episode notes):
+ *   encode = random +-1 signs, Hadamard transform over head_dim, low-bit group
+ *            quantization, then a lossless codec over the quantized payload;
+ *   decode = the exact inverse of the lossless codec, then dequantization,
+ *            inverse Hadamard and unsigning.
+ * The pages name the stages only. Every exact rule here (butterfly order, sign
+ * generator, meta rounding, stream format) is a stated reading, listed in the
+ * design notes with its justification.
+ *
+ * Floating point: the method's arithmetic is fp32 with one IEEE rounding per
+ * operation (no fused multiply-add). Build with -ffp-contract=off
+ * -fno-fast-math. Status codes use the same numbering as the library ABI.
+ */
+#ifndef KVC_ORACLE_H
+#define KVC_ORACLE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  ORC_OK = 0,
+  ORC_ERR_INVALID_ARG = 1,
+  ORC_ERR_UNSUPPORTED = 2,
+  ORC_ERR_CAPACITY = 3,
+  ORC_ERR_NONFINITE = 4,
+  ORC_ERR_RANGE = 5,
+  ORC_ERR_CORRUPT = 6
+};
+
+#define ORC_CHUNK 16384      /* lossless chunk length in bytes            */
+#define ORC_BITMAP 2048      /* zero-byte-elimination bitmap bytes        */
+#define ORC_HEADER 64        /* stream header bytes                       */
+#define ORC_MAGIC 0x3143564Bu /* "KVC1" little-endian                    */
+#define ORC_MAX_D 256
+
+/* ---- scalar building blocks (each pinned by its own test) ---------------- */
+uint64_t orc_splitmix64_next(uint64_t *state);
+void orc_sign_words(uint64_t seed, int d, uint64_t *words);
+void orc_fwht(float *y, int d);
+int orc_meta_shift(int d);
+float orc_bf16_to_f32(uint16_t b);
+uint16_t orc_f32_to_bf16_rne(float x);
+float orc_f16_to_f32(uint16_t h);
+uint16_t orc_f32_to_f16_rd(float x);
+uint16_t orc_f32_to_f16_ru(float x);
+
+/* ---- one vector ----------------------------------------------------------- */
+int orc_quantize_vector(const uint16_t *x, int d, int bits, int g,
+                        const uint64_t *sign_words, uint8_t *codes,
+                        uint8_t *meta);
+void orc_dequantize_vector(const uint8_t *codes, const uint8_t *meta, int d,
+                           int bits, int g, const uint64_t *sign_words,
+                           uint16_t *xhat);
+void orc_pack_codes(const uint8_t *q, int d, int bits, uint8_t *packed);
+void orc_unpack_codes(const uint8_t *packed, int d, int bits, uint8_t *q);
+
+/* ---- lossless stage on one chunk ------------------------------------------ */
+void orc_bitplane_shuffle(const uint8_t *in, uint8_t *out);
+void orc_bitplane_unshuffle(const uint8_t *in, uint8_t *out);
+uint32_t orc_lossless_encode_chunk(const uint8_t *in, uint32_t len,
+                                   uint8_t *out);
+int orc_lossless_decode_chunk(const uint8_t *in, uint32_t size, uint32_t len,
+                              uint8_t *out);
+
+/* ---- stream --------------------------------------------------------------- */
+typedef struct {
+  int32_t bits, group, head_dim, layers, kv_heads, origin, n_requests;
+  uint64_t sign_seed;
+  const uint32_t *token_lens; /* [n_requests] tokens per request          */
+} orc_desc;
+
+typedef struct {
+  uint64_t V;             /* vectors                                       */
+  uint32_t code_bytes;    /* packed code bytes per vector                  */
+  uint32_t meta_bytes;    /* meta bytes per vector                         */
+  uint32_t vec_per_code;  /* vectors per code chunk                        */
+  uint32_t code_per_seg;  /* code chunks per meta chunk (segment)          */
+  uint64_t n_code, n_meta, n_chunks, n_seg;
+  uint64_t data_base;     /* byte offset of the first chunk                */
+  uint64_t max_bytes;     /* worst-case stream length                      */
+} orc_layout;
+
+int orc_check_desc(const orc_desc *d);
+int orc_layout_of(const orc_desc *d, orc_layout *lay);
+uint64_t orc_max_compressed_bytes(const orc_desc *d);
+
+/* Stream chunk index of code chunk c and of meta chunk s. */
+uint64_t orc_code_chunk_index(const orc_layout *lay, uint64_t c);
+uint64_t orc_meta_chunk_index(const orc_layout *lay, uint64_t s);
+
+/* Encodes segment s from its vectors (vectors [s*VM, min((s+1)*VM, V)) in
+ * logical order, d bf16 each). Writes the segment's chunks, unpadded, back to
+ * back into chunks (capacity (code_per_seg+1)*ORC_CHUNK) and their sizes into
+ * sizes[] (code chunks first, then the meta chunk). Returns the status and the
+ * number of chunks through n_out. */
+int orc_encode_segment(const orc_desc *d, uint64_t s, const uint16_t *vectors,
+                       uint8_t *chunks, uint32_t *sizes, uint32_t *n_out);
+int orc_decode_segment(const orc_desc *d, uint64_t s, const uint8_t *chunks,
+                       const uint32_t *sizes, uint16_t *vectors);
+
+int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
+                 uint64_t capacity, uint64_t *out_bytes);
+int orc_decompress(const uint8_t *stream, uint64_t stream_bytes,
+                   const orc_desc *expect, uint16_t *vectors);
+
+/* ---- layouts: logical vector order [layer][kv][head][request][token] ------ */
+void orc_gather_dense(const uint16_t *base, int layers, int kv_heads,
+                      int64_t tokens, int d, int64_t s_layer, int64_t s_kv,
+                      int64_t s_head, int64_t s_token, uint64_t v_begin,
+                      uint64_t v_end, uint16_t *out);
+void orc_gather_paged(const uint16_t *pool, int layers, int kv_heads, int d,
+                      int64_t s_layer, int64_t s_page, int64_t s_kv,
+                      int64_t s_head, int64_t s_slot, int page_tokens,
+                      int n_requests, const uint32_t *seq_lens,
+                      const int32_t *page_table, int64_t pt_stride,
+                      uint64_t v_begin, uint64_t v_end, uint16_t *out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

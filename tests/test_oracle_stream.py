@@ -1,0 +1,186 @@
+"""Pins of the oracle's stream layer: the header against a hand-written golden,
+layout counts against hand arithmetic, the whole-codec error bound, corrupt
+streams, and the logical vector order of dense and paged gathers against
+independent numpy/torch indexing."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_compression_04_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _u(b, off, n):
+    return int.from_bytes(bytes(b[off:off + n]), "little")
+
+
+def tiny_desc_and_vectors():
+    w = synth.workload("tiny")
+    kv = synth.dense_kv(w)
+    x = synth.bf16_bits(kv).reshape(-1, w.head_dim)   # contiguous = logical order
+    d = oracle.StreamDesc(w.bits, w.group, w.head_dim, w.layers, w.kv_heads,
+                          [w.tokens], w.sign_seed)
+    return w, d, x
+
+
+def test_header_golden():
+    _, d, x = tiny_desc_and_vectors()
+    st, s = oracle.compress(d, x)
+    assert st == oracle.OK
+    rows = {}
+    with open(os.path.join(GOLDEN, "header_tiny.txt")) as f:
+        for l in f:
+            l = l.split("#")[0].split()
+            if l:
+                rows[l[0]] = l[1:]
+    for key, val in rows.items():
+        if key.isdigit():
+            assert _u(s, int(key), int(val[0])) == int(val[1], 0), key
+    lay = d.layout()
+    assert lay.data_base == int(rows["data_base"][0])
+    assert d.max_bytes() == int(rows["max_bytes"][0])
+    assert _u(s, 56, 8) == s.size                               # stream_bytes
+    assert _u(s, 64 + 8 * 5, 4) == 64                           # token length
+    assert not s[64 + 8 * 5 + 4:112].any()                      # zero padding
+
+
+@pytest.mark.parametrize("name,n_code,n_meta", [("tiny", 4, 1), ("llama8b", 8192, 512),
+                                                ("qwen7b", 14336, 7168)])
+def test_layout_counts(name, n_code, n_meta):
+    """Hand arithmetic: code chunks = V*d*b/8/16384, meta chunks =
+    V*(d/g)*4/16384 (rounded up)."""
+    w = synth.workload(name)
+    d = oracle.StreamDesc(w.bits, w.group, w.head_dim, w.layers, w.kv_heads,
+                          [w.tokens])
+    lay = d.layout()
+    assert lay.V == w.vectors
+    assert (lay.n_code, lay.n_meta, lay.n_chunks) == (n_code, n_meta, n_code + n_meta)
+    assert lay.code_per_seg == w.group * w.bits // 32
+
+
+def test_chunk_order_is_segment_by_segment():
+    lay = oracle.StreamDesc(2, 32, 128, 1, 1, [1250]).layout()   # V = 2500, R = 2
+    assert lay.code_per_seg == 2 and lay.n_code == 5 and lay.n_meta == 3
+    idx = sorted([("c", c, oracle.code_chunk_index(lay, c)) for c in range(5)] +
+                 [("m", s, oracle.meta_chunk_index(lay, s)) for s in range(3)],
+                 key=lambda t: t[2])
+    assert [(k, i) for k, i, _ in idx] == [("c", 0), ("c", 1), ("m", 0), ("c", 2),
+                                           ("c", 3), ("m", 1), ("c", 4), ("m", 2)]
+    assert [t[2] for t in idx] == list(range(8))
+
+
+def test_roundtrip_error_bound_tiny():
+    """x^ - x = D H (y^ - y) / d up to the final bf16 rounding, and H/sqrt(d)
+    is orthonormal, so ||x^ - x||_2 <= ||y^ - y||_2 / sqrt(d) + bf16 term,
+    with |y^ - y| <= sf/2 per element in each group."""
+    w, d, x = tiny_desc_and_vectors()
+    st, s = oracle.compress(d, x)
+    assert st == oracle.OK and s.size <= d.max_bytes()
+    st, xh = oracle.decompress(s, d)
+    assert st == oracle.OK
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).double().numpy()
+    xhf = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).double().numpy()
+    _, codes, meta = oracle.quantize_vectors(x, w.bits, w.group, 0)
+    sh = meta.reshape(x.shape[0], -1, 4)
+    sh = (sh[..., 0].astype(np.uint16) | (sh[..., 1].astype(np.uint16) << 8)).view(np.float16)
+    sf = sh.astype(np.float64) * 8
+    ybound = np.sqrt((sf / 2) ** 2 * w.group).sum(axis=1) if sf.shape[1] == 1 else \
+        np.sqrt(((sf / 2) ** 2 * w.group).sum(axis=1))
+    err = np.linalg.norm(xhf - xf, axis=1)
+    bf16_term = np.linalg.norm(xhf, axis=1) * 2.0 ** -8
+    assert np.all(err <= ybound / np.sqrt(w.head_dim) * (1 + 1e-4) + bf16_term)
+    # and it is a real codec: 4-bit relative error well below 1
+    assert err.mean() / np.linalg.norm(xf, axis=1).mean() < 0.15
+
+
+def test_stream_is_deterministic_and_segments_agree():
+    w, d, x = tiny_desc_and_vectors()
+    st1, s1 = oracle.compress(d, x)
+    st2, s2 = oracle.compress(d, x)
+    assert np.array_equal(s1, s2)
+    lay = d.layout()
+    st, chunks = oracle.encode_segment(d, 0, x)
+    base = lay.data_base
+    off = 0
+    for i, ch in enumerate(chunks):
+        e = _u(s1, 64 + 8 * i, 8)
+        assert e & 0xFFFF == ch.size and (e >> 16) * 16 == off
+        assert np.array_equal(s1[base + off: base + off + ch.size], ch)
+        off += (ch.size + 15) // 16 * 16
+
+
+def test_corrupt_streams():
+    _, d, x = tiny_desc_and_vectors()
+    _, s = oracle.compress(d, x)
+    assert oracle.decompress(s[:-16], d)[0] == oracle.CORRUPT       # truncated
+    for off, val in ((0, 0x4A), (8, 2), (12, 64), (24, 4), (52, 6)):
+        bad = s.copy()
+        bad[off] = val
+        assert oracle.decompress(bad, d)[0] == oracle.CORRUPT, off
+    bad = s.copy()
+    bad[64] ^= 0x10                                                   # chunk 0 size
+    assert oracle.decompress(bad, d)[0] == oracle.CORRUPT
+    bad = s.copy()
+    bad[64 + 8 + 2] ^= 0x01                                           # chunk 1 offset
+    assert oracle.decompress(bad, d)[0] == oracle.CORRUPT
+
+
+def test_mode1_chunks_roundtrip():
+    """Half of the tokens zero: code chunks of zero vectors compress to a
+    bitmap plus few bytes; the stream still decodes bit-exactly to what the
+    per-vector decode gives."""
+    w, d, x = tiny_desc_and_vectors()
+    x = x.copy()
+    x[: x.shape[0] // 2] = 0
+    st, s = oracle.compress(d, x)
+    assert st == oracle.OK
+    lay = d.layout()
+    sizes = [_u(s, 64 + 8 * i, 8) & 0xFFFF for i in range(lay.n_chunks)]
+    assert min(sizes[:2]) < 16384                                     # mode-1 chunks
+    st, xh = oracle.decompress(s, d)
+    _, codes, meta = oracle.quantize_vectors(x, w.bits, w.group, 0)
+    ref = oracle.dequantize_vectors(codes, meta, 128, w.bits, w.group, 0)
+    assert st == oracle.OK and np.array_equal(xh, ref)
+
+
+def test_empty_stream():
+    d = oracle.StreamDesc(4, 128, 128, 2, 8, [0])
+    st, s = oracle.compress(d, np.zeros((0, 128), np.uint16))
+    assert st == oracle.OK and s.size == d.layout().data_base == 80
+    st, xh = oracle.decompress(s, d)
+    assert st == oracle.OK and xh.shape == (0, 128)
+
+
+def test_gather_dense_matches_permuted_indexing():
+    rng = np.random.default_rng(0)
+    L, H, T, D = 2, 3, 5, 64
+    store = rng.integers(0, 65536, (T, L, H, 2, D)).astype(np.uint16)   # odd layout
+    st = [s // 2 for s in store.strides]                              # elements
+    strides = (st[1], st[3], st[2], st[0])                            # layer, kv, head, token
+    out = oracle.gather_dense(store.reshape(-1), L, H, T, D, strides, 0, L * 2 * H * T)
+    ref = store.transpose(1, 3, 2, 0, 4).reshape(-1, D)               # [l][kv][h][t]
+    assert np.array_equal(out, ref)
+    out2 = oracle.gather_dense(store.reshape(-1), L, H, T, D, strides, 7, 23)
+    assert np.array_equal(out2, ref[7:23])
+
+
+def test_gather_paged_matches_python_walk():
+    w = synth.Workload("t", 2, 2, 64, 4, 64, 5, "lognormal", seq_lens=[20, 0, 33, 16])
+    pk = synth.paged_kv(w)
+    pool = synth.bf16_bits(pk.pool)
+    pt = pk.page_table.numpy()
+    ref = []
+    for l in range(2):
+        for kv in range(2):
+            for h in range(2):
+                for r, n in enumerate(w.seq_lens):
+                    for t in range(n):
+                        ref.append(pool[l, pt[r, t // 16], kv, h, t % 16])
+    ref = np.array(ref)
+    out = oracle.gather_paged(pool.reshape(-1), 2, 2, 64, pk.strides(), 16, w.seq_lens,
+                              pt, 0, len(ref))
+    assert np.array_equal(out, ref)
