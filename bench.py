@@ -1,0 +1,378 @@
+"""Throughput of the B200 KV-cache codec: one step = fused encode + fused decode
+of one synthetic KV cache resident in HBM (Llama-3-8B shape by default:
+[32, 2, 8, 4096, 128] bf16, 4-bit, group 128).
+
+Prints ONE JSON line (rank 0):
+  value      raw bf16 bytes per second of encode + decode, all ranks (GB/s)
+  e2e        the same metric through the C ABI with pinned host buffers:
+             H2D KV, compress, D2H stream, H2D stream, decompress, D2H KV
+  roofline   the slower kernel: algorithmic bytes per launch / its CUDA-event
+             duration against the measured HBM copy bandwidth
+  cpu_baseline  the CPU oracle on a bounded sample of the same workload
+Also: per-direction GB/s, compression ratio, break-even link speed, net wire
+time saved at 100 and 400 Gbit/s, SM clocks sampled during the timed region.
+
+Multi-GPU (torchrun): every rank compresses its own KV cache (weak scaling);
+the only collectives are a barrier and a max over ranks of the timings.
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "encode/decode GB/s of raw bf16 KV on 1 B200 and % of HBM roofline; ratio"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        self.file.seek(0)
+        rows = [l.strip().split(", ") for l in self.file.read().splitlines() if l.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except Exception:
+                continue
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# -------------------------------------------------------------- workloads --
+def make_input(wname: str, device, rank: int):
+    import torch
+    from kv_cache_compression_04_b200 import synth
+    import kv_cache_compression_04_b200 as kvc
+    w = synth.workload(wname)
+    w.seed += 1000 * rank
+    if w.paged:
+        pk = synth.paged_kv(w, device=device)
+        desc = kvc.paged_desc(pk.pool, pk.page_table, w.seq_lens)
+
+        def out_desc():
+            pool2 = torch.empty_like(pk.pool)
+            return kvc.paged_desc(pool2, pk.page_table, w.seq_lens), pool2
+        return w, desc, out_desc, pk
+    kv = synth.dense_kv(w, device=device)
+    desc = kvc.dense_desc(kv)
+
+    def out_desc():
+        o = torch.empty_like(kv)
+        return kvc.dense_desc(o), o
+    return w, desc, out_desc, kv
+
+
+def describe(w) -> str:
+    if w.paged:
+        return (f"{w.name}: {w.layers} layers x 2 x {w.kv_heads} heads x d{w.head_dim}, "
+                f"{len(w.seq_lens)} requests, {w.total_tokens} tokens in 16-token pages, "
+                f"{w.bits}-bit g{w.group}")
+    return (f"{w.name}: [{w.layers}, 2, {w.kv_heads}, {w.tokens}, {w.head_dim}] bf16, "
+            f"{w.bits}-bit g{w.group}")
+
+
+# ------------------------------------------------------------ CPU oracle --
+def oracle_sample(wname: str, budget_s: float, seed_offset: int = 0):
+    """Round trip of whole segments through the CPU oracle until `budget_s`
+    of CPU time is spent. Returns (raw bytes processed, seconds, segments)."""
+    import numpy as np
+    import torch
+    import oracle
+    from kv_cache_compression_04_b200 import synth
+    w = synth.workload(wname)
+    od = oracle.StreamDesc(w.bits, w.group, w.head_dim, w.layers, w.kv_heads,
+                           w.seq_lens if w.paged else [w.tokens])
+    lay = od.layout()
+    vm = lay.vec_per_code * lay.code_per_seg
+    g = torch.Generator().manual_seed(w.seed + seed_offset)
+    done_bytes, spent, segs = 0, 0.0, 0
+    while spent < budget_s and segs < lay.n_seg:
+        # a segment of vectors drawn with the workload's key distribution
+        x = torch.randn(vm, w.head_dim, generator=g) * torch.exp(
+            w.scale_sigma * torch.randn(1, w.head_dim, generator=g))
+        x = synth.bf16_bits(x.to(torch.bfloat16))
+        t0 = time.perf_counter()
+        st, chunks = oracle.encode_segment(od, segs, x)
+        _, y = oracle.decode_segment(od, segs, chunks, vm)
+        spent += time.perf_counter() - t0
+        done_bytes += x.nbytes
+        segs += 1
+    return done_bytes, spent, segs
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    per_step = max(0.5, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(args.workload, per_step / 4)
+    tot_b, tot_s, segs = 0, 0.0, 0
+    for _ in range(args.steps):
+        b, s, n = oracle_sample(args.workload, per_step)
+        tot_b += b
+        tot_s += s
+        segs += n
+    from kv_cache_compression_04_b200 import synth
+    w = synth.workload(args.workload)
+    v = tot_b / tot_s / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": describe(w), "sample": f"{segs} segments"},
+            "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"{segs} whole segments of {args.workload} vectors, "
+                                       "encode + decode, single thread"},
+            "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    import torch
+    import kv_cache_compression_04_b200 as kvc
+    from kv_cache_compression_04_b200 import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    build.build()
+    dev = torch.device("cuda", local)
+
+    w, desc, out_desc_fn, keep = make_input(args.workload, dev, rank)
+    codec = kvc.Codec(w.bits, w.group, w.sign_seed)
+    out, ws, nb = codec.buffers(desc, dev)
+    odesc, obuf = out_desc_fn()
+    dws = torch.empty(kvc.KVC_DECOMPRESS_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = kvc._stream_ptr(stream)
+    raw = w.raw_bytes
+
+    def enc():
+        st = kvc.kvc_compress(desc, codec.params, out.data_ptr(), out.numel(), nb.data_ptr(),
+                              ws.data_ptr(), ws.numel(), sp)
+        assert st == kvc.KVC_OK, kvc.STATUS[st]
+
+    def dec(n):
+        st = kvc.kvc_decompress(out.data_ptr(), n, odesc, dws.data_ptr(), dws.numel(), sp)
+        assert st == kvc.KVC_OK, kvc.STATUS[st]
+
+    # correctness gate + stream size
+    enc()
+    assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+    nbytes = int(nb.item())
+    dec(nbytes)
+    assert kvc.kvc_stream_status(dws.data_ptr(), sp) == kvc.KVC_OK
+
+    for _ in range(args.warmup):
+        enc()
+        dec(nbytes)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            enc()
+            ev[i][1].record(stream)
+            dec(nbytes)
+            ev[i][2].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    total_ms = start.elapsed_time(stop)
+    enc_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    dec_ms = [b.elapsed_time(c) for _, b, c in ev]
+    stats = torch.tensor([total_ms, sum(enc_ms) / K, sum(dec_ms) / K], device=dev,
+                         dtype=torch.float64)
+    if dist:
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+    total_ms, enc_avg, dec_avg = stats.tolist()
+    assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+    assert kvc.kvc_stream_status(dws.data_ptr(), sp) == kvc.KVC_OK
+
+    # ------------------------------------------------ end to end via host --
+    e2e = None
+    if args.e2e_steps > 0:
+        src = (keep.pool if w.paged else keep)
+        h_in = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
+        h_in.copy_(src)
+        h_stream = torch.empty(out.numel(), dtype=torch.uint8, pin_memory=True)
+        h_out = torch.empty(obuf.shape, dtype=obuf.dtype, pin_memory=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def e2e_step():
+            src.copy_(h_in, non_blocking=True)
+            enc()
+            h_stream[:nbytes].copy_(out[:nbytes], non_blocking=True)
+            out[:nbytes].copy_(h_stream[:nbytes], non_blocking=True)
+            dec(nbytes)
+            h_out.copy_(obuf, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if dist:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        t = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+        if dist:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item() / args.e2e_steps
+        inb = src.numel() * src.element_size()
+        e2e = {"value": round(raw * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": inb + nbytes, "d2h_bytes_per_step": nbytes + inb,
+               "ms_per_step": round(e2e_ms, 3)}
+        assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    hbm, peak_kind = peaks()
+    step_ms = total_ms / K
+    value = raw * world / (step_ms * 1e-3) / 1e9
+    enc_bytes = raw + nbytes            # algorithmic: read KV, write stream
+    dec_bytes = nbytes + raw            # read stream, write KV
+    enc_gbs = enc_bytes / (enc_avg * 1e-3) / 1e9
+    dec_gbs = dec_bytes / (dec_avg * 1e-3) / 1e9
+    dom = "encode" if enc_avg >= dec_avg else "decode"
+    achieved = enc_gbs if dom == "encode" else dec_gbs
+    ratio = raw / nbytes
+    saved_bits = 8 * (raw - nbytes)
+    t_codec = (enc_avg + dec_avg) * 1e-3
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; shapes and distributions of the named workload)",
+        "config": {"workload": describe(w), "raw_bytes_per_step_per_gpu": raw,
+                   "stream_bytes": nbytes, "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"weak x{world}, no data-path collective"},
+        "encode_GBps": round(raw / (enc_avg * 1e-3) / 1e9, 3),
+        "decode_GBps": round(raw / (dec_avg * 1e-3) / 1e9, 3),
+        "encode_ms": round(enc_avg, 4), "decode_ms": round(dec_avg, 4),
+        "ratio": round(ratio, 4),
+        "break_even_gbit_s": round(saved_bits / t_codec / 1e9, 1),
+        "net_gain_ms": {"100Gbit": round((saved_bits / 100e9 - t_codec) * 1e3, 3),
+                        "400Gbit": round((saved_bits / 400e9 - t_codec) * 1e3, 3)},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                     "peak_kind": peak_kind, "traffic": None,
+                     "encode_frac": round(enc_gbs / hbm, 4),
+                     "decode_frac": round(dec_gbs / hbm, 4)},
+        "gpu_launches": 2 * K,
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if world == 1 and args.cpu_budget > 0:
+        b, s, n = oracle_sample(args.workload, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(b / s / 1e9, 6), "unit": "GB/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"{n} whole segments ({b} raw bytes) of "
+                                          f"{args.workload} vectors, encode + decode, "
+                                          "single thread"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

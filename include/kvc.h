@@ -1,0 +1,171 @@
+/*
+ * kvc.h — C ABI of libkvc.so, a B200 (sm_100a) KV-cache codec in the manner of
+ * FastKVComp ("Beyond Compression Ratio: High-Throughput KV Compression for
+ * Disaggregated LLM Serving", Abstract and Methodology; podcast page
+ * "FastKVComp: checking whether high-throughput KV compression pays off",
+ * episode notes).
+ *
+ * Encode: random +-1 signs and an fp32 Walsh-Hadamard transform over head_dim,
+ * 2- or 4-bit asymmetric group quantization with fp16 scale/zero, code packing,
+ * then a lossless stage over 16 KB chunks (bit-plane shuffle, zero-byte
+ * elimination with a bitmap, device-wide prefix sum of chunk sizes and
+ * compaction) into one self-describing byte stream. Decode inverts every step.
+ * Only the quantization loses information.
+ *
+ * Conventions shared by every entry point:
+ *  - Memory. The caller owns every buffer (input, output, page table,
+ *    workspace, stream). The library allocates nothing and keeps no global
+ *    state; calls are re-entrant, but concurrent calls need distinct
+ *    workspaces.
+ *  - Asynchrony. All device work is enqueued on `stream` (a cudaStream_t; 0 is
+ *    the legacy default stream). Pointers marked DEVICE must stay valid until
+ *    that work completes.
+ *  - Synchronous errors. Argument, shape and capacity errors are returned
+ *    before anything is enqueued: KVC_ERR_INVALID_ARG, KVC_ERR_UNSUPPORTED,
+ *    KVC_ERR_CAPACITY. A failed CUDA launch returns KVC_ERR_CUDA.
+ *  - Data-dependent errors (non-finite input, fp16 meta overflow, a corrupt
+ *    stream, an invalid page index, a device wait that ran out) are written to
+ *    a status word in the workspace; kvc_stream_status() reads it. The first
+ *    error of a call wins; each call clears the word when it starts.
+ *  - Bounds. Encode never writes outside [out, out + out_capacity) or the
+ *    workspace; decode never writes outside the output slots its descriptor
+ *    names. On an error the output content is unspecified.
+ *  - Alignment. `data`, `out`, the stream passed to decode and `workspace`
+ *    must be 16-byte aligned; every vector start (all strides times 2 bytes)
+ *    must be 16-byte aligned, i.e. strides are multiples of 8 elements.
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; declared here so that this header
+ * needs no CUDA include. */
+typedef struct CUstream_st *kvc_stream_t;
+
+typedef enum {
+  KVC_OK = 0,
+  KVC_ERR_INVALID_ARG = 1, /* null pointer, bad shape, stride or alignment     */
+  KVC_ERR_UNSUPPORTED = 2, /* bits / group / head_dim outside the built set    */
+  KVC_ERR_CAPACITY = 3,    /* out_capacity or workspace too small              */
+  KVC_ERR_NONFINITE = 4,   /* an input vector transforms to inf or NaN         */
+  KVC_ERR_RANGE = 5,       /* a group's zero or scale overflows fp16           */
+  KVC_ERR_CORRUPT = 6,     /* stream header, table or chunk inconsistent, or a
+                              page index outside the pool                     */
+  KVC_ERR_TIMEOUT = 7,     /* a bounded device wait gave up                   */
+  KVC_ERR_CUDA = 8         /* CUDA runtime error (launch, copy, device)       */
+} kvc_status;
+
+/* Quantization parameters.
+ *  bits       2 or 4 bits per code.
+ *  group_size 32, 64 or 128 consecutive channels of the transformed vector
+ *             share one fp16 zero and scale; must divide head_dim.
+ *  sign_seed  seeds the +-1 diagonal: channel c is negated iff bit (c mod 64)
+ *             of SplitMix64 output number floor(c/64), counted from state =
+ *             sign_seed, is 1. */
+typedef struct {
+  int32_t bits;
+  int32_t group_size;
+  uint64_t sign_seed;
+} kvc_params;
+
+enum { KVC_DENSE = 0, KVC_PAGED = 1 };
+
+/* Largest request count of a paged descriptor. */
+#define KVC_MAX_REQUESTS 1024
+/* Workspace bytes kvc_decompress needs (it only keeps a status word). */
+#define KVC_DECOMPRESS_WORKSPACE_BYTES 256
+
+/* A KV cache: logical shape [layers, 2 (K, V), kv_heads, tokens, head_dim],
+ * bf16, head_dim contiguous. Vectors are coded in the logical order
+ * [layer][kv][head][request][token]; a dense tensor is one request.
+ *
+ * kind = KVC_DENSE:
+ *   element (l, kv, h, t, c) at data + l*stride_layer + kv*stride_kv +
+ *   h*stride_head + t*stride_token + c (strides in elements).
+ * kind = KVC_PAGED (a pool of pages of page_tokens token slots):
+ *   token t of request r sits in page p = page_table[r*page_table_stride +
+ *   t/page_tokens], slot t % page_tokens; element (l, kv, h, r, t, c) at
+ *   data + l*stride_layer + p*stride_page + kv*stride_kv + h*stride_head +
+ *   (t % page_tokens)*stride_slot + c. Pages are checked against
+ *   [0, num_pages); a page outside it sets KVC_ERR_CORRUPT and its vectors
+ *   are neither read nor written.
+ *
+ * head_dim is 64 or 128 in this build (256 returns KVC_ERR_UNSUPPORTED). */
+typedef struct {
+  int32_t kind;
+  int32_t layers;
+  int32_t kv_heads;
+  int32_t head_dim;
+  void *data;                 /* DEVICE bf16 tensor or page pool             */
+  int64_t stride_layer;       /* elements, both kinds                        */
+  int64_t stride_kv;          /* elements, both kinds                        */
+  int64_t stride_head;        /* elements, both kinds                        */
+  /* dense */
+  int64_t tokens;             /* T >= 0                                      */
+  int64_t stride_token;       /* elements                                    */
+  /* paged */
+  int32_t page_tokens;        /* token slots per page, >= 1                  */
+  int32_t n_requests;         /* 0 .. KVC_MAX_REQUESTS                       */
+  int64_t stride_page;        /* elements                                    */
+  int64_t stride_slot;        /* elements                                    */
+  int64_t num_pages;          /* pages in the pool                           */
+  const int32_t *seq_lens;    /* HOST [n_requests], tokens per request >= 0  */
+  const int32_t *page_table;  /* DEVICE int32 [n_requests][page_table_stride] */
+  int64_t page_table_stride;  /* entries per request row                     */
+} kvc_kv_desc;
+
+/* Exact worst-case stream length for this shape and these parameters: the
+ * header and tables plus every chunk at its raw length, each rounded up to
+ * 16 bytes. Host only, pure; returns 0 for an invalid description. */
+size_t kvc_max_compressed_bytes(const kvc_kv_desc *kv, const kvc_params *params);
+
+/* Workspace bytes kvc_compress needs for this shape (DEVICE memory, 16-byte
+ * aligned, caller-owned, contents need not be initialized). kvc_decompress
+ * needs KVC_DECOMPRESS_WORKSPACE_BYTES. Returns 0 for an invalid
+ * description. */
+size_t kvc_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params);
+
+/* Compresses `kv` into `out` (DEVICE, out_capacity bytes, which must be at
+ * least kvc_max_compressed_bytes). The stream length is written to the
+ * header's stream_bytes field and, if out_bytes_dev (DEVICE) is not null, to
+ * *out_bytes_dev. Stream layout (little-endian): 64-byte header; u64 chunk
+ * table (bits 0..15 unpadded chunk size, bits 16..63 offset from the data base
+ * in 16-byte units); u32 token count per request; zero padding to 16 bytes;
+ * the chunks, each zero-padded to 16 bytes. The code and meta regions are cut
+ * into 16 KB chunks; a meta chunk covers group_size*bits/32 code chunks and
+ * follows them. */
+kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params,
+                        void *out, size_t out_capacity, uint64_t *out_bytes_dev,
+                        void *workspace, size_t workspace_bytes,
+                        kvc_stream_t stream);
+
+/* Decompresses the stream at `in` (DEVICE, in_bytes readable bytes) into the
+ * slots described by `out`. Bits, group size and sign seed come from the
+ * stream. The logical shape must match the stream's: layers, kv_heads,
+ * head_dim and total tokens; a paged receiver must also match the stream's
+ * request count and per-request token counts. The receiver's layout (dense or
+ * paged, page table, strides) may differ from the sender's. A mismatch or any
+ * inconsistency in the stream sets KVC_ERR_CORRUPT; reads stay inside
+ * [in, in + in_bytes). Slots outside the described tokens are not written. */
+kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *out,
+                          void *workspace, size_t workspace_bytes,
+                          kvc_stream_t stream);
+
+/* Waits for `stream`, then returns the status word of the last call that used
+ * this workspace (KVC_OK if it found no data-dependent error), or
+ * KVC_ERR_CUDA if the stream reports a CUDA error. */
+kvc_status kvc_stream_status(const void *workspace, kvc_stream_t stream);
+
+/* Static, human-readable name of a status. */
+const char *kvc_status_string(kvc_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVC_H */

@@ -1,0 +1,258 @@
+// Host side of the C ABI in include/kvc.h: argument validation, stream layout
+// arithmetic, workspace layout, kernel parameters and launches. Allocates
+// nothing and keeps no state beyond per-kernel launch attributes.
+#include <string.h>
+
+#include <cuda_runtime.h>
+
+#include "kvc_internal.h"
+
+using namespace kvc;
+
+namespace {
+
+struct Shape {
+  int D = 0, bits = 0, G = 0;
+  uint64_t T = 0;      // tokens per (layer, kv, head), summed over requests
+  uint64_t V = 0;      // vectors
+  uint32_t n_req = 0;
+  uint64_t CB = 0, MB = 0, VC = 0, R = 0;
+  uint64_t n_code = 0, n_seg = 0, n_chunks = 0;
+  uint64_t data_base = 0, max_bytes = 0, ws_bytes = 0;
+};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool stride_ok(int64_t s) { return s % 8 == 0; }  // 16-byte vector starts
+
+// Shape and layout checks shared by both directions (bits/group optional).
+kvc_status describe(const kvc_kv_desc *kv, const kvc_params *p, Shape &s) {
+  if (!kv) return KVC_ERR_INVALID_ARG;
+  if (kv->kind != KVC_DENSE && kv->kind != KVC_PAGED) return KVC_ERR_INVALID_ARG;
+  if (kv->layers < 0 || kv->kv_heads < 0) return KVC_ERR_INVALID_ARG;
+  if (kv->head_dim != 64 && kv->head_dim != 128) return KVC_ERR_UNSUPPORTED;
+  s.D = kv->head_dim;
+  if (!stride_ok(kv->stride_layer) || !stride_ok(kv->stride_kv) || !stride_ok(kv->stride_head))
+    return KVC_ERR_INVALID_ARG;
+  if (kv->kind == KVC_DENSE) {
+    if (kv->tokens < 0 || kv->tokens >= (int64_t(1) << 31)) return KVC_ERR_INVALID_ARG;
+    if (!stride_ok(kv->stride_token)) return KVC_ERR_INVALID_ARG;
+    s.T = uint64_t(kv->tokens);
+    s.n_req = 1;
+  } else {
+    if (kv->n_requests < 0 || kv->n_requests > KVC_MAX_REQUESTS) return KVC_ERR_INVALID_ARG;
+    if (kv->n_requests > 0 && !kv->seq_lens) return KVC_ERR_INVALID_ARG;
+    if (kv->page_tokens < 1 || !stride_ok(kv->stride_page) || !stride_ok(kv->stride_slot))
+      return KVC_ERR_INVALID_ARG;
+    int64_t maxlen = 0;
+    for (int r = 0; r < kv->n_requests; ++r) {
+      if (kv->seq_lens[r] < 0) return KVC_ERR_INVALID_ARG;
+      s.T += uint64_t(kv->seq_lens[r]);
+      maxlen = kv->seq_lens[r] > maxlen ? kv->seq_lens[r] : maxlen;
+    }
+    if (s.T >= (uint64_t(1) << 31)) return KVC_ERR_INVALID_ARG;
+    if (s.T > 0) {
+      if (!kv->page_table || kv->num_pages < 1) return KVC_ERR_INVALID_ARG;
+      if (kv->page_table_stride < (maxlen + kv->page_tokens - 1) / kv->page_tokens)
+        return KVC_ERR_INVALID_ARG;
+    }
+    s.n_req = uint32_t(kv->n_requests);
+  }
+  s.V = uint64_t(kv->layers) * 2u * uint64_t(kv->kv_heads) * s.T;
+  if (s.V >= (uint64_t(1) << 31)) return KVC_ERR_UNSUPPORTED;
+  if (s.V > 0 && (!kv->data || !aligned16(kv->data))) return KVC_ERR_INVALID_ARG;
+  if (!p) return KVC_OK;
+  if (p->bits != 2 && p->bits != 4) return KVC_ERR_UNSUPPORTED;
+  if (p->group_size != 32 && p->group_size != 64 && p->group_size != 128)
+    return KVC_ERR_UNSUPPORTED;
+  if (p->group_size > s.D) return KVC_ERR_UNSUPPORTED;
+  s.bits = p->bits;
+  s.G = p->group_size;
+  // Stream layout (readings R12/R13): codes and meta chunked separately into
+  // 16 KB chunks; one meta chunk covers R = G*bits/32 code chunks.
+  s.CB = uint64_t(s.D) * s.bits / 8;
+  s.MB = uint64_t(s.D / s.G) * 4;
+  s.VC = kChunk / s.CB;
+  s.R = uint64_t(s.G) * s.bits / 32;
+  s.n_code = (s.V + s.VC - 1) / s.VC;
+  s.n_seg = (s.n_code + s.R - 1) / s.R;
+  s.n_chunks = s.n_code + s.n_seg;
+  s.data_base = round16(kHeader + 8 * s.n_chunks + 4 * uint64_t(s.n_req));
+  s.max_bytes = s.data_base;
+  if (s.n_code) {
+    const uint64_t VM = s.VC * s.R;
+    s.max_bytes += (s.n_code - 1) * kChunk + round16((s.V - (s.n_code - 1) * s.VC) * s.CB);
+    s.max_bytes += (s.n_seg - 1) * kChunk + round16((s.V - (s.n_seg - 1) * VM) * s.MB);
+  }
+  s.ws_bytes = kWsCtl + round256(8 * s.n_code) + s.n_seg * kChunk;
+  return KVC_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+DenseLayout dense_layout(const kvc_kv_desc *kv, const Shape &s) {
+  DenseLayout L{};
+  L.base = static_cast<uint8_t *>(kv->data);
+  L.s_l = kv->stride_layer * 2;
+  L.s_kv = kv->stride_kv * 2;
+  L.s_h = kv->stride_head * 2;
+  L.s_t = kv->stride_token * 2;
+  L.T = make_fastdiv(s.T ? uint32_t(s.T) : 1u);
+  L.H = make_fastdiv(kv->kv_heads ? uint32_t(kv->kv_heads) : 1u);
+  L.tokens = uint32_t(s.T);
+  return L;
+}
+
+void paged_layout(const kvc_kv_desc *kv, const Shape &s, PagedLayout &L) {
+  L.base = static_cast<uint8_t *>(kv->data);
+  L.s_l = kv->stride_layer * 2;
+  L.s_p = kv->stride_page * 2;
+  L.s_kv = kv->stride_kv * 2;
+  L.s_h = kv->stride_head * 2;
+  L.s_slot = kv->stride_slot * 2;
+  L.page_table = kv->page_table;
+  L.pt_stride = kv->page_table_stride;
+  L.num_pages = kv->num_pages;
+  L.T = make_fastdiv(s.T ? uint32_t(s.T) : 1u);
+  L.H = make_fastdiv(kv->kv_heads ? uint32_t(kv->kv_heads) : 1u);
+  L.PT = make_fastdiv(uint32_t(kv->page_tokens));
+  L.n_req = s.n_req;
+  L.cum[0] = 0;
+  for (uint32_t r = 0; r < s.n_req; ++r) L.cum[r + 1] = L.cum[r] + uint32_t(kv->seq_lens[r]);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvc_max_compressed_bytes(const kvc_kv_desc *kv, const kvc_params *params) {
+  Shape s;
+  if (!params || describe(kv, params, s) != KVC_OK) return 0;
+  return size_t(s.max_bytes);
+}
+
+size_t kvc_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params) {
+  Shape s;
+  if (!params || describe(kv, params, s) != KVC_OK) return 0;
+  return size_t(s.ws_bytes);
+}
+
+kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *out,
+                        size_t out_capacity, uint64_t *out_bytes_dev, void *workspace,
+                        size_t workspace_bytes, kvc_stream_t stream) {
+  Shape s;
+  if (!params) return KVC_ERR_INVALID_ARG;
+  kvc_status st = describe(kv, params, s);
+  if (st != KVC_OK) return st;
+  if (!out || !aligned16(out) || !workspace || !aligned16(workspace)) return KVC_ERR_INVALID_ARG;
+  if (out_capacity < s.max_bytes || workspace_bytes < s.ws_bytes) return KVC_ERR_CAPACITY;
+  const int sms = sm_count();
+  if (sms <= 0) return KVC_ERR_CUDA;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  EncArgs a{};
+  a.V = uint32_t(s.V);
+  a.n_tiles = uint32_t(s.n_code);
+  a.n_seg = uint32_t(s.n_seg);
+  a.n_chunks = uint32_t(s.n_chunks);
+  a.out = static_cast<uint8_t *>(out);
+  a.out_capacity = out_capacity;
+  a.data_base = s.data_base;
+  a.out_bytes_dev = out_bytes_dev;
+  a.status = reinterpret_cast<uint32_t *>(ws);
+  a.ticket = reinterpret_cast<uint32_t *>(ws + 4);
+  a.tile_state = reinterpret_cast<uint64_t *>(ws + kWsCtl);
+  a.ws_meta = ws + kWsCtl + round256(8 * s.n_code);
+  a.layers = uint32_t(kv->layers);
+  a.kv_heads = uint32_t(kv->kv_heads);
+  a.head_dim = uint32_t(s.D);
+  a.group = uint32_t(s.G);
+  a.bits = uint32_t(s.bits);
+  a.k = (s.D == 64 ? 6u : s.D == 128 ? 7u : 8u) / 2;
+  a.origin = kv->kind == KVC_PAGED ? 1u : 0u;
+  a.n_req = s.n_req;
+  a.tokens = s.T;
+  a.seed = params->sign_seed;
+  sign_masks(params->sign_seed, s.D, a.sign_mask);
+
+  if (cudaMemsetAsync(ws, 0, kWsCtl + 8 * s.n_code, cs) != cudaSuccess) return KVC_ERR_CUDA;
+  cudaError_t e;
+  if (kv->kind == KVC_DENSE) {
+    const DenseLayout L = dense_layout(kv, s);
+    e = s.D == 128 ? launch_encode_dense_d128(s.bits, s.G, a, L, sms, cs)
+                   : launch_encode_dense_d64(s.bits, s.G, a, L, sms, cs);
+  } else {
+    static thread_local PagedLayout L;  // large (4 KB) parameter block
+    paged_layout(kv, s, L);
+    e = s.D == 128 ? launch_encode_paged_d128(s.bits, s.G, a, L, sms, cs)
+                   : launch_encode_paged_d64(s.bits, s.G, a, L, sms, cs);
+  }
+  return e == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *out,
+                          void *workspace, size_t workspace_bytes, kvc_stream_t stream) {
+  Shape s;
+  kvc_status st = describe(out, nullptr, s);
+  if (st != KVC_OK) return st;
+  if (!in || !aligned16(in) || !workspace || !aligned16(workspace)) return KVC_ERR_INVALID_ARG;
+  if (workspace_bytes < KVC_DECOMPRESS_WORKSPACE_BYTES) return KVC_ERR_CAPACITY;
+  const int sms = sm_count();
+  if (sms <= 0) return KVC_ERR_CUDA;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  DecArgs a{};
+  a.in = static_cast<const uint8_t *>(in);
+  a.in_bytes = in_bytes;
+  a.status = static_cast<uint32_t *>(workspace);
+  a.layers = uint32_t(out->layers);
+  a.kv_heads = uint32_t(out->kv_heads);
+  a.head_dim = uint32_t(s.D);
+  a.n_req = s.n_req;
+  a.tokens = s.T;
+  a.V = uint32_t(s.V);
+  a.paged_receiver = out->kind == KVC_PAGED ? 1u : 0u;
+  if (cudaMemsetAsync(workspace, 0, KVC_DECOMPRESS_WORKSPACE_BYTES, cs) != cudaSuccess)
+    return KVC_ERR_CUDA;
+  cudaError_t e;
+  if (out->kind == KVC_DENSE) {
+    const DenseLayout L = dense_layout(out, s);
+    e = s.D == 128 ? launch_decode_dense_d128(a, L, sms, cs) : launch_decode_dense_d64(a, L, sms, cs);
+  } else {
+    static thread_local PagedLayout L;
+    paged_layout(out, s, L);
+    e = s.D == 128 ? launch_decode_paged_d128(a, L, sms, cs) : launch_decode_paged_d64(a, L, sms, cs);
+  }
+  return e == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+kvc_status kvc_stream_status(const void *workspace, kvc_stream_t stream) {
+  if (!workspace) return KVC_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return KVC_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return KVC_ERR_CUDA;
+  return v <= KVC_ERR_CUDA ? static_cast<kvc_status>(v) : KVC_ERR_CUDA;
+}
+
+const char *kvc_status_string(kvc_status status) {
+  switch (status) {
+    case KVC_OK: return "KVC_OK";
+    case KVC_ERR_INVALID_ARG: return "KVC_ERR_INVALID_ARG";
+    case KVC_ERR_UNSUPPORTED: return "KVC_ERR_UNSUPPORTED";
+    case KVC_ERR_CAPACITY: return "KVC_ERR_CAPACITY";
+    case KVC_ERR_NONFINITE: return "KVC_ERR_NONFINITE";
+    case KVC_ERR_RANGE: return "KVC_ERR_RANGE";
+    case KVC_ERR_CORRUPT: return "KVC_ERR_CORRUPT";
+    case KVC_ERR_TIMEOUT: return "KVC_ERR_TIMEOUT";
+    case KVC_ERR_CUDA: return "KVC_ERR_CUDA";
+  }
+  return "KVC_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,275 @@
+// Device building blocks of libkvc (sm_100a): mbarriers and bulk-async copies,
+// memory-model helpers, paired fp32 arithmetic, the register Walsh-Hadamard
+// butterfly, the 32x32 bit transpose, block scans and vector addressing.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "kvc_internal.h"
+
+namespace kvc {
+
+// Every device wait is bounded: after this many nanoseconds of %globaltimer
+// (or the iteration cap) the waiter records KVC_ERR_TIMEOUT and goes on. A
+// recorded timeout is sticky: every other wait of the call sees it in the
+// status word and gives up at once, so a failed call ends within about one
+// wait limit.
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t kWaitIters = 1u << 26;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// First error of a call wins.
+__device__ __forceinline__ void set_status(uint32_t *status, uint32_t code) {
+  atomicCAS(status, 0u, code);
+}
+__device__ __forceinline__ bool timed_out(const uint32_t *status) {
+  return *reinterpret_cast<const volatile uint32_t *>(status) == KVC_ERR_TIMEOUT;
+}
+// Poll step of a bounded spin: true means give up (time, iterations, or a
+// timeout already recorded by another waiter). Checks every 64 iterations.
+__device__ __forceinline__ bool spin_expired(uint32_t it, uint64_t t0, const uint32_t *status) {
+  if (it >= kWaitIters) return true;
+  if ((it & 63u) != 63u) return false;
+  return globaltimer() - t0 > kWaitNs || timed_out(status);
+}
+
+// ---------------------------------------------------------------- mbarrier --
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the phase with the given parity; false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const uint32_t *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (spin_expired(i, t0, status)) return false;
+  }
+}
+
+// ---------------------------------------------------- bulk-async copies --
+// global -> shared, completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *sdst, const void *gsrc, uint32_t bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(sdst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// shared -> global, tracked by this thread's bulk groups.
+__device__ __forceinline__ void bulk_s2g(void *gdst, const void *ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later
+// bulk-async reads of them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// ------------------------------------------------------- memory model --
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u64(uint64_t *p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// Invalidates an L2 line without writing it back (its content is dead).
+__device__ __forceinline__ void discard_l2(const void *p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
+// ---------------------------------------------------- fp32 arithmetic --
+// Paired fp32 ops (sm_100 f32x2): each lane of the pair is one IEEE
+// round-to-nearest-even operation, identical to the scalar op.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&r);
+}
+// min / max that return NaN if any input is NaN.
+__device__ __forceinline__ float min3n(float a, float b, float c) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float max3n(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float min2n(float a, float b) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+__device__ __forceinline__ float max2n(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// Walsh-Hadamard butterfly of one head_dim vector held as HALF = d/2 pairs,
+// p[i] = (y[i], y[i + d/2]). Strides h = 1, 2, ..., d/2 in ascending order;
+// each pair (i, i+h) with (i & h) == 0 becomes (a+b, a-b), one rounding each.
+// Strides below d/2 act on both halves at once (paired ops); the last stride
+// pairs the two lanes of each p[i].
+template <int HALF>
+__device__ __forceinline__ void fwht_pairs(float2 (&p)[HALF]) {
+#pragma unroll
+  for (int h = 1; h < HALF; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < HALF; ++i) {
+      if ((i & h) == 0) {
+        const float2 a = p[i], b = p[i + h];
+        p[i] = add2(a, b);
+        p[i + h] = sub2(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) {
+    const float a = p[i].x, b = p[i].y;
+    p[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+}
+
+// In-register transpose of a 32x32 bit matrix: afterwards bit l of a[p] is
+// bit p of the original a[l]. Recursive exchange of off-diagonal blocks of
+// 16, 8, 4, 2 and 1 bits.
+KVC_HD void transpose32(uint32_t (&a)[32]) {
+  const uint32_t masks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+  for (int lvl = 0; lvl < 5; ++lvl) {
+    const int j = 16 >> lvl;
+    const uint32_t m = masks[lvl];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      if ((k & j) == 0) {
+        const uint32_t t = ((a[k] >> j) ^ a[k + j]) & m;
+        a[k] ^= t << j;
+        a[k + j] ^= t;
+      }
+    }
+  }
+}
+
+// -------------------------------------------------------------- scans --
+// Exclusive sum over the kThreads compute threads (named barrier 1); also
+// returns the total. `red` holds kThreads/32 words of shared memory.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *red,
+                                                    uint32_t &total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) red[warp] = incl;
+  named_bar_sync(1, kThreads);
+  uint32_t before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) {
+    const uint32_t r = red[w];
+    before += (w < warp) ? r : 0u;
+    all += r;
+  }
+  named_bar_sync(1, kThreads);
+  total = all;
+  return before + incl - x;
+}
+__device__ __forceinline__ uint32_t block_sum(uint32_t x, uint32_t *red) {
+  uint32_t total;
+  block_excl_scan(x, red, total);
+  return total;
+}
+
+// --------------------------------------------------------- addressing --
+// Dense: v = ((l*2 + kv)*H + h)*T + t.
+__device__ __forceinline__ uint8_t *vec_addr(const DenseLayout &L, const uint32_t *,
+                                             uint32_t v, bool &ok) {
+  const uint32_t lkh = fdiv(L.T, v), t = v - lkh * L.T.d;
+  const uint32_t lk = fdiv(L.H, lkh), h = lkh - lk * L.H.d;
+  ok = true;
+  return L.base + int64_t(lk >> 1) * L.s_l + int64_t(lk & 1u) * L.s_kv + int64_t(h) * L.s_h +
+         int64_t(t) * L.s_t;
+}
+// Paged: v = ((l*2 + kv)*H + h)*Ttot + cum[r] + t; page from the page table.
+__device__ __forceinline__ uint8_t *vec_addr(const PagedLayout &L, const uint32_t *cum,
+                                             uint32_t v, bool &ok) {
+  const uint32_t lkh = fdiv(L.T, v), u = v - lkh * L.T.d;
+  const uint32_t lk = fdiv(L.H, lkh), h = lkh - lk * L.H.d;
+  uint32_t lo = 0, hi = L.n_req - 1;  // largest r with cum[r] <= u
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi + 1) >> 1;
+    if (cum[mid] <= u)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  const uint32_t t = u - cum[lo];
+  const uint32_t pi = fdiv(L.PT, t), slot = t - pi * L.PT.d;
+  const int32_t page = __ldg(L.page_table + int64_t(lo) * L.pt_stride + pi);
+  ok = page >= 0 && int64_t(page) < L.num_pages;
+  return L.base + int64_t(lk >> 1) * L.s_l + int64_t(page) * L.s_p + int64_t(lk & 1u) * L.s_kv +
+         int64_t(h) * L.s_h + int64_t(slot) * L.s_slot;
+}
+
+}  // namespace kvc

@@ -1,0 +1,9 @@
+// Encode instantiations: head_dim 128, paged input.
+#include "kvc_launch.cuh"
+
+namespace kvc {
+cudaError_t launch_encode_paged_d128(int bits, int group, const EncArgs &a, const PagedLayout &lay,
+                                  int sms, cudaStream_t st) {
+  return launch_enc_dispatch<128>(bits, group, a, lay, sms, st);
+}
+}  // namespace kvc

@@ -1,0 +1,9 @@
+// Encode instantiations: head_dim 64, dense input.
+#include "kvc_launch.cuh"
+
+namespace kvc {
+cudaError_t launch_encode_dense_d64(int bits, int group, const EncArgs &a, const DenseLayout &lay,
+                                  int sms, cudaStream_t st) {
+  return launch_enc_dispatch<64>(bits, group, a, lay, sms, st);
+}
+}  // namespace kvc

@@ -1,0 +1,9 @@
+// Encode instantiations: head_dim 64, paged input.
+#include "kvc_launch.cuh"
+
+namespace kvc {
+cudaError_t launch_encode_paged_d64(int bits, int group, const EncArgs &a, const PagedLayout &lay,
+                                  int sms, cudaStream_t st) {
+  return launch_enc_dispatch<64>(bits, group, a, lay, sms, st);
+}
+}  // namespace kvc

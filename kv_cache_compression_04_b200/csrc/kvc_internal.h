@@ -1,0 +1,141 @@
+// Definitions shared by the host launcher and the sm_100a kernels of libkvc.
+//
+// Stream format and arithmetic follow the readings stated in include/kvc.h:
+// stage list from "Beyond Compression Ratio: High-Throughput KV Compression
+// for Disaggregated LLM Serving" (Abstract, Methodology) and the podcast page
+// "FastKVComp: checking whether high-throughput KV compression pays off"
+// (episode notes); exact rules are this library's readings.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kvc.h"
+
+#if defined(__CUDACC__)
+#define KVC_HD __host__ __device__ __forceinline__
+#else
+#define KVC_HD inline
+#endif
+
+namespace kvc {
+
+constexpr int kChunk = 16384;   // lossless chunk bytes
+constexpr int kBitmap = 2048;   // zero-byte-elimination bitmap bytes
+constexpr int kHeader = 64;     // stream header bytes
+constexpr uint32_t kMagic = 0x3143564Bu;  // "KVC1"
+constexpr int kThreads = 256;   // compute threads per CTA (one vector each)
+constexpr uint32_t kNoTile = 0xFFFFFFFFu;
+
+// Workspace layout of kvc_compress: [status, ticket, ...] control block,
+// then one u64 look-back word per tile, then one 16 KB meta staging chunk per
+// segment. Only the first two parts need zeroing per call.
+constexpr size_t kWsCtl = 256;
+
+KVC_HD uint64_t round16(uint64_t x) { return (x + 15u) & ~uint64_t(15); }
+KVC_HD uint64_t round256(uint64_t x) { return (x + 255u) & ~uint64_t(255); }
+
+// SplitMix64 (Steele, Lea, Flood, OOPSLA 2014): sign words of the +-1
+// diagonal are its outputs counted from state = seed.
+KVC_HD uint64_t splitmix64(uint64_t &state) {
+  state += 0x9E3779B97F4A7C15ull;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// XOR masks that flip the bf16 sign bits of channel pair (2j, 2j+1).
+KVC_HD void sign_masks(uint64_t seed, int d, uint32_t *mask) {
+  uint64_t st = seed, w = 0;
+  for (int c = 0; c < d; c += 2) {
+    if (c % 64 == 0) w = splitmix64(st);
+    uint32_t lo = uint32_t((w >> (c % 64)) & 1u), hi = uint32_t((w >> (c % 64 + 1)) & 1u);
+    mask[c / 2] = (lo << 15) | (hi << 31);
+  }
+}
+
+// Unsigned 32-bit division by a run-time constant (Granlund and Montgomery,
+// "Division by invariant integers using multiplication", PLDI 1994, the
+// round-up variant): q = (umulhi(n, m) + n) >> s, exact for every n < 2^32.
+struct FastDiv {
+  uint32_t d, m, s;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{d, 0, 0};
+  uint32_t l = 0;
+  while ((uint64_t(1) << l) < d) l++;
+  f.s = l;
+  f.m = uint32_t(((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1);
+  return f;
+}
+KVC_HD uint32_t fdiv(const FastDiv &f, uint32_t n) {
+  uint32_t hi = uint32_t((uint64_t(n) * f.m) >> 32);
+  return uint32_t((uint64_t(hi) + n) >> f.s);
+}
+
+// Vector addressing. Vector v (logical order [layer][kv][head][request]
+// [token]) -> byte address of its head_dim contiguous bf16 values.
+struct DenseLayout {
+  uint8_t *base;
+  int64_t s_l, s_kv, s_h, s_t;  // bytes
+  FastDiv T, H;                 // tokens, kv_heads
+  uint32_t tokens;
+};
+
+struct PagedLayout {
+  uint8_t *base;
+  int64_t s_l, s_p, s_kv, s_h, s_slot;  // bytes
+  const int32_t *page_table;
+  int64_t pt_stride;
+  int64_t num_pages;
+  FastDiv T, H, PT;                     // total tokens, kv_heads, page tokens
+  uint32_t n_req;
+  uint32_t cum[KVC_MAX_REQUESTS + 1];   // token prefix per request
+};
+
+struct EncArgs {
+  uint32_t V;          // vectors
+  uint32_t n_tiles;    // code chunks (one tile = one code chunk)
+  uint32_t n_seg;      // segments = meta chunks
+  uint32_t n_chunks;
+  uint8_t *out;
+  uint64_t out_capacity;
+  uint64_t data_base;
+  uint64_t *out_bytes_dev;
+  uint32_t *status;
+  uint32_t *ticket;
+  uint64_t *tile_state;
+  uint8_t *ws_meta;
+  // header fields
+  uint32_t layers, kv_heads, head_dim, group, bits, k, origin, n_req;
+  uint64_t tokens, seed;
+  uint32_t sign_mask[128];
+};
+
+struct DecArgs {
+  const uint8_t *in;
+  uint64_t in_bytes;
+  uint32_t *status;
+  uint32_t layers, kv_heads, head_dim, n_req;
+  uint64_t tokens;
+  uint32_t V;
+  uint32_t paged_receiver;   // 1: request count and lengths must match
+};
+
+// Launchers, one translation unit per (head_dim, layout).
+#define KVC_DECLARE_LAUNCHERS(D)                                                          \
+  cudaError_t launch_encode_dense_d##D(int bits, int group, const EncArgs &a,             \
+                                       const DenseLayout &lay, int sms, cudaStream_t st); \
+  cudaError_t launch_encode_paged_d##D(int bits, int group, const EncArgs &a,             \
+                                       const PagedLayout &lay, int sms, cudaStream_t st); \
+  cudaError_t launch_decode_dense_d##D(const DecArgs &a, const DenseLayout &lay, int sms, \
+                                       cudaStream_t st);                                  \
+  cudaError_t launch_decode_paged_d##D(const DecArgs &a, const PagedLayout &lay, int sms, \
+                                       cudaStream_t st);
+KVC_DECLARE_LAUNCHERS(128)
+KVC_DECLARE_LAUNCHERS(64)
+#undef KVC_DECLARE_LAUNCHERS
+
+}  // namespace kvc

@@ -1,0 +1,68 @@
+// Launch helpers shared by the per-head_dim translation units.
+#pragma once
+
+#include <atomic>
+
+#include "kvc_decode.cuh"
+
+namespace kvc {
+
+// Opt each instantiation into large dynamic shared memory once per device.
+template <class Kernel>
+inline cudaError_t prepare(Kernel k, size_t smem) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+template <int D, int BITS, int G, class Layout>
+cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
+  auto k = encode_kernel<D, BITS, G, Layout>;
+  const size_t smem = enc_smem_bytes<D, BITS, G>(kIsPaged<Layout>);
+  cudaError_t e = prepare(k, smem);
+  if (e != cudaSuccess) return e;
+  const int grid = a.n_tiles == 0 ? 1 : int(a.n_tiles < uint32_t(sms) ? a.n_tiles : uint32_t(sms));
+  k<<<grid, kThreads + 32, smem, st>>>(a, lay);
+  return cudaGetLastError();
+}
+
+template <int D, class Layout>
+cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_t st) {
+  auto k = decode_kernel<D, Layout>;
+  const size_t smem = dec_smem_bytes<D>(kIsPaged<Layout>);
+  cudaError_t e = prepare(k, smem);
+  if (e != cudaSuccess) return e;
+  // one CTA per SM; tiles are the code chunks (at least 128 vectors each)
+  const uint64_t min_vc = uint64_t(kChunk) / (uint64_t(D) * 4 / 8);
+  const uint64_t tiles = (uint64_t(a.V) + min_vc - 1) / min_vc;
+  const int grid = tiles == 0 ? 1 : int(tiles < uint64_t(sms) ? tiles : uint64_t(sms));
+  k<<<grid, kThreads, smem, st>>>(a, lay);
+  return cudaGetLastError();
+}
+
+template <int D, class Layout>
+cudaError_t launch_enc_dispatch(int bits, int group, const EncArgs &a, const Layout &lay, int sms,
+                                cudaStream_t st) {
+  if constexpr (D == 128) {
+    if (bits == 4 && group == 128) return launch_enc<128, 4, 128>(a, lay, sms, st);
+    if (bits == 4 && group == 64) return launch_enc<128, 4, 64>(a, lay, sms, st);
+    if (bits == 4 && group == 32) return launch_enc<128, 4, 32>(a, lay, sms, st);
+    if (bits == 2 && group == 128) return launch_enc<128, 2, 128>(a, lay, sms, st);
+    if (bits == 2 && group == 64) return launch_enc<128, 2, 64>(a, lay, sms, st);
+    if (bits == 2 && group == 32) return launch_enc<128, 2, 32>(a, lay, sms, st);
+  } else {
+    if (bits == 4 && group == 64) return launch_enc<64, 4, 64>(a, lay, sms, st);
+    if (bits == 4 && group == 32) return launch_enc<64, 4, 32>(a, lay, sms, st);
+    if (bits == 2 && group == 64) return launch_enc<64, 2, 64>(a, lay, sms, st);
+    if (bits == 2 && group == 32) return launch_enc<64, 2, 32>(a, lay, sms, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kvc

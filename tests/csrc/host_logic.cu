@@ -1,0 +1,14 @@
+// Host-side exports of the library's host/device helpers (compiled host-only
+// by the tests): fast division, the 32x32 bit transpose, sign masks.
+#include "../../kv_cache_compression_04_b200/csrc/kvc_device.cuh"
+
+extern "C" {
+uint32_t hl_fdiv(uint32_t d, uint32_t n) { return kvc::fdiv(kvc::make_fastdiv(d), n); }
+void hl_transpose32(const uint32_t *in, uint32_t *out) {
+  uint32_t a[32];
+  for (int i = 0; i < 32; ++i) a[i] = in[i];
+  kvc::transpose32(a);
+  for (int i = 0; i < 32; ++i) out[i] = a[i];
+}
+void hl_sign_masks(uint64_t seed, int d, uint32_t *out) { kvc::sign_masks(seed, d, out); }
+}

@@ -1,0 +1,200 @@
+"""The C ABI without a GPU: libkvc.so loads and exports every declared symbol,
+host-pure sizing agrees with the oracle's independent layout arithmetic,
+invalid arguments are refused before anything is enqueued, and the host
+helpers (fast division, bit transpose, sign masks) are exact."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import kv_cache_compression_04_b200 as kvc
+from kv_cache_compression_04_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return kvc.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    with open(os.path.join(ROOT, "include", "kvc.h")) as f:
+        hdr = f.read()
+    declared = set(re.findall(r"\b(kvc_[a-z_]+)\s*\(", hdr))
+    assert declared == set(kvc.EXPORTS)
+    for name in declared:
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", kvc.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    for name in declared:
+        assert re.search(rf"\bT {name}$", out, re.M), name
+
+
+def test_status_strings(L):
+    for i, name in enumerate(kvc.STATUS):
+        assert kvc.kvc_status_string(i) == name
+    assert kvc.kvc_status_string(99) == "KVC_ERR_UNKNOWN"
+
+
+FAKE = 0x7F0000000000  # never dereferenced: validation happens on the host
+
+
+def dense(L_, H, T, D, data=FAKE):
+    d = kvc.kvc_kv_desc()
+    d.kind, d.layers, d.kv_heads, d.head_dim = kvc.KVC_DENSE, L_, H, D
+    d.data = data
+    d.stride_token = D
+    d.stride_head = T * D
+    d.stride_kv = H * T * D
+    d.stride_layer = 2 * H * T * D
+    d.tokens = T
+    return d
+
+
+def paged(L_, H, D, seq, pt_stride=None, page_tokens=16):
+    d = kvc.kvc_kv_desc()
+    d.kind, d.layers, d.kv_heads, d.head_dim = kvc.KVC_PAGED, L_, H, D
+    d.data = FAKE
+    d.stride_slot = D
+    d.stride_head = page_tokens * D
+    d.stride_kv = H * page_tokens * D
+    d.stride_page = 2 * H * page_tokens * D
+    npages = sum((s + page_tokens - 1) // page_tokens for s in seq) + 1
+    d.stride_layer = npages * d.stride_page
+    d.page_tokens, d.n_requests, d.num_pages = page_tokens, len(seq), npages
+    arr = (C.c_int32 * max(1, len(seq)))(*seq)
+    d.seq_lens = C.cast(arr, C.POINTER(C.c_int32))
+    d.page_table = FAKE
+    d.page_table_stride = pt_stride if pt_stride is not None else max(
+        [(s + page_tokens - 1) // page_tokens for s in seq] + [1])
+    d._keep = (arr,)
+    return d
+
+
+SHAPES = [(1, 8, 64, 128, 4, 128), (32, 8, 4096, 128, 4, 128), (28, 4, 32768, 128, 2, 32),
+          (2, 3, 1000, 128, 4, 64), (1, 1, 1, 64, 2, 64), (3, 2, 777, 64, 4, 32),
+          (2, 8, 0, 128, 4, 128), (0, 8, 16, 128, 2, 32), (5, 1, 513, 128, 2, 128)]
+
+
+@pytest.mark.parametrize("Ln,H,T,D,bits,g", SHAPES)
+def test_max_bytes_matches_oracle_dense(L, Ln, H, T, D, bits, g):
+    p = kvc.params(bits, g)
+    od = oracle.StreamDesc(bits, g, D, Ln, H, [T])
+    assert kvc.kvc_max_compressed_bytes(dense(Ln, H, T, D), p) == od.max_bytes()
+    lay = od.layout()
+    ws = kvc.kvc_workspace_bytes(dense(Ln, H, T, D), p)
+    assert ws >= 8 * lay.n_code + 16384 * lay.n_meta
+
+
+@pytest.mark.parametrize("seq,bits,g", [([20, 0, 33, 16], 4, 64), ([512, 8192, 3000], 2, 32),
+                                        ([0], 4, 128), ([1] * 1024, 2, 64)])
+def test_max_bytes_matches_oracle_paged(L, seq, bits, g):
+    p = kvc.params(bits, g)
+    od = oracle.StreamDesc(bits, g, 128, 3, 2, seq)
+    assert kvc.kvc_max_compressed_bytes(paged(3, 2, 128, seq), p) == od.max_bytes()
+
+
+def _compress(d, p, out=FAKE, cap=1 << 40, ws=FAKE, wsb=1 << 40):
+    return kvc.kvc_compress(d, p, out, cap, None, ws, wsb, None)
+
+
+def test_invalid_arguments_refused_on_host(L):
+    p = kvc.params(4, 128)
+    d = dense(2, 2, 64, 128)
+    assert _compress(d, kvc.params(3, 128)) == kvc.KVC_ERR_UNSUPPORTED
+    assert _compress(d, kvc.params(4, 48)) == kvc.KVC_ERR_UNSUPPORTED
+    assert _compress(dense(2, 2, 64, 64), kvc.params(4, 128)) == kvc.KVC_ERR_UNSUPPORTED
+    assert _compress(dense(2, 2, 64, 96), p) == kvc.KVC_ERR_UNSUPPORTED
+    assert _compress(dense(2, 2, 64, 256), p) == kvc.KVC_ERR_UNSUPPORTED
+    assert _compress(d, p, out=FAKE + 8) == kvc.KVC_ERR_INVALID_ARG
+    assert _compress(d, p, ws=FAKE + 4) == kvc.KVC_ERR_INVALID_ARG
+    assert _compress(d, p, out=None) == kvc.KVC_ERR_INVALID_ARG
+    assert _compress(dense(2, 2, 64, 128, data=FAKE + 2), p) == kvc.KVC_ERR_INVALID_ARG
+    need = kvc.kvc_max_compressed_bytes(d, p)
+    assert _compress(d, p, cap=need - 1) == kvc.KVC_ERR_CAPACITY
+    assert _compress(d, p, wsb=kvc.kvc_workspace_bytes(d, p) - 1) == kvc.KVC_ERR_CAPACITY
+    bad = dense(2, 2, 64, 128)
+    bad.stride_token = 132                               # 264 B: not 16-byte aligned
+    assert _compress(bad, p) == kvc.KVC_ERR_INVALID_ARG
+    bad = dense(2, 2, 64, 128)
+    bad.kind = 7
+    assert _compress(bad, p) == kvc.KVC_ERR_INVALID_ARG
+    bad = dense(2, 2, 64, 128)
+    bad.tokens = -1
+    assert _compress(bad, p) == kvc.KVC_ERR_INVALID_ARG
+    assert kvc.lib().kvc_compress(None, C.byref(p), FAKE, 1 << 40, None, FAKE, 1 << 40,
+                                  None) == kvc.KVC_ERR_INVALID_ARG
+    # paged
+    assert _compress(paged(2, 2, 128, [5] * 1025), p) == kvc.KVC_ERR_INVALID_ARG
+    assert _compress(paged(2, 2, 128, [5, -1]), p) == kvc.KVC_ERR_INVALID_ARG
+    assert _compress(paged(2, 2, 128, [40, 3], pt_stride=2), p) == kvc.KVC_ERR_INVALID_ARG
+    pg = paged(2, 2, 128, [40, 3])
+    pg.page_tokens = 0
+    assert _compress(pg, p) == kvc.KVC_ERR_INVALID_ARG
+    # too many vectors for 32-bit indexing
+    assert _compress(dense(1 << 10, 8, 1 << 20, 128), p) == kvc.KVC_ERR_UNSUPPORTED
+    assert kvc.kvc_max_compressed_bytes(dense(2, 2, 64, 96), p) == 0
+    assert kvc.kvc_workspace_bytes(dense(2, 2, 64, 96), p) == 0
+
+
+def test_decompress_refuses_bad_arguments_on_host(L):
+    d = dense(2, 2, 64, 128)
+    assert kvc.kvc_decompress(FAKE + 8, 100, d, FAKE, 256, None) == kvc.KVC_ERR_INVALID_ARG
+    assert kvc.kvc_decompress(FAKE, 100, d, FAKE, 255, None) == kvc.KVC_ERR_CAPACITY
+    assert kvc.kvc_decompress(FAKE, 100, dense(2, 2, 64, 96), FAKE, 256,
+                              None) == kvc.KVC_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------ host helpers --
+@pytest.fixture(scope="module")
+def host_logic():
+    out = os.path.join(ROOT, "tests", "_build")
+    os.makedirs(out, exist_ok=True)
+    so = os.path.join(out, f"host_logic_{os.getpid()}.so")
+    subprocess.run([build.nvcc(), *build.ARCH, "-std=c++17", "-O2", "-Xcompiler", "-fPIC", "-shared",
+                    os.path.join(ROOT, "tests", "csrc", "host_logic.cu"), "-o", so], check=True)
+    lib = C.CDLL(so)
+    os.unlink(so)
+    lib.hl_fdiv.restype = C.c_uint32
+    lib.hl_fdiv.argtypes = [C.c_uint32, C.c_uint32]
+    lib.hl_transpose32.argtypes = [C.c_void_p, C.c_void_p]
+    lib.hl_sign_masks.argtypes = [C.c_uint64, C.c_int, C.c_void_p]
+    return lib
+
+
+def test_fast_division_exact(host_logic):
+    rng = np.random.default_rng(0)
+    divisors = list(range(1, 300)) + [1000, 4096, 4352, 32768, 69632, 2 ** 20 + 7,
+                                      2 ** 30 - 1, 2 ** 30, 2 ** 31 - 1]
+    ns = [0, 1, 2 ** 31 - 1, 2 ** 31, 2 ** 32 - 1] + list(rng.integers(0, 2 ** 32, 300))
+    for dv in divisors:
+        for n in ns:
+            assert host_logic.hl_fdiv(dv, int(n)) == int(n) // dv, (dv, n)
+
+
+def test_transpose32_is_bit_matrix_transpose(host_logic):
+    rng = np.random.default_rng(1)
+    for _ in range(20):
+        a = rng.integers(0, 2 ** 32, 32, dtype=np.uint64).astype(np.uint32)
+        out = np.zeros(32, np.uint32)
+        host_logic.hl_transpose32(a.ctypes.data, out.ctypes.data)
+        bits = (a[:, None] >> np.arange(32, dtype=np.uint32)) & 1       # [row l, bit p]
+        want = (bits.T.astype(np.uint64) << np.arange(32, dtype=np.uint64)).sum(1)
+        assert np.array_equal(out, want.astype(np.uint32))
+
+
+@pytest.mark.parametrize("seed,d", [(0, 128), (12345, 64), (2 ** 63 + 5, 128)])
+def test_sign_masks_match_oracle_sign_words(host_logic, seed, d):
+    m = np.zeros(d // 2, np.uint32)
+    host_logic.hl_sign_masks(seed, d, m.ctypes.data)
+    w = [int(x) for x in oracle.sign_words(seed, d)]
+    for j in range(d // 2):
+        lo = (w[(2 * j) // 64] >> ((2 * j) % 64)) & 1
+        hi = (w[(2 * j + 1) // 64] >> ((2 * j + 1) % 64)) & 1
+        assert m[j] == (lo << 15) | (hi << 31)
