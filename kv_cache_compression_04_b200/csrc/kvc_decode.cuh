@@ -126,7 +126,9 @@ struct Dec : Cfg<D, BITS, G> {
       const float2 q = sub2(make_float2(__uint_as_float(kMagicBits | qa), __uint_as_float(kMagicBits | qb)),
                             make_float2(kMagic, kMagic));
       const int ga = ca / G, gb = cb / G;
-      p[i] = add2(make_float2(zf[ga], zf[gb]), mul2(q, make_float2(sf[ga], sf[gb])));
+      // q * sf is exact (q < 16 times an fp16 value times 2^K needs at most 15
+      // significant bits), so one fused rounding equals fl(zf + fl(q * sf)).
+      p[i] = fma2(q, make_float2(sf[ga], sf[gb]), make_float2(zf[ga], zf[gb]));
     }
     fwht_pairs<C::HALF>(p);
     const float inv = 1.0f / float(D);

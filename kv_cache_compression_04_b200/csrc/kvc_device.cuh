@@ -132,17 +132,37 @@ __device__ __forceinline__ void discard_l2(const void *p) {
 }
 
 // ---------------------------------------------------- fp32 arithmetic --
-// Paired fp32 ops (sm_100 f32x2): each lane of the pair is one IEEE
-// round-to-nearest-even operation, identical to the scalar op.
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+// Paired fp32 ops (sm_100 f32x2): each lane is one IEEE round-to-nearest-even
+// operation. Written as PTX with an explicit .rn modifier, which the compiler
+// never contracts into a fused multiply-add (the codec's bit-exactness
+// depends on every product and sum being rounded separately).
+__device__ __forceinline__ uint64_t f2_bits(float2 a) { return *reinterpret_cast<uint64_t *>(&a); }
+__device__ __forceinline__ float2 bits_f2(uint64_t r) { return *reinterpret_cast<float2 *>(&r); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(r);
+}
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;"
-      : "=l"(r)
-      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
-  return *reinterpret_cast<float2 *>(&r);
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(r);
 }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(r);
+}
+// a*b + c with one rounding. Used only where a*b is exact, so the result
+// equals the separately rounded product-then-sum.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(r);
+}
+// Measured on sm_100a: a paired multiply followed by a paired add can be
+// fused even when both carry .rn, so no product that needs its own rounding
+// feeds an add here; products are rounded to integers with cvt.rni instead.
 // min / max that return NaN if any input is NaN.
 __device__ __forceinline__ float min3n(float a, float b, float c) {
   float d;

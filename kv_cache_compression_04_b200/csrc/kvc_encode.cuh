@@ -128,15 +128,15 @@ struct Enc : Cfg<D, BITS, G> {
       nzf[g] = zf;
       meta[g] = uint32_t(sb) | (uint32_t(zb) << 16);
     }
-    // E6: q = RNE((y - zf) * r). (y - zf) >= 0 and (y - zf) * r < 2^b - 0.5
-    // for every finite group (zf <= min, sf >= (max - zf)/(2^b-1)), so adding
-    // 1.5*2^23 leaves q in the low mantissa bits with no clamp needed.
-    constexpr float kMagic = 12582912.0f;
+    // E6: q = RNE(fl(fl(y - zf) * r)) by cvt.rni on the rounded product. The
+    // clamp to [0, 2^b - 1] never acts for a finite group: y - zf >= 0 since
+    // zf <= min, and sf >= (max - zf)/(2^b - 1) bounds the product below
+    // 2^b - 1 + 2^-20, so the integers are stored as they come.
 #pragma unroll
     for (int i = 0; i < C::HALF; ++i) {
       const int ga = i / G, gb = (i + C::HALF) / G;
       const float2 t = mul2(sub2(p[i], make_float2(nzf[ga], nzf[gb])), make_float2(rr[ga], rr[gb]));
-      p[i] = add2(t, make_float2(kMagic, kMagic));
+      p[i] = make_float2(__int_as_float(__float2int_rn(t.x)), __int_as_float(__float2int_rn(t.y)));
     }
     // E7: pack (reading R6), channel order, LSB first.
 #pragma unroll

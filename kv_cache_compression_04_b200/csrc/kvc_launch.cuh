@@ -8,7 +8,8 @@
 namespace kvc {
 
 // Opt each instantiation into large dynamic shared memory once per device.
-template <class Kernel>
+// `Tag` makes the flag per kernel instantiation (kernels share a pointer type).
+template <class Tag, class Kernel>
 inline cudaError_t prepare(Kernel k, size_t smem) {
   static std::atomic<uint64_t> done{0};
   int dev = 0;
@@ -25,7 +26,8 @@ template <int D, int BITS, int G, class Layout>
 cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
   auto k = encode_kernel<D, BITS, G, Layout>;
   const size_t smem = enc_smem_bytes<D, BITS, G>(kIsPaged<Layout>);
-  cudaError_t e = prepare(k, smem);
+  struct Tag {};
+  cudaError_t e = prepare<Tag>(k, smem);
   if (e != cudaSuccess) return e;
   const int grid = a.n_tiles == 0 ? 1 : int(a.n_tiles < uint32_t(sms) ? a.n_tiles : uint32_t(sms));
   k<<<grid, kThreads + 32, smem, st>>>(a, lay);
@@ -36,7 +38,8 @@ template <int D, class Layout>
 cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_t st) {
   auto k = decode_kernel<D, Layout>;
   const size_t smem = dec_smem_bytes<D>(kIsPaged<Layout>);
-  cudaError_t e = prepare(k, smem);
+  struct Tag {};
+  cudaError_t e = prepare<Tag>(k, smem);
   if (e != cudaSuccess) return e;
   // one CTA per SM; tiles are the code chunks (at least 128 vectors each)
   const uint64_t min_vc = uint64_t(kChunk) / (uint64_t(D) * 4 / 8);
