@@ -391,10 +391,10 @@ int orc_lossless_decode_chunk(const uint8_t *in, uint32_t size, uint32_t len,
 /*   then      zeros up to a 16-byte boundary = data base;                    */
 /*   then      the chunks, each zero-padded to 16 bytes, at their offsets.    */
 /* The codes region (packed codes of all vectors in logical order) and the    */
-/* meta region (4 bytes per group) are cut into 16 KB chunks separately. A    */
-/* meta chunk covers R = g*b/32 code chunks; stream order is segment by       */
-/* segment: the R code chunks of a segment, then its meta chunk. Chunk        */
-/* offsets are the exclusive prefix sum of the padded chunk sizes.            */
+/* meta region (4 bytes per group) are cut into 16 KB chunks separately (a    */
+/* meta chunk covers R = g*b/32 code chunks: a "segment"). Stream order is    */
+/* every code chunk, then every meta chunk. Chunk offsets are the exclusive   */
+/* prefix sum of the padded chunk sizes in that order.                        */
 /* ========================================================================== */
 static uint64_t round16(uint64_t x) { return (x + 15u) & ~(uint64_t)15u; }
 
@@ -454,13 +454,12 @@ uint64_t orc_max_compressed_bytes(const orc_desc *d) {
 }
 
 uint64_t orc_code_chunk_index(const orc_layout *lay, uint64_t c) {
-  return c + c / lay->code_per_seg;
+  (void)lay;
+  return c;
 }
 
 uint64_t orc_meta_chunk_index(const orc_layout *lay, uint64_t s) {
-  uint64_t end = (s + 1) * lay->code_per_seg;
-  if (end > lay->n_code) end = lay->n_code;
-  return end + s;
+  return lay->n_code + s;
 }
 
 static void put16(uint8_t *p, uint16_t v) {
@@ -567,9 +566,10 @@ int orc_decode_segment(const orc_desc *d, uint64_t s, const uint8_t *chunks,
 int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
                  uint64_t capacity, uint64_t *out_bytes) {
   orc_layout lay;
-  uint64_t s, off = 0, T = 0, vm;
-  uint8_t *seg;
-  uint32_t sizes[17], n, i;
+  uint64_t s, off = 0, T = 0, vm, i;
+  uint8_t *seg, *store;
+  uint32_t sizes[17], n, k, *all_sizes;
+  uint64_t *where; /* chunk index -> position in store */
   int st = orc_layout_of(d, &lay), sst, r;
   if (st != ORC_OK) return st;
   if (capacity < lay.max_bytes) return ORC_ERR_CAPACITY;
@@ -593,23 +593,37 @@ int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
   put32(out + 52, (uint32_t)lay.n_chunks);
   for (r = 0; r < d->n_requests; r++)
     put32(out + ORC_HEADER + 8 * lay.n_chunks + 4 * r, d->token_lens[r]);
+  /* encode every segment, remembering where each chunk's bytes are */
   vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
   seg = (uint8_t *)malloc((size_t)(lay.code_per_seg + 1) * ORC_CHUNK);
+  store = (uint8_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1) * ORC_CHUNK);
+  all_sizes = (uint32_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1) * 4);
+  where = (uint64_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1) * 8);
   for (s = 0; s < lay.n_seg; s++) {
-    uint64_t first = orc_code_chunk_index(&lay, s * lay.code_per_seg);
     uint32_t pos = 0;
     sst = orc_encode_segment(d, s, vectors + s * vm * d->head_dim, seg, sizes, &n);
     if (sst != ORC_OK && st == ORC_OK) st = sst;
-    for (i = 0; i < n; i++) {
-      uint64_t padded = round16(sizes[i]);
-      put64(out + ORC_HEADER + 8 * (first + i), ((off / 16) << 16) | sizes[i]);
-      memset(out + lay.data_base + off, 0, (size_t)padded);
-      memcpy(out + lay.data_base + off, seg + pos, sizes[i]);
-      pos += sizes[i];
-      off += padded;
+    for (k = 0; k < n; k++) {
+      uint64_t idx = (k + 1 < n) ? orc_code_chunk_index(&lay, s * lay.code_per_seg + k)
+                                 : orc_meta_chunk_index(&lay, s);
+      memcpy(store + idx * ORC_CHUNK, seg + pos, sizes[k]);
+      all_sizes[idx] = sizes[k];
+      where[idx] = idx * ORC_CHUNK;
+      pos += sizes[k];
     }
   }
+  /* lay the chunks out in index order */
+  for (i = 0; i < lay.n_chunks; i++) {
+    uint64_t padded = round16(all_sizes[i]);
+    put64(out + ORC_HEADER + 8 * i, ((off / 16) << 16) | all_sizes[i]);
+    memset(out + lay.data_base + off, 0, (size_t)padded);
+    memcpy(out + lay.data_base + off, store + where[i], all_sizes[i]);
+    off += padded;
+  }
   free(seg);
+  free(store);
+  free(all_sizes);
+  free(where);
   put64(out + 56, lay.data_base + off);
   *out_bytes = lay.data_base + off;
   return st;
@@ -642,30 +656,31 @@ int orc_decompress(const uint8_t *stream, uint64_t stream_bytes,
     if (get32(stream + ORC_HEADER + 8 * lay.n_chunks + 4 * r) !=
         expect->token_lens[r])
       return ORC_ERR_CORRUPT;
+  /* the table: offsets are the prefix sum of padded sizes, in index order */
+  for (s = 0; s < lay.n_chunks; s++) {
+    uint64_t e = get64(stream + ORC_HEADER + 8 * s);
+    uint32_t sz = (uint32_t)(e & 0xFFFFu);
+    uint64_t off = (e >> 16) * 16;
+    if (off != expect_off || sz > ORC_CHUNK || lay.data_base + off + round16(sz) > total)
+      return ORC_ERR_CORRUPT;
+    expect_off = off + round16(sz);
+  }
   vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
   seg = (uint8_t *)malloc((size_t)(lay.code_per_seg + 1) * ORC_CHUNK);
   for (s = 0; s < lay.n_seg && st == ORC_OK; s++) {
-    uint64_t first = orc_code_chunk_index(&lay, s * lay.code_per_seg);
-    uint64_t last = orc_meta_chunk_index(&lay, s);
-    uint64_t i;
+    uint64_t c0 = s * lay.code_per_seg;
+    uint64_t c1 = c0 + lay.code_per_seg < lay.n_code ? c0 + lay.code_per_seg : lay.n_code;
+    uint64_t i, k = 0;
     uint32_t pos = 0;
-    for (i = first; i <= last; i++) {
-      uint64_t e = get64(stream + ORC_HEADER + 8 * i);
+    for (i = c0; i <= c1; i++, k++) { /* code chunks c0..c1-1, then the meta chunk */
+      uint64_t idx = i < c1 ? orc_code_chunk_index(&lay, i) : orc_meta_chunk_index(&lay, s);
+      uint64_t e = get64(stream + ORC_HEADER + 8 * idx);
       uint32_t sz = (uint32_t)(e & 0xFFFFu);
-      uint64_t off = (e >> 16) * 16;
-      if (off != expect_off || sz > ORC_CHUNK ||
-          lay.data_base + off + round16(sz) > total) {
-        st = ORC_ERR_CORRUPT;
-        break;
-      }
-      memcpy(seg + pos, stream + lay.data_base + off, sz);
-      sizes[i - first] = sz;
+      memcpy(seg + pos, stream + lay.data_base + (e >> 16) * 16, sz);
+      sizes[k] = sz;
       pos += sz;
-      expect_off = off + round16(sz);
     }
-    if (st == ORC_OK)
-      st = orc_decode_segment(expect, s, seg, sizes,
-                              vectors + s * vm * expect->head_dim);
+    st = orc_decode_segment(expect, s, seg, sizes, vectors + s * vm * expect->head_dim);
   }
   free(seg);
   if (st == ORC_OK && lay.data_base + expect_off != total) st = ORC_ERR_CORRUPT;

@@ -196,12 +196,12 @@ def _segment_check(w, od, gstream, x_of_range, segs):
         v0, v1 = oracle.segment_vectors(lay, s)
         st, chunks = oracle.encode_segment(od, s, x_of_range(v0, v1))
         assert st == oracle.OK
-        first = oracle.code_chunk_index(lay, s * lay.code_per_seg)
-        for i, ch in enumerate(chunks):
-            ci = first + i
-            assert sizes[ci] == ch.size, (s, i)
+        idx = [oracle.code_chunk_index(lay, s * lay.code_per_seg + i)
+               for i in range(len(chunks) - 1)] + [oracle.meta_chunk_index(lay, s)]
+        for ch, ci in zip(chunks, idx):
+            assert sizes[ci] == ch.size, (s, ci)
             a = lay.data_base + offs[ci]
-            assert np.array_equal(gstream[a:a + ch.size], ch), (s, i)
+            assert np.array_equal(gstream[a:a + ch.size], ch), (s, ci)
     return sizes, offs
 
 

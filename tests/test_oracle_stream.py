@@ -62,14 +62,14 @@ def test_layout_counts(name, n_code, n_meta):
     assert lay.code_per_seg == w.group * w.bits // 32
 
 
-def test_chunk_order_is_segment_by_segment():
+def test_chunk_order_codes_then_meta():
     lay = oracle.StreamDesc(2, 32, 128, 1, 1, [1250]).layout()   # V = 2500, R = 2
     assert lay.code_per_seg == 2 and lay.n_code == 5 and lay.n_meta == 3
     idx = sorted([("c", c, oracle.code_chunk_index(lay, c)) for c in range(5)] +
                  [("m", s, oracle.meta_chunk_index(lay, s)) for s in range(3)],
                  key=lambda t: t[2])
-    assert [(k, i) for k, i, _ in idx] == [("c", 0), ("c", 1), ("m", 0), ("c", 2),
-                                           ("c", 3), ("m", 1), ("c", 4), ("m", 2)]
+    assert [(k, i) for k, i, _ in idx] == [("c", 0), ("c", 1), ("c", 2), ("c", 3),
+                                           ("c", 4), ("m", 0), ("m", 1), ("m", 2)]
     assert [t[2] for t in idx] == list(range(8))
 
 
@@ -98,19 +98,28 @@ def test_roundtrip_error_bound_tiny():
 
 
 def test_stream_is_deterministic_and_segments_agree():
-    w, d, x = tiny_desc_and_vectors()
+    """Three segments (R = 2 code chunks per meta chunk at 2-bit, group 32):
+    each chunk of encode_segment sits in the stream at the index the layout
+    gives it, and offsets are the prefix sum of padded sizes."""
+    w = synth.Workload("t", 1, 2, 128, 2, 32, seed=3, kind="lognormal", tokens=600)
+    x = synth.bf16_bits(synth.dense_kv(w)).reshape(-1, 128)
+    d = oracle.StreamDesc(2, 32, 128, 1, 2, [600])
     st1, s1 = oracle.compress(d, x)
     st2, s2 = oracle.compress(d, x)
-    assert np.array_equal(s1, s2)
+    assert st1 == oracle.OK and np.array_equal(s1, s2)
     lay = d.layout()
-    st, chunks = oracle.encode_segment(d, 0, x)
-    base = lay.data_base
-    off = 0
-    for i, ch in enumerate(chunks):
-        e = _u(s1, 64 + 8 * i, 8)
-        assert e & 0xFFFF == ch.size and (e >> 16) * 16 == off
-        assert np.array_equal(s1[base + off: base + off + ch.size], ch)
-        off += (ch.size + 15) // 16 * 16
+    assert lay.n_code == 5 and lay.n_seg == 3       # 2400 vectors, 512 per code chunk
+    sizes = [_u(s1, 64 + 8 * i, 8) & 0xFFFF for i in range(lay.n_chunks)]
+    offs = [(_u(s1, 64 + 8 * i, 8) >> 16) * 16 for i in range(lay.n_chunks)]
+    assert offs == [sum((z + 15) // 16 * 16 for z in sizes[:i]) for i in range(lay.n_chunks)]
+    for seg in range(lay.n_seg):
+        v0, v1 = oracle.segment_vectors(lay, seg)
+        st, chunks = oracle.encode_segment(d, seg, x[v0:v1])
+        idx = [oracle.code_chunk_index(lay, seg * lay.code_per_seg + i)
+               for i in range(len(chunks) - 1)] + [oracle.meta_chunk_index(lay, seg)]
+        for i, ch in zip(idx, chunks):
+            a = lay.data_base + offs[i]
+            assert sizes[i] == ch.size and np.array_equal(s1[a:a + ch.size], ch)
 
 
 def test_corrupt_streams():
