@@ -358,7 +358,7 @@ def main():
                      "peak_kind": peak_kind, "traffic": None,
                      "encode_frac": round(enc_gbs / hbm, 4),
                      "decode_frac": round(dec_gbs / hbm, 4)},
-        "gpu_launches": 2 * K,
+        "gpu_launches": 4 * K,  # encode, finish, compaction (returns at once unless a code chunk shrank), decode
         "clocks": clk.summary(),
     }
     if e2e:

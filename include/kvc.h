@@ -138,8 +138,10 @@ size_t kvc_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params);
  * table (bits 0..15 unpadded chunk size, bits 16..63 offset from the data base
  * in 16-byte units); u32 token count per request; zero padding to 16 bytes;
  * the chunks, each zero-padded to 16 bytes. The code and meta regions are cut
- * into 16 KB chunks; a meta chunk covers group_size*bits/32 code chunks and
- * follows them. */
+ * into 16 KB chunks; a meta chunk covers group_size*bits/32 code chunks. Chunk
+ * order (table and data): every code chunk, then every meta chunk. The call
+ * launches up to three kernels on `stream` (encode; table, meta chunks and
+ * header; compaction, which returns at once unless a code chunk shrank). */
 kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params,
                         void *out, size_t out_capacity, uint64_t *out_bytes_dev,
                         void *workspace, size_t workspace_bytes,

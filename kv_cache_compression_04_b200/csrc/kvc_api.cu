@@ -83,7 +83,7 @@ kvc_status describe(const kvc_kv_desc *kv, const kvc_params *p, Shape &s) {
     s.max_bytes += (s.n_code - 1) * kChunk + round16((s.V - (s.n_code - 1) * s.VC) * s.CB);
     s.max_bytes += (s.n_seg - 1) * kChunk + round16((s.V - (s.n_seg - 1) * VM) * s.MB);
   }
-  s.ws_bytes = kWsCtl + round256(8 * s.n_code) + s.n_seg * kChunk;
+  s.ws_bytes = ws_layout(s.n_code, s.n_seg).total;
   return KVC_OK;
 }
 
@@ -155,42 +155,68 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *o
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const WsLayout w = ws_layout(s.n_code, s.n_seg);
+  uint32_t *ctl = reinterpret_cast<uint32_t *>(ws);  // status, flags, ticket, reads
   EncArgs a{};
   a.V = uint32_t(s.V);
   a.n_tiles = uint32_t(s.n_code);
-  a.n_seg = uint32_t(s.n_seg);
-  a.n_chunks = uint32_t(s.n_chunks);
   a.out = static_cast<uint8_t *>(out);
-  a.out_capacity = out_capacity;
   a.data_base = s.data_base;
-  a.out_bytes_dev = out_bytes_dev;
-  a.status = reinterpret_cast<uint32_t *>(ws);
-  a.ticket = reinterpret_cast<uint32_t *>(ws + 4);
-  a.tile_state = reinterpret_cast<uint64_t *>(ws + kWsCtl);
-  a.ws_meta = ws + kWsCtl + round256(8 * s.n_code);
-  a.layers = uint32_t(kv->layers);
-  a.kv_heads = uint32_t(kv->kv_heads);
-  a.head_dim = uint32_t(s.D);
-  a.group = uint32_t(s.G);
-  a.bits = uint32_t(s.bits);
-  a.k = (s.D == 64 ? 6u : s.D == 128 ? 7u : 8u) / 2;
-  a.origin = kv->kind == KVC_PAGED ? 1u : 0u;
-  a.n_req = s.n_req;
-  a.tokens = s.T;
-  a.seed = params->sign_seed;
+  a.status = ctl;
+  a.flags = ctl + 1;
+  a.code_size = reinterpret_cast<uint32_t *>(ws + w.code_size);
+  a.meta_nnz = reinterpret_cast<uint32_t *>(ws + w.meta_nnz);
+  a.ws_meta = ws + w.meta;
   sign_masks(params->sign_seed, s.D, a.sign_mask);
 
-  if (cudaMemsetAsync(ws, 0, kWsCtl + 8 * s.n_code, cs) != cudaSuccess) return KVC_ERR_CUDA;
-  cudaError_t e;
+  FinArgs f{};
+  f.V = uint32_t(s.V);
+  f.n_code = uint32_t(s.n_code);
+  f.n_meta = uint32_t(s.n_seg);
+  f.n_chunks = uint32_t(s.n_chunks);
+  f.cb = uint32_t(s.CB);
+  f.mb = uint32_t(s.MB);
+  f.vc = uint32_t(s.VC);
+  f.vm = uint32_t(s.VC * s.R);
+  f.out = a.out;
+  f.out_capacity = out_capacity;
+  f.data_base = s.data_base;
+  f.out_bytes_dev = out_bytes_dev;
+  f.status = ctl;
+  f.flags = ctl + 1;
+  f.ticket = ctl + 2;  // ticket[0]: next code chunk to move, ticket[1]: chunks read
+  f.code_size = a.code_size;
+  f.meta_nnz = a.meta_nnz;
+  f.done = reinterpret_cast<uint32_t *>(ws + w.done);
+  f.meta_size = reinterpret_cast<uint32_t *>(ws + w.meta_size);
+  f.code_off = reinterpret_cast<uint64_t *>(ws + w.code_off);
+  f.ws_meta = a.ws_meta;
+  f.layers = uint32_t(kv->layers);
+  f.kv_heads = uint32_t(kv->kv_heads);
+  f.head_dim = uint32_t(s.D);
+  f.group = uint32_t(s.G);
+  f.bits = uint32_t(s.bits);
+  f.k = (s.D == 64 ? 6u : s.D == 128 ? 7u : 8u) / 2;
+  f.origin = kv->kind == KVC_PAGED ? 1u : 0u;
+  f.n_req = s.n_req;
+  f.tokens = s.T;
+  f.seed = params->sign_seed;
+
+  if (cudaMemsetAsync(ws, 0, w.zero_bytes, cs) != cudaSuccess) return KVC_ERR_CUDA;
+  cudaError_t e = cudaSuccess;
   if (kv->kind == KVC_DENSE) {
     const DenseLayout L = dense_layout(kv, s);
-    e = s.D == 128 ? launch_encode_dense_d128(s.bits, s.G, a, L, sms, cs)
-                   : launch_encode_dense_d64(s.bits, s.G, a, L, sms, cs);
+    if (s.n_code)
+      e = s.D == 128 ? launch_encode_dense_d128(s.bits, s.G, a, L, sms, cs)
+                     : launch_encode_dense_d64(s.bits, s.G, a, L, sms, cs);
+    if (e == cudaSuccess) e = launch_finish_dense(f, L, sms, cs);
   } else {
     static thread_local PagedLayout L;  // large (4 KB) parameter block
     paged_layout(kv, s, L);
-    e = s.D == 128 ? launch_encode_paged_d128(s.bits, s.G, a, L, sms, cs)
-                   : launch_encode_paged_d64(s.bits, s.G, a, L, sms, cs);
+    if (s.n_code)
+      e = s.D == 128 ? launch_encode_paged_d128(s.bits, s.G, a, L, sms, cs)
+                     : launch_encode_paged_d64(s.bits, s.G, a, L, sms, cs);
+    if (e == cudaSuccess) e = launch_finish_paged(f, L, sms, cs);
   }
   return e == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }

@@ -32,7 +32,7 @@ struct DecCtl {
   uint32_t hdr_ok;
   uint32_t bits, group, n_req_stream, n_chunks;
   uint64_t data_base, stream_bytes, seed;
-  uint32_t mask[128];
+  alignas(16) uint32_t mask[128];  // read as uint4
 };
 
 template <int D>
@@ -48,57 +48,20 @@ __device__ __forceinline__ uint64_t ld_u64(const uint8_t *p) {
   return *reinterpret_cast<const uint64_t *>(p);
 }
 
-// Undo zero-byte elimination (buf: bitmap + nonzero bytes, `size` bytes) into
-// scr, then undo the bit-plane shuffle from scr back into buf. Compute threads.
-// Returns false (for all threads) if the bitmap's popcount disagrees with the
-// size.
-__device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *red,
-                                          uint32_t size) {
-  const int tid = threadIdx.x;
-  const uint2 bm = reinterpret_cast<const uint2 *>(buf)[tid];
-  uint32_t total;
-  const uint32_t pos = block_excl_scan(__popc(bm.x) + __popc(bm.y), red, total);
-  const bool good = total == size - kBitmap;
-  uint32_t w[16];
-  const uint8_t *src = buf + kBitmap + pos;
-  int n = 0;
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    uint32_t v = 0;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int i = 4 * q + b;
-      const uint32_t bit = ((i < 32 ? bm.x >> i : bm.y >> (i - 32)) & 1u);
-      if (bit && good) v |= uint32_t(src[n++]) << (8 * b);
-    }
-    w[q] = v;
-  }
-  uint4 *d4 = reinterpret_cast<uint4 *>(scr + tid * 64);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) d4[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-  named_bar_sync(1, kThreads);
-  if (tid < 128) {  // plane words (p, m) -> words 32m .. 32m+31
-    uint32_t a[32];
-    const uint32_t *s = reinterpret_cast<const uint32_t *>(scr);
-#pragma unroll
-    for (int p = 0; p < 32; ++p) a[p] = s[p * 128 + tid];
-    transpose32(a);
-    uint4 *o = reinterpret_cast<uint4 *>(buf + tid * 128);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) o[q] = make_uint4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
-  }
-  named_bar_sync(1, kThreads);
-  return good;
-}
-
 template <int D, int BITS, int G>
-struct Dec : Cfg<D, BITS, G> {
-  using C = Cfg<D, BITS, G>;
+struct Dec : Cfg<D, BITS, G, kThreads> {
+  using C = Cfg<D, BITS, G, kThreads>;
 
-  // Reading R9: y^ = zf + q*sf (product rounded, then sum), butterfly,
-  // x 2^-log2(d), unsign, bf16 round-to-nearest-even.
+  // Reading R9: y^ = fl(zf + fl(q*sf)), the encoder's butterfly, then
+  // x^ = bf16_RNE(sign * (u * 2^-log2 d)). Computed here in an exactly
+  // equivalent order: zf and sf are pre-scaled by 2^-log2 d (exact), so every
+  // value of the butterfly is the reference value times 2^-log2 d; no value
+  // can become subnormal (all are 0 or at least 2^-28 in magnitude: fp16
+  // meta values are multiples of 2^-24), so scaling commutes with every
+  // rounding. q*sf is exact (q < 16 times an fp16 value needs at most 15
+  // significant bits), so one fused multiply-add equals fl(zf + fl(q*sf)).
   static __device__ __forceinline__ void vector(const uint8_t *codes, const uint8_t *meta,
-                                                const uint32_t *mask, uint32_t (&out)[C::HALF]) {
+                                                const uint32_t *mask, uint32_t (&out)[D / 2]) {
     uint32_t cw[C::CW];
     const uint4 *c4 = reinterpret_cast<const uint4 *>(codes);
 #pragma unroll
@@ -107,40 +70,47 @@ struct Dec : Cfg<D, BITS, G> {
       cw[4 * q] = v.x, cw[4 * q + 1] = v.y, cw[4 * q + 2] = v.z, cw[4 * q + 3] = v.w;
     }
     float zf[C::NG], sf[C::NG];
-    const float up = float(1 << C::K);
+    const float up = float(1 << C::K) / float(D);
 #pragma unroll
     for (int g = 0; g < C::NG; ++g) {
       const uint32_t m = reinterpret_cast<const uint32_t *>(meta)[g];
       sf[g] = __fmul_rn(__half2float(__ushort_as_half(uint16_t(m & 0xFFFFu))), up);
       zf[g] = __fmul_rn(__half2float(__ushort_as_half(uint16_t(m >> 16))), up);
     }
-    constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
+    // Code -> float: a byte permute puts the code in the low byte of the bit
+    // pattern 0x4B4000qq = 1.5*2^23 + q, and subtracting 1.5*2^23 gives q
+    // exactly.
+    constexpr uint32_t kMagicBits = 0x4B400000u;
     constexpr float kMagic = 12582912.0f;
-    constexpr int per_word = 32 / BITS;
-    float2 p[C::HALF];
+    float y[D];
 #pragma unroll
-    for (int i = 0; i < C::HALF; ++i) {
-      const int ca = i, cb = i + C::HALF;
-      const uint32_t qa = (cw[ca / per_word] >> ((ca % per_word) * BITS)) & C::QMAX;
-      const uint32_t qb = (cw[cb / per_word] >> ((cb % per_word) * BITS)) & C::QMAX;
-      const float2 q = sub2(make_float2(__uint_as_float(kMagicBits | qa), __uint_as_float(kMagicBits | qb)),
-                            make_float2(kMagic, kMagic));
-      const int ga = ca / G, gb = cb / G;
-      // q * sf is exact (q < 16 times an fp16 value times 2^K needs at most 15
-      // significant bits), so one fused rounding equals fl(zf + fl(q * sf)).
-      p[i] = fma2(q, make_float2(sf[ga], sf[gb]), make_float2(zf[ga], zf[gb]));
+    for (int W = 0; W < C::CW; ++W) {
+      constexpr int per_byte = 8 / BITS;
+      uint32_t part[per_byte];  // part[e] byte k = code of channel (4W + k)*per_byte + e
+#pragma unroll
+      for (int e = 0; e < per_byte; ++e)
+        part[e] = (cw[W] >> (e * BITS)) & (BITS == 4 ? 0x0F0F0F0Fu : 0x03030303u);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+#pragma unroll
+        for (int e = 0; e < per_byte; ++e) {
+          const int c = (4 * W + k) * per_byte + e, g = c / G;
+          const float qf = __fsub_rn(__uint_as_float(__byte_perm(part[e], kMagicBits, 0x7640 | k)), kMagic);
+          y[c] = __fmaf_rn(qf, sf[g], zf[g]);
+        }
+      }
     }
-    fwht_pairs<C::HALF>(p);
-    const float inv = 1.0f / float(D);
+    fwht<D>(y);
 #pragma unroll
-    for (int i = 0; i < C::HALF; ++i) p[i] = mul2(p[i], make_float2(inv, inv));
+    for (int q = 0; q < D / 8; ++q) {
+      const uint4 m4 = reinterpret_cast<const uint4 *>(mask)[q];
+      const uint32_t m[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-    for (int j = 0; j < C::HALF; ++j) {
-      const int c0 = 2 * j, c1 = 2 * j + 1;
-      const float v0 = c0 < C::HALF ? p[c0].x : p[c0 - C::HALF].y;
-      const float v1 = c1 < C::HALF ? p[c1].x : p[c1 - C::HALF].y;
-      const __nv_bfloat162 b = __floats2bfloat162_rn(v0, v1);
-      out[j] = *reinterpret_cast<const uint32_t *>(&b) ^ mask[j];
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * q + e;
+        const __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
+        out[j] = *reinterpret_cast<const uint32_t *>(&b) ^ m[e];
+      }
     }
   }
 };
@@ -149,7 +119,7 @@ template <int D, int BITS, int G, class Layout>
 __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, uint8_t *s_out,
                             uint8_t *s_cbuf, uint8_t *s_mbuf, uint8_t *s_scr,
                             const uint32_t *cum) {
-  using C = Cfg<D, BITS, G>;
+  using C = Cfg<D, BITS, G, kThreads>;
   using Dc = Dec<D, BITS, G>;
   const int tid = threadIdx.x;
   const uint32_t V = a.V;
@@ -167,9 +137,9 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     uint32_t bytes = 0;
     const uint32_t nvec = min(uint32_t(C::VC), V - tile * C::VC);
     const uint32_t seg = tile / C::R, tis = tile - seg * C::R;
-    const uint32_t seg_tiles = min(uint32_t(C::R), n_tiles - seg * C::R);
-    const uint64_t ic = uint64_t(tile) + seg;
-    const uint64_t im = uint64_t(seg) * (C::R + 1) + seg_tiles;
+    // reading R13: code chunk c is entry c, meta chunk s is entry n_code + s
+    const uint64_t ic = tile;
+    const uint64_t im = uint64_t(n_tiles) + seg;
     auto entry = [&](uint64_t i, uint64_t &off, uint32_t &size) {
       const uint64_t e = ld_u64(in + kHeader + 8 * i);
       off = (e >> 16) << 4;
@@ -241,8 +211,8 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     }
     uint8_t *cb = s_cbuf + b * kChunk, *mb = s_mbuf + b * kChunk;
     bool good = true;
-    if (io.code_mode) good &= ze_decode(cb, s_scr, ctl->red, io.code_size);
-    if (io.meta_mode) good &= ze_decode(mb, s_scr, ctl->red, io.meta_size);
+    if (io.code_mode) good &= ze_decode<kThreads>(cb, s_scr, ctl->red, io.code_size);
+    if (io.meta_mode) good &= ze_decode<kThreads>(mb, s_scr, ctl->red, io.meta_size);
     if (!good) {
       if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
       named_bar_sync(1, kThreads);
@@ -260,13 +230,13 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
         set_status(a.status, KVC_ERR_CORRUPT);
         continue;
       }
-      uint32_t out[C::HALF];
+      uint32_t out[D / 2];
       Dc::vector(cb + j * C::CB, mb + tis * C::SLICE + j * C::MB, ctl->mask, out);
       uint8_t *row = s_out + (outbuf * kThreads + tid) * C::ROWP;
       bulk_wait_read<1>();  // the store issued two rows ago has read this buffer
       uint4 *r4 = reinterpret_cast<uint4 *>(row);
 #pragma unroll
-      for (int q = 0; q < C::HALF / 4; ++q)
+      for (int q = 0; q < D / 8; ++q)
         r4[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
       fence_proxy_async_smem();
       bulk_s2g(dst, row, C::ROW);
@@ -341,12 +311,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       sum += n;
       if constexpr (kPaged) bad |= n != s_cum[r + 1] - s_cum[r];
     }
-    const uint32_t hi = block_sum(uint32_t(sum >> 32), ctl->red);
-    const uint32_t lo_bad = block_sum(bad, ctl->red);
+    const uint32_t hi = block_sum<kThreads>(uint32_t(sum >> 32), ctl->red);
+    const uint32_t lo_bad = block_sum<kThreads>(bad, ctl->red);
     // low 32 bits: sum of low halves may carry; recombine in 64 bits
     uint32_t lo32 = uint32_t(sum);
-    const uint32_t lo_sum = block_sum(lo32 & 0xFFFFu, ctl->red);
-    const uint32_t lo_hi = block_sum(lo32 >> 16, ctl->red);
+    const uint32_t lo_sum = block_sum<kThreads>(lo32 & 0xFFFFu, ctl->red);
+    const uint32_t lo_hi = block_sum<kThreads>(lo32 >> 16, ctl->red);
     const uint64_t total = (uint64_t(hi) << 32) + (uint64_t(lo_hi) << 16) + lo_sum;
     ok = !lo_bad && total == a.tokens;
   }

@@ -185,28 +185,21 @@ __device__ __forceinline__ float max2n(float a, float b) {
   return d;
 }
 
-// Walsh-Hadamard butterfly of one head_dim vector held as HALF = d/2 pairs,
-// p[i] = (y[i], y[i + d/2]). Strides h = 1, 2, ..., d/2 in ascending order;
-// each pair (i, i+h) with (i & h) == 0 becomes (a+b, a-b), one rounding each.
-// Strides below d/2 act on both halves at once (paired ops); the last stride
-// pairs the two lanes of each p[i].
-template <int HALF>
-__device__ __forceinline__ void fwht_pairs(float2 (&p)[HALF]) {
+// Walsh-Hadamard butterfly of one head_dim vector in registers (reading R2):
+// strides h = 1, 2, ..., d/2 in ascending order; each pair (i, i+h) with
+// (i & h) == 0 becomes (a+b, a-b), one rounding each.
+template <int D>
+__device__ __forceinline__ void fwht(float (&y)[D]) {
 #pragma unroll
-  for (int h = 1; h < HALF; h <<= 1) {
+  for (int h = 1; h < D; h <<= 1) {
 #pragma unroll
-    for (int i = 0; i < HALF; ++i) {
+    for (int i = 0; i < D; ++i) {
       if ((i & h) == 0) {
-        const float2 a = p[i], b = p[i + h];
-        p[i] = add2(a, b);
-        p[i + h] = sub2(a, b);
+        const float a = y[i], b = y[i + h];
+        y[i] = __fadd_rn(a, b);
+        y[i + h] = __fsub_rn(a, b);
       }
     }
-  }
-#pragma unroll
-  for (int i = 0; i < HALF; ++i) {
-    const float a = p[i].x, b = p[i].y;
-    p[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
   }
 }
 
@@ -231,10 +224,10 @@ KVC_HD void transpose32(uint32_t (&a)[32]) {
 }
 
 // -------------------------------------------------------------- scans --
-// Exclusive sum over the kThreads compute threads (named barrier 1); also
-// returns the total. `red` holds kThreads/32 words of shared memory.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *red,
-                                                    uint32_t &total) {
+// Exclusive sum over the first NT threads of the block (named barrier 1);
+// also returns the total. `red` holds NT/32 words of shared memory.
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *red, uint32_t &total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = x;
 #pragma unroll
@@ -243,22 +236,135 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *red,
     if (lane >= o) incl += y;
   }
   if (lane == 31) red[warp] = incl;
-  named_bar_sync(1, kThreads);
+  named_bar_sync(1, NT);
   uint32_t before = 0, all = 0;
 #pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     const uint32_t r = red[w];
     before += (w < warp) ? r : 0u;
     all += r;
   }
-  named_bar_sync(1, kThreads);
+  named_bar_sync(1, NT);
   total = all;
   return before + incl - x;
 }
+template <int NT>
 __device__ __forceinline__ uint32_t block_sum(uint32_t x, uint32_t *red) {
   uint32_t total;
-  block_excl_scan(x, red, total);
+  block_excl_scan<NT>(x, red, total);
   return total;
+}
+
+// ------------------------------------------- lossless stage (16 KB chunk) --
+// Reading R10 (bit planes of 32-bit little-endian words) and R11 (zero-byte
+// elimination: 2048-byte bitmap + nonzero bytes), on a chunk in shared
+// memory, by the first NT threads.
+
+// Nonzero bytes the bit-plane shuffle of the chunk would have: byte i of
+// plane p is nonzero iff bit p of (w[8i] | ... | w[8i+7]) is set, so the
+// count is the sum of popcounts of 8-word ORs; no shuffle is needed to
+// decide between raw and eliminated storage. This thread's part.
+template <int NT>
+__device__ __forceinline__ uint32_t chunk_nnz_part(const uint8_t *buf) {
+  constexpr int kGroups = kChunk / 32 / NT;  // 8-word groups per thread
+  const uint4 *s = reinterpret_cast<const uint4 *>(buf) + threadIdx.x * 2 * kGroups;
+  uint32_t n = 0;
+#pragma unroll
+  for (int q = 0; q < kGroups; ++q) {
+    const uint4 a = s[2 * q], b = s[2 * q + 1];
+    n += __popc(a.x | a.y | a.z | a.w | b.x | b.y | b.z | b.w);
+  }
+  return n;
+}
+
+// buf holds a full 16 KB chunk; on return it holds bitmap + nonzero bytes
+// (the caller knows their count from chunk_nnz_part). scr: 16 KB scratch.
+template <int NT>
+__device__ __forceinline__ void ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *red) {
+  const int tid = threadIdx.x;
+  for (int m = tid; m < 128; m += NT) {  // block m = words 32m .. 32m+31
+    uint32_t a[32];
+    const uint4 *src = reinterpret_cast<const uint4 *>(buf + m * 128);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint4 v = src[q];
+      a[4 * q] = v.x, a[4 * q + 1] = v.y, a[4 * q + 2] = v.z, a[4 * q + 3] = v.w;
+    }
+    transpose32(a);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(scr);
+#pragma unroll
+    for (int p = 0; p < 32; ++p) dst[p * 128 + m] = a[p];
+  }
+  named_bar_sync(1, NT);
+  constexpr int kBytes = kChunk / NT;  // shuffled bytes per thread
+  constexpr int kMaskWords = kBytes / 32;
+  const uint32_t *w = reinterpret_cast<const uint32_t *>(scr + tid * kBytes);
+  uint32_t mask[kMaskWords], cnt = 0;
+#pragma unroll
+  for (int mw = 0; mw < kMaskWords; ++mw) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) m |= (((w[mw * 8 + i / 4] >> (8 * (i % 4))) & 0xFFu) ? 1u : 0u) << i;
+    mask[mw] = m;
+    cnt += __popc(m);
+  }
+  uint32_t total;
+  const uint32_t pos = block_excl_scan<NT>(cnt, red, total);
+  uint32_t *bm = reinterpret_cast<uint32_t *>(buf) + tid * kMaskWords;
+#pragma unroll
+  for (int mw = 0; mw < kMaskWords; ++mw) bm[mw] = mask[mw];
+  uint32_t o = kBitmap + pos;
+#pragma unroll 4
+  for (int i = 0; i < kBytes; ++i) {
+    const uint32_t byte = (w[i / 4] >> (8 * (i % 4))) & 0xFFu;
+    if (byte && o < uint32_t(kChunk)) buf[o++] = uint8_t(byte);
+  }
+  named_bar_sync(1, NT);
+}
+
+// Inverse: buf holds bitmap + nonzero bytes (`size` bytes); on return it
+// holds the 16 KB chunk. Returns false (for every thread) if the bitmap's
+// popcount disagrees with the size; then buf is unspecified.
+template <int NT>
+__device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *red, uint32_t size) {
+  const int tid = threadIdx.x;
+  constexpr int kBytes = kChunk / NT;
+  constexpr int kMaskWords = kBytes / 32;
+  uint32_t mask[kMaskWords], cnt = 0;
+#pragma unroll
+  for (int mw = 0; mw < kMaskWords; ++mw) {
+    mask[mw] = reinterpret_cast<const uint32_t *>(buf)[tid * kMaskWords + mw];
+    cnt += __popc(mask[mw]);
+  }
+  uint32_t total;
+  const uint32_t pos = block_excl_scan<NT>(cnt, red, total);
+  const bool good = total == size - kBitmap;
+  const uint8_t *src = buf + kBitmap + pos;
+  uint32_t *d = reinterpret_cast<uint32_t *>(scr + tid * kBytes);
+  int n = 0;
+#pragma unroll
+  for (int q = 0; q < kBytes / 4; ++q) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int i = 4 * q + b;
+      if (good && ((mask[i / 32] >> (i % 32)) & 1u)) v |= uint32_t(src[n++]) << (8 * b);
+    }
+    d[q] = v;
+  }
+  named_bar_sync(1, NT);
+  for (int m = tid; m < 128; m += NT) {  // plane words (p, m) -> words 32m .. 32m+31
+    uint32_t a[32];
+    const uint32_t *s = reinterpret_cast<const uint32_t *>(scr);
+#pragma unroll
+    for (int p = 0; p < 32; ++p) a[p] = s[p * 128 + m];
+    transpose32(a);
+    uint4 *o = reinterpret_cast<uint4 *>(buf + m * 128);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) o[q] = make_uint4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+  }
+  named_bar_sync(1, NT);
+  return good;
 }
 
 // --------------------------------------------------------- addressing --

@@ -1,0 +1,301 @@
+// Finishing kernels of kvc_compress (after the main encode kernel):
+//
+// finish_kernel: the device-wide prefix sum of chunk sizes (readings R12,
+//   R13: every code chunk, then every meta chunk; offsets are the exclusive
+//   prefix sum of the 16-byte-padded sizes), the meta chunks' lossless stage
+//   (each meta chunk's shuffled-byte count was accumulated by the encode
+//   kernel, so the raw / zero-byte decision needs no pass over the data),
+//   compaction of the meta chunks into place, the chunk table and the header.
+//   CTA b takes a contiguous range of meta chunks and of code-table entries;
+//   the few prefix sums a CTA needs are block reductions over the size
+//   arrays, so CTAs never wait on one another.
+//
+// compact_kernel: runs only when some code chunk shrank (zero-byte
+//   elimination paid), which leaves later code chunks to the right of their
+//   final offsets. Chunks move left in ticket order; a chunk is moved only
+//   after every chunk whose source it would overwrite has been read, and the
+//   meta chunks (parked in the workspace by finish_kernel) are placed after
+//   every code chunk has been read. All waits are bounded.
+#pragma once
+
+#include "kvc_encode.cuh"
+
+namespace kvc {
+
+constexpr int kFinThreads = 256;
+
+struct FinCtl {
+  uint64_t full;
+  uint32_t red[kFinThreads / 32];
+  uint32_t flag;
+  uint32_t tick;
+};
+
+constexpr size_t fin_smem_bytes(bool paged) {
+  return 2 * size_t(kChunk) + sizeof(FinCtl) +
+         (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
+}
+
+// 64-bit block sum over the first NT threads.
+template <int NT>
+__device__ __forceinline__ uint64_t block_sum64(uint64_t x, uint32_t *red) {
+  const uint32_t hi = block_sum<NT>(uint32_t(x >> 32), red);
+  const uint32_t mid = block_sum<NT>(uint32_t(x >> 16) & 0xFFFFu, red);
+  const uint32_t lo = block_sum<NT>(uint32_t(x) & 0xFFFFu, red);
+  return (uint64_t(hi) << 32) + (uint64_t(mid) << 16) + lo;
+}
+
+__device__ __forceinline__ void st_u16(uint8_t *p, uint32_t v) {
+  *reinterpret_cast<uint16_t *>(p) = uint16_t(v);
+}
+__device__ __forceinline__ void st_u32(uint8_t *p, uint32_t v) {
+  *reinterpret_cast<uint32_t *>(p) = v;
+}
+__device__ __forceinline__ void st_u64(uint8_t *p, uint64_t v) {
+  *reinterpret_cast<uint64_t *>(p) = v;
+}
+
+__device__ __forceinline__ uint32_t meta_len(const FinArgs &a, uint32_t s) {
+  return min(a.vm, a.V - s * a.vm) * a.mb;
+}
+// Reading R11: zero-byte elimination only when strictly shorter, full chunks only.
+__device__ __forceinline__ uint32_t meta_stored_size(const FinArgs &a, uint32_t s) {
+  const uint32_t len = meta_len(a, s), n = a.meta_nnz[s];
+  return (len == uint32_t(kChunk) && kBitmap + n < uint32_t(kChunk)) ? kBitmap + n : len;
+}
+
+template <class Layout>
+__device__ void fin_header(const FinArgs &a, const uint32_t *cum, uint64_t stream_bytes) {
+  uint8_t *o = a.out;
+  st_u32(o + 0, kMagic);
+  st_u16(o + 4, 1);
+  st_u16(o + 6, kHeader);
+  st_u32(o + 8, a.bits | (a.k << 8) | (a.origin << 16));
+  st_u32(o + 12, a.group);
+  st_u32(o + 16, a.layers);
+  st_u32(o + 20, 2);
+  st_u32(o + 24, a.kv_heads);
+  st_u32(o + 28, a.head_dim);
+  st_u64(o + 32, a.tokens);
+  st_u64(o + 40, a.seed);
+  st_u32(o + 48, a.n_req);
+  st_u32(o + 52, a.n_chunks);
+  st_u64(o + 56, stream_bytes);
+  uint8_t *tt = o + kHeader + 8ull * a.n_chunks;
+  for (uint32_t r = 0; r < a.n_req; ++r) {
+    uint32_t n;
+    if constexpr (kIsPaged<Layout>)
+      n = cum[r + 1] - cum[r];
+    else
+      n = uint32_t(a.tokens);
+    st_u32(tt + 4ull * r, n);
+  }
+  for (uint64_t b = kHeader + 8ull * a.n_chunks + 4ull * a.n_req; b < a.data_base; ++b) o[b] = 0;
+  if (a.out_bytes_dev) *a.out_bytes_dev = stream_bytes;
+}
+
+template <class Layout>
+__global__ void __launch_bounds__(kFinThreads, 1)
+    finish_kernel(const __grid_constant__ FinArgs a, const __grid_constant__ Layout lay) {
+  constexpr int NT = kFinThreads;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t *buf = smem;
+  uint8_t *scr = smem + kChunk;
+  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + 2 * kChunk);
+  uint32_t *s_cum = reinterpret_cast<uint32_t *>(ctl + 1);
+  const int tid = threadIdx.x;
+  const uint32_t nb = gridDim.x, b = blockIdx.x;
+  if (tid == 0) {
+    mbar_init(&ctl->full, 1);
+    mbar_fence_init();
+    ctl->flag = *reinterpret_cast<volatile uint32_t *>(a.flags);
+  }
+  if constexpr (kIsPaged<Layout>) {
+    for (uint32_t r = tid; r <= lay.n_req; r += NT) s_cum[r] = lay.cum[r];
+  }
+  __syncthreads();
+  const bool shrank = ctl->flag & 1u;
+
+  // Bytes of all code chunks, padded.
+  uint64_t total_code = 0;
+  if (a.n_code) {
+    if (!shrank) {
+      total_code = uint64_t(a.n_code - 1) * kChunk +
+                   round16(uint64_t(a.V - (a.n_code - 1) * a.vc) * a.cb);
+    } else {
+      uint64_t part = 0;
+      for (uint32_t c = tid; c < a.n_code; c += NT) part += round16(a.code_size[c]);
+      total_code = block_sum64<NT>(part, ctl->red);
+    }
+  }
+
+  // -------------------------------------------------- this CTA's meta chunks --
+  const uint32_t s0 = uint32_t(uint64_t(b) * a.n_meta / nb);
+  const uint32_t s1 = uint32_t(uint64_t(b + 1) * a.n_meta / nb);
+  uint64_t prefix = 0;
+  {
+    uint64_t part = 0;
+    for (uint32_t s = tid; s < s0; s += NT) part += round16(meta_stored_size(a, s));
+    prefix = block_sum64<NT>(part, ctl->red);
+  }
+  uint32_t phase = 0;
+#pragma unroll 1
+  for (uint32_t s = s0; s < s1; ++s, ++phase) {
+    const uint32_t len = meta_len(a, s), size = meta_stored_size(a, s);
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&ctl->full, uint32_t(round16(len)));
+      bulk_g2s(buf, a.ws_meta + uint64_t(s) * kChunk, uint32_t(round16(len)), &ctl->full);
+    }
+    if (!mbar_wait(&ctl->full, phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+    if (size < len) ze_encode<NT>(buf, scr, ctl->red);
+    for (uint32_t i = size + tid; i < round16(size); i += NT) buf[i] = 0;
+    fence_proxy_async_smem();
+    named_bar_sync(1, NT);
+    if (tid == 0) {
+      const uint64_t off = total_code + prefix;
+      if (a.data_base + off + round16(size) <= a.out_capacity) {
+        // Without a shrunken code chunk the code region is final, so the
+        // chunk goes to its place; otherwise it is parked in its workspace
+        // slot until compact_kernel has moved the code chunks.
+        uint8_t *dst = shrank ? a.ws_meta + uint64_t(s) * kChunk : a.out + a.data_base + off;
+        bulk_s2g(dst, buf, uint32_t(round16(size)));
+        bulk_commit();
+        st_u64(a.out + kHeader + 8ull * (a.n_code + s), ((off >> 4) << 16) | size);
+      } else {
+        set_status(a.status, KVC_ERR_CAPACITY);
+      }
+      a.meta_size[s] = size;
+      bulk_wait_read<0>();
+    }
+    prefix += round16(size);
+    named_bar_sync(1, NT);  // buf free
+  }
+
+  // -------------------------------------------------- code-table entries --
+  const uint32_t c0 = uint32_t(uint64_t(b) * a.n_code / nb);
+  const uint32_t c1 = uint32_t(uint64_t(b + 1) * a.n_code / nb);
+  if (!shrank) {
+    for (uint32_t c = c0 + tid; c < c1; c += NT)
+      st_u64(a.out + kHeader + 8ull * c, ((uint64_t(c) * kChunk >> 4) << 16) | a.code_size[c]);
+  } else {
+    uint64_t part = 0;
+    for (uint32_t c = tid; c < c0; c += NT) part += round16(a.code_size[c]);
+    uint64_t base = block_sum64<NT>(part, ctl->red);
+    for (uint32_t c = c0; c < c1; c += NT) {  // block-wide scan, NT chunks at a time
+      const uint32_t me = c + tid;
+      const uint32_t sz = me < c1 ? a.code_size[me] : 0u;
+      uint32_t total;
+      const uint32_t ex = block_excl_scan<NT>(uint32_t(round16(sz)) >> 4, ctl->red, total);
+      if (me < c1) {
+        const uint64_t off = base + (uint64_t(ex) << 4);
+        a.code_off[me] = off;
+        st_u64(a.out + kHeader + 8ull * me, ((off >> 4) << 16) | sz);
+      }
+      base += uint64_t(total) << 4;
+    }
+  }
+
+  // -------------------------------------------------------------- header --
+  if (b == 0) {
+    uint64_t part = 0;
+    for (uint32_t s = tid; s < a.n_meta; s += NT) part += round16(meta_stored_size(a, s));
+    const uint64_t total_meta = block_sum64<NT>(part, ctl->red);
+    if (tid == 0) fin_header<Layout>(a, s_cum, a.data_base + total_code + total_meta);
+  }
+  if (tid == 0) bulk_wait_all<0>();
+}
+
+// Moves code chunks left when some code chunk shrank, then places the meta
+// chunks. Chunk c (source data_base + c * 16 KB, destination data_base +
+// code_off[c] <= source) may overwrite only sources of chunks j <= c whose
+// 16 KB slot overlaps its destination; it waits for their read flags.
+__global__ void __launch_bounds__(kFinThreads, 1) compact_kernel(const __grid_constant__ FinArgs a) {
+  constexpr int NT = kFinThreads;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t *buf = smem;
+  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + 2 * kChunk);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    mbar_init(&ctl->full, 1);
+    mbar_fence_init();
+    ctl->flag = *reinterpret_cast<volatile uint32_t *>(a.flags);
+  }
+  __syncthreads();
+  if (!(ctl->flag & 1u)) return;
+  uint32_t phase = 0;
+#pragma unroll 1
+  while (true) {
+    if (tid == 0) ctl->tick = atomicAdd(a.ticket, 1u);
+    named_bar_sync(1, NT);
+    const uint32_t c = ctl->tick;
+    named_bar_sync(1, NT);
+    if (c >= a.n_code) break;
+    const uint32_t size = a.code_size[c];
+    const uint64_t src = uint64_t(c) * kChunk, dst = a.code_off[c];
+    if (dst != src) {
+      // sources overlapping [dst, dst + padded size) must have been read
+      const uint32_t j0 = uint32_t(dst / kChunk);
+      for (uint32_t j = j0 + tid; j < c; j += NT) {
+        const uint64_t t0 = globaltimer();
+        for (uint32_t it = 0; *reinterpret_cast<volatile uint32_t *>(a.done + j) == 0; ++it) {
+          if (spin_expired(it, t0, a.status)) {
+            set_status(a.status, KVC_ERR_TIMEOUT);
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+      __threadfence();
+      named_bar_sync(1, NT);
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&ctl->full, uint32_t(round16(size)));
+        bulk_g2s(buf, a.out + a.data_base + src, uint32_t(round16(size)), &ctl->full);
+      }
+      if (!mbar_wait(&ctl->full, phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+      ++phase;
+      if (tid == 0) {
+        __threadfence();
+        atomicExch(a.done + c, 1u);  // source read
+        atomicAdd(a.ticket + 1, 1u);
+        bulk_s2g(a.out + a.data_base + dst, buf, uint32_t(round16(size)));
+        bulk_commit();
+        bulk_wait_read<0>();
+      }
+      named_bar_sync(1, NT);
+    } else if (tid == 0) {
+      atomicExch(a.done + c, 1u);
+      atomicAdd(a.ticket + 1, 1u);
+    }
+  }
+  // meta chunks, parked in the workspace, go after the code region once
+  // every code chunk has been read (their destinations overlap old sources)
+  if (tid == 0) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0; *reinterpret_cast<volatile uint32_t *>(a.ticket + 1) < a.n_code; ++it) {
+      if (spin_expired(it, t0, a.status)) {
+        set_status(a.status, KVC_ERR_TIMEOUT);
+        break;
+      }
+      __nanosleep(128);
+    }
+    __threadfence();
+  }
+  named_bar_sync(1, NT);
+#pragma unroll 1
+  for (uint32_t s = blockIdx.x; s < a.n_meta; s += gridDim.x) {
+    if (tid == 0) {
+      const uint32_t size = a.meta_size[s];
+      const uint64_t e = *reinterpret_cast<const uint64_t *>(a.out + kHeader + 8ull * (a.n_code + s));
+      mbar_arrive_expect_tx(&ctl->full, uint32_t(round16(size)));
+      bulk_g2s(buf, a.ws_meta + uint64_t(s) * kChunk, uint32_t(round16(size)), &ctl->full);
+      if (!mbar_wait(&ctl->full, phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+      bulk_s2g(a.out + a.data_base + ((e >> 16) << 4), buf, uint32_t(round16(size)));
+      bulk_commit();
+      bulk_wait_read<0>();
+    }
+    ++phase;
+  }
+  if (tid == 0) bulk_wait_all<0>();
+}
+
+}  // namespace kvc

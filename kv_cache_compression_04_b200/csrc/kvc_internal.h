@@ -28,13 +28,37 @@ constexpr uint32_t kMagic = 0x3143564Bu;  // "KVC1"
 constexpr int kThreads = 256;   // compute threads per CTA (one vector each)
 constexpr uint32_t kNoTile = 0xFFFFFFFFu;
 
-// Workspace layout of kvc_compress: [status, ticket, ...] control block,
-// then one u64 look-back word per tile, then one 16 KB meta staging chunk per
-// segment. Only the first two parts need zeroing per call.
+// Workspace of kvc_compress, in this order (each part 256-byte aligned):
+//   control   status word, flags word (bit 0: some code chunk shrank),
+//             compaction ticket
+//   meta_nnz  u32 per meta chunk: shuffled-byte nonzero count (accumulated)
+//   done      u32 per code chunk: compaction read flags
+//   code_size u32 per code chunk
+//   meta_size u32 per meta chunk
+//   code_off  u64 per code chunk: final offsets (compaction only)
+//   meta      16 KB per meta chunk: raw meta, then (compaction only) the
+//             chunk as stored
+// Only control, meta_nnz and done need zeroing per call.
 constexpr size_t kWsCtl = 256;
+struct WsLayout {
+  size_t meta_nnz, done, code_size, meta_size, code_off, meta, total, zero_bytes;
+};
 
 KVC_HD uint64_t round16(uint64_t x) { return (x + 15u) & ~uint64_t(15); }
 KVC_HD uint64_t round256(uint64_t x) { return (x + 255u) & ~uint64_t(255); }
+
+inline WsLayout ws_layout(uint64_t n_code, uint64_t n_meta) {
+  WsLayout w{};
+  w.meta_nnz = kWsCtl;
+  w.done = w.meta_nnz + round256(4 * n_meta);
+  w.code_size = w.done + round256(4 * n_code);
+  w.meta_size = w.code_size + round256(4 * n_code);
+  w.code_off = w.meta_size + round256(4 * n_meta);
+  w.meta = w.code_off + round256(8 * n_code);
+  w.total = w.meta + n_meta * uint64_t(kChunk);
+  w.zero_bytes = w.code_size;
+  return w;
+}
 
 // SplitMix64 (Steele, Lea, Flood, OOPSLA 2014): sign words of the +-1
 // diagonal are its outputs counted from state = seed.
@@ -95,23 +119,42 @@ struct PagedLayout {
   uint32_t cum[KVC_MAX_REQUESTS + 1];   // token prefix per request
 };
 
+// Main encode kernel: quantize and place every code chunk at its raw-layout
+// position (data base + c * 16 KB); meta slices go to the workspace.
 struct EncArgs {
   uint32_t V;          // vectors
   uint32_t n_tiles;    // code chunks (one tile = one code chunk)
-  uint32_t n_seg;      // segments = meta chunks
-  uint32_t n_chunks;
+  uint8_t *out;
+  uint64_t data_base;
+  uint32_t *status;
+  uint32_t *flags;
+  uint32_t *code_size;
+  uint32_t *meta_nnz;
+  uint8_t *ws_meta;
+  uint32_t sign_mask[128];
+};
+
+// Finishing kernels: sizes and offsets of every chunk, meta chunks,
+// chunk table, header; compaction when a code chunk shrank.
+struct FinArgs {
+  uint32_t V, n_code, n_meta, n_chunks;
+  uint32_t cb, mb, vc, vm;  // code / meta bytes per vector, vectors per code / meta chunk
   uint8_t *out;
   uint64_t out_capacity;
   uint64_t data_base;
   uint64_t *out_bytes_dev;
   uint32_t *status;
+  uint32_t *flags;
   uint32_t *ticket;
-  uint64_t *tile_state;
+  const uint32_t *code_size;
+  const uint32_t *meta_nnz;
+  uint32_t *done;
+  uint32_t *meta_size;
+  uint64_t *code_off;
   uint8_t *ws_meta;
   // header fields
   uint32_t layers, kv_heads, head_dim, group, bits, k, origin, n_req;
   uint64_t tokens, seed;
-  uint32_t sign_mask[128];
 };
 
 struct DecArgs {
@@ -137,5 +180,7 @@ struct DecArgs {
 KVC_DECLARE_LAUNCHERS(128)
 KVC_DECLARE_LAUNCHERS(64)
 #undef KVC_DECLARE_LAUNCHERS
+cudaError_t launch_finish_dense(const FinArgs &a, const DenseLayout &lay, int sms, cudaStream_t st);
+cudaError_t launch_finish_paged(const FinArgs &a, const PagedLayout &lay, int sms, cudaStream_t st);
 
 }  // namespace kvc

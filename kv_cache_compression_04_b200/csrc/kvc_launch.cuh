@@ -29,8 +29,8 @@ cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_
   struct Tag {};
   cudaError_t e = prepare<Tag>(k, smem);
   if (e != cudaSuccess) return e;
-  const int grid = a.n_tiles == 0 ? 1 : int(a.n_tiles < uint32_t(sms) ? a.n_tiles : uint32_t(sms));
-  k<<<grid, kThreads + 32, smem, st>>>(a, lay);
+  const int grid = int(a.n_tiles < uint32_t(sms) ? a.n_tiles : uint32_t(sms));
+  k<<<grid, kEncThreads, smem, st>>>(a, lay);
   return cudaGetLastError();
 }
 

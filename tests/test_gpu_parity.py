@@ -133,6 +133,24 @@ def test_structured_inputs(kind, bits, g):
         assert (sizes < 16384).any()              # zero-byte elimination was exercised
 
 
+def test_compaction_many_chunks_mixed():
+    """Shrunken code chunks scattered through more code chunks than CTAs (each
+    CTA moves several): a random half of the 16 KB code chunks are all-zero
+    codes, so later chunks move left by varying distances."""
+    L, H, T, D = 4, 8, 4096, 128
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(L, 2, H, T, D, generator=g)
+    blocks = x.view(L, 2, H, T // 256, 256, D)
+    zero = torch.rand(L, 2, H, T // 256, generator=g) < 0.5
+    blocks[zero] = 0
+    s = _roundtrip_dense(x.to(torch.bfloat16).cuda(), 4, 128)
+    od = oracle_desc(4, 128, D, L, H, [T])
+    sizes, _ = chunk_table(s, od.layout().n_chunks)
+    n_code = od.layout().n_code
+    assert n_code > 2 * 148
+    assert 0.3 < (sizes[:n_code] < 16384).mean() < 0.7
+
+
 # -------------------------------------------------------------------- paged --
 def _paged_setup(seq, L=2, H=3, D=128, bits=4, g=64, seed=3):
     w = synth.Workload("p", L, H, D, bits, g, seed=seed, kind="lognormal", scale_sigma=1.5,
