@@ -14,8 +14,9 @@
  *
  * Conventions shared by every entry point:
  *  - Memory. The caller owns every buffer (input, output, page table,
- *    workspace, stream). The library allocates nothing and keeps no global
- *    state; calls are re-entrant, but concurrent calls need distinct
+ *    workspace, stream). The library allocates nothing; its only global state
+ *    is the static workspace block of kvc_compress_noalloc (end of this
+ *    file). Calls are re-entrant, but concurrent calls need distinct
  *    workspaces.
  *  - Asynchrony. All device work is enqueued on `stream` (a cudaStream_t; 0 is
  *    the legacy default stream). Pointers marked DEVICE must stay valid until
@@ -166,6 +167,41 @@ kvc_status kvc_stream_status(const void *workspace, kvc_stream_t stream);
 
 /* Static, human-readable name of a status. */
 const char *kvc_status_string(kvc_status status);
+
+/* ---- Compression without a caller-provided workspace (the pages have no
+ * counterpart; this is a deployment convenience).
+ *
+ * Some callers cannot hand out device memory at transfer time: a serving
+ * engine typically gives nearly all of HBM to its paged KV pool when it
+ * starts, and its transfer path must not ask any allocator for more (a
+ * request may block, synchronize the device or fail under memory pressure at
+ * exactly the moment a KV cache is leaving). kvc_compress_noalloc does the
+ * same work as kvc_compress, with the same arguments and results, but its
+ * workspace is a fixed block of the library's own static device memory
+ * (KVC_NOALLOC_SCRATCH_BYTES per device, reserved when the library's module
+ * is loaded on that device) instead of caller memory. It allocates nothing.
+ *
+ *  - Limit. Shapes whose kvc_workspace_bytes exceeds KVC_NOALLOC_SCRATCH_BYTES
+ *    return KVC_ERR_CAPACITY before anything is enqueued. The workspace is
+ *    about 16 KB per 16 KB of meta (fp16 scale and zero per group), so 16 MiB
+ *    holds e.g. 32 layers x 8 kv_heads x 4096 tokens x head_dim 128 at group
+ *    128 (8.1 MiB), not at group 64 (16.1 MiB).
+ *  - Set-up. The first call on each device (with that device current) looks
+ *    up the block's device address once and keeps it; make that first call
+ *    before any stream capture on the device. A failed look-up returns
+ *    KVC_ERR_CUDA.
+ *  - Status. If status_dev (DEVICE, 4 bytes, 4-byte aligned) is not null, the
+ *    call's status word is copied there on `stream` after the encode; pass
+ *    status_dev to kvc_stream_status() to read it.
+ *  - Concurrency. There is one block per device, so calls on the same device
+ *    must not overlap: a call enqueued on one stream while another is still
+ *    running on a different stream (or from another thread) races on the
+ *    block and corrupts both streams. Serialize them, e.g. on one stream. */
+#define KVC_NOALLOC_SCRATCH_BYTES (16u << 20)
+kvc_status kvc_compress_noalloc(const kvc_kv_desc *kv, const kvc_params *params,
+                                void *out, size_t out_capacity,
+                                uint64_t *out_bytes_dev, uint32_t *status_dev,
+                                kvc_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(PKG, "libkvc.so")
 KVC_DENSE, KVC_PAGED = 0, 1
 KVC_MAX_REQUESTS = 1024
 KVC_DECOMPRESS_WORKSPACE_BYTES = 256
+KVC_NOALLOC_SCRATCH_BYTES = 16 << 20
 STATUS = ["KVC_OK", "KVC_ERR_INVALID_ARG", "KVC_ERR_UNSUPPORTED", "KVC_ERR_CAPACITY",
           "KVC_ERR_NONFINITE", "KVC_ERR_RANGE", "KVC_ERR_CORRUPT", "KVC_ERR_TIMEOUT",
           "KVC_ERR_CUDA"]
@@ -26,7 +27,7 @@ STATUS = ["KVC_OK", "KVC_ERR_INVALID_ARG", "KVC_ERR_UNSUPPORTED", "KVC_ERR_CAPAC
 
 # Every symbol include/kvc.h declares.
 EXPORTS = ["kvc_max_compressed_bytes", "kvc_workspace_bytes", "kvc_compress",
-           "kvc_decompress", "kvc_stream_status", "kvc_status_string"]
+           "kvc_decompress", "kvc_stream_status", "kvc_status_string", "kvc_compress_noalloc"]
 
 
 class KvcError(RuntimeError):
@@ -77,6 +78,9 @@ def lib() -> C.CDLL:
         L.kvc_stream_status.argtypes = [C.c_void_p, C.c_void_p]
         L.kvc_status_string.restype = C.c_char_p
         L.kvc_status_string.argtypes = [C.c_int]
+        L.kvc_compress_noalloc.restype = C.c_int
+        L.kvc_compress_noalloc.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p,
+                                           C.c_void_p, C.c_void_p]
         _lib = L
     return _lib
 
@@ -94,6 +98,12 @@ def kvc_compress(desc, params, out_ptr, out_capacity, out_bytes_dev_ptr, ws_ptr,
                  stream) -> int:
     return lib().kvc_compress(C.byref(desc), C.byref(params), out_ptr, out_capacity,
                               out_bytes_dev_ptr, ws_ptr, ws_bytes, stream)
+
+
+def kvc_compress_noalloc(desc, params, out_ptr, out_capacity, out_bytes_dev_ptr, status_dev_ptr,
+                         stream) -> int:
+    return lib().kvc_compress_noalloc(C.byref(desc), C.byref(params), out_ptr, out_capacity,
+                                      out_bytes_dev_ptr, status_dev_ptr, stream)
 
 
 def kvc_decompress(in_ptr, in_bytes, desc, ws_ptr, ws_bytes, stream) -> int:
