@@ -159,12 +159,11 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *o
   uint32_t *ctl = reinterpret_cast<uint32_t *>(ws);  // status, flags, ticket, reads
   EncArgs a{};
   a.V = uint32_t(s.V);
-  a.n_tiles = uint32_t(s.n_code);
   a.out = static_cast<uint8_t *>(out);
   a.data_base = s.data_base;
   a.status = ctl;
   a.flags = ctl + 1;
-  a.code_size = reinterpret_cast<uint32_t *>(ws + w.code_size);
+  a.code_nnz = reinterpret_cast<unsigned long long *>(ws + w.code_nnz);
   a.meta_nnz = reinterpret_cast<uint32_t *>(ws + w.meta_nnz);
   a.ws_meta = ws + w.meta;
   sign_masks(params->sign_seed, s.D, a.sign_mask);
@@ -185,8 +184,9 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *o
   f.status = ctl;
   f.flags = ctl + 1;
   f.ticket = ctl + 2;  // ticket[0]: next code chunk to move, ticket[1]: chunks read
-  f.code_size = a.code_size;
+  f.code_nnz = a.code_nnz;
   f.meta_nnz = a.meta_nnz;
+  f.code_size = reinterpret_cast<uint32_t *>(ws + w.code_size);
   f.done = reinterpret_cast<uint32_t *>(ws + w.done);
   f.meta_size = reinterpret_cast<uint32_t *>(ws + w.meta_size);
   f.code_off = reinterpret_cast<uint64_t *>(ws + w.code_off);

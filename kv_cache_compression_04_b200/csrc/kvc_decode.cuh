@@ -1,45 +1,59 @@
-// Fused decode kernel: parse and validate the stream -> per tile (one code
-// chunk): bulk-async load of the code chunk and of the tile's meta -> undo
-// zero-byte elimination and the bit-plane shuffle when the chunk used them ->
-// unpack -> dequantize -> fp32 Walsh-Hadamard (same butterfly as the encoder)
-// -> scale by 2^-log2(d) -> unsign -> bf16 -> bulk store (dense) or scatter
-// through the receiver's page table (paged). The decoder is the inverse path
-// the podcast page "FastKVComp: checking whether high-throughput KV
-// compression pays off" (episode notes) places on the decode GPU.
+// Fused decode kernel: parse and validate the stream -> per meta chunk: load
+// it and undo zero-byte elimination and the bit-plane shuffle when it used
+// them -> per code chunk of the CTA's tile range: blocks of 32 vectors, one
+// per lane, code bytes loaded by bulk-async copy (a chunk that used zero-byte
+// elimination is first expanded by the whole CTA) -> unpack -> dequantize ->
+// fp32 Walsh-Hadamard (the encoder's butterfly) -> scale by 2^-log2(d) ->
+// unsign -> bf16 -> bulk store (dense) or scatter through the receiver's page
+// table (paged). The decoder is the inverse path the podcast page
+// "FastKVComp: checking whether high-throughput KV compression pays off"
+// (episode notes) places on the decode GPU.
 //
 // The chunk table stores every chunk's offset, so each CTA takes a contiguous
-// range of tiles and reads its chunks directly: no scan, no inter-CTA waits.
-// Every table entry is checked against its predecessor (offset = previous
-// offset + padded previous size), so a consistent table is a prefix sum.
+// range of code chunks (tiles) and reads its chunks directly: no scan, no
+// inter-CTA waits. Every table entry is checked against its predecessor
+// (offset = previous offset + padded previous size) by the CTA whose range
+// holds it, so a consistent table is a prefix sum. Warps decode blocks
+// independently; the CTA synchronizes only when it moves to the next meta
+// chunk or expands a zero-byte-eliminated code chunk.
 #pragma once
 
 #include "kvc_encode.cuh"
 
 namespace kvc {
 
-struct TileIO {
-  uint32_t ok;        // chunk entries valid
-  uint32_t code_mode; // 0 raw, 1 zero-byte eliminated
-  uint32_t code_size;
-  uint32_t meta_mode;
-  uint32_t meta_size;
-};
+constexpr int kDecWarps = 12;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kZeThreads = 256;  // threads that run the chunk expansion
 
 struct DecCtl {
-  uint64_t full[2];
-  TileIO io[2];
-  uint32_t red[kThreads / 32];
-  uint32_t hdr_ok;
+  uint64_t cbar[kDecWarps][2];  // per-warp code blocks loaded (two buffers)
+  uint64_t mbar;             // meta chunk loaded
+  uint64_t zbar;             // zero-byte-eliminated code chunk loaded
+  uint32_t red[kDecThreads / 32];
+  uint32_t hdr_ok, bad;
   uint32_t bits, group, n_req_stream, n_chunks;
   uint64_t data_base, stream_bytes, seed;
   alignas(16) uint32_t mask[128];  // read as uint4
 };
 
+// Shared memory: output rows | per-warp code blocks | meta chunk | expanded
+// code chunk | expansion scratch | control | request prefix (paged).
 template <int D>
-constexpr size_t dec_smem_bytes(bool paged) {
-  return size_t(2) * kThreads * (2 * D + 16) + 5 * size_t(kChunk) + sizeof(DecCtl) +
-         (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
-}
+struct DecSmem {
+  static constexpr size_t ROWP = 2 * D + 16;
+  static constexpr size_t BLK = 32 * size_t(D) / 2;  // widest code block (4-bit)
+  static constexpr size_t rows = 0;
+  static constexpr size_t code = rows + kDecThreads * ROWP;
+  static constexpr size_t meta = code + 2 * kDecWarps * BLK;
+  static constexpr size_t zchunk = meta + kChunk;
+  static constexpr size_t scr = zchunk + kChunk;
+  static constexpr size_t ctl = scr + kChunk;
+  static constexpr size_t cum = ctl + ((sizeof(DecCtl) + 15) & ~size_t(15));
+  static constexpr size_t bytes(bool paged) {
+    return cum + (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
+  }
+};
 
 __device__ __forceinline__ uint32_t ld_u32(const uint8_t *p) {
   return *reinterpret_cast<const uint32_t *>(p);
@@ -49,8 +63,8 @@ __device__ __forceinline__ uint64_t ld_u64(const uint8_t *p) {
 }
 
 template <int D, int BITS, int G>
-struct Dec : Cfg<D, BITS, G, kThreads> {
-  using C = Cfg<D, BITS, G, kThreads>;
+struct Dec : Cfg<D, BITS, G> {
+  using C = Cfg<D, BITS, G>;
 
   // Reading R9: y^ = fl(zf + fl(q*sf)), the encoder's butterfly, then
   // x^ = bf16_RNE(sign * (u * 2^-log2 d)). Computed here in an exactly
@@ -60,15 +74,9 @@ struct Dec : Cfg<D, BITS, G, kThreads> {
   // meta values are multiples of 2^-24), so scaling commutes with every
   // rounding. q*sf is exact (q < 16 times an fp16 value needs at most 15
   // significant bits), so one fused multiply-add equals fl(zf + fl(q*sf)).
+  // The vector is held as pairs (c, c + d/2) like the encoder's.
   static __device__ __forceinline__ void vector(const uint8_t *codes, const uint8_t *meta,
                                                 const uint32_t *mask, uint32_t (&out)[D / 2]) {
-    uint32_t cw[C::CW];
-    const uint4 *c4 = reinterpret_cast<const uint4 *>(codes);
-#pragma unroll
-    for (int q = 0; q < C::CW / 4; ++q) {
-      const uint4 v = c4[q];
-      cw[4 * q] = v.x, cw[4 * q + 1] = v.y, cw[4 * q + 2] = v.z, cw[4 * q + 3] = v.w;
-    }
     float zf[C::NG], sf[C::NG];
     const float up = float(1 << C::K) / float(D);
 #pragma unroll
@@ -78,196 +86,267 @@ struct Dec : Cfg<D, BITS, G, kThreads> {
       zf[g] = __fmul_rn(__half2float(__ushort_as_half(uint16_t(m >> 16))), up);
     }
     // Code -> float: a byte permute puts the code in the low byte of the bit
-    // pattern 0x4B4000qq = 1.5*2^23 + q, and subtracting 1.5*2^23 gives q
-    // exactly.
+    // pattern 0x4B4000qq = 1.5*2^23 + q; subtracting 1.5*2^23 gives q exactly.
+    // Pair j takes channel j from the first half of the code words and
+    // channel j + d/2 from the second; each 16-byte piece of either half is
+    // loaded when the pairs reach it.
+    constexpr int per_word = 32 / BITS;          // codes per word
+    constexpr int per_byte = 8 / BITS;
+    constexpr int HW = C::CW / 2;                // words per half
+    constexpr int PW = HW < 4 ? HW : 4;          // words per piece
+    constexpr int NP = HW / PW;                  // pieces per half
+    constexpr int JP = PW * per_word;            // pairs per piece
     constexpr uint32_t kMagicBits = 0x4B400000u;
     constexpr float kMagic = 12582912.0f;
-    float y[D];
+    const float2 mag = make_float2(kMagic, kMagic);
+    Pairs<D> y;
 #pragma unroll
-    for (int W = 0; W < C::CW; ++W) {
-      constexpr int per_byte = 8 / BITS;
-      uint32_t part[per_byte];  // part[e] byte k = code of channel (4W + k)*per_byte + e
+    for (int piece = 0; piece < NP; ++piece) {
+      uint32_t lo[PW], hi[PW];
+      if constexpr (PW == 4) {
+        const uint4 a = reinterpret_cast<const uint4 *>(codes)[piece];
+        const uint4 b = reinterpret_cast<const uint4 *>(codes)[NP + piece];
+        lo[0] = a.x, lo[1] = a.y, lo[2] = a.z, lo[3] = a.w;
+        hi[0] = b.x, hi[1] = b.y, hi[2] = b.z, hi[3] = b.w;
+      } else {
+        const uint4 a = reinterpret_cast<const uint4 *>(codes)[0];
+        lo[0] = a.x, lo[1] = a.y, hi[0] = a.z, hi[1] = a.w;
+      }
+      auto code_float = [&](const uint32_t (&w)[PW], int c) -> float {
+        const int W = c / per_word, r = c % per_word, k = r / per_byte, e = r % per_byte;
+        const uint32_t part = (w[W] >> (e * BITS)) & (BITS == 4 ? 0x0F0F0F0Fu : 0x03030303u);
+        return __uint_as_float(__byte_perm(part, kMagicBits, 0x7640 | k));
+      };
 #pragma unroll
-      for (int e = 0; e < per_byte; ++e)
-        part[e] = (cw[W] >> (e * BITS)) & (BITS == 4 ? 0x0F0F0F0Fu : 0x03030303u);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-#pragma unroll
-        for (int e = 0; e < per_byte; ++e) {
-          const int c = (4 * W + k) * per_byte + e, g = c / G;
-          const float qf = __fsub_rn(__uint_as_float(__byte_perm(part[e], kMagicBits, 0x7640 | k)), kMagic);
-          y[c] = __fmaf_rn(qf, sf[g], zf[g]);
-        }
+      for (int i = 0; i < JP; ++i) {
+        const int j = piece * JP + i;
+        const int ga = j / G, gb = (j + D / 2) / G;
+        const float2 q = sub2(make_float2(code_float(lo, i), code_float(hi, i)), mag);
+        y.p[j] = fma2(q, make_float2(sf[ga], sf[gb]), make_float2(zf[ga], zf[gb]));
       }
     }
-    fwht<D>(y);
+    fwht_pairs<D>(y);
 #pragma unroll
     for (int q = 0; q < D / 8; ++q) {
       const uint4 m4 = reinterpret_cast<const uint4 *>(mask)[q];
       const uint32_t m[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int j = 4 * q + e;
-        const __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
-        out[j] = *reinterpret_cast<const uint32_t *>(&b) ^ m[e];
+        const int k = 4 * q + e;
+        const __nv_bfloat162 b = __floats2bfloat162_rn(y.at(2 * k), y.at(2 * k + 1));
+        out[k] = *reinterpret_cast<const uint32_t *>(&b) ^ m[e];
       }
     }
   }
 };
 
+// Decodes vectors v0 .. v0 + nvec - 1 (one per lane) whose codes start at
+// `codes` (CB bytes each, lane order) and meta at `meta` (MB bytes each).
 template <int D, int BITS, int G, class Layout>
-__device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, uint8_t *s_out,
-                            uint8_t *s_cbuf, uint8_t *s_mbuf, uint8_t *s_scr,
+__device__ __forceinline__ void decode_block(const DecArgs &a, const Layout &lay, const uint32_t *cum,
+                                             const uint8_t *codes, const uint8_t *meta, uint32_t v0,
+                                             uint32_t nvec, const uint32_t *mask, uint8_t *row,
+                                             bool &row_busy) {
+  using C = Cfg<D, BITS, G>;
+  const int lane = threadIdx.x & 31;
+  if (uint32_t(lane) >= nvec) return;
+  uint32_t out[D / 2];
+  Dec<D, BITS, G>::vector(codes + lane * C::CB, meta + lane * C::MB, mask, out);
+  bool ok;
+  uint8_t *dst = vec_addr(lay, cum, v0 + lane, ok);  // after the vector: fewer live registers
+  if (!ok) {
+    set_status(a.status, KVC_ERR_CORRUPT);
+    return;
+  }
+  if (row_busy) bulk_wait_read<0>();  // this thread's previous store has read the row
+  uint4 *r4 = reinterpret_cast<uint4 *>(row);
+#pragma unroll
+  for (int q = 0; q < D / 8; ++q)
+    r4[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+  fence_proxy_async_smem();
+  bulk_s2g(dst, row, C::ROW);
+  bulk_commit();
+  row_busy = true;
+}
+
+template <int D, int BITS, int G, class Layout>
+__device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, uint8_t *smem,
                             const uint32_t *cum) {
-  using C = Cfg<D, BITS, G, kThreads>;
-  using Dc = Dec<D, BITS, G>;
-  const int tid = threadIdx.x;
+  using C = Cfg<D, BITS, G>;
+  using S = DecSmem<D>;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t V = a.V;
   const uint32_t n_tiles = (V + C::VC - 1) / C::VC;
   const uint32_t t0 = uint32_t(uint64_t(blockIdx.x) * n_tiles / gridDim.x);
   const uint32_t t1 = uint32_t(uint64_t(blockIdx.x + 1) * n_tiles / gridDim.x);
+  if (t0 >= t1) return;
   const uint8_t *in = a.in;
   const uint64_t base = ctl->data_base;
   const uint64_t limit = min(a.in_bytes, ctl->stream_bytes);
+  const uint8_t *table = in + kHeader;
+  uint8_t *row = smem + S::rows + tid * S::ROWP;
+  uint8_t *cbuf = smem + S::code + 2 * warp * S::BLK;
+  uint8_t *mbuf = smem + S::meta;
+  uint8_t *zbuf = smem + S::zchunk;
+  uint8_t *scr = smem + S::scr;
+  const uint32_t seg0 = t0 / C::R, seg1 = (t1 - 1) / C::R;
 
-  // Thread 0: check the table entries of `tile`, then start its loads.
-  auto prefetch = [&](uint32_t tile, int b) {
-    uint64_t *bar = &ctl->full[b];
-    TileIO io{1, 0, 0, 0, 0};
-    uint32_t bytes = 0;
-    const uint32_t nvec = min(uint32_t(C::VC), V - tile * C::VC);
-    const uint32_t seg = tile / C::R, tis = tile - seg * C::R;
-    // reading R13: code chunk c is entry c, meta chunk s is entry n_code + s
-    const uint64_t ic = tile;
-    const uint64_t im = uint64_t(n_tiles) + seg;
-    auto entry = [&](uint64_t i, uint64_t &off, uint32_t &size) {
-      const uint64_t e = ld_u64(in + kHeader + 8 * i);
-      off = (e >> 16) << 4;
-      size = uint32_t(e & 0xFFFFu);
-      uint64_t expect = 0;
-      if (i > 0) {
-        const uint64_t p = ld_u64(in + kHeader + 8 * (i - 1));
-        expect = ((p >> 16) << 4) + round16(p & 0xFFFFu);
-      }
-      return off == expect && base + off + round16(size) <= limit;
-    };
-    uint64_t oc, om;
-    uint32_t sc, sm;
-    const uint32_t code_len = nvec * C::CB;
-    const uint32_t seg_vec = min(uint32_t(C::VM), V - seg * C::VM);
-    const uint32_t meta_len = seg_vec * C::MB;
-    bool ok = entry(ic, oc, sc) && entry(im, om, sm);
-    if (ok) {
-      if (sc == code_len)
-        io.code_mode = 0;
-      else if (code_len == kChunk && sc >= kBitmap && sc < kChunk)
-        io.code_mode = 1;
-      else
-        ok = false;
-      if (sm == meta_len)
-        io.meta_mode = 0;
-      else if (meta_len == kChunk && sm >= kBitmap && sm < kChunk)
-        io.meta_mode = 1;
-      else
-        ok = false;
-      // the last chunk must end the stream
-      if (im + 1 == ctl->n_chunks && base + om + round16(sm) != ctl->stream_bytes) ok = false;
+  // D2: table entries of this range (code chunks t0..t1-1, meta chunks
+  // seg0..seg1): each offset continues its predecessor, stays inside the
+  // stream, and each size is the chunk's raw length or a valid eliminated
+  // size (full chunks only); the last chunk ends the stream.
+  auto entry_ok = [&](uint64_t i, uint32_t len) {
+    const uint64_t e = ld_u64(table + 8 * i);
+    const uint64_t off = (e >> 16) << 4;
+    const uint32_t size = uint32_t(e & 0xFFFFu);
+    uint64_t expect = 0;
+    if (i > 0) {
+      const uint64_t p = ld_u64(table + 8 * (i - 1));
+      expect = ((p >> 16) << 4) + round16(p & 0xFFFFu);
     }
-    io.ok = ok;
-    io.code_size = sc;
-    io.meta_size = sm;
-    ctl->io[b] = io;
-    if (!ok) {
-      set_status(a.status, KVC_ERR_CORRUPT);
-      mbar_arrive(bar);
+    bool ok = off == expect && base + off + round16(size) <= limit &&
+              (size == len || (len == uint32_t(kChunk) && size >= kBitmap && size < len));
+    if (i + 1 == ctl->n_chunks) ok = ok && base + off + round16(size) == ctl->stream_bytes;
+    return ok;
+  };
+  {
+    uint32_t bad = 0;
+    for (uint32_t t = t0 + tid; t < t1; t += kDecThreads)
+      bad |= !entry_ok(t, min(uint32_t(C::VC), V - t * C::VC) * C::CB);
+    for (uint32_t s = seg0 + tid; s <= seg1; s += kDecThreads)
+      bad |= !entry_ok(uint64_t(n_tiles) + s, min(uint32_t(C::VM), V - s * C::VM) * C::MB);
+    if (block_sum<kDecThreads>(bad, ctl->red)) {
+      if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
       return;
     }
-    const uint32_t cbytes = uint32_t(round16(sc));
-    uint32_t mbytes, moff;
-    if (io.meta_mode == 0) {  // only this tile's slice
-      moff = tis * C::SLICE;
-      mbytes = uint32_t(round16(uint64_t(nvec) * C::MB));
-    } else {
-      moff = 0;
-      mbytes = uint32_t(round16(sm));
-    }
-    bytes = cbytes + mbytes;
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_g2s(s_cbuf + b * kChunk, in + base + oc, cbytes, bar);
-    bulk_g2s(s_mbuf + b * kChunk + moff, in + base + om + moff, mbytes, bar);
-  };
+  }
 
-  if (t0 < t1 && tid == 0) prefetch(t0, 0);
-  uint32_t outbuf = 0;
+  uint32_t mphase = 0, zphase = 0, cphase = 0;  // cphase: bit k for code buffer k
+  bool row_busy = false;
 #pragma unroll 1
-  for (uint32_t tile = t0, i = 0; tile < t1; ++tile, ++i) {
-    const int b = i & 1;
-    if (tile + 1 < t1 && tid == 0) prefetch(tile + 1, b ^ 1);
-    if (!mbar_wait(&ctl->full[b], (i >> 1) & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
-    const TileIO io = ctl->io[b];
-    if (!io.ok) {
-      named_bar_sync(1, kThreads);
-      continue;
-    }
-    uint8_t *cb = s_cbuf + b * kChunk, *mb = s_mbuf + b * kChunk;
-    bool good = true;
-    if (io.code_mode) good &= ze_decode<kThreads>(cb, s_scr, ctl->red, io.code_size);
-    if (io.meta_mode) good &= ze_decode<kThreads>(mb, s_scr, ctl->red, io.meta_size);
-    if (!good) {
-      if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
-      named_bar_sync(1, kThreads);
-      continue;
-    }
-    const uint32_t nvec = min(uint32_t(C::VC), V - tile * C::VC);
-    const uint32_t seg = tile / C::R, tis = tile - seg * C::R;
-#pragma unroll 1
-    for (int sub = 0; sub < C::NSUB; ++sub) {
-      const uint32_t j = sub * kThreads + tid;
-      if (j >= nvec) break;
-      bool ok;
-      uint8_t *dst = vec_addr(lay, cum, tile * C::VC + j, ok);
-      if (!ok) {
-        set_status(a.status, KVC_ERR_CORRUPT);
-        continue;
-      }
-      uint32_t out[D / 2];
-      Dc::vector(cb + j * C::CB, mb + tis * C::SLICE + j * C::MB, ctl->mask, out);
-      uint8_t *row = s_out + (outbuf * kThreads + tid) * C::ROWP;
-      bulk_wait_read<1>();  // the store issued two rows ago has read this buffer
-      uint4 *r4 = reinterpret_cast<uint4 *>(row);
-#pragma unroll
-      for (int q = 0; q < D / 8; ++q)
-        r4[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+  for (uint32_t s = seg0; s <= seg1; ++s) {
+    // D3: the meta chunk, expanded if it used zero-byte elimination.
+    const uint64_t me = ld_u64(table + 8 * (uint64_t(n_tiles) + s));
+    const uint32_t msize = uint32_t(me & 0xFFFFu);
+    const uint32_t mlen = min(uint32_t(C::VM), V - s * C::VM) * C::MB;
+    __syncthreads();  // every warp is done with the previous meta chunk
+    if (tid == 0) {
       fence_proxy_async_smem();
-      bulk_s2g(dst, row, C::ROW);
-      bulk_commit();
-      outbuf ^= 1;
+      mbar_arrive_expect_tx(&ctl->mbar, uint32_t(round16(msize)));
+      bulk_g2s(mbuf, in + base + ((me >> 16) << 4), uint32_t(round16(msize)), &ctl->mbar);
     }
-    named_bar_sync(1, kThreads);  // buffers b free for the prefetch two tiles on
+    if (!mbar_wait(&ctl->mbar, mphase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+    mphase ^= 1;
+    if (msize != mlen) {
+      bool good = true;
+      if (tid < kZeThreads) good = ze_decode<kZeThreads>(mbuf, scr, ctl->red, msize);
+      if (tid == 0) ctl->bad = !good;
+      __syncthreads();
+      if (ctl->bad) {
+        if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
+        return;
+      }
+    }
+    const uint32_t ts0 = max(t0, s * C::R), ts1 = min(t1, (s + 1) * C::R);
+
+    // Code chunks of this segment that used zero-byte elimination (rare):
+    // the CTA expands each one, then the warps decode its blocks.
+#pragma unroll 1
+    for (uint32_t t = ts0; t < ts1; ++t) {
+      const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
+      const uint32_t csize = uint32_t(ce & 0xFFFFu);
+      const uint32_t nvec = min(uint32_t(C::VC), V - t * C::VC);
+      if (csize == nvec * C::CB) continue;
+      __syncthreads();  // zbuf free
+      if (tid == 0) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&ctl->zbar, uint32_t(round16(csize)));
+        bulk_g2s(zbuf, in + base + ((ce >> 16) << 4), uint32_t(round16(csize)), &ctl->zbar);
+      }
+      if (!mbar_wait(&ctl->zbar, zphase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+      zphase ^= 1;
+      bool good = true;
+      if (tid < kZeThreads) good = ze_decode<kZeThreads>(zbuf, scr, ctl->red, csize);
+      if (tid == 0) ctl->bad = !good;
+      __syncthreads();
+      if (ctl->bad) {
+        if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
+        return;
+      }
+      for (uint32_t b = warp; b * 32 < nvec; b += kDecWarps) {
+        const uint32_t v0 = t * C::VC + b * 32;
+        decode_block<D, BITS, G>(a, lay, cum, zbuf + b * 32 * C::CB,
+                                 mbuf + (v0 - s * C::VM) * C::MB, v0, min(32u, nvec - b * 32),
+                                 ctl->mask, row, row_busy);
+      }
+    }
+
+    // Raw code chunks: blocks of 32 vectors round-robin over the warps, each
+    // warp loading a block's code bytes with one bulk copy into one of its two
+    // buffers while it decodes the previous block from the other.
+    const uint32_t vs0 = ts0 * C::VC, vs1 = min(ts1 * C::VC, V);
+    const uint32_t nblk = (vs1 - vs0 + 31) / 32;
+    auto raw_block = [&](uint32_t b) {  // block b lies in a raw code chunk
+      const uint32_t t = (vs0 + b * 32) / C::VC;
+      const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
+      return uint32_t(ce & 0xFFFFu) == min(uint32_t(C::VC), V - t * C::VC) * C::CB;
+    };
+    auto next_raw = [&](uint32_t b) {
+      while (b < nblk && !raw_block(b)) b += kDecWarps;
+      return b;
+    };
+    auto issue = [&](uint32_t b, uint32_t k) {
+      if (lane == 0) {
+        const uint32_t v0 = vs0 + b * 32, t = v0 / C::VC, bytes = min(32u, vs1 - v0) * C::CB;
+        const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&ctl->cbar[warp][k], bytes);
+        bulk_g2s(cbuf + k * S::BLK, in + base + ((ce >> 16) << 4) + uint64_t(v0 - t * C::VC) * C::CB,
+                 bytes, &ctl->cbar[warp][k]);
+      }
+    };
+    uint32_t b = next_raw(warp), k = 0;
+    if (b < nblk) issue(b, 0);
+#pragma unroll 1
+    while (b < nblk) {
+      const uint32_t nb = next_raw(b + kDecWarps);
+      __syncwarp();  // every lane is done with buffer k ^ 1 (the block before b)
+      if (nb < nblk) issue(nb, k ^ 1);
+      if (!mbar_wait(&ctl->cbar[warp][k], (cphase >> k) & 1, a.status))
+        set_status(a.status, KVC_ERR_TIMEOUT);
+      cphase ^= 1u << k;
+      const uint32_t v0 = vs0 + b * 32;
+      decode_block<D, BITS, G>(a, lay, cum, cbuf + k * S::BLK, mbuf + (v0 - s * C::VM) * C::MB, v0,
+                               min(32u, vs1 - v0), ctl->mask, row, row_busy);
+      b = nb;
+      k ^= 1;
+    }
   }
   bulk_wait_all<0>();
 }
 
 template <int D, class Layout>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, 1)
     decode_kernel(const __grid_constant__ DecArgs a, const __grid_constant__ Layout lay) {
   constexpr bool kPaged = kIsPaged<Layout>;
+  using S = DecSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t *s_out = smem;
-  uint8_t *s_cbuf = s_out + 2 * kThreads * (2 * D + 16);
-  uint8_t *s_mbuf = s_cbuf + 2 * kChunk;
-  uint8_t *s_scr = s_mbuf + 2 * kChunk;
-  DecCtl *ctl = reinterpret_cast<DecCtl *>(s_scr + kChunk);
-  uint32_t *s_cum = reinterpret_cast<uint32_t *>(ctl + 1);
+  DecCtl *ctl = reinterpret_cast<DecCtl *>(smem + S::ctl);
+  uint32_t *s_cum = reinterpret_cast<uint32_t *>(smem + S::cum);
   const int tid = threadIdx.x;
   constexpr uint32_t kLog2D = D == 64 ? 6 : D == 128 ? 7 : 8;
 
   if constexpr (kPaged) {
     for (uint32_t r = tid; r <= lay.n_req; r += blockDim.x) s_cum[r] = lay.cum[r];
   }
+  if (tid < kDecWarps) {
+    mbar_init(&ctl->cbar[tid][0], 1);
+    mbar_init(&ctl->cbar[tid][1], 1);
+    mbar_fence_init();
+  }
   if (tid == 0) {
-    mbar_init(&ctl->full[0], 1);
-    mbar_init(&ctl->full[1], 1);
+    mbar_init(&ctl->mbar, 1);
+    mbar_init(&ctl->zbar, 1);
     mbar_fence_init();
     // D1: header (reading R12) against the receiver's description.
     const uint8_t *h = a.in;
@@ -311,14 +390,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       sum += n;
       if constexpr (kPaged) bad |= n != s_cum[r + 1] - s_cum[r];
     }
-    const uint32_t hi = block_sum<kThreads>(uint32_t(sum >> 32), ctl->red);
-    const uint32_t lo_bad = block_sum<kThreads>(bad, ctl->red);
-    // low 32 bits: sum of low halves may carry; recombine in 64 bits
-    uint32_t lo32 = uint32_t(sum);
-    const uint32_t lo_sum = block_sum<kThreads>(lo32 & 0xFFFFu, ctl->red);
-    const uint32_t lo_hi = block_sum<kThreads>(lo32 >> 16, ctl->red);
-    const uint64_t total = (uint64_t(hi) << 32) + (uint64_t(lo_hi) << 16) + lo_sum;
-    ok = !lo_bad && total == a.tokens;
+    const uint32_t hi = block_sum<kDecThreads>(uint32_t(sum >> 32), ctl->red);
+    const uint32_t any_bad = block_sum<kDecThreads>(bad, ctl->red);
+    const uint32_t lo32 = uint32_t(sum);
+    const uint32_t lo_lo = block_sum<kDecThreads>(lo32 & 0xFFFFu, ctl->red);
+    const uint32_t lo_hi = block_sum<kDecThreads>(lo32 >> 16, ctl->red);
+    const uint64_t total = (uint64_t(hi) << 32) + (uint64_t(lo_hi) << 16) + lo_lo;
+    ok = !any_bad && total == a.tokens;
   }
   if (!ok) {
     if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
@@ -327,26 +405,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bits = ctl->bits, group = ctl->group;
   if constexpr (D == 128) {
     if (bits == 4 && group == 128)
-      decode_body<128, 4, 128>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<128, 4, 128>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 64)
-      decode_body<128, 4, 64>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<128, 4, 64>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 32)
-      decode_body<128, 4, 32>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<128, 4, 32>(a, lay, ctl, smem, s_cum);
     else if (bits == 2 && group == 128)
-      decode_body<128, 2, 128>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<128, 2, 128>(a, lay, ctl, smem, s_cum);
     else if (bits == 2 && group == 64)
-      decode_body<128, 2, 64>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<128, 2, 64>(a, lay, ctl, smem, s_cum);
     else
-      decode_body<128, 2, 32>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<128, 2, 32>(a, lay, ctl, smem, s_cum);
   } else {
     if (bits == 4 && group == 64)
-      decode_body<64, 4, 64>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<64, 4, 64>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 32)
-      decode_body<64, 4, 32>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<64, 4, 32>(a, lay, ctl, smem, s_cum);
     else if (bits == 2 && group == 64)
-      decode_body<64, 2, 64>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<64, 2, 64>(a, lay, ctl, smem, s_cum);
     else
-      decode_body<64, 2, 32>(a, lay, ctl, s_out, s_cbuf, s_mbuf, s_scr, s_cum);
+      decode_body<64, 2, 32>(a, lay, ctl, smem, s_cum);
   }
 }
 

@@ -13,8 +13,9 @@ cudaError_t launch_fin(const FinArgs &a, const Layout &lay, int sms, cudaStream_
   struct FinTag {};
   cudaError_t e = prepare<FinTag>(fk, fsmem);
   if (e != cudaSuccess) return e;
-  const uint32_t want = a.n_meta > 1 ? a.n_meta : 1u;
-  const int grid = int(want < uint32_t(sms) ? want : uint32_t(sms));
+  // one meta chunk per CTA where possible (several CTAs share an SM)
+  const uint32_t want = a.n_meta > 1 ? a.n_meta : 1u, cap = 4u * uint32_t(sms);
+  const int grid = int(want < cap ? want : cap);
   fk<<<grid, kFinThreads, fsmem, st>>>(a, lay);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.n_code == 0) return e;

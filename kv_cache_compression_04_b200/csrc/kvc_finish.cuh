@@ -1,21 +1,21 @@
 // Finishing kernels of kvc_compress (after the main encode kernel):
 //
-// finish_kernel: the device-wide prefix sum of chunk sizes (readings R12,
-//   R13: every code chunk, then every meta chunk; offsets are the exclusive
-//   prefix sum of the 16-byte-padded sizes), the meta chunks' lossless stage
-//   (each meta chunk's shuffled-byte count was accumulated by the encode
-//   kernel, so the raw / zero-byte decision needs no pass over the data),
-//   compaction of the meta chunks into place, the chunk table and the header.
-//   CTA b takes a contiguous range of meta chunks and of code-table entries;
-//   the few prefix sums a CTA needs are block reductions over the size
-//   arrays, so CTAs never wait on one another.
+// finish_kernel: every chunk's stored size, from the shuffled-byte nonzero
+//   counts the encode kernel accumulated (reading R11: zero-byte elimination
+//   only for full chunks and only when strictly shorter), the device-wide
+//   prefix sum of the padded sizes (readings R12, R13: every code chunk, then
+//   every meta chunk), the meta chunks' lossless stage and their placement,
+//   the chunk table and the header. CTA b takes a contiguous range of meta
+//   chunks and of code-table entries; the prefix sums a CTA needs are block
+//   reductions over the count arrays, so CTAs never wait on one another.
 //
-// compact_kernel: runs only when some code chunk shrank (zero-byte
-//   elimination paid), which leaves later code chunks to the right of their
-//   final offsets. Chunks move left in ticket order; a chunk is moved only
-//   after every chunk whose source it would overwrite has been read, and the
-//   meta chunks (parked in the workspace by finish_kernel) are placed after
-//   every code chunk has been read. All waits are bounded.
+// compact_kernel: runs only when some code chunk shrinks (zero-byte
+//   elimination pays), which is rare for Hadamard-rotated codes. The encode
+//   kernel left every code chunk raw at data base + c * 16 KB; chunks are
+//   re-encoded and moved left in ticket order, a chunk only after every chunk
+//   whose raw bytes its destination overlaps has been read; the meta chunks
+//   (parked in the workspace by finish_kernel) are placed after every code
+//   chunk has been read. All waits are bounded.
 #pragma once
 
 #include "kvc_encode.cuh"
@@ -55,6 +55,13 @@ __device__ __forceinline__ void st_u64(uint8_t *p, uint64_t v) {
   *reinterpret_cast<uint64_t *>(p) = v;
 }
 
+__device__ __forceinline__ uint32_t code_len(const FinArgs &a, uint32_t c) {
+  return min(a.vc, a.V - c * a.vc) * a.cb;
+}
+__device__ __forceinline__ uint32_t code_stored_size(const FinArgs &a, uint32_t c) {
+  const uint32_t len = code_len(a, c), n = uint32_t(a.code_nnz[c]);
+  return (len == uint32_t(kChunk) && kBitmap + n < uint32_t(kChunk)) ? kBitmap + n : len;
+}
 __device__ __forceinline__ uint32_t meta_len(const FinArgs &a, uint32_t s) {
   return min(a.vm, a.V - s * a.vm) * a.mb;
 }
@@ -95,7 +102,7 @@ __device__ void fin_header(const FinArgs &a, const uint32_t *cum, uint64_t strea
 }
 
 template <class Layout>
-__global__ void __launch_bounds__(kFinThreads, 1)
+__global__ void __launch_bounds__(kFinThreads, 4)
     finish_kernel(const __grid_constant__ FinArgs a, const __grid_constant__ Layout lay) {
   constexpr int NT = kFinThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -114,19 +121,19 @@ __global__ void __launch_bounds__(kFinThreads, 1)
     for (uint32_t r = tid; r <= lay.n_req; r += NT) s_cum[r] = lay.cum[r];
   }
   __syncthreads();
-  const bool shrank = ctl->flag & 1u;
 
-  // Bytes of all code chunks, padded.
+  // Bytes of all code chunks, padded. The encode kernel flagged the call if
+  // any code chunk shrinks; otherwise every code chunk is raw and the code
+  // region is the plain array of codes.
+  const bool shrank = ctl->flag & 1u;
   uint64_t total_code = 0;
-  if (a.n_code) {
-    if (!shrank) {
-      total_code = uint64_t(a.n_code - 1) * kChunk +
-                   round16(uint64_t(a.V - (a.n_code - 1) * a.vc) * a.cb);
-    } else {
-      uint64_t part = 0;
-      for (uint32_t c = tid; c < a.n_code; c += NT) part += round16(a.code_size[c]);
-      total_code = block_sum64<NT>(part, ctl->red);
-    }
+  if (!shrank) {
+    if (a.n_code)
+      total_code = uint64_t(a.n_code - 1) * kChunk + round16(code_len(a, a.n_code - 1));
+  } else {
+    uint64_t part = 0;
+    for (uint32_t c = tid; c < a.n_code; c += NT) part += round16(code_stored_size(a, c));
+    total_code = block_sum64<NT>(part, ctl->red);
   }
 
   // -------------------------------------------------- this CTA's meta chunks --
@@ -176,14 +183,15 @@ __global__ void __launch_bounds__(kFinThreads, 1)
   const uint32_t c1 = uint32_t(uint64_t(b + 1) * a.n_code / nb);
   if (!shrank) {
     for (uint32_t c = c0 + tid; c < c1; c += NT)
-      st_u64(a.out + kHeader + 8ull * c, ((uint64_t(c) * kChunk >> 4) << 16) | a.code_size[c]);
+      st_u64(a.out + kHeader + 8ull * c, ((uint64_t(c) * kChunk >> 4) << 16) | code_len(a, c));
   } else {
     uint64_t part = 0;
-    for (uint32_t c = tid; c < c0; c += NT) part += round16(a.code_size[c]);
+    for (uint32_t c = tid; c < c0; c += NT) part += round16(code_stored_size(a, c));
     uint64_t base = block_sum64<NT>(part, ctl->red);
     for (uint32_t c = c0; c < c1; c += NT) {  // block-wide scan, NT chunks at a time
       const uint32_t me = c + tid;
-      const uint32_t sz = me < c1 ? a.code_size[me] : 0u;
+      const uint32_t sz = me < c1 ? code_stored_size(a, me) : 0u;
+      if (me < c1) a.code_size[me] = sz;
       uint32_t total;
       const uint32_t ex = block_excl_scan<NT>(uint32_t(round16(sz)) >> 4, ctl->red, total);
       if (me < c1) {
@@ -205,14 +213,16 @@ __global__ void __launch_bounds__(kFinThreads, 1)
   if (tid == 0) bulk_wait_all<0>();
 }
 
-// Moves code chunks left when some code chunk shrank, then places the meta
-// chunks. Chunk c (source data_base + c * 16 KB, destination data_base +
-// code_off[c] <= source) may overwrite only sources of chunks j <= c whose
-// 16 KB slot overlaps its destination; it waits for their read flags.
+// Re-encodes and moves code chunks when some code chunk shrank, then places
+// the meta chunks. Chunk c (raw bytes at data_base + c * 16 KB, destination
+// data_base + code_off[c] <= that) may overwrite only raw bytes of chunks
+// j <= c whose 16 KB slot overlaps its destination; it waits for their read
+// flags.
 __global__ void __launch_bounds__(kFinThreads, 1) compact_kernel(const __grid_constant__ FinArgs a) {
   constexpr int NT = kFinThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *buf = smem;
+  uint8_t *scr = smem + kChunk;
   FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + 2 * kChunk);
   const int tid = threadIdx.x;
   if (tid == 0) {
@@ -230,10 +240,10 @@ __global__ void __launch_bounds__(kFinThreads, 1) compact_kernel(const __grid_co
     const uint32_t c = ctl->tick;
     named_bar_sync(1, NT);
     if (c >= a.n_code) break;
-    const uint32_t size = a.code_size[c];
+    const uint32_t len = code_len(a, c), size = a.code_size[c];
     const uint64_t src = uint64_t(c) * kChunk, dst = a.code_off[c];
-    if (dst != src) {
-      // sources overlapping [dst, dst + padded size) must have been read
+    if (dst != src || size != len) {
+      // raw bytes of chunks overlapping [dst, dst + padded size) must have been read
       const uint32_t j0 = uint32_t(dst / kChunk);
       for (uint32_t j = j0 + tid; j < c; j += NT) {
         const uint64_t t0 = globaltimer();
@@ -248,15 +258,23 @@ __global__ void __launch_bounds__(kFinThreads, 1) compact_kernel(const __grid_co
       __threadfence();
       named_bar_sync(1, NT);
       if (tid == 0) {
-        mbar_arrive_expect_tx(&ctl->full, uint32_t(round16(size)));
-        bulk_g2s(buf, a.out + a.data_base + src, uint32_t(round16(size)), &ctl->full);
+        mbar_arrive_expect_tx(&ctl->full, len);
+        bulk_g2s(buf, a.out + a.data_base + src, len, &ctl->full);
       }
       if (!mbar_wait(&ctl->full, phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
       ++phase;
       if (tid == 0) {
         __threadfence();
-        atomicExch(a.done + c, 1u);  // source read
+        atomicExch(a.done + c, 1u);  // raw bytes read
         atomicAdd(a.ticket + 1, 1u);
+      }
+      if (size != len) {  // shrinks: bit-plane shuffle + zero-byte elimination
+        ze_encode<NT>(buf, scr, ctl->red);
+        for (uint32_t i = size + tid; i < round16(size); i += NT) buf[i] = 0;
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, NT);
+      if (tid == 0) {
         bulk_s2g(a.out + a.data_base + dst, buf, uint32_t(round16(size)));
         bulk_commit();
         bulk_wait_read<0>();

@@ -30,18 +30,20 @@ constexpr uint32_t kNoTile = 0xFFFFFFFFu;
 
 // Workspace of kvc_compress, in this order (each part 256-byte aligned):
 //   control   status word, flags word (bit 0: some code chunk shrank),
-//             compaction ticket
+//             compaction ticket, compaction read count
 //   meta_nnz  u32 per meta chunk: shuffled-byte nonzero count (accumulated)
+//   code_nnz  u64 per code chunk: the same count (low half) and the number
+//             of 32-vector blocks accumulated so far (high half)
 //   done      u32 per code chunk: compaction read flags
-//   code_size u32 per code chunk
-//   meta_size u32 per meta chunk
+//   code_size u32 per code chunk: stored size
+//   meta_size u32 per meta chunk: stored size
 //   code_off  u64 per code chunk: final offsets (compaction only)
-//   meta      16 KB per meta chunk: raw meta, then (compaction only) the
-//             chunk as stored
-// Only control, meta_nnz and done need zeroing per call.
+//   meta      raw meta of every vector (meta chunk s at s * 16 KB), then
+//             (compaction only) each meta chunk as stored
+// Only control, meta_nnz, code_nnz and done need zeroing per call.
 constexpr size_t kWsCtl = 256;
 struct WsLayout {
-  size_t meta_nnz, done, code_size, meta_size, code_off, meta, total, zero_bytes;
+  size_t meta_nnz, code_nnz, done, code_size, meta_size, code_off, meta, total, zero_bytes;
 };
 
 KVC_HD uint64_t round16(uint64_t x) { return (x + 15u) & ~uint64_t(15); }
@@ -50,7 +52,8 @@ KVC_HD uint64_t round256(uint64_t x) { return (x + 255u) & ~uint64_t(255); }
 inline WsLayout ws_layout(uint64_t n_code, uint64_t n_meta) {
   WsLayout w{};
   w.meta_nnz = kWsCtl;
-  w.done = w.meta_nnz + round256(4 * n_meta);
+  w.code_nnz = w.meta_nnz + round256(4 * n_meta);
+  w.done = w.code_nnz + round256(8 * n_code);
   w.code_size = w.done + round256(4 * n_code);
   w.meta_size = w.code_size + round256(4 * n_code);
   w.code_off = w.meta_size + round256(4 * n_meta);
@@ -119,16 +122,15 @@ struct PagedLayout {
   uint32_t cum[KVC_MAX_REQUESTS + 1];   // token prefix per request
 };
 
-// Main encode kernel: quantize and place every code chunk at its raw-layout
-// position (data base + c * 16 KB); meta slices go to the workspace.
+// Main encode kernel: codes of vector v to data base + v * CB (the raw code
+// region), raw meta to the workspace, nonzero counts per chunk.
 struct EncArgs {
   uint32_t V;          // vectors
-  uint32_t n_tiles;    // code chunks (one tile = one code chunk)
   uint8_t *out;
   uint64_t data_base;
   uint32_t *status;
-  uint32_t *flags;
-  uint32_t *code_size;
+  uint32_t *flags;     // bit 0: some code chunk shrinks
+  unsigned long long *code_nnz;
   uint32_t *meta_nnz;
   uint8_t *ws_meta;
   uint32_t sign_mask[128];
@@ -146,8 +148,9 @@ struct FinArgs {
   uint32_t *status;
   uint32_t *flags;
   uint32_t *ticket;
-  const uint32_t *code_size;
+  const unsigned long long *code_nnz;
   const uint32_t *meta_nnz;
+  uint32_t *code_size;
   uint32_t *done;
   uint32_t *meta_size;
   uint64_t *code_off;

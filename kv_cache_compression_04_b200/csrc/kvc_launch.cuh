@@ -25,11 +25,14 @@ inline cudaError_t prepare(Kernel k, size_t smem) {
 template <int D, int BITS, int G, class Layout>
 cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
   auto k = encode_kernel<D, BITS, G, Layout>;
-  const size_t smem = enc_smem_bytes<D, BITS, G>(kIsPaged<Layout>);
+  const size_t smem = enc_smem_bytes<D>(kIsPaged<Layout>);
   struct Tag {};
   cudaError_t e = prepare<Tag>(k, smem);
   if (e != cudaSuccess) return e;
-  const int grid = int(a.n_tiles < uint32_t(sms) ? a.n_tiles : uint32_t(sms));
+  // one CTA per SM; warps take blocks of 32 vectors round-robin
+  const uint32_t n_blocks = (a.V + 31) / 32;
+  const uint32_t want = (n_blocks + kEncWarps - 1) / kEncWarps;
+  const int grid = int(want < uint32_t(sms) ? want : uint32_t(sms));
   k<<<grid, kEncThreads, smem, st>>>(a, lay);
   return cudaGetLastError();
 }
@@ -37,7 +40,7 @@ cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_
 template <int D, class Layout>
 cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_t st) {
   auto k = decode_kernel<D, Layout>;
-  const size_t smem = dec_smem_bytes<D>(kIsPaged<Layout>);
+  const size_t smem = DecSmem<D>::bytes(kIsPaged<Layout>);
   struct Tag {};
   cudaError_t e = prepare<Tag>(k, smem);
   if (e != cudaSuccess) return e;
@@ -45,7 +48,7 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
   const uint64_t min_vc = uint64_t(kChunk) / (uint64_t(D) * 4 / 8);
   const uint64_t tiles = (uint64_t(a.V) + min_vc - 1) / min_vc;
   const int grid = tiles == 0 ? 1 : int(tiles < uint64_t(sms) ? tiles : uint64_t(sms));
-  k<<<grid, kThreads, smem, st>>>(a, lay);
+  k<<<grid, kDecThreads, smem, st>>>(a, lay);
   return cudaGetLastError();
 }
 

@@ -95,6 +95,7 @@ def lib():
                 "orc_f16_to_f32": (C.c_float, [C.c_uint16]),
                 "orc_f32_to_f16_rd": (C.c_uint16, [C.c_float]),
                 "orc_f32_to_f16_ru": (C.c_uint16, [C.c_float]),
+                "orc_quantize_scalar": (C.c_int, [C.c_float, C.c_float, C.c_float, C.c_int]),
                 "orc_quantize_vector": (C.c_int, [u16p, C.c_int, C.c_int,
                                                   C.c_int, u64p, u8p, u8p]),
                 "orc_dequantize_vector": (None, [u8p, u8p, C.c_int, C.c_int,
@@ -188,6 +189,10 @@ def bf16_to_f32(b: int) -> float:
 # --------------------------------------------------------------------------
 # vectors
 # --------------------------------------------------------------------------
+def quantize_scalar(y: float, zf: float, r: float, qmax: int) -> int:
+    return lib().orc_quantize_scalar(y, zf, r, qmax)
+
+
 def quantize_vectors(x: np.ndarray, bits: int, group: int, seed: int):
     """x: uint16 [V, d] bf16 bits -> (status, codes [V, d*b/8], meta [V, d/g*4])."""
     x = np.ascontiguousarray(x, np.uint16)

@@ -177,6 +177,18 @@ void orc_unpack_codes(const uint8_t *packed, int d, int bits, uint8_t *q) {
     q[c] = (uint8_t)((packed[c / per] >> ((c % per) * bits)) & mask);
 }
 
+/* One code of reading R5: t = fl(y - zf), then the exact real t*r rounded to
+ * the nearest integer (ties to even) and clamped to [0, qmax]. t and r are
+ * fp32, so their product has at most 48 significant bits and is exact in
+ * double; rint() in the default rounding mode is round-half-even. */
+int orc_quantize_scalar(float y, float zf, float r, int qmax) {
+  float t = y - zf;
+  double n = nearbyint((double)t * (double)r);
+  if (n < 0.0) n = 0.0;
+  if (n > (double)qmax) n = (double)qmax;
+  return (int)n;
+}
+
 /* ========================================================================== */
 /* Quantization of one vector ([P2] Methodology: distribution transformation  */
 /* then low-bit quantization; [P3]: only this step loses information).        */
@@ -185,8 +197,9 @@ void orc_unpack_codes(const uint8_t *packed, int d, int bits, uint8_t *q) {
 /*   mn, mx = group min and max, then mn+0, mx+0 (so -0 becomes +0);          */
 /*   z_h = RD16(mn * 2^-k),  zf = f32(z_h) * 2^k;                             */
 /*   s32 = (mx - zf) / (2^b - 1),  s_h = RU16(s32 * 2^-k), sf = f32(s_h)*2^k; */
-/*   r = 0 if s_h == 0 else 1/sf;                                             */
-/*   q = clamp(RNE((y - zf) * r), 0, 2^b - 1).                                */
+/*   r = 0 if s_h == 0 else 1/sf;  t = y - zf (one fp32 rounding);         */
+/*   q = clamp(nearest integer to the exact product t*r, ties to even,       */
+/*             0, 2^b - 1): the product is not rounded to fp32 first.        */
 /* Directed rounding makes the grid zf + q*sf cover [mn, mx]. A non-finite y  */
 /* gives NONFINITE; an infinite z_h or s_h gives RANGE (reading R8). The meta */
 /* of group j is 4 bytes: s_h then z_h, little-endian.                        */
@@ -236,13 +249,7 @@ int orc_quantize_vector(const uint16_t *x, int d, int bits, int g,
       for (c = 0; c < g; c++) q[j * g + c] = 0;
     } else {
       r = ((sh & 0x7FFFu) == 0) ? 0.0f : 1.0f / sf;
-      for (c = 0; c < g; c++) {
-        float t = (yg[c] - zf) * r;
-        float n = nearbyintf(t); /* default mode: nearest, ties to even */
-        if (n < 0.0f) n = 0.0f;
-        if (n > (float)qmax) n = (float)qmax;
-        q[j * g + c] = (uint8_t)n;
-      }
+      for (c = 0; c < g; c++) q[j * g + c] = (uint8_t)orc_quantize_scalar(yg[c], zf, r, qmax);
     }
     meta[4 * j + 0] = (uint8_t)(sh & 0xFF);
     meta[4 * j + 1] = (uint8_t)(sh >> 8);

@@ -60,6 +60,7 @@ uint16_t orc_f32_to_f16_rd(float x);
 uint16_t orc_f32_to_f16_ru(float x);
 
 /* ---- one vector ----------------------------------------------------------- */
+int orc_quantize_scalar(float y, float zf, float r, int qmax);
 int orc_quantize_vector(const uint16_t *x, int d, int bits, int g,
                         const uint64_t *sign_words, uint8_t *codes,
                         uint8_t *meta);

@@ -197,3 +197,50 @@ def test_nonfinite_and_range_errors():
     assert st == oracle.OK
     assert int(meta[0, 2]) | (int(meta[0, 3]) << 8) == f16_bits(65504.0)
     assert int(meta[0, 0]) | (int(meta[0, 1]) << 8) == f16_bits(1095.0)
+
+
+def _nearest_even(fr):
+    """Nearest integer to a Fraction, ties to even (exact)."""
+    from fractions import Fraction
+    n = fr.numerator // fr.denominator
+    rem = fr - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return n
+
+
+def test_quantizer_rounds_the_exact_product():
+    """Reading R5: the code is the nearest integer to the exact real t*r, not
+    to fl32(t*r). Cases are built where t*r lies within half an fp32 ulp of
+    n + 1/2 (so fl32(t*r) is the tie n + 1/2) but not on it; the two readings
+    then differ, and exact rational arithmetic decides."""
+    from fractions import Fraction
+    rng = np.random.default_rng(7)
+    found = {"up": 0, "down": 0, "tie": 0}
+    for _ in range(4000):
+        sf = np.float32(np.float16(rng.uniform(0.01, 4.0))) * np.float32(8)
+        r = np.float32(1) / sf
+        qmax = 15
+        n = int(rng.integers(0, qmax))
+        t0 = np.float32((n + 0.5) / float(r))
+        for t in (np.nextafter(t0, np.float32(-np.inf)), t0, np.nextafter(t0, np.float32(np.inf))):
+            exact = Fraction(float(t)) * Fraction(float(r))
+            want = min(max(_nearest_even(exact), 0), qmax)
+            got = oracle.quantize_scalar(float(t), 0.0, float(r), qmax)
+            assert got == want, (float(t), float(r), got, want)
+            sep = int(np.rint(np.float32(t) * np.float32(r)))
+            if exact == Fraction(2 * n + 1, 2):
+                found["tie"] += 1
+            elif sep != want:
+                found["up" if want > sep else "down"] += 1
+    # the readings really were separated, in both directions
+    assert found["up"] > 0 and found["down"] > 0, found
+
+
+def test_quantizer_scalar_clamps_and_subtracts_once():
+    # t = fl(y - zf) is rounded before the product: y - zf = 1 + 2^-24 rounds to 1
+    y, zf = float(np.float32(1.0)), float(np.float32(-2.0 ** -24))
+    assert oracle.quantize_scalar(y, zf, 2.5, 15) == 2      # exact 2.5 -> even
+    assert oracle.quantize_scalar(y, zf, 3.5, 15) == 4      # exact 3.5 -> even
+    assert oracle.quantize_scalar(100.0, 0.0, 1.0, 15) == 15
+    assert oracle.quantize_scalar(0.0, 1.0, 1.0, 15) == 0
