@@ -277,47 +277,102 @@ __device__ __forceinline__ uint32_t chunk_nnz_part(const uint8_t *buf) {
   return n;
 }
 
+// Plane words: the shuffled chunk as 4096 little-endian words, word
+// p * 128 + m holding bit p of words 32m .. 32m+31 (bytes p*512 + 4m ..).
+//
+// Thread m (< 128) transposes words 32m .. 32m+31 in registers. It moves its
+// eight 16-byte pieces in an order rotated by m, so that the eight threads of
+// a shared-memory phase hit eight different bank groups; the rotation of the
+// words by r = 4 * (m % 8) becomes a rotation of every transposed word by r,
+// undone (or applied) by a funnel shift.
+__device__ __forceinline__ void planes_from_words(const uint8_t *buf, uint32_t *pw, int m) {
+  const uint4 *src = reinterpret_cast<const uint4 *>(buf + m * 128);
+  uint32_t a[32];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint4 v = src[(q + m) & 7];  // words 4q + r .. (mod 32)
+    a[4 * q] = v.x, a[4 * q + 1] = v.y, a[4 * q + 2] = v.z, a[4 * q + 3] = v.w;
+  }
+  transpose32(a);
+  const int r = 4 * (m & 7);
+#pragma unroll
+  for (int p = 0; p < 32; ++p) pw[p * 128 + m] = __funnelshift_l(a[p], a[p], r);
+}
+__device__ __forceinline__ void words_from_planes(const uint32_t *pw, uint8_t *buf, int m) {
+  const int r = 4 * (m & 7);
+  uint32_t a[32];
+#pragma unroll
+  for (int p = 0; p < 32; ++p) {
+    const uint32_t x = pw[p * 128 + m];
+    a[p] = __funnelshift_r(x, x, r);
+  }
+  transpose32(a);  // a[l] = word (l + r) mod 32 of the group
+  uint4 *dst = reinterpret_cast<uint4 *>(buf + m * 128);
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    dst[(q + m) & 7] = make_uint4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+}
+
+// Nonzero-byte mask of a word: bit b set iff byte b is nonzero.
+__device__ __forceinline__ uint32_t nz_nibble(uint32_t x) {
+  uint32_t t = x | (x >> 4);
+  t |= t >> 2;
+  t |= t >> 1;
+  t &= 0x01010101u;
+  return (t | (t >> 7) | (t >> 14) | (t >> 21)) & 0xFu;
+}
+
+// Inclusive prefix sum over the warp.
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x;
+}
+
 // buf holds a full 16 KB chunk; on return it holds bitmap + nonzero bytes
 // (the caller knows their count from chunk_nnz_part). scr: 16 KB scratch.
+// Run by the first NT threads (NT >= 128, a multiple of 32 dividing 4096).
+// Each warp compacts a contiguous eighth (for NT = 256) of the plane words:
+// one pass counts its nonzero bytes, a block scan of the warp totals gives
+// each warp's output base, a second pass places bytes and bitmap words.
 template <int NT>
 __device__ __forceinline__ void ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *red) {
-  const int tid = threadIdx.x;
-  for (int m = tid; m < 128; m += NT) {  // block m = words 32m .. 32m+31
-    uint32_t a[32];
-    const uint4 *src = reinterpret_cast<const uint4 *>(buf + m * 128);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const uint4 v = src[q];
-      a[4 * q] = v.x, a[4 * q + 1] = v.y, a[4 * q + 2] = v.z, a[4 * q + 3] = v.w;
-    }
-    transpose32(a);
-    uint32_t *dst = reinterpret_cast<uint32_t *>(scr);
-#pragma unroll
-    for (int p = 0; p < 32; ++p) dst[p * 128 + m] = a[p];
-  }
+  constexpr int NW = NT / 32, PER_WARP = 4096 / NW, ROUNDS = PER_WARP / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t *pw = reinterpret_cast<uint32_t *>(scr);
+  for (int m = tid; m < 128; m += NT) planes_from_words(buf, pw, m);
   named_bar_sync(1, NT);
-  constexpr int kBytes = kChunk / NT;  // shuffled bytes per thread
-  constexpr int kMaskWords = kBytes / 32;
-  const uint32_t *w = reinterpret_cast<const uint32_t *>(scr + tid * kBytes);
-  uint32_t mask[kMaskWords], cnt = 0;
-#pragma unroll
-  for (int mw = 0; mw < kMaskWords; ++mw) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) m |= (((w[mw * 8 + i / 4] >> (8 * (i % 4))) & 0xFFu) ? 1u : 0u) << i;
-    mask[mw] = m;
-    cnt += __popc(m);
-  }
-  uint32_t total;
-  const uint32_t pos = block_excl_scan<NT>(cnt, red, total);
-  uint32_t *bm = reinterpret_cast<uint32_t *>(buf) + tid * kMaskWords;
-#pragma unroll
-  for (int mw = 0; mw < kMaskWords; ++mw) bm[mw] = mask[mw];
-  uint32_t o = kBitmap + pos;
+  const int w0 = warp * PER_WARP;
+  uint32_t cnt = 0;
 #pragma unroll 4
-  for (int i = 0; i < kBytes; ++i) {
-    const uint32_t byte = (w[i / 4] >> (8 * (i % 4))) & 0xFFu;
-    if (byte && o < uint32_t(kChunk)) buf[o++] = uint8_t(byte);
+  for (int r = 0; r < ROUNDS; ++r) cnt += __popc(nz_nibble(pw[w0 + 32 * r + lane]));
+  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+  if (lane == 0) red[warp] = cnt;
+  named_bar_sync(1, NT);
+  uint32_t run = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) run += w < warp ? red[w] : 0u;
+  named_bar_sync(1, NT);  // red may be reused by the caller
+  uint32_t *bm = reinterpret_cast<uint32_t *>(buf);
+#pragma unroll 2
+  for (int r = 0; r < ROUNDS; ++r) {
+    const int i = w0 + 32 * r + lane;
+    const uint32_t x = pw[i], n = nz_nibble(x), c = __popc(n);
+    const uint32_t incl = warp_incl_scan(c);
+    uint32_t off = kBitmap + run + incl - c;
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      if ((n >> b) & 1u) buf[off++] = uint8_t(x >> (8 * b));
+    uint32_t word = n << (4 * (lane & 7));
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+    if ((lane & 7) == 0) bm[i >> 3] = word;
+    run += __shfl_sync(0xFFFFFFFFu, incl, 31);
   }
   named_bar_sync(1, NT);
 }
@@ -327,44 +382,41 @@ __device__ __forceinline__ void ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *
 // popcount disagrees with the size; then buf is unspecified.
 template <int NT>
 __device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *red, uint32_t size) {
-  const int tid = threadIdx.x;
-  constexpr int kBytes = kChunk / NT;
-  constexpr int kMaskWords = kBytes / 32;
-  uint32_t mask[kMaskWords], cnt = 0;
+  constexpr int NW = NT / 32, PER_WARP = 4096 / NW, ROUNDS = PER_WARP / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t *pw = reinterpret_cast<uint32_t *>(scr);
+  const uint32_t *bm = reinterpret_cast<const uint32_t *>(buf);
+  const int w0 = warp * PER_WARP;
+  uint32_t cnt = 0;
+  for (int j = lane; j < PER_WARP / 8; j += 32) cnt += __popc(bm[w0 / 8 + j]);
+  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+  if (lane == 0) red[warp] = cnt;
+  named_bar_sync(1, NT);
+  uint32_t run = 0, total = 0;
 #pragma unroll
-  for (int mw = 0; mw < kMaskWords; ++mw) {
-    mask[mw] = reinterpret_cast<const uint32_t *>(buf)[tid * kMaskWords + mw];
-    cnt += __popc(mask[mw]);
+  for (int w = 0; w < NW; ++w) {
+    const uint32_t r = red[w];
+    run += w < warp ? r : 0u;
+    total += r;
   }
-  uint32_t total;
-  const uint32_t pos = block_excl_scan<NT>(cnt, red, total);
-  const bool good = total == size - kBitmap;
-  const uint8_t *src = buf + kBitmap + pos;
-  uint32_t *d = reinterpret_cast<uint32_t *>(scr + tid * kBytes);
-  int n = 0;
+  named_bar_sync(1, NT);  // red may be reused by the caller
+  if (total != size - kBitmap) return false;
+#pragma unroll 2
+  for (int r = 0; r < ROUNDS; ++r) {
+    const int i = w0 + 32 * r + lane;
+    const uint32_t n = (bm[i >> 3] >> (4 * (i & 7))) & 0xFu, c = __popc(n);
+    const uint32_t incl = warp_incl_scan(c);
+    uint32_t off = kBitmap + run + incl - c, x = 0;
 #pragma unroll
-  for (int q = 0; q < kBytes / 4; ++q) {
-    uint32_t v = 0;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int i = 4 * q + b;
-      if (good && ((mask[i / 32] >> (i % 32)) & 1u)) v |= uint32_t(src[n++]) << (8 * b);
-    }
-    d[q] = v;
+    for (int b = 0; b < 4; ++b)
+      if ((n >> b) & 1u) x |= uint32_t(buf[off++]) << (8 * b);
+    pw[i] = x;
+    run += __shfl_sync(0xFFFFFFFFu, incl, 31);
   }
   named_bar_sync(1, NT);
-  for (int m = tid; m < 128; m += NT) {  // plane words (p, m) -> words 32m .. 32m+31
-    uint32_t a[32];
-    const uint32_t *s = reinterpret_cast<const uint32_t *>(scr);
-#pragma unroll
-    for (int p = 0; p < 32; ++p) a[p] = s[p * 128 + m];
-    transpose32(a);
-    uint4 *o = reinterpret_cast<uint4 *>(buf + m * 128);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) o[q] = make_uint4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
-  }
+  for (int m = tid; m < 128; m += NT) words_from_planes(pw, buf, m);
   named_bar_sync(1, NT);
-  return good;
+  return true;
 }
 
 // --------------------------------------------------------- addressing --

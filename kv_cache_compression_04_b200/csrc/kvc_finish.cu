@@ -25,7 +25,7 @@ cudaError_t launch_fin(const FinArgs &a, const Layout &lay, int sms, cudaStream_
   struct CompactTag {};
   e = prepare<CompactTag>(ck, csmem);
   if (e != cudaSuccess) return e;
-  const int cgrid = int(a.n_code < uint32_t(sms) ? a.n_code : uint32_t(sms));
+  const int cgrid = int(a.n_code < cap ? a.n_code : cap);
   ck<<<cgrid, kFinThreads, csmem, st>>>(a);
   return cudaGetLastError();
 }

@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kFinThreads, 4)
 // data_base + code_off[c] <= that) may overwrite only raw bytes of chunks
 // j <= c whose 16 KB slot overlaps its destination; it waits for their read
 // flags.
-__global__ void __launch_bounds__(kFinThreads, 1) compact_kernel(const __grid_constant__ FinArgs a) {
+__global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_constant__ FinArgs a) {
   constexpr int NT = kFinThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *buf = smem;
@@ -243,20 +243,10 @@ __global__ void __launch_bounds__(kFinThreads, 1) compact_kernel(const __grid_co
     const uint32_t len = code_len(a, c), size = a.code_size[c];
     const uint64_t src = uint64_t(c) * kChunk, dst = a.code_off[c];
     if (dst != src || size != len) {
-      // raw bytes of chunks overlapping [dst, dst + padded size) must have been read
-      const uint32_t j0 = uint32_t(dst / kChunk);
-      for (uint32_t j = j0 + tid; j < c; j += NT) {
-        const uint64_t t0 = globaltimer();
-        for (uint32_t it = 0; *reinterpret_cast<volatile uint32_t *>(a.done + j) == 0; ++it) {
-          if (spin_expired(it, t0, a.status)) {
-            set_status(a.status, KVC_ERR_TIMEOUT);
-            break;
-          }
-          __nanosleep(64);
-        }
-      }
-      __threadfence();
-      named_bar_sync(1, NT);
+      // The raw bytes of chunk c are never overwritten before it reads them
+      // (chunk j < c writes below code_off[j + 1] <= code_off[c] <= c * 16 KB),
+      // so every chunk loads at once; only its store waits, for the chunks
+      // whose raw bytes [dst, dst + padded size) overlaps to have been read.
       if (tid == 0) {
         mbar_arrive_expect_tx(&ctl->full, len);
         bulk_g2s(buf, a.out + a.data_base + src, len, &ctl->full);
@@ -272,6 +262,19 @@ __global__ void __launch_bounds__(kFinThreads, 1) compact_kernel(const __grid_co
         ze_encode<NT>(buf, scr, ctl->red);
         for (uint32_t i = size + tid; i < round16(size); i += NT) buf[i] = 0;
       }
+      const uint32_t j0 = uint32_t(dst / kChunk);
+      const uint32_t j1 = uint32_t((dst + round16(size) - 1) / kChunk);  // <= c
+      for (uint32_t j = j0 + tid; j <= j1 && j < c; j += NT) {
+        const uint64_t t0 = globaltimer();
+        for (uint32_t it = 0; *reinterpret_cast<volatile uint32_t *>(a.done + j) == 0; ++it) {
+          if (spin_expired(it, t0, a.status)) {
+            set_status(a.status, KVC_ERR_TIMEOUT);
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+      __threadfence();
       fence_proxy_async_smem();
       named_bar_sync(1, NT);
       if (tid == 0) {
