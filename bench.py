@@ -35,6 +35,39 @@ METRIC = "encode/decode GB/s of raw bf16 KV on 1 B200 and % of HBM roofline; rat
 FALLBACK_HBM_GBS = 6650.0
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_llama8b.txt")
+
+
+def kernel_source_sha() -> str:
+    """Digest of the CUDA sources and the ABI header (a recorded DRAM-traffic
+    figure is stale once any of them changed)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kv_cache_compression_04_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
+                   glob.glob(os.path.join(csrc, "*.h"))) + [os.path.join(ROOT, "include", "kvc.h")]
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per compress / decompress call from the committed ncu
+    summary, or None if it is missing, for another workload, or stale."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            kv = dict(l.split(":", 1) for l in f.read().splitlines() if ":" in l and not l.startswith("#"))
+        kv = {k.strip(): v.strip() for k, v in kv.items()}
+        if kv.get("source_sha") != kernel_source_sha() or kv.get("workload") != workload:
+            return None
+        return {"encode": int(kv["compress_dram_bytes_per_call"]),
+                "decode": int(kv["decompress_dram_bytes_per_call"])}
+    except Exception:
+        return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -46,57 +79,97 @@ def peaks():
 
 # ------------------------------------------------------------------ clocks --
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """SM clocks and clock-event (throttle) reasons sampled while the timed
+    region runs: NVML polled every millisecond from a thread (the region can
+    be tens of milliseconds, shorter than nvidia-smi's sampling period);
+    nvidia-smi in loop mode if NVML is unavailable. Reads only."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
-        self.file = None
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []          # (sm_mhz, max_mhz, set of reason names)
+        self.mode = None
+        self.stop = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+        return pynvml, pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+
+    def _poll(self, nv, h):
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+
+        def sample():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), {n for n, b in bits.items() if r & b}))
+            except Exception:
+                pass
+        sample()  # at least one sample at each end of a very short region
+        while not self.stop.is_set():
+            time.sleep(0.001)
+            sample()
 
     def __enter__(self):
         try:
+            nv, h = self._nvml_handle()
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.mode = "nvml"
+            self.thread.start()
+            return self
+        except Exception:
+            pass
+        try:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                ["nvidia-smi", f"--id={self.cuda_index}", f"--query-gpu={self.Q}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.file, stderr=subprocess.DEVNULL)
+            self.mode = "nvidia-smi"
         except Exception:
-            self.proc = None
+            self.mode = None
         return self
 
     def __exit__(self, *a):
-        if self.proc is not None:
+        if self.mode == "nvml":
+            self.stop.set()
+            self.thread.join(timeout=5)
+        elif self.mode == "nvidia-smi":
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+            self.file.flush()
+            self.file.seek(0)
+            for line in self.file.read().splitlines():
+                r = line.strip().split(", ")
+                try:
+                    self.samples.append((float(r[1]), float(r[2]),
+                                         {n for n, v in zip(self.NAMES, r[5:9])
+                                          if v.strip().lower() == "active"}))
+                except Exception:
+                    continue
+            os.unlink(self.file.name)
 
     def summary(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.file.flush()
-        self.file.seek(0)
-        rows = [l.strip().split(", ") for l in self.file.read().splitlines() if l.strip()]
-        os.unlink(self.file.name)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
-                for n, v in zip(names, r[5:9]):
-                    if v.strip().lower() == "active":
-                        reasons.add(n)
-            except Exception:
-                continue
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None,
+                    "reasons": ["no samples" if self.mode else "no NVML / nvidia-smi"]}
+        reasons = set().union(*(s[2] for s in self.samples))
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples), "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": self.mode}
 
 
 # -------------------------------------------------------------- workloads --
@@ -192,11 +265,28 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------ multi-rank timing --
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of per-rank timings (every rank gets the result).
+    Each rank times its own work on the device; the job's time is the
+    slowest rank's."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_gbs(raw_bytes_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the raw bytes all ranks processed / the time."""
+    return raw_bytes_per_rank * world / (ms * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ main --
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama8b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -270,17 +360,17 @@ def main():
             dec(nbytes)
             ev[i][2].record(stream)
         stop.record(stream)
+        # poll instead of blocking so the clock sampler thread keeps running
+        while not stop.query():
+            time.sleep(0.0002)
         torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
     total_ms = start.elapsed_time(stop)
     enc_ms = [a.elapsed_time(b) for a, b, _ in ev]
     dec_ms = [b.elapsed_time(c) for _, b, c in ev]
-    stats = torch.tensor([total_ms, sum(enc_ms) / K, sum(dec_ms) / K], device=dev,
-                         dtype=torch.float64)
-    if dist:
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
-    total_ms, enc_avg, dec_avg = stats.tolist()
+    total_ms, enc_avg, dec_avg = max_over_ranks([total_ms, sum(enc_ms) / K, sum(dec_ms) / K],
+                                                dist, dev)
     assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
     assert kvc.kvc_stream_status(dws.data_ptr(), sp) == kvc.KVC_OK
 
@@ -310,12 +400,9 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        t = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-        if dist:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item() / args.e2e_steps
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0] / args.e2e_steps
         inb = src.numel() * src.element_size()
-        e2e = {"value": round(raw * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+        e2e = {"value": round(job_gbs(raw, world, e2e_ms), 3), "unit": "GB/s",
                "h2d_bytes_per_step": inb + nbytes, "d2h_bytes_per_step": nbytes + inb,
                "ms_per_step": round(e2e_ms, 3)}
         assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
@@ -327,8 +414,9 @@ def main():
         return 0
 
     hbm, peak_kind = peaks()
+    traffic = recorded_traffic(args.workload)
     step_ms = total_ms / K
-    value = raw * world / (step_ms * 1e-3) / 1e9
+    value = job_gbs(raw, world, step_ms)
     enc_bytes = raw + nbytes            # algorithmic: read KV, write stream
     dec_bytes = nbytes + raw            # read stream, write KV
     enc_gbs = enc_bytes / (enc_avg * 1e-3) / 1e9
@@ -353,9 +441,9 @@ def main():
         "break_even_gbit_s": round(saved_bits / t_codec / 1e9, 1),
         "net_gain_ms": {"100Gbit": round((saved_bits / 100e9 - t_codec) * 1e3, 3),
                         "400Gbit": round((saved_bits / 400e9 - t_codec) * 1e3, 3)},
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+        "roofline": {"bound": "hbm", "kernel": {"encode": "kvc_compress call (encode + finish + compaction kernels)", "decode": "kvc_decompress call (decode kernel)"}[dom], "achieved": round(achieved, 1),
                      "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                     "peak_kind": peak_kind, "traffic": None,
+                     "peak_kind": peak_kind, "traffic": traffic[dom] if traffic else None,
                      "encode_frac": round(enc_gbs / hbm, 4),
                      "decode_frac": round(dec_gbs / hbm, 4)},
         "gpu_launches": 4 * K,  # encode, finish, compaction (returns at once unless a code chunk shrank), decode

@@ -292,3 +292,40 @@ def test_full_paged_sampled():
     _segment_check(w, od, gstream, rows, segs)
     del pk
     torch.cuda.empty_cache()
+
+
+# -------------------------------------------------------------------- sweep --
+@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("i", [0, 2, 5])
+def test_sweep_small_sizes_full(i, bits):
+    """Message-size sweep, small end (T = 8 * 2^i tokens): whole streams and
+    whole decodes compared."""
+    w = synth.workload(f"sweep-{i}-{bits}")
+    kv = synth.dense_kv(w, device="cuda")
+    _roundtrip_dense(kv, w.bits, w.group)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_sweep_largest_size_sampled(bits):
+    """Message-size sweep, 4 GiB end (T = 32768): chunk table consistency over
+    the whole stream, sampled segments against the oracle, sampled decode."""
+    w = synth.workload(f"sweep-12-{bits}")
+    kv = synth.dense_kv(w, device="cuda")
+    flat = kv.view(-1, 128)
+    od = oracle_desc(w.bits, w.group, 128, w.layers, w.kv_heads, [w.tokens])
+    st, gstream, _, _ = gpu_compress(kvc.dense_desc(kv), w.bits, w.group)
+    assert st == kvc.KVC_OK
+    lay = od.layout()
+    rng = np.random.default_rng(12 + bits)
+    segs = sorted({0, int(lay.n_seg) - 1, *rng.integers(0, lay.n_seg, 6).tolist()})
+    _segment_check(w, od, gstream, lambda a, b: u16(flat[a:b]), segs)
+    out = torch.empty_like(kv)
+    assert gpu_decompress(gstream, kvc.dense_desc(out)) == kvc.KVC_OK
+    oflat = out.view(-1, 128)
+    for s in segs[:3]:
+        v0, v1 = oracle.segment_vectors(lay, s)
+        _, chunks = oracle.encode_segment(od, s, u16(flat[v0:v1]))
+        _, ref = oracle.decode_segment(od, s, chunks, v1 - v0)
+        assert np.array_equal(u16(oflat[v0:v1]), ref), s
+    del kv, out, flat, oflat
+    torch.cuda.empty_cache()
