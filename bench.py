@@ -320,7 +320,7 @@ def main():
     codec = kvc.Codec(w.bits, w.group, w.sign_seed)
     out, ws, nb = codec.buffers(desc, dev)
     odesc, obuf = out_desc_fn()
-    dws = torch.empty(kvc.KVC_DECOMPRESS_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
+    dws = torch.empty(kvc.kvc_decompress_workspace_bytes(odesc), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     sp = kvc._stream_ptr(stream)
     raw = w.raw_bytes

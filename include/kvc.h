@@ -79,8 +79,6 @@ enum { KVC_DENSE = 0, KVC_PAGED = 1 };
 
 /* Largest request count of a paged descriptor. */
 #define KVC_MAX_REQUESTS 1024
-/* Workspace bytes kvc_decompress needs (it only keeps a status word). */
-#define KVC_DECOMPRESS_WORKSPACE_BYTES 256
 
 /* A KV cache: logical shape [layers, 2 (K, V), kv_heads, tokens, head_dim],
  * bf16, head_dim contiguous. Vectors are coded in the logical order
@@ -127,10 +125,17 @@ typedef struct {
 size_t kvc_max_compressed_bytes(const kvc_kv_desc *kv, const kvc_params *params);
 
 /* Workspace bytes kvc_compress needs for this shape (DEVICE memory, 16-byte
- * aligned, caller-owned, contents need not be initialized). kvc_decompress
- * needs KVC_DECOMPRESS_WORKSPACE_BYTES. Returns 0 for an invalid
- * description. */
+ * aligned, caller-owned, contents need not be initialized). Returns 0 for an
+ * invalid description. */
 size_t kvc_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params);
+
+/* Workspace bytes kvc_decompress needs to decode into `out` (DEVICE memory,
+ * 16-byte aligned, caller-owned, contents need not be initialized): a status
+ * word plus room to expand the meta chunks that used zero-byte elimination,
+ * sized for the largest meta region any group size gives this shape
+ * (head_dim / 8 bytes per vector, about 6% of the raw bf16 size). Returns 0
+ * for an invalid description. */
+size_t kvc_decompress_workspace_bytes(const kvc_kv_desc *out);
 
 /* Compresses `kv` into `out` (DEVICE, out_capacity bytes, which must be at
  * least kvc_max_compressed_bytes). The stream length is written to the
@@ -149,7 +154,8 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params,
                         kvc_stream_t stream);
 
 /* Decompresses the stream at `in` (DEVICE, in_bytes readable bytes) into the
- * slots described by `out`. Bits, group size and sign seed come from the
+ * slots described by `out`; workspace_bytes must be at least
+ * kvc_decompress_workspace_bytes(out). Bits, group size and sign seed come from the
  * stream. The logical shape must match the stream's: layers, kv_heads,
  * head_dim and total tokens; a paged receiver must also match the stream's
  * request count and per-request token counts. The receiver's layout (dense or

@@ -17,7 +17,6 @@ LIB_PATH = os.path.join(PKG, "libkvc.so")
 
 KVC_DENSE, KVC_PAGED = 0, 1
 KVC_MAX_REQUESTS = 1024
-KVC_DECOMPRESS_WORKSPACE_BYTES = 256
 KVC_NOALLOC_SCRATCH_BYTES = 16 << 20
 STATUS = ["KVC_OK", "KVC_ERR_INVALID_ARG", "KVC_ERR_UNSUPPORTED", "KVC_ERR_CAPACITY",
           "KVC_ERR_NONFINITE", "KVC_ERR_RANGE", "KVC_ERR_CORRUPT", "KVC_ERR_TIMEOUT",
@@ -27,7 +26,8 @@ STATUS = ["KVC_OK", "KVC_ERR_INVALID_ARG", "KVC_ERR_UNSUPPORTED", "KVC_ERR_CAPAC
 
 # Every symbol include/kvc.h declares.
 EXPORTS = ["kvc_max_compressed_bytes", "kvc_workspace_bytes", "kvc_compress",
-           "kvc_decompress", "kvc_stream_status", "kvc_status_string", "kvc_compress_noalloc"]
+           "kvc_decompress", "kvc_stream_status", "kvc_status_string", "kvc_compress_noalloc",
+           "kvc_decompress_workspace_bytes"]
 
 
 class KvcError(RuntimeError):
@@ -68,6 +68,8 @@ def lib() -> C.CDLL:
         L.kvc_max_compressed_bytes.argtypes = [D, P]
         L.kvc_workspace_bytes.restype = C.c_size_t
         L.kvc_workspace_bytes.argtypes = [D, P]
+        L.kvc_decompress_workspace_bytes.restype = C.c_size_t
+        L.kvc_decompress_workspace_bytes.argtypes = [D]
         L.kvc_compress.restype = C.c_int
         L.kvc_compress.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p,
                                    C.c_size_t, C.c_void_p]
@@ -92,6 +94,10 @@ def kvc_max_compressed_bytes(desc: kvc_kv_desc, params: kvc_params) -> int:
 
 def kvc_workspace_bytes(desc: kvc_kv_desc, params: kvc_params) -> int:
     return lib().kvc_workspace_bytes(C.byref(desc), C.byref(params))
+
+
+def kvc_decompress_workspace_bytes(desc: kvc_kv_desc) -> int:
+    return lib().kvc_decompress_workspace_bytes(C.byref(desc))
 
 
 def kvc_compress(desc, params, out_ptr, out_capacity, out_bytes_dev_ptr, ws_ptr, ws_bytes,
@@ -185,7 +191,8 @@ class Codec:
         if cap == 0 or wsb == 0:
             raise KvcError(KVC_ERR_INVALID_ARG, "kvc_max_compressed_bytes")
         out = torch.empty(cap, dtype=torch.uint8, device=device)
-        ws = torch.empty(max(wsb, KVC_DECOMPRESS_WORKSPACE_BYTES), dtype=torch.uint8,
+        # one workspace serves both directions for this shape
+        ws = torch.empty(max(wsb, kvc_decompress_workspace_bytes(desc)), dtype=torch.uint8,
                          device=device)
         nbytes = torch.zeros(1, dtype=torch.int64, device=device)
         return out, ws, nbytes

@@ -87,6 +87,14 @@ kvc_status describe(const kvc_kv_desc *kv, const kvc_params *p, Shape &s) {
   return KVC_OK;
 }
 
+// Meta chunks of the largest meta region any supported group size gives for
+// this shape (group 32: head_dim / 8 bytes per vector).
+uint64_t max_meta_chunks(const Shape &s) {
+  const uint64_t mb = uint64_t(s.D / 32) * 4;
+  return (s.V * mb + kChunk - 1) / kChunk;
+}
+uint64_t decompress_ws_bytes(const Shape &s) { return kWsCtl + max_meta_chunks(s) * kChunk; }
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -133,6 +141,12 @@ size_t kvc_max_compressed_bytes(const kvc_kv_desc *kv, const kvc_params *params)
   Shape s;
   if (!params || describe(kv, params, s) != KVC_OK) return 0;
   return size_t(s.max_bytes);
+}
+
+size_t kvc_decompress_workspace_bytes(const kvc_kv_desc *out) {
+  Shape s;
+  if (describe(out, nullptr, s) != KVC_OK) return 0;
+  return size_t(decompress_ws_bytes(s));
 }
 
 size_t kvc_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params) {
@@ -227,7 +241,7 @@ kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *ou
   kvc_status st = describe(out, nullptr, s);
   if (st != KVC_OK) return st;
   if (!in || !aligned16(in) || !workspace || !aligned16(workspace)) return KVC_ERR_INVALID_ARG;
-  if (workspace_bytes < KVC_DECOMPRESS_WORKSPACE_BYTES) return KVC_ERR_CAPACITY;
+  if (workspace_bytes < decompress_ws_bytes(s)) return KVC_ERR_CAPACITY;
   const int sms = sm_count();
   if (sms <= 0) return KVC_ERR_CUDA;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -242,7 +256,9 @@ kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *ou
   a.tokens = s.T;
   a.V = uint32_t(s.V);
   a.paged_receiver = out->kind == KVC_PAGED ? 1u : 0u;
-  if (cudaMemsetAsync(workspace, 0, KVC_DECOMPRESS_WORKSPACE_BYTES, cs) != cudaSuccess)
+  a.ws_meta = static_cast<uint8_t *>(workspace) + kWsCtl;
+  a.ws_meta_chunks = uint32_t(max_meta_chunks(s));
+  if (cudaMemsetAsync(workspace, 0, kWsCtl, cs) != cudaSuccess)
     return KVC_ERR_CUDA;
   cudaError_t e;
   if (out->kind == KVC_DENSE) {

@@ -27,9 +27,8 @@ constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kZeThreads = 256;  // threads that run the chunk expansion
 
 struct DecCtl {
-  uint64_t cbar[kDecWarps][2];  // per-warp code blocks loaded (two buffers)
-  uint64_t mbar;             // meta chunk loaded
-  uint64_t zbar;             // zero-byte-eliminated code chunk loaded
+  uint64_t cbar[kDecWarps][2];  // per-warp code + meta blocks loaded (two buffers)
+  uint64_t zbar;                // zero-byte-eliminated code chunk loaded
   uint32_t red[kDecThreads / 32];
   uint32_t hdr_ok, bad;
   uint32_t bits, group, n_req_stream, n_chunks;
@@ -37,16 +36,17 @@ struct DecCtl {
   alignas(16) uint32_t mask[128];  // read as uint4
 };
 
-// Shared memory: output rows | per-warp code blocks | meta chunk | expanded
-// code chunk | expansion scratch | control | request prefix (paged).
+// Shared memory: output rows | per-warp code blocks | per-warp meta blocks |
+// expanded code chunk | expansion scratch | control | request prefix (paged).
 template <int D>
 struct DecSmem {
   static constexpr size_t ROWP = 2 * D + 16;
-  static constexpr size_t BLK = 32 * size_t(D) / 2;  // widest code block (4-bit)
+  static constexpr size_t BLK = 32 * size_t(D) / 2;       // widest code block (4-bit)
+  static constexpr size_t MBLK = 32 * (size_t(D) / 32) * 4;  // widest meta block (group 32)
   static constexpr size_t rows = 0;
   static constexpr size_t code = rows + kDecThreads * ROWP;
   static constexpr size_t meta = code + 2 * kDecWarps * BLK;
-  static constexpr size_t zchunk = meta + kChunk;
+  static constexpr size_t zchunk = meta + 2 * kDecWarps * MBLK;
   static constexpr size_t scr = zchunk + kChunk;
   static constexpr size_t ctl = scr + kChunk;
   static constexpr size_t cum = ctl + ((sizeof(DecCtl) + 15) & ~size_t(15));
@@ -60,6 +60,43 @@ __device__ __forceinline__ uint32_t ld_u32(const uint8_t *p) {
 }
 __device__ __forceinline__ uint64_t ld_u64(const uint8_t *p) {
   return *reinterpret_cast<const uint64_t *>(p);
+}
+
+// D1: the header (reading R12) against the receiver's description.
+struct StreamHdr {
+  uint32_t ok, bits, group, n_req, n_chunks;
+  uint64_t data_base, stream_bytes, seed;
+};
+template <int D>
+__device__ __forceinline__ StreamHdr parse_header(const DecArgs &a) {
+  constexpr uint32_t kLog2D = D == 64 ? 6 : D == 128 ? 7 : 8;
+  StreamHdr r{};
+  const uint8_t *h = a.in;
+  if (a.in_bytes < kHeader) return r;
+  const uint32_t bits = h[8], k = h[9], group = ld_u32(h + 12);
+  bool ok = ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 &&
+            (ld_u32(h + 4) >> 16) == kHeader && (bits == 2 || bits == 4) && k == kLog2D / 2 &&
+            (group == 32 || group == 64 || group == 128) && group <= D &&
+            ld_u32(h + 16) == a.layers && ld_u32(h + 20) == 2 && ld_u32(h + 24) == a.kv_heads &&
+            ld_u32(h + 28) == a.head_dim && ld_u64(h + 32) == a.tokens;
+  if (!ok) return r;
+  const uint32_t n_req = ld_u32(h + 48), n_chunks = ld_u32(h + 52);
+  const uint64_t stream_bytes = ld_u64(h + 56);
+  const uint64_t cb = uint64_t(D) * bits / 8, mbv = uint64_t(D / group) * 4;
+  const uint64_t n_code = (uint64_t(a.V) * cb + kChunk - 1) / kChunk;
+  const uint64_t n_meta = (uint64_t(a.V) * mbv + kChunk - 1) / kChunk;
+  const uint64_t base = round16(kHeader + 8ull * n_chunks + 4ull * n_req);
+  ok = n_chunks == n_code + n_meta && base <= stream_bytes && stream_bytes <= a.in_bytes &&
+       (!a.paged_receiver || n_req == a.n_req);
+  r.ok = ok;
+  r.bits = bits;
+  r.group = group;
+  r.n_req = n_req;
+  r.n_chunks = n_chunks;
+  r.data_base = base;
+  r.stream_bytes = stream_bytes;
+  r.seed = ld_u64(h + 40);
+  return r;
 }
 
 template <int D, int BITS, int G>
@@ -186,7 +223,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   const uint8_t *table = in + kHeader;
   uint8_t *row = smem + S::rows + tid * S::ROWP;
   uint8_t *cbuf = smem + S::code + 2 * warp * S::BLK;
-  uint8_t *mbuf = smem + S::meta;
+  uint8_t *mbuf = smem + S::meta + 2 * warp * S::MBLK;
   uint8_t *zbuf = smem + S::zchunk;
   uint8_t *scr = smem + S::scr;
   const uint32_t seg0 = t0 / C::R, seg1 = (t1 - 1) / C::R;
@@ -221,106 +258,106 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     }
   }
 
-  uint32_t mphase = 0, zphase = 0, cphase = 0;  // cphase: bit k for code buffer k
-  bool row_busy = false;
-#pragma unroll 1
-  for (uint32_t s = seg0; s <= seg1; ++s) {
-    // D3: the meta chunk, expanded if it used zero-byte elimination.
+  // D3 for meta: a raw meta chunk is read in place; an eliminated one was
+  // expanded into the workspace by meta_expand_kernel.
+  auto meta_src = [&](uint32_t v0) -> const uint8_t * {
+    const uint32_t s = v0 / C::VM;
     const uint64_t me = ld_u64(table + 8 * (uint64_t(n_tiles) + s));
-    const uint32_t msize = uint32_t(me & 0xFFFFu);
     const uint32_t mlen = min(uint32_t(C::VM), V - s * C::VM) * C::MB;
-    __syncthreads();  // every warp is done with the previous meta chunk
+    const uint8_t *chunk = uint32_t(me & 0xFFFFu) == mlen ? in + base + ((me >> 16) << 4)
+                                                          : a.ws_meta + uint64_t(s) * kChunk;
+    return chunk + uint64_t(v0 - s * C::VM) * C::MB;
+  };
+  // Lane 0 starts the loads of a block's meta bytes and, unless they are
+  // already in shared memory (csrc null), its code bytes, into buffer k.
+  auto issue = [&](uint32_t v0, uint32_t nvec, const uint8_t *csrc, uint32_t k) {
+    if (lane == 0) {
+      const uint32_t cbytes = csrc ? nvec * C::CB : 0u;
+      const uint32_t mbytes = uint32_t(round16(nvec * C::MB));
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&ctl->cbar[warp][k], cbytes + mbytes);
+      if (csrc) bulk_g2s(cbuf + k * S::BLK, csrc, cbytes, &ctl->cbar[warp][k]);
+      bulk_g2s(mbuf + k * S::MBLK, meta_src(v0), mbytes, &ctl->cbar[warp][k]);
+    }
+  };
+  uint32_t cphase = 0;  // bit k: phase of buffer k
+  auto wait = [&](uint32_t k) {
+    if (!mbar_wait(&ctl->cbar[warp][k], (cphase >> k) & 1, a.status))
+      set_status(a.status, KVC_ERR_TIMEOUT);
+    cphase ^= 1u << k;
+  };
+  bool row_busy = false;
+
+  // Phase 1 (rare): code chunks that used zero-byte elimination. The CTA
+  // expands each one into shared memory, then the warps decode its blocks.
+  uint32_t zphase = 0;
+#pragma unroll 1
+  for (uint32_t t = t0; t < t1; ++t) {
+    const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
+    const uint32_t csize = uint32_t(ce & 0xFFFFu);
+    const uint32_t nvec = min(uint32_t(C::VC), V - t * C::VC);
+    if (csize == nvec * C::CB) continue;
+    __syncthreads();  // zbuf free
     if (tid == 0) {
       fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&ctl->mbar, uint32_t(round16(msize)));
-      bulk_g2s(mbuf, in + base + ((me >> 16) << 4), uint32_t(round16(msize)), &ctl->mbar);
+      mbar_arrive_expect_tx(&ctl->zbar, uint32_t(round16(csize)));
+      bulk_g2s(zbuf, in + base + ((ce >> 16) << 4), uint32_t(round16(csize)), &ctl->zbar);
     }
-    if (!mbar_wait(&ctl->mbar, mphase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
-    mphase ^= 1;
-    if (msize != mlen) {
-      bool good = true;
-      if (tid < kZeThreads) good = ze_decode<kZeThreads>(mbuf, scr, ctl->red, msize);
-      if (tid == 0) ctl->bad = !good;
-      __syncthreads();
-      if (ctl->bad) {
-        if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
-        return;
-      }
+    if (!mbar_wait(&ctl->zbar, zphase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+    zphase ^= 1;
+    bool good = true;
+    if (tid < kZeThreads) good = ze_decode<kZeThreads>(zbuf, scr, ctl->red, csize);
+    if (tid == 0) ctl->bad = !good;
+    __syncthreads();
+    if (ctl->bad) {
+      if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
+      return;
     }
-    const uint32_t ts0 = max(t0, s * C::R), ts1 = min(t1, (s + 1) * C::R);
-
-    // Code chunks of this segment that used zero-byte elimination (rare):
-    // the CTA expands each one, then the warps decode its blocks.
 #pragma unroll 1
-    for (uint32_t t = ts0; t < ts1; ++t) {
-      const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
-      const uint32_t csize = uint32_t(ce & 0xFFFFu);
-      const uint32_t nvec = min(uint32_t(C::VC), V - t * C::VC);
-      if (csize == nvec * C::CB) continue;
-      __syncthreads();  // zbuf free
-      if (tid == 0) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&ctl->zbar, uint32_t(round16(csize)));
-        bulk_g2s(zbuf, in + base + ((ce >> 16) << 4), uint32_t(round16(csize)), &ctl->zbar);
-      }
-      if (!mbar_wait(&ctl->zbar, zphase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
-      zphase ^= 1;
-      bool good = true;
-      if (tid < kZeThreads) good = ze_decode<kZeThreads>(zbuf, scr, ctl->red, csize);
-      if (tid == 0) ctl->bad = !good;
-      __syncthreads();
-      if (ctl->bad) {
-        if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
-        return;
-      }
-      for (uint32_t b = warp; b * 32 < nvec; b += kDecWarps) {
-        const uint32_t v0 = t * C::VC + b * 32;
-        decode_block<D, BITS, G>(a, lay, cum, zbuf + b * 32 * C::CB,
-                                 mbuf + (v0 - s * C::VM) * C::MB, v0, min(32u, nvec - b * 32),
-                                 ctl->mask, row, row_busy);
-      }
+    for (uint32_t b = warp; b * 32 < nvec; b += kDecWarps) {
+      const uint32_t v0 = t * C::VC + b * 32, nv = min(32u, nvec - b * 32);
+      __syncwarp();
+      issue(v0, nv, nullptr, 0);
+      wait(0);
+      decode_block<D, BITS, G>(a, lay, cum, zbuf + b * 32 * C::CB, mbuf, v0, nv, ctl->mask, row,
+                               row_busy);
     }
+  }
 
-    // Raw code chunks: blocks of 32 vectors round-robin over the warps, each
-    // warp loading a block's code bytes with one bulk copy into one of its two
-    // buffers while it decodes the previous block from the other.
-    const uint32_t vs0 = ts0 * C::VC, vs1 = min(ts1 * C::VC, V);
-    const uint32_t nblk = (vs1 - vs0 + 31) / 32;
-    auto raw_block = [&](uint32_t b) {  // block b lies in a raw code chunk
-      const uint32_t t = (vs0 + b * 32) / C::VC;
-      const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
-      return uint32_t(ce & 0xFFFFu) == min(uint32_t(C::VC), V - t * C::VC) * C::CB;
-    };
-    auto next_raw = [&](uint32_t b) {
-      while (b < nblk && !raw_block(b)) b += kDecWarps;
-      return b;
-    };
-    auto issue = [&](uint32_t b, uint32_t k) {
-      if (lane == 0) {
-        const uint32_t v0 = vs0 + b * 32, t = v0 / C::VC, bytes = min(32u, vs1 - v0) * C::CB;
-        const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&ctl->cbar[warp][k], bytes);
-        bulk_g2s(cbuf + k * S::BLK, in + base + ((ce >> 16) << 4) + uint64_t(v0 - t * C::VC) * C::CB,
-                 bytes, &ctl->cbar[warp][k]);
-      }
-    };
-    uint32_t b = next_raw(warp), k = 0;
-    if (b < nblk) issue(b, 0);
+  // Phase 2: raw code chunks, blocks of 32 vectors round-robin over the
+  // warps; each warp loads a block's code and meta bytes with bulk copies
+  // into one of its two buffers while it decodes the previous block.
+  const uint32_t vs0 = t0 * C::VC, vs1 = min(t1 * C::VC, V);
+  const uint32_t nblk = (vs1 - vs0 + 31) / 32;
+  auto raw_block = [&](uint32_t b) {  // block b lies in a raw code chunk
+    const uint32_t t = (vs0 + b * 32) / C::VC;
+    const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
+    return uint32_t(ce & 0xFFFFu) == min(uint32_t(C::VC), V - t * C::VC) * C::CB;
+  };
+  auto next_raw = [&](uint32_t b) {
+    while (b < nblk && !raw_block(b)) b += kDecWarps;
+    return b;
+  };
+  auto issue_raw = [&](uint32_t b, uint32_t k) {
+    const uint32_t v0 = vs0 + b * 32, t = v0 / C::VC;
+    const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
+    issue(v0, min(32u, vs1 - v0),
+          in + base + ((ce >> 16) << 4) + uint64_t(v0 - t * C::VC) * C::CB, k);
+  };
+  uint32_t b = next_raw(warp), k = 0;
+  __syncwarp();
+  if (b < nblk) issue_raw(b, 0);
 #pragma unroll 1
-    while (b < nblk) {
-      const uint32_t nb = next_raw(b + kDecWarps);
-      __syncwarp();  // every lane is done with buffer k ^ 1 (the block before b)
-      if (nb < nblk) issue(nb, k ^ 1);
-      if (!mbar_wait(&ctl->cbar[warp][k], (cphase >> k) & 1, a.status))
-        set_status(a.status, KVC_ERR_TIMEOUT);
-      cphase ^= 1u << k;
-      const uint32_t v0 = vs0 + b * 32;
-      decode_block<D, BITS, G>(a, lay, cum, cbuf + k * S::BLK, mbuf + (v0 - s * C::VM) * C::MB, v0,
-                               min(32u, vs1 - v0), ctl->mask, row, row_busy);
-      b = nb;
-      k ^= 1;
-    }
+  while (b < nblk) {
+    const uint32_t nb = next_raw(b + kDecWarps);
+    __syncwarp();  // every lane is done with buffer k ^ 1 (the block before b)
+    if (nb < nblk) issue_raw(nb, k ^ 1);
+    wait(k);
+    const uint32_t v0 = vs0 + b * 32;
+    decode_block<D, BITS, G>(a, lay, cum, cbuf + k * S::BLK, mbuf + k * S::MBLK, v0,
+                             min(32u, vs1 - v0), ctl->mask, row, row_busy);
+    b = nb;
+    k ^= 1;
   }
   bulk_wait_all<0>();
 }
@@ -334,7 +371,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   DecCtl *ctl = reinterpret_cast<DecCtl *>(smem + S::ctl);
   uint32_t *s_cum = reinterpret_cast<uint32_t *>(smem + S::cum);
   const int tid = threadIdx.x;
-  constexpr uint32_t kLog2D = D == 64 ? 6 : D == 128 ? 7 : 8;
 
   if constexpr (kPaged) {
     for (uint32_t r = tid; r <= lay.n_req; r += blockDim.x) s_cum[r] = lay.cum[r];
@@ -345,39 +381,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     mbar_fence_init();
   }
   if (tid == 0) {
-    mbar_init(&ctl->mbar, 1);
     mbar_init(&ctl->zbar, 1);
     mbar_fence_init();
-    // D1: header (reading R12) against the receiver's description.
-    const uint8_t *h = a.in;
-    bool ok = a.in_bytes >= kHeader;
-    if (ok) {
-      const uint32_t bits = h[8], k = h[9], group = ld_u32(h + 12);
-      ok = ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 &&
-           (ld_u32(h + 4) >> 16) == kHeader && (bits == 2 || bits == 4) && k == kLog2D / 2 &&
-           (group == 32 || group == 64 || group == 128) && group <= D &&
-           ld_u32(h + 16) == a.layers && ld_u32(h + 20) == 2 && ld_u32(h + 24) == a.kv_heads &&
-           ld_u32(h + 28) == a.head_dim && ld_u64(h + 32) == a.tokens;
-      const uint32_t n_req = ld_u32(h + 48), n_chunks = ld_u32(h + 52);
-      const uint64_t stream_bytes = ld_u64(h + 56);
-      if (ok) {
-        const uint64_t cb = uint64_t(D) * bits / 8, mbv = uint64_t(D / group) * 4;
-        const uint64_t n_code = (uint64_t(a.V) * cb + kChunk - 1) / kChunk;
-        const uint64_t n_meta = (uint64_t(a.V) * mbv + kChunk - 1) / kChunk;
-        const uint64_t base = round16(kHeader + 8ull * n_chunks + 4ull * n_req);
-        ok = n_chunks == n_code + n_meta && base <= stream_bytes && stream_bytes <= a.in_bytes &&
-             (!a.paged_receiver || n_req == a.n_req);
-        ctl->bits = bits;
-        ctl->group = group;
-        ctl->n_req_stream = n_req;
-        ctl->n_chunks = n_chunks;
-        ctl->data_base = base;
-        ctl->stream_bytes = stream_bytes;
-        ctl->seed = ld_u64(h + 40);
-      }
-    }
-    ctl->hdr_ok = ok;
-    if (ok) sign_masks(ctl->seed, D, ctl->mask);
+    const StreamHdr h = parse_header<D>(a);
+    ctl->hdr_ok = h.ok;
+    ctl->bits = h.bits;
+    ctl->group = h.group;
+    ctl->n_req_stream = h.n_req;
+    ctl->n_chunks = h.n_chunks;
+    ctl->data_base = h.data_base;
+    ctl->stream_bytes = h.stream_bytes;
+    ctl->seed = h.seed;
+    if (h.ok) sign_masks(h.seed, D, ctl->mask);
   }
   __syncthreads();
   bool ok = ctl->hdr_ok;
@@ -426,6 +441,82 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     else
       decode_body<64, 2, 32>(a, lay, ctl, smem, s_cum);
   }
+}
+
+
+// Pre-pass of kvc_decompress: expands every meta chunk that used zero-byte
+// elimination (D3, D4) into the workspace, slot s at ws_meta + s * 16 KB, so
+// that the decode kernel reads each block's meta with one bulk copy and never
+// stops for a meta chunk. A raw meta chunk is left where it is. Every table
+// entry used here is bounds-checked on its own (the decode kernel checks the
+// whole table); a bad one only records KVC_ERR_CORRUPT.
+constexpr int kMetaThreads = 256;
+struct MetaCtl {
+  uint64_t full;
+  uint32_t red[kMetaThreads / 32];
+  uint32_t ok, bits, group, n_chunks;
+  uint64_t base, limit;
+};
+constexpr size_t meta_smem_bytes() { return 2 * size_t(kChunk) + sizeof(MetaCtl); }
+
+template <int D>
+__global__ void __launch_bounds__(kMetaThreads, 4)
+    meta_expand_kernel(const __grid_constant__ DecArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t *buf = smem, *scr = smem + kChunk;
+  MetaCtl *ctl = reinterpret_cast<MetaCtl *>(smem + 2 * kChunk);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    mbar_init(&ctl->full, 1);
+    mbar_fence_init();
+    const StreamHdr h = parse_header<D>(a);
+    ctl->ok = h.ok;
+    ctl->bits = h.bits;
+    ctl->group = h.group;
+    ctl->n_chunks = h.n_chunks;
+    ctl->base = h.data_base;
+    ctl->limit = min(a.in_bytes, h.stream_bytes);
+  }
+  __syncthreads();
+  if (!ctl->ok) return;  // the decode kernel reports the header
+  const uint32_t cb = D * ctl->bits / 8, mb = (D / ctl->group) * 4;
+  const uint32_t vc = kChunk / cb, vm = vc * (ctl->group * ctl->bits / 32);
+  const uint32_t n_code = (a.V + vc - 1) / vc, n_meta = (a.V + vm - 1) / vm;
+  if (n_meta > a.ws_meta_chunks) return;  // cannot happen for a consistent header
+  const uint8_t *table = a.in + kHeader;
+  uint32_t phase = 0;
+#pragma unroll 1
+  for (uint32_t s = blockIdx.x; s < n_meta; s += gridDim.x) {
+    const uint64_t e = ld_u64(table + 8 * (uint64_t(n_code) + s));
+    const uint64_t off = (e >> 16) << 4;
+    const uint32_t size = uint32_t(e & 0xFFFFu), len = min(vm, a.V - s * vm) * mb;
+    if (size == len) continue;
+    if (!(len == uint32_t(kChunk) && size >= kBitmap && size < len &&
+          ctl->base + off + round16(size) <= ctl->limit)) {
+      if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
+      continue;
+    }
+    if (tid == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&ctl->full, uint32_t(round16(size)));
+      bulk_g2s(buf, a.in + ctl->base + off, uint32_t(round16(size)), &ctl->full);
+    }
+    if (!mbar_wait(&ctl->full, phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+    phase ^= 1;
+    if (!ze_decode<kMetaThreads>(buf, scr, ctl->red, size)) {
+      if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
+      continue;
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, kMetaThreads);
+    if (tid == 0) {
+      bulk_s2g(a.ws_meta + uint64_t(s) * kChunk, buf, kChunk);
+      bulk_commit();
+      bulk_wait_read<0>();
+    }
+    named_bar_sync(1, kMetaThreads);  // buf free
+  }
+  if (tid == 0) bulk_wait_all<0>();
 }
 
 }  // namespace kvc

@@ -168,6 +168,8 @@ struct DecArgs {
   uint64_t tokens;
   uint32_t V;
   uint32_t paged_receiver;   // 1: request count and lengths must match
+  uint8_t *ws_meta;          // expanded meta chunks, 16 KB each
+  uint32_t ws_meta_chunks;   // slots in ws_meta
 };
 
 // Launchers, one translation unit per (head_dim, layout).

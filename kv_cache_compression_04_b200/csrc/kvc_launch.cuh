@@ -48,6 +48,16 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
   const uint64_t min_vc = uint64_t(kChunk) / (uint64_t(D) * 4 / 8);
   const uint64_t tiles = (uint64_t(a.V) + min_vc - 1) / min_vc;
   const int grid = tiles == 0 ? 1 : int(tiles < uint64_t(sms) ? tiles : uint64_t(sms));
+  // pre-pass: expand zero-byte-eliminated meta chunks into the workspace
+  auto mk = meta_expand_kernel<D>;
+  struct MetaTag {};
+  e = prepare<MetaTag>(mk, meta_smem_bytes());
+  if (e != cudaSuccess) return e;
+  const uint32_t mcap = 4u * uint32_t(sms);
+  const int mgrid = int(a.ws_meta_chunks == 0 ? 1u : (a.ws_meta_chunks < mcap ? a.ws_meta_chunks : mcap));
+  mk<<<mgrid, kMetaThreads, meta_smem_bytes(), st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   k<<<grid, kDecThreads, smem, st>>>(a, lay);
   return cudaGetLastError();
 }

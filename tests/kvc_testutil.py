@@ -36,7 +36,7 @@ def gpu_decompress(stream: np.ndarray | torch.Tensor, desc, nbytes: int | None =
     buf = stream if isinstance(stream, torch.Tensor) else torch.from_numpy(
         np.ascontiguousarray(stream)).cuda()
     n = buf.numel() if nbytes is None else nbytes
-    ws = torch.empty(kvc.KVC_DECOMPRESS_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(kvc.kvc_decompress_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
     st = kvc.kvc_decompress(buf.data_ptr(), n, desc, ws.data_ptr(), ws.numel(),
                             kvc._stream_ptr(None))
     assert st == kvc.KVC_OK, kvc.STATUS[st]
