@@ -452,22 +452,23 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // whole table); a bad one only records KVC_ERR_CORRUPT.
 constexpr int kMetaThreads = 256;
 struct MetaCtl {
-  uint64_t full;
+  uint64_t full[2];
   uint32_t red[kMetaThreads / 32];
   uint32_t ok, bits, group, n_chunks;
   uint64_t base, limit;
 };
-constexpr size_t meta_smem_bytes() { return 2 * size_t(kChunk) + sizeof(MetaCtl); }
+constexpr size_t meta_smem_bytes() { return 3 * size_t(kChunk) + sizeof(MetaCtl); }
 
 template <int D>
 __global__ void __launch_bounds__(kMetaThreads, 4)
     meta_expand_kernel(const __grid_constant__ DecArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t *buf = smem, *scr = smem + kChunk;
-  MetaCtl *ctl = reinterpret_cast<MetaCtl *>(smem + 2 * kChunk);
+  uint8_t *scr = smem + 2 * kChunk;  // buffers 0 and 1 below it
+  MetaCtl *ctl = reinterpret_cast<MetaCtl *>(smem + 3 * kChunk);
   const int tid = threadIdx.x;
   if (tid == 0) {
-    mbar_init(&ctl->full, 1);
+    mbar_init(&ctl->full[0], 1);
+    mbar_init(&ctl->full[1], 1);
     mbar_fence_init();
     const StreamHdr h = parse_header<D>(a);
     ctl->ok = h.ok;
@@ -484,37 +485,62 @@ __global__ void __launch_bounds__(kMetaThreads, 4)
   const uint32_t n_code = (a.V + vc - 1) / vc, n_meta = (a.V + vm - 1) / vm;
   if (n_meta > a.ws_meta_chunks) return;  // cannot happen for a consistent header
   const uint8_t *table = a.in + kHeader;
-  uint32_t phase = 0;
-#pragma unroll 1
-  for (uint32_t s = blockIdx.x; s < n_meta; s += gridDim.x) {
-    const uint64_t e = ld_u64(table + 8 * (uint64_t(n_code) + s));
-    const uint64_t off = (e >> 16) << 4;
+  const uint64_t base = ctl->base, limit = ctl->limit;
+
+  // this CTA's chunks s = blockIdx.x + i * gridDim.x that used elimination
+  auto entry = [&](uint32_t s) { return ld_u64(table + 8 * (uint64_t(n_code) + s)); };
+  auto eliminated = [&](uint32_t s) {
+    return uint32_t(entry(s) & 0xFFFFu) != min(vm, a.V - s * vm) * mb;
+  };
+  auto next = [&](uint32_t s) {
+    while (s < n_meta && !eliminated(s)) s += gridDim.x;
+    return s;
+  };
+  // starts loading chunk s into buffer k; false (and CORRUPT) for a bad entry
+  auto load = [&](uint32_t s, uint32_t k) {
+    const uint64_t e = entry(s), off = (e >> 16) << 4;
     const uint32_t size = uint32_t(e & 0xFFFFu), len = min(vm, a.V - s * vm) * mb;
-    if (size == len) continue;
-    if (!(len == uint32_t(kChunk) && size >= kBitmap && size < len &&
-          ctl->base + off + round16(size) <= ctl->limit)) {
-      if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
-      continue;
-    }
+    const bool ok = len == uint32_t(kChunk) && size >= kBitmap && size < len &&
+                    base + off + round16(size) <= limit;
     if (tid == 0) {
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&ctl->full, uint32_t(round16(size)));
-      bulk_g2s(buf, a.in + ctl->base + off, uint32_t(round16(size)), &ctl->full);
+      if (ok) {
+        mbar_arrive_expect_tx(&ctl->full[k], uint32_t(round16(size)));
+        bulk_g2s(smem + k * kChunk, a.in + base + off, uint32_t(round16(size)), &ctl->full[k]);
+      } else {
+        set_status(a.status, KVC_ERR_CORRUPT);
+        mbar_arrive(&ctl->full[k]);  // completes the phase without data
+      }
     }
-    if (!mbar_wait(&ctl->full, phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
-    phase ^= 1;
-    if (!ze_decode<kMetaThreads>(buf, scr, ctl->red, size)) {
-      if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
-      continue;
+    return ok;
+  };
+  uint32_t s = next(blockIdx.x), k = 0, phase = 0;
+  bool ok = s < n_meta && load(s, 0);
+#pragma unroll 1
+  while (s < n_meta) {
+    const uint32_t ns = next(s + gridDim.x);
+    bool nok = false;
+    if (ns < n_meta) {
+      if (tid == 0) bulk_wait_read<0>();  // the store from buffer k ^ 1 has read it
+      nok = load(ns, k ^ 1);
     }
-    fence_proxy_async_smem();
-    named_bar_sync(1, kMetaThreads);
-    if (tid == 0) {
-      bulk_s2g(a.ws_meta + uint64_t(s) * kChunk, buf, kChunk);
-      bulk_commit();
-      bulk_wait_read<0>();
+    if (!mbar_wait(&ctl->full[k], (phase >> k) & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+    phase ^= 1u << k;
+    uint8_t *buf = smem + k * kChunk;
+    if (ok) {
+      if (ze_decode<kMetaThreads>(buf, scr, ctl->red, uint32_t(entry(s) & 0xFFFFu))) {
+        fence_proxy_async_smem();
+        named_bar_sync(1, kMetaThreads);
+        if (tid == 0) {
+          bulk_s2g(a.ws_meta + uint64_t(s) * kChunk, buf, kChunk);
+          bulk_commit();
+        }
+      } else if (tid == 0) {
+        set_status(a.status, KVC_ERR_CORRUPT);
+      }
     }
-    named_bar_sync(1, kMetaThreads);  // buf free
+    s = ns;
+    ok = nok;
+    k ^= 1;
   }
   if (tid == 0) bulk_wait_all<0>();
 }

@@ -313,13 +313,14 @@ __device__ __forceinline__ void words_from_planes(const uint32_t *pw, uint8_t *b
     dst[(q + m) & 7] = make_uint4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
 }
 
-// Nonzero-byte mask of a word: bit b set iff byte b is nonzero.
-__device__ __forceinline__ uint32_t nz_nibble(uint32_t x) {
-  uint32_t t = x | (x >> 4);
-  t |= t >> 2;
-  t |= t >> 1;
-  t &= 0x01010101u;
-  return (t | (t >> 7) | (t >> 14) | (t >> 21)) & 0xFu;
+// Nonzero-byte mask of a word: bit b set iff byte b is nonzero. The top bit
+// of each byte of ((x & 0x7F..) + 0x7F..) | x is set iff the byte is
+// nonzero (the add cannot carry out of a byte); one multiply then gathers
+// bits 7, 15, 23, 31 into bits 28..31 (the other partial products land on
+// distinct bits below 28 or above 31, so nothing carries into 28..31).
+KVC_HD uint32_t nz_nibble(uint32_t x) {
+  const uint32_t m = (((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x) & 0x80808080u;
+  return (m * 0x00204081u) >> 28;
 }
 
 // Inclusive prefix sum over the warp.
@@ -333,86 +334,108 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
   return x;
 }
 
+// Byte-permute selectors, indexed by a 4-bit nonzero-byte mask n:
+// expand: byte b takes source byte #(set bits of n below b) if bit b is set,
+//         zero otherwise;
+// compact: byte i takes the position of the i-th set bit of n, zero beyond.
+__device__ __forceinline__ uint32_t expand_selector(uint32_t n) {
+  uint32_t sel = 0, j = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const bool on = (n >> b) & 1u;
+    sel |= (on ? j : 4u) << (4 * b);
+    j += on;
+  }
+  return sel;
+}
+__device__ __forceinline__ uint32_t compact_selector(uint32_t n) {
+  uint32_t sel = 0x4444u, j = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    if ((n >> b) & 1u) {
+      sel = (sel & ~(0xFu << (4 * j))) | (uint32_t(b) << (4 * j));
+      ++j;
+    }
+  }
+  return sel;
+}
+
 // buf holds a full 16 KB chunk; on return it holds bitmap + nonzero bytes
 // (the caller knows their count from chunk_nnz_part). scr: 16 KB scratch.
-// Run by the first NT threads (NT >= 128, a multiple of 32 dividing 4096).
-// Each warp compacts a contiguous eighth (for NT = 256) of the plane words:
-// one pass counts its nonzero bytes, a block scan of the warp totals gives
-// each warp's output base, a second pass places bytes and bitmap words.
+// Run by the first 256 threads. Thread t owns plane words 16t .. 16t+15
+// (bitmap words 2t, 2t+1): it compacts the nonzero bytes of each with one
+// byte permute and writes them after the bytes of threads < t (block scan).
 template <int NT>
 __device__ __forceinline__ void ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *red) {
-  constexpr int NW = NT / 32, PER_WARP = 4096 / NW, ROUNDS = PER_WARP / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  static_assert(NT == 256, "16 plane words per thread");
+  __shared__ uint32_t lut[16];
+  const int tid = threadIdx.x;
   uint32_t *pw = reinterpret_cast<uint32_t *>(scr);
+  if (tid < 16) lut[tid] = compact_selector(tid);
   for (int m = tid; m < 128; m += NT) planes_from_words(buf, pw, m);
   named_bar_sync(1, NT);
-  const int w0 = warp * PER_WARP;
-  uint32_t cnt = 0;
-#pragma unroll 4
-  for (int r = 0; r < ROUNDS; ++r) cnt += __popc(nz_nibble(pw[w0 + 32 * r + lane]));
-  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-  if (lane == 0) red[warp] = cnt;
-  named_bar_sync(1, NT);
-  uint32_t run = 0;
+  uint32_t x[16], n[16], cnt = 0, bw0 = 0, bw1 = 0;
+  const uint4 *src = reinterpret_cast<const uint4 *>(pw + 16 * tid);
 #pragma unroll
-  for (int w = 0; w < NW; ++w) run += w < warp ? red[w] : 0u;
-  named_bar_sync(1, NT);  // red may be reused by the caller
-  uint32_t *bm = reinterpret_cast<uint32_t *>(buf);
-#pragma unroll 2
-  for (int r = 0; r < ROUNDS; ++r) {
-    const int i = w0 + 32 * r + lane;
-    const uint32_t x = pw[i], n = nz_nibble(x), c = __popc(n);
-    const uint32_t incl = warp_incl_scan(c);
-    uint32_t off = kBitmap + run + incl - c;
+  for (int q = 0; q < 4; ++q) {
+    const uint4 v = src[q];
+    x[4 * q] = v.x, x[4 * q + 1] = v.y, x[4 * q + 2] = v.z, x[4 * q + 3] = v.w;
+  }
 #pragma unroll
-    for (int b = 0; b < 4; ++b)
-      if ((n >> b) & 1u) buf[off++] = uint8_t(x >> (8 * b));
-    uint32_t word = n << (4 * (lane & 7));
-    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
-    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
-    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-    if ((lane & 7) == 0) bm[i >> 3] = word;
-    run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+  for (int k = 0; k < 16; ++k) {
+    n[k] = nz_nibble(x[k]);
+    cnt += __popc(n[k]);
+    if (k < 8)
+      bw0 |= n[k] << (4 * k);
+    else
+      bw1 |= n[k] << (4 * (k - 8));
+  }
+  uint32_t total;
+  uint32_t q = kBitmap + block_excl_scan<NT>(cnt, red, total);  // buf is free after this
+  reinterpret_cast<uint2 *>(buf)[tid] = make_uint2(bw0, bw1);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t c = __byte_perm(x[k], 0, lut[n[k]]), nb = __popc(n[k]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (uint32_t(i) < nb) buf[q + i] = uint8_t(c >> (8 * i));
+    q += nb;
   }
   named_bar_sync(1, NT);
 }
 
 // Inverse: buf holds bitmap + nonzero bytes (`size` bytes); on return it
 // holds the 16 KB chunk. Returns false (for every thread) if the bitmap's
-// popcount disagrees with the size; then buf is unspecified.
+// popcount disagrees with the size; then buf is unspecified. Thread t
+// rebuilds plane words 16t .. 16t+15: each takes the next popcount(n) source
+// bytes (an unaligned 4-byte window) and spreads them with one byte permute.
 template <int NT>
 __device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *red, uint32_t size) {
-  constexpr int NW = NT / 32, PER_WARP = 4096 / NW, ROUNDS = PER_WARP / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  static_assert(NT == 256, "16 plane words per thread");
+  __shared__ uint32_t lut[16];
+  const int tid = threadIdx.x;
   uint32_t *pw = reinterpret_cast<uint32_t *>(scr);
-  const uint32_t *bm = reinterpret_cast<const uint32_t *>(buf);
-  const int w0 = warp * PER_WARP;
-  uint32_t cnt = 0;
-  for (int j = lane; j < PER_WARP / 8; j += 32) cnt += __popc(bm[w0 / 8 + j]);
-  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-  if (lane == 0) red[warp] = cnt;
-  named_bar_sync(1, NT);
-  uint32_t run = 0, total = 0;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) {
-    const uint32_t r = red[w];
-    run += w < warp ? r : 0u;
-    total += r;
-  }
-  named_bar_sync(1, NT);  // red may be reused by the caller
+  if (tid < 16) lut[tid] = expand_selector(tid);
+  const uint2 bw = reinterpret_cast<const uint2 *>(buf)[tid];
+  uint32_t total;
+  uint32_t p = kBitmap +
+               block_excl_scan<NT>(__popc(bw.x) + __popc(bw.y), red, total);  // lut visible after
   if (total != size - kBitmap) return false;
-#pragma unroll 2
-  for (int r = 0; r < ROUNDS; ++r) {
-    const int i = w0 + 32 * r + lane;
-    const uint32_t n = (bm[i >> 3] >> (4 * (i & 7))) & 0xFu, c = __popc(n);
-    const uint32_t incl = warp_incl_scan(c);
-    uint32_t off = kBitmap + run + incl - c, x = 0;
+  // the window's words are clamped to the buffer: a byte it needs lies below
+  // `size` <= 16384, so a clamped word is never one whose bytes are used
+  const uint32_t *b32 = reinterpret_cast<const uint32_t *>(buf);
+  uint32_t o[16];
 #pragma unroll
-    for (int b = 0; b < 4; ++b)
-      if ((n >> b) & 1u) x |= uint32_t(buf[off++]) << (8 * b);
-    pw[i] = x;
-    run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t n = ((k < 8 ? bw.x : bw.y) >> (4 * (k & 7))) & 0xFu;
+    const uint32_t a = min(p >> 2, 4095u), a1 = min((p >> 2) + 1, 4095u);
+    const uint32_t win = __funnelshift_r(b32[a], b32[a1], 8 * (p & 3));
+    o[k] = __byte_perm(win, 0, lut[n]);
+    p += __popc(n);
   }
+  uint4 *dst = reinterpret_cast<uint4 *>(pw + 16 * tid);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
   named_bar_sync(1, NT);
   for (int m = tid; m < 128; m += NT) words_from_planes(pw, buf, m);
   named_bar_sync(1, NT);

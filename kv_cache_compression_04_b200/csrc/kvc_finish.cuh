@@ -25,14 +25,14 @@ namespace kvc {
 constexpr int kFinThreads = 256;
 
 struct FinCtl {
-  uint64_t full;
+  uint64_t full[2];
   uint32_t red[kFinThreads / 32];
   uint32_t flag;
   uint32_t tick;
 };
 
 constexpr size_t fin_smem_bytes(bool paged) {
-  return 2 * size_t(kChunk) + sizeof(FinCtl) +
+  return 3 * size_t(kChunk) + sizeof(FinCtl) +
          (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
 }
 
@@ -106,14 +106,14 @@ __global__ void __launch_bounds__(kFinThreads, 4)
     finish_kernel(const __grid_constant__ FinArgs a, const __grid_constant__ Layout lay) {
   constexpr int NT = kFinThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t *buf = smem;
-  uint8_t *scr = smem + kChunk;
-  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + 2 * kChunk);
+  uint8_t *scr = smem + 2 * kChunk;  // buffers 0 and 1 below it
+  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + 3 * kChunk);
   uint32_t *s_cum = reinterpret_cast<uint32_t *>(ctl + 1);
   const int tid = threadIdx.x;
   const uint32_t nb = gridDim.x, b = blockIdx.x;
   if (tid == 0) {
-    mbar_init(&ctl->full, 1);
+    mbar_init(&ctl->full[0], 1);
+    mbar_init(&ctl->full[1], 1);
     mbar_fence_init();
     ctl->flag = *reinterpret_cast<volatile uint32_t *>(a.flags);
   }
@@ -145,15 +145,27 @@ __global__ void __launch_bounds__(kFinThreads, 4)
     for (uint32_t s = tid; s < s0; s += NT) part += round16(meta_stored_size(a, s));
     prefix = block_sum64<NT>(part, ctl->red);
   }
-  uint32_t phase = 0;
-#pragma unroll 1
-  for (uint32_t s = s0; s < s1; ++s, ++phase) {
-    const uint32_t len = meta_len(a, s), size = meta_stored_size(a, s);
+  // Two buffers: the raw meta of chunk s + 1 loads while chunk s is encoded;
+  // a buffer is refilled only after its store has read it.
+  auto load = [&](uint32_t s, uint32_t k) {
     if (tid == 0) {
-      mbar_arrive_expect_tx(&ctl->full, uint32_t(round16(len)));
-      bulk_g2s(buf, a.ws_meta + uint64_t(s) * kChunk, uint32_t(round16(len)), &ctl->full);
+      const uint32_t bytes = uint32_t(round16(meta_len(a, s)));
+      mbar_arrive_expect_tx(&ctl->full[k], bytes);
+      bulk_g2s(smem + k * kChunk, a.ws_meta + uint64_t(s) * kChunk, bytes, &ctl->full[k]);
     }
-    if (!mbar_wait(&ctl->full, phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+  };
+  if (s0 < s1) load(s0, 0);
+  uint32_t phase = 0;  // bit k: phase of buffer k
+#pragma unroll 1
+  for (uint32_t s = s0, k = 0; s < s1; ++s, k ^= 1) {
+    uint8_t *buf = smem + k * kChunk;
+    if (s + 1 < s1) {
+      if (tid == 0) bulk_wait_read<0>();  // the store of chunk s - 1 has read buffer k ^ 1
+      load(s + 1, k ^ 1);
+    }
+    if (!mbar_wait(&ctl->full[k], (phase >> k) & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+    phase ^= 1u << k;
+    const uint32_t len = meta_len(a, s), size = meta_stored_size(a, s);
     if (size < len) ze_encode<NT>(buf, scr, ctl->red);
     for (uint32_t i = size + tid; i < round16(size); i += NT) buf[i] = 0;
     fence_proxy_async_smem();
@@ -172,10 +184,8 @@ __global__ void __launch_bounds__(kFinThreads, 4)
         set_status(a.status, KVC_ERR_CAPACITY);
       }
       a.meta_size[s] = size;
-      bulk_wait_read<0>();
     }
     prefix += round16(size);
-    named_bar_sync(1, NT);  // buf free
   }
 
   // -------------------------------------------------- code-table entries --
@@ -223,10 +233,10 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *buf = smem;
   uint8_t *scr = smem + kChunk;
-  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + 2 * kChunk);
+  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + 3 * kChunk);
   const int tid = threadIdx.x;
   if (tid == 0) {
-    mbar_init(&ctl->full, 1);
+    mbar_init(&ctl->full[0], 1);
     mbar_fence_init();
     ctl->flag = *reinterpret_cast<volatile uint32_t *>(a.flags);
   }
@@ -248,10 +258,10 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
       // so every chunk loads at once; only its store waits, for the chunks
       // whose raw bytes [dst, dst + padded size) overlaps to have been read.
       if (tid == 0) {
-        mbar_arrive_expect_tx(&ctl->full, len);
-        bulk_g2s(buf, a.out + a.data_base + src, len, &ctl->full);
+        mbar_arrive_expect_tx(&ctl->full[0], len);
+        bulk_g2s(buf, a.out + a.data_base + src, len, &ctl->full[0]);
       }
-      if (!mbar_wait(&ctl->full, phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+      if (!mbar_wait(&ctl->full[0], phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
       ++phase;
       if (tid == 0) {
         __threadfence();
@@ -307,9 +317,9 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
     if (tid == 0) {
       const uint32_t size = a.meta_size[s];
       const uint64_t e = *reinterpret_cast<const uint64_t *>(a.out + kHeader + 8ull * (a.n_code + s));
-      mbar_arrive_expect_tx(&ctl->full, uint32_t(round16(size)));
-      bulk_g2s(buf, a.ws_meta + uint64_t(s) * kChunk, uint32_t(round16(size)), &ctl->full);
-      if (!mbar_wait(&ctl->full, phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+      mbar_arrive_expect_tx(&ctl->full[0], uint32_t(round16(size)));
+      bulk_g2s(buf, a.ws_meta + uint64_t(s) * kChunk, uint32_t(round16(size)), &ctl->full[0]);
+      if (!mbar_wait(&ctl->full[0], phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
       bulk_s2g(a.out + a.data_base + ((e >> 16) << 4), buf, uint32_t(round16(size)));
       bulk_commit();
       bulk_wait_read<0>();

@@ -11,4 +11,16 @@ void hl_transpose32(const uint32_t *in, uint32_t *out) {
   for (int i = 0; i < 32; ++i) out[i] = a[i];
 }
 void hl_sign_masks(uint64_t seed, int d, uint32_t *out) { kvc::sign_masks(seed, d, out); }
+// Mismatches of the library's nonzero-byte mask against a byte-by-byte
+// reference over words [start, start + count).
+uint64_t hl_nz_nibble_mismatches(uint64_t start, uint64_t count) {
+  uint64_t bad = 0;
+  for (uint64_t i = 0; i < count; ++i) {
+    const uint32_t x = uint32_t(start + i);
+    uint32_t ref = 0;
+    for (int b = 0; b < 4; ++b) ref |= (((x >> (8 * b)) & 0xFFu) != 0 ? 1u : 0u) << b;
+    bad += kvc::nz_nibble(x) != ref;
+  }
+  return bad;
+}
 }

@@ -164,6 +164,8 @@ def host_logic():
     lib.hl_fdiv.restype = C.c_uint32
     lib.hl_fdiv.argtypes = [C.c_uint32, C.c_uint32]
     lib.hl_transpose32.argtypes = [C.c_void_p, C.c_void_p]
+    lib.hl_nz_nibble_mismatches.restype = C.c_uint64
+    lib.hl_nz_nibble_mismatches.argtypes = [C.c_uint64, C.c_uint64]
     lib.hl_sign_masks.argtypes = [C.c_uint64, C.c_int, C.c_void_p]
     return lib
 
@@ -198,3 +200,16 @@ def test_sign_masks_match_oracle_sign_words(host_logic, seed, d):
         lo = (w[(2 * j) // 64] >> ((2 * j) % 64)) & 1
         hi = (w[(2 * j + 1) // 64] >> ((2 * j + 1) % 64)) & 1
         assert m[j] == (lo << 15) | (hi << 31)
+
+
+def test_nonzero_byte_mask(host_logic):
+    """The lossless stage's nonzero-byte mask (add-and-gather identity)
+    against a byte-by-byte reference: every word in several 2^24 ranges that
+    cover all byte patterns' boundaries, and all 2^32 words under -m slow."""
+    for start in (0, 0x007F0000, 0x7F7F0000, 0x80800000, 0xFF000000, 0xFFFF0000 - (1 << 24)):
+        assert host_logic.hl_nz_nibble_mismatches(start, 1 << 24) == 0, hex(start)
+
+
+@pytest.mark.slow
+def test_nonzero_byte_mask_exhaustive(host_logic):
+    assert host_logic.hl_nz_nibble_mismatches(0, 1 << 32) == 0
