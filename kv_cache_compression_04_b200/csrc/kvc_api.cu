@@ -115,6 +115,44 @@ DenseLayout dense_layout(const kvc_kv_desc *kv, const Shape &s) {
   return L;
 }
 
+// Tensor map of a dense input for the encoder's per-warp tensor loads:
+// 5-D [layers][2][kv_heads][tokens][head_dim], boxes of 32 tokens x 64
+// channels with 128-byte swizzle. Only when every 32-vector block lies in one
+// head row (tokens % 32 == 0); the encoder copies rows one by one otherwise.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return EncodeTiledFn(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+void add_tensor_map(const kvc_kv_desc *kv, const Shape &s, DenseLayout &L) {
+  L.tma = 0;
+  if (s.V == 0 || s.T % 32 != 0) return;
+  const EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return;
+  const cuuint64_t dims[5] = {cuuint64_t(s.D), cuuint64_t(s.T), cuuint64_t(kv->kv_heads), 2,
+                              cuuint64_t(kv->layers)};
+  const cuuint64_t strides[4] = {cuuint64_t(L.s_t), cuuint64_t(L.s_h), cuuint64_t(L.s_kv),
+                                 cuuint64_t(L.s_l)};
+  const cuuint32_t box[5] = {64, 32, 1, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  if (fn(&L.tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, kv->data, dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+    L.tma = 1;
+}
+
 void paged_layout(const kvc_kv_desc *kv, const Shape &s, PagedLayout &L) {
   L.base = static_cast<uint8_t *>(kv->data);
   L.s_l = kv->stride_layer * 2;
@@ -219,7 +257,8 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *o
   if (cudaMemsetAsync(ws, 0, w.zero_bytes, cs) != cudaSuccess) return KVC_ERR_CUDA;
   cudaError_t e = cudaSuccess;
   if (kv->kind == KVC_DENSE) {
-    const DenseLayout L = dense_layout(kv, s);
+    DenseLayout L = dense_layout(kv, s);
+    add_tensor_map(kv, s, L);
     if (s.n_code)
       e = s.D == 128 ? launch_encode_dense_d128(s.bits, s.G, a, L, sms, cs)
                      : launch_encode_dense_d64(s.bits, s.G, a, L, sms, cs);

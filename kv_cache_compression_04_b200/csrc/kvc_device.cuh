@@ -81,6 +81,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
 }
 
 // ---------------------------------------------------- bulk-async copies --
+// Tensor-map load of a 5-D box into shared memory, completion counted in
+// bytes on `bar` (no multicast). c0 is the innermost coordinate.
+__device__ __forceinline__ void tma_load_5d(void *sdst, const CUtensorMap *map, int c0, int c1,
+                                            int c2, int c3, int c4, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(sdst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
 // global -> shared, completion counted in bytes on `bar`.
 __device__ __forceinline__ void bulk_g2s(void *sdst, const void *gsrc, uint32_t bytes,
                                          uint64_t *bar) {

@@ -52,10 +52,23 @@ struct Cfg {
   static_assert(SLICE % 32 == 0, "meta slices hold whole 8-word groups");
 };
 
+// Shared memory: [per-thread padded rows | per-warp tensor-load buffers (a
+// union: one load path runs)] | per-thread mbarriers | per-warp mbarriers |
+// request prefix (paged).
+template <int D>
+struct EncSmem {
+  static constexpr size_t ROWP = 2 * D + 16;
+  static constexpr size_t WBUF = size_t(D / 64) * 32 * 128;  // 32 rows, 128-byte swizzled halves
+  static constexpr size_t A = kEncThreads * ROWP > kEncWarps * WBUF ? kEncThreads * ROWP
+                                                                    : kEncWarps * WBUF;
+  static constexpr size_t bars = (A + 1023) & ~size_t(1023);
+  static constexpr size_t wbars = bars + kEncThreads * 8;
+  static constexpr size_t cum = wbars + kEncWarps * 8;
+  static_assert(WBUF % 1024 == 0, "swizzled buffers stay 1024-byte aligned");
+};
 template <int D>
 constexpr size_t enc_smem_bytes(bool paged) {
-  return size_t(kEncThreads) * (2 * D + 16) + size_t(kEncThreads) * 8 +
-         (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
+  return EncSmem<D>::cum + (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
 }
 
 template <class L>
@@ -106,6 +119,31 @@ struct Enc : Cfg<D, BITS, G> {
 #pragma unroll
     for (int q = 0; q < D / 16; ++q) {
       const uint4 va = r4[q], vb = r4[q + D / 16];  // words 4q.., 4q + d/4..
+      const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = 4 * q + e;
+        const uint32_t x0 = wa[e] ^ mask[k], x1 = wb[e] ^ mask[k + D / 4];
+        y.p[2 * k] = make_float2(__uint_as_float(x0 << 16), __uint_as_float(x1 << 16));
+        y.p[2 * k + 1] =
+            make_float2(__uint_as_float(x0 & 0xFFFF0000u), __uint_as_float(x1 & 0xFFFF0000u));
+      }
+    }
+  }
+
+  // E1/E2 from a per-warp tensor-load buffer: lane r's row r of each 64-channel
+  // half, 16-byte chunk c stored at r * 128 + ((c ^ (r % 8)) * 16) (the
+  // tensor map's 128-byte swizzle, which keeps these reads conflict-free).
+  static __device__ __forceinline__ void unpack_swz(const uint8_t *wbuf, int lane,
+                                                    const uint32_t *__restrict__ mask, Pairs<D> &y) {
+    const int sw = lane & 7;
+    auto chunk = [&](int q) {
+      return *reinterpret_cast<const uint4 *>(wbuf + (q >> 3) * 4096 + lane * 128 +
+                                              (((q & 7) ^ sw) << 4));
+    };
+#pragma unroll
+    for (int q = 0; q < D / 16; ++q) {
+      const uint4 va = chunk(q), vb = chunk(q + D / 16);  // words 4q.., 4q + d/4..
       const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -201,14 +239,19 @@ __global__ void __launch_bounds__(kEncThreads, 1)
   using C = Cfg<D, BITS, G>;
   using E = Enc<D, BITS, G>;
   constexpr bool kPaged = kIsPaged<Layout>;
+  using S = EncSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint8_t *row = smem + tid * C::ROWP;
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kEncThreads * C::ROWP) + tid;
-  uint32_t *s_cum = reinterpret_cast<uint32_t *>(smem + kEncThreads * (C::ROWP + 8));
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S::bars) + tid;
+  uint8_t *wbuf = smem + warp * S::WBUF;
+  uint64_t *wbar = reinterpret_cast<uint64_t *>(smem + S::wbars) + warp;
+  uint32_t *s_cum = reinterpret_cast<uint32_t *>(smem + S::cum);
 
   mbar_init(bar, 1);
+  if (lane == 0) mbar_init(wbar, 1);
   mbar_fence_init();
+  __syncwarp();  // the warp's barrier is initialized before any lane waits on it
   if constexpr (kPaged) {
     for (uint32_t r = tid; r <= lay.n_req; r += blockDim.x) s_cum[r] = lay.cum[r];
     __syncthreads();
@@ -234,22 +277,10 @@ __global__ void __launch_bounds__(kEncThreads, 1)
     return true;
   };
 
-  bool pending = blk < n_blocks && issue(blk * 32 + lane);
   uint32_t phase = 0, err = 0;
-#pragma unroll 1
-  for (; blk < n_blocks; blk += stride) {
-    const uint32_t v = blk * 32 + lane;
-    const bool valid = v < V;
-    Pairs<D> y;
-    if (pending) {
-      if (!mbar_wait(bar, phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
-      phase ^= 1;
-    }
-    if (valid) E::unpack(row, a.sign_mask, y);
-    // the row has been read into registers; the next copy may overwrite it
-    fence_proxy_async_smem();
-    pending = blk + stride < n_blocks && issue((blk + stride) * 32 + lane);
-
+  // E3..E7 of this lane's vector v of block blk, its stores, and the block's
+  // shuffled-byte nonzero counts.
+  auto finish_block = [&](uint32_t blk, uint32_t v, bool valid, Pairs<D> &y) {
     uint32_t code[C::CW], meta[C::NG];
     if (valid) {
       err |= E::vector(y, code, meta);
@@ -307,6 +338,57 @@ __global__ void __launch_bounds__(kEncThreads, 1)
           kBitmap + uint32_t(old) + cs < uint32_t(kChunk))
         atomicOr(a.flags, 1u);
       atomicAdd(a.meta_nnz + blk * 32 / C::VM, ms);
+    }
+  };
+
+  bool use_tma = false;
+  if constexpr (!kPaged) use_tma = lay.tma != 0;
+  if constexpr (!kPaged) {
+    if (use_tma) {
+      // Per-warp tensor loads: every block is 32 vectors of one head row
+      // (tokens % 32 == 0, so V % 32 == 0 and no block is partial).
+      auto issue_tma = [&](uint32_t b) {
+        if (lane == 0) {
+          const uint32_t v0 = b * 32, lkh = fdiv(lay.T, v0), t0 = v0 - lkh * lay.T.d;
+          const uint32_t lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
+          mbar_arrive_expect_tx(wbar, uint32_t(S::WBUF));
+#pragma unroll
+          for (int hh = 0; hh < D / 64; ++hh)
+            tma_load_5d(wbuf + hh * 4096, &lay.tmap, hh * 64, int(t0), int(h), int(lk & 1u),
+                        int(lk >> 1), wbar);
+        }
+      };
+      if (blk < n_blocks) issue_tma(blk);
+#pragma unroll 1
+      for (; blk < n_blocks; blk += stride) {
+        if (!mbar_wait(wbar, phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+        phase ^= 1;
+        Pairs<D> y;
+        E::unpack_swz(wbuf, lane, a.sign_mask, y);
+        // every lane has read the buffer; the next load may overwrite it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (blk + stride < n_blocks) issue_tma(blk + stride);
+        finish_block(blk, blk * 32 + lane, true, y);
+      }
+    }
+  }
+  if (!use_tma) {
+    bool pending = blk < n_blocks && issue(blk * 32 + lane);
+#pragma unroll 1
+    for (; blk < n_blocks; blk += stride) {
+      const uint32_t v = blk * 32 + lane;
+      const bool valid = v < V;
+      Pairs<D> y;
+      if (pending) {
+        if (!mbar_wait(bar, phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+        phase ^= 1;
+      }
+      if (valid) E::unpack(row, a.sign_mask, y);
+      // the row has been read into registers; the next copy may overwrite it
+      fence_proxy_async_smem();
+      pending = blk + stride < n_blocks && issue((blk + stride) * 32 + lane);
+      finish_block(blk, v, valid, y);
     }
   }
   err = __reduce_or_sync(0xFFFFFFFFu, err);

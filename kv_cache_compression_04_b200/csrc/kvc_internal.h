@@ -7,6 +7,7 @@
 // (episode notes); exact rules are this library's readings.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -105,10 +106,16 @@ KVC_HD uint32_t fdiv(const FastDiv &f, uint32_t n) {
 // Vector addressing. Vector v (logical order [layer][kv][head][request]
 // [token]) -> byte address of its head_dim contiguous bf16 values.
 struct DenseLayout {
+  // Tensor map of the input as 5-D [layers][2][kv_heads][tokens][head_dim]
+  // (boxes of 32 tokens x 64 channels, 128-byte swizzle), valid iff tma != 0:
+  // set by the host when tokens % 32 == 0, so a 32-vector block lies in one
+  // head row.
+  alignas(64) CUtensorMap tmap;
   uint8_t *base;
   int64_t s_l, s_kv, s_h, s_t;  // bytes
   FastDiv T, H;                 // tokens, kv_heads
   uint32_t tokens;
+  uint32_t tma;
 };
 
 struct PagedLayout {
