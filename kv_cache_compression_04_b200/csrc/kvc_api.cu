@@ -301,7 +301,8 @@ kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *ou
     return KVC_ERR_CUDA;
   cudaError_t e;
   if (out->kind == KVC_DENSE) {
-    const DenseLayout L = dense_layout(out, s);
+    DenseLayout L = dense_layout(out, s);
+    add_tensor_map(out, s, L);
     e = s.D == 128 ? launch_decode_dense_d128(a, L, sms, cs) : launch_decode_dense_d64(a, L, sms, cs);
   } else {
     static thread_local PagedLayout L;

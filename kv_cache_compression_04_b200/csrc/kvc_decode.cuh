@@ -43,8 +43,9 @@ struct DecSmem {
   static constexpr size_t ROWP = 2 * D + 16;
   static constexpr size_t BLK = 32 * size_t(D) / 2;       // widest code block (4-bit)
   static constexpr size_t MBLK = 32 * (size_t(D) / 32) * 4;  // widest meta block (group 32)
-  static constexpr size_t rows = 0;
+  static constexpr size_t rows = 0;  // also the per-warp tensor-store staging buffers
   static constexpr size_t code = rows + kDecThreads * ROWP;
+  static_assert(kDecThreads * ROWP >= kDecWarps * (size_t(D / 64) * 4096), "staging fits");
   static constexpr size_t meta = code + 2 * kDecWarps * BLK;
   static constexpr size_t zchunk = meta + 2 * kDecWarps * MBLK;
   static constexpr size_t scr = zchunk + kChunk;
@@ -206,6 +207,38 @@ __device__ __forceinline__ void decode_block(const DecArgs &a, const Layout &lay
   row_busy = true;
 }
 
+// Dense receiver with a tensor map (tokens % 32 == 0, so the block is 32
+// vectors of one head row): the lanes write their rows into the warp's
+// staging buffer in the map's 128-byte swizzle (conflict-free), then lane 0
+// stores the block with one tensor copy per 64-channel half.
+template <int D, int BITS, int G>
+__device__ __forceinline__ void decode_block_tma(const DenseLayout &lay, const uint8_t *codes,
+                                                 const uint8_t *meta, uint32_t v0,
+                                                 const uint32_t *mask, uint8_t *stage,
+                                                 bool &stage_busy) {
+  using C = Cfg<D, BITS, G>;
+  const int lane = threadIdx.x & 31, sw = lane & 7;
+  uint32_t out[D / 2];
+  Dec<D, BITS, G>::vector(codes + lane * C::CB, meta + lane * C::MB, mask, out);
+  if (stage_busy && lane == 0) bulk_wait_read<0>();  // the previous block's stores have read it
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c)
+    *reinterpret_cast<uint4 *>(stage + (c >> 3) * 4096 + lane * 128 + (((c & 7) ^ sw) << 4)) =
+        make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    const uint32_t lkh = fdiv(lay.T, v0), t0 = v0 - lkh * lay.T.d;
+    const uint32_t lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh)
+      tma_store_5d(&lay.tmap, hh * 64, int(t0), int(h), int(lk & 1u), int(lk >> 1), stage + hh * 4096);
+    bulk_commit();
+  }
+  stage_busy = true;
+}
+
 template <int D, int BITS, int G, class Layout>
 __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, uint8_t *smem,
                             const uint32_t *cum) {
@@ -287,6 +320,21 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     cphase ^= 1u << k;
   };
   bool row_busy = false;
+  // Dense receivers with a tensor map store whole blocks from a per-warp
+  // staging buffer (aliasing the per-thread rows, which that path leaves
+  // unused); other receivers store each row with its own bulk copy.
+  bool use_tma = false;
+  if constexpr (!kIsPaged<Layout>) use_tma = lay.tma != 0;
+  uint8_t *stage = smem + S::rows + warp * (size_t(D / 64) * 4096);
+  auto emit = [&](const uint8_t *codes, const uint8_t *meta, uint32_t v0, uint32_t nv) {
+    if constexpr (!kIsPaged<Layout>) {
+      if (use_tma) {
+        decode_block_tma<D, BITS, G>(lay, codes, meta, v0, ctl->mask, stage, row_busy);
+        return;
+      }
+    }
+    decode_block<D, BITS, G>(a, lay, cum, codes, meta, v0, nv, ctl->mask, row, row_busy);
+  };
 
   // Phase 1 (rare): code chunks that used zero-byte elimination. The CTA
   // expands each one into shared memory, then the warps decode its blocks.
@@ -319,8 +367,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
       __syncwarp();
       issue(v0, nv, nullptr, 0);
       wait(0);
-      decode_block<D, BITS, G>(a, lay, cum, zbuf + b * 32 * C::CB, mbuf, v0, nv, ctl->mask, row,
-                               row_busy);
+      emit(zbuf + b * 32 * C::CB, mbuf, v0, nv);
     }
   }
 
@@ -354,8 +401,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     if (nb < nblk) issue_raw(nb, k ^ 1);
     wait(k);
     const uint32_t v0 = vs0 + b * 32;
-    decode_block<D, BITS, G>(a, lay, cum, cbuf + k * S::BLK, mbuf + k * S::MBLK, v0,
-                             min(32u, vs1 - v0), ctl->mask, row, row_busy);
+    emit(cbuf + k * S::BLK, mbuf + k * S::MBLK, v0, min(32u, vs1 - v0));
     b = nb;
     k ^= 1;
   }

@@ -93,6 +93,16 @@ __device__ __forceinline__ void tma_load_5d(void *sdst, const CUtensorMap *map, 
       : "memory");
 }
 
+// Tensor-map store of a 5-D box from shared memory (bulk group completion).
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap *map, int c0, int c1, int c2, int c3,
+                                             int c4, const void *ssrc) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group"
+      " [%0, {%1, %2, %3, %4, %5}], [%6];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(ssrc))
+      : "memory");
+}
+
 // global -> shared, completion counted in bytes on `bar`.
 __device__ __forceinline__ void bulk_g2s(void *sdst, const void *gsrc, uint32_t bytes,
                                          uint64_t *bar) {
