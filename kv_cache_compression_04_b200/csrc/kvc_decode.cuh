@@ -178,20 +178,14 @@ struct Dec : Cfg<D, BITS, G> {
   }
 };
 
-// Decodes vectors v0 .. v0 + nvec - 1 (one per lane) whose codes start at
-// `codes` (CB bytes each, lane order) and meta at `meta` (MB bytes each).
-template <int D, int BITS, int G, class Layout>
-__device__ __forceinline__ void decode_block(const DecArgs &a, const Layout &lay, const uint32_t *cum,
-                                             const uint8_t *codes, const uint8_t *meta, uint32_t v0,
-                                             uint32_t nvec, const uint32_t *mask, uint8_t *row,
-                                             bool &row_busy) {
-  using C = Cfg<D, BITS, G>;
-  const int lane = threadIdx.x & 31;
-  if (uint32_t(lane) >= nvec) return;
-  uint32_t out[D / 2];
-  Dec<D, BITS, G>::vector(codes + lane * C::CB, meta + lane * C::MB, mask, out);
+// Stores this lane's decoded vector v (bf16 words `out`) with its own bulk
+// copy from the lane's row buffer.
+template <int D, class Layout>
+__device__ __forceinline__ void store_row(const DecArgs &a, const Layout &lay, const uint32_t *cum,
+                                          const uint32_t (&out)[D / 2], uint32_t v, uint8_t *row,
+                                          bool &row_busy) {
   bool ok;
-  uint8_t *dst = vec_addr(lay, cum, v0 + lane, ok);  // after the vector: fewer live registers
+  uint8_t *dst = vec_addr(lay, cum, v, ok);
   if (!ok) {
     set_status(a.status, KVC_ERR_CORRUPT);
     return;
@@ -202,7 +196,7 @@ __device__ __forceinline__ void decode_block(const DecArgs &a, const Layout &lay
   for (int q = 0; q < D / 8; ++q)
     r4[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
   fence_proxy_async_smem();
-  bulk_s2g(dst, row, C::ROW);
+  bulk_s2g(dst, row, uint32_t(D) * 2);
   bulk_commit();
   row_busy = true;
 }
@@ -211,15 +205,10 @@ __device__ __forceinline__ void decode_block(const DecArgs &a, const Layout &lay
 // vectors of one head row): the lanes write their rows into the warp's
 // staging buffer in the map's 128-byte swizzle (conflict-free), then lane 0
 // stores the block with one tensor copy per 64-channel half.
-template <int D, int BITS, int G>
-__device__ __forceinline__ void decode_block_tma(const DenseLayout &lay, const uint8_t *codes,
-                                                 const uint8_t *meta, uint32_t v0,
-                                                 const uint32_t *mask, uint8_t *stage,
-                                                 bool &stage_busy) {
-  using C = Cfg<D, BITS, G>;
+template <int D>
+__device__ __forceinline__ void store_block_tma(const DenseLayout &lay, const uint32_t (&out)[D / 2],
+                                                uint32_t v0, uint8_t *stage, bool &stage_busy) {
   const int lane = threadIdx.x & 31, sw = lane & 7;
-  uint32_t out[D / 2];
-  Dec<D, BITS, G>::vector(codes + lane * C::CB, meta + lane * C::MB, mask, out);
   if (stage_busy && lane == 0) bulk_wait_read<0>();  // the previous block's stores have read it
   __syncwarp();
 #pragma unroll
@@ -279,16 +268,24 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     if (i + 1 == ctl->n_chunks) ok = ok && base + off + round16(size) == ctl->stream_bytes;
     return ok;
   };
+  // Also counts the range's code chunks that used zero-byte elimination
+  // (usually none: then phase 1 and the per-block raw test are skipped).
+  bool any_elim;
   {
-    uint32_t bad = 0;
-    for (uint32_t t = t0 + tid; t < t1; t += kDecThreads)
-      bad |= !entry_ok(t, min(uint32_t(C::VC), V - t * C::VC) * C::CB);
+    uint32_t bad = 0, elim = 0;
+    for (uint32_t t = t0 + tid; t < t1; t += kDecThreads) {
+      const uint32_t len = min(uint32_t(C::VC), V - t * C::VC) * C::CB;
+      bad |= !entry_ok(t, len);
+      elim |= uint32_t(ld_u64(table + 8 * uint64_t(t)) & 0xFFFFu) != len;
+    }
     for (uint32_t s = seg0 + tid; s <= seg1; s += kDecThreads)
       bad |= !entry_ok(uint64_t(n_tiles) + s, min(uint32_t(C::VM), V - s * C::VM) * C::MB);
-    if (block_sum<kDecThreads>(bad, ctl->red)) {
+    const uint32_t sum = block_sum<kDecThreads>(bad | (elim << 16), ctl->red);
+    if (sum & 0xFFFFu) {
       if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
       return;
     }
+    any_elim = sum != 0;
   }
 
   // D3 for meta: a raw meta chunk is read in place; an eliminated one was
@@ -326,21 +323,27 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   bool use_tma = false;
   if constexpr (!kIsPaged<Layout>) use_tma = lay.tma != 0;
   uint8_t *stage = smem + S::rows + warp * (size_t(D / 64) * 4096);
+  // Decodes vectors v0 .. v0 + nv - 1 (one per lane) whose codes start at
+  // `codes` (CB bytes each, lane order) and meta at `meta` (MB bytes each).
+  // One copy of the unrolled vector code serves both store paths.
   auto emit = [&](const uint8_t *codes, const uint8_t *meta, uint32_t v0, uint32_t nv) {
+    uint32_t out[D / 2];
+    const bool act = uint32_t(lane) < nv;
+    if (act) Dec<D, BITS, G>::vector(codes + lane * C::CB, meta + lane * C::MB, ctl->mask, out);
     if constexpr (!kIsPaged<Layout>) {
       if (use_tma) {
-        decode_block_tma<D, BITS, G>(lay, codes, meta, v0, ctl->mask, stage, row_busy);
+        store_block_tma<D>(lay, out, v0, stage, row_busy);
         return;
       }
     }
-    decode_block<D, BITS, G>(a, lay, cum, codes, meta, v0, nv, ctl->mask, row, row_busy);
+    if (act) store_row<D>(a, lay, cum, out, v0 + lane, row, row_busy);
   };
 
   // Phase 1 (rare): code chunks that used zero-byte elimination. The CTA
   // expands each one into shared memory, then the warps decode its blocks.
   uint32_t zphase = 0;
 #pragma unroll 1
-  for (uint32_t t = t0; t < t1; ++t) {
+  for (uint32_t t = t0; any_elim && t < t1; ++t) {
     const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
     const uint32_t csize = uint32_t(ce & 0xFFFFu);
     const uint32_t nvec = min(uint32_t(C::VC), V - t * C::VC);
@@ -382,7 +385,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     return uint32_t(ce & 0xFFFFu) == min(uint32_t(C::VC), V - t * C::VC) * C::CB;
   };
   auto next_raw = [&](uint32_t b) {
-    while (b < nblk && !raw_block(b)) b += kDecWarps;
+    while (any_elim && b < nblk && !raw_block(b)) b += kDecWarps;
     return b;
   };
   auto issue_raw = [&](uint32_t b, uint32_t k) {

@@ -245,6 +245,52 @@ KVC_HD void transpose32(uint32_t (&a)[32]) {
   }
 }
 
+// Byte permute (PRMT semantics: selector nibble i picks byte i of the result
+// from the eight bytes y:x, x being bytes 0..3), usable on the host as well.
+KVC_HD uint32_t prmt(uint32_t x, uint32_t y, uint32_t sel) {
+#ifdef __CUDA_ARCH__
+  return __byte_perm(x, y, sel);
+#else
+  const uint64_t v = (uint64_t(y) << 32) | x;
+  uint32_t r = 0;
+  for (int i = 0; i < 4; ++i) r |= uint32_t((v >> (8 * ((sel >> (4 * i)) & 7))) & 0xFFu) << (8 * i);
+  return r;
+#endif
+}
+
+// transpose32 split between two threads. Half h holds rows 16h .. 16h+15 of
+// the 32x32 bit matrix (a[i] = row 16h + i), `other` the partner's a[i].
+// The 16-bit block exchange is one byte permute per row:
+//   row i      keeps its low half and takes the low half of row i + 16 on top,
+//   row i + 16 keeps its high half and takes the high half of row i below.
+KVC_HD uint32_t transpose_split_stage16(uint32_t mine, uint32_t other, int h) {
+  return prmt(mine, other, h ? 0x3276u : 0x5410u);
+}
+// The remaining levels (8, 4, 2, 1 bits) act within each half. The 8-bit
+// level is a byte permute too.
+KVC_HD void transpose_split_rest(uint32_t (&a)[16]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t x = a[k], y = a[k + 8];
+    a[k] = prmt(x, y, 0x6240u);      // bytes x0 y0 x2 y2
+    a[k + 8] = prmt(x, y, 0x7351u);  // bytes x1 y1 x3 y3
+  }
+  const uint32_t masks[3] = {0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+  for (int lvl = 0; lvl < 3; ++lvl) {
+    const int j = 4 >> lvl;
+    const uint32_t m = masks[lvl];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if ((k & j) == 0) {
+        const uint32_t t = ((a[k] >> j) ^ a[k + j]) & m;
+        a[k] ^= t << j;
+        a[k + j] ^= t;
+      }
+    }
+  }
+}
+
 // -------------------------------------------------------------- scans --
 // Exclusive sum over the first NT threads of the block (named barrier 1);
 // also returns the total. `red` holds NT/32 words of shared memory.
@@ -280,7 +326,7 @@ __device__ __forceinline__ uint32_t block_sum(uint32_t x, uint32_t *red) {
 // ------------------------------------------- lossless stage (16 KB chunk) --
 // Reading R10 (bit planes of 32-bit little-endian words) and R11 (zero-byte
 // elimination: 2048-byte bitmap + nonzero bytes), on a chunk in shared
-// memory, by the first NT threads.
+// memory, by the first 256 threads.
 
 // Nonzero bytes the bit-plane shuffle of the chunk would have: byte i of
 // plane p is nonzero iff bit p of (w[8i] | ... | w[8i+7]) is set, so the
@@ -301,38 +347,62 @@ __device__ __forceinline__ uint32_t chunk_nnz_part(const uint8_t *buf) {
 
 // Plane words: the shuffled chunk as 4096 little-endian words, word
 // p * 128 + m holding bit p of words 32m .. 32m+31 (bytes p*512 + 4m ..).
-//
-// Thread m (< 128) transposes words 32m .. 32m+31 in registers. It moves its
-// eight 16-byte pieces in an order rotated by m, so that the eight threads of
-// a shared-memory phase hit eight different bank groups; the rotation of the
-// words by r = 4 * (m % 8) becomes a rotation of every transposed word by r,
-// undone (or applied) by a funnel shift.
-__device__ __forceinline__ void planes_from_words(const uint8_t *buf, uint32_t *pw, int m) {
-  const uint4 *src = reinterpret_cast<const uint4 *>(buf + m * 128);
-  uint32_t a[32];
+// Their shared-memory image (scratch between the transpose and the byte
+// compaction) keeps word (p, m) at p * 128 + (m ^ 16 * (p >> 4)).
+__device__ __forceinline__ uint32_t pw_index(uint32_t p, uint32_t m) {
+  return p * 128 + (m ^ ((p >> 4) << 4));
+}
+
+// The 128 groups of 32 words are transposed by thread pairs (the first 256
+// threads): lane l of warp w takes group m = 16w + 4(l >> 3) + (l & 3) and
+// half h = (l >> 2) & 1; its partner is lane l ^ 4. The pair transposes the
+// group's rows rotated by r = 4s, s = l & 3 (half h reads its four 16-byte
+// pieces from piece 4h + s on, so the eight lanes of a shared-memory phase
+// hit eight different bank groups); rotating the rows rotates every
+// transposed word by r bits, which a funnel shift undoes. In the image the
+// partners' words (same m, planes p and p + 16) fall in different banks.
+struct PairLane {
+  int m, h, s;
+};
+__device__ __forceinline__ PairLane pair_lane() {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  return {16 * warp + 4 * (lane >> 3) + (lane & 3), (lane >> 2) & 1, lane & 3};
+}
+
+__device__ __forceinline__ void planes_from_words(const uint8_t *buf, uint32_t *pw) {
+  const PairLane L = pair_lane();
+  const uint4 *src = reinterpret_cast<const uint4 *>(buf + L.m * 128);
+  uint32_t a[16];  // rows 16h .. 16h+15 of the rotated group
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const uint4 v = src[(q + m) & 7];  // words 4q + r .. (mod 32)
+  for (int q = 0; q < 4; ++q) {
+    const uint4 v = src[(4 * L.h + q + L.s) & 7];
     a[4 * q] = v.x, a[4 * q + 1] = v.y, a[4 * q + 2] = v.z, a[4 * q + 3] = v.w;
   }
-  transpose32(a);
-  const int r = 4 * (m & 7);
 #pragma unroll
-  for (int p = 0; p < 32; ++p) pw[p * 128 + m] = __funnelshift_l(a[p], a[p], r);
+  for (int i = 0; i < 16; ++i)
+    a[i] = transpose_split_stage16(a[i], __shfl_xor_sync(0xFFFFFFFFu, a[i], 4), L.h);
+  transpose_split_rest(a);
+  const int r = 4 * L.s;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pw[pw_index(16 * L.h + i, L.m)] = __funnelshift_l(a[i], a[i], r);
 }
-__device__ __forceinline__ void words_from_planes(const uint32_t *pw, uint8_t *buf, int m) {
-  const int r = 4 * (m & 7);
-  uint32_t a[32];
+__device__ __forceinline__ void words_from_planes(const uint32_t *pw, uint8_t *buf) {
+  const PairLane L = pair_lane();
+  const int r = 4 * L.s;
+  uint32_t a[16];
 #pragma unroll
-  for (int p = 0; p < 32; ++p) {
-    const uint32_t x = pw[p * 128 + m];
-    a[p] = __funnelshift_r(x, x, r);
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t x = pw[pw_index(16 * L.h + i, L.m)];
+    a[i] = __funnelshift_r(x, x, r);
   }
-  transpose32(a);  // a[l] = word (l + r) mod 32 of the group
-  uint4 *dst = reinterpret_cast<uint4 *>(buf + m * 128);
 #pragma unroll
-  for (int q = 0; q < 8; ++q)
-    dst[(q + m) & 7] = make_uint4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+  for (int i = 0; i < 16; ++i)
+    a[i] = transpose_split_stage16(a[i], __shfl_xor_sync(0xFFFFFFFFu, a[i], 4), L.h);
+  transpose_split_rest(a);  // a[i] = word (16h + i + r) mod 32 of the group
+  uint4 *dst = reinterpret_cast<uint4 *>(buf + L.m * 128);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    dst[(4 * L.h + q + L.s) & 7] = make_uint4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
 }
 
 // Nonzero-byte mask of a word: bit b set iff byte b is nonzero. The top bit
@@ -382,84 +452,122 @@ __device__ __forceinline__ uint32_t compact_selector(uint32_t n) {
   return sel;
 }
 
-// buf holds a full 16 KB chunk; on return it holds bitmap + nonzero bytes
-// (the caller knows their count from chunk_nnz_part). scr: 16 KB scratch.
-// Run by the first 256 threads. Thread t owns plane words 16t .. 16t+15
-// (bitmap words 2t, 2t+1): it compacts the nonzero bytes of each with one
-// byte permute and writes them after the bytes of threads < t (block scan).
+// Byte positions of the compaction. Warp w covers plane words 512w ..
+// 512w + 511 in four rounds; in round k lane l takes the four words
+// j = 512w + 128k + 4l .. + 3 (plane 4w + k), whose bitmap bits are the
+// 16-bit bitmap word j / 4. cnt[k] is the lane's nonzero-byte count in round
+// k; q[k] receives the exclusive prefix over all words before its first one
+// (plus the bitmap), `total` the chunk's count. Two rounds share one warp
+// scan (a round's warp total is at most 512, so 16-bit halves cannot
+// overflow); warp totals go through red[] (named barrier 1, first NT
+// threads). The caller passes another barrier before red is reused.
+template <int NT>
+__device__ __forceinline__ void ze_positions(const uint32_t (&cnt)[4], uint32_t *red,
+                                             uint32_t (&q)[4], uint32_t &total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t i01 = warp_incl_scan(cnt[0] | (cnt[1] << 16));
+  const uint32_t i23 = warp_incl_scan(cnt[2] | (cnt[3] << 16));
+  const uint32_t t01 = __shfl_sync(0xFFFFFFFFu, i01, 31), t23 = __shfl_sync(0xFFFFFFFFu, i23, 31);
+  const uint32_t r0 = t01 & 0xFFFFu, r1 = t01 >> 16, r2 = t23 & 0xFFFFu, r3 = t23 >> 16;
+  if (lane == 0) red[warp] = r0 + r1 + r2 + r3;
+  named_bar_sync(1, NT);
+  uint32_t base = kBitmap, all = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const uint32_t v = red[w];
+    base += (w < warp) ? v : 0u;
+    all += v;
+  }
+  total = all;
+  q[0] = base + (i01 & 0xFFFFu) - cnt[0];
+  q[1] = base + r0 + (i01 >> 16) - cnt[1];
+  q[2] = base + r0 + r1 + (i23 & 0xFFFFu) - cnt[2];
+  q[3] = base + r0 + r1 + r2 + (i23 >> 16) - cnt[3];
+}
+
+// buf holds a full chunk (first 256 threads); on return it holds bitmap + nonzero bytes (the
+// caller knows their count from chunk_nnz_part). scr: 16 KB scratch. Each
+// word's nonzero bytes are packed by one byte permute and stored at its
+// position; the lanes of a warp store next to one another.
 template <int NT>
 __device__ __forceinline__ void ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *red) {
-  static_assert(NT == 256, "16 plane words per thread");
+  static_assert(NT == 256, "eight warps of 512 plane words");
   __shared__ uint32_t lut[16];
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t *pw = reinterpret_cast<uint32_t *>(scr);
   if (tid < 16) lut[tid] = compact_selector(tid);
-  for (int m = tid; m < 128; m += NT) planes_from_words(buf, pw, m);
-  named_bar_sync(1, NT);
-  uint32_t x[16], n[16], cnt = 0, bw0 = 0, bw1 = 0;
-  const uint4 *src = reinterpret_cast<const uint4 *>(pw + 16 * tid);
+  planes_from_words(buf, pw);
+  named_bar_sync(1, NT);  // buf is free from here on
+  uint32_t x[4][4], nib[4], cnt[4];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 v = src[q];
-    x[4 * q] = v.x, x[4 * q + 1] = v.y, x[4 * q + 2] = v.z, x[4 * q + 3] = v.w;
+  for (int k = 0; k < 4; ++k) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(pw + pw_index(4 * warp + k, 4 * lane));
+    x[k][0] = v.x, x[k][1] = v.y, x[k][2] = v.z, x[k][3] = v.w;
+    nib[k] = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) nib[k] |= nz_nibble(x[k][e]) << (4 * e);
+    cnt[k] = __popc(nib[k]);
+    reinterpret_cast<uint16_t *>(buf)[128 * warp + 32 * k + lane] = uint16_t(nib[k]);
   }
+  uint32_t q[4], total;
+  ze_positions<NT>(cnt, red, q, total);
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    n[k] = nz_nibble(x[k]);
-    cnt += __popc(n[k]);
-    if (k < 8)
-      bw0 |= n[k] << (4 * k);
-    else
-      bw1 |= n[k] << (4 * (k - 8));
-  }
-  uint32_t total;
-  uint32_t q = kBitmap + block_excl_scan<NT>(cnt, red, total);  // buf is free after this
-  reinterpret_cast<uint2 *>(buf)[tid] = make_uint2(bw0, bw1);
+  for (int k = 0; k < 4; ++k) {
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const uint32_t c = __byte_perm(x[k], 0, lut[n[k]]), nb = __popc(n[k]);
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t n = (nib[k] >> (4 * e)) & 0xFu;
+      const uint32_t c = __byte_perm(x[k][e], 0, lut[n]), nb = __popc(n);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (uint32_t(i) < nb) buf[q + i] = uint8_t(c >> (8 * i));
-    q += nb;
+      for (int i = 0; i < 4; ++i)
+        if (uint32_t(i) < nb) buf[q[k] + i] = uint8_t(c >> (8 * i));
+      q[k] += nb;
+    }
   }
   named_bar_sync(1, NT);
 }
 
 // Inverse: buf holds bitmap + nonzero bytes (`size` bytes); on return it
 // holds the 16 KB chunk. Returns false (for every thread) if the bitmap's
-// popcount disagrees with the size; then buf is unspecified. Thread t
-// rebuilds plane words 16t .. 16t+15: each takes the next popcount(n) source
-// bytes (an unaligned 4-byte window) and spreads them with one byte permute.
+// popcount disagrees with the size; then buf is unspecified. Each plane word
+// takes the next popcount(n) source bytes (an unaligned 4-byte window) and
+// spreads them with one byte permute.
 template <int NT>
 __device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *red, uint32_t size) {
-  static_assert(NT == 256, "16 plane words per thread");
+  static_assert(NT == 256, "eight warps of 512 plane words");
   __shared__ uint32_t lut[16];
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t *pw = reinterpret_cast<uint32_t *>(scr);
   if (tid < 16) lut[tid] = expand_selector(tid);
-  const uint2 bw = reinterpret_cast<const uint2 *>(buf)[tid];
-  uint32_t total;
-  uint32_t p = kBitmap +
-               block_excl_scan<NT>(__popc(bw.x) + __popc(bw.y), red, total);  // lut visible after
-  if (total != size - kBitmap) return false;
+  uint32_t nib[4], cnt[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    nib[k] = reinterpret_cast<const uint16_t *>(buf)[128 * warp + 32 * k + lane];
+    cnt[k] = __popc(nib[k]);
+  }
+  uint32_t q[4], total;
+  ze_positions<NT>(cnt, red, q, total);  // lut visible after its barrier
+  if (total != size - kBitmap) {
+    named_bar_sync(1, NT);  // red read by all before anyone reuses it
+    return false;
+  }
   // the window's words are clamped to the buffer: a byte it needs lies below
   // `size` <= 16384, so a clamped word is never one whose bytes are used
   const uint32_t *b32 = reinterpret_cast<const uint32_t *>(buf);
-  uint32_t o[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const uint32_t n = ((k < 8 ? bw.x : bw.y) >> (4 * (k & 7))) & 0xFu;
-    const uint32_t a = min(p >> 2, 4095u), a1 = min((p >> 2) + 1, 4095u);
-    const uint32_t win = __funnelshift_r(b32[a], b32[a1], 8 * (p & 3));
-    o[k] = __byte_perm(win, 0, lut[n]);
-    p += __popc(n);
+  for (int k = 0; k < 4; ++k) {
+    uint32_t o[4], p = q[k];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t n = (nib[k] >> (4 * e)) & 0xFu;
+      const uint32_t a = min(p >> 2, 4095u), a1 = min((p >> 2) + 1, 4095u);
+      const uint32_t win = __funnelshift_r(b32[a], b32[a1], 8 * (p & 3));
+      o[e] = __byte_perm(win, 0, lut[n]);
+      p += __popc(n);
+    }
+    *reinterpret_cast<uint4 *>(pw + pw_index(4 * warp + k, 4 * lane)) = make_uint4(o[0], o[1], o[2], o[3]);
   }
-  uint4 *dst = reinterpret_cast<uint4 *>(pw + 16 * tid);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
   named_bar_sync(1, NT);
-  for (int m = tid; m < 128; m += NT) words_from_planes(pw, buf, m);
+  words_from_planes(pw, buf);
   named_bar_sync(1, NT);
   return true;
 }

@@ -10,6 +10,20 @@ void hl_transpose32(const uint32_t *in, uint32_t *out) {
   kvc::transpose32(a);
   for (int i = 0; i < 32; ++i) out[i] = a[i];
 }
+// The two-thread split of the transpose: each half runs the byte-permute
+// exchange against the other half's rows, then the in-half levels.
+void hl_transpose32_split(const uint32_t *in, uint32_t *out) {
+  uint32_t lo[16], hi[16];
+  for (int i = 0; i < 16; ++i) lo[i] = in[i], hi[i] = in[16 + i];
+  uint32_t nlo[16], nhi[16];
+  for (int i = 0; i < 16; ++i) {
+    nlo[i] = kvc::transpose_split_stage16(lo[i], hi[i], 0);
+    nhi[i] = kvc::transpose_split_stage16(hi[i], lo[i], 1);
+  }
+  kvc::transpose_split_rest(nlo);
+  kvc::transpose_split_rest(nhi);
+  for (int i = 0; i < 16; ++i) out[i] = nlo[i], out[16 + i] = nhi[i];
+}
 void hl_sign_masks(uint64_t seed, int d, uint32_t *out) { kvc::sign_masks(seed, d, out); }
 // Mismatches of the library's nonzero-byte mask against a byte-by-byte
 // reference over words [start, start + count).

@@ -164,6 +164,7 @@ def host_logic():
     lib.hl_fdiv.restype = C.c_uint32
     lib.hl_fdiv.argtypes = [C.c_uint32, C.c_uint32]
     lib.hl_transpose32.argtypes = [C.c_void_p, C.c_void_p]
+    lib.hl_transpose32_split.argtypes = [C.c_void_p, C.c_void_p]
     lib.hl_nz_nibble_mismatches.restype = C.c_uint64
     lib.hl_nz_nibble_mismatches.argtypes = [C.c_uint64, C.c_uint64]
     lib.hl_sign_masks.argtypes = [C.c_uint64, C.c_int, C.c_void_p]
@@ -180,12 +181,17 @@ def test_fast_division_exact(host_logic):
             assert host_logic.hl_fdiv(dv, int(n)) == int(n) // dv, (dv, n)
 
 
-def test_transpose32_is_bit_matrix_transpose(host_logic):
+@pytest.mark.parametrize("fn", ["hl_transpose32", "hl_transpose32_split"])
+def test_transpose32_is_bit_matrix_transpose(host_logic, fn):
+    """Both the one-thread transpose and its two-thread split (the kernels'
+    form) are the bit-matrix transpose: bit l of out[p] = bit p of in[l]."""
     rng = np.random.default_rng(1)
-    for _ in range(20):
-        a = rng.integers(0, 2 ** 32, 32, dtype=np.uint64).astype(np.uint32)
+    cases = [rng.integers(0, 2 ** 32, 32, dtype=np.uint64).astype(np.uint32) for _ in range(20)]
+    cases += [np.array([1 << ((3 * i) % 32) for i in range(32)], np.uint32),
+              np.eye(32, dtype=np.uint32)[0] * 0xFFFFFFFF]
+    for a in cases:
         out = np.zeros(32, np.uint32)
-        host_logic.hl_transpose32(a.ctypes.data, out.ctypes.data)
+        getattr(host_logic, fn)(a.ctypes.data, out.ctypes.data)
         bits = (a[:, None] >> np.arange(32, dtype=np.uint32)) & 1       # [row l, bit p]
         want = (bits.T.astype(np.uint64) << np.arange(32, dtype=np.uint64)).sum(1)
         assert np.array_equal(out, want.astype(np.uint32))
