@@ -36,16 +36,16 @@ struct DecCtl {
   alignas(16) uint32_t mask[128];  // read as uint4
 };
 
-// Shared memory: output rows | per-warp code blocks | per-warp meta blocks |
-// expanded code chunk | expansion scratch | control | request prefix (paged).
+// Shared memory: per-warp output staging | per-warp code blocks | per-warp
+// meta blocks | expanded code chunk | expansion scratch | control | request
+// prefix (paged).
 template <int D>
 struct DecSmem {
-  static constexpr size_t ROWP = 2 * D + 16;
+  static constexpr size_t WBUF = size_t(D / 64) * 4096;    // 32 rows, 128-byte swizzled halves
   static constexpr size_t BLK = 32 * size_t(D) / 2;       // widest code block (4-bit)
   static constexpr size_t MBLK = 32 * (size_t(D) / 32) * 4;  // widest meta block (group 32)
-  static constexpr size_t rows = 0;  // also the per-warp tensor-store staging buffers
-  static constexpr size_t code = rows + kDecThreads * ROWP;
-  static_assert(kDecThreads * ROWP >= kDecWarps * (size_t(D / 64) * 4096), "staging fits");
+  static constexpr size_t rows = 0;
+  static constexpr size_t code = rows + kDecWarps * WBUF;
   static constexpr size_t meta = code + 2 * kDecWarps * BLK;
   static constexpr size_t zchunk = meta + 2 * kDecWarps * MBLK;
   static constexpr size_t scr = zchunk + kChunk;
@@ -178,43 +178,27 @@ struct Dec : Cfg<D, BITS, G> {
   }
 };
 
-// Stores this lane's decoded vector v (bf16 words `out`) with its own bulk
-// copy from the lane's row buffer.
-template <int D, class Layout>
-__device__ __forceinline__ void store_row(const DecArgs &a, const Layout &lay, const uint32_t *cum,
-                                          const uint32_t (&out)[D / 2], uint32_t v, uint8_t *row,
-                                          bool &row_busy) {
-  bool ok;
-  uint8_t *dst = vec_addr(lay, cum, v, ok);
-  if (!ok) {
-    set_status(a.status, KVC_ERR_CORRUPT);
-    return;
-  }
-  if (row_busy) bulk_wait_read<0>();  // this thread's previous store has read the row
-  uint4 *r4 = reinterpret_cast<uint4 *>(row);
+// Writes this lane's decoded row (bf16 words `out`) into the warp's staging
+// buffer as row `lane` of the 128-byte swizzle (conflict-free).
+template <int D>
+__device__ __forceinline__ void stage_row(const uint32_t (&out)[D / 2], uint8_t *stage) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int q = 0; q < D / 8; ++q)
-    r4[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
-  fence_proxy_async_smem();
-  bulk_s2g(dst, row, uint32_t(D) * 2);
-  bulk_commit();
-  row_busy = true;
+  for (int c = 0; c < D / 8; ++c)
+    *reinterpret_cast<uint4 *>(stage + swz_offset(lane, c)) =
+        make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
 }
 
 // Dense receiver with a tensor map (tokens % 32 == 0, so the block is 32
-// vectors of one head row): the lanes write their rows into the warp's
-// staging buffer in the map's 128-byte swizzle (conflict-free), then lane 0
-// stores the block with one tensor copy per 64-channel half.
+// vectors of one head row): lane 0 stores the staged block with one tensor
+// copy per 64-channel half.
 template <int D>
 __device__ __forceinline__ void store_block_tma(const DenseLayout &lay, const uint32_t (&out)[D / 2],
                                                 uint32_t v0, uint8_t *stage, bool &stage_busy) {
-  const int lane = threadIdx.x & 31, sw = lane & 7;
+  const int lane = threadIdx.x & 31;
   if (stage_busy && lane == 0) bulk_wait_read<0>();  // the previous block's stores have read it
   __syncwarp();
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c)
-    *reinterpret_cast<uint4 *>(stage + (c >> 3) * 4096 + lane * 128 + (((c & 7) ^ sw) << 4)) =
-        make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+  stage_row<D>(out, stage);
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
@@ -243,7 +227,6 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   const uint64_t base = ctl->data_base;
   const uint64_t limit = min(a.in_bytes, ctl->stream_bytes);
   const uint8_t *table = in + kHeader;
-  uint8_t *row = smem + S::rows + tid * S::ROWP;
   uint8_t *cbuf = smem + S::code + 2 * warp * S::BLK;
   uint8_t *mbuf = smem + S::meta + 2 * warp * S::MBLK;
   uint8_t *zbuf = smem + S::zchunk;
@@ -316,13 +299,13 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
       set_status(a.status, KVC_ERR_TIMEOUT);
     cphase ^= 1u << k;
   };
-  bool row_busy = false;
-  // Dense receivers with a tensor map store whole blocks from a per-warp
-  // staging buffer (aliasing the per-thread rows, which that path leaves
-  // unused); other receivers store each row with its own bulk copy.
+  bool stage_busy = false;
+  // Decoded blocks go through a per-warp staging buffer: dense receivers with
+  // a tensor map store them with tensor copies, other receivers with 16-byte
+  // stores, half a warp per row (scatter_rows).
   bool use_tma = false;
   if constexpr (!kIsPaged<Layout>) use_tma = lay.tma != 0;
-  uint8_t *stage = smem + S::rows + warp * (size_t(D / 64) * 4096);
+  uint8_t *stage = smem + S::rows + warp * S::WBUF;
   // Decodes vectors v0 .. v0 + nv - 1 (one per lane) whose codes start at
   // `codes` (CB bytes each, lane order) and meta at `meta` (MB bytes each).
   // One copy of the unrolled vector code serves both store paths.
@@ -332,11 +315,23 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     if (act) Dec<D, BITS, G>::vector(codes + lane * C::CB, meta + lane * C::MB, ctl->mask, out);
     if constexpr (!kIsPaged<Layout>) {
       if (use_tma) {
-        store_block_tma<D>(lay, out, v0, stage, row_busy);
+        store_block_tma<D>(lay, out, v0, stage, stage_busy);
         return;
       }
     }
-    if (act) store_row<D>(a, lay, cum, out, v0 + lane, row, row_busy);
+    uint8_t *dst = nullptr;
+    if (act) {
+      bool ok;
+      dst = vec_addr(lay, cum, v0 + lane, ok);
+      if (!ok) {
+        set_status(a.status, KVC_ERR_CORRUPT);
+        dst = nullptr;
+      }
+    }
+    __syncwarp();  // the previous block's scatter has read the buffer
+    stage_row<D>(out, stage);
+    __syncwarp();
+    scatter_rows<D>(stage, dst);
   };
 
   // Phase 1 (rare): code chunks that used zero-byte elimination. The CTA

@@ -129,6 +129,21 @@ template <int N>
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
+// 16-byte asynchronous global -> shared copy issued by this thread (L2 only);
+// src_bytes 0 zero-fills the destination and reads nothing.
+__device__ __forceinline__ void cp_async16(void *sdst, const void *gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(sdst)), "l"(gsrc),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Waits for all of this thread's committed 16-byte copies.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // bulk-async reads of them.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -570,6 +585,63 @@ __device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *
   words_from_planes(pw, buf);
   named_bar_sync(1, NT);
   return true;
+}
+
+// ------------------------------------------- warp row blocks (32 rows) --
+// A per-warp buffer of 32 rows of D bf16 in 64-channel halves of 32 x 128
+// bytes, 16-byte piece c of row r at (c / 8) * 4096 + r * 128 +
+// ((c % 8) ^ (r % 8)) * 16: the tensor maps' 128-byte swizzle, in which lane
+// r reading its own row, or a group of lanes reading one row, hits distinct
+// bank groups.
+__device__ __forceinline__ uint32_t swz_offset(int r, int c) {
+  return uint32_t((c >> 3) * 4096 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Gathers the 32 rows whose global addresses the lanes hold (lane r: row r;
+// null: zeros) into the buffer with 16-byte asynchronous copies. Each copy
+// instruction covers D/8-lane groups, one whole row per group, so every
+// group reads 2*D contiguous bytes. `dummy` is any valid global address
+// (passed with zero-fill copies). Completion: cp_async_wait_all + __syncwarp.
+template <int D>
+__device__ __forceinline__ void gather_rows(uint8_t *wbuf, const uint8_t *row, const void *dummy) {
+  constexpr int P = D / 8, RPI = 32 / P;  // pieces per row, rows per instruction
+  const int lane = threadIdx.x & 31, c = lane % P, rs = lane / P;
+  const uint64_t me = reinterpret_cast<uint64_t>(row);
+#pragma unroll
+  for (int i = 0; i < 32 / RPI; ++i) {
+    const int r = i * RPI + rs;
+    const uint64_t s = __shfl_sync(0xFFFFFFFFu, me, r);
+    const void *src = s ? reinterpret_cast<const void *>(s + 16u * c) : dummy;
+    cp_async16(wbuf + swz_offset(r, c), src, s ? 16u : 0u);
+  }
+  cp_async_commit();
+}
+
+// The inverse move: the buffer's rows to the lanes' global addresses (null:
+// not stored), one whole row per lane group and instruction. The caller
+// orders the buffer's writes before it (__syncwarp); the buffer may be
+// rewritten after a __syncwarp that follows it.
+// Pieces are read eight rows' worth at a time before any of them is stored,
+// so the shared loads are not held behind the global stores.
+template <int D>
+__device__ __forceinline__ void scatter_rows(const uint8_t *wbuf, uint8_t *row) {
+  constexpr int P = D / 8, RPI = 32 / P, N = 32 / RPI, B = 8;
+  const int lane = threadIdx.x & 31, c = lane % P, rs = lane / P;
+  const uint64_t me = reinterpret_cast<uint64_t>(row);
+#pragma unroll
+  for (int i0 = 0; i0 < N; i0 += B) {
+    uint4 v[B];
+    uint64_t d[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+      const int r = (i0 + i) * RPI + rs;
+      d[i] = __shfl_sync(0xFFFFFFFFu, me, r);
+      v[i] = *reinterpret_cast<const uint4 *>(wbuf + swz_offset(r, c));
+    }
+#pragma unroll
+    for (int i = 0; i < B; ++i)
+      if (d[i]) *reinterpret_cast<uint4 *>(d[i] + 16u * c) = v[i];
+  }
 }
 
 // --------------------------------------------------------- addressing --

@@ -18,9 +18,11 @@
 // Work: blocks of 32 consecutive vectors, one per lane; warps are fully
 // independent and take blocks round-robin over the grid. Each thread holds
 // one head_dim vector in registers as head_dim/2 pairs (c, c + d/2), so every
-// butterfly stage but the last is a paired f32x2 add/subtract, and copies its
-// next row into its own padded shared-memory slot (bulk-async copy, one
-// mbarrier per thread) as soon as it has read the current one.
+// butterfly stage but the last is a paired f32x2 add/subtract. A warp loads
+// its next block's 32 rows into its shared-memory buffer as soon as every
+// lane has read the current one: one tensor-map copy per 64-channel half for
+// a dense tensor whose blocks are head-row tiles, otherwise a gather of
+// 16-byte asynchronous copies, half a warp per row.
 #pragma once
 
 #include <type_traits>
@@ -52,17 +54,12 @@ struct Cfg {
   static_assert(SLICE % 32 == 0, "meta slices hold whole 8-word groups");
 };
 
-// Shared memory: [per-thread padded rows | per-warp tensor-load buffers (a
-// union: one load path runs)] | per-thread mbarriers | per-warp mbarriers |
-// request prefix (paged).
+// Shared memory: per-warp row buffers | per-warp mbarriers | request prefix
+// (paged).
 template <int D>
 struct EncSmem {
-  static constexpr size_t ROWP = 2 * D + 16;
   static constexpr size_t WBUF = size_t(D / 64) * 32 * 128;  // 32 rows, 128-byte swizzled halves
-  static constexpr size_t A = kEncThreads * ROWP > kEncWarps * WBUF ? kEncThreads * ROWP
-                                                                    : kEncWarps * WBUF;
-  static constexpr size_t bars = (A + 1023) & ~size_t(1023);
-  static constexpr size_t wbars = bars + kEncThreads * 8;
+  static constexpr size_t wbars = kEncWarps * WBUF;
   static constexpr size_t cum = wbars + kEncWarps * 8;
   static_assert(WBUF % 1024 == 0, "swizzled buffers stay 1024-byte aligned");
 };
@@ -242,15 +239,14 @@ __global__ void __launch_bounds__(kEncThreads, 1)
   using S = EncSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint8_t *row = smem + tid * C::ROWP;
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S::bars) + tid;
   uint8_t *wbuf = smem + warp * S::WBUF;
   uint64_t *wbar = reinterpret_cast<uint64_t *>(smem + S::wbars) + warp;
   uint32_t *s_cum = reinterpret_cast<uint32_t *>(smem + S::cum);
 
-  mbar_init(bar, 1);
-  if (lane == 0) mbar_init(wbar, 1);
-  mbar_fence_init();
+  if (lane == 0) {
+    mbar_init(wbar, 1);
+    mbar_fence_init();
+  }
   __syncwarp();  // the warp's barrier is initialized before any lane waits on it
   if constexpr (kPaged) {
     for (uint32_t r = tid; r <= lay.n_req; r += blockDim.x) s_cum[r] = lay.cum[r];
@@ -262,19 +258,17 @@ __global__ void __launch_bounds__(kEncThreads, 1)
   const uint32_t stride = gridDim.x * kEncWarps;
   uint32_t blk = blockIdx.x * kEncWarps + (tid >> 5);
 
-  // Starts the copy of vector v's row; false if nothing was started.
-  auto issue = [&](uint32_t v) -> bool {
-    if (v >= V) return false;
+  // Source row of vector v for the gather path (null past the end or for a
+  // page outside the pool, which is recorded).
+  auto src_of = [&](uint32_t v) -> const uint8_t * {
+    if (v >= V) return nullptr;
     bool ok;
-    const uint8_t *src = vec_addr(lay, s_cum, v, ok);
+    const uint8_t *p = vec_addr(lay, s_cum, v, ok);
     if (!ok) {
       set_status(a.status, KVC_ERR_CORRUPT);
-      mbar_arrive(bar);  // completes the phase without data
-      return true;
+      return nullptr;
     }
-    mbar_arrive_expect_tx(bar, C::ROW);
-    bulk_g2s(row, src, C::ROW, bar);
-    return true;
+    return p;
   };
 
   uint32_t phase = 0, err = 0;
@@ -374,21 +368,21 @@ __global__ void __launch_bounds__(kEncThreads, 1)
     }
   }
   if (!use_tma) {
-    bool pending = blk < n_blocks && issue(blk * 32 + lane);
+    // Row addresses are looked up one block ahead of their gather, so the
+    // page-table read overlaps a block of arithmetic.
+    if (blk < n_blocks) gather_rows<D>(wbuf, src_of(blk * 32 + lane), a.out);
+    const uint8_t *next = src_of((blk + stride) * 32 + lane);
 #pragma unroll 1
     for (; blk < n_blocks; blk += stride) {
       const uint32_t v = blk * 32 + lane;
-      const bool valid = v < V;
+      cp_async_wait_all();
+      __syncwarp();  // every lane's copies have landed
       Pairs<D> y;
-      if (pending) {
-        if (!mbar_wait(bar, phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
-        phase ^= 1;
-      }
-      if (valid) E::unpack(row, a.sign_mask, y);
-      // the row has been read into registers; the next copy may overwrite it
-      fence_proxy_async_smem();
-      pending = blk + stride < n_blocks && issue((blk + stride) * 32 + lane);
-      finish_block(blk, v, valid, y);
+      E::unpack_swz(wbuf, lane, a.sign_mask, y);
+      __syncwarp();  // every lane has read the buffer; the next gather may overwrite it
+      if (blk + stride < n_blocks) gather_rows<D>(wbuf, next, a.out);
+      next = src_of((blk + 2 * stride) * 32 + lane);
+      finish_block(blk, v, v < V, y);
     }
   }
   err = __reduce_or_sync(0xFFFFFFFFu, err);

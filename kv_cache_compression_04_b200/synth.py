@@ -20,6 +20,7 @@ Workloads (logical shape [layers, 2 (K, V), kv_heads, tokens, head_dim], bf16):
   paged   80 layers, 8 heads, d 128, 16 requests of U{512..8192} tokens in
           16-token pages placed by a seeded permutation of the pool; llama8b
           distributions; 4-bit, group 64
+  paged-L the paged batch with L layers (a smaller case of the same kernels)
   sweep   [32, 2, 8, T, 128], T = 8 * 2^i (1 MiB .. 4 GiB), llama8b
           distributions; 4-bit/group 128 and 2-bit/group 32
 """
@@ -80,6 +81,10 @@ def workload(name: str) -> Workload:
         return Workload("qwen7b", 28, 4, 128, 2, 32, 2, "outlier_t", tokens=32768)
     if name == "paged":
         return Workload("paged", 80, 8, 128, 4, 64, 3, "lognormal", 1.5,
+                        seq_lens=paged_seq_lens(3))
+    if name.startswith("paged-"):
+        # paged-<layers>: the paged batch with fewer layers (profiling size)
+        return Workload(name, int(name.split("-")[1]), 8, 128, 4, 64, 3, "lognormal", 1.5,
                         seq_lens=paged_seq_lens(3))
     if name.startswith("sweep"):
         # sweep-<i>-<bits>: T = 8 * 2^i tokens
