@@ -208,13 +208,14 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *o
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   const WsLayout w = ws_layout(s.n_code, s.n_seg);
-  uint32_t *ctl = reinterpret_cast<uint32_t *>(ws);  // status, flags, ticket, reads
+  uint32_t *ctl = reinterpret_cast<uint32_t *>(ws);  // status, flags, ticket, reads, first
   EncArgs a{};
   a.V = uint32_t(s.V);
   a.out = static_cast<uint8_t *>(out);
   a.data_base = s.data_base;
   a.status = ctl;
   a.flags = ctl + 1;
+  a.first_inv = ctl + 4;
   a.code_nnz = reinterpret_cast<unsigned long long *>(ws + w.code_nnz);
   a.meta_nnz = reinterpret_cast<uint32_t *>(ws + w.meta_nnz);
   a.ws_meta = ws + w.meta;
@@ -235,6 +236,7 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *o
   f.out_bytes_dev = out_bytes_dev;
   f.status = ctl;
   f.flags = ctl + 1;
+  f.first_inv = ctl + 4;
   f.ticket = ctl + 2;  // ticket[0]: next code chunk to move, ticket[1]: chunks read
   f.code_nnz = a.code_nnz;
   f.meta_nnz = a.meta_nnz;

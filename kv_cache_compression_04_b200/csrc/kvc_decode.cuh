@@ -1,21 +1,27 @@
-// Fused decode kernel: parse and validate the stream -> per meta chunk: load
-// it and undo zero-byte elimination and the bit-plane shuffle when it used
-// them -> per code chunk of the CTA's tile range: blocks of 32 vectors, one
-// per lane, code bytes loaded by bulk-async copy (a chunk that used zero-byte
-// elimination is first expanded by the whole CTA) -> unpack -> dequantize ->
-// fp32 Walsh-Hadamard (the encoder's butterfly) -> scale by 2^-log2(d) ->
-// unsign -> bf16 -> bulk store (dense) or scatter through the receiver's page
-// table (paged). The decoder is the inverse path the podcast page
+// Decode kernels (D1..D9): parse and validate the stream -> undo zero-byte
+// elimination and the bit-plane shuffle of the chunks that used them ->
+// unpack -> dequantize -> fp32 Walsh-Hadamard (the encoder's butterfly) ->
+// scale by 2^-log2(d) -> unsign -> bf16 -> store (tensor copies for a dense
+// receiver with a tensor map, else 16-byte stores through the receiver's
+// layout or page table). The decoder is the inverse path the podcast page
 // "FastKVComp: checking whether high-throughput KV compression pays off"
 // (episode notes) places on the decode GPU.
 //
-// The chunk table stores every chunk's offset, so each CTA takes a contiguous
-// range of code chunks (tiles) and reads its chunks directly: no scan, no
-// inter-CTA waits. Every table entry is checked against its predecessor
-// (offset = previous offset + padded previous size) by the CTA whose range
-// holds it, so a consistent table is a prefix sum. Warps decode blocks
-// independently; the CTA synchronizes only when it moves to the next meta
-// chunk or expands a zero-byte-eliminated code chunk.
+// Three kernels per call:
+//  meta_expand_kernel   expands the meta chunks that used elimination into
+//                       the workspace;
+//  elim_decode_kernel   decodes the (rare) code chunks that used elimination,
+//                       spread over the CTAs; returns at once unless the
+//                       header says there are some;
+//  decode_kernel        decodes every raw code chunk. The chunk table stores
+//                       every chunk's offset, so each CTA takes a contiguous
+//                       range of code chunks (tiles) and reads its chunks
+//                       directly: no scan, no inter-CTA waits. Every table
+//                       entry is checked against its predecessor (offset =
+//                       previous offset + padded previous size) by the CTA
+//                       whose range holds it, so a consistent table is a
+//                       prefix sum. Warps decode blocks of 32 vectors
+//                       independently.
 #pragma once
 
 #include "kvc_encode.cuh"
@@ -24,21 +30,18 @@ namespace kvc {
 
 constexpr int kDecWarps = 12;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kZeThreads = 256;  // threads that run the chunk expansion
 
 struct DecCtl {
   uint64_t cbar[kDecWarps][2];  // per-warp code + meta blocks loaded (two buffers)
-  uint64_t zbar;                // zero-byte-eliminated code chunk loaded
   uint32_t red[kDecThreads / 32];
-  uint32_t hdr_ok, bad;
-  uint32_t bits, group, n_req_stream, n_chunks;
+  uint32_t hdr_ok;
+  uint32_t bits, group, n_req_stream, n_chunks, code_elim;
   uint64_t data_base, stream_bytes, seed;
   alignas(16) uint32_t mask[128];  // read as uint4
 };
 
 // Shared memory: per-warp output staging | per-warp code blocks | per-warp
-// meta blocks | expanded code chunk | expansion scratch | control | request
-// prefix (paged).
+// meta blocks | control | request prefix (paged).
 template <int D>
 struct DecSmem {
   static constexpr size_t WBUF = size_t(D / 64) * 4096;    // 32 rows, 128-byte swizzled halves
@@ -47,9 +50,7 @@ struct DecSmem {
   static constexpr size_t rows = 0;
   static constexpr size_t code = rows + kDecWarps * WBUF;
   static constexpr size_t meta = code + 2 * kDecWarps * BLK;
-  static constexpr size_t zchunk = meta + 2 * kDecWarps * MBLK;
-  static constexpr size_t scr = zchunk + kChunk;
-  static constexpr size_t ctl = scr + kChunk;
+  static constexpr size_t ctl = meta + 2 * kDecWarps * MBLK;
   static constexpr size_t cum = ctl + ((sizeof(DecCtl) + 15) & ~size_t(15));
   static constexpr size_t bytes(bool paged) {
     return cum + (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
@@ -65,7 +66,7 @@ __device__ __forceinline__ uint64_t ld_u64(const uint8_t *p) {
 
 // D1: the header (reading R12) against the receiver's description.
 struct StreamHdr {
-  uint32_t ok, bits, group, n_req, n_chunks;
+  uint32_t ok, bits, group, n_req, n_chunks, code_elim;
   uint64_t data_base, stream_bytes, seed;
 };
 template <int D>
@@ -75,7 +76,7 @@ __device__ __forceinline__ StreamHdr parse_header(const DecArgs &a) {
   const uint8_t *h = a.in;
   if (a.in_bytes < kHeader) return r;
   const uint32_t bits = h[8], k = h[9], group = ld_u32(h + 12);
-  bool ok = ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 &&
+  bool ok = ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 && h[11] <= 1 &&
             (ld_u32(h + 4) >> 16) == kHeader && (bits == 2 || bits == 4) && k == kLog2D / 2 &&
             (group == 32 || group == 64 || group == 128) && group <= D &&
             ld_u32(h + 16) == a.layers && ld_u32(h + 20) == 2 && ld_u32(h + 24) == a.kv_heads &&
@@ -97,6 +98,7 @@ __device__ __forceinline__ StreamHdr parse_header(const DecArgs &a) {
   r.data_base = base;
   r.stream_bytes = stream_bytes;
   r.seed = ld_u64(h + 40);
+  r.code_elim = h[11];
   return r;
 }
 
@@ -229,8 +231,6 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   const uint8_t *table = in + kHeader;
   uint8_t *cbuf = smem + S::code + 2 * warp * S::BLK;
   uint8_t *mbuf = smem + S::meta + 2 * warp * S::MBLK;
-  uint8_t *zbuf = smem + S::zchunk;
-  uint8_t *scr = smem + S::scr;
   const uint32_t seg0 = t0 / C::R, seg1 = (t1 - 1) / C::R;
 
   // D2: table entries of this range (code chunks t0..t1-1, meta chunks
@@ -264,11 +264,13 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     for (uint32_t s = seg0 + tid; s <= seg1; s += kDecThreads)
       bad |= !entry_ok(uint64_t(n_tiles) + s, min(uint32_t(C::VM), V - s * C::VM) * C::MB);
     const uint32_t sum = block_sum<kDecThreads>(bad | (elim << 16), ctl->red);
-    if (sum & 0xFFFFu) {
+    any_elim = sum != 0;
+    // such chunks must be announced by the header (elim_decode_kernel
+    // decodes them only then)
+    if ((sum & 0xFFFFu) || (any_elim && !ctl->code_elim)) {
       if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
       return;
     }
-    any_elim = sum != 0;
   }
 
   // D3 for meta: a raw meta chunk is read in place; an eliminated one was
@@ -334,44 +336,10 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     scatter_rows<D>(stage, dst);
   };
 
-  // Phase 1 (rare): code chunks that used zero-byte elimination. The CTA
-  // expands each one into shared memory, then the warps decode its blocks.
-  uint32_t zphase = 0;
-#pragma unroll 1
-  for (uint32_t t = t0; any_elim && t < t1; ++t) {
-    const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
-    const uint32_t csize = uint32_t(ce & 0xFFFFu);
-    const uint32_t nvec = min(uint32_t(C::VC), V - t * C::VC);
-    if (csize == nvec * C::CB) continue;
-    __syncthreads();  // zbuf free
-    if (tid == 0) {
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&ctl->zbar, uint32_t(round16(csize)));
-      bulk_g2s(zbuf, in + base + ((ce >> 16) << 4), uint32_t(round16(csize)), &ctl->zbar);
-    }
-    if (!mbar_wait(&ctl->zbar, zphase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
-    zphase ^= 1;
-    bool good = true;
-    if (tid < kZeThreads) good = ze_decode<kZeThreads>(zbuf, scr, ctl->red, csize);
-    if (tid == 0) ctl->bad = !good;
-    __syncthreads();
-    if (ctl->bad) {
-      if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
-      return;
-    }
-#pragma unroll 1
-    for (uint32_t b = warp; b * 32 < nvec; b += kDecWarps) {
-      const uint32_t v0 = t * C::VC + b * 32, nv = min(32u, nvec - b * 32);
-      __syncwarp();
-      issue(v0, nv, nullptr, 0);
-      wait(0);
-      emit(zbuf + b * 32 * C::CB, mbuf, v0, nv);
-    }
-  }
-
-  // Phase 2: raw code chunks, blocks of 32 vectors round-robin over the
-  // warps; each warp loads a block's code and meta bytes with bulk copies
-  // into one of its two buffers while it decodes the previous block.
+  // Raw code chunks, blocks of 32 vectors round-robin over the warps (chunks
+  // that used zero-byte elimination are decoded by elim_decode_kernel); each
+  // warp loads a block's code and meta bytes with bulk copies into one of its
+  // two buffers while it decodes the previous block.
   const uint32_t vs0 = t0 * C::VC, vs1 = min(t1 * C::VC, V);
   const uint32_t nblk = (vs1 - vs0 + 31) / 32;
   auto raw_block = [&](uint32_t b) {  // block b lies in a raw code chunk
@@ -425,14 +393,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     mbar_fence_init();
   }
   if (tid == 0) {
-    mbar_init(&ctl->zbar, 1);
-    mbar_fence_init();
     const StreamHdr h = parse_header<D>(a);
     ctl->hdr_ok = h.ok;
     ctl->bits = h.bits;
     ctl->group = h.group;
     ctl->n_req_stream = h.n_req;
     ctl->n_chunks = h.n_chunks;
+    ctl->code_elim = h.code_elim;
     ctl->data_base = h.data_base;
     ctl->stream_bytes = h.stream_bytes;
     ctl->seed = h.seed;
@@ -587,6 +554,211 @@ __global__ void __launch_bounds__(kMetaThreads, 4)
     k ^= 1;
   }
   if (tid == 0) bulk_wait_all<0>();
+}
+
+// ------------------------------------------------------------------------
+// Code chunks that used zero-byte elimination (rare: e.g. the heads whose
+// keys have the largest outlier channels, where many codes sit at one end of
+// the grid). The header's flag says whether there are any; without it this
+// kernel returns at once. CTA b tests code chunks b, b + grid, ... 256 at a
+// time (such chunks come in runs, which this spreads over the CTAs), expands
+// each eliminated one in shared memory (D3, D4) and decodes its vectors like
+// decode_kernel, which skips them. Table entries used here are bounds-checked
+// on their own (decode_kernel checks the whole table).
+// ------------------------------------------------------------------------
+constexpr int kElimWarps = 8;
+constexpr int kElimThreads = kElimWarps * 32;
+struct ElimCtl {
+  uint64_t zbar;
+  uint64_t mbar[kElimWarps];
+  uint32_t red[kElimThreads / 32];
+  uint32_t ok, bits, group, nlist;
+  uint64_t base, limit;
+  alignas(16) uint32_t mask[128];
+  uint32_t list[kElimThreads];
+};
+// Shared memory: per-warp staging | per-warp meta blocks | chunk | scratch |
+// control | request prefix (paged).
+template <int D>
+struct ElimSmem {
+  static constexpr size_t WBUF = size_t(D / 64) * 4096;
+  static constexpr size_t MBLK = 32 * (size_t(D) / 32) * 4;
+  static constexpr size_t meta = kElimWarps * WBUF;
+  static constexpr size_t chunk = meta + kElimWarps * MBLK;
+  static constexpr size_t scr = chunk + kChunk;
+  static constexpr size_t ctl = scr + kChunk;
+  static constexpr size_t cum = ctl + ((sizeof(ElimCtl) + 15) & ~size_t(15));
+  static constexpr size_t bytes(bool paged) {
+    return cum + (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
+  }
+};
+
+template <int D, int BITS, int G, class Layout>
+__device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uint8_t *smem,
+                          const uint32_t *cum) {
+  using C = Cfg<D, BITS, G>;
+  using S = ElimSmem<D>;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t V = a.V;
+  const uint32_t n_code = (V + C::VC - 1) / C::VC;
+  const uint8_t *table = a.in + kHeader;
+  const uint64_t base = ctl->base, limit = ctl->limit;
+  uint8_t *stage = smem + warp * S::WBUF;
+  uint8_t *mbuf = smem + S::meta + warp * S::MBLK;
+  uint8_t *chunk = smem + S::chunk;
+  uint8_t *scr = smem + S::scr;
+  bool use_tma = false;
+  if constexpr (!kIsPaged<Layout>) use_tma = lay.tma != 0;
+  bool stage_busy = false;
+  uint32_t zphase = 0, mphase = 0;
+  auto len_of = [&](uint32_t c) { return min(uint32_t(C::VC), V - c * C::VC) * C::CB; };
+  // meta of vectors v0 .. v0 + nv - 1 (one meta chunk): raw in the stream or
+  // expanded by meta_expand_kernel; null for an entry out of bounds
+  auto meta_src = [&](uint32_t v0, uint32_t nv) -> const uint8_t * {
+    const uint32_t s = v0 / C::VM;
+    const uint64_t e = ld_u64(table + 8 * (uint64_t(n_code) + s));
+    const uint32_t mlen = min(uint32_t(C::VM), V - s * C::VM) * C::MB;
+    const uint64_t off = (e >> 16) << 4;
+    if (uint32_t(e & 0xFFFFu) != mlen) return a.ws_meta + uint64_t(s) * kChunk + (v0 - s * C::VM) * C::MB;
+    const uint64_t at = off + uint64_t(v0 - s * C::VM) * C::MB;
+    return base + at + round16(nv * C::MB) <= limit ? a.in + base + at : nullptr;
+  };
+#pragma unroll 1
+  for (uint64_t j0 = 0; uint64_t(blockIdx.x) + j0 * gridDim.x < n_code; j0 += kElimThreads) {
+    if (tid == 0) ctl->nlist = 0;
+    __syncthreads();
+    const uint64_t cc = uint64_t(blockIdx.x) + (j0 + tid) * gridDim.x;
+    if (cc < n_code && uint32_t(ld_u64(table + 8 * cc) & 0xFFFFu) != len_of(uint32_t(cc)))
+      ctl->list[atomicAdd(&ctl->nlist, 1u)] = uint32_t(cc);
+    __syncthreads();
+    const uint32_t nl = ctl->nlist;
+#pragma unroll 1
+    for (uint32_t i = 0; i < nl; ++i) {
+      const uint32_t c = ctl->list[i];
+      const uint64_t e = ld_u64(table + 8 * uint64_t(c)), off = (e >> 16) << 4;
+      const uint32_t size = uint32_t(e & 0xFFFFu), len = len_of(c);
+      const bool good = len == uint32_t(kChunk) && size >= kBitmap && size < len &&
+                        base + off + round16(size) <= limit;
+      if (tid == 0) {
+        if (good) {
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&ctl->zbar, uint32_t(round16(size)));
+          bulk_g2s(chunk, a.in + base + off, uint32_t(round16(size)), &ctl->zbar);
+        } else {
+          set_status(a.status, KVC_ERR_CORRUPT);
+        }
+      }
+      if (!good) continue;  // uniform over the CTA
+      if (!mbar_wait(&ctl->zbar, zphase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+      zphase ^= 1;
+      const bool ok = ze_decode<kElimThreads>(chunk, scr, ctl->red, size);
+      if (!ok) {
+        if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
+        __syncthreads();
+        continue;
+      }
+      const uint32_t nvec = len / C::CB;
+#pragma unroll 1
+      for (uint32_t b = warp; b * 32 < nvec; b += kElimWarps) {
+        const uint32_t v0 = c * C::VC + b * 32, nv = min(32u, nvec - b * 32);
+        const uint8_t *msrc = meta_src(v0, nv);
+        if (!msrc) {
+          if (lane == 0) set_status(a.status, KVC_ERR_CORRUPT);
+          continue;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t mbytes = uint32_t(round16(nv * C::MB));
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&ctl->mbar[warp], mbytes);
+          bulk_g2s(mbuf, msrc, mbytes, &ctl->mbar[warp]);
+        }
+        if (!mbar_wait(&ctl->mbar[warp], mphase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+        mphase ^= 1;
+        uint32_t out[D / 2];
+        const bool act = uint32_t(lane) < nv;
+        if (act)
+          Dec<D, BITS, G>::vector(chunk + (b * 32 + lane) * C::CB, mbuf + lane * C::MB, ctl->mask, out);
+        if constexpr (!kIsPaged<Layout>) {
+          if (use_tma) {
+            store_block_tma<D>(lay, out, v0, stage, stage_busy);
+            continue;
+          }
+        }
+        uint8_t *dst = nullptr;
+        if (act) {
+          bool vok;
+          dst = vec_addr(lay, cum, v0 + lane, vok);
+          if (!vok) {
+            set_status(a.status, KVC_ERR_CORRUPT);
+            dst = nullptr;
+          }
+        }
+        __syncwarp();  // the previous block's scatter has read the buffer
+        stage_row<D>(out, stage);
+        __syncwarp();
+        scatter_rows<D>(stage, dst);
+      }
+      fence_proxy_async_smem();
+      __syncthreads();  // the chunk buffer is reused
+    }
+  }
+  if (lane == 0) bulk_wait_all<0>();
+}
+
+template <int D, class Layout>
+__global__ void __launch_bounds__(kElimThreads, 1)
+    elim_decode_kernel(const __grid_constant__ DecArgs a, const __grid_constant__ Layout lay) {
+  using S = ElimSmem<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  ElimCtl *ctl = reinterpret_cast<ElimCtl *>(smem + S::ctl);
+  uint32_t *s_cum = reinterpret_cast<uint32_t *>(smem + S::cum);
+  const int tid = threadIdx.x;
+  if (a.in_bytes < kHeader || a.in[11] != 1) return;  // no code chunk uses elimination
+  if (tid < kElimWarps) {
+    mbar_init(&ctl->mbar[tid], 1);
+    mbar_fence_init();
+  }
+  if (tid == 0) {
+    mbar_init(&ctl->zbar, 1);
+    mbar_fence_init();
+    const StreamHdr h = parse_header<D>(a);
+    ctl->ok = h.ok;
+    ctl->bits = h.bits;
+    ctl->group = h.group;
+    ctl->base = h.data_base;
+    ctl->limit = min(a.in_bytes, h.stream_bytes);
+    if (h.ok) sign_masks(h.seed, D, ctl->mask);
+  }
+  if constexpr (kIsPaged<Layout>) {
+    for (uint32_t r = tid; r <= lay.n_req; r += blockDim.x) s_cum[r] = lay.cum[r];
+  }
+  __syncthreads();
+  if (!ctl->ok) return;  // decode_kernel reports the header
+  const uint32_t bits = ctl->bits, group = ctl->group;
+  if constexpr (D == 128) {
+    if (bits == 4 && group == 128)
+      elim_body<128, 4, 128>(a, lay, ctl, smem, s_cum);
+    else if (bits == 4 && group == 64)
+      elim_body<128, 4, 64>(a, lay, ctl, smem, s_cum);
+    else if (bits == 4 && group == 32)
+      elim_body<128, 4, 32>(a, lay, ctl, smem, s_cum);
+    else if (bits == 2 && group == 128)
+      elim_body<128, 2, 128>(a, lay, ctl, smem, s_cum);
+    else if (bits == 2 && group == 64)
+      elim_body<128, 2, 64>(a, lay, ctl, smem, s_cum);
+    else
+      elim_body<128, 2, 32>(a, lay, ctl, smem, s_cum);
+  } else {
+    if (bits == 4 && group == 64)
+      elim_body<64, 4, 64>(a, lay, ctl, smem, s_cum);
+    else if (bits == 4 && group == 32)
+      elim_body<64, 4, 32>(a, lay, ctl, smem, s_cum);
+    else if (bits == 2 && group == 64)
+      elim_body<64, 2, 64>(a, lay, ctl, smem, s_cum);
+    else
+      elim_body<64, 2, 32>(a, lay, ctl, smem, s_cum);
+  }
 }
 
 }  // namespace kvc

@@ -329,8 +329,10 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       const unsigned long long old = atomicAdd(a.code_nnz + c, (1ull << 32) | cs);
       const uint32_t blocks = (min(uint32_t(C::VC), V - c * C::VC) + 31) / 32;
       if (uint32_t(old >> 32) + 1 == blocks && blocks * 32 == uint32_t(C::VC) &&
-          kBitmap + uint32_t(old) + cs < uint32_t(kChunk))
+          kBitmap + uint32_t(old) + cs < uint32_t(kChunk)) {
         atomicOr(a.flags, 1u);
+        atomicMax(a.first_inv, ~c);
+      }
       atomicAdd(a.meta_nnz + blk * 32 / C::VM, ms);
     }
   };

@@ -71,13 +71,16 @@ __device__ __forceinline__ uint32_t meta_stored_size(const FinArgs &a, uint32_t 
   return (len == uint32_t(kChunk) && kBitmap + n < uint32_t(kChunk)) ? kBitmap + n : len;
 }
 
+// Header (reading R12); byte 11 bit 0: some code chunk uses zero-byte
+// elimination (`code_elim`).
 template <class Layout>
-__device__ void fin_header(const FinArgs &a, const uint32_t *cum, uint64_t stream_bytes) {
+__device__ void fin_header(const FinArgs &a, const uint32_t *cum, uint64_t stream_bytes,
+                           uint32_t code_elim) {
   uint8_t *o = a.out;
   st_u32(o + 0, kMagic);
   st_u16(o + 4, 1);
   st_u16(o + 6, kHeader);
-  st_u32(o + 8, a.bits | (a.k << 8) | (a.origin << 16));
+  st_u32(o + 8, a.bits | (a.k << 8) | (a.origin << 16) | (code_elim << 24));
   st_u32(o + 12, a.group);
   st_u32(o + 16, a.layers);
   st_u32(o + 20, 2);
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(kFinThreads, 4)
     uint64_t part = 0;
     for (uint32_t s = tid; s < a.n_meta; s += NT) part += round16(meta_stored_size(a, s));
     const uint64_t total_meta = block_sum64<NT>(part, ctl->red);
-    if (tid == 0) fin_header<Layout>(a, s_cum, a.data_base + total_code + total_meta);
+    if (tid == 0) fin_header<Layout>(a, s_cum, a.data_base + total_code + total_meta, shrank ? 1u : 0u);
   }
   if (tid == 0) bulk_wait_all<0>();
 }
@@ -227,7 +230,8 @@ __global__ void __launch_bounds__(kFinThreads, 4)
 // the meta chunks. Chunk c (raw bytes at data_base + c * 16 KB, destination
 // data_base + code_off[c] <= that) may overwrite only raw bytes of chunks
 // j <= c whose 16 KB slot overlaps its destination; it waits for their read
-// flags.
+// flags. Chunks before the first shrinking chunk c0 stay where they are
+// (every destination lies at or above c0's slot).
 __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_constant__ FinArgs a) {
   constexpr int NT = kFinThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -242,14 +246,18 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
   }
   __syncthreads();
   if (!(ctl->flag & 1u)) return;
+  // Chunks before the first shrinking one keep their place: tickets start
+  // there. The next ticket is taken while the current chunk moves.
+  const uint32_t c0 = ~*reinterpret_cast<volatile uint32_t *>(a.first_inv);
   uint32_t phase = 0;
+  if (tid == 0) ctl->tick = atomicAdd(a.ticket, 1u);
 #pragma unroll 1
   while (true) {
-    if (tid == 0) ctl->tick = atomicAdd(a.ticket, 1u);
     named_bar_sync(1, NT);
-    const uint32_t c = ctl->tick;
+    const uint32_t c = c0 + ctl->tick;
     named_bar_sync(1, NT);
     if (c >= a.n_code) break;
+    if (tid == 0) ctl->tick = atomicAdd(a.ticket, 1u);
     const uint32_t len = code_len(a, c), size = a.code_size[c];
     const uint64_t src = uint64_t(c) * kChunk, dst = a.code_off[c];
     if (dst != src || size != len) {
@@ -302,7 +310,7 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
   // every code chunk has been read (their destinations overlap old sources)
   if (tid == 0) {
     const uint64_t t0 = globaltimer();
-    for (uint32_t it = 0; *reinterpret_cast<volatile uint32_t *>(a.ticket + 1) < a.n_code; ++it) {
+    for (uint32_t it = 0; *reinterpret_cast<volatile uint32_t *>(a.ticket + 1) < a.n_code - c0; ++it) {
       if (spin_expired(it, t0, a.status)) {
         set_status(a.status, KVC_ERR_TIMEOUT);
         break;

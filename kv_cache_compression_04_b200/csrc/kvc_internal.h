@@ -31,7 +31,8 @@ constexpr uint32_t kNoTile = 0xFFFFFFFFu;
 
 // Workspace of kvc_compress, in this order (each part 256-byte aligned):
 //   control   status word, flags word (bit 0: some code chunk shrank),
-//             compaction ticket, compaction read count
+//             compaction ticket, compaction read count, ~(first shrinking
+//             code chunk)
 //   meta_nnz  u32 per meta chunk: shuffled-byte nonzero count (accumulated)
 //   code_nnz  u64 per code chunk: the same count (low half) and the number
 //             of 32-vector blocks accumulated so far (high half)
@@ -137,6 +138,7 @@ struct EncArgs {
   uint64_t data_base;
   uint32_t *status;
   uint32_t *flags;     // bit 0: some code chunk shrinks
+  uint32_t *first_inv; // max over shrinking code chunks c of ~c (0: none)
   unsigned long long *code_nnz;
   uint32_t *meta_nnz;
   uint8_t *ws_meta;
@@ -154,6 +156,7 @@ struct FinArgs {
   uint64_t *out_bytes_dev;
   uint32_t *status;
   uint32_t *flags;
+  uint32_t *first_inv;  // ~(first shrinking code chunk), 0 if none
   uint32_t *ticket;
   const unsigned long long *code_nnz;
   const uint32_t *meta_nnz;

@@ -58,6 +58,18 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
   mk<<<mgrid, kMetaThreads, meta_smem_bytes(), st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // code chunks that used zero-byte elimination (returns at once if none);
+  // 256 chunks per CTA and scan step, for the largest code region (4-bit)
+  auto ek = elim_decode_kernel<D, Layout>;
+  const size_t esmem = ElimSmem<D>::bytes(kIsPaged<Layout>);
+  struct ElimTag {};
+  e = prepare<ElimTag>(ek, esmem);
+  if (e != cudaSuccess) return e;
+  const uint64_t egrid_want = (tiles + kElimThreads - 1) / kElimThreads;
+  const int egrid = egrid_want == 0 ? 1 : int(egrid_want < uint64_t(sms) ? egrid_want : uint64_t(sms));
+  ek<<<egrid, kElimThreads, esmem, st>>>(a, lay);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   k<<<grid, kDecThreads, smem, st>>>(a, lay);
   return cudaGetLastError();
 }

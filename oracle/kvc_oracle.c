@@ -388,7 +388,8 @@ int orc_lossless_decode_chunk(const uint8_t *in, uint32_t size, uint32_t len,
 /* ========================================================================== */
 /* Stream layout. Reading R12 (self-describing stream, little-endian):        */
 /*   [0,64)    header: u32 magic "KVC1", u16 version 1, u16 header bytes 64,  */
-/*             u8 bits, u8 k, u8 origin (0 dense, 1 paged), u8 0, u32 group,  */
+/*             u8 bits, u8 k, u8 origin (0 dense, 1 paged), u8 flags (bit 0: */
+/*             some code chunk uses zero-byte elimination), u32 group,        */
 /*             u32 layers, u32 kv (=2), u32 kv_heads, u32 head_dim,           */
 /*             u64 tokens (sum over requests), u64 sign_seed,                 */
 /*             u32 n_requests, u32 n_chunks, u64 stream_bytes;                */
@@ -627,6 +628,16 @@ int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
     memcpy(out + lay.data_base + off, store + where[i], all_sizes[i]);
     off += padded;
   }
+  /* header flags, bit 0: some code chunk uses zero-byte elimination (a
+     decoder may use it to skip looking for such chunks) */
+  for (i = 0; i < lay.n_code; i++) {
+    uint64_t nv = lay.V - i * lay.vec_per_code;
+    if (nv > lay.vec_per_code) nv = lay.vec_per_code;
+    if (all_sizes[orc_code_chunk_index(&lay, i)] != nv * lay.code_bytes) {
+      out[11] = 1;
+      break;
+    }
+  }
   free(seg);
   free(store);
   free(all_sizes);
@@ -671,6 +682,16 @@ int orc_decompress(const uint8_t *stream, uint64_t stream_bytes,
     if (off != expect_off || sz > ORC_CHUNK || lay.data_base + off + round16(sz) > total)
       return ORC_ERR_CORRUPT;
     expect_off = off + round16(sz);
+  }
+  /* header flags: only bit 0, which must be set if a code chunk uses
+     zero-byte elimination */
+  if (stream[11] > 1) return ORC_ERR_CORRUPT;
+  for (s = 0; s < lay.n_code && !stream[11]; s++) {
+    uint64_t nv = lay.V - s * lay.vec_per_code;
+    if (nv > lay.vec_per_code) nv = lay.vec_per_code;
+    if ((get64(stream + ORC_HEADER + 8 * orc_code_chunk_index(&lay, s)) & 0xFFFFu) !=
+        nv * lay.code_bytes)
+      return ORC_ERR_CORRUPT;
   }
   vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
   seg = (uint8_t *)malloc((size_t)(lay.code_per_seg + 1) * ORC_CHUNK);

@@ -80,7 +80,7 @@ def test_good_stream_decodes():
 @pytest.mark.parametrize("field,offset,value", [
     ("magic", 0, 0x4A), ("version", 4, 2), ("bits", 8, 3), ("k", 9, 4), ("group", 12, 48),
     ("layers", 16, 3), ("kv", 20, 3), ("heads", 24, 5), ("head_dim", 28, 64),
-    ("tokens", 32, 0x11), ("n_chunks", 52, 0x77), ("stream_bytes", 61, 0x7F)])
+    ("tokens", 32, 0x11), ("n_chunks", 52, 0x77), ("stream_bytes", 61, 0x7F), ("flags", 11, 2)])
 def test_corrupt_header(field, offset, value):
     _, s = _good_stream()
     bad = s.copy()
@@ -121,6 +121,22 @@ def test_corrupt_zero_byte_bitmap():
     bad[base + offs[i]] ^= 0x01                  # bitmap popcount no longer matches
     st, guard = _decode_guarded(bad)
     assert st == kvc.KVC_ERR_CORRUPT and guard
+
+
+def test_code_elimination_flag_cleared():
+    """Code chunks that use zero-byte elimination but a header that does not
+    announce them: CORRUPT, like the oracle decoder."""
+    kv = _kv(T=2000)
+    kv[:, :, :, :1000] = 0                       # mode-1 code chunks
+    st, s, _, _ = gpu_compress(kvc.dense_desc(kv.cuda()), 4, 128)
+    assert st == kvc.KVC_OK and s[11] == 1
+    bad = s.copy()
+    bad[11] = 0
+    st, guard = _decode_guarded(bad)
+    assert st == kvc.KVC_ERR_CORRUPT and guard
+    od = oracle.StreamDesc(4, 128, 128, 2, 2, [2000])
+    assert oracle.decompress(bad, od)[0] == oracle.CORRUPT
+    assert oracle.decompress(s, od)[0] == oracle.OK
 
 
 def test_shape_mismatch():

@@ -48,6 +48,24 @@ def test_header_golden():
     assert not s[64 + 8 * 5 + 4:112].any()                      # zero padding
 
 
+@pytest.mark.parametrize("zero_chunk", [False, True])
+def test_header_flag_code_elimination(zero_chunk):
+    """Header byte 11, bit 0 says whether some code chunk uses zero-byte
+    elimination: an all-zero tensor's 16 KB code chunks are all-zero codes
+    (2048-byte bitmap only); random data gives none."""
+    w, d, x = tiny_desc_and_vectors()
+    if zero_chunk:
+        x = x.copy()
+        x[:256] = 0                      # the first code chunk's 256 vectors
+    st, s = oracle.compress(d, x)
+    assert st == oracle.OK
+    sizes = np.frombuffer(bytes(s[64:64 + 8 * 5]), "<u8") & 0xFFFF
+    assert (sizes[:4] < 16384).any() == zero_chunk
+    assert s[11] == (1 if zero_chunk else 0)
+    st, y = oracle.decompress(s, d)
+    assert st == oracle.OK
+
+
 @pytest.mark.parametrize("name,n_code,n_meta", [("tiny", 4, 1), ("llama8b", 8192, 512),
                                                 ("qwen7b", 14336, 7168)])
 def test_layout_counts(name, n_code, n_meta):
@@ -136,6 +154,11 @@ def test_corrupt_streams():
     bad = s.copy()
     bad[64 + 8 + 2] ^= 0x01                                           # chunk 1 offset
     assert oracle.decompress(bad, d)[0] == oracle.CORRUPT
+    bad = s.copy()
+    bad[11] = 2                                                       # unknown flag bit
+    assert oracle.decompress(bad, d)[0] == oracle.CORRUPT
+    bad[11] = 1                   # announced elimination that no chunk uses: accepted
+    assert oracle.decompress(bad, d)[0] == oracle.OK
 
 
 def test_mode1_chunks_roundtrip():
@@ -150,6 +173,10 @@ def test_mode1_chunks_roundtrip():
     lay = d.layout()
     sizes = [_u(s, 64 + 8 * i, 8) & 0xFFFF for i in range(lay.n_chunks)]
     assert min(sizes[:2]) < 16384                                     # mode-1 chunks
+    assert s[11] == 1
+    bad = s.copy()
+    bad[11] = 0                                  # not announced: corrupt
+    assert oracle.decompress(bad, d)[0] == oracle.CORRUPT
     st, xh = oracle.decompress(s, d)
     _, codes, meta = oracle.quantize_vectors(x, w.bits, w.group, 0)
     ref = oracle.dequantize_vectors(codes, meta, 128, w.bits, w.group, 0)
