@@ -375,7 +375,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
 }
 
 template <int D, class Layout>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads)
     decode_kernel(const __grid_constant__ DecArgs a, const __grid_constant__ Layout lay) {
   constexpr bool kPaged = kIsPaged<Layout>;
   using S = DecSmem<D>;
