@@ -15,6 +15,8 @@ time saved at 100 and 400 Gbit/s, SM clocks sampled during the timed region.
 Multi-GPU (torchrun): every rank compresses its own KV cache (weak scaling);
 the only collectives are a barrier and a max over ranks of the timings.
 `--impl reference` times the CPU oracle instead (rank 0 only).
+`--sweep` runs the message-size sweep instead (1 GPU): Llama-3-8B-shaped KV
+of 1 MiB .. 4 GiB, 4-bit g128 and 2-bit g32, one JSON line per point.
 """
 from __future__ import annotations
 
@@ -283,6 +285,82 @@ def job_gbs(raw_bytes_per_rank: int, world: int, ms: float) -> float:
 
 
 # ------------------------------------------------------------------ main --
+def run_sweep(args):
+    """Message-size sweep: [32, 2, 8, T, 128] with T = 8 * 2^i tokens (1 MiB ..
+    4 GiB), 4-bit g128 and 2-bit g32. Each step times one compress and one
+    decompress with CUDA events after flushing L2 (a 256 MiB write outside the
+    events), so small sizes are not served from cache."""
+    import torch
+    import kv_cache_compression_04_b200 as kvc
+    from kv_cache_compression_04_b200 import build, synth
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = kvc._stream_ptr(stream)
+    for bits in (4, 2):
+        for i in range(13):
+            w = synth.workload(f"sweep-{i}-{bits}")
+            kv = synth.dense_kv(w, device=dev)
+            desc = kvc.dense_desc(kv)
+            codec = kvc.Codec(w.bits, w.group, w.sign_seed)
+            out, ws, nb = codec.buffers(desc, dev)
+            o = torch.empty_like(kv)
+            odesc = kvc.dense_desc(o)
+            dws = torch.empty(kvc.kvc_decompress_workspace_bytes(odesc), dtype=torch.uint8,
+                              device=dev)
+
+            def enc():
+                assert kvc.kvc_compress(desc, codec.params, out.data_ptr(), out.numel(),
+                                        nb.data_ptr(), ws.data_ptr(), ws.numel(), sp) == kvc.KVC_OK
+
+            enc()
+            assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+            n = int(nb.item())
+
+            def dec():
+                assert kvc.kvc_decompress(out.data_ptr(), n, odesc, dws.data_ptr(), dws.numel(),
+                                          sp) == kvc.KVC_OK
+
+            dec()
+            assert kvc.kvc_stream_status(dws.data_ptr(), sp) == kvc.KVC_OK
+            steps = max(5, min(100, int(4e9 / w.raw_bytes)))
+            te, td = [], []
+            for it in range(args.warmup + steps):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                e[0].record(stream)
+                enc()
+                e[1].record(stream)
+                dec()
+                e[2].record(stream)
+                torch.cuda.synchronize(dev)
+                if it >= args.warmup:
+                    te.append(e[0].elapsed_time(e[1]))
+                    td.append(e[1].elapsed_time(e[2]))
+            assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+            enc_ms, dec_ms = statistics.median(te), statistics.median(td)
+            raw = w.raw_bytes
+            saved_bits = 8 * (raw - n)
+            t_codec = (enc_ms + dec_ms) * 1e-3
+            print(json.dumps({
+                "sweep": w.name, "bits": w.bits, "group": w.group, "raw_bytes": raw,
+                "stream_bytes": n, "ratio": round(raw / n, 4), "steps": steps,
+                "encode_us": round(enc_ms * 1e3, 2), "decode_us": round(dec_ms * 1e3, 2),
+                "encode_GBps": round(raw / (enc_ms * 1e-3) / 1e9, 1),
+                "decode_GBps": round(raw / (dec_ms * 1e-3) / 1e9, 1),
+                "roundtrip_GBps": round(raw / t_codec / 1e9, 1),
+                "break_even_gbit_s": round(saved_bits / t_codec / 1e9, 1),
+                "net_gain_ms": {"100Gbit": round((saved_bits / 100e9 - t_codec) * 1e3, 4),
+                                "400Gbit": round((saved_bits / 400e9 - t_codec) * 1e3, 4)},
+                "l2": "flushed before every step (256 MiB write)", "timing": "median of steps"}),
+                flush=True)
+            del kv, out, ws, nb, o, dws
+            torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -292,7 +370,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--sweep", action="store_true")
     args = ap.parse_args()
+    if args.sweep:
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     assert args.warmup >= 3, "at least 3 warm-up steps"

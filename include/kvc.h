@@ -161,7 +161,10 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params,
  * request count and per-request token counts. The receiver's layout (dense or
  * paged, page table, strides) may differ from the sender's. A mismatch or any
  * inconsistency in the stream sets KVC_ERR_CORRUPT; reads stay inside
- * [in, in + in_bytes). Slots outside the described tokens are not written. */
+ * [in, in + in_bytes). Slots outside the described tokens are not written.
+ * The call launches three kernels on `stream` (meta chunk expansion; decode
+ * of the code chunks that used zero-byte elimination, which returns at once
+ * unless the header flags some; decode of the raw code chunks). */
 kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *out,
                           void *workspace, size_t workspace_bytes,
                           kvc_stream_t stream);

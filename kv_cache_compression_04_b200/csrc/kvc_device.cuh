@@ -29,6 +29,15 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
+// Programmatic dependent launch: a kernel launched with launch_after() is
+// set up while the previous kernel on the stream runs; it calls
+// grid_dependency_wait() before anything else, which returns once that
+// kernel has completed and its writes are visible. (No kernel triggers its
+// dependents early: measured slower, their CTAs then wait on busy SMs.)
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // First error of a call wins.
 __device__ __forceinline__ void set_status(uint32_t *status, uint32_t code) {
   atomicCAS(status, 0u, code);

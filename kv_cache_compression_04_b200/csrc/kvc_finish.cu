@@ -16,8 +16,7 @@ cudaError_t launch_fin(const FinArgs &a, const Layout &lay, int sms, cudaStream_
   // one meta chunk per CTA where possible (several CTAs share an SM)
   const uint32_t want = a.n_meta > 1 ? a.n_meta : 1u, cap = 4u * uint32_t(sms);
   const int grid = int(want < cap ? want : cap);
-  fk<<<grid, kFinThreads, fsmem, st>>>(a, lay);
-  e = cudaGetLastError();
+  e = launch_after(fk, grid, kFinThreads, fsmem, st, a, lay);
   if (e != cudaSuccess || a.n_code == 0) return e;
   // Returns at once unless a code chunk shrank (flag set by the encode kernel).
   auto ck = compact_kernel;
@@ -26,8 +25,7 @@ cudaError_t launch_fin(const FinArgs &a, const Layout &lay, int sms, cudaStream_
   e = prepare<CompactTag>(ck, csmem);
   if (e != cudaSuccess) return e;
   const int cgrid = int(a.n_code < cap ? a.n_code : cap);
-  ck<<<cgrid, kFinThreads, csmem, st>>>(a);
-  return cudaGetLastError();
+  return launch_after(ck, cgrid, kFinThreads, csmem, st, a);
 }
 
 }  // namespace

@@ -107,6 +107,7 @@ __device__ void fin_header(const FinArgs &a, const uint32_t *cum, uint64_t strea
 template <class Layout>
 __global__ void __launch_bounds__(kFinThreads, 4)
     finish_kernel(const __grid_constant__ FinArgs a, const __grid_constant__ Layout lay) {
+  grid_dependency_wait();  // the encode kernel's counts and meta
   constexpr int NT = kFinThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *scr = smem + 2 * kChunk;  // buffers 0 and 1 below it
@@ -233,6 +234,7 @@ __global__ void __launch_bounds__(kFinThreads, 4)
 // flags. Chunks before the first shrinking chunk c0 stay where they are
 // (every destination lies at or above c0's slot).
 __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_constant__ FinArgs a) {
+  grid_dependency_wait();  // finish_kernel's sizes, offsets and parked meta
   constexpr int NT = kFinThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *buf = smem;

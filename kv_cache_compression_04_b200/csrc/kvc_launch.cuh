@@ -2,10 +2,30 @@
 #pragma once
 
 #include <atomic>
+#include <utility>
 
 #include "kvc_decode.cuh"
 
 namespace kvc {
+
+// Launches kernel k so that it may begin while the previous kernel on the
+// stream finishes (programmatic dependent launch); k must start with
+// grid_dependency_wait().
+template <class... KArgs, class... Args>
+inline cudaError_t launch_after(void (*k)(KArgs...), int grid, int threads, size_t smem,
+                                cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(unsigned(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
 
 // Opt each instantiation into large dynamic shared memory once per device.
 // `Tag` makes the flag per kernel instantiation (kernels share a pointer type).
@@ -67,11 +87,9 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
   if (e != cudaSuccess) return e;
   const uint64_t egrid_want = (tiles + kElimThreads - 1) / kElimThreads;
   const int egrid = egrid_want == 0 ? 1 : int(egrid_want < uint64_t(sms) ? egrid_want : uint64_t(sms));
-  ek<<<egrid, kElimThreads, esmem, st>>>(a, lay);
-  e = cudaGetLastError();
+  e = launch_after(ek, egrid, kElimThreads, esmem, st, a, lay);
   if (e != cudaSuccess) return e;
-  k<<<grid, kDecThreads, smem, st>>>(a, lay);
-  return cudaGetLastError();
+  return launch_after(k, grid, kDecThreads, smem, st, a, lay);
 }
 
 template <int D, class Layout>
