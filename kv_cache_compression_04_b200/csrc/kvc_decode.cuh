@@ -377,7 +377,6 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
 template <int D, class Layout>
 __global__ void __launch_bounds__(kDecThreads)
     decode_kernel(const __grid_constant__ DecArgs a, const __grid_constant__ Layout lay) {
-  grid_dependency_wait();  // the meta pre-pass and elim_decode_kernel
   constexpr bool kPaged = kIsPaged<Layout>;
   using S = DecSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -710,7 +709,6 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
 template <int D, class Layout>
 __global__ void __launch_bounds__(kElimThreads, 1)
     elim_decode_kernel(const __grid_constant__ DecArgs a, const __grid_constant__ Layout lay) {
-  grid_dependency_wait();  // the meta pre-pass
   using S = ElimSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   ElimCtl *ctl = reinterpret_cast<ElimCtl *>(smem + S::ctl);

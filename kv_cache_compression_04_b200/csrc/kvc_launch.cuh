@@ -87,9 +87,13 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
   if (e != cudaSuccess) return e;
   const uint64_t egrid_want = (tiles + kElimThreads - 1) / kElimThreads;
   const int egrid = egrid_want == 0 ? 1 : int(egrid_want < uint64_t(sms) ? egrid_want : uint64_t(sms));
-  e = launch_after(ek, egrid, kElimThreads, esmem, st, a, lay);
+  // (plain launches: dependent launches measured slower on this side when
+  // compress and decompress calls alternate on a stream)
+  ek<<<egrid, kElimThreads, esmem, st>>>(a, lay);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_after(k, grid, kDecThreads, smem, st, a, lay);
+  k<<<grid, kDecThreads, smem, st>>>(a, lay);
+  return cudaGetLastError();
 }
 
 template <int D, class Layout>
