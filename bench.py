@@ -370,6 +370,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--unfused-steps", type=int, default=20)
     ap.add_argument("--sweep", action="store_true")
     args = ap.parse_args()
     if args.sweep:
@@ -488,6 +489,37 @@ def main():
                "ms_per_step": round(e2e_ms, 3)}
         assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
 
+    # ------------------------------------- unfused baseline (fusion gain) --
+    # The same compress call as two kernels with the fp32 transformed tensor
+    # in HBM between them (kvc_compress_unfused; identical stream), timed the
+    # same way, outside the timed region above.
+    unfused = None
+    if args.unfused_steps > 0:
+        uws = torch.empty(kvc.kvc_unfused_workspace_bytes(desc, codec.params), dtype=torch.uint8,
+                          device=dev)
+
+        def enc_unfused():
+            st = kvc.kvc_compress_unfused(desc, codec.params, out.data_ptr(), out.numel(),
+                                          nb.data_ptr(), uws.data_ptr(), uws.numel(), sp)
+            assert st == kvc.KVC_OK, kvc.STATUS[st]
+
+        for _ in range(3):
+            enc_unfused()
+        u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        u0.record(stream)
+        for _ in range(args.unfused_steps):
+            enc_unfused()
+        u1.record(stream)
+        torch.cuda.synchronize(dev)
+        assert kvc.kvc_stream_status(uws.data_ptr(), sp) == kvc.KVC_OK
+        assert int(nb.item()) == nbytes
+        u_ms = max_over_ranks([u0.elapsed_time(u1) / args.unfused_steps], dist, dev)[0]
+        unfused = {"encode_ms": round(u_ms, 4), "fusion_speedup": round(u_ms / enc_avg, 3),
+                   "intermediate_bytes": int(w.vectors) * w.head_dim * 4,
+                   "what": "kvc_compress_unfused: transform kernel -> fp32 tensor in HBM -> "
+                           "quantize kernel, same finishing kernels, same stream"}
+        del uws
+
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -534,6 +566,8 @@ def main():
     }
     if e2e:
         line["e2e"] = e2e
+    if unfused:
+        line["unfused_baseline"] = unfused
     if world == 1 and args.cpu_budget > 0:
         b, s, n = oracle_sample(args.workload, args.cpu_budget)
         line["cpu_baseline"] = {"value": round(b / s / 1e9, 6), "unit": "GB/s", "cores": 1,

@@ -212,6 +212,21 @@ kvc_status kvc_compress_noalloc(const kvc_kv_desc *kv, const kvc_params *params,
                                 uint64_t *out_bytes_dev, uint32_t *status_dev,
                                 kvc_stream_t stream);
 
+/* Unfused baseline, for measurement only ("Beyond Compression Ratio:
+ * High-Throughput KV Compression for Disaggregated LLM Serving", Abstract:
+ * the fused transform + quantization kernel is compared against separate
+ * kernels). kvc_compress_unfused writes exactly the stream kvc_compress
+ * writes, with the same arguments and errors, but runs the transform (signs
+ * and Walsh-Hadamard) and the quantization as two kernels with the
+ * transformed vectors in HBM between them (fp32, 4 * head_dim bytes per
+ * vector, at the end of the workspace). workspace_bytes must be at least
+ * kvc_unfused_workspace_bytes(kv, params) (0 for an invalid description). */
+size_t kvc_unfused_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params);
+kvc_status kvc_compress_unfused(const kvc_kv_desc *kv, const kvc_params *params,
+                                void *out, size_t out_capacity,
+                                uint64_t *out_bytes_dev, void *workspace,
+                                size_t workspace_bytes, kvc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

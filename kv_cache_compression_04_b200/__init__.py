@@ -27,7 +27,8 @@ STATUS = ["KVC_OK", "KVC_ERR_INVALID_ARG", "KVC_ERR_UNSUPPORTED", "KVC_ERR_CAPAC
 # Every symbol include/kvc.h declares.
 EXPORTS = ["kvc_max_compressed_bytes", "kvc_workspace_bytes", "kvc_compress",
            "kvc_decompress", "kvc_stream_status", "kvc_status_string", "kvc_compress_noalloc",
-           "kvc_decompress_workspace_bytes"]
+           "kvc_decompress_workspace_bytes", "kvc_unfused_workspace_bytes",
+           "kvc_compress_unfused"]
 
 
 class KvcError(RuntimeError):
@@ -83,6 +84,11 @@ def lib() -> C.CDLL:
         L.kvc_compress_noalloc.restype = C.c_int
         L.kvc_compress_noalloc.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p,
                                            C.c_void_p, C.c_void_p]
+        L.kvc_unfused_workspace_bytes.restype = C.c_size_t
+        L.kvc_unfused_workspace_bytes.argtypes = [D, P]
+        L.kvc_compress_unfused.restype = C.c_int
+        L.kvc_compress_unfused.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p,
+                                           C.c_size_t, C.c_void_p]
         _lib = L
     return _lib
 
@@ -104,6 +110,16 @@ def kvc_compress(desc, params, out_ptr, out_capacity, out_bytes_dev_ptr, ws_ptr,
                  stream) -> int:
     return lib().kvc_compress(C.byref(desc), C.byref(params), out_ptr, out_capacity,
                               out_bytes_dev_ptr, ws_ptr, ws_bytes, stream)
+
+
+def kvc_unfused_workspace_bytes(desc: kvc_kv_desc, params: kvc_params) -> int:
+    return lib().kvc_unfused_workspace_bytes(C.byref(desc), C.byref(params))
+
+
+def kvc_compress_unfused(desc, params, out_ptr, out_capacity, out_bytes_dev_ptr, ws_ptr, ws_bytes,
+                         stream) -> int:
+    return lib().kvc_compress_unfused(C.byref(desc), C.byref(params), out_ptr, out_capacity,
+                                      out_bytes_dev_ptr, ws_ptr, ws_bytes, stream)
 
 
 def kvc_compress_noalloc(desc, params, out_ptr, out_capacity, out_bytes_dev_ptr, status_dev_ptr,

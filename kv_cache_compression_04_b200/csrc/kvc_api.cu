@@ -193,15 +193,26 @@ size_t kvc_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params) {
   return size_t(s.ws_bytes);
 }
 
-kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *out,
-                        size_t out_capacity, uint64_t *out_bytes_dev, void *workspace,
-                        size_t workspace_bytes, kvc_stream_t stream) {
+size_t kvc_unfused_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params) {
+  Shape s;
+  if (!params || describe(kv, params, s) != KVC_OK) return 0;
+  return size_t(round256(s.ws_bytes) + s.V * uint64_t(s.D) * 4);
+}
+
+namespace {
+
+// kvc_compress, or (unfused) the two-kernel baseline that keeps the
+// transformed vectors in the workspace after the compress workspace.
+kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *out,
+                         size_t out_capacity, uint64_t *out_bytes_dev, void *workspace,
+                         size_t workspace_bytes, kvc_stream_t stream, bool unfused) {
   Shape s;
   if (!params) return KVC_ERR_INVALID_ARG;
   kvc_status st = describe(kv, params, s);
   if (st != KVC_OK) return st;
   if (!out || !aligned16(out) || !workspace || !aligned16(workspace)) return KVC_ERR_INVALID_ARG;
-  if (out_capacity < s.max_bytes || workspace_bytes < s.ws_bytes) return KVC_ERR_CAPACITY;
+  const uint64_t need = unfused ? round256(s.ws_bytes) + s.V * uint64_t(s.D) * 4 : s.ws_bytes;
+  if (out_capacity < s.max_bytes || workspace_bytes < need) return KVC_ERR_CAPACITY;
   const int sms = sm_count();
   if (sms <= 0) return KVC_ERR_CUDA;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -219,6 +230,7 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *o
   a.code_nnz = reinterpret_cast<unsigned long long *>(ws + w.code_nnz);
   a.meta_nnz = reinterpret_cast<uint32_t *>(ws + w.meta_nnz);
   a.ws_meta = ws + w.meta;
+  a.ymid = unfused ? reinterpret_cast<float *>(ws + round256(s.ws_bytes)) : nullptr;
   sign_masks(params->sign_seed, s.D, a.sign_mask);
 
   FinArgs f{};
@@ -261,19 +273,43 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *o
   if (kv->kind == KVC_DENSE) {
     DenseLayout L = dense_layout(kv, s);
     add_tensor_map(kv, s, L);
-    if (s.n_code)
+    if (s.n_code && unfused) {
+      e = launch_transform_dense(s.D, a, L, sms, cs);
+      if (e == cudaSuccess) e = launch_quantize(s.D, s.bits, s.G, a, sms, cs);
+    } else if (s.n_code) {
       e = s.D == 128 ? launch_encode_dense_d128(s.bits, s.G, a, L, sms, cs)
                      : launch_encode_dense_d64(s.bits, s.G, a, L, sms, cs);
+    }
     if (e == cudaSuccess) e = launch_finish_dense(f, L, sms, cs);
   } else {
     static thread_local PagedLayout L;  // large (4 KB) parameter block
     paged_layout(kv, s, L);
-    if (s.n_code)
+    if (s.n_code && unfused) {
+      e = launch_transform_paged(s.D, a, L, sms, cs);
+      if (e == cudaSuccess) e = launch_quantize(s.D, s.bits, s.G, a, sms, cs);
+    } else if (s.n_code) {
       e = s.D == 128 ? launch_encode_paged_d128(s.bits, s.G, a, L, sms, cs)
                      : launch_encode_paged_d64(s.bits, s.G, a, L, sms, cs);
+    }
     if (e == cudaSuccess) e = launch_finish_paged(f, L, sms, cs);
   }
   return e == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+}  // namespace
+
+kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params, void *out,
+                        size_t out_capacity, uint64_t *out_bytes_dev, void *workspace,
+                        size_t workspace_bytes, kvc_stream_t stream) {
+  return compress_impl(kv, params, out, out_capacity, out_bytes_dev, workspace, workspace_bytes,
+                       stream, false);
+}
+
+kvc_status kvc_compress_unfused(const kvc_kv_desc *kv, const kvc_params *params, void *out,
+                                size_t out_capacity, uint64_t *out_bytes_dev, void *workspace,
+                                size_t workspace_bytes, kvc_stream_t stream) {
+  return compress_impl(kv, params, out, out_capacity, out_bytes_dev, workspace, workspace_bytes,
+                       stream, true);
 }
 
 kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *out,

@@ -597,11 +597,11 @@ __device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *
 }
 
 // ------------------------------------------- warp row blocks (32 rows) --
-// A per-warp buffer of 32 rows of D bf16 in 64-channel halves of 32 x 128
-// bytes, 16-byte piece c of row r at (c / 8) * 4096 + r * 128 +
-// ((c % 8) ^ (r % 8)) * 16: the tensor maps' 128-byte swizzle, in which lane
-// r reading its own row, or a group of lanes reading one row, hits distinct
-// bank groups.
+// A per-warp buffer of 32 rows in column blocks of 32 x 128 bytes (64 bf16
+// channels, or 32 fp32), 16-byte piece c of row r at (c / 8) * 4096 +
+// r * 128 + ((c % 8) ^ (r % 8)) * 16: the tensor maps' 128-byte swizzle, in
+// which lane r reading its own row, or a group of lanes reading one row, hits
+// distinct bank groups.
 __device__ __forceinline__ uint32_t swz_offset(int r, int c) {
   return uint32_t((c >> 3) * 4096 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
@@ -611,9 +611,9 @@ __device__ __forceinline__ uint32_t swz_offset(int r, int c) {
 // instruction covers D/8-lane groups, one whole row per group, so every
 // group reads 2*D contiguous bytes. `dummy` is any valid global address
 // (passed with zero-fill copies). Completion: cp_async_wait_all + __syncwarp.
-template <int D>
-__device__ __forceinline__ void gather_rows(uint8_t *wbuf, const uint8_t *row, const void *dummy) {
-  constexpr int P = D / 8, RPI = 32 / P;  // pieces per row, rows per instruction
+template <int P>  // 16-byte pieces per row: 8, 16 or 32
+__device__ __forceinline__ void gather_rows_p(uint8_t *wbuf, const uint8_t *row, const void *dummy) {
+  constexpr int RPI = 32 / P;  // rows per instruction
   const int lane = threadIdx.x & 31, c = lane % P, rs = lane / P;
   const uint64_t me = reinterpret_cast<uint64_t>(row);
 #pragma unroll
@@ -632,9 +632,9 @@ __device__ __forceinline__ void gather_rows(uint8_t *wbuf, const uint8_t *row, c
 // rewritten after a __syncwarp that follows it.
 // Pieces are read eight rows' worth at a time before any of them is stored,
 // so the shared loads are not held behind the global stores.
-template <int D>
-__device__ __forceinline__ void scatter_rows(const uint8_t *wbuf, uint8_t *row) {
-  constexpr int P = D / 8, RPI = 32 / P, N = 32 / RPI, B = 8;
+template <int P>
+__device__ __forceinline__ void scatter_rows_p(const uint8_t *wbuf, uint8_t *row) {
+  constexpr int RPI = 32 / P, N = 32 / RPI, B = 8;
   const int lane = threadIdx.x & 31, c = lane % P, rs = lane / P;
   const uint64_t me = reinterpret_cast<uint64_t>(row);
 #pragma unroll
@@ -651,6 +651,16 @@ __device__ __forceinline__ void scatter_rows(const uint8_t *wbuf, uint8_t *row) 
     for (int i = 0; i < B; ++i)
       if (d[i]) *reinterpret_cast<uint4 *>(d[i] + 16u * c) = v[i];
   }
+}
+
+// Rows of D bf16 (2*D bytes, D/8 pieces).
+template <int D>
+__device__ __forceinline__ void gather_rows(uint8_t *wbuf, const uint8_t *row, const void *dummy) {
+  gather_rows_p<D / 8>(wbuf, row, dummy);
+}
+template <int D>
+__device__ __forceinline__ void scatter_rows(const uint8_t *wbuf, uint8_t *row) {
+  scatter_rows_p<D / 8>(wbuf, row);
 }
 
 // --------------------------------------------------------- addressing --

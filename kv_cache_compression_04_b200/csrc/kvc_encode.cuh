@@ -181,6 +181,11 @@ struct Enc : Cfg<D, BITS, G> {
   static __device__ __forceinline__ uint32_t vector(Pairs<D> &y, uint32_t (&code)[C::CW],
                                                     uint32_t (&meta)[C::NG]) {
     fwht_pairs<D>(y);
+    return quantize(y, code, meta);
+  }
+  // E4..E7 on the transformed vector.
+  static __device__ __forceinline__ uint32_t quantize(Pairs<D> &y, uint32_t (&code)[C::CW],
+                                                      uint32_t (&meta)[C::NG]) {
     uint32_t err = 0;
     float zf[C::NG], rr[C::NG];
 #pragma unroll
@@ -227,6 +232,81 @@ struct Enc : Cfg<D, BITS, G> {
   }
 };
 
+// E3..E7 (kFwht) or E4..E7 of this lane's vector v of block blk, its stores
+// (codes in place, meta to the workspace), and the block's shuffled-byte
+// nonzero counts, accumulated per code and meta chunk.
+template <int D, int BITS, int G, bool kFwht>
+__device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t blk, uint32_t v,
+                                                    bool valid, Pairs<D> &y, uint32_t &err) {
+  using C = Cfg<D, BITS, G>;
+  using E = Enc<D, BITS, G>;
+  const int lane = threadIdx.x & 31;
+  const uint32_t V = a.V;
+  uint32_t code[C::CW], meta[C::NG];
+  if (valid) {
+    if constexpr (kFwht)
+      err |= E::vector(y, code, meta);
+    else
+      err |= E::quantize(y, code, meta);
+    uint4 *cd = reinterpret_cast<uint4 *>(a.out + a.data_base + uint64_t(v) * C::CB);
+#pragma unroll
+    for (int q = 0; q < C::CW / 4; ++q)
+      cd[q] = make_uint4(code[4 * q], code[4 * q + 1], code[4 * q + 2], code[4 * q + 3]);
+    uint8_t *md = a.ws_meta + uint64_t(v) * C::MB;
+    if constexpr (C::NG == 1) {
+      *reinterpret_cast<uint32_t *>(md) = meta[0];
+    } else if constexpr (C::NG == 2) {
+      *reinterpret_cast<uint2 *>(md) = make_uint2(meta[0], meta[1]);
+    } else {
+      *reinterpret_cast<uint4 *>(md) = make_uint4(meta[0], meta[1], meta[2], meta[3]);
+    }
+  } else {
+#pragma unroll
+    for (int w = 0; w < C::CW; ++w) code[w] = 0;
+#pragma unroll
+    for (int g = 0; g < C::NG; ++g) meta[g] = 0;
+  }
+
+  // Shuffled-byte nonzero counts (chunk_nnz_part): 8-word groups of the
+  // code region and of the meta region, summed per chunk.
+  uint32_t cn = 0;
+  if constexpr (C::CW >= 8) {
+#pragma unroll
+    for (int q = 0; q < C::CW / 8; ++q) {
+      uint32_t o = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) o |= code[8 * q + w];
+      cn += __popc(o);
+    }
+  } else {  // 4 words: two lanes form a group
+    uint32_t o = code[0] | code[1] | code[2] | code[3];
+    o |= __shfl_xor_sync(0xFFFFFFFFu, o, 1);
+    cn = (lane & 1) ? 0u : __popc(o);
+  }
+  uint32_t mo = 0;
+#pragma unroll
+  for (int g = 0; g < C::NG; ++g) mo |= meta[g];
+  constexpr int kVecPerGroup = 32 / C::MB;  // vectors per 8-word meta group
+#pragma unroll
+  for (int o = 1; o < kVecPerGroup; o <<= 1) mo |= __shfl_xor_sync(0xFFFFFFFFu, mo, o);
+  const uint32_t mcnt = (lane % kVecPerGroup) ? 0u : __popc(mo);
+  const uint32_t cs = __reduce_add_sync(0xFFFFFFFFu, cn);
+  const uint32_t ms = __reduce_add_sync(0xFFFFFFFFu, mcnt);
+  if (lane == 0) {
+    // The block that completes a full code chunk sees its final count and
+    // flags the chunk if zero-byte elimination pays (reading R11).
+    const uint32_t c = blk * 32 / C::VC;
+    const unsigned long long old = atomicAdd(a.code_nnz + c, (1ull << 32) | cs);
+    const uint32_t blocks = (min(uint32_t(C::VC), V - c * C::VC) + 31) / 32;
+    if (uint32_t(old >> 32) + 1 == blocks && blocks * 32 == uint32_t(C::VC) &&
+        kBitmap + uint32_t(old) + cs < uint32_t(kChunk)) {
+      atomicOr(a.flags, 1u);
+      atomicMax(a.first_inv, ~c);
+    }
+    atomicAdd(a.meta_nnz + blk * 32 / C::VM, ms);
+  }
+}
+
 // ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
@@ -272,69 +352,8 @@ __global__ void __launch_bounds__(kEncThreads, 1)
   };
 
   uint32_t phase = 0, err = 0;
-  // E3..E7 of this lane's vector v of block blk, its stores, and the block's
-  // shuffled-byte nonzero counts.
   auto finish_block = [&](uint32_t blk, uint32_t v, bool valid, Pairs<D> &y) {
-    uint32_t code[C::CW], meta[C::NG];
-    if (valid) {
-      err |= E::vector(y, code, meta);
-      uint4 *cd = reinterpret_cast<uint4 *>(a.out + a.data_base + uint64_t(v) * C::CB);
-#pragma unroll
-      for (int q = 0; q < C::CW / 4; ++q)
-        cd[q] = make_uint4(code[4 * q], code[4 * q + 1], code[4 * q + 2], code[4 * q + 3]);
-      uint8_t *md = a.ws_meta + uint64_t(v) * C::MB;
-      if constexpr (C::NG == 1) {
-        *reinterpret_cast<uint32_t *>(md) = meta[0];
-      } else if constexpr (C::NG == 2) {
-        *reinterpret_cast<uint2 *>(md) = make_uint2(meta[0], meta[1]);
-      } else {
-        *reinterpret_cast<uint4 *>(md) = make_uint4(meta[0], meta[1], meta[2], meta[3]);
-      }
-    } else {
-#pragma unroll
-      for (int w = 0; w < C::CW; ++w) code[w] = 0;
-#pragma unroll
-      for (int g = 0; g < C::NG; ++g) meta[g] = 0;
-    }
-
-    // Shuffled-byte nonzero counts (chunk_nnz_part): 8-word groups of the
-    // code region and of the meta region, summed per chunk.
-    uint32_t cn = 0;
-    if constexpr (C::CW >= 8) {
-#pragma unroll
-      for (int q = 0; q < C::CW / 8; ++q) {
-        uint32_t o = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) o |= code[8 * q + w];
-        cn += __popc(o);
-      }
-    } else {  // 4 words: two lanes form a group
-      uint32_t o = code[0] | code[1] | code[2] | code[3];
-      o |= __shfl_xor_sync(0xFFFFFFFFu, o, 1);
-      cn = (lane & 1) ? 0u : __popc(o);
-    }
-    uint32_t mo = 0;
-#pragma unroll
-    for (int g = 0; g < C::NG; ++g) mo |= meta[g];
-    constexpr int kVecPerGroup = 32 / C::MB;  // vectors per 8-word meta group
-#pragma unroll
-    for (int o = 1; o < kVecPerGroup; o <<= 1) mo |= __shfl_xor_sync(0xFFFFFFFFu, mo, o);
-    const uint32_t mcnt = (lane % kVecPerGroup) ? 0u : __popc(mo);
-    const uint32_t cs = __reduce_add_sync(0xFFFFFFFFu, cn);
-    const uint32_t ms = __reduce_add_sync(0xFFFFFFFFu, mcnt);
-    if (lane == 0) {
-      // The block that completes a full code chunk sees its final count and
-      // flags the chunk if zero-byte elimination pays (reading R11).
-      const uint32_t c = blk * 32 / C::VC;
-      const unsigned long long old = atomicAdd(a.code_nnz + c, (1ull << 32) | cs);
-      const uint32_t blocks = (min(uint32_t(C::VC), V - c * C::VC) + 31) / 32;
-      if (uint32_t(old >> 32) + 1 == blocks && blocks * 32 == uint32_t(C::VC) &&
-          kBitmap + uint32_t(old) + cs < uint32_t(kChunk)) {
-        atomicOr(a.flags, 1u);
-        atomicMax(a.first_inv, ~c);
-      }
-      atomicAdd(a.meta_nnz + blk * 32 / C::VM, ms);
-    }
+    encode_finish_block<D, BITS, G, true>(a, blk, v, valid, y, err);
   };
 
   bool use_tma = false;

@@ -142,6 +142,7 @@ struct EncArgs {
   unsigned long long *code_nnz;
   uint32_t *meta_nnz;
   uint8_t *ws_meta;
+  float *ymid;         // unfused baseline only: transformed vectors, d fp32 each
   uint32_t sign_mask[128];
 };
 
@@ -195,6 +196,12 @@ struct DecArgs {
 KVC_DECLARE_LAUNCHERS(128)
 KVC_DECLARE_LAUNCHERS(64)
 #undef KVC_DECLARE_LAUNCHERS
+// Unfused baseline: transform kernel (per layout), quantize kernel.
+cudaError_t launch_transform_dense(int d, const EncArgs &a, const DenseLayout &lay, int sms,
+                                   cudaStream_t st);
+cudaError_t launch_transform_paged(int d, const EncArgs &a, const PagedLayout &lay, int sms,
+                                   cudaStream_t st);
+cudaError_t launch_quantize(int d, int bits, int group, const EncArgs &a, int sms, cudaStream_t st);
 cudaError_t launch_finish_dense(const FinArgs &a, const DenseLayout &lay, int sms, cudaStream_t st);
 cudaError_t launch_finish_paged(const FinArgs &a, const PagedLayout &lay, int sms, cudaStream_t st);
 

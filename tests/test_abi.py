@@ -219,3 +219,25 @@ def test_nonzero_byte_mask(host_logic):
 @pytest.mark.slow
 def test_nonzero_byte_mask_exhaustive(host_logic):
     assert host_logic.hl_nz_nibble_mismatches(0, 1 << 32) == 0
+
+
+def test_unfused_workspace_and_argument_checks(L):
+    """The unfused baseline's workspace is the fused one (rounded to 256
+    bytes) plus d fp32 per vector; it validates like kvc_compress, on the
+    host, before anything runs."""
+    p = kvc.params(4, 128, 0)
+    for Ln, H, T, D in [(1, 8, 64, 128), (32, 8, 4096, 128), (2, 3, 333, 64)]:
+        d = dense(Ln, H, T, D)
+        pp = kvc.params(4, 64, 0) if D == 64 else p
+        base = kvc.kvc_workspace_bytes(d, pp)
+        V = Ln * 2 * H * T
+        assert kvc.kvc_unfused_workspace_bytes(d, pp) == (base + 255) // 256 * 256 + V * D * 4
+    d = dense(2, 2, 64, 128)
+    cap = kvc.kvc_max_compressed_bytes(d, p)
+    wsb = kvc.kvc_unfused_workspace_bytes(d, p)
+    nb = FAKE
+    assert kvc.kvc_compress_unfused(d, p, FAKE, cap, nb, FAKE, wsb - 1, None) == kvc.KVC_ERR_CAPACITY
+    assert kvc.kvc_compress_unfused(d, p, FAKE, cap - 1, nb, FAKE, wsb, None) == kvc.KVC_ERR_CAPACITY
+    assert kvc.kvc_compress_unfused(d, kvc.params(3, 128, 0), FAKE, cap, nb, FAKE, wsb,
+                                    None) == kvc.KVC_ERR_UNSUPPORTED
+    assert kvc.kvc_unfused_workspace_bytes(dense(2, 2, 64, 96), p) == 0
