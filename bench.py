@@ -17,6 +17,8 @@ the only collectives are a barrier and a max over ranks of the timings.
 `--impl reference` times the CPU oracle instead (rank 0 only).
 `--sweep` runs the message-size sweep instead (1 GPU): Llama-3-8B-shaped KV
 of 1 MiB .. 4 GiB, 4-bit g128 and 2-bit g32, one JSON line per point.
+`--pipeline` times a layer-pipelined transfer of the llama8b cache over a
+simulated 100 and 400 Gbit/s link instead (1 GPU), one JSON line per speed.
 """
 from __future__ import annotations
 
@@ -361,6 +363,141 @@ def run_sweep(args):
     return 0
 
 
+def run_pipeline(args):
+    """Layer-pipelined transfer of the llama8b cache: layer l is compressed on
+    one stream, held on a 'wire' stream for its stream bytes / link speed (a
+    spin of that many SM cycles at the sampled clock), then decompressed on a
+    third stream into the receiver's cache, so compression, transfer and
+    decompression of different layers overlap. Compared with sending the raw
+    bf16 cache over the same link. The receiver's cache is checked against a
+    whole-cache round trip (decoding is per vector, so the chunking does not
+    change it)."""
+    import torch
+    import kv_cache_compression_04_b200 as kvc
+    from kv_cache_compression_04_b200 import build, synth
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.workload("llama8b")
+    kv = synth.dense_kv(w, device=dev)
+    rx = torch.empty_like(kv)
+    codec = kvc.Codec(w.bits, w.group, w.sign_seed)
+    L = w.layers
+    descs = [kvc.dense_desc(kv[l:l + 1]) for l in range(L)]
+    odescs = [kvc.dense_desc(rx[l:l + 1]) for l in range(L)]
+    bufs = [codec.buffers(d, dev) for d in descs]
+    dws = [torch.empty(kvc.kvc_decompress_workspace_bytes(d), dtype=torch.uint8, device=dev)
+           for d in odescs]
+    se, sw, sd = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    pe, pdd = kvc._stream_ptr(se), kvc._stream_ptr(sd)
+
+    def enc(l):
+        out, ws, nb = bufs[l]
+        assert kvc.kvc_compress(descs[l], codec.params, out.data_ptr(), out.numel(),
+                                nb.data_ptr(), ws.data_ptr(), ws.numel(), pe) == kvc.KVC_OK
+
+    def dec(l, n):
+        out = bufs[l][0]
+        assert kvc.kvc_decompress(out.data_ptr(), n, odescs[l], dws[l].data_ptr(),
+                                  dws[l].numel(), pdd) == kvc.KVC_OK
+
+    for l in range(L):
+        enc(l)
+    torch.cuda.synchronize(dev)
+    n = [int(b[2].item()) for b in bufs]
+    # whole-cache reference for the receiver's check
+    ref = torch.empty_like(kv)
+    with torch.cuda.stream(se):
+        cout, cws, cnb = codec.buffers(kvc.dense_desc(kv), dev)
+        sp = kvc._stream_ptr(se)
+        assert kvc.kvc_compress(kvc.dense_desc(kv), codec.params, cout.data_ptr(), cout.numel(),
+                                cnb.data_ptr(), cws.data_ptr(), cws.numel(), sp) == kvc.KVC_OK
+        rdesc = kvc.dense_desc(ref)
+        rws = torch.empty(kvc.kvc_decompress_workspace_bytes(rdesc), dtype=torch.uint8,
+                          device=dev)
+        torch.cuda.synchronize(dev)
+        assert kvc.kvc_decompress(cout.data_ptr(), int(cnb.item()), rdesc, rws.data_ptr(),
+                                  rws.numel(), sp) == kvc.KVC_OK
+    torch.cuda.synchronize(dev)
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        sm_hz = pynvml.nvmlDeviceGetMaxClockInfo(pynvml.nvmlDeviceGetHandleByIndex(0),
+                                                 pynvml.NVML_CLOCK_SM) * 1e6
+    except Exception:
+        sm_hz = 1.965e9
+    raw_l = w.raw_bytes // L
+    # per-layer compress and decompress times, each stage alone (for the
+    # two-GPU model: sender and receiver are different GPUs)
+    te = [torch.cuda.Event(enable_timing=True) for _ in range(L + 1)]
+    td = [torch.cuda.Event(enable_timing=True) for _ in range(L + 1)]
+    enc_ms, dec_ms = [0.0] * L, [0.0] * L
+    for rep in range(args.warmup + 3):
+        te[0].record(se)
+        for l in range(L):
+            enc(l)
+            te[l + 1].record(se)
+        torch.cuda.synchronize(dev)
+        td[0].record(sd)
+        for l in range(L):
+            dec(l, n[l])
+            td[l + 1].record(sd)
+        torch.cuda.synchronize(dev)
+        if rep >= args.warmup:
+            for l in range(L):
+                enc_ms[l] += te[l].elapsed_time(te[l + 1]) / 3
+                dec_ms[l] += td[l].elapsed_time(td[l + 1]) / 3
+    for gbit in (100, 400):
+        link = gbit * 1e9 / 8  # bytes per second
+        times = []
+        for rep in range(args.warmup + 3):
+            rx.zero_()
+            torch.cuda.synchronize(dev)
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(se)
+            for l in range(L):
+                enc(l)
+                e1 = torch.cuda.Event()
+                e1.record(se)
+                sw.wait_event(e1)
+                with torch.cuda.stream(sw):
+                    torch.cuda._sleep(int(n[l] / link * sm_hz))
+                e2 = torch.cuda.Event()
+                e2.record(sw)
+                sd.wait_event(e2)
+                dec(l, n[l])
+            t1.record(sd)
+            torch.cuda.synchronize(dev)
+            if rep >= args.warmup:
+                times.append(t0.elapsed_time(t1))
+        for l in range(L):
+            assert kvc.kvc_stream_status(dws[l].data_ptr(), pdd) == kvc.KVC_OK
+        assert torch.equal(rx.view(torch.int16), ref.view(torch.int16))
+        pipe_ms = statistics.median(times)
+        raw_ms = w.raw_bytes / link * 1e3
+        e_t = w_t = d_t = 0.0  # three-stage pipeline, sender and receiver on two GPUs
+        for l in range(L):
+            e_t += enc_ms[l]
+            w_t = max(e_t, w_t) + n[l] / link * 1e3
+            d_t = max(w_t, d_t) + dec_ms[l]
+        print(json.dumps({
+            "pipeline": "llama8b cache, one batch per layer (32), compress -> simulated link -> "
+                        "decompress on three streams",
+            "link_gbit_s": gbit, "raw_bytes": w.raw_bytes, "stream_bytes": sum(n),
+            "raw_transfer_ms": round(raw_ms, 3),
+            "compressed_transfer_only_ms": round(sum(n) / link * 1e3, 3),
+            "pipelined_one_gpu_ms": round(pipe_ms, 3),
+            "speedup_vs_raw_one_gpu": round(raw_ms / pipe_ms, 3),
+            "pipelined_two_gpu_model_ms": round(d_t, 3),
+            "speedup_vs_raw_two_gpu_model": round(raw_ms / d_t, 3),
+            "per_layer_compress_us": round(sum(enc_ms) / L * 1e3, 2),
+            "per_layer_decompress_us": round(sum(dec_ms) / L * 1e3, 2),
+            "per_layer_raw_bytes": raw_l, "link_model": "spin of stream bytes / link seconds "
+                                                        "at the max SM clock",
+            "receiver_check": "equal to a whole-cache round trip"}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -372,9 +509,12 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--unfused-steps", type=int, default=20)
     ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--pipeline", action="store_true")
     args = ap.parse_args()
     if args.sweep:
         return run_sweep(args)
+    if args.pipeline:
+        return run_pipeline(args)
     if args.impl == "reference":
         return run_reference(args)
     assert args.warmup >= 3, "at least 3 warm-up steps"
