@@ -709,6 +709,7 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
 template <int D, class Layout>
 __global__ void __launch_bounds__(kElimThreads, 1)
     elim_decode_kernel(const __grid_constant__ DecArgs a, const __grid_constant__ Layout lay) {
+  grid_dependency_wait();  // the meta pre-pass
   using S = ElimSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   ElimCtl *ctl = reinterpret_cast<ElimCtl *>(smem + S::ctl);

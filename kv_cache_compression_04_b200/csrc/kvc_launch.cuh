@@ -87,10 +87,10 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
   if (e != cudaSuccess) return e;
   const uint64_t egrid_want = (tiles + kElimThreads - 1) / kElimThreads;
   const int egrid = egrid_want == 0 ? 1 : int(egrid_want < uint64_t(sms) ? egrid_want : uint64_t(sms));
-  // (plain launches: dependent launches measured slower on this side when
-  // compress and decompress calls alternate on a stream)
-  ek<<<egrid, kElimThreads, esmem, st>>>(a, lay);
-  e = cudaGetLastError();
+  // The elimination kernel (which usually returns at once) is a dependent
+  // launch; the decode kernel is not (as a dependent launch it measured
+  // slower when compress and decompress calls alternate on a stream).
+  e = launch_after(ek, egrid, kElimThreads, esmem, st, a, lay);
   if (e != cudaSuccess) return e;
   k<<<grid, kDecThreads, smem, st>>>(a, lay);
   return cudaGetLastError();
