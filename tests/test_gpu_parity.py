@@ -201,6 +201,39 @@ def test_paged_parity_and_cross_layout_decode(seq, bits, g):
     assert np.array_equal(u16(dense).reshape(-1, 128), ox)
 
 
+@pytest.mark.parametrize("bits,g", [(4, 64), (2, 32)])
+def test_paged_parity_head_dim_64(bits, g):
+    """head_dim 64 through the paged gather (encode) and scatter (decode)."""
+    seq = [300, 17, 1025]
+    w, pk, x = _paged_setup(seq, D=64, bits=bits, g=g)
+    od = oracle_desc(bits, g, 64, w.layers, w.kv_heads, seq, origin=1)
+    ost, ostream = oracle.compress(od, x)
+    assert ost == oracle.OK
+    st, gstream, _, _ = gpu_compress(kvc.paged_desc(pk.pool, pk.page_table, seq), bits, g)
+    assert st == kvc.KVC_OK
+    assert np.array_equal(gstream, ostream), first_diff(gstream, ostream, od.layout())
+    _, ox = oracle.decompress(ostream, od)
+    pt2 = synth.page_table_for(seq, 16, pk.pool.shape[1], 99, device="cuda")
+    pool2 = torch.full_like(pk.pool, 1.5)
+    assert gpu_decompress(ostream, kvc.paged_desc(pool2, pt2, seq)) == kvc.KVC_OK
+    got = oracle.gather_paged(u16(pool2).reshape(-1), w.layers, w.kv_heads, 64,
+                              [s for s in pool2.stride()][:5], 16, seq, pt2.cpu().numpy(), 0,
+                              w.vectors)
+    assert np.array_equal(got, ox)
+
+
+@pytest.mark.parametrize("kind", ["zeros", "half_zero_tokens"])
+@pytest.mark.parametrize("bits,g", [(4, 64), (2, 32)])
+def test_structured_head_dim_64(kind, bits, g):
+    """Zero-byte-eliminated code chunks at head_dim 64 (the eliminated-chunk
+    decode kernel's 64-channel bodies)."""
+    kv = _structured(kind, D=64).cuda()
+    s = _roundtrip_dense(kv, bits, g)
+    od = oracle_desc(bits, g, 64, 2, 2, [1024])
+    sizes, _ = chunk_table(s, od.layout().n_chunks)
+    assert (sizes[:od.layout().n_code] < 16384).any()
+
+
 # ----------------------------------------------------------- full workloads --
 def _segment_check(w, od, gstream, x_of_range, segs):
     """Compare the chunks of sampled segments with the oracle's, and the table's
