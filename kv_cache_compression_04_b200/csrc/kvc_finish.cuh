@@ -115,10 +115,19 @@ __global__ void __launch_bounds__(kFinThreads, 4)
   uint32_t *s_cum = reinterpret_cast<uint32_t *>(ctl + 1);
   const int tid = threadIdx.x;
   const uint32_t nb = gridDim.x, b = blockIdx.x;
+  // this CTA's meta chunks s0 .. s1 - 1; the first one starts loading at once
+  // (its raw bytes need none of the prefix sums below)
+  const uint32_t s0 = uint32_t(uint64_t(b) * a.n_meta / nb);
+  const uint32_t s1 = uint32_t(uint64_t(b + 1) * a.n_meta / nb);
   if (tid == 0) {
     mbar_init(&ctl->full[0], 1);
     mbar_init(&ctl->full[1], 1);
     mbar_fence_init();
+    if (s0 < s1) {
+      const uint32_t bytes = uint32_t(round16(meta_len(a, s0)));
+      mbar_arrive_expect_tx(&ctl->full[0], bytes);
+      bulk_g2s(smem, a.ws_meta + uint64_t(s0) * kChunk, bytes, &ctl->full[0]);
+    }
     ctl->flag = *reinterpret_cast<volatile uint32_t *>(a.flags);
   }
   if constexpr (kIsPaged<Layout>) {
@@ -141,8 +150,6 @@ __global__ void __launch_bounds__(kFinThreads, 4)
   }
 
   // -------------------------------------------------- this CTA's meta chunks --
-  const uint32_t s0 = uint32_t(uint64_t(b) * a.n_meta / nb);
-  const uint32_t s1 = uint32_t(uint64_t(b + 1) * a.n_meta / nb);
   uint64_t prefix = 0;
   {
     uint64_t part = 0;
@@ -158,7 +165,6 @@ __global__ void __launch_bounds__(kFinThreads, 4)
       bulk_g2s(smem + k * kChunk, a.ws_meta + uint64_t(s) * kChunk, bytes, &ctl->full[k]);
     }
   };
-  if (s0 < s1) load(s0, 0);
   uint32_t phase = 0;  // bit k: phase of buffer k
 #pragma unroll 1
   for (uint32_t s = s0, k = 0; s < s1; ++s, k ^= 1) {
