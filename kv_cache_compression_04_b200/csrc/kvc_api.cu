@@ -22,6 +22,21 @@ struct Shape {
 };
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Clears n 16-byte words (the per-call part of a workspace), so that the
+// next kernel can be a dependent launch of it.
+__global__ void __launch_bounds__(256) clear_words_kernel(uint4 *p, uint64_t n) {
+  for (uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += uint64_t(gridDim.x) * blockDim.x)
+    p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+inline cudaError_t clear_words(void *p, uint64_t bytes, int sms, cudaStream_t st) {
+  const uint64_t n = bytes / 16, want = (n + 255) / 256, cap = uint64_t(sms) * 4;
+  const int grid = int(want == 0 ? 1 : (want < cap ? want : cap));
+  clear_words_kernel<<<grid, 256, 0, st>>>(static_cast<uint4 *>(p), n);
+  return cudaGetLastError();
+}
+
 bool stride_ok(int64_t s) { return s % 8 == 0; }  // 16-byte vector starts
 
 // Shape and layout checks shared by both directions (bits/group optional).
@@ -268,7 +283,7 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   f.tokens = s.T;
   f.seed = params->sign_seed;
 
-  if (cudaMemsetAsync(ws, 0, w.zero_bytes, cs) != cudaSuccess) return KVC_ERR_CUDA;
+  if (clear_words(ws, w.zero_bytes, sms, cs) != cudaSuccess) return KVC_ERR_CUDA;
   cudaError_t e = cudaSuccess;
   if (kv->kind == KVC_DENSE) {
     DenseLayout L = dense_layout(kv, s);
@@ -335,8 +350,7 @@ kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *ou
   a.paged_receiver = out->kind == KVC_PAGED ? 1u : 0u;
   a.ws_meta = static_cast<uint8_t *>(workspace) + kWsCtl;
   a.ws_meta_chunks = uint32_t(max_meta_chunks(s));
-  if (cudaMemsetAsync(workspace, 0, kWsCtl, cs) != cudaSuccess)
-    return KVC_ERR_CUDA;
+  if (clear_words(workspace, kWsCtl, sms, cs) != cudaSuccess) return KVC_ERR_CUDA;
   cudaError_t e;
   if (out->kind == KVC_DENSE) {
     DenseLayout L = dense_layout(out, s);

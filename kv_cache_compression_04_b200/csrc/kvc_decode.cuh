@@ -473,6 +473,7 @@ constexpr size_t meta_smem_bytes() { return 3 * size_t(kChunk) + sizeof(MetaCtl)
 template <int D>
 __global__ void __launch_bounds__(kMetaThreads, 4)
     meta_expand_kernel(const __grid_constant__ DecArgs a) {
+  grid_dependency_wait();  // the status clear
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *scr = smem + 2 * kChunk;  // buffers 0 and 1 below it
   MetaCtl *ctl = reinterpret_cast<MetaCtl *>(smem + 3 * kChunk);

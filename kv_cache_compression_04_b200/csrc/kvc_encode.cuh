@@ -374,6 +374,9 @@ __global__ void __launch_bounds__(kEncThreads, 1)
         }
       };
       if (blk < n_blocks) issue_tma(blk);
+      // The launch may overlap the workspace clear before it: the first
+      // rows load meanwhile; counts and status are touched only after this.
+      grid_dependency_wait();
 #pragma unroll 1
       for (; blk < n_blocks; blk += stride) {
         if (!mbar_wait(wbar, phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
@@ -389,6 +392,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
     }
   }
   if (!use_tma) {
+    grid_dependency_wait();  // the workspace clear (src_of may record a status)
     // Row addresses are looked up one block ahead of their gather, so the
     // page-table read overlaps a block of arithmetic.
     if (blk < n_blocks) gather_rows<D>(wbuf, src_of(blk * 32 + lane), a.out);

@@ -53,8 +53,8 @@ cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_
   const uint32_t n_blocks = (a.V + 31) / 32;
   const uint32_t want = (n_blocks + kEncWarps - 1) / kEncWarps;
   const int grid = int(want < uint32_t(sms) ? want : uint32_t(sms));
-  k<<<grid, kEncThreads, smem, st>>>(a, lay);
-  return cudaGetLastError();
+  // a dependent launch after the workspace clear: see encode_kernel
+  return launch_after(k, grid, kEncThreads, smem, st, a, lay);
 }
 
 template <int D, class Layout>
@@ -75,8 +75,7 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
   if (e != cudaSuccess) return e;
   const uint32_t mcap = 4u * uint32_t(sms);
   const int mgrid = int(a.ws_meta_chunks == 0 ? 1u : (a.ws_meta_chunks < mcap ? a.ws_meta_chunks : mcap));
-  mk<<<mgrid, kMetaThreads, meta_smem_bytes(), st>>>(a);
-  e = cudaGetLastError();
+  e = launch_after(mk, mgrid, kMetaThreads, meta_smem_bytes(), st, a);  // after the status clear
   if (e != cudaSuccess) return e;
   // code chunks that used zero-byte elimination (returns at once if none);
   // 256 chunks per CTA and scan step, for the largest code region (4-bit)
