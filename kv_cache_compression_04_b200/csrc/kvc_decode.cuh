@@ -463,24 +463,24 @@ __global__ void __launch_bounds__(kDecThreads)
 // whole table); a bad one only records KVC_ERR_CORRUPT.
 constexpr int kMetaThreads = 256;
 struct MetaCtl {
-  uint64_t full[2];
+  uint64_t full[1];
   uint32_t red[kMetaThreads / 32];
   uint32_t ok, bits, group, n_chunks;
   uint64_t base, limit;
 };
-constexpr size_t meta_smem_bytes() { return 3 * size_t(kChunk) + sizeof(MetaCtl); }
+constexpr int kMetaCtas = 6;  // per SM: one chunk buffer each, so latency hides across CTAs
+constexpr size_t meta_smem_bytes() { return 2 * size_t(kChunk) + sizeof(MetaCtl); }
 
 template <int D>
-__global__ void __launch_bounds__(kMetaThreads, 4)
+__global__ void __launch_bounds__(kMetaThreads, kMetaCtas)
     meta_expand_kernel(const __grid_constant__ DecArgs a) {
   grid_dependency_wait();  // the status clear
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t *scr = smem + 2 * kChunk;  // buffers 0 and 1 below it
-  MetaCtl *ctl = reinterpret_cast<MetaCtl *>(smem + 3 * kChunk);
+  uint8_t *buf = smem, *scr = smem + kChunk;
+  MetaCtl *ctl = reinterpret_cast<MetaCtl *>(smem + 2 * kChunk);
   const int tid = threadIdx.x;
   if (tid == 0) {
     mbar_init(&ctl->full[0], 1);
-    mbar_init(&ctl->full[1], 1);
     mbar_fence_init();
     const StreamHdr h = parse_header<D>(a);
     ctl->ok = h.ok;
@@ -498,61 +498,37 @@ __global__ void __launch_bounds__(kMetaThreads, 4)
   if (n_meta > a.ws_meta_chunks) return;  // cannot happen for a consistent header
   const uint8_t *table = a.in + kHeader;
   const uint64_t base = ctl->base, limit = ctl->limit;
-
+  uint32_t phase = 0;
   // this CTA's chunks s = blockIdx.x + i * gridDim.x that used elimination
-  auto entry = [&](uint32_t s) { return ld_u64(table + 8 * (uint64_t(n_code) + s)); };
-  auto eliminated = [&](uint32_t s) {
-    return uint32_t(entry(s) & 0xFFFFu) != min(vm, a.V - s * vm) * mb;
-  };
-  auto next = [&](uint32_t s) {
-    while (s < n_meta && !eliminated(s)) s += gridDim.x;
-    return s;
-  };
-  // starts loading chunk s into buffer k; false (and CORRUPT) for a bad entry
-  auto load = [&](uint32_t s, uint32_t k) {
-    const uint64_t e = entry(s), off = (e >> 16) << 4;
+#pragma unroll 1
+  for (uint32_t s = blockIdx.x; s < n_meta; s += gridDim.x) {
+    const uint64_t e = ld_u64(table + 8 * (uint64_t(n_code) + s)), off = (e >> 16) << 4;
     const uint32_t size = uint32_t(e & 0xFFFFu), len = min(vm, a.V - s * vm) * mb;
+    if (size == len) continue;  // raw: read in place by the decode kernel
     const bool ok = len == uint32_t(kChunk) && size >= kBitmap && size < len &&
                     base + off + round16(size) <= limit;
+    if (!ok) {
+      if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
+      continue;
+    }
     if (tid == 0) {
-      if (ok) {
-        mbar_arrive_expect_tx(&ctl->full[k], uint32_t(round16(size)));
-        bulk_g2s(smem + k * kChunk, a.in + base + off, uint32_t(round16(size)), &ctl->full[k]);
-      } else {
-        set_status(a.status, KVC_ERR_CORRUPT);
-        mbar_arrive(&ctl->full[k]);  // completes the phase without data
+      bulk_wait_read<0>();  // the previous chunk's store has read the buffer
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&ctl->full[0], uint32_t(round16(size)));
+      bulk_g2s(buf, a.in + base + off, uint32_t(round16(size)), &ctl->full[0]);
+    }
+    if (!mbar_wait(&ctl->full[0], phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+    phase ^= 1;
+    if (ze_decode<kMetaThreads>(buf, scr, ctl->red, size)) {
+      fence_proxy_async_smem();
+      named_bar_sync(1, kMetaThreads);
+      if (tid == 0) {
+        bulk_s2g(a.ws_meta + uint64_t(s) * kChunk, buf, kChunk);
+        bulk_commit();
       }
+    } else if (tid == 0) {
+      set_status(a.status, KVC_ERR_CORRUPT);
     }
-    return ok;
-  };
-  uint32_t s = next(blockIdx.x), k = 0, phase = 0;
-  bool ok = s < n_meta && load(s, 0);
-#pragma unroll 1
-  while (s < n_meta) {
-    const uint32_t ns = next(s + gridDim.x);
-    bool nok = false;
-    if (ns < n_meta) {
-      if (tid == 0) bulk_wait_read<0>();  // the store from buffer k ^ 1 has read it
-      nok = load(ns, k ^ 1);
-    }
-    if (!mbar_wait(&ctl->full[k], (phase >> k) & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
-    phase ^= 1u << k;
-    uint8_t *buf = smem + k * kChunk;
-    if (ok) {
-      if (ze_decode<kMetaThreads>(buf, scr, ctl->red, uint32_t(entry(s) & 0xFFFFu))) {
-        fence_proxy_async_smem();
-        named_bar_sync(1, kMetaThreads);
-        if (tid == 0) {
-          bulk_s2g(a.ws_meta + uint64_t(s) * kChunk, buf, kChunk);
-          bulk_commit();
-        }
-      } else if (tid == 0) {
-        set_status(a.status, KVC_ERR_CORRUPT);
-      }
-    }
-    s = ns;
-    ok = nok;
-    k ^= 1;
   }
   if (tid == 0) bulk_wait_all<0>();
 }

@@ -73,7 +73,7 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
   struct MetaTag {};
   e = prepare<MetaTag>(mk, meta_smem_bytes());
   if (e != cudaSuccess) return e;
-  const uint32_t mcap = 4u * uint32_t(sms);
+  const uint32_t mcap = uint32_t(kMetaCtas) * uint32_t(sms);
   const int mgrid = int(a.ws_meta_chunks == 0 ? 1u : (a.ws_meta_chunks < mcap ? a.ws_meta_chunks : mcap));
   e = launch_after(mk, mgrid, kMetaThreads, meta_smem_bytes(), st, a);  // after the status clear
   if (e != cudaSuccess) return e;
