@@ -119,6 +119,7 @@ def lib():
                                                  u16p, u8p, u32p, u32p]),
                 "orc_decode_segment": (C.c_int, [C.POINTER(Desc), C.c_uint64,
                                                  u8p, u32p, u16p]),
+                "orc_code_elim_pays": (C.c_int, [u32p, u32p, C.c_uint64]),
                 "orc_compress": (C.c_int, [C.POINTER(Desc), u16p, u8p,
                                            C.c_uint64, u64p]),
                 "orc_decompress": (C.c_int, [u8p, C.c_uint64,
@@ -265,6 +266,16 @@ def lossless_encode_chunk(chunk: np.ndarray) -> np.ndarray:
     n = lib().orc_lossless_encode_chunk(_p(chunk, C.c_uint8), chunk.size,
                                         _p(out, C.c_uint8))
     return out[:n].copy()
+
+
+def code_elim_pays(sizes, lens) -> bool:
+    """Reading R16: does zero-byte elimination in the code region pay for the
+    shift of the code chunks after the first shrinking one?"""
+    sizes = np.ascontiguousarray(sizes, np.uint32)
+    lens = np.ascontiguousarray(lens, np.uint32)
+    assert sizes.shape == lens.shape
+    return bool(lib().orc_code_elim_pays(_p(sizes, C.c_uint32), _p(lens, C.c_uint32),
+                                         sizes.size))
 
 
 def lossless_decode_chunk(enc: np.ndarray, length: int):

@@ -571,6 +571,30 @@ int orc_decode_segment(const orc_desc *d, uint64_t s, const uint8_t *chunks,
   return st;
 }
 
+/* Reading R16 (the encoder's choice for the code region; a decoder accepts
+ * either outcome). Storing a code chunk eliminated shifts every later code
+ * chunk, so elimination in the code region is kept only if it pays for that
+ * shift: with S = the padded bytes it saves over all code chunks and T = the
+ * padded bytes of the code chunks from the first shrinking one to the end of
+ * the region, it is kept iff 64 * S >= T; otherwise every code chunk is
+ * stored raw. 1/64 is where the time to move T bytes through HBM twice (read
+ * and write, about 6.4 TB/s) equals the time to send S bytes over a
+ * 400 Gbit/s link. sizes[c] and lens[c] are the eliminated-or-raw size and
+ * the raw length of code chunk c, in code-chunk order. Returns 1 if some
+ * chunk shrinks and elimination pays, 0 otherwise. */
+int orc_code_elim_pays(const uint32_t *sizes, const uint32_t *lens, uint64_t n_code) {
+  uint64_t c, S = 0, T = 0;
+  int seen = 0;
+  for (c = 0; c < n_code; c++) {
+    if (sizes[c] != lens[c]) seen = 1;
+    if (seen) {
+      T += round16(lens[c]);
+      S += round16(lens[c]) - round16(sizes[c]);
+    }
+  }
+  return seen && 64 * S >= T;
+}
+
 int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
                  uint64_t capacity, uint64_t *out_bytes) {
   orc_layout lay;
@@ -619,6 +643,32 @@ int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
       where[idx] = idx * ORC_CHUNK;
       pos += sizes[k];
     }
+  }
+  /* reading R16: keep elimination in the code region only if it pays for
+     the shift of the code chunks after the first shrinking one */
+  if (lay.n_code) {
+    uint32_t *csz = (uint32_t *)malloc((size_t)lay.n_code * 4);
+    uint32_t *clen = (uint32_t *)malloc((size_t)lay.n_code * 4);
+    for (i = 0; i < lay.n_code; i++) {
+      uint64_t nv = lay.V - i * lay.vec_per_code;
+      if (nv > lay.vec_per_code) nv = lay.vec_per_code;
+      csz[i] = all_sizes[orc_code_chunk_index(&lay, i)];
+      clen[i] = (uint32_t)(nv * lay.code_bytes);
+    }
+    if (!orc_code_elim_pays(csz, clen, lay.n_code)) {
+      uint8_t raw[ORC_CHUNK];
+      for (i = 0; i < lay.n_code; i++) {
+        uint64_t idx = orc_code_chunk_index(&lay, i);
+        if (csz[i] == clen[i]) continue;
+        if (orc_lossless_decode_chunk(store + where[idx], csz[i], clen[i], raw) != ORC_OK &&
+            st == ORC_OK)
+          st = ORC_ERR_CORRUPT; /* cannot happen: the chunk was just encoded */
+        memcpy(store + where[idx], raw, clen[i]);
+        all_sizes[idx] = clen[i];
+      }
+    }
+    free(csz);
+    free(clen);
   }
   /* lay the chunks out in index order */
   for (i = 0; i < lay.n_chunks; i++) {

@@ -114,6 +114,9 @@ int orc_encode_segment(const orc_desc *d, uint64_t s, const uint16_t *vectors,
 int orc_decode_segment(const orc_desc *d, uint64_t s, const uint8_t *chunks,
                        const uint32_t *sizes, uint16_t *vectors);
 
+/* Reading R16: 1 iff some code chunk shrinks and the padded bytes saved are
+ * at least 1/64 of the padded bytes from the first shrinking code chunk on. */
+int orc_code_elim_pays(const uint32_t *sizes, const uint32_t *lens, uint64_t n_code);
 int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
                  uint64_t capacity, uint64_t *out_bytes);
 int orc_decompress(const uint8_t *stream, uint64_t stream_bytes,

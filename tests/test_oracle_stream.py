@@ -66,6 +66,65 @@ def test_header_flag_code_elimination(zero_chunk):
     assert st == oracle.OK
 
 
+def test_code_elim_rule_arithmetic():
+    """Reading R16 by hand: S = padded bytes saved, T = padded bytes from the
+    first shrinking code chunk on; elimination is kept iff 64 * S >= T."""
+    F = 16384
+    pays = oracle.code_elim_pays
+    assert not pays([F] * 5, [F] * 5)                         # nothing shrinks
+    assert not pays([], [])
+    # one all-zero chunk (bitmap only, saves 14336 = 56 * 256) at position 1:
+    # T = 56 chunks -> 64 * 14336 = 917504 = T, kept (tie); 57 chunks -> not
+    assert pays([F, 2048] + [F] * 55, [F] * 57)
+    assert not pays([F, 2048] + [F] * 56, [F] * 58)
+    # chunks before the first shrinking one are not part of T
+    assert pays([F] * 1000 + [2048] + [F] * 55, [F] * 1056)
+    # sizes count padded: 2049 -> 2064 saves 14320, so 56 chunks no longer pay
+    assert not pays([2049] + [F] * 55, [F] * 56)
+    assert pays([2049] + [F] * 54, [F] * 55)
+    # a short last chunk counts with its padded length: 55 full + 1000 -> 1008
+    assert pays([2048] + [F] * 54 + [1000], [F] * 55 + [1000])
+    # two shrinking chunks: S adds up
+    assert pays([2048, F, 2048] + [F] * 109, [F] * 112)
+    assert not pays([2048, F, 2048] + [F] * 110, [F] * 113)
+
+
+def _one_zero_chunk(bits, group, zero_chunk, n_code=64, seed=11):
+    """Random vectors except the `zero_chunk`-th code chunk's vectors, which
+    are zero: all-zero codes, stored as the 2048-byte bitmap alone when
+    eliminated."""
+    per = 16384 * 8 // (128 * bits)                           # vectors per code chunk
+    V = per * n_code
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(V, 128, generator=g)
+    x[zero_chunk * per:(zero_chunk + 1) * per] = 0
+    x = synth.bf16_bits(x.to(torch.bfloat16)).reshape(V, 128)
+    d = oracle.StreamDesc(bits, group, 128, 1, V // 2048, [1024], 0)
+    return d, x
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (2, 32)])
+@pytest.mark.parametrize("zero_chunk,kept", [(8, True), (7, False), (63, True), (0, False)])
+def test_code_elim_rule_in_stream(bits, group, zero_chunk, kept):
+    """64 code chunks, one of them all-zero codes: eliminated (and the later
+    chunks shifted) only if the 56 * 256 saved bytes are at least 1/64 of the
+    code chunks from it to the end, i.e. if at most 56 chunks remain."""
+    d, x = _one_zero_chunk(bits, group, zero_chunk)
+    lay = d.layout()
+    assert lay.n_code == 64
+    st, s = oracle.compress(d, x)
+    assert st == oracle.OK
+    table = np.frombuffer(bytes(s[64:64 + 8 * lay.n_chunks]), "<u8")
+    code = [int(table[oracle.code_chunk_index(lay, c)] & 0xFFFF) for c in range(64)]
+    assert code[zero_chunk] == (2048 if kept else 16384)
+    assert all(code[c] == 16384 for c in range(64) if c != zero_chunk)
+    assert s[11] == (1 if kept else 0)
+    st, y = oracle.decompress(s, d)
+    assert st == oracle.OK
+    zero = y[zero_chunk * (lay.V // 64):(zero_chunk + 1) * (lay.V // 64)]
+    assert not (zero & 0x7FFF).any()                          # +-0 (signs flip zeros)
+
+
 @pytest.mark.parametrize("name,n_code,n_meta", [("tiny", 4, 1), ("llama8b", 8192, 512),
                                                 ("qwen7b", 14336, 7168)])
 def test_layout_counts(name, n_code, n_meta):
