@@ -145,9 +145,14 @@ size_t kvc_decompress_workspace_bytes(const kvc_kv_desc *out);
  * in 16-byte units); u32 token count per request; zero padding to 16 bytes;
  * the chunks, each zero-padded to 16 bytes. The code and meta regions are cut
  * into 16 KB chunks; a meta chunk covers group_size*bits/32 code chunks. Chunk
- * order (table and data): every code chunk, then every meta chunk. The call
- * launches up to three kernels on `stream` (encode; table, meta chunks and
- * header; compaction, which returns at once unless a code chunk shrank). */
+ * order (table and data): every code chunk, then every meta chunk. A chunk is
+ * stored zero-byte eliminated only if that makes it shorter; in the code
+ * region, only if moreover the padded bytes saved there are at least 1/64 of
+ * the padded bytes from the first shrinking code chunk to the region's end
+ * (the bytes that shift), else every code chunk is stored raw. The call
+ * launches four kernels on `stream` (workspace clear; encode; table, meta
+ * chunks and header; compaction, which returns at once unless code chunks
+ * are stored eliminated). */
 kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params,
                         void *out, size_t out_capacity, uint64_t *out_bytes_dev,
                         void *workspace, size_t workspace_bytes,

@@ -234,7 +234,7 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   const WsLayout w = ws_layout(s.n_code, s.n_seg);
-  uint32_t *ctl = reinterpret_cast<uint32_t *>(ws);  // status, flags, ticket, reads, first
+  uint32_t *ctl = reinterpret_cast<uint32_t *>(ws);  // status, flags, ticket, reads, first, -, saved
   EncArgs a{};
   a.V = uint32_t(s.V);
   a.out = static_cast<uint8_t *>(out);
@@ -242,6 +242,7 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   a.status = ctl;
   a.flags = ctl + 1;
   a.first_inv = ctl + 4;
+  a.saved = reinterpret_cast<unsigned long long *>(ctl + 6);
   a.code_nnz = reinterpret_cast<unsigned long long *>(ws + w.code_nnz);
   a.meta_nnz = reinterpret_cast<uint32_t *>(ws + w.meta_nnz);
   a.ws_meta = ws + w.meta;
@@ -264,6 +265,7 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   f.status = ctl;
   f.flags = ctl + 1;
   f.first_inv = ctl + 4;
+  f.saved = a.saved;
   f.ticket = ctl + 2;  // ticket[0]: next code chunk to move, ticket[1]: chunks read
   f.code_nnz = a.code_nnz;
   f.meta_nnz = a.meta_nnz;

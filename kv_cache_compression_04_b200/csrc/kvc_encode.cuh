@@ -294,14 +294,17 @@ __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t b
   const uint32_t ms = __reduce_add_sync(0xFFFFFFFFu, mcnt);
   if (lane == 0) {
     // The block that completes a full code chunk sees its final count and
-    // flags the chunk if zero-byte elimination pays (reading R11).
+    // flags the chunk if zero-byte elimination makes it shorter (reading
+    // R11), adding the padded bytes it would save (reading R16 weighs them).
     const uint32_t c = blk * 32 / C::VC;
     const unsigned long long old = atomicAdd(a.code_nnz + c, (1ull << 32) | cs);
     const uint32_t blocks = (min(uint32_t(C::VC), V - c * C::VC) + 31) / 32;
+    const uint32_t size = kBitmap + uint32_t(old) + cs;
     if (uint32_t(old >> 32) + 1 == blocks && blocks * 32 == uint32_t(C::VC) &&
-        kBitmap + uint32_t(old) + cs < uint32_t(kChunk)) {
+        size < uint32_t(kChunk)) {
       atomicOr(a.flags, 1u);
       atomicMax(a.first_inv, ~c);
+      atomicAdd(a.saved, (unsigned long long)(uint32_t(kChunk) - uint32_t(round16(size))));
     }
     atomicAdd(a.meta_nnz + blk * 32 / C::VM, ms);
   }

@@ -10,7 +10,9 @@
 //   reductions over the count arrays, so CTAs never wait on one another.
 //
 // compact_kernel: runs only when some code chunk shrinks (zero-byte
-//   elimination pays), which is rare for Hadamard-rotated codes. The encode
+//   elimination makes it shorter, reading R11) and eliminating pays for the
+//   shift of the later code chunks (reading R16), which is rare for
+//   Hadamard-rotated codes. The encode
 //   kernel left every code chunk raw at data base + c * 16 KB; chunks are
 //   re-encoded and moved left in ticket order, a chunk only after every chunk
 //   whose raw bytes its destination overlaps has been read; the meta chunks
@@ -71,6 +73,20 @@ __device__ __forceinline__ uint32_t meta_stored_size(const FinArgs &a, uint32_t 
   return (len == uint32_t(kChunk) && kBitmap + n < uint32_t(kChunk)) ? kBitmap + n : len;
 }
 
+// Reading R16: some code chunk shrank (flag bit 0); keep zero-byte
+// elimination in the code region only if the padded bytes it saves are at
+// least 1/64 of the padded bytes from the first shrinking code chunk to the
+// region's end, the bytes the compaction would move. Otherwise every code
+// chunk stays raw where the encode kernel wrote it.
+__device__ __forceinline__ bool code_elim_kept(const FinArgs &a, uint32_t flags) {
+  if (!(flags & 1u) || a.n_code == 0) return false;
+  const uint32_t c0 = ~*reinterpret_cast<const volatile uint32_t *>(a.first_inv);
+  const uint64_t saved = *reinterpret_cast<const volatile unsigned long long *>(a.saved);
+  const uint64_t moved =
+      uint64_t(a.n_code - 1 - c0) * kChunk + round16(code_len(a, a.n_code - 1));
+  return 64 * saved >= moved;
+}
+
 // Header (reading R12); byte 11 bit 0: some code chunk uses zero-byte
 // elimination (`code_elim`).
 template <class Layout>
@@ -128,15 +144,15 @@ __global__ void __launch_bounds__(kFinThreads, 4)
       mbar_arrive_expect_tx(&ctl->full[0], bytes);
       bulk_g2s(smem, a.ws_meta + uint64_t(s0) * kChunk, bytes, &ctl->full[0]);
     }
-    ctl->flag = *reinterpret_cast<volatile uint32_t *>(a.flags);
+    ctl->flag = code_elim_kept(a, *reinterpret_cast<volatile uint32_t *>(a.flags)) ? 1u : 0u;
   }
   if constexpr (kIsPaged<Layout>) {
     for (uint32_t r = tid; r <= lay.n_req; r += NT) s_cum[r] = lay.cum[r];
   }
   __syncthreads();
 
-  // Bytes of all code chunks, padded. The encode kernel flagged the call if
-  // any code chunk shrinks; otherwise every code chunk is raw and the code
+  // Bytes of all code chunks, padded. Unless some code chunk shrank and
+  // eliminating pays (reading R16), every code chunk is raw and the code
   // region is the plain array of codes.
   const bool shrank = ctl->flag & 1u;
   uint64_t total_code = 0;
@@ -250,7 +266,7 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
   if (tid == 0) {
     mbar_init(&ctl->full[0], 1);
     mbar_fence_init();
-    ctl->flag = *reinterpret_cast<volatile uint32_t *>(a.flags);
+    ctl->flag = code_elim_kept(a, *reinterpret_cast<volatile uint32_t *>(a.flags)) ? 1u : 0u;
   }
   __syncthreads();
   if (!(ctl->flag & 1u)) return;

@@ -32,7 +32,8 @@ constexpr uint32_t kNoTile = 0xFFFFFFFFu;
 // Workspace of kvc_compress, in this order (each part 256-byte aligned):
 //   control   status word, flags word (bit 0: some code chunk shrank),
 //             compaction ticket, compaction read count, ~(first shrinking
-//             code chunk)
+//             code chunk), (u64 at byte 24) padded bytes the shrinking code
+//             chunks save
 //   meta_nnz  u32 per meta chunk: shuffled-byte nonzero count (accumulated)
 //   code_nnz  u64 per code chunk: the same count (low half) and the number
 //             of 32-vector blocks accumulated so far (high half)
@@ -139,6 +140,7 @@ struct EncArgs {
   uint32_t *status;
   uint32_t *flags;     // bit 0: some code chunk shrinks
   uint32_t *first_inv; // max over shrinking code chunks c of ~c (0: none)
+  unsigned long long *saved;  // padded bytes the shrinking code chunks save
   unsigned long long *code_nnz;
   uint32_t *meta_nnz;
   uint8_t *ws_meta;
@@ -158,6 +160,7 @@ struct FinArgs {
   uint32_t *status;
   uint32_t *flags;
   uint32_t *first_inv;  // ~(first shrinking code chunk), 0 if none
+  const unsigned long long *saved;  // padded bytes the shrinking code chunks save
   uint32_t *ticket;
   const unsigned long long *code_nnz;
   const uint32_t *meta_nnz;

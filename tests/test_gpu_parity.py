@@ -133,6 +133,28 @@ def test_structured_inputs(kind, bits, g):
         assert (sizes < 16384).any()              # zero-byte elimination was exercised
 
 
+@pytest.mark.parametrize("bits,g", [(4, 128), (2, 32)])
+@pytest.mark.parametrize("zero_chunk,kept", [(8, True), (7, False), (63, True), (0, False)])
+def test_code_elimination_threshold(bits, g, zero_chunk, kept):
+    """Reading R16 on the GPU: 64 code chunks, one of them all-zero codes.
+    Its elimination saves 56 * 256 padded bytes, so it is kept only if at most
+    56 code chunks (itself included) follow from it: 8 and 63 keep it (8 is
+    the tie), 7 and 0 store every code chunk raw, with the flag clear and no
+    compaction. Stream bytes and decoded values equal the oracle's."""
+    per = 16384 * 8 // (128 * bits)                           # vectors per code chunk
+    V = per * 64
+    x = torch.randn(V, 128, generator=torch.Generator().manual_seed(11))
+    x[zero_chunk * per:(zero_chunk + 1) * per] = 0
+    kv = x.to(torch.bfloat16).reshape(1, 2, V // 2048, 1024, 128).cuda()
+    s = _roundtrip_dense(kv, bits, g)
+    od = oracle_desc(bits, g, 128, 1, V // 2048, [1024])
+    lay = od.layout()
+    sizes, _ = chunk_table(s, lay.n_chunks)
+    code = [int(sizes[oracle.code_chunk_index(lay, c)]) for c in range(64)]
+    assert code[zero_chunk] == (2048 if kept else 16384)
+    assert s[11] == (1 if kept else 0)
+
+
 def test_compaction_many_chunks_mixed():
     """Shrunken code chunks scattered through more code chunks than CTAs (each
     CTA moves several): a random half of the 16 KB code chunks are all-zero
