@@ -224,6 +224,34 @@ def test_paged_parity_and_cross_layout_decode(seq, bits, g):
 
 
 @pytest.mark.parametrize("bits,g", [(4, 64), (2, 32)])
+def test_paged_parity_eliminated_code_chunks(bits, g):
+    """A paged batch whose middle request is all zeros: the code chunks inside
+    it are stored eliminated (they save far more than 1/64 of what follows,
+    reading R16) between raw ones, so the paged gather feeds the compaction,
+    and the eliminated-chunk decode scatters through another page table."""
+    seq = [700, 600, 300]
+    w, pk, _ = _paged_setup(seq, bits=bits, g=g)
+    pages = pk.page_table[1, :(600 + 15) // 16].long()
+    pk.pool[:, pages] = 0
+    x = oracle.gather_paged(u16(pk.pool).reshape(-1), w.layers, w.kv_heads, 128,
+                            pk.strides(), 16, seq, pk.page_table.cpu().numpy(), 0, w.vectors)
+    od = oracle_desc(bits, g, 128, w.layers, w.kv_heads, seq, origin=1)
+    ost, ostream = oracle.compress(od, x)
+    assert ost == oracle.OK and ostream[11] == 1
+    st, gstream, _, _ = gpu_compress(kvc.paged_desc(pk.pool, pk.page_table, seq), bits, g)
+    assert st == kvc.KVC_OK
+    assert np.array_equal(gstream, ostream), first_diff(gstream, ostream, od.layout())
+    _, ox = oracle.decompress(ostream, od)
+    pt2 = synth.page_table_for(seq, 16, pk.pool.shape[1], 41, device="cuda")
+    pool2 = torch.full_like(pk.pool, 1.5)
+    assert gpu_decompress(ostream, kvc.paged_desc(pool2, pt2, seq)) == kvc.KVC_OK
+    got = oracle.gather_paged(u16(pool2).reshape(-1), w.layers, w.kv_heads, 128,
+                              [s for s in pool2.stride()][:5], 16, seq, pt2.cpu().numpy(), 0,
+                              w.vectors)
+    assert np.array_equal(got, ox)
+
+
+@pytest.mark.parametrize("bits,g", [(4, 64), (2, 32)])
 def test_paged_parity_head_dim_64(bits, g):
     """head_dim 64 through the paged gather (encode) and scatter (decode)."""
     seq = [300, 17, 1025]
