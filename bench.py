@@ -5,7 +5,8 @@ of one synthetic KV cache resident in HBM (Llama-3-8B shape by default:
 Prints ONE JSON line (rank 0):
   value      raw bf16 bytes per second of encode + decode, all ranks (GB/s)
   e2e        the same metric through the C ABI with pinned host buffers:
-             H2D KV, compress, D2H stream, H2D stream, decompress, D2H KV
+             H2D KV, compress, D2H stream, H2D stream, decompress, D2H KV,
+             in layer groups whose copies overlap in both directions
   roofline   the slower kernel: algorithmic bytes per launch / its CUDA-event
              duration against the measured HBM copy bandwidth
   cpu_baseline  the CPU oracle on a bounded sample of the same workload
@@ -177,6 +178,101 @@ class ClockSampler:
 
 
 # -------------------------------------------------------------- workloads --
+def run_e2e(args, w, codec, keep, obuf, stream, dev, dist, world, raw):
+    """End to end through the C ABI with pinned host buffers: every step
+    uploads the KV cache, compresses it, downloads the stream, uploads it
+    again, decompresses it and downloads the KV cache. The cache goes in
+    layer groups (one kvc_compress / kvc_decompress call per group, each with
+    its own stream, workspace and pinned buffers) on five CUDA streams (KV
+    upload, compress, stream download, stream upload + decompress, KV
+    download) ordered by events, so uploads and downloads of different groups
+    overlap on the two copy directions."""
+    import torch
+    import kv_cache_compression_04_b200 as kvc
+    src = keep.pool if w.paged else keep
+    L = src.shape[0]
+    G = min(8, L)
+    bounds = [(L * g // G, L * (g + 1) // G) for g in range(G)]
+
+    def desc_of(t):
+        return kvc.paged_desc(t, keep.page_table, w.seq_lens) if w.paged else kvc.dense_desc(t)
+
+    h_in = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
+    h_in.copy_(src)
+    h_out = torch.empty(obuf.shape, dtype=obuf.dtype, pin_memory=True)
+    groups = []
+    for l0, l1 in bounds:
+        sd, od = desc_of(src[l0:l1]), desc_of(obuf[l0:l1])
+        out, ws, nb = codec.buffers(sd, dev)
+        dws = torch.empty(kvc.kvc_decompress_workspace_bytes(od), dtype=torch.uint8, device=dev)
+        groups.append(dict(l=(l0, l1), sd=sd, od=od, out=out, ws=ws, nb=nb, dws=dws,
+                           hs=torch.empty(out.numel(), dtype=torch.uint8, pin_memory=True)))
+    sk_in, s_enc, s_st_out, s_st_in, sk_out = (torch.cuda.Stream(dev) for _ in range(5))
+    ptr = kvc._stream_ptr
+
+    def compress(g, st):
+        assert kvc.kvc_compress(g["sd"], codec.params, g["out"].data_ptr(), g["out"].numel(),
+                                g["nb"].data_ptr(), g["ws"].data_ptr(), g["ws"].numel(),
+                                ptr(st)) == kvc.KVC_OK
+
+    def decompress(g, st):
+        assert kvc.kvc_decompress(g["out"].data_ptr(), g["n"], g["od"], g["dws"].data_ptr(),
+                                  g["dws"].numel(), ptr(st)) == kvc.KVC_OK
+
+    for g in groups:  # stream sizes (fixed for a fixed input)
+        compress(g, stream)
+        g["n"] = int(g["nb"].item())
+    n_total = sum(g["n"] for g in groups)
+    before = obuf.view(torch.int16).sum(dtype=torch.int64)
+
+    def e2e_step():
+        go = torch.cuda.Event()
+        go.record(stream)
+        for s_ in (sk_in, s_enc, s_st_out, s_st_in, sk_out):
+            s_.wait_event(go)
+        ends = []
+        for g in groups:
+            (l0, l1), n = g["l"], g["n"]
+            with torch.cuda.stream(sk_in):
+                src[l0:l1].copy_(h_in[l0:l1], non_blocking=True)
+            e = torch.cuda.Event(); e.record(sk_in); s_enc.wait_event(e)
+            compress(g, s_enc)
+            e = torch.cuda.Event(); e.record(s_enc); s_st_out.wait_event(e)
+            with torch.cuda.stream(s_st_out):
+                g["hs"][:n].copy_(g["out"][:n], non_blocking=True)
+            e = torch.cuda.Event(); e.record(s_st_out); s_st_in.wait_event(e)
+            with torch.cuda.stream(s_st_in):
+                g["out"][:n].copy_(g["hs"][:n], non_blocking=True)
+            decompress(g, s_st_in)
+            e = torch.cuda.Event(); e.record(s_st_in); sk_out.wait_event(e)
+            with torch.cuda.stream(sk_out):
+                h_out[l0:l1].copy_(obuf[l0:l1], non_blocking=True)
+        for s_ in (sk_in, s_enc, s_st_out, s_st_in, sk_out):
+            e = torch.cuda.Event(); e.record(s_); stream.wait_event(e)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0] / args.e2e_steps
+    for g in groups:
+        assert kvc.kvc_stream_status(g["ws"].data_ptr(), ptr(stream)) == kvc.KVC_OK
+        assert kvc.kvc_stream_status(g["dws"].data_ptr(), ptr(stream)) == kvc.KVC_OK
+    # the groups' decode equals the whole-cache decode left in obuf
+    assert int(obuf.view(torch.int16).sum(dtype=torch.int64)) == int(before)
+    inb = src.numel() * src.element_size()
+    return {"value": round(job_gbs(raw, world, e2e_ms), 3), "unit": "GB/s",
+            "h2d_bytes_per_step": inb + n_total, "d2h_bytes_per_step": n_total + inb,
+            "ms_per_step": round(e2e_ms, 3), "layer_groups": G,
+            "copies": "uploads and downloads of different layer groups overlap"}
+
+
 def make_input(wname: str, device, rank: int):
     import torch
     from kv_cache_compression_04_b200 import synth
@@ -599,35 +695,7 @@ def main():
     # ------------------------------------------------ end to end via host --
     e2e = None
     if args.e2e_steps > 0:
-        src = (keep.pool if w.paged else keep)
-        h_in = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
-        h_in.copy_(src)
-        h_stream = torch.empty(out.numel(), dtype=torch.uint8, pin_memory=True)
-        h_out = torch.empty(obuf.shape, dtype=obuf.dtype, pin_memory=True)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-        def e2e_step():
-            src.copy_(h_in, non_blocking=True)
-            enc()
-            h_stream[:nbytes].copy_(out[:nbytes], non_blocking=True)
-            out[:nbytes].copy_(h_stream[:nbytes], non_blocking=True)
-            dec(nbytes)
-            h_out.copy_(obuf, non_blocking=True)
-        e2e_step()
-        torch.cuda.synchronize(dev)
-        if dist:
-            dist.barrier()
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0] / args.e2e_steps
-        inb = src.numel() * src.element_size()
-        e2e = {"value": round(job_gbs(raw, world, e2e_ms), 3), "unit": "GB/s",
-               "h2d_bytes_per_step": inb + nbytes, "d2h_bytes_per_step": nbytes + inb,
-               "ms_per_step": round(e2e_ms, 3)}
-        assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+        e2e = run_e2e(args, w, codec, keep, obuf, stream, dev, dist, world, raw)
 
     # ------------------------------------- unfused baseline (fusion gain) --
     # The same compress call as two kernels with the fp32 transformed tensor
