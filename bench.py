@@ -767,9 +767,10 @@ def main():
                      "peak_kind": peak_kind, "traffic": traffic[dom] if traffic else None,
                      "encode_frac": round(enc_gbs / hbm, 4),
                      "decode_frac": round(dec_gbs / hbm, 4)},
-        "gpu_launches": 6 * K,  # encode, finish, compaction (returns at once unless a code chunk
-        # shrank), meta expansion, eliminated-chunk decode (returns at once unless the header
-        # flags such chunks), decode
+        "gpu_launches": 8 * K,  # per step: workspace clear, encode, finish, compaction
+        # (returns at once unless code chunks are stored eliminated); status clear, meta
+        # expansion, eliminated-chunk decode (returns at once unless the header flags such
+        # chunks), decode
         "clocks": clk.summary(),
     }
     if e2e:
