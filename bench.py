@@ -191,7 +191,7 @@ def run_e2e(args, w, codec, keep, obuf, stream, dev, dist, world, raw):
     import kv_cache_compression_04_b200 as kvc
     src = keep.pool if w.paged else keep
     L = src.shape[0]
-    G = min(8, L)
+    G = max(1, min(args.e2e_groups, L))
     bounds = [(L * g // G, L * (g + 1) // G) for g in range(G)]
 
     def desc_of(t):
@@ -602,6 +602,8 @@ def main():
     ap.add_argument("--workload", default="llama8b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-groups", type=int, default=8,
+                    help="layer groups of the end-to-end timing (one call pair each)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--unfused-steps", type=int, default=20)
     ap.add_argument("--sweep", action="store_true")
