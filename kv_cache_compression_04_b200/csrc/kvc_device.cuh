@@ -91,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
 
 // ---------------------------------------------------- bulk-async copies --
 // Tensor-map load of a 5-D box into shared memory, completion counted in
-// bytes on `bar` (no multicast). c0 is the innermost coordinate.
+// bytes on `bar` (this CTA's buffer only). c0 is the innermost coordinate.
 __device__ __forceinline__ void tma_load_5d(void *sdst, const CUtensorMap *map, int c0, int c1,
                                             int c2, int c3, int c4, uint64_t *bar) {
   asm volatile(

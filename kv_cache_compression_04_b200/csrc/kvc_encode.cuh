@@ -11,8 +11,9 @@
 // decided from the number of nonzero bytes its bit-plane shuffle would have,
 // which this kernel accumulates per chunk (chunk_nnz_part's OR-popcount
 // identity); the finishing kernels (kvc_finish.cuh) write the table, the meta
-// chunks and the header, and, only when some chunk shrinks, re-encode and
-// move code chunks. This kernel therefore has no dependency between threads
+// chunks and the header, and, only when some chunk shrinks and storing it
+// eliminated pays for the shift of the later chunks (reading R16), re-encode
+// and move code chunks. This kernel therefore has no dependency between threads
 // beyond the warp reductions of those counts.
 //
 // Work: blocks of 32 consecutive vectors, one per lane; warps are fully
@@ -37,7 +38,6 @@ constexpr int kEncThreads = kEncWarps * 32;
 template <int D, int BITS, int G>
 struct Cfg {
   static constexpr int ROW = D * 2;              // bytes of one bf16 vector
-  static constexpr int ROWP = ROW + 16;          // padded smem row (no bank conflicts)
   static constexpr int CB = D * BITS / 8;        // code bytes per vector
   static constexpr int CW = CB / 4;              // code words per vector
   static constexpr int NG = D / G;               // groups per vector
