@@ -125,6 +125,41 @@ def test_code_elim_rule_in_stream(bits, group, zero_chunk, kept):
     assert not (zero & 0x7FFF).any()                          # +-0 (signs flip zeros)
 
 
+@pytest.mark.parametrize("pattern", range(6))
+def test_code_elim_rule_matches_per_chunk_sizes(pattern):
+    """The stream's code sizes and flag follow from the separately pinned
+    parts: each code chunk's own lossless encoding (raw codes from the
+    quantizer) and the rule on those sizes; random sets of all-zero chunks
+    among 64, some of which keep elimination and some not."""
+    rng = np.random.default_rng(100 + pattern)
+    zeros = sorted(rng.choice(64, size=int(rng.integers(1, 5)), replace=False).tolist())
+    if pattern == 0:
+        zeros = [3]                                           # a long tail: raw
+    if pattern == 1:
+        zeros = [60, 61, 62]                                  # a short tail: kept
+    d, x = _one_zero_chunk(4, 128, zeros[0], seed=20 + pattern)
+    for z in zeros[1:]:
+        x[z * 256:(z + 1) * 256] = 0
+    lay = d.layout()
+    st, codes, _ = oracle.quantize_vectors(x, 4, 128, 0)
+    assert st == oracle.OK
+    lens = [16384] * 64
+    sizes = [oracle.lossless_encode_chunk(codes[c * 256:(c + 1) * 256].reshape(-1)).size
+             for c in range(64)]
+    keep = oracle.code_elim_pays(sizes, lens)
+    st, s = oracle.compress(d, x)
+    assert st == oracle.OK
+    table = np.frombuffer(bytes(s[64:64 + 8 * lay.n_chunks]), "<u8")
+    got = [int(table[oracle.code_chunk_index(lay, c)] & 0xFFFF) for c in range(64)]
+    assert got == (sizes if keep else lens)
+    assert s[11] == int(keep)
+    if pattern == 0:
+        assert not keep
+    if pattern == 1:
+        assert keep
+    assert oracle.decompress(s, d)[0] == oracle.OK
+
+
 @pytest.mark.parametrize("name,n_code,n_meta", [("tiny", 4, 1), ("llama8b", 8192, 512),
                                                 ("qwen7b", 14336, 7168)])
 def test_layout_counts(name, n_code, n_meta):
