@@ -177,13 +177,15 @@ void orc_unpack_codes(const uint8_t *packed, int d, int bits, uint8_t *q) {
     q[c] = (uint8_t)((packed[c / per] >> ((c % per) * bits)) & mask);
 }
 
-/* One code of reading R5: t = fl(y - zf), then the exact real t*r rounded to
- * the nearest integer (ties to even) and clamped to [0, qmax]. t and r are
- * fp32, so their product has at most 48 significant bits and is exact in
- * double; rint() in the default rounding mode is round-half-even. */
+/* One code of reading R5: t = fl(y - zf), p = fl(t * r) (two separate fp32
+ * operations, each rounded to nearest even; the file is built without FMA
+ * contraction), then p rounded to the nearest integer, ties to even, and
+ * clamped to [0, qmax]. nearbyint() in the default rounding mode is
+ * round-half-even, and p is an fp32 value, exact in double. */
 int orc_quantize_scalar(float y, float zf, float r, int qmax) {
   float t = y - zf;
-  double n = nearbyint((double)t * (double)r);
+  float p = t * r;
+  double n = nearbyint((double)p);
   if (n < 0.0) n = 0.0;
   if (n > (double)qmax) n = (double)qmax;
   return (int)n;
@@ -197,9 +199,9 @@ int orc_quantize_scalar(float y, float zf, float r, int qmax) {
 /*   mn, mx = group min and max, then mn+0, mx+0 (so -0 becomes +0);          */
 /*   z_h = RD16(mn * 2^-k),  zf = f32(z_h) * 2^k;                             */
 /*   s32 = (mx - zf) / (2^b - 1),  s_h = RU16(s32 * 2^-k), sf = f32(s_h)*2^k; */
-/*   r = 0 if s_h == 0 else 1/sf;  t = y - zf (one fp32 rounding);         */
-/*   q = clamp(nearest integer to the exact product t*r, ties to even,       */
-/*             0, 2^b - 1): the product is not rounded to fp32 first.        */
+/*   r = 0 if s_h == 0 else 1/sf;  t = y - zf, p = t * r (each one fp32   */
+/*   rounding, no fused multiply-add);                                       */
+/*   q = clamp(nearest integer to p, ties to even, 0, 2^b - 1).              */
 /* Directed rounding makes the grid zf + q*sf cover [mn, mx]. A non-finite y  */
 /* gives NONFINITE; an infinite z_h or s_h gives RANGE (reading R8). The meta */
 /* of group j is 4 bytes: s_h then z_h, little-endian.                        */

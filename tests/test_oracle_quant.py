@@ -122,7 +122,8 @@ def test_quantizer_nearest_grid_and_meta_bounds(d, bits, g):
     """Brute force: with y from the (separately pinned) butterfly, the meta
     brackets each group (z_h <= min/2^k < next16(z_h); s_h the smallest fp16
     >= s32/2^k), and every code is the nearest grid point to y up to the
-    rounding of (y - zf) * r: |y - (zf + q sf)| <= sf/2 * (1 + 2^-20)."""
+    roundings of t = y - zf, r = 1/sf and t * r (each at most half an fp32
+    ulp; t * r < 16): |y - (zf + q sf)| <= sf * (1/2 + 2^-18)."""
     rng = np.random.default_rng(d + bits + g)
     seed = 99
     k = {64: 3, 128: 3, 256: 4}[d]
@@ -150,7 +151,7 @@ def test_quantizer_nearest_grid_and_meta_bounds(d, bits, g):
             qg = q[j * g:(j + 1) * g]
             assert qg.min() >= 0 and qg.max() <= qmax
             err = np.abs(yg - (zf + qg * sf))
-            assert np.all(err <= sf / 2 * (1 + 2.0 ** -20) + 1e-30)
+            assert np.all(err <= sf * (0.5 + 2.0 ** -18) + 1e-30)
 
 
 def test_constant_and_zero_groups():
@@ -209,11 +210,29 @@ def _nearest_even(fr):
     return n
 
 
-def test_quantizer_rounds_the_exact_product():
-    """Reading R5: the code is the nearest integer to the exact real t*r, not
-    to fl32(t*r). Cases are built where t*r lies within half an fp32 ulp of
-    n + 1/2 (so fl32(t*r) is the tie n + 1/2) but not on it; the two readings
-    then differ, and exact rational arithmetic decides."""
+def _f32_product(t, r):
+    """The fp32 product, correctly rounded (IEEE binary32 multiply, round to
+    nearest even), taken from numpy's float32 arithmetic as a library routine
+    and checked here against exact rationals: it is the fp32 value nearest to
+    the exact product."""
+    from fractions import Fraction
+    p = np.float32(t) * np.float32(r)
+    exact = Fraction(float(t)) * Fraction(float(r))
+    lo = Fraction(float(np.nextafter(p, np.float32(-np.inf))))
+    hi = Fraction(float(np.nextafter(p, np.float32(np.inf))))
+    here = Fraction(float(p))
+    assert abs(exact - here) <= abs(exact - lo) and abs(exact - here) <= abs(exact - hi)
+    return here
+
+
+def test_quantizer_rounds_the_fp32_product():
+    """Reading R5 (no fused multiply-add): the code is the nearest integer,
+    ties to even, to p = fl32(t*r), the product rounded to fp32 on its own.
+    Cases are built where the exact t*r lies within half an fp32 ulp of
+    n + 1/2 but not on it, so p is the tie n + 1/2 and goes to the even
+    integer, while the exact product would round the other way half of the
+    time: a quantizer that fuses the product and the rounding (one FMA with
+    a rounding constant) fails here in both directions."""
     from fractions import Fraction
     rng = np.random.default_rng(7)
     found = {"up": 0, "down": 0, "tie": 0}
@@ -224,16 +243,17 @@ def test_quantizer_rounds_the_exact_product():
         n = int(rng.integers(0, qmax))
         t0 = np.float32((n + 0.5) / float(r))
         for t in (np.nextafter(t0, np.float32(-np.inf)), t0, np.nextafter(t0, np.float32(np.inf))):
-            exact = Fraction(float(t)) * Fraction(float(r))
-            want = min(max(_nearest_even(exact), 0), qmax)
+            p = _f32_product(t, r)
+            want = min(max(_nearest_even(p), 0), qmax)
             got = oracle.quantize_scalar(float(t), 0.0, float(r), qmax)
             assert got == want, (float(t), float(r), got, want)
-            sep = int(np.rint(np.float32(t) * np.float32(r)))
-            if exact == Fraction(2 * n + 1, 2):
+            fused = min(max(_nearest_even(Fraction(float(t)) * Fraction(float(r))), 0), qmax)
+            if p == Fraction(2 * n + 1, 2) and fused != want:
+                found["up" if fused > want else "down"] += 1
+            elif p == Fraction(2 * n + 1, 2):
                 found["tie"] += 1
-            elif sep != want:
-                found["up" if want > sep else "down"] += 1
-    # the readings really were separated, in both directions
+    # the fp32-product rule and the exact-product rule really were separated,
+    # in both directions
     assert found["up"] > 0 and found["down"] > 0, found
 
 
