@@ -29,7 +29,7 @@ _HDR = os.path.join(_HERE, "kvc_oracle.h")
 _BUILD = os.path.join(_HERE, "_build")
 _SO = os.path.join(_BUILD, "liboracle.so")
 
-CFLAGS = ["-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+CFLAGS = ["-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-pthread",
           "-Wall", "-Wextra", "-Wno-unused-parameter"]
 
 OK, INVALID_ARG, UNSUPPORTED, CAPACITY, NONFINITE, RANGE, CORRUPT = range(7)
@@ -124,6 +124,10 @@ def lib():
                                            C.c_uint64, u64p]),
                 "orc_decompress": (C.c_int, [u8p, C.c_uint64,
                                              C.POINTER(Desc), u16p]),
+                "orc_compress_mt": (C.c_int, [C.POINTER(Desc), u16p, u8p,
+                                              C.c_uint64, u64p, C.c_int]),
+                "orc_decompress_mt": (C.c_int, [u8p, C.c_uint64,
+                                                C.POINTER(Desc), u16p, C.c_int]),
                 "orc_gather_dense": (None, [u16p, C.c_int, C.c_int, C.c_int64,
                                             C.c_int, C.c_int64, C.c_int64,
                                             C.c_int64, C.c_int64, C.c_uint64,
@@ -322,23 +326,33 @@ def meta_chunk_index(lay: Layout, s: int) -> int:
     return lib().orc_meta_chunk_index(C.byref(lay), s)
 
 
-def compress(desc: StreamDesc, vectors: np.ndarray):
-    """vectors: uint16 [V, d] in logical order -> (status, stream bytes)."""
+def compress(desc: StreamDesc, vectors: np.ndarray, threads: int = 1):
+    """vectors: uint16 [V, d] in logical order -> (status, stream bytes).
+    threads > 1 spreads the per-segment loop over POSIX threads (same bytes).
+    The returned stream is a view of a buffer of the worst-case length."""
     vectors = np.ascontiguousarray(vectors, np.uint16)
     cap = desc.max_bytes()
-    out = np.zeros(cap, np.uint8)
+    out = np.empty(cap, np.uint8)
     n = C.c_uint64(0)
-    st = lib().orc_compress(C.byref(desc.c), _p(vectors, C.c_uint16),
-                            _p(out, C.c_uint8), cap, C.byref(n))
-    return st, out[: n.value].copy()
+    if threads > 1:
+        st = lib().orc_compress_mt(C.byref(desc.c), _p(vectors, C.c_uint16),
+                                   _p(out, C.c_uint8), cap, C.byref(n), int(threads))
+    else:
+        st = lib().orc_compress(C.byref(desc.c), _p(vectors, C.c_uint16),
+                                _p(out, C.c_uint8), cap, C.byref(n))
+    return st, out[: n.value]
 
 
-def decompress(stream: np.ndarray, desc: StreamDesc):
+def decompress(stream: np.ndarray, desc: StreamDesc, threads: int = 1):
     stream = np.ascontiguousarray(stream, np.uint8)
     lay = desc.layout()
-    out = np.zeros((lay.V, desc.head_dim), np.uint16)
-    st = lib().orc_decompress(_p(stream, C.c_uint8), stream.size,
-                              C.byref(desc.c), _p(out, C.c_uint16))
+    out = np.empty((lay.V, desc.head_dim), np.uint16)
+    if threads > 1:
+        st = lib().orc_decompress_mt(_p(stream, C.c_uint8), stream.size,
+                                     C.byref(desc.c), _p(out, C.c_uint16), int(threads))
+    else:
+        st = lib().orc_decompress(_p(stream, C.c_uint8), stream.size,
+                                  C.byref(desc.c), _p(out, C.c_uint16))
     return st, out
 
 

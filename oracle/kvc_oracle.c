@@ -24,6 +24,7 @@
 #include "kvc_oracle.h"
 
 #include <math.h>
+#include <pthread.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -493,42 +494,88 @@ static uint64_t get64(const uint8_t *p) {
   return (uint64_t)get32(p) | ((uint64_t)get32(p + 4) << 32);
 }
 
-int orc_encode_segment(const orc_desc *d, uint64_t s, const uint16_t *vectors,
-                       uint8_t *chunks, uint32_t *sizes, uint32_t *n_out) {
-  orc_layout lay;
+/* Segment s's chunks from its vectors, for a layout computed once by the
+ * caller (orc_encode_segment and the compressor below). */
+static int encode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t s,
+                             const uint16_t *vectors, uint8_t *chunks,
+                             uint32_t *sizes, uint32_t *n_out) {
   uint64_t vm, v0, nv, v, c0, c1, c;
   uint8_t *codes, *meta;
   uint64_t sw[4];
   uint32_t pos = 0;
-  int st = orc_layout_of(d, &lay), vst;
-  if (st != ORC_OK) return st;
-  if (s >= lay.n_seg) return ORC_ERR_INVALID_ARG;
-  vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
+  int st = ORC_OK, vst;
+  vm = (uint64_t)lay->vec_per_code * lay->code_per_seg;
   v0 = s * vm;
-  nv = lay.V - v0 < vm ? lay.V - v0 : vm;
+  nv = lay->V - v0 < vm ? lay->V - v0 : vm;
   orc_sign_words(d->sign_seed, d->head_dim, sw);
-  codes = (uint8_t *)malloc((size_t)(nv * lay.code_bytes));
-  meta = (uint8_t *)malloc((size_t)(nv * lay.meta_bytes));
+  codes = (uint8_t *)malloc((size_t)(nv * lay->code_bytes));
+  meta = (uint8_t *)malloc((size_t)(nv * lay->meta_bytes));
   for (v = 0; v < nv; v++) {
     vst = orc_quantize_vector(vectors + v * d->head_dim, d->head_dim, d->bits,
-                              d->group, sw, codes + v * lay.code_bytes,
-                              meta + v * lay.meta_bytes);
+                              d->group, sw, codes + v * lay->code_bytes,
+                              meta + v * lay->meta_bytes);
     if (vst != ORC_OK && st == ORC_OK) st = vst;
   }
-  c0 = s * lay.code_per_seg;
-  c1 = c0 + lay.code_per_seg < lay.n_code ? c0 + lay.code_per_seg : lay.n_code;
+  c0 = s * lay->code_per_seg;
+  c1 = c0 + lay->code_per_seg < lay->n_code ? c0 + lay->code_per_seg : lay->n_code;
   *n_out = 0;
   for (c = c0; c < c1; c++) {
-    uint64_t a = (c - c0) * lay.vec_per_code;
-    uint64_t b = a + lay.vec_per_code < nv ? a + lay.vec_per_code : nv;
+    uint64_t a = (c - c0) * lay->vec_per_code;
+    uint64_t b = a + lay->vec_per_code < nv ? a + lay->vec_per_code : nv;
     uint32_t sz = orc_lossless_encode_chunk(
-        codes + a * lay.code_bytes, (uint32_t)((b - a) * lay.code_bytes),
+        codes + a * lay->code_bytes, (uint32_t)((b - a) * lay->code_bytes),
         chunks + pos);
     sizes[(*n_out)++] = sz;
     pos += sz;
   }
   sizes[(*n_out)++] =
-      orc_lossless_encode_chunk(meta, (uint32_t)(nv * lay.meta_bytes), chunks + pos);
+      orc_lossless_encode_chunk(meta, (uint32_t)(nv * lay->meta_bytes), chunks + pos);
+  free(codes);
+  free(meta);
+  return st;
+}
+
+int orc_encode_segment(const orc_desc *d, uint64_t s, const uint16_t *vectors,
+                       uint8_t *chunks, uint32_t *sizes, uint32_t *n_out) {
+  orc_layout lay;
+  int st = orc_layout_of(d, &lay);
+  if (st != ORC_OK) return st;
+  if (s >= lay.n_seg) return ORC_ERR_INVALID_ARG;
+  return encode_segment_in(d, &lay, s, vectors, chunks, sizes, n_out);
+}
+
+static int decode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t s,
+                             const uint8_t *chunks, const uint32_t *sizes,
+                             uint16_t *vectors) {
+  uint64_t vm, v0, nv, v, c0, c1, c, i = 0;
+  uint8_t *codes, *meta;
+  uint64_t sw[4];
+  uint32_t pos = 0;
+  int st = ORC_OK;
+  vm = (uint64_t)lay->vec_per_code * lay->code_per_seg;
+  v0 = s * vm;
+  nv = lay->V - v0 < vm ? lay->V - v0 : vm;
+  orc_sign_words(d->sign_seed, d->head_dim, sw);
+  codes = (uint8_t *)malloc((size_t)(nv * lay->code_bytes));
+  meta = (uint8_t *)malloc((size_t)(nv * lay->meta_bytes));
+  c0 = s * lay->code_per_seg;
+  c1 = c0 + lay->code_per_seg < lay->n_code ? c0 + lay->code_per_seg : lay->n_code;
+  for (c = c0; c < c1 && st == ORC_OK; c++, i++) {
+    uint64_t a = (c - c0) * lay->vec_per_code;
+    uint64_t b = a + lay->vec_per_code < nv ? a + lay->vec_per_code : nv;
+    st = orc_lossless_decode_chunk(chunks + pos, sizes[i],
+                                   (uint32_t)((b - a) * lay->code_bytes),
+                                   codes + a * lay->code_bytes);
+    pos += sizes[i];
+  }
+  if (st == ORC_OK)
+    st = orc_lossless_decode_chunk(chunks + pos, sizes[i],
+                                   (uint32_t)(nv * lay->meta_bytes), meta);
+  if (st == ORC_OK)
+    for (v = 0; v < nv; v++)
+      orc_dequantize_vector(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
+                            d->head_dim, d->bits, d->group, sw,
+                            vectors + v * d->head_dim);
   free(codes);
   free(meta);
   return st;
@@ -537,40 +584,52 @@ int orc_encode_segment(const orc_desc *d, uint64_t s, const uint16_t *vectors,
 int orc_decode_segment(const orc_desc *d, uint64_t s, const uint8_t *chunks,
                        const uint32_t *sizes, uint16_t *vectors) {
   orc_layout lay;
-  uint64_t vm, v0, nv, v, c0, c1, c, i = 0;
-  uint8_t *codes, *meta;
-  uint64_t sw[4];
-  uint32_t pos = 0;
   int st = orc_layout_of(d, &lay);
   if (st != ORC_OK) return st;
   if (s >= lay.n_seg) return ORC_ERR_INVALID_ARG;
-  vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
-  v0 = s * vm;
-  nv = lay.V - v0 < vm ? lay.V - v0 : vm;
-  orc_sign_words(d->sign_seed, d->head_dim, sw);
-  codes = (uint8_t *)malloc((size_t)(nv * lay.code_bytes));
-  meta = (uint8_t *)malloc((size_t)(nv * lay.meta_bytes));
-  c0 = s * lay.code_per_seg;
-  c1 = c0 + lay.code_per_seg < lay.n_code ? c0 + lay.code_per_seg : lay.n_code;
-  for (c = c0; c < c1 && st == ORC_OK; c++, i++) {
-    uint64_t a = (c - c0) * lay.vec_per_code;
-    uint64_t b = a + lay.vec_per_code < nv ? a + lay.vec_per_code : nv;
-    st = orc_lossless_decode_chunk(chunks + pos, sizes[i],
-                                   (uint32_t)((b - a) * lay.code_bytes),
-                                   codes + a * lay.code_bytes);
-    pos += sizes[i];
+  return decode_segment_in(d, &lay, s, chunks, sizes, vectors);
+}
+
+/* Runs fn(job, s) for every segment s in [0, n_seg) on n_threads threads
+ * (segment s on thread s mod n_threads; 1 thread: the caller, in order).
+ * Segments are independent, so the order does not change any result. */
+typedef struct {
+  void *job;
+  void (*fn)(void *job, uint64_t s);
+  uint64_t first, n_seg, step;
+} seg_pool_part;
+
+static void *seg_pool_run(void *arg) {
+  seg_pool_part *p = (seg_pool_part *)arg;
+  uint64_t s;
+  for (s = p->first; s < p->n_seg; s += p->step) p->fn(p->job, s);
+  return NULL;
+}
+
+static void for_each_segment(uint64_t n_seg, int n_threads, void *job,
+                             void (*fn)(void *job, uint64_t s)) {
+  pthread_t th[ORC_MAX_THREADS];
+  seg_pool_part part[ORC_MAX_THREADS];
+  int t, started = 0;
+  if (n_threads < 1) n_threads = 1;
+  if (n_threads > ORC_MAX_THREADS) n_threads = ORC_MAX_THREADS;
+  if ((uint64_t)n_threads > n_seg) n_threads = n_seg ? (int)n_seg : 1;
+  for (t = 0; t < n_threads; t++) {
+    part[t].job = job;
+    part[t].fn = fn;
+    part[t].first = (uint64_t)t;
+    part[t].n_seg = n_seg;
+    part[t].step = (uint64_t)n_threads;
   }
-  if (st == ORC_OK)
-    st = orc_lossless_decode_chunk(chunks + pos, sizes[i],
-                                   (uint32_t)(nv * lay.meta_bytes), meta);
-  if (st == ORC_OK)
-    for (v = 0; v < nv; v++)
-      orc_dequantize_vector(codes + v * lay.code_bytes, meta + v * lay.meta_bytes,
-                            d->head_dim, d->bits, d->group, sw,
-                            vectors + v * d->head_dim);
-  free(codes);
-  free(meta);
-  return st;
+  for (t = 1; t < n_threads; t++)
+    if (pthread_create(&th[t], NULL, seg_pool_run, &part[t]) == 0) started = t;
+    else break;
+  /* threads that could not start leave their segments to this thread */
+  if (started + 1 < n_threads) {
+    for (t = started + 1; t < n_threads; t++) seg_pool_run(&part[t]);
+  }
+  seg_pool_run(&part[0]);
+  for (t = 1; t <= started; t++) pthread_join(th[t], NULL);
 }
 
 /* Reading R16 (the encoder's choice for the code region; a decoder accepts
@@ -597,14 +656,52 @@ int orc_code_elim_pays(const uint32_t *sizes, const uint32_t *lens, uint64_t n_c
   return seen && 64 * S >= T;
 }
 
+/* One segment of the compressor: its chunks go to the store slots of their
+ * stream chunk indices. */
+typedef struct {
+  const orc_desc *d;
+  const orc_layout *lay;
+  const uint16_t *vectors;
+  uint8_t *store;
+  uint32_t *all_sizes;
+  uint64_t *where;
+  int *seg_status;
+} enc_job;
+
+static void enc_one_segment(void *arg, uint64_t s) {
+  enc_job *j = (enc_job *)arg;
+  const orc_layout *lay = j->lay;
+  uint64_t vm = (uint64_t)lay->vec_per_code * lay->code_per_seg;
+  uint8_t *seg = (uint8_t *)malloc((size_t)(lay->code_per_seg + 1) * ORC_CHUNK);
+  uint32_t sizes[17], n, k, pos = 0;
+  j->seg_status[s] = encode_segment_in(j->d, lay, s, j->vectors + s * vm * j->d->head_dim,
+                                       seg, sizes, &n);
+  for (k = 0; k < n; k++) {
+    uint64_t idx = (k + 1 < n) ? orc_code_chunk_index(lay, s * lay->code_per_seg + k)
+                               : orc_meta_chunk_index(lay, s);
+    memcpy(j->store + idx * ORC_CHUNK, seg + pos, sizes[k]);
+    j->all_sizes[idx] = sizes[k];
+    j->where[idx] = idx * ORC_CHUNK;
+    pos += sizes[k];
+  }
+  free(seg);
+}
+
 int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
                  uint64_t capacity, uint64_t *out_bytes) {
+  return orc_compress_mt(d, vectors, out, capacity, out_bytes, 1);
+}
+
+int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
+                    uint64_t capacity, uint64_t *out_bytes, int n_threads) {
   orc_layout lay;
-  uint64_t s, off = 0, T = 0, vm, i;
-  uint8_t *seg, *store;
-  uint32_t sizes[17], n, k, *all_sizes;
+  uint64_t s, off = 0, T = 0, i;
+  uint8_t *store;
+  uint32_t *all_sizes;
   uint64_t *where; /* chunk index -> position in store */
-  int st = orc_layout_of(d, &lay), sst, r;
+  int *seg_status;
+  enc_job job;
+  int st = orc_layout_of(d, &lay), r;
   if (st != ORC_OK) return st;
   if (capacity < lay.max_bytes) return ORC_ERR_CAPACITY;
   for (r = 0; r < d->n_requests; r++) T += d->token_lens[r];
@@ -628,24 +725,22 @@ int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
   for (r = 0; r < d->n_requests; r++)
     put32(out + ORC_HEADER + 8 * lay.n_chunks + 4 * r, d->token_lens[r]);
   /* encode every segment, remembering where each chunk's bytes are */
-  vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
-  seg = (uint8_t *)malloc((size_t)(lay.code_per_seg + 1) * ORC_CHUNK);
   store = (uint8_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1) * ORC_CHUNK);
   all_sizes = (uint32_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1) * 4);
   where = (uint64_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1) * 8);
-  for (s = 0; s < lay.n_seg; s++) {
-    uint32_t pos = 0;
-    sst = orc_encode_segment(d, s, vectors + s * vm * d->head_dim, seg, sizes, &n);
-    if (sst != ORC_OK && st == ORC_OK) st = sst;
-    for (k = 0; k < n; k++) {
-      uint64_t idx = (k + 1 < n) ? orc_code_chunk_index(&lay, s * lay.code_per_seg + k)
-                                 : orc_meta_chunk_index(&lay, s);
-      memcpy(store + idx * ORC_CHUNK, seg + pos, sizes[k]);
-      all_sizes[idx] = sizes[k];
-      where[idx] = idx * ORC_CHUNK;
-      pos += sizes[k];
-    }
-  }
+  seg_status = (int *)malloc((size_t)(lay.n_seg ? lay.n_seg : 1) * sizeof(int));
+  job.d = d;
+  job.lay = &lay;
+  job.vectors = vectors;
+  job.store = store;
+  job.all_sizes = all_sizes;
+  job.where = where;
+  job.seg_status = seg_status;
+  for_each_segment(lay.n_seg, n_threads, &job, enc_one_segment);
+  /* the first error in segment order wins */
+  for (s = 0; s < lay.n_seg; s++)
+    if (seg_status[s] != ORC_OK && st == ORC_OK) st = seg_status[s];
+  free(seg_status);
   /* reading R16: keep elimination in the code region only if it pays for
      the shift of the code chunks after the first shrinking one */
   if (lay.n_code) {
@@ -690,7 +785,6 @@ int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
       break;
     }
   }
-  free(seg);
   free(store);
   free(all_sizes);
   free(where);
@@ -699,12 +793,49 @@ int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
   return st;
 }
 
+/* One segment of the decompressor: its chunks are gathered from the stream
+ * by the (already validated) chunk table and decoded. */
+typedef struct {
+  const orc_desc *d;
+  const orc_layout *lay;
+  const uint8_t *stream;
+  uint16_t *vectors;
+  int *seg_status;
+} dec_job;
+
+static void dec_one_segment(void *arg, uint64_t s) {
+  dec_job *j = (dec_job *)arg;
+  const orc_layout *lay = j->lay;
+  uint64_t vm = (uint64_t)lay->vec_per_code * lay->code_per_seg;
+  uint64_t c0 = s * lay->code_per_seg;
+  uint64_t c1 = c0 + lay->code_per_seg < lay->n_code ? c0 + lay->code_per_seg : lay->n_code;
+  uint64_t i, k = 0;
+  uint32_t pos = 0, sizes[17];
+  uint8_t *seg = (uint8_t *)malloc((size_t)(lay->code_per_seg + 1) * ORC_CHUNK);
+  for (i = c0; i <= c1; i++, k++) { /* code chunks c0..c1-1, then the meta chunk */
+    uint64_t idx = i < c1 ? orc_code_chunk_index(lay, i) : orc_meta_chunk_index(lay, s);
+    uint64_t e = get64(j->stream + ORC_HEADER + 8 * idx);
+    uint32_t sz = (uint32_t)(e & 0xFFFFu);
+    memcpy(seg + pos, j->stream + lay->data_base + (e >> 16) * 16, sz);
+    sizes[k] = sz;
+    pos += sz;
+  }
+  j->seg_status[s] = decode_segment_in(j->d, lay, s, seg, sizes,
+                                       j->vectors + s * vm * j->d->head_dim);
+  free(seg);
+}
+
 int orc_decompress(const uint8_t *stream, uint64_t stream_bytes,
                    const orc_desc *expect, uint16_t *vectors) {
+  return orc_decompress_mt(stream, stream_bytes, expect, vectors, 1);
+}
+
+int orc_decompress_mt(const uint8_t *stream, uint64_t stream_bytes,
+                      const orc_desc *expect, uint16_t *vectors, int n_threads) {
   orc_layout lay;
-  uint64_t s, T = 0, vm, expect_off = 0, total;
-  uint8_t *seg;
-  uint32_t sizes[17];
+  uint64_t s, T = 0, expect_off = 0, total;
+  int *seg_status;
+  dec_job job;
   int st = orc_layout_of(expect, &lay), r;
   if (st != ORC_OK) return st;
   if (stream_bytes < ORC_HEADER) return ORC_ERR_CORRUPT;
@@ -745,24 +876,17 @@ int orc_decompress(const uint8_t *stream, uint64_t stream_bytes,
         nv * lay.code_bytes)
       return ORC_ERR_CORRUPT;
   }
-  vm = (uint64_t)lay.vec_per_code * lay.code_per_seg;
-  seg = (uint8_t *)malloc((size_t)(lay.code_per_seg + 1) * ORC_CHUNK);
-  for (s = 0; s < lay.n_seg && st == ORC_OK; s++) {
-    uint64_t c0 = s * lay.code_per_seg;
-    uint64_t c1 = c0 + lay.code_per_seg < lay.n_code ? c0 + lay.code_per_seg : lay.n_code;
-    uint64_t i, k = 0;
-    uint32_t pos = 0;
-    for (i = c0; i <= c1; i++, k++) { /* code chunks c0..c1-1, then the meta chunk */
-      uint64_t idx = i < c1 ? orc_code_chunk_index(&lay, i) : orc_meta_chunk_index(&lay, s);
-      uint64_t e = get64(stream + ORC_HEADER + 8 * idx);
-      uint32_t sz = (uint32_t)(e & 0xFFFFu);
-      memcpy(seg + pos, stream + lay.data_base + (e >> 16) * 16, sz);
-      sizes[k] = sz;
-      pos += sz;
-    }
-    st = orc_decode_segment(expect, s, seg, sizes, vectors + s * vm * expect->head_dim);
-  }
-  free(seg);
+  seg_status = (int *)malloc((size_t)(lay.n_seg ? lay.n_seg : 1) * sizeof(int));
+  job.d = expect;
+  job.lay = &lay;
+  job.stream = stream;
+  job.vectors = vectors;
+  job.seg_status = seg_status;
+  for_each_segment(lay.n_seg, n_threads, &job, dec_one_segment);
+  /* the first error in segment order wins */
+  for (s = 0; s < lay.n_seg; s++)
+    if (seg_status[s] != ORC_OK && st == ORC_OK) st = seg_status[s];
+  free(seg_status);
   if (st == ORC_OK && lay.data_base + expect_off != total) st = ORC_ERR_CORRUPT;
   return st;
 }

@@ -122,6 +122,16 @@ int orc_compress(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
 int orc_decompress(const uint8_t *stream, uint64_t stream_bytes,
                    const orc_desc *expect, uint16_t *vectors);
 
+/* The same two calls with their per-segment loop spread over n_threads
+ * POSIX threads (segment s on thread s mod n_threads). Segments are
+ * independent and every result is placed by its segment index, so the
+ * output and status equal the single-thread calls'. */
+#define ORC_MAX_THREADS 256
+int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
+                    uint64_t capacity, uint64_t *out_bytes, int n_threads);
+int orc_decompress_mt(const uint8_t *stream, uint64_t stream_bytes,
+                      const orc_desc *expect, uint16_t *vectors, int n_threads);
+
 /* ---- layouts: logical vector order [layer][kv][head][request][token] ------ */
 void orc_gather_dense(const uint16_t *base, int layers, int kv_heads,
                       int64_t tokens, int d, int64_t s_layer, int64_t s_kv,

@@ -314,3 +314,43 @@ def test_gather_paged_matches_python_walk():
     out = oracle.gather_paged(pool.reshape(-1), 2, 2, 64, pk.strides(), 16, w.seq_lens,
                               pt, 0, len(ref))
     assert np.array_equal(out, ref)
+
+
+@pytest.mark.parametrize("threads", [2, 3, 8])
+def test_threaded_oracle_equals_single_thread(threads):
+    """The thread-pool compress/decompress (the per-segment loop spread over
+    POSIX threads) give the single-thread calls' bytes and status: a mixed
+    lognormal input with all-zero stretches (eliminated code and meta chunks,
+    reading R16 both ways), a ragged tail, and more segments than threads."""
+    w = synth.Workload("m", 3, 2, 128, 2, 32, seed=5, kind="lognormal", scale_sigma=1.5,
+                       tokens=1500)
+    x = synth.bf16_bits(synth.dense_kv(w)).reshape(-1, 128).copy()
+    x[4000:6200] = 0
+    for bits, g in [(2, 32), (4, 64), (4, 128)]:
+        d = oracle.StreamDesc(bits, g, 128, 3, 2, [1500], 7)
+        st1, s1 = oracle.compress(d, x)
+        stn, sn = oracle.compress(d, x, threads=threads)
+        assert st1 == stn == oracle.OK and np.array_equal(s1, sn)
+        dst1, x1 = oracle.decompress(s1, d)
+        dstn, xn = oracle.decompress(s1, d, threads=threads)
+        assert dst1 == dstn == oracle.OK and np.array_equal(x1, xn)
+
+
+def test_threaded_oracle_first_error_in_segment_order():
+    """With errors in several segments the threaded call reports the one of
+    the lowest segment, as the single-thread loop does: RANGE in segment 1,
+    NONFINITE in segment 3 -> RANGE; swapped -> NONFINITE."""
+    d = oracle.StreamDesc(4, 128, 128, 1, 1, [2048 * 4], 0)
+    lay = d.layout()
+    assert lay.n_seg == 4
+    s0 = -1 if oracle.sign_words(0, 128)[0] & 1 else 1     # sign of channel 0
+    big = np.float32(-s0 * 655360.0).view(np.uint32) >> 16   # one-hot -> RANGE
+    for rng_seg, nan_seg, want in [(1, 3, oracle.RANGE), (3, 1, oracle.NONFINITE)]:
+        x = np.zeros((lay.V, 128), np.uint16)
+        v0, _ = oracle.segment_vectors(lay, rng_seg)
+        x[v0, 0] = big
+        v1, _ = oracle.segment_vectors(lay, nan_seg)
+        x[v1, 5] = 0x7FC0
+        st1, s1 = oracle.compress(d, x)
+        st4, s4 = oracle.compress(d, x, threads=4)
+        assert st1 == st4 == want and np.array_equal(s1, s4)
