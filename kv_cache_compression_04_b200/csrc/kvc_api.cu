@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include "kvc_internal.h"
+#include "../../include/kvc_test.h"
 
 using namespace kvc;
 
@@ -220,7 +221,8 @@ namespace {
 // transformed vectors in the workspace after the compress workspace.
 kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *out,
                          size_t out_capacity, uint64_t *out_bytes_dev, void *workspace,
-                         size_t workspace_bytes, kvc_stream_t stream, bool unfused) {
+                         size_t workspace_bytes, kvc_stream_t stream, bool unfused,
+                         uint32_t ticket_skip = 0, uint64_t wait_ns = kWaitNs) {
   Shape s;
   if (!params) return KVC_ERR_INVALID_ARG;
   kvc_status st = describe(kv, params, s);
@@ -247,6 +249,7 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   a.meta_nnz = reinterpret_cast<uint32_t *>(ws + w.meta_nnz);
   a.ws_meta = ws + w.meta;
   a.ymid = unfused ? reinterpret_cast<float *>(ws + round256(s.ws_bytes)) : nullptr;
+  a.one = 1.0f;
   sign_masks(params->sign_seed, s.D, a.sign_mask);
 
   FinArgs f{};
@@ -284,6 +287,8 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   f.n_req = s.n_req;
   f.tokens = s.T;
   f.seed = params->sign_seed;
+  f.wait_ns = wait_ns;
+  f.ticket_skip = ticket_skip;
 
   if (clear_words(ws, w.zero_bytes, sms, cs) != cudaSuccess) return KVC_ERR_CUDA;
   cudaError_t e = cudaSuccess;
@@ -327,6 +332,16 @@ kvc_status kvc_compress_unfused(const kvc_kv_desc *kv, const kvc_params *params,
                                 size_t workspace_bytes, kvc_stream_t stream) {
   return compress_impl(kv, params, out, out_capacity, out_bytes_dev, workspace, workspace_bytes,
                        stream, true);
+}
+
+kvc_status kvc_test_compress_stalled(const kvc_kv_desc *kv, const kvc_params *params, void *out,
+                                     size_t out_capacity, uint64_t *out_bytes_dev,
+                                     void *workspace, size_t workspace_bytes,
+                                     uint32_t skip_chunks, uint64_t wait_ns,
+                                     kvc_stream_t stream) {
+  if (skip_chunks == 0 || wait_ns == 0 || wait_ns > kWaitNs) return KVC_ERR_INVALID_ARG;
+  return compress_impl(kv, params, out, out_capacity, out_bytes_dev, workspace, workspace_bytes,
+                       stream, false, skip_chunks, wait_ns);
 }
 
 kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *out,

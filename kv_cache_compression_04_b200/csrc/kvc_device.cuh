@@ -11,14 +11,6 @@
 
 namespace kvc {
 
-// Every device wait is bounded: after this many nanoseconds of %globaltimer
-// (or the iteration cap) the waiter records KVC_ERR_TIMEOUT and goes on. A
-// recorded timeout is sticky: every other wait of the call sees it in the
-// status word and gives up at once, so a failed call ends within about one
-// wait limit.
-constexpr uint64_t kWaitNs = 1000000000ull;
-constexpr uint32_t kWaitIters = 1u << 26;
-
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -47,10 +39,11 @@ __device__ __forceinline__ bool timed_out(const uint32_t *status) {
 }
 // Poll step of a bounded spin: true means give up (time, iterations, or a
 // timeout already recorded by another waiter). Checks every 64 iterations.
-__device__ __forceinline__ bool spin_expired(uint32_t it, uint64_t t0, const uint32_t *status) {
+__device__ __forceinline__ bool spin_expired(uint32_t it, uint64_t t0, const uint32_t *status,
+                                             uint64_t limit_ns = kWaitNs) {
   if (it >= kWaitIters) return true;
   if ((it & 63u) != 63u) return false;
-  return globaltimer() - t0 > kWaitNs || timed_out(status);
+  return globaltimer() - t0 > limit_ns || timed_out(status);
 }
 
 // ---------------------------------------------------------------- mbarrier --
@@ -199,16 +192,18 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
   return bits_f2(r);
 }
-// a*b + c with one rounding. Used only where a*b is exact, so the result
-// equals the separately rounded product-then-sum.
+// a*b + c with one rounding. Used only where a*b is exact (a small integer
+// times an fp16 value, or a value times 1.0), so the result equals the
+// separately rounded product-then-sum.
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   uint64_t r;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
   return bits_f2(r);
 }
 // Measured on sm_100a: a paired multiply followed by a paired add can be
-// fused even when both carry .rn, so no product that needs its own rounding
-// feeds an add here; products are rounded to integers with cvt.rni instead.
+// fused, so no product that needs its own rounding feeds an add here; the
+// quantizer rounds its product to an integer with a multiply-add by a
+// run-time 1.0 instead (kvc_encode.cuh).
 // min / max that return NaN if any input is NaN.
 __device__ __forceinline__ float min3n(float a, float b, float c) {
   float d;

@@ -171,21 +171,26 @@ struct Enc : Cfg<D, BITS, G> {
   }
 
   // E3..E7. Reading R5: asymmetric min/max group quantization, fp16 zero
-  // (round down) and scale (round up), both x 2^-K; q = nearest integer to
-  // the exact t * r with t = fl(y - zf), by one fused multiply-add with
-  // 1.5 * 2^23, which leaves q in the low bits of the sum (the sum lies in
-  // [2^23, 2^24), where the fp32 spacing is 1, and 1.5 * 2^23 is even, so
-  // ties go to even q). The clamp to [0, 2^b - 1] never acts for a finite
-  // group: t >= 0 since zf <= min, and sf >= (max - zf) / (2^b - 1) keeps
-  // t * r below 2^b - 1 + 2^-20. Codes pack LSB first (reading R6).
+  // (round down) and scale (round up), both x 2^-K; t = fl(y - zf),
+  // p = fl(t * r), q = nearest integer to p, ties to even, each step rounded
+  // on its own (no fused multiply-add). The integer rounding is
+  // fl(p * one + 1.5 * 2^23) with `one` = 1.0 passed in at run time: p * 1
+  // is exact, so this is the rounded sum p + 1.5 * 2^23, which leaves q in
+  // the low bits (the sum lies in [2^23, 2^24), where the fp32 spacing is 1,
+  // and 1.5 * 2^23 is even, so ties go to even q). Because that operation is
+  // itself a multiply-add whose multiplier the compiler cannot see, the
+  // product t * r before it can never be contracted into it. The clamp to
+  // [0, 2^b - 1] never acts for a finite group: t >= 0 since zf <= min, and
+  // sf >= (max - zf) / (2^b - 1) keeps p below 2^b - 1 + 2^-18. Codes pack
+  // LSB first (reading R6).
   static __device__ __forceinline__ uint32_t vector(Pairs<D> &y, uint32_t (&code)[C::CW],
-                                                    uint32_t (&meta)[C::NG]) {
+                                                    uint32_t (&meta)[C::NG], float one) {
     fwht_pairs<D>(y);
-    return quantize(y, code, meta);
+    return quantize(y, code, meta, one);
   }
   // E4..E7 on the transformed vector.
   static __device__ __forceinline__ uint32_t quantize(Pairs<D> &y, uint32_t (&code)[C::CW],
-                                                      uint32_t (&meta)[C::NG]) {
+                                                      uint32_t (&meta)[C::NG], float one) {
     uint32_t err = 0;
     float zf[C::NG], rr[C::NG];
 #pragma unroll
@@ -207,12 +212,13 @@ struct Enc : Cfg<D, BITS, G> {
       meta[g] = uint32_t(sb) | (uint32_t(zb) << 16);
     }
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-    const float2 mag = make_float2(kMagic, kMagic);
+    const float2 mag = make_float2(kMagic, kMagic), one2 = make_float2(one, one);
 #pragma unroll
     for (int j = 0; j < D / 2; ++j) {
       const int ga = j / G, gb = (j + D / 2) / G;
       const float2 t = sub2(y.p[j], make_float2(zf[ga], zf[gb]));
-      y.p[j] = fma2(t, make_float2(rr[ga], rr[gb]), mag);
+      const float2 p = mul2(t, make_float2(rr[ga], rr[gb]));
+      y.p[j] = fma2(p, one2, mag);
     }
     constexpr int per = 8 / BITS;  // codes per byte
 #pragma unroll
@@ -245,9 +251,9 @@ __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t b
   uint32_t code[C::CW], meta[C::NG];
   if (valid) {
     if constexpr (kFwht)
-      err |= E::vector(y, code, meta);
+      err |= E::vector(y, code, meta, a.one);
     else
-      err |= E::quantize(y, code, meta);
+      err |= E::quantize(y, code, meta, a.one);
     uint4 *cd = reinterpret_cast<uint4 *>(a.out + a.data_base + uint64_t(v) * C::CB);
 #pragma unroll
     for (int q = 0; q < C::CW / 4; ++q)

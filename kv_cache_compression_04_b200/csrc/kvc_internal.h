@@ -29,6 +29,14 @@ constexpr uint32_t kMagic = 0x3143564Bu;  // "KVC1"
 constexpr int kThreads = 256;   // compute threads per CTA (one vector each)
 constexpr uint32_t kNoTile = 0xFFFFFFFFu;
 
+// Every device wait is bounded: after this many nanoseconds of %globaltimer
+// (or the iteration cap) the waiter records KVC_ERR_TIMEOUT and goes on. A
+// recorded timeout is sticky: every other wait of the call sees it in the
+// status word and gives up at once, so a failed call ends within about one
+// wait limit.
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t kWaitIters = 1u << 26;
+
 // Workspace of kvc_compress, in this order (each part 256-byte aligned):
 //   control   status word, flags word (bit 0: some code chunk shrank),
 //             compaction ticket, compaction read count, ~(first shrinking
@@ -145,6 +153,7 @@ struct EncArgs {
   uint32_t *meta_nnz;
   uint8_t *ws_meta;
   float *ymid;         // unfused baseline only: transformed vectors, d fp32 each
+  float one;           // 1.0: the quantizer's integer rounding multiplies by it
   uint32_t sign_mask[128];
 };
 
@@ -172,6 +181,11 @@ struct FinArgs {
   // header fields
   uint32_t layers, kv_heads, head_dim, group, bits, k, origin, n_req;
   uint64_t tokens, seed;
+  // compaction waits give up after wait_ns (kWaitNs in every product call);
+  // ticket_skip > 0 (a test of that limit only) starts the compaction's
+  // tickets that many chunks late, so those chunks' read flags are never set
+  uint64_t wait_ns;
+  uint32_t ticket_skip;
 };
 
 struct DecArgs {
