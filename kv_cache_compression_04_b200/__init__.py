@@ -28,7 +28,7 @@ STATUS = ["KVC_OK", "KVC_ERR_INVALID_ARG", "KVC_ERR_UNSUPPORTED", "KVC_ERR_CAPAC
 EXPORTS = ["kvc_max_compressed_bytes", "kvc_workspace_bytes", "kvc_compress",
            "kvc_decompress", "kvc_stream_status", "kvc_status_string", "kvc_compress_noalloc",
            "kvc_decompress_workspace_bytes", "kvc_unfused_workspace_bytes",
-           "kvc_compress_unfused"]
+           "kvc_compress_unfused", "kvc_test_compress_stalled"]
 
 
 class KvcError(RuntimeError):
@@ -89,6 +89,10 @@ def lib() -> C.CDLL:
         L.kvc_compress_unfused.restype = C.c_int
         L.kvc_compress_unfused.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p,
                                            C.c_size_t, C.c_void_p]
+        L.kvc_test_compress_stalled.restype = C.c_int
+        L.kvc_test_compress_stalled.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p,
+                                                C.c_void_p, C.c_size_t, C.c_uint32, C.c_uint64,
+                                                C.c_void_p]
         _lib = L
     return _lib
 
@@ -126,6 +130,15 @@ def kvc_compress_noalloc(desc, params, out_ptr, out_capacity, out_bytes_dev_ptr,
                          stream) -> int:
     return lib().kvc_compress_noalloc(C.byref(desc), C.byref(params), out_ptr, out_capacity,
                                       out_bytes_dev_ptr, status_dev_ptr, stream)
+
+
+def kvc_test_compress_stalled(desc, params, out_ptr, out_capacity, out_bytes_dev_ptr, ws_ptr,
+                              ws_bytes, skip_chunks, wait_ns, stream) -> int:
+    """Test-only (include/kvc_test.h): kvc_compress whose compaction skips
+    `skip_chunks` chunks and gives up its waits after `wait_ns`."""
+    return lib().kvc_test_compress_stalled(C.byref(desc), C.byref(params), out_ptr, out_capacity,
+                                           out_bytes_dev_ptr, ws_ptr, ws_bytes, skip_chunks,
+                                           wait_ns, stream)
 
 
 def kvc_decompress(in_ptr, in_bytes, desc, ws_ptr, ws_bytes, stream) -> int:

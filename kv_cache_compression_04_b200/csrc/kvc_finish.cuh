@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
 #pragma unroll 1
   while (true) {
     named_bar_sync(1, NT);
-    const uint32_t c = c0 + ctl->tick;
+    const uint32_t c = c0 + a.ticket_skip + ctl->tick;
     named_bar_sync(1, NT);
     if (c >= a.n_code) break;
     if (tid == 0) ctl->tick = atomicAdd(a.ticket, 1u);
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
       for (uint32_t j = j0 + tid; j <= j1 && j < c; j += NT) {
         const uint64_t t0 = globaltimer();
         for (uint32_t it = 0; *reinterpret_cast<volatile uint32_t *>(a.done + j) == 0; ++it) {
-          if (spin_expired(it, t0, a.status)) {
+          if (spin_expired(it, t0, a.status, a.wait_ns)) {
             set_status(a.status, KVC_ERR_TIMEOUT);
             break;
           }
@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
   if (tid == 0) {
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0; *reinterpret_cast<volatile uint32_t *>(a.ticket + 1) < a.n_code - c0; ++it) {
-      if (spin_expired(it, t0, a.status)) {
+      if (spin_expired(it, t0, a.status, a.wait_ns)) {
         set_status(a.status, KVC_ERR_TIMEOUT);
         break;
       }

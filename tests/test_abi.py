@@ -24,8 +24,11 @@ def L():
 
 
 def test_exports_every_declared_symbol(L):
-    with open(os.path.join(ROOT, "include", "kvc.h")) as f:
-        hdr = f.read()
+    import glob
+    hdr = ""
+    for path in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))):
+        with open(path) as f:
+            hdr += f.read()
     declared = set(re.findall(r"\b(kvc_[a-z_]+)\s*\(", hdr))
     assert declared == set(kvc.EXPORTS)
     for name in declared:

@@ -177,3 +177,45 @@ def test_status_is_cleared_per_call():
     kv[0, 0, 0, 0, 0] = float("nan")
     assert gpu_compress(kvc.dense_desc(kv.cuda()), 4, 128)[0] == kvc.KVC_ERR_NONFINITE
     assert gpu_compress(kvc.dense_desc(_kv().cuda()), 4, 128)[0] == kvc.KVC_OK
+
+
+def test_compaction_wait_runs_out_to_timeout():
+    """A bounded device wait that runs out ends the call with KVC_ERR_TIMEOUT
+    and leaves the context usable. The test entry point starts the
+    compaction's tickets one chunk late, so the first shrinking code chunk is
+    never read and its read flag never set; the next chunk stores into that
+    chunk's slot and waits for the flag, which runs out after 1 ms. Writes stay
+    inside the output buffer (guard bytes after it intact), and an ordinary
+    compress on the same stream afterwards still matches the oracle."""
+    L, H, T, D = 2, 4, 4096, 128
+    g = torch.Generator().manual_seed(21)
+    x = torch.randn(L, 2, H, T, D, generator=g)
+    blocks = x.view(L, 2, H, T // 256, 256, D)
+    zero = torch.rand(L, 2, H, T // 256, generator=g) < 0.5
+    blocks[zero] = 0
+    kv = x.to(torch.bfloat16).cuda()
+    desc = kvc.dense_desc(kv)
+    p = kvc.params(4, 128, 0)
+    cap = kvc.kvc_max_compressed_bytes(desc, p)
+    wsb = kvc.kvc_workspace_bytes(desc, p)
+    out = torch.full((cap + 4096,), 0xA5, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    nb = torch.zeros(1, dtype=torch.int64, device="cuda")
+    sp = kvc._stream_ptr(None)
+    # invalid hook arguments are refused before anything runs
+    for skip, ns in [(0, 10**6), (1, 0), (1, 2 * 10**9)]:
+        assert kvc.kvc_test_compress_stalled(desc, p, out.data_ptr(), cap, nb.data_ptr(),
+                                             ws.data_ptr(), wsb, skip, ns,
+                                             sp) == kvc.KVC_ERR_INVALID_ARG
+    st = kvc.kvc_test_compress_stalled(desc, p, out.data_ptr(), cap, nb.data_ptr(),
+                                       ws.data_ptr(), wsb, 1, 10**6, sp)
+    assert st == kvc.KVC_OK
+    assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_ERR_TIMEOUT
+    assert torch.all(out[cap:] == 0xA5), "a write went past the output buffer"
+    # the context is still usable: the ordinary call gives the oracle's stream
+    st, gstream, _, _ = gpu_compress(desc, 4, 128)
+    assert st == kvc.KVC_OK
+    od = oracle.StreamDesc(4, 128, D, L, H, [T], 0)
+    ost, ostream = oracle.compress(od, u16(kv.cpu()).reshape(-1, D))
+    assert ost == oracle.OK and ostream[11] == 1       # code chunks stored eliminated
+    assert np.array_equal(gstream, ostream)
