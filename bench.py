@@ -43,18 +43,30 @@ FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_llama8b.txt")
 
 
+def strip_c_comments(text: str) -> str:
+    """C/C++ source without its comments and with runs of white space
+    collapsed, so that a comment-only edit leaves the digest below unchanged
+    (string literals are kept whole)."""
+    import re
+    tok = re.compile(r'"(?:\\.|[^"\\])*"|/\*.*?\*/|//[^\n]*', re.S)
+    code = tok.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", text)
+    return " ".join(code.split())
+
+
 def kernel_source_sha() -> str:
-    """Digest of the CUDA sources and the ABI header (a recorded DRAM-traffic
-    figure is stale once any of them changed)."""
+    """Digest of the CUDA sources and the ABI headers without their comments
+    (a recorded DRAM-traffic figure is stale once any code in them changed)."""
     import glob
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kv_cache_compression_04_b200", "csrc")
     files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
-                   glob.glob(os.path.join(csrc, "*.h"))) + [os.path.join(ROOT, "include", "kvc.h")]
+                   glob.glob(os.path.join(csrc, "*.h"))) + sorted(
+                       glob.glob(os.path.join(ROOT, "include", "*.h")))
     for f in files:
-        with open(f, "rb") as fh:
-            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" +
+                     strip_c_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -459,15 +471,73 @@ def run_sweep(args):
     return 0
 
 
-def run_pipeline(args):
-    """Layer-pipelined transfer of the llama8b cache: layer l is compressed on
+class LayerPipeline:
+    """Layer-pipelined transfer of a dense KV cache: layer l is compressed on
     one stream, held on a 'wire' stream for its stream bytes / link speed (a
-    spin of that many SM cycles at the sampled clock), then decompressed on a
+    spin of that many SM cycles at the given clock), then decompressed on a
     third stream into the receiver's cache, so compression, transfer and
-    decompression of different layers overlap. Compared with sending the raw
-    bf16 cache over the same link. The receiver's cache is checked against a
-    whole-cache round trip (decoding is per vector, so the chunking does not
-    change it)."""
+    decompression of different layers overlap. One kvc_compress and one
+    kvc_decompress call per layer, each with its own buffers."""
+
+    def __init__(self, kv, rx, codec, dev):
+        import torch
+        import kv_cache_compression_04_b200 as kvc
+        self.kvc, self.torch, self.dev, self.codec = kvc, torch, dev, codec
+        self.L = kv.shape[0]
+        self.descs = [kvc.dense_desc(kv[l:l + 1]) for l in range(self.L)]
+        self.odescs = [kvc.dense_desc(rx[l:l + 1]) for l in range(self.L)]
+        self.bufs = [codec.buffers(d, dev) for d in self.descs]
+        self.dws = [torch.empty(kvc.kvc_decompress_workspace_bytes(d), dtype=torch.uint8,
+                                device=dev) for d in self.odescs]
+        self.se, self.sw, self.sd = (torch.cuda.Stream(dev) for _ in range(3))
+        self.pe, self.pd = kvc._stream_ptr(self.se), kvc._stream_ptr(self.sd)
+        for l in range(self.L):
+            self.enc(l)
+        torch.cuda.synchronize(dev)
+        self.n = [int(b[2].item()) for b in self.bufs]
+
+    def enc(self, l):
+        out, ws, nb = self.bufs[l]
+        assert self.kvc.kvc_compress(self.descs[l], self.codec.params, out.data_ptr(),
+                                     out.numel(), nb.data_ptr(), ws.data_ptr(), ws.numel(),
+                                     self.pe) == self.kvc.KVC_OK
+
+    def dec(self, l):
+        out = self.bufs[l][0]
+        assert self.kvc.kvc_decompress(out.data_ptr(), self.n[l], self.odescs[l],
+                                       self.dws[l].data_ptr(), self.dws[l].numel(),
+                                       self.pd) == self.kvc.KVC_OK
+
+    def transfer(self, link_bytes_per_s: float, sm_hz: float) -> float:
+        """One pipelined transfer; returns its CUDA-event time in ms."""
+        torch = self.torch
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(self.se)
+        for l in range(self.L):
+            self.enc(l)
+            e1 = torch.cuda.Event()
+            e1.record(self.se)
+            self.sw.wait_event(e1)
+            with torch.cuda.stream(self.sw):
+                torch.cuda._sleep(int(self.n[l] / link_bytes_per_s * sm_hz))
+            e2 = torch.cuda.Event()
+            e2.record(self.sw)
+            self.sd.wait_event(e2)
+            self.dec(l)
+        t1.record(self.sd)
+        torch.cuda.synchronize(self.dev)
+        return t0.elapsed_time(t1)
+
+    def statuses_ok(self) -> bool:
+        return all(self.kvc.kvc_stream_status(d.data_ptr(), self.pd) == self.kvc.KVC_OK
+                   for d in self.dws)
+
+
+def run_pipeline(args):
+    """Layer-pipelined transfer of the llama8b cache over a simulated 100 and
+    400 Gbit/s link (LayerPipeline), compared with sending the raw bf16 cache
+    over the same link. The receiver's cache is checked against a whole-cache
+    round trip (decoding is per vector, so the chunking does not change it)."""
     import torch
     import kv_cache_compression_04_b200 as kvc
     from kv_cache_compression_04_b200 import build, synth
@@ -479,30 +549,11 @@ def run_pipeline(args):
     rx = torch.empty_like(kv)
     codec = kvc.Codec(w.bits, w.group, w.sign_seed)
     L = w.layers
-    descs = [kvc.dense_desc(kv[l:l + 1]) for l in range(L)]
-    odescs = [kvc.dense_desc(rx[l:l + 1]) for l in range(L)]
-    bufs = [codec.buffers(d, dev) for d in descs]
-    dws = [torch.empty(kvc.kvc_decompress_workspace_bytes(d), dtype=torch.uint8, device=dev)
-           for d in odescs]
-    se, sw, sd = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    pe, pdd = kvc._stream_ptr(se), kvc._stream_ptr(sd)
-
-    def enc(l):
-        out, ws, nb = bufs[l]
-        assert kvc.kvc_compress(descs[l], codec.params, out.data_ptr(), out.numel(),
-                                nb.data_ptr(), ws.data_ptr(), ws.numel(), pe) == kvc.KVC_OK
-
-    def dec(l, n):
-        out = bufs[l][0]
-        assert kvc.kvc_decompress(out.data_ptr(), n, odescs[l], dws[l].data_ptr(),
-                                  dws[l].numel(), pdd) == kvc.KVC_OK
-
-    for l in range(L):
-        enc(l)
-    torch.cuda.synchronize(dev)
-    n = [int(b[2].item()) for b in bufs]
+    pipe = LayerPipeline(kv, rx, codec, dev)
+    n = pipe.n
     # whole-cache reference for the receiver's check
     ref = torch.empty_like(kv)
+    se = pipe.se
     with torch.cuda.stream(se):
         cout, cws, cnb = codec.buffers(kvc.dense_desc(kv), dev)
         sp = kvc._stream_ptr(se)
@@ -531,13 +582,13 @@ def run_pipeline(args):
     for rep in range(args.warmup + 3):
         te[0].record(se)
         for l in range(L):
-            enc(l)
+            pipe.enc(l)
             te[l + 1].record(se)
         torch.cuda.synchronize(dev)
-        td[0].record(sd)
+        td[0].record(pipe.sd)
         for l in range(L):
-            dec(l, n[l])
-            td[l + 1].record(sd)
+            pipe.dec(l)
+            td[l + 1].record(pipe.sd)
         torch.cuda.synchronize(dev)
         if rep >= args.warmup:
             for l in range(L):
@@ -549,25 +600,10 @@ def run_pipeline(args):
         for rep in range(args.warmup + 3):
             rx.zero_()
             torch.cuda.synchronize(dev)
-            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            t0.record(se)
-            for l in range(L):
-                enc(l)
-                e1 = torch.cuda.Event()
-                e1.record(se)
-                sw.wait_event(e1)
-                with torch.cuda.stream(sw):
-                    torch.cuda._sleep(int(n[l] / link * sm_hz))
-                e2 = torch.cuda.Event()
-                e2.record(sw)
-                sd.wait_event(e2)
-                dec(l, n[l])
-            t1.record(sd)
-            torch.cuda.synchronize(dev)
+            ms = pipe.transfer(link, sm_hz)
             if rep >= args.warmup:
-                times.append(t0.elapsed_time(t1))
-        for l in range(L):
-            assert kvc.kvc_stream_status(dws[l].data_ptr(), pdd) == kvc.KVC_OK
+                times.append(ms)
+        assert pipe.statuses_ok()
         assert torch.equal(rx.view(torch.int16), ref.view(torch.int16))
         pipe_ms = statistics.median(times)
         raw_ms = w.raw_bytes / link * 1e3

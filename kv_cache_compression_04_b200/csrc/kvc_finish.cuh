@@ -78,6 +78,11 @@ __device__ __forceinline__ uint32_t meta_stored_size(const FinArgs &a, uint32_t 
 // least 1/64 of the padded bytes from the first shrinking code chunk to the
 // region's end, the bytes the compaction would move. Otherwise every code
 // chunk stays raw where the encode kernel wrote it.
+// Both kernels that call this read the encode kernel's counters after
+// grid_dependency_wait(), which returns only once the encode kernel (and the
+// kernels before it) has completed and its memory operations, atomics
+// included, are visible to this grid; plain volatile loads then see the final
+// values, so no acquire ordering is needed here.
 __device__ __forceinline__ bool code_elim_kept(const FinArgs &a, uint32_t flags) {
   if (!(flags & 1u) || a.n_code == 0) return false;
   const uint32_t c0 = ~*reinterpret_cast<const volatile uint32_t *>(a.first_inv);
