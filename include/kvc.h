@@ -121,10 +121,19 @@ typedef struct {
 
 /* Exact worst-case stream length for this shape and these parameters: the
  * header and tables plus every chunk at its raw length, each rounded up to
- * 16 bytes. Host only, pure; returns 0 for an invalid description. */
+ * 16 bytes. Host only, pure; returns 0 for an invalid description.
+ * Source: no page defines a size bound; it follows from the lossless stage
+ * keeping a chunk raw whenever coding would not shorten it ("Beyond
+ * Compression Ratio: High-Throughput KV Compression for Disaggregated LLM
+ * Serving", Methodology: the LC-based backend of composed primitives), so the
+ * stream never exceeds the quantized payload plus its tables. */
 size_t kvc_max_compressed_bytes(const kvc_kv_desc *kv, const kvc_params *params);
 
-/* Workspace bytes kvc_compress needs for this shape (DEVICE memory, 16-byte
+/* (No page defines the workspace calls and the status read below: they
+ * exist because this library allocates nothing and reports data-dependent
+ * errors from the device.)
+ *
+ * Workspace bytes kvc_compress needs for this shape (DEVICE memory, 16-byte
  * aligned, caller-owned, contents need not be initialized). Returns 0 for an
  * invalid description. */
 size_t kvc_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params);
@@ -137,7 +146,16 @@ size_t kvc_workspace_bytes(const kvc_kv_desc *kv, const kvc_params *params);
  * for an invalid description. */
 size_t kvc_decompress_workspace_bytes(const kvc_kv_desc *out);
 
-/* Compresses `kv` into `out` (DEVICE, out_capacity bytes, which must be at
+/* Source of the operation: "Beyond Compression Ratio: High-Throughput KV
+ * Compression for Disaggregated LLM Serving", Abstract and Methodology (the
+ * distribution transformation and the low-bit quantization fused in one
+ * kernel with no intermediate tensor, then the LC-based lossless backend);
+ * podcast page "FastKVComp: checking whether high-throughput KV compression
+ * pays off", episode notes (the stages are a randomized Hadamard transform,
+ * low-bit quantization and a lossless codec; the prefill side compresses the
+ * cache before it crosses the link to the decode GPU).
+ *
+ * Compresses `kv` into `out` (DEVICE, out_capacity bytes, which must be at
  * least kvc_max_compressed_bytes). The stream length is written to the
  * header's stream_bytes field and, if out_bytes_dev (DEVICE) is not null, to
  * *out_bytes_dev. Stream layout (little-endian): 64-byte header; u64 chunk
@@ -158,7 +176,14 @@ kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params,
                         void *workspace, size_t workspace_bytes,
                         kvc_stream_t stream);
 
-/* Decompresses the stream at `in` (DEVICE, in_bytes readable bytes) into the
+/* Source of the operation: podcast page "FastKVComp: checking whether
+ * high-throughput KV compression pays off", episode notes (the decode GPU
+ * receives the compressed cache; encode plus decode time is what the wire
+ * time saved must exceed; only the quantization loses information, so the
+ * decoder inverts the lossless codec exactly and the transform up to the
+ * quantization error).
+ *
+ * Decompresses the stream at `in` (DEVICE, in_bytes readable bytes) into the
  * slots described by `out`; workspace_bytes must be at least
  * kvc_decompress_workspace_bytes(out). Bits, group size and sign seed come from the
  * stream. The logical shape must match the stream's: layers, kv_heads,
@@ -200,10 +225,13 @@ const char *kvc_status_string(kvc_status status);
  *    about 16 KB per 16 KB of meta (fp16 scale and zero per group), so 16 MiB
  *    holds e.g. 32 layers x 8 kv_heads x 4096 tokens x head_dim 128 at group
  *    128 (8.1 MiB), not at group 64 (16.1 MiB).
- *  - Set-up. The first call on each device (with that device current) looks
- *    up the block's device address once and keeps it; make that first call
- *    before any stream capture on the device. A failed look-up returns
- *    KVC_ERR_CUDA.
+ *  - Set-up. The first call in each CUDA context (per device, with that
+ *    device current) looks up the block's device address and keeps it for
+ *    that context; later calls in the same context only compare the current
+ *    context's ID with the kept one. After a device reset (a new primary
+ *    context) the next call looks the address up again. Make the first call
+ *    in a context before any stream capture on the device. A failed look-up
+ *    returns KVC_ERR_CUDA.
  *  - Status. If status_dev (DEVICE, 4 bytes, 4-byte aligned) is not null, the
  *    call's status word is copied there on `stream` after the encode; pass
  *    status_dev to kvc_stream_status() to read it.

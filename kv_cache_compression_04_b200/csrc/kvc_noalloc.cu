@@ -1,10 +1,12 @@
 // kvc_compress_noalloc: kvc_compress with its workspace in this file's static
 // device block instead of caller memory. Nothing here allocates: the block is
-// part of the module image, its address is looked up once per device with
-// cudaGetSymbolAddress, and kvc_compress clears the part of it that must
-// start at zero on the caller's stream.
+// part of the module image, its address is looked up with
+// cudaGetSymbolAddress once per CUDA context (a context's address stays valid
+// for its lifetime), and kvc_compress clears the part of it that must start
+// at zero on the caller's stream.
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/kvc.h"
@@ -15,17 +17,47 @@ __device__ __align__(256) uint8_t g_noalloc_scratch[KVC_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
+// Per device: the context the address was looked up in (by its process-unique
+// ID, so a context created after a device reset never matches an old entry,
+// even if it reuses the old handle value) and the address.
+unsigned long long g_ctx_id[kMaxDevices];
 void *g_scratch_ptr[kMaxDevices];
 
-// Device address of the block on the current device (looked up once).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+template <class Fn>
+Fn driver_fn(const char *name) {
+  void *p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Device address of the block in the current context (looked up again
+// whenever the current context is not the one of the cached address).
 kvc_status scratch_ptr(void **p) {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return KVC_ERR_CUDA;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVC_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return KVC_ERR_CUDA;
+  if (!ctx) {  // no context current in this thread yet: cudaSetDevice makes the primary one so
+    if (cudaSetDevice(dev) != cudaSuccess || get_current(&ctx) != CUDA_SUCCESS || !ctx)
+      return KVC_ERR_CUDA;
+  }
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return KVC_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || g_ctx_id[dev] != id) {
     void *q = nullptr;
     if (cudaGetSymbolAddress(&q, g_noalloc_scratch) != cudaSuccess || !q) return KVC_ERR_CUDA;
     g_scratch_ptr[dev] = q;
+    g_ctx_id[dev] = id;
   }
   *p = g_scratch_ptr[dev];
   return KVC_OK;

@@ -6,8 +6,11 @@ operation sequence with round-to-nearest-even and no contraction).
 
 Sizes: small shapes that still span several tiles, segments and a ragged tail
 (oracle in seconds), structured inputs that exercise zero-byte elimination,
-and the full-size workloads in the benchmark's launch configuration (full
-comparison for llama8b, sampled segments for qwen7b and the paged batch)."""
+and every full-size workload in the benchmark's launch configuration (llama8b,
+qwen7b, the paged batch and all 26 points of the message-size sweep), each
+compared whole: every stream byte and every decoded value."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -285,130 +288,134 @@ def test_structured_head_dim_64(kind, bits, g):
 
 
 # ----------------------------------------------------------- full workloads --
-def _segment_check(w, od, gstream, x_of_range, segs):
-    """Compare the chunks of sampled segments with the oracle's, and the table's
-    offsets with the prefix sum of padded sizes."""
-    lay = od.layout()
-    sizes, offs = chunk_table(gstream, lay.n_chunks)
-    padded = (sizes + 15) // 16 * 16
-    assert np.array_equal(offs[1:], np.cumsum(padded)[:-1]) and offs[0] == 0
-    assert gstream.size == lay.data_base + offs[-1] + padded[-1]
-    for s in segs:
-        v0, v1 = oracle.segment_vectors(lay, s)
-        st, chunks = oracle.encode_segment(od, s, x_of_range(v0, v1))
-        assert st == oracle.OK
-        idx = [oracle.code_chunk_index(lay, s * lay.code_per_seg + i)
-               for i in range(len(chunks) - 1)] + [oracle.meta_chunk_index(lay, s)]
-        for ch, ci in zip(chunks, idx):
-            assert sizes[ci] == ch.size, (s, ci)
-            a = lay.data_base + offs[ci]
-            assert np.array_equal(gstream[a:a + ch.size], ch), (s, ci)
-    return sizes, offs
+# Whole streams and whole decodes at the benchmark's sizes, in its launch
+# configuration, against the oracle's thread pool over segments (the same
+# bytes as its single-thread calls). Host memory is checked first: a full
+# comparison holds the input, the oracle's stream and its decode on the host.
+THREADS = max(1, min(os.cpu_count() or 1, 128))
+
+
+def _need_host_ram(nbytes: int):
+    import psutil
+    avail = psutil.virtual_memory().available
+    if avail < nbytes:
+        pytest.skip(f"needs {nbytes / 2**30:.1f} GiB of free host memory, "
+                    f"{avail / 2**30:.1f} GiB available")
+
+
+def _compare_decode(out_rows, ox, piece=1 << 22):
+    """out_rows(a, b) -> uint16 [b - a, d] of the GPU decode; ox the oracle's."""
+    V = ox.shape[0]
+    for a in range(0, V, piece):
+        b = min(V, a + piece)
+        got = out_rows(a, b)
+        if not np.array_equal(got, ox[a:b]):
+            i = int(np.flatnonzero((got != ox[a:b]).any(axis=1))[0])
+            raise AssertionError(f"decoded vector {a + i} differs from the oracle's")
+
+
+def _full_dense(w):
+    """GPU stream == oracle stream, and GPU decode of it == oracle decode,
+    over the whole tensor."""
+    _need_host_ram(int(w.raw_bytes * 2.2))
+    kv = synth.dense_kv(w, device="cuda")
+    x = u16(kv).reshape(-1, w.head_dim)
+    od = oracle_desc(w.bits, w.group, w.head_dim, w.layers, w.kv_heads, [w.tokens])
+    st, gstream, gbuf, n = gpu_compress(kvc.dense_desc(kv), w.bits, w.group)
+    assert st == kvc.KVC_OK
+    ost, ostream = oracle.compress(od, x, threads=THREADS)
+    assert ost == oracle.OK
+    assert np.array_equal(gstream, ostream), first_diff(gstream, ostream, od.layout())
+    del x, gstream
+    out = torch.empty_like(kv)
+    del kv
+    assert gpu_decompress(gbuf, kvc.dense_desc(out), n) == kvc.KVC_OK
+    dst, ox = oracle.decompress(ostream, od, threads=THREADS)
+    assert dst == oracle.OK
+    flat = out.view(-1, w.head_dim)
+    _compare_decode(lambda a, b: u16(flat[a:b]), ox)
+    del out, flat, gbuf
+    torch.cuda.empty_cache()
+    return ostream
 
 
 def test_full_llama8b():
-    w = synth.workload("llama8b")
-    kv = synth.dense_kv(w, device="cuda")
-    x = u16(kv).reshape(-1, 128)
-    od = oracle_desc(w.bits, w.group, 128, w.layers, w.kv_heads, [w.tokens])
-    st, gstream, _, _ = gpu_compress(kvc.dense_desc(kv), w.bits, w.group)
-    assert st == kvc.KVC_OK
-    ost, ostream = oracle.compress(od, x)
-    assert np.array_equal(gstream, ostream), first_diff(gstream, ostream, od.layout())
-    out = torch.empty_like(kv)
-    assert gpu_decompress(gstream, kvc.dense_desc(out)) == kvc.KVC_OK
-    lay = od.layout()
-    got = u16(out).reshape(-1, 128)
-    for s in [0, 1, 77, 255, lay.n_seg - 1]:
-        v0, v1 = oracle.segment_vectors(lay, s)
-        _, chunks = oracle.encode_segment(od, s, x[v0:v1])
-        dst, ref = oracle.decode_segment(od, s, chunks, v1 - v0)
-        assert dst == oracle.OK and np.array_equal(got[v0:v1], ref), s
+    _full_dense(synth.workload("llama8b"))
 
 
-def test_full_qwen7b_sampled():
-    w = synth.workload("qwen7b")
-    kv = synth.dense_kv(w, device="cuda")
-    flat = kv.view(-1, 128)
-    od = oracle_desc(w.bits, w.group, 128, w.layers, w.kv_heads, [w.tokens])
-    st, gstream, _, _ = gpu_compress(kvc.dense_desc(kv), w.bits, w.group)
-    assert st == kvc.KVC_OK
-    lay = od.layout()
-    rng = np.random.default_rng(0)
-    segs = sorted({0, 1, int(lay.n_seg) - 1, *rng.integers(0, lay.n_seg, 12).tolist()})
-    _segment_check(w, od, gstream, lambda a, b: u16(flat[a:b]), segs)
-    out = torch.empty_like(kv)
-    assert gpu_decompress(gstream, kvc.dense_desc(out)) == kvc.KVC_OK
-    oflat = out.view(-1, 128)
-    for s in segs[:6]:
-        v0, v1 = oracle.segment_vectors(lay, s)
-        _, chunks = oracle.encode_segment(od, s, u16(flat[v0:v1]))
-        _, ref = oracle.decode_segment(od, s, chunks, v1 - v0)
-        assert np.array_equal(u16(oflat[v0:v1]), ref), s
+def test_full_qwen7b():
+    _full_dense(synth.workload("qwen7b"))
 
 
-def test_full_paged_sampled():
-    w = synth.workload("paged")
-    pk = synth.paged_kv(w, device="cuda")
-    seq = w.seq_lens
-    od = oracle_desc(w.bits, w.group, 128, w.layers, w.kv_heads, seq, origin=1)
-    st, gstream, _, _ = gpu_compress(kvc.paged_desc(pk.pool, pk.page_table, seq), w.bits,
-                                     w.group)
-    assert st == kvc.KVC_OK
-    lay = od.layout()
-    # logical vectors of a range via torch indexing (independent of both sides)
-    cum = np.concatenate([[0], np.cumsum(seq)])
+def _paged_rows(pk, w, cum):
+    """Logical vectors [a, b) of a paged pool by torch indexing on the GPU
+    (independent of both codecs)."""
     T = int(cum[-1])
     pt = pk.page_table
+    cum_d = torch.tensor(cum, device=pt.device)
 
     def rows(a, b):
-        v = torch.arange(a, b, device="cuda")
+        v = torch.arange(a, b, device=pt.device)
         lkh, u = v // T, v % T
-        r = torch.searchsorted(torch.tensor(cum[1:], device="cuda"), u, right=True)
-        t = u - torch.tensor(cum, device="cuda")[r]
-        page = pt[r, t // 16].long()
+        r = torch.searchsorted(cum_d[1:], u, right=True)
+        t = u - cum_d[r]
+        page = pt[r, t // w.page_tokens].long()
         lk, h = lkh // w.kv_heads, lkh % w.kv_heads
-        return u16(pk.pool[lk // 2, page, lk % 2, h, t % 16])
+        return u16(pk.pool[lk // 2, page, lk % 2, h, t % w.page_tokens])
+    return rows
 
-    rng = np.random.default_rng(1)
-    segs = sorted({0, int(lay.n_seg) - 1, *rng.integers(0, lay.n_seg, 10).tolist()})
-    _segment_check(w, od, gstream, rows, segs)
+
+def test_full_paged():
+    """The paged batch (80 layers, 16 ragged requests, shuffled page table) at
+    full size: the whole stream against the oracle's, then the whole decode
+    into a second, differently shuffled page table against the oracle's
+    decode, with every slot outside the requests left untouched."""
+    w = synth.workload("paged")
+    _need_host_ram(int(w.raw_bytes * 2.4))
+    pk = synth.paged_kv(w, device="cuda")
+    seq = w.seq_lens
+    cum = np.concatenate([[0], np.cumsum(seq)]).astype(np.int64)
+    od = oracle_desc(w.bits, w.group, 128, w.layers, w.kv_heads, seq, origin=1)
+    st, gstream, gbuf, n = gpu_compress(kvc.paged_desc(pk.pool, pk.page_table, seq), w.bits,
+                                        w.group)
+    assert st == kvc.KVC_OK
+    rows = _paged_rows(pk, w, cum)
+    x = np.empty((w.vectors, 128), np.uint16)
+    for a in range(0, w.vectors, 1 << 22):
+        b = min(w.vectors, a + (1 << 22))
+        x[a:b] = rows(a, b)
+    ost, ostream = oracle.compress(od, x, threads=THREADS)
+    assert ost == oracle.OK
+    assert np.array_equal(gstream, ostream), first_diff(gstream, ostream, od.layout())
+    del x, gstream
+    # decode into a second pool with another page table, pre-filled with a canary
+    pool_shape, n_pages = pk.pool.shape, pk.pool.shape[1]
     del pk
+    torch.cuda.empty_cache()
+    pt2 = synth.page_table_for(seq, 16, n_pages, 4321, device="cuda")
+    pool2 = torch.full(pool_shape, 1.5, dtype=torch.bfloat16, device="cuda")
+    assert gpu_decompress(gbuf, kvc.paged_desc(pool2, pt2, seq), n) == kvc.KVC_OK
+    del gbuf
+    dst, ox = oracle.decompress(ostream, od, threads=THREADS)
+    assert dst == oracle.OK
+    pk2 = synth.PagedKV(pool2, pt2, seq)
+    _compare_decode(_paged_rows(pk2, w, cum), ox)
+    # slots that belong to no request still hold the canary
+    used = torch.zeros(n_pages, 16, dtype=torch.bool, device="cuda")
+    for r, ln in enumerate(seq):
+        t = torch.arange(ln, device="cuda")
+        used[pt2[r, t // 16].long(), t % 16] = True
+    for l in range(w.layers):
+        sl = pool2[l].permute(0, 3, 1, 2, 4)[~used]           # [unused slots, 2, H, d]
+        assert torch.all(sl == 1.5), f"decode wrote an unused slot in layer {l}"
+    del pool2, pk2
     torch.cuda.empty_cache()
 
 
 # -------------------------------------------------------------------- sweep --
 @pytest.mark.parametrize("bits", [4, 2])
-@pytest.mark.parametrize("i", [0, 2, 5])
-def test_sweep_small_sizes_full(i, bits):
-    """Message-size sweep, small end (T = 8 * 2^i tokens): whole streams and
-    whole decodes compared."""
-    w = synth.workload(f"sweep-{i}-{bits}")
-    kv = synth.dense_kv(w, device="cuda")
-    _roundtrip_dense(kv, w.bits, w.group)
-
-
-@pytest.mark.parametrize("bits", [4, 2])
-def test_sweep_largest_size_sampled(bits):
-    """Message-size sweep, 4 GiB end (T = 32768): chunk table consistency over
-    the whole stream, sampled segments against the oracle, sampled decode."""
-    w = synth.workload(f"sweep-12-{bits}")
-    kv = synth.dense_kv(w, device="cuda")
-    flat = kv.view(-1, 128)
-    od = oracle_desc(w.bits, w.group, 128, w.layers, w.kv_heads, [w.tokens])
-    st, gstream, _, _ = gpu_compress(kvc.dense_desc(kv), w.bits, w.group)
-    assert st == kvc.KVC_OK
-    lay = od.layout()
-    rng = np.random.default_rng(12 + bits)
-    segs = sorted({0, int(lay.n_seg) - 1, *rng.integers(0, lay.n_seg, 6).tolist()})
-    _segment_check(w, od, gstream, lambda a, b: u16(flat[a:b]), segs)
-    out = torch.empty_like(kv)
-    assert gpu_decompress(gstream, kvc.dense_desc(out)) == kvc.KVC_OK
-    oflat = out.view(-1, 128)
-    for s in segs[:3]:
-        v0, v1 = oracle.segment_vectors(lay, s)
-        _, chunks = oracle.encode_segment(od, s, u16(flat[v0:v1]))
-        _, ref = oracle.decode_segment(od, s, chunks, v1 - v0)
-        assert np.array_equal(u16(oflat[v0:v1]), ref), s
-    del kv, out, flat, oflat
-    torch.cuda.empty_cache()
+@pytest.mark.parametrize("i", list(range(13)))
+def test_sweep_full(i, bits):
+    """Message-size sweep, every point (T = 8 * 2^i tokens, 1 MiB .. 4 GiB):
+    whole streams and whole decodes compared."""
+    _full_dense(synth.workload(f"sweep-{i}-{bits}"))
