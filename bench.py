@@ -1,6 +1,9 @@
 """Throughput of the B200 KV-cache codec: one step = fused encode + fused decode
-of one synthetic KV cache resident in HBM (Llama-3-8B shape by default:
-[32, 2, 8, 4096, 128] bf16, 4-bit, group 128).
+of one synthetic KV cache resident in HBM. The headline workload is the
+largest single-GPU configuration, the paged ragged batch (80 layers x 2 x 8
+heads x d128, 16 requests of 512..8192 tokens in 16-token pages placed by a
+shuffled page table, 4-bit, group 64); Llama-3-8B- and Qwen-7B-shaped caches
+and the message-size sweep are timed the same way under `per_config`.
 
 Prints ONE JSON line (rank 0):
   value      raw bf16 bytes per second of encode + decode, all ranks (GB/s)
@@ -40,7 +43,8 @@ METRIC = "encode/decode GB/s of raw bf16 KV on 1 B200 and % of HBM roofline; rat
 FALLBACK_HBM_GBS = 6650.0
 
 
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_llama8b.txt")
+def traffic_file(workload: str) -> str:
+    return os.path.join(ROOT, "profiles", f"dram_traffic_{workload}.txt")
 
 
 def strip_c_comments(text: str) -> str:
@@ -74,7 +78,7 @@ def recorded_traffic(workload: str):
     """DRAM bytes per compress / decompress call from the committed ncu
     summary, or None if it is missing, for another workload, or stale."""
     try:
-        with open(TRAFFIC_FILE) as f:
+        with open(traffic_file(workload)) as f:
             kv = dict(l.split(":", 1) for l in f.read().splitlines() if ":" in l and not l.startswith("#"))
         kv = {k.strip(): v.strip() for k, v in kv.items()}
         if kv.get("source_sha") != kernel_source_sha() or kv.get("workload") != workload:
@@ -318,10 +322,38 @@ def describe(w) -> str:
 
 
 # ------------------------------------------------------------ CPU oracle --
-def oracle_sample(wname: str, budget_s: float, seed_offset: int = 0):
-    """Round trip of whole segments through the CPU oracle until `budget_s`
-    of CPU time is spent. Returns (raw bytes processed, seconds, segments)."""
-    import numpy as np
+def host_cpu():
+    """(logical CPUs, CPU model name) of this host."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+def _sample_vectors(w, n, g):
+    """n vectors drawn like the workload's keys (per-channel lognormal scales;
+    Student-t values for the outlier workload), as bf16 bits."""
+    import torch
+    from kv_cache_compression_04_b200 import synth
+    x = torch.randn(n, w.head_dim, generator=g)
+    if w.kind == "lognormal":
+        x = x * torch.exp(w.scale_sigma * torch.randn(1, w.head_dim, generator=g))
+    return synth.bf16_bits(x.to(torch.bfloat16))
+
+
+def oracle_sample(wname: str, budget_s: float, threads: int = 1, seed_offset: int = 0):
+    """Round trips through the CPU oracle, as it stands, on vectors drawn like
+    the workload's, until `budget_s` seconds are spent. One thread: whole
+    segments one at a time (encode_segment + decode_segment). More threads:
+    batches of `threads` x 4 segments through the oracle's thread pool
+    (compress + decompress of a stream of that many segments). Returns (raw
+    bytes processed, seconds, segments)."""
     import torch
     import oracle
     from kv_cache_compression_04_b200 import synth
@@ -332,33 +364,60 @@ def oracle_sample(wname: str, budget_s: float, seed_offset: int = 0):
     vm = lay.vec_per_code * lay.code_per_seg
     g = torch.Generator().manual_seed(w.seed + seed_offset)
     done_bytes, spent, segs = 0, 0.0, 0
-    while spent < budget_s and segs < lay.n_seg:
-        # a segment of vectors drawn with the workload's key distribution
-        x = torch.randn(vm, w.head_dim, generator=g) * torch.exp(
-            w.scale_sigma * torch.randn(1, w.head_dim, generator=g))
-        x = synth.bf16_bits(x.to(torch.bfloat16))
+    if threads <= 1:
+        while spent < budget_s and segs < lay.n_seg:
+            x = _sample_vectors(w, vm, g)
+            t0 = time.perf_counter()
+            st, chunks, pipes = oracle.encode_segment(od, segs, x)
+            _, y = oracle.decode_segment(od, segs, chunks, vm, pipes)
+            spent += time.perf_counter() - t0
+            done_bytes += x.nbytes
+            segs += 1
+        return done_bytes, spent, segs
+    nseg = 4 * threads
+    # a stream of nseg whole segments: one layer, one head, K and V
+    bd = oracle.StreamDesc(w.bits, w.group, w.head_dim, 1, 1, [nseg * vm // 2])
+    assert bd.layout().n_seg == nseg
+    x = _sample_vectors(w, nseg * vm, g)
+    while spent < budget_s:
         t0 = time.perf_counter()
-        st, chunks = oracle.encode_segment(od, segs, x)
-        _, y = oracle.decode_segment(od, segs, chunks, vm)
+        st, stream = oracle.compress(bd, x, threads=threads)
+        dst, y = oracle.decompress(stream, bd, threads=threads)
         spent += time.perf_counter() - t0
+        assert st == oracle.OK and dst == oracle.OK
         done_bytes += x.nbytes
-        segs += 1
+        segs += nseg
     return done_bytes, spent, segs
+
+
+def cpu_baseline(wname: str, budget_s: float):
+    """The oracle on this host: one thread, and every logical CPU."""
+    n, model = host_cpu()
+    b1, s1, n1 = oracle_sample(wname, budget_s / 2, threads=1)
+    bn, sn, nn = oracle_sample(wname, budget_s / 2, threads=n) if n > 1 else (b1, s1, n1)
+    return {"value": round(bn / sn / 1e9, 6), "unit": "GB/s", "cores": n, "kind": "oracle",
+            "sample": f"{nn} whole segments ({bn} raw bytes) of vectors drawn like {wname}'s, "
+                      f"encode + decode through the oracle's thread pool over segments, "
+                      f"{n} threads",
+            "single_thread": {"value": round(b1 / s1 / 1e9, 6), "unit": "GB/s", "cores": 1,
+                              "sample": f"{n1} whole segments ({b1} raw bytes), one at a time"},
+            "cpu_model": model, "host_logical_cpus": n}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    n, model = host_cpu()
     per_step = max(0.5, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(args.workload, per_step / 4)
+        oracle_sample(args.workload, per_step / 4, threads=n)
     tot_b, tot_s, segs = 0, 0.0, 0
     for _ in range(args.steps):
-        b, s, n = oracle_sample(args.workload, per_step)
+        b, s, k = oracle_sample(args.workload, per_step, threads=n)
         tot_b += b
         tot_s += s
-        segs += n
+        segs += k
     from kv_cache_compression_04_b200 import synth
     w = synth.workload(args.workload)
     v = tot_b / tot_s / 1e9
@@ -367,10 +426,11 @@ def run_reference(args):
             "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": describe(w), "sample": f"{segs} segments"},
-            "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "cores": 1,
-                             "kind": "oracle",
-                             "sample": f"{segs} whole segments of {args.workload} vectors, "
-                                       "encode + decode, single thread"},
+            "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "cores": n,
+                             "kind": "oracle", "cpu_model": model,
+                             "sample": f"{segs} whole segments of vectors drawn like "
+                                       f"{args.workload}'s, encode + decode through the "
+                                       f"oracle's thread pool, {n} threads"},
             "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -395,6 +455,81 @@ def job_gbs(raw_bytes_per_rank: int, world: int, ms: float) -> float:
 
 
 # ------------------------------------------------------------------ main --
+def time_config(wname: str, dev, steps: int, warmup: int, hbm: float, flush=None,
+                brief: bool = False):
+    """kvc_compress and kvc_decompress of one workload resident in HBM, timed
+    like the headline step (CUDA events on the launching stream around each
+    call, after `warmup` untimed steps; with `flush`, a write of it before
+    every step so small inputs are not served from L2). Returns the per-call
+    times, GB/s of raw input, roofline fractions (algorithmic bytes = raw
+    bytes + stream bytes, against `hbm` GB/s), ratio and break-even."""
+    import torch
+    import kv_cache_compression_04_b200 as kvc
+    w, desc, out_desc_fn, keep = make_input(wname, dev, 0)
+    codec = kvc.Codec(w.bits, w.group, w.sign_seed)
+    out, ws, nb = codec.buffers(desc, dev)
+    odesc, obuf = out_desc_fn()
+    dws = torch.empty(kvc.kvc_decompress_workspace_bytes(odesc), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = kvc._stream_ptr(stream)
+
+    def enc():
+        assert kvc.kvc_compress(desc, codec.params, out.data_ptr(), out.numel(), nb.data_ptr(),
+                                ws.data_ptr(), ws.numel(), sp) == kvc.KVC_OK
+
+    enc()
+    assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+    n = int(nb.item())
+
+    def dec():
+        assert kvc.kvc_decompress(out.data_ptr(), n, odesc, dws.data_ptr(), dws.numel(),
+                                  sp) == kvc.KVC_OK
+
+    dec()
+    assert kvc.kvc_stream_status(dws.data_ptr(), sp) == kvc.KVC_OK
+    te, td = [], []
+    for it in range(warmup + steps):
+        if flush is not None:
+            flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        enc()
+        e[1].record(stream)
+        dec()
+        e[2].record(stream)
+        if it >= warmup:
+            te.append(e)
+    torch.cuda.synchronize(dev)
+    assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+    assert kvc.kvc_stream_status(dws.data_ptr(), sp) == kvc.KVC_OK
+    enc_ms = statistics.median(e[0].elapsed_time(e[1]) for e in te)
+    dec_ms = statistics.median(e[1].elapsed_time(e[2]) for e in te)
+    raw = w.raw_bytes
+    alg = raw + n
+    saved_bits = 8 * (raw - n)
+    t_codec = (enc_ms + dec_ms) * 1e-3
+    r = {"workload": describe(w), "raw_bytes": raw, "stream_bytes": n,
+         "encode_ms": round(enc_ms, 4), "decode_ms": round(dec_ms, 4),
+         "encode_GBps": round(raw / (enc_ms * 1e-3) / 1e9, 1),
+         "decode_GBps": round(raw / (dec_ms * 1e-3) / 1e9, 1),
+         "roundtrip_GBps": round(raw / t_codec / 1e9, 1),
+         "encode_frac": round(alg / (enc_ms * 1e-3) / 1e9 / hbm, 4),
+         "decode_frac": round(alg / (dec_ms * 1e-3) / 1e9 / hbm, 4),
+         "ratio": round(raw / n, 4),
+         "break_even_gbit_s": round(saved_bits / t_codec / 1e9, 1),
+         "net_gain_ms": {"100Gbit": round((saved_bits / 100e9 - t_codec) * 1e3, 4),
+                         "400Gbit": round((saved_bits / 400e9 - t_codec) * 1e3, 4)},
+         "steps": steps, "timing": "median of steps",
+         "l2": "flushed before every step" if flush is not None else "inputs larger than L2"}
+    if brief:
+        for k in ("workload", "steps", "timing", "l2", "raw_bytes"):
+            r.pop(k)
+        r["name"] = wname
+    del keep, out, ws, nb, obuf, dws
+    torch.cuda.empty_cache()
+    return r
+
+
 def run_sweep(args):
     """Message-size sweep: [32, 2, 8, T, 128] with T = 8 * 2^i tokens (1 MiB ..
     4 GiB), 4-bit g128 and 2-bit g32. Each step times one compress and one
@@ -635,7 +770,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--workload", default="paged",
+                    help="the headline workload (the largest single-GPU configuration)")
+    ap.add_argument("--per-config", default="llama8b,qwen7b",
+                    help="other workloads timed after the headline one ('' for none)")
+    ap.add_argument("--config-steps", type=int, default=20)
+    ap.add_argument("--sweep-points", type=int, default=1,
+                    help="1: also time every message-size sweep point into per_config")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--e2e-groups", type=int, default=8,
@@ -766,6 +907,24 @@ def main():
                            "quantize kernel, same finishing kernels, same stream"}
         del uws
 
+    # -------------------------- the other workloads, timed the same way --
+    # (after the timed region, with the headline workload's buffers freed)
+    per_config = None
+    if world == 1 and args.per_config:
+        del out, ws, nb, obuf, dws, keep
+        torch.cuda.empty_cache()
+        hbm_, _ = peaks()
+        per_config = {}
+        for wname in [x for x in args.per_config.split(",") if x and x != args.workload]:
+            per_config[wname] = time_config(wname, dev, args.config_steps, args.warmup, hbm_)
+        if args.sweep_points:
+            flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+            per_config["sweep"] = [time_config(f"sweep-{i}-{b}", dev, args.config_steps,
+                                               args.warmup, hbm_, flush=flush, brief=True)
+                                   for b in (4, 2) for i in range(13)]
+            del flush
+            torch.cuda.empty_cache()
+
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -815,13 +974,10 @@ def main():
         line["e2e"] = e2e
     if unfused:
         line["unfused_baseline"] = unfused
+    if per_config:
+        line["per_config"] = per_config
     if world == 1 and args.cpu_budget > 0:
-        b, s, n = oracle_sample(args.workload, args.cpu_budget)
-        line["cpu_baseline"] = {"value": round(b / s / 1e9, 6), "unit": "GB/s", "cores": 1,
-                                "kind": "oracle",
-                                "sample": f"{n} whole segments ({b} raw bytes) of "
-                                          f"{args.workload} vectors, encode + decode, "
-                                          "single thread"}
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_budget)
     print(json.dumps(line), flush=True)
     return 0
 

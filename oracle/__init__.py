@@ -60,7 +60,13 @@ class Desc(C.Structure):
                 ("head_dim", C.c_int32), ("layers", C.c_int32),
                 ("kv_heads", C.c_int32), ("origin", C.c_int32),
                 ("n_requests", C.c_int32), ("sign_seed", C.c_uint64),
-                ("token_lens", C.POINTER(C.c_uint32))]
+                ("token_lens", C.POINTER(C.c_uint32)), ("lossless", C.c_int32)]
+
+
+# Lossless pipeline ids of a chunk and encoder modes (reading R17).
+PIPE_ZE, PIPE_XOR_ZE, PIPE_ZE2, PIPE_XOR_ZE2 = range(4)
+LOSSLESS_FIXED, LOSSLESS_SEARCH, LOSSLESS_NONE = range(3)
+BITMAP2 = 256
 
 
 class Layout(C.Structure):
@@ -116,9 +122,19 @@ def lib():
                 "orc_meta_chunk_index": (C.c_uint64, [C.POINTER(Layout),
                                                       C.c_uint64]),
                 "orc_encode_segment": (C.c_int, [C.POINTER(Desc), C.c_uint64,
-                                                 u16p, u8p, u32p, u32p]),
+                                                 u16p, u8p, u32p, u8p, u32p]),
                 "orc_decode_segment": (C.c_int, [C.POINTER(Desc), C.c_uint64,
-                                                 u8p, u32p, u16p]),
+                                                 u8p, u32p, u8p, u16p]),
+                "orc_xor_words": (None, [u8p, C.c_uint32, C.c_int]),
+                "orc_unxor_words": (None, [u8p, C.c_uint32, C.c_int]),
+                "orc_ze2_encode": (C.c_uint32, [u8p, u8p]),
+                "orc_ze2_decode": (C.c_int, [u8p, C.c_uint32, u8p]),
+                "orc_chunk_encode_pipe": (C.c_uint32, [u8p, C.c_int, C.c_int, u8p]),
+                "orc_chunk_decode_pipe": (C.c_int, [u8p, C.c_uint32, C.c_uint32,
+                                                    C.c_int, C.c_int, u8p]),
+                "orc_chunk_encode_select": (C.c_uint32, [u8p, C.c_uint32, C.c_int,
+                                                         C.c_int, C.c_int, u8p,
+                                                         C.POINTER(C.c_int)]),
                 "orc_code_elim_pays": (C.c_int, [u32p, u32p, C.c_uint64]),
                 "orc_compress": (C.c_int, [C.POINTER(Desc), u16p, u8p,
                                            C.c_uint64, u64p]),
@@ -297,11 +313,11 @@ class StreamDesc:
     """Shape and parameters of one stream (the oracle's own description)."""
 
     def __init__(self, bits, group, head_dim, layers, kv_heads, token_lens,
-                 sign_seed=0, origin=0):
+                 sign_seed=0, origin=0, lossless=LOSSLESS_FIXED):
         self.token_lens = np.ascontiguousarray(np.asarray(token_lens, np.uint32))
         self.c = Desc(bits, group, head_dim, layers, kv_heads, origin,
                       len(self.token_lens), sign_seed,
-                      _p(self.token_lens, C.c_uint32))
+                      _p(self.token_lens, C.c_uint32), lossless)
 
     @property
     def head_dim(self):
@@ -357,30 +373,90 @@ def decompress(stream: np.ndarray, desc: StreamDesc, threads: int = 1):
 
 
 def encode_segment(desc: StreamDesc, s: int, vectors: np.ndarray):
-    """-> (status, [chunk bytes ...]) for segment s (code chunks, then meta)."""
+    """-> (status, [chunk bytes ...], [pipeline ids]) for segment s (code
+    chunks, then meta), each chunk as the encoder mode chooses it (the
+    stream-wide code-region rule R16 is not applied here)."""
     vectors = np.ascontiguousarray(vectors, np.uint16)
     lay = desc.layout()
     buf = np.zeros((lay.code_per_seg + 1) * CHUNK, np.uint8)
     sizes = np.zeros(lay.code_per_seg + 1, np.uint32)
+    pipes = np.zeros(lay.code_per_seg + 1, np.uint8)
     n = C.c_uint32(0)
     st = lib().orc_encode_segment(C.byref(desc.c), s, _p(vectors, C.c_uint16),
                                   _p(buf, C.c_uint8), _p(sizes, C.c_uint32),
-                                  C.byref(n))
+                                  _p(pipes, C.c_uint8), C.byref(n))
     chunks, pos = [], 0
     for i in range(n.value):
         chunks.append(buf[pos:pos + sizes[i]].copy())
         pos += int(sizes[i])
-    return st, chunks
+    return st, chunks, [int(p) for p in pipes[:n.value]]
 
 
-def decode_segment(desc: StreamDesc, s: int, chunks: list, nvec: int):
+def decode_segment(desc: StreamDesc, s: int, chunks: list, nvec: int, pipes=None):
     lay = desc.layout()
     buf = np.concatenate(chunks).astype(np.uint8) if chunks else np.zeros(1, np.uint8)
     sizes = np.array([c.size for c in chunks], np.uint32)
+    pp = np.zeros(max(len(chunks), 1), np.uint8)
+    if pipes is not None:
+        pp[:len(pipes)] = pipes
     out = np.zeros((nvec, desc.head_dim), np.uint16)
     st = lib().orc_decode_segment(C.byref(desc.c), s, _p(buf, C.c_uint8),
-                                  _p(sizes, C.c_uint32), _p(out, C.c_uint16))
+                                  _p(sizes, C.c_uint32), _p(pp, C.c_uint8),
+                                  _p(out, C.c_uint16))
     return st, out
+
+
+def xor_words(chunk: np.ndarray, run_words: int) -> np.ndarray:
+    c = np.ascontiguousarray(chunk, np.uint8).copy()
+    lib().orc_xor_words(_p(c, C.c_uint8), c.size // 4, run_words)
+    return c
+
+
+def unxor_words(chunk: np.ndarray, run_words: int) -> np.ndarray:
+    c = np.ascontiguousarray(chunk, np.uint8).copy()
+    lib().orc_unxor_words(_p(c, C.c_uint8), c.size // 4, run_words)
+    return c
+
+
+def ze2_encode(shuffled: np.ndarray) -> np.ndarray:
+    sh = np.ascontiguousarray(shuffled, np.uint8)
+    assert sh.size == CHUNK
+    out = np.zeros(CHUNK + BITMAP2 + BITMAP, np.uint8)
+    n = lib().orc_ze2_encode(_p(sh, C.c_uint8), _p(out, C.c_uint8))
+    return out[:n].copy()
+
+
+def ze2_decode(enc: np.ndarray):
+    enc = np.ascontiguousarray(enc, np.uint8)
+    out = np.zeros(CHUNK, np.uint8)
+    st = lib().orc_ze2_decode(_p(enc, C.c_uint8), enc.size, _p(out, C.c_uint8))
+    return st, out
+
+
+def chunk_encode_pipe(chunk: np.ndarray, pipe: int, words_per_vector: int) -> np.ndarray:
+    c = np.ascontiguousarray(chunk, np.uint8)
+    assert c.size == CHUNK
+    out = np.zeros(CHUNK + BITMAP2 + BITMAP, np.uint8)
+    n = lib().orc_chunk_encode_pipe(_p(c, C.c_uint8), pipe, words_per_vector, _p(out, C.c_uint8))
+    return out[:n].copy()
+
+
+def chunk_decode_pipe(enc: np.ndarray, length: int, pipe: int, words_per_vector: int):
+    enc = np.ascontiguousarray(enc, np.uint8)
+    out = np.zeros(max(length, 1), np.uint8)
+    st = lib().orc_chunk_decode_pipe(_p(enc, C.c_uint8), enc.size, length, pipe,
+                                     words_per_vector, _p(out, C.c_uint8))
+    return st, out[:length]
+
+
+def chunk_encode_select(chunk: np.ndarray, is_meta: bool, words_per_vector: int, mode: int):
+    """-> (encoded bytes, pipeline id) under reading R17."""
+    c = np.ascontiguousarray(chunk, np.uint8)
+    out = np.zeros(CHUNK + BITMAP2 + BITMAP, np.uint8)
+    pipe = C.c_int(0)
+    n = lib().orc_chunk_encode_select(_p(c, C.c_uint8), c.size, int(is_meta), words_per_vector,
+                                      mode, _p(out, C.c_uint8), C.byref(pipe))
+    return out[:n].copy(), pipe.value
 
 
 def segment_vectors(lay: Layout, s: int) -> tuple[int, int]:

@@ -389,6 +389,173 @@ int orc_lossless_decode_chunk(const uint8_t *in, uint32_t size, uint32_t len,
 }
 
 /* ========================================================================== */
+/* Composable lossless pipelines ([P2]: the backend is "searchable", built   */
+/* from primitives composed into pipelines). Reading R17 adds two primitives */
+/* to the bit-plane shuffle and zero-byte elimination above, each pinned on  */
+/* its own: an XOR of each 32-bit word with the previous word, restarting at */
+/* every run of 32 vectors (the fp16 scale/zero pairs of neighbouring groups */
+/* and tokens share their sign and exponent bits, so the XOR clears most of  */
+/* those bit planes), and a second level of zero-byte elimination applied to */
+/* the 2048-byte bitmap. A chunk's pipeline id (0..3, see kvc_oracle.h) says */
+/* which were applied.                                                        */
+/* ========================================================================== */
+static void put_word(uint8_t *b, int j, uint32_t w) {
+  b[4 * j] = (uint8_t)w;
+  b[4 * j + 1] = (uint8_t)(w >> 8);
+  b[4 * j + 2] = (uint8_t)(w >> 16);
+  b[4 * j + 3] = (uint8_t)(w >> 24);
+}
+
+/* w'[j] = w[j] XOR w[j-1] unless j starts a run (j mod run_words == 0), with
+ * w the original words; in place, so from the last word down. run_words is
+ * 32 vectors' worth of words. */
+void orc_xor_words(uint8_t *chunk, uint32_t n_words, int run_words) {
+  int64_t j;
+  for (j = (int64_t)n_words - 1; j >= 1; j--)
+    if (j % run_words != 0)
+      put_word(chunk, (int)j, word_at(chunk, (int)j) ^ word_at(chunk, (int)j - 1));
+}
+
+/* The inverse: from the first word up, each word XOR the restored previous
+ * one, except at the start of a run. */
+void orc_unxor_words(uint8_t *chunk, uint32_t n_words, int run_words) {
+  uint32_t j;
+  for (j = 1; j < n_words; j++)
+    if (j % run_words != 0)
+      put_word(chunk, (int)j, word_at(chunk, (int)j) ^ word_at(chunk, (int)j - 1));
+}
+
+/* Two-level zero-byte elimination of a shuffled chunk: the 2048-byte bitmap B
+ * of the one-level form (bit i = shuffled byte i is nonzero) is itself
+ * reduced to a 256-byte bitmap B2 (bit i = byte i of B is nonzero) and its
+ * nonzero bytes. Output: B2, then the nonzero bytes of B in order, then the
+ * nonzero shuffled bytes in order. Returns the size. */
+uint32_t orc_ze2_encode(const uint8_t *sh, uint8_t *out) {
+  uint8_t b[ORC_BITMAP];
+  uint32_t i, pos;
+  memset(b, 0, sizeof b);
+  for (i = 0; i < ORC_CHUNK; i++)
+    if (sh[i]) b[i / 8] |= (uint8_t)(1u << (i % 8));
+  memset(out, 0, ORC_BITMAP2);
+  pos = ORC_BITMAP2;
+  for (i = 0; i < ORC_BITMAP; i++)
+    if (b[i]) {
+      out[i / 8] |= (uint8_t)(1u << (i % 8));
+      out[pos++] = b[i];
+    }
+  for (i = 0; i < ORC_CHUNK; i++)
+    if (sh[i]) out[pos++] = sh[i];
+  return pos;
+}
+
+int orc_ze2_decode(const uint8_t *in, uint32_t size, uint8_t *sh) {
+  uint8_t b[ORC_BITMAP];
+  uint32_t i, pos = ORC_BITMAP2;
+  if (size < ORC_BITMAP2) return ORC_ERR_CORRUPT;
+  for (i = 0; i < ORC_BITMAP; i++) {
+    if ((in[i / 8] >> (i % 8)) & 1u) {
+      if (pos >= size) return ORC_ERR_CORRUPT;
+      b[i] = in[pos++];
+    } else {
+      b[i] = 0;
+    }
+  }
+  for (i = 0; i < ORC_CHUNK; i++) {
+    if ((b[i / 8] >> (i % 8)) & 1u) {
+      if (pos >= size) return ORC_ERR_CORRUPT;
+      sh[i] = in[pos++];
+    } else {
+      sh[i] = 0;
+    }
+  }
+  return pos == size ? ORC_OK : ORC_ERR_CORRUPT;
+}
+
+/* A full chunk through pipeline `pipe` (no raw fallback, so `out` needs room
+ * for ORC_BITMAP2 + ORC_BITMAP + ORC_CHUNK bytes). s: words per vector (the
+ * XOR of pipelines 1 and 3 restarts every 32 vectors, 32 * s words). Returns
+ * the size. */
+uint32_t orc_chunk_encode_pipe(const uint8_t *in, int pipe, int s, uint8_t *out) {
+  uint8_t w[ORC_CHUNK], sh[ORC_CHUNK];
+  uint32_t i, nnz = 0;
+  memcpy(w, in, ORC_CHUNK);
+  if (pipe == ORC_PIPE_XOR_ZE || pipe == ORC_PIPE_XOR_ZE2) orc_xor_words(w, ORC_CHUNK / 4, 32 * s);
+  orc_bitplane_shuffle(w, sh);
+  if (pipe == ORC_PIPE_ZE2 || pipe == ORC_PIPE_XOR_ZE2) return orc_ze2_encode(sh, out);
+  memset(out, 0, ORC_BITMAP);
+  for (i = 0; i < ORC_CHUNK; i++) {
+    if (sh[i]) {
+      out[i / 8] |= (uint8_t)(1u << (i % 8));
+      out[ORC_BITMAP + nnz++] = sh[i];
+    }
+  }
+  return ORC_BITMAP + nnz;
+}
+
+/* Inverse of any pipeline, or a raw chunk (size == len, pipe 0). */
+int orc_chunk_decode_pipe(const uint8_t *in, uint32_t size, uint32_t len, int pipe, int s,
+                          uint8_t *out) {
+  uint8_t sh[ORC_CHUNK];
+  int st;
+  if (pipe < 0 || pipe > 3) return ORC_ERR_CORRUPT;
+  if (size == len) {
+    if (pipe != 0) return ORC_ERR_CORRUPT;
+    memcpy(out, in, len);
+    return ORC_OK;
+  }
+  if (len != ORC_CHUNK || size >= ORC_CHUNK) return ORC_ERR_CORRUPT;
+  if (pipe == ORC_PIPE_ZE || pipe == ORC_PIPE_XOR_ZE) {
+    st = orc_lossless_decode_chunk(in, size, len, out);
+    if (st != ORC_OK) return st;
+  } else {
+    st = orc_ze2_decode(in, size, sh);
+    if (st != ORC_OK) return st;
+    orc_bitplane_unshuffle(sh, out);
+  }
+  if (pipe == ORC_PIPE_XOR_ZE || pipe == ORC_PIPE_XOR_ZE2)
+    orc_unxor_words(out, ORC_CHUNK / 4, 32 * s);
+  return ORC_OK;
+}
+
+/* Reading R17, the encoder's choice for one chunk: FIXED tries pipeline 0,
+ * SEARCH every candidate of the region (code chunks 0 and 2; meta chunks 0..3
+ * when a vector holds at least two meta words, else 0 and 1), NONE none. The
+ * shortest candidate wins, ties to the lower id; it is used only if strictly
+ * shorter than the chunk, which is otherwise stored raw (pipeline 0). Short
+ * chunks are always raw. */
+uint32_t orc_chunk_encode_select(const uint8_t *in, uint32_t len, int is_meta, int s, int mode,
+                                 uint8_t *out, int *pipe) {
+  uint8_t tmp[ORC_BITMAP2 + ORC_BITMAP + ORC_CHUNK]; /* a candidate may exceed the chunk */
+  int cand[4], n = 0, k, best = -1;
+  uint32_t best_size = len, sz;
+  *pipe = 0;
+  if (len < ORC_CHUNK || mode == ORC_LOSSLESS_NONE) {
+    memcpy(out, in, len);
+    return len;
+  }
+  cand[n++] = ORC_PIPE_ZE;
+  if (mode == ORC_LOSSLESS_SEARCH) {
+    if (is_meta) cand[n++] = ORC_PIPE_XOR_ZE;
+    if (!is_meta || s >= 2) cand[n++] = ORC_PIPE_ZE2;
+    if (is_meta && s >= 2) cand[n++] = ORC_PIPE_XOR_ZE2;
+  }
+  for (k = 0; k < n; k++) {
+    sz = orc_chunk_encode_pipe(in, cand[k], s, tmp);
+    if (sz < best_size) {
+      best_size = sz;
+      best = cand[k];
+    }
+  }
+  if (best < 0) {
+    memcpy(out, in, len);
+    return len;
+  }
+  orc_chunk_encode_pipe(in, best, s, out);
+  *pipe = best;
+  return best_size;
+}
+
+/* ========================================================================== */
 /* Stream layout. Reading R12 (self-describing stream, little-endian):        */
 /*   [0,64)    header: u32 magic "KVC1", u16 version 1, u16 header bytes 64,  */
 /*             u8 bits, u8 k, u8 origin (0 dense, 1 paged), u8 flags (bit 0: */
@@ -397,7 +564,8 @@ int orc_lossless_decode_chunk(const uint8_t *in, uint32_t size, uint32_t len,
 /*             u64 tokens (sum over requests), u64 sign_seed,                 */
 /*             u32 n_requests, u32 n_chunks, u64 stream_bytes;                */
 /*   then      u64 chunk table [n_chunks]: bits 0..15 = unpadded size,        */
-/*             bits 16..63 = offset from the data base in 16-byte units;      */
+/*             bits 16..59 = offset from the data base in 16-byte units,      */
+/*             bits 60..63 = the chunk's lossless pipeline id (R17; 0 raw);   */
 /*   then      u32 token lengths [n_requests];                                */
 /*   then      zeros up to a 16-byte boundary = data base;                    */
 /*   then      the chunks, each zero-padded to 16 bytes, at their offsets.    */
@@ -408,6 +576,9 @@ int orc_lossless_decode_chunk(const uint8_t *in, uint32_t size, uint32_t len,
 /* prefix sum of the padded chunk sizes in that order.                        */
 /* ========================================================================== */
 static uint64_t round16(uint64_t x) { return (x + 15u) & ~(uint64_t)15u; }
+
+/* Byte offset (from the data base) held in bits 16..59 of a table entry. */
+#define ENTRY_OFFSET(e) ((((e) >> 16) & 0xFFFFFFFFFFFull) * 16)
 
 int orc_check_desc(const orc_desc *d) {
   int r;
@@ -498,7 +669,8 @@ static uint64_t get64(const uint8_t *p) {
  * caller (orc_encode_segment and the compressor below). */
 static int encode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t s,
                              const uint16_t *vectors, uint8_t *chunks,
-                             uint32_t *sizes, uint32_t *n_out) {
+                             uint32_t *sizes, uint8_t *pipes, uint32_t *n_out) {
+  int pipe;
   uint64_t vm, v0, nv, v, c0, c1, c;
   uint8_t *codes, *meta;
   uint64_t sw[4];
@@ -522,31 +694,34 @@ static int encode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t 
   for (c = c0; c < c1; c++) {
     uint64_t a = (c - c0) * lay->vec_per_code;
     uint64_t b = a + lay->vec_per_code < nv ? a + lay->vec_per_code : nv;
-    uint32_t sz = orc_lossless_encode_chunk(
-        codes + a * lay->code_bytes, (uint32_t)((b - a) * lay->code_bytes),
-        chunks + pos);
+    uint32_t sz = orc_chunk_encode_select(
+        codes + a * lay->code_bytes, (uint32_t)((b - a) * lay->code_bytes), 0,
+        (int)(lay->code_bytes / 4), d->lossless, chunks + pos, &pipe);
+    pipes[*n_out] = (uint8_t)pipe;
     sizes[(*n_out)++] = sz;
     pos += sz;
   }
-  sizes[(*n_out)++] =
-      orc_lossless_encode_chunk(meta, (uint32_t)(nv * lay->meta_bytes), chunks + pos);
+  sizes[*n_out] = orc_chunk_encode_select(meta, (uint32_t)(nv * lay->meta_bytes), 1,
+                                          (int)(lay->meta_bytes / 4), d->lossless,
+                                          chunks + pos, &pipe);
+  pipes[(*n_out)++] = (uint8_t)pipe;
   free(codes);
   free(meta);
   return st;
 }
 
 int orc_encode_segment(const orc_desc *d, uint64_t s, const uint16_t *vectors,
-                       uint8_t *chunks, uint32_t *sizes, uint32_t *n_out) {
+                       uint8_t *chunks, uint32_t *sizes, uint8_t *pipes, uint32_t *n_out) {
   orc_layout lay;
   int st = orc_layout_of(d, &lay);
   if (st != ORC_OK) return st;
   if (s >= lay.n_seg) return ORC_ERR_INVALID_ARG;
-  return encode_segment_in(d, &lay, s, vectors, chunks, sizes, n_out);
+  return encode_segment_in(d, &lay, s, vectors, chunks, sizes, pipes, n_out);
 }
 
 static int decode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t s,
                              const uint8_t *chunks, const uint32_t *sizes,
-                             uint16_t *vectors) {
+                             const uint8_t *pipes, uint16_t *vectors) {
   uint64_t vm, v0, nv, v, c0, c1, c, i = 0;
   uint8_t *codes, *meta;
   uint64_t sw[4];
@@ -563,14 +738,17 @@ static int decode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t 
   for (c = c0; c < c1 && st == ORC_OK; c++, i++) {
     uint64_t a = (c - c0) * lay->vec_per_code;
     uint64_t b = a + lay->vec_per_code < nv ? a + lay->vec_per_code : nv;
-    st = orc_lossless_decode_chunk(chunks + pos, sizes[i],
-                                   (uint32_t)((b - a) * lay->code_bytes),
-                                   codes + a * lay->code_bytes);
+    /* code chunks: pipelines 0 and 2 only */
+    if (pipes[i] != ORC_PIPE_ZE && pipes[i] != ORC_PIPE_ZE2) st = ORC_ERR_CORRUPT;
+    else
+      st = orc_chunk_decode_pipe(chunks + pos, sizes[i], (uint32_t)((b - a) * lay->code_bytes),
+                                 pipes[i], (int)(lay->code_bytes / 4),
+                                 codes + a * lay->code_bytes);
     pos += sizes[i];
   }
   if (st == ORC_OK)
-    st = orc_lossless_decode_chunk(chunks + pos, sizes[i],
-                                   (uint32_t)(nv * lay->meta_bytes), meta);
+    st = orc_chunk_decode_pipe(chunks + pos, sizes[i], (uint32_t)(nv * lay->meta_bytes),
+                               pipes[i], (int)(lay->meta_bytes / 4), meta);
   if (st == ORC_OK)
     for (v = 0; v < nv; v++)
       orc_dequantize_vector(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
@@ -582,12 +760,12 @@ static int decode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t 
 }
 
 int orc_decode_segment(const orc_desc *d, uint64_t s, const uint8_t *chunks,
-                       const uint32_t *sizes, uint16_t *vectors) {
+                       const uint32_t *sizes, const uint8_t *pipes, uint16_t *vectors) {
   orc_layout lay;
   int st = orc_layout_of(d, &lay);
   if (st != ORC_OK) return st;
   if (s >= lay.n_seg) return ORC_ERR_INVALID_ARG;
-  return decode_segment_in(d, &lay, s, chunks, sizes, vectors);
+  return decode_segment_in(d, &lay, s, chunks, sizes, pipes, vectors);
 }
 
 /* Runs fn(job, s) for every segment s in [0, n_seg) on n_threads threads
@@ -664,6 +842,7 @@ typedef struct {
   const uint16_t *vectors;
   uint8_t *store;
   uint32_t *all_sizes;
+  uint8_t *all_pipes;
   uint64_t *where;
   int *seg_status;
 } enc_job;
@@ -674,13 +853,15 @@ static void enc_one_segment(void *arg, uint64_t s) {
   uint64_t vm = (uint64_t)lay->vec_per_code * lay->code_per_seg;
   uint8_t *seg = (uint8_t *)malloc((size_t)(lay->code_per_seg + 1) * ORC_CHUNK);
   uint32_t sizes[17], n, k, pos = 0;
+  uint8_t pipes[17];
   j->seg_status[s] = encode_segment_in(j->d, lay, s, j->vectors + s * vm * j->d->head_dim,
-                                       seg, sizes, &n);
+                                       seg, sizes, pipes, &n);
   for (k = 0; k < n; k++) {
     uint64_t idx = (k + 1 < n) ? orc_code_chunk_index(lay, s * lay->code_per_seg + k)
                                : orc_meta_chunk_index(lay, s);
     memcpy(j->store + idx * ORC_CHUNK, seg + pos, sizes[k]);
     j->all_sizes[idx] = sizes[k];
+    j->all_pipes[idx] = pipes[k];
     j->where[idx] = idx * ORC_CHUNK;
     pos += sizes[k];
   }
@@ -698,6 +879,7 @@ int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
   uint64_t s, off = 0, T = 0, i;
   uint8_t *store;
   uint32_t *all_sizes;
+  uint8_t *all_pipes;
   uint64_t *where; /* chunk index -> position in store */
   int *seg_status;
   enc_job job;
@@ -727,6 +909,7 @@ int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
   /* encode every segment, remembering where each chunk's bytes are */
   store = (uint8_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1) * ORC_CHUNK);
   all_sizes = (uint32_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1) * 4);
+  all_pipes = (uint8_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1));
   where = (uint64_t *)malloc((size_t)(lay.n_chunks ? lay.n_chunks : 1) * 8);
   seg_status = (int *)malloc((size_t)(lay.n_seg ? lay.n_seg : 1) * sizeof(int));
   job.d = d;
@@ -734,6 +917,7 @@ int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
   job.vectors = vectors;
   job.store = store;
   job.all_sizes = all_sizes;
+  job.all_pipes = all_pipes;
   job.where = where;
   job.seg_status = seg_status;
   for_each_segment(lay.n_seg, n_threads, &job, enc_one_segment);
@@ -757,11 +941,13 @@ int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
       for (i = 0; i < lay.n_code; i++) {
         uint64_t idx = orc_code_chunk_index(&lay, i);
         if (csz[i] == clen[i]) continue;
-        if (orc_lossless_decode_chunk(store + where[idx], csz[i], clen[i], raw) != ORC_OK &&
+        if (orc_chunk_decode_pipe(store + where[idx], csz[i], clen[i], all_pipes[idx],
+                                  (int)(lay.code_bytes / 4), raw) != ORC_OK &&
             st == ORC_OK)
           st = ORC_ERR_CORRUPT; /* cannot happen: the chunk was just encoded */
         memcpy(store + where[idx], raw, clen[i]);
         all_sizes[idx] = clen[i];
+        all_pipes[idx] = 0;
       }
     }
     free(csz);
@@ -770,7 +956,9 @@ int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
   /* lay the chunks out in index order */
   for (i = 0; i < lay.n_chunks; i++) {
     uint64_t padded = round16(all_sizes[i]);
-    put64(out + ORC_HEADER + 8 * i, ((off / 16) << 16) | all_sizes[i]);
+    /* entry: bits 0..15 size, 16..59 offset / 16, 60..63 pipeline id */
+    put64(out + ORC_HEADER + 8 * i,
+          ((uint64_t)all_pipes[i] << 60) | ((off / 16) << 16) | all_sizes[i]);
     memset(out + lay.data_base + off, 0, (size_t)padded);
     memcpy(out + lay.data_base + off, store + where[i], all_sizes[i]);
     off += padded;
@@ -787,6 +975,7 @@ int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
   }
   free(store);
   free(all_sizes);
+  free(all_pipes);
   free(where);
   put64(out + 56, lay.data_base + off);
   *out_bytes = lay.data_base + off;
@@ -811,16 +1000,18 @@ static void dec_one_segment(void *arg, uint64_t s) {
   uint64_t c1 = c0 + lay->code_per_seg < lay->n_code ? c0 + lay->code_per_seg : lay->n_code;
   uint64_t i, k = 0;
   uint32_t pos = 0, sizes[17];
+  uint8_t pipes[17];
   uint8_t *seg = (uint8_t *)malloc((size_t)(lay->code_per_seg + 1) * ORC_CHUNK);
   for (i = c0; i <= c1; i++, k++) { /* code chunks c0..c1-1, then the meta chunk */
     uint64_t idx = i < c1 ? orc_code_chunk_index(lay, i) : orc_meta_chunk_index(lay, s);
     uint64_t e = get64(j->stream + ORC_HEADER + 8 * idx);
     uint32_t sz = (uint32_t)(e & 0xFFFFu);
-    memcpy(seg + pos, j->stream + lay->data_base + (e >> 16) * 16, sz);
+    memcpy(seg + pos, j->stream + lay->data_base + ENTRY_OFFSET(e), sz);
     sizes[k] = sz;
+    pipes[k] = (uint8_t)(e >> 60);
     pos += sz;
   }
-  j->seg_status[s] = decode_segment_in(j->d, lay, s, seg, sizes,
+  j->seg_status[s] = decode_segment_in(j->d, lay, s, seg, sizes, pipes,
                                        j->vectors + s * vm * j->d->head_dim);
   free(seg);
 }
@@ -861,7 +1052,7 @@ int orc_decompress_mt(const uint8_t *stream, uint64_t stream_bytes,
   for (s = 0; s < lay.n_chunks; s++) {
     uint64_t e = get64(stream + ORC_HEADER + 8 * s);
     uint32_t sz = (uint32_t)(e & 0xFFFFu);
-    uint64_t off = (e >> 16) * 16;
+    uint64_t off = ENTRY_OFFSET(e);
     if (off != expect_off || sz > ORC_CHUNK || lay.data_base + off + round16(sz) > total)
       return ORC_ERR_CORRUPT;
     expect_off = off + round16(sz);

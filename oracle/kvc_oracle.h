@@ -44,6 +44,7 @@ enum {
 
 #define ORC_CHUNK 16384      /* lossless chunk length in bytes            */
 #define ORC_BITMAP 2048      /* zero-byte-elimination bitmap bytes        */
+#define ORC_BITMAP2 256      /* second-level bitmap bytes (pipelines 2, 3) */
 #define ORC_HEADER 64        /* stream header bytes                       */
 #define ORC_MAGIC 0x3143564Bu /* "KVC1" little-endian                    */
 #define ORC_MAX_D 256
@@ -78,11 +79,44 @@ uint32_t orc_lossless_encode_chunk(const uint8_t *in, uint32_t len,
 int orc_lossless_decode_chunk(const uint8_t *in, uint32_t size, uint32_t len,
                               uint8_t *out);
 
+/* ---- composable lossless pipelines (LC-style search, reading R17) --------- */
+/* Pipeline ids of a stored chunk (bits 60..63 of its table entry):
+ *   0  bit-plane shuffle, zero-byte elimination with a 2048-byte bitmap
+ *   1  XOR of each word with the previous word, restarting at every run of
+ *      32 vectors (meta chunks), then as 0
+ *   2  bit-plane shuffle, two-level zero-byte elimination (the 2048-byte
+ *      bitmap itself zero-byte eliminated under a 256-byte bitmap)
+ *   3  the XOR of 1, then as 2
+ * A raw chunk (size == length) has id 0. */
+#define ORC_PIPE_ZE 0
+#define ORC_PIPE_XOR_ZE 1
+#define ORC_PIPE_ZE2 2
+#define ORC_PIPE_XOR_ZE2 3
+/* Encoder modes (orc_desc.lossless): FIXED uses pipeline 0 only; SEARCH picks,
+ * per full chunk, the shortest candidate (code chunks: 0, 2; meta chunks with
+ * at least two groups per vector: 0..3; other meta chunks: 0, 1), ties to the
+ * lower id; NONE stores every chunk raw. */
+#define ORC_LOSSLESS_FIXED 0
+#define ORC_LOSSLESS_SEARCH 1
+#define ORC_LOSSLESS_NONE 2
+void orc_xor_words(uint8_t *chunk, uint32_t n_words, int run_words);
+void orc_unxor_words(uint8_t *chunk, uint32_t n_words, int run_words);
+uint32_t orc_ze2_encode(const uint8_t *shuffled, uint8_t *out);
+int orc_ze2_decode(const uint8_t *in, uint32_t size, uint8_t *shuffled);
+uint32_t orc_chunk_encode_pipe(const uint8_t *in, int pipe, int words_per_vector,
+                               uint8_t *out);
+int orc_chunk_decode_pipe(const uint8_t *in, uint32_t size, uint32_t len, int pipe,
+                          int words_per_vector, uint8_t *out);
+uint32_t orc_chunk_encode_select(const uint8_t *in, uint32_t len, int is_meta,
+                                 int words_per_vector, int mode, uint8_t *out,
+                                 int *pipe);
+
 /* ---- stream --------------------------------------------------------------- */
 typedef struct {
   int32_t bits, group, head_dim, layers, kv_heads, origin, n_requests;
   uint64_t sign_seed;
   const uint32_t *token_lens; /* [n_requests] tokens per request          */
+  int32_t lossless;           /* ORC_LOSSLESS_* (encoder only)            */
 } orc_desc;
 
 typedef struct {
@@ -106,13 +140,15 @@ uint64_t orc_meta_chunk_index(const orc_layout *lay, uint64_t s);
 
 /* Encodes segment s from its vectors (vectors [s*VM, min((s+1)*VM, V)) in
  * logical order, d bf16 each). Writes the segment's chunks, unpadded, back to
- * back into chunks (capacity (code_per_seg+1)*ORC_CHUNK) and their sizes into
- * sizes[] (code chunks first, then the meta chunk). Returns the status and the
- * number of chunks through n_out. */
+ * back into chunks (capacity (code_per_seg+1)*ORC_CHUNK), their sizes into
+ * sizes[] and their pipeline ids into pipes[] (code chunks first, then the
+ * meta chunk), per chunk as chosen by d->lossless (the code-region rule R16
+ * is applied by orc_compress over the whole stream, not here). Returns the
+ * status and the number of chunks through n_out. */
 int orc_encode_segment(const orc_desc *d, uint64_t s, const uint16_t *vectors,
-                       uint8_t *chunks, uint32_t *sizes, uint32_t *n_out);
+                       uint8_t *chunks, uint32_t *sizes, uint8_t *pipes, uint32_t *n_out);
 int orc_decode_segment(const orc_desc *d, uint64_t s, const uint8_t *chunks,
-                       const uint32_t *sizes, uint16_t *vectors);
+                       const uint32_t *sizes, const uint8_t *pipes, uint16_t *vectors);
 
 /* Reading R16: 1 iff some code chunk shrinks and the padded bytes saved are
  * at least 1/64 of the padded bytes from the first shrinking code chunk on. */

@@ -226,7 +226,7 @@ def test_stream_is_deterministic_and_segments_agree():
     assert offs == [sum((z + 15) // 16 * 16 for z in sizes[:i]) for i in range(lay.n_chunks)]
     for seg in range(lay.n_seg):
         v0, v1 = oracle.segment_vectors(lay, seg)
-        st, chunks = oracle.encode_segment(d, seg, x[v0:v1])
+        st, chunks, _ = oracle.encode_segment(d, seg, x[v0:v1])
         idx = [oracle.code_chunk_index(lay, seg * lay.code_per_seg + i)
                for i in range(len(chunks) - 1)] + [oracle.meta_chunk_index(lay, seg)]
         for i, ch in zip(idx, chunks):
@@ -354,3 +354,100 @@ def test_threaded_oracle_first_error_in_segment_order():
         st1, s1 = oracle.compress(d, x)
         st4, s4 = oracle.compress(d, x, threads=4)
         assert st1 == st4 == want and np.array_equal(s1, s4)
+
+
+def _search_desc(bits, g, L, H, T, seed=0, mode=None):
+    return oracle.StreamDesc(bits, g, 128, L, H, [T], seed,
+                             lossless=oracle.LOSSLESS_SEARCH if mode is None else mode)
+
+
+def _entries(stream, n_chunks):
+    e = stream[64:64 + 8 * n_chunks].view("<u8").astype(np.uint64)
+    return (e & 0xFFFF).astype(np.int64), (e >> 60).astype(np.int64)
+
+
+@pytest.mark.parametrize("bits,g", [(4, 128), (4, 64), (2, 32)])
+def test_search_mode_round_trip_and_table_ids(bits, g):
+    """Search-mode streams decode to the fixed-mode decode (the lossless
+    stage is exact), their meta chunks use the XOR pipelines on these inputs
+    and are shorter than in the fixed mode, and each table entry's id equals
+    the one encode_segment chose for that chunk."""
+    w = synth.Workload("s", 2, 4, 128, bits, g, seed=3, kind="lognormal", scale_sigma=1.5,
+                       tokens=4096)
+    x = synth.bf16_bits(synth.dense_kv(w)).reshape(-1, 128)
+    ds, df = _search_desc(bits, g, 2, 4, 4096), _search_desc(bits, g, 2, 4, 4096,
+                                                              mode=oracle.LOSSLESS_FIXED)
+    st, s = oracle.compress(ds, x)
+    stf, sf = oracle.compress(df, x)
+    assert st == stf == oracle.OK
+    lay = ds.layout()
+    sizes, ids = _entries(s, lay.n_chunks)
+    fsizes, fids = _entries(sf, lay.n_chunks)
+    meta = [oracle.meta_chunk_index(lay, k) for k in range(lay.n_meta)]
+    assert not fids.any()
+    assert set(ids[meta].tolist()) <= {1, 3} and sizes[meta].sum() < fsizes[meta].sum()
+    for seg in (0, lay.n_seg - 1):
+        v0, v1 = oracle.segment_vectors(lay, seg)
+        _, chunks, pipes = oracle.encode_segment(ds, seg, x[v0:v1])
+        assert pipes[-1] == ids[oracle.meta_chunk_index(lay, seg)]
+        assert chunks[-1].size == sizes[oracle.meta_chunk_index(lay, seg)]
+    dst, y = oracle.decompress(s, ds)
+    dstf, yf = oracle.decompress(sf, df)
+    assert dst == dstf == oracle.OK and np.array_equal(y, yf)
+    # the thread pool gives the same bytes in search mode
+    st4, s4 = oracle.compress(ds, x, threads=4)
+    assert st4 == oracle.OK and np.array_equal(s4, s)
+
+
+@pytest.mark.parametrize("zero_chunk,fixed_kept,search_kept", [(1, False, True), (7, False, True),
+                                                                (8, True, True), (0, False, False)])
+def test_code_rule_threshold_moves_with_search(zero_chunk, fixed_kept, search_kept):
+    """Reading R16 with the chosen sizes: an all-zero code chunk saves
+    16384 - 2048 padded bytes in the fixed mode and 16384 - 256 in the search
+    mode (two-level form), so among 64 code chunks elimination is kept when
+    at most 56 (fixed) or 63 (search) chunks follow from it, itself
+    included: 64 * 14336 = 917504 >= 56 * 16384, 64 * 16128 = 1032192 ==
+    63 * 16384."""
+    per = 16384 * 8 // (128 * 4)
+    V = per * 64
+    x = torch.randn(V, 128, generator=torch.Generator().manual_seed(11))
+    x[zero_chunk * per:(zero_chunk + 1) * per] = 0
+    xb = synth.bf16_bits(x.to(torch.bfloat16))
+    for mode, kept, size in [(oracle.LOSSLESS_FIXED, fixed_kept, 2048),
+                             (oracle.LOSSLESS_SEARCH, search_kept, 256)]:
+        d = oracle.StreamDesc(4, 128, 128, 1, V // 2048, [1024], 0, lossless=mode)
+        st, s = oracle.compress(d, xb)
+        assert st == oracle.OK
+        sizes, ids = _entries(s, d.layout().n_chunks)
+        assert sizes[zero_chunk] == (size if kept else 16384), mode
+        assert ids[zero_chunk] == (2 if kept and size == 256 else 0)
+        assert s[11] == (1 if kept else 0)
+        dst, y = oracle.decompress(s, d)
+        assert dst == oracle.OK and np.array_equal(y, oracle.decompress(
+            oracle.compress(oracle.StreamDesc(4, 128, 128, 1, V // 2048, [1024], 0), xb)[1],
+            oracle.StreamDesc(4, 128, 128, 1, V // 2048, [1024], 0))[1])
+
+
+def test_decoder_rejects_bad_pipeline_ids():
+    """A table id above 3, a nonzero id on a raw chunk, and an XOR id on a
+    code chunk are corrupt streams."""
+    w = synth.Workload("s", 1, 2, 128, 2, 32, seed=4, kind="lognormal", scale_sigma=1.5,
+                       tokens=4096)
+    x = synth.bf16_bits(synth.dense_kv(w)).reshape(-1, 128).copy()
+    x[:512] = 0                                         # an all-zero code chunk (id 2)
+    d = _search_desc(2, 32, 1, 2, 4096)
+    st, s = oracle.compress(d, x)
+    lay = d.layout()
+    sizes, ids = _entries(s, lay.n_chunks)
+    assert st == oracle.OK and ids[0] == 2 and s[11] == 1
+    m = oracle.meta_chunk_index(lay, 0)
+    raw = next(i for i in range(lay.n_code) if sizes[i] == 16384)
+
+    def with_id(i, new_id):
+        t = s.copy()
+        e = t[64 + 8 * i:72 + 8 * i].view("<u8")
+        e[0] = (int(e[0]) & ((1 << 60) - 1)) | (new_id << 60)
+        return t
+    assert oracle.decompress(s, d)[0] == oracle.OK
+    for i, new_id in [(m, 4), (m, 15), (raw, 2), (0, 1), (0, 3)]:
+        assert oracle.decompress(with_id(i, new_id), d)[0] == oracle.CORRUPT, (i, new_id)
