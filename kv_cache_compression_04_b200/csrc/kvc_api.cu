@@ -3,6 +3,9 @@
 // nothing and keeps no state beyond per-kernel launch attributes.
 #include <string.h>
 
+#include <initializer_list>
+#include <utility>
+
 #include <cuda_runtime.h>
 
 #include "kvc_internal.h"
@@ -118,6 +121,17 @@ int sm_count() {
   return n;
 }
 
+// Rows at non-negative offsets below 64 GB from the base can be named by a
+// 32-bit count of 16-byte units (the kernels' narrow row copies).
+bool narrow_extent(std::initializer_list<std::pair<int64_t, int64_t>> dims, int64_t row_bytes) {
+  int64_t hi = row_bytes;
+  for (const auto &d : dims) {  // (stride in bytes, index count)
+    if (d.first < 0) return false;
+    if (d.second > 1) hi += d.first * (d.second - 1);
+  }
+  return hi <= (int64_t(1) << 36);
+}
+
 DenseLayout dense_layout(const kvc_kv_desc *kv, const Shape &s) {
   DenseLayout L{};
   L.base = static_cast<uint8_t *>(kv->data);
@@ -128,6 +142,9 @@ DenseLayout dense_layout(const kvc_kv_desc *kv, const Shape &s) {
   L.T = make_fastdiv(s.T ? uint32_t(s.T) : 1u);
   L.H = make_fastdiv(kv->kv_heads ? uint32_t(kv->kv_heads) : 1u);
   L.tokens = uint32_t(s.T);
+  L.narrow = narrow_extent({{L.s_l, kv->layers}, {L.s_kv, 2}, {L.s_h, kv->kv_heads},
+                            {L.s_t, int64_t(s.T)}},
+                           2 * int64_t(s.D));
   return L;
 }
 
@@ -183,6 +200,9 @@ void paged_layout(const kvc_kv_desc *kv, const Shape &s, PagedLayout &L) {
   L.H = make_fastdiv(kv->kv_heads ? uint32_t(kv->kv_heads) : 1u);
   L.PT = make_fastdiv(uint32_t(kv->page_tokens));
   L.n_req = s.n_req;
+  L.narrow = narrow_extent({{L.s_l, kv->layers}, {L.s_p, kv->num_pages}, {L.s_kv, 2},
+                            {L.s_h, kv->kv_heads}, {L.s_slot, kv->page_tokens}},
+                           2 * int64_t(s.D));
   L.cum[0] = 0;
   for (uint32_t r = 0; r < s.n_req; ++r) L.cum[r + 1] = L.cum[r] + uint32_t(kv->seq_lens[r]);
 }

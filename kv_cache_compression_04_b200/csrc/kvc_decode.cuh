@@ -214,7 +214,7 @@ __device__ __forceinline__ void store_block_tma(const DenseLayout &lay, const ui
   stage_busy = true;
 }
 
-template <int D, int BITS, int G, class Layout>
+template <int D, int BITS, int G, class Layout, bool kNarrow>
 __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, uint8_t *smem,
                             const uint32_t *cum) {
   using C = Cfg<D, BITS, G>;
@@ -333,7 +333,10 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     __syncwarp();  // the previous block's scatter has read the buffer
     stage_row<D>(out, stage);
     __syncwarp();
-    scatter_rows<D>(stage, dst);
+    if constexpr (kNarrow)
+      scatter_rows_narrow<D / 8>(stage, lay.base, dst ? uint32_t((dst - lay.base) >> 4) : ~0u);
+    else
+      scatter_rows<D>(stage, dst);
   };
 
   // Raw code chunks, blocks of 32 vectors round-robin over the warps (chunks
@@ -374,7 +377,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   bulk_wait_all<0>();
 }
 
-template <int D, class Layout>
+template <int D, class Layout, bool kNarrow>
 __global__ void __launch_bounds__(kDecThreads)
     decode_kernel(const __grid_constant__ DecArgs a, const __grid_constant__ Layout lay) {
   constexpr bool kPaged = kIsPaged<Layout>;
@@ -431,26 +434,26 @@ __global__ void __launch_bounds__(kDecThreads)
   const uint32_t bits = ctl->bits, group = ctl->group;
   if constexpr (D == 128) {
     if (bits == 4 && group == 128)
-      decode_body<128, 4, 128>(a, lay, ctl, smem, s_cum);
+      decode_body<128, 4, 128, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 64)
-      decode_body<128, 4, 64>(a, lay, ctl, smem, s_cum);
+      decode_body<128, 4, 64, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 32)
-      decode_body<128, 4, 32>(a, lay, ctl, smem, s_cum);
+      decode_body<128, 4, 32, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else if (bits == 2 && group == 128)
-      decode_body<128, 2, 128>(a, lay, ctl, smem, s_cum);
+      decode_body<128, 2, 128, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else if (bits == 2 && group == 64)
-      decode_body<128, 2, 64>(a, lay, ctl, smem, s_cum);
+      decode_body<128, 2, 64, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else
-      decode_body<128, 2, 32>(a, lay, ctl, smem, s_cum);
+      decode_body<128, 2, 32, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
   } else {
     if (bits == 4 && group == 64)
-      decode_body<64, 4, 64>(a, lay, ctl, smem, s_cum);
+      decode_body<64, 4, 64, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 32)
-      decode_body<64, 4, 32>(a, lay, ctl, smem, s_cum);
+      decode_body<64, 4, 32, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else if (bits == 2 && group == 64)
-      decode_body<64, 2, 64>(a, lay, ctl, smem, s_cum);
+      decode_body<64, 2, 64, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else
-      decode_body<64, 2, 32>(a, lay, ctl, smem, s_cum);
+      decode_body<64, 2, 32, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
   }
 }
 

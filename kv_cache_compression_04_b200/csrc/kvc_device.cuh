@@ -648,6 +648,78 @@ __device__ __forceinline__ void scatter_rows_p(const uint8_t *wbuf, uint8_t *row
   }
 }
 
+// The same two moves with each lane's row given as a 32-bit offset from
+// `base` in 16-byte units (layouts whose rows all lie in [base, base + 64 GB)
+// at non-negative offsets, flagged `narrow` by the host): one shuffle per row
+// instead of two, and the swizzled shared-memory positions of a lane's pieces
+// computed once per call. Piece c = lane % P of row r = i * RPI + lane / P is
+// at swz_offset(r, c), whose bank term ((c ^ r) & 7) depends on i only
+// through (i * RPI) & 7, so its K = 8 / RPI (at least 1) distinct addresses
+// serve every i with a constant added.
+__device__ __forceinline__ void cp_async16_s(uint32_t sdst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sdst), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t saddr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(saddr));
+  return v;
+}
+template <int P>
+struct RowPieces {
+  static constexpr int RPI = 32 / P;              // rows per copy instruction
+  static constexpr int NI = 32 / RPI;             // instructions per 32 rows
+  static constexpr int K = RPI >= 8 ? 1 : 8 / RPI;
+  uint32_t s[K];
+  int c, rs;
+  __device__ __forceinline__ explicit RowPieces(const uint8_t *wbuf) {
+    const int lane = threadIdx.x & 31;
+    c = lane % P;
+    rs = lane / P;
+    const uint32_t sb = smem_u32(wbuf) + uint32_t((c >> 3) * 4096 + rs * 128);
+    const uint32_t k = uint32_t((c & 7) ^ (rs & 7));
+#pragma unroll
+    for (int j = 0; j < K; ++j) s[j] = sb + ((k ^ uint32_t((j * RPI) & 7)) << 4);
+  }
+  __device__ __forceinline__ uint32_t at(int i) const { return s[i % K] + uint32_t(i * RPI * 128); }
+};
+// Lanes without a row pass offset 0 (their row reads base's first row,
+// which is not used).
+template <int P>
+__device__ __forceinline__ void gather_rows_narrow(uint8_t *wbuf, const uint8_t *base,
+                                                   uint32_t off16) {
+  const RowPieces<P> rp(wbuf);
+  const uint8_t *g = base + 16 * rp.c;
+#pragma unroll
+  for (int i = 0; i < RowPieces<P>::NI; ++i) {
+    const uint32_t o = __shfl_sync(0xFFFFFFFFu, off16, i * RowPieces<P>::RPI + rp.rs);
+    cp_async16_s(rp.at(i), g + uint64_t(o) * 16);
+  }
+  cp_async_commit();
+}
+// Lanes without a row pass ~0u (nothing is stored for them).
+template <int P>
+__device__ __forceinline__ void scatter_rows_narrow(const uint8_t *wbuf, uint8_t *base,
+                                                    uint32_t off16) {
+  constexpr int N = RowPieces<P>::NI, B = 8;
+  const RowPieces<P> rp(wbuf);
+  uint8_t *g = base + 16 * rp.c;
+#pragma unroll
+  for (int i0 = 0; i0 < N; i0 += B) {
+    uint4 v[B];
+    uint32_t d[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+      d[i] = __shfl_sync(0xFFFFFFFFu, off16, (i0 + i) * RowPieces<P>::RPI + rp.rs);
+      v[i] = lds128(rp.at(i0 + i));
+    }
+#pragma unroll
+    for (int i = 0; i < B; ++i)
+      if (d[i] != ~0u) *reinterpret_cast<uint4 *>(g + uint64_t(d[i]) * 16) = v[i];
+  }
+}
+
 // Rows of D bf16 (2*D bytes, D/8 pieces).
 template <int D>
 __device__ __forceinline__ void gather_rows(uint8_t *wbuf, const uint8_t *row, const void *dummy) {

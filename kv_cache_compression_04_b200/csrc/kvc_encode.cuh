@@ -319,7 +319,7 @@ __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t b
 // ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
-template <int D, int BITS, int G, class Layout>
+template <int D, int BITS, int G, class Layout, bool kNarrow>
 __global__ void __launch_bounds__(kEncThreads, 1)
     encode_kernel(const __grid_constant__ EncArgs a, const __grid_constant__ Layout lay) {
   using C = Cfg<D, BITS, G>;
@@ -403,8 +403,15 @@ __global__ void __launch_bounds__(kEncThreads, 1)
   if (!use_tma) {
     grid_dependency_wait();  // the workspace clear (src_of may record a status)
     // Row addresses are looked up one block ahead of their gather, so the
-    // page-table read overlaps a block of arithmetic.
-    if (blk < n_blocks) gather_rows<D>(wbuf, src_of(blk * 32 + lane), a.out);
+    // page-table read overlaps a block of arithmetic; a layout whose rows fit
+    // 32-bit offsets from its base (the common case) uses the narrow copies.
+    auto gather = [&](const uint8_t *rowp) {
+      if constexpr (kNarrow)
+        gather_rows_narrow<D / 8>(wbuf, lay.base, rowp ? uint32_t((rowp - lay.base) >> 4) : 0u);
+      else
+        gather_rows<D>(wbuf, rowp, a.out);
+    };
+    if (blk < n_blocks) gather(src_of(blk * 32 + lane));
     const uint8_t *next = src_of((blk + stride) * 32 + lane);
 #pragma unroll 1
     for (; blk < n_blocks; blk += stride) {
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       Pairs<D> y;
       E::unpack_swz(wbuf, lane, a.sign_mask, y);
       __syncwarp();  // every lane has read the buffer; the next gather may overwrite it
-      if (blk + stride < n_blocks) gather_rows<D>(wbuf, next, a.out);
+      if (blk + stride < n_blocks) gather(next);
       next = src_of((blk + 2 * stride) * 32 + lane);
       finish_block(blk, v, v < V, y);
     }

@@ -126,6 +126,7 @@ struct DenseLayout {
   FastDiv T, H;                 // tokens, kv_heads
   uint32_t tokens;
   uint32_t tma;
+  uint32_t narrow;  // 1: every row at a non-negative offset below 64 GB from base
 };
 
 struct PagedLayout {
@@ -136,6 +137,7 @@ struct PagedLayout {
   int64_t num_pages;
   FastDiv T, H, PT;                     // total tokens, kv_heads, page tokens
   uint32_t n_req;
+  uint32_t narrow;  // 1: every row at a non-negative offset below 64 GB from base
   uint32_t cum[KVC_MAX_REQUESTS + 1];   // token prefix per request
 };
 

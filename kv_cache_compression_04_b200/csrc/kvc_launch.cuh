@@ -42,9 +42,9 @@ inline cudaError_t prepare(Kernel k, size_t smem) {
   return e;
 }
 
-template <int D, int BITS, int G, class Layout>
-cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
-  auto k = encode_kernel<D, BITS, G, Layout>;
+template <int D, int BITS, int G, class Layout, bool kNarrow>
+cudaError_t launch_enc_k(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
+  auto k = encode_kernel<D, BITS, G, Layout, kNarrow>;
   const size_t smem = enc_smem_bytes<D>(kIsPaged<Layout>);
   struct Tag {};
   cudaError_t e = prepare<Tag>(k, smem);
@@ -56,13 +56,30 @@ cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_
   // a dependent launch after the workspace clear: see encode_kernel
   return launch_after(k, grid, kEncThreads, smem, st, a, lay);
 }
+// Paged rows named by 32-bit offsets when the pool allows (narrow row
+// copies). Dense inputs keep the 64-bit gather next to their tensor-map
+// loads: both paths in one kernel would not fit its registers.
+template <int D, int BITS, int G, class Layout>
+cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
+  if constexpr (kIsPaged<Layout>) {
+    if (lay.narrow) return launch_enc_k<D, BITS, G, Layout, true>(a, lay, sms, st);
+  }
+  return launch_enc_k<D, BITS, G, Layout, false>(a, lay, sms, st);
+}
+
+template <int D, class Layout, bool kNarrow>
+cudaError_t prepare_dec(const size_t smem) {
+  struct Tag {};
+  return prepare<Tag>(decode_kernel<D, Layout, kNarrow>, smem);
+}
 
 template <int D, class Layout>
 cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_t st) {
-  auto k = decode_kernel<D, Layout>;
+  // rows named by 32-bit offsets when the layout allows (narrow row copies)
+  auto k = lay.narrow ? decode_kernel<D, Layout, true> : decode_kernel<D, Layout, false>;
   const size_t smem = DecSmem<D>::bytes(kIsPaged<Layout>);
-  struct Tag {};
-  cudaError_t e = prepare<Tag>(k, smem);
+  cudaError_t e = lay.narrow ? prepare_dec<D, Layout, true>(smem)
+                             : prepare_dec<D, Layout, false>(smem);
   if (e != cudaSuccess) return e;
   // one CTA per SM; tiles are the code chunks (at least 128 vectors each)
   const uint64_t min_vc = uint64_t(kChunk) / (uint64_t(D) * 4 / 8);
