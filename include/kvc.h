@@ -62,17 +62,43 @@ typedef enum {
   KVC_ERR_CUDA = 8         /* CUDA runtime error (launch, copy, device)       */
 } kvc_status;
 
-/* Quantization parameters.
+/* Lossless-stage modes of the encoder ("Beyond Compression Ratio: High-
+ * Throughput KV Compression for Disaggregated LLM Serving", Abstract and
+ * Methodology: a searchable backend that composes primitives into
+ * pipelines). A stored chunk's pipeline id (bits 60..63 of its table entry)
+ * says which primitives were applied:
+ *   0  bit-plane shuffle of 32-bit words, zero-byte elimination with a
+ *      2048-byte bitmap
+ *   1  each 32-bit word XOR the previous word, restarting every 32 vectors
+ *      (meta chunks only), then as 0
+ *   2  bit-plane shuffle, two-level zero-byte elimination: the 2048-byte
+ *      bitmap itself eliminated under a 256-byte bitmap
+ *   3  the XOR of 1, then as 2
+ * KVC_LOSSLESS_FIXED uses pipeline 0 only. KVC_LOSSLESS_SEARCH gives every
+ * full chunk the shortest of its candidates (code chunks: 0 and 2; meta
+ * chunks: 0..3, or 0 and 1 when a vector has one group), ties to the lower
+ * id. KVC_LOSSLESS_NONE stores every chunk raw (no lossless stage). In every
+ * mode a chunk is stored transformed only if that makes it strictly shorter,
+ * and the code region follows the elimination rule documented at
+ * kvc_compress. A decoder handles every mode. */
+enum { KVC_LOSSLESS_FIXED = 0, KVC_LOSSLESS_SEARCH = 1, KVC_LOSSLESS_NONE = 2 };
+
+/* Quantization and lossless parameters.
  *  bits       2 or 4 bits per code.
  *  group_size 32, 64 or 128 consecutive channels of the transformed vector
  *             share one fp16 zero and scale; must divide head_dim.
  *  sign_seed  seeds the +-1 diagonal: channel c is negated iff bit (c mod 64)
  *             of SplitMix64 output number floor(c/64), counted from state =
- *             sign_seed, is 1. */
+ *             sign_seed, is 1.
+ *  lossless   KVC_LOSSLESS_* (encoder only); other values are refused with
+ *             KVC_ERR_UNSUPPORTED.
+ *  reserved   must be 0. */
 typedef struct {
   int32_t bits;
   int32_t group_size;
   uint64_t sign_seed;
+  int32_t lossless;
+  int32_t reserved;
 } kvc_params;
 
 enum { KVC_DENSE = 0, KVC_PAGED = 1 };
@@ -159,12 +185,14 @@ size_t kvc_decompress_workspace_bytes(const kvc_kv_desc *out);
  * least kvc_max_compressed_bytes). The stream length is written to the
  * header's stream_bytes field and, if out_bytes_dev (DEVICE) is not null, to
  * *out_bytes_dev. Stream layout (little-endian): 64-byte header; u64 chunk
- * table (bits 0..15 unpadded chunk size, bits 16..63 offset from the data base
- * in 16-byte units); u32 token count per request; zero padding to 16 bytes;
+ * table (bits 0..15 unpadded chunk size, bits 16..59 offset from the data base
+ * in 16-byte units, bits 60..63 the chunk's lossless pipeline id, 0 for a
+ * raw chunk); u32 token count per request; zero padding to 16 bytes;
  * the chunks, each zero-padded to 16 bytes. The code and meta regions are cut
  * into 16 KB chunks; a meta chunk covers group_size*bits/32 code chunks. Chunk
  * order (table and data): every code chunk, then every meta chunk. A chunk is
- * stored zero-byte eliminated only if that makes it shorter; in the code
+ * stored through a lossless pipeline (params->lossless) only if that makes it
+ * shorter; in the code
  * region, only if moreover the padded bytes saved there are at least 1/64 of
  * the padded bytes from the first shrinking code chunk to the region's end
  * (the bytes that shift), else every code chunk is stored raw. The call
@@ -259,6 +287,26 @@ kvc_status kvc_compress_unfused(const kvc_kv_desc *kv, const kvc_params *params,
                                 void *out, size_t out_capacity,
                                 uint64_t *out_bytes_dev, void *workspace,
                                 size_t workspace_bytes, kvc_stream_t stream);
+
+/* Measurement only (no page defines these; they let a benchmark time each
+ * kernel of a call with CUDA events on the call's own stream). The same work
+ * and results as kvc_compress / kvc_decompress, with n_events == 5 caller-
+ * created CUDA events (cudaEvent_t, passed as void *) recorded on `stream`:
+ * events[0] before the call's first kernel and events[i] after its i-th
+ * kernel. Compress: workspace clear, encode, finishing (table, meta chunks,
+ * header), compaction. Decompress: status clear, meta chunk expansion,
+ * decode of eliminated code chunks, decode. A kernel that a call does not
+ * need gets an empty interval. The kernels of a timed call start in plain
+ * stream order, without overlapping the previous kernel's tail, so a timed
+ * call can take a few microseconds longer than an ordinary one. Other
+ * n_events or a null event: KVC_ERR_INVALID_ARG. */
+kvc_status kvc_compress_timed(const kvc_kv_desc *kv, const kvc_params *params, void *out,
+                              size_t out_capacity, uint64_t *out_bytes_dev, void *workspace,
+                              size_t workspace_bytes, void *const *events, int n_events,
+                              kvc_stream_t stream);
+kvc_status kvc_decompress_timed(const void *in, size_t in_bytes, const kvc_kv_desc *out,
+                                void *workspace, size_t workspace_bytes, void *const *events,
+                                int n_events, kvc_stream_t stream);
 
 #ifdef __cplusplus
 }

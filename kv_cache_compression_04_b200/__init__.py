@@ -28,7 +28,8 @@ STATUS = ["KVC_OK", "KVC_ERR_INVALID_ARG", "KVC_ERR_UNSUPPORTED", "KVC_ERR_CAPAC
 EXPORTS = ["kvc_max_compressed_bytes", "kvc_workspace_bytes", "kvc_compress",
            "kvc_decompress", "kvc_stream_status", "kvc_status_string", "kvc_compress_noalloc",
            "kvc_decompress_workspace_bytes", "kvc_unfused_workspace_bytes",
-           "kvc_compress_unfused", "kvc_test_compress_stalled"]
+           "kvc_compress_unfused", "kvc_test_compress_stalled", "kvc_compress_timed",
+           "kvc_decompress_timed"]
 
 
 class KvcError(RuntimeError):
@@ -38,7 +39,12 @@ class KvcError(RuntimeError):
 
 
 class kvc_params(C.Structure):
-    _fields_ = [("bits", C.c_int32), ("group_size", C.c_int32), ("sign_seed", C.c_uint64)]
+    _fields_ = [("bits", C.c_int32), ("group_size", C.c_int32), ("sign_seed", C.c_uint64),
+                ("lossless", C.c_int32), ("reserved", C.c_int32)]
+
+
+# Lossless-stage modes (kvc_params.lossless) and pipeline ids of a chunk.
+KVC_LOSSLESS_FIXED, KVC_LOSSLESS_SEARCH, KVC_LOSSLESS_NONE = range(3)
 
 
 class kvc_kv_desc(C.Structure):
@@ -89,6 +95,12 @@ def lib() -> C.CDLL:
         L.kvc_compress_unfused.restype = C.c_int
         L.kvc_compress_unfused.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p,
                                            C.c_size_t, C.c_void_p]
+        L.kvc_compress_timed.restype = C.c_int
+        L.kvc_compress_timed.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p,
+                                         C.c_size_t, C.POINTER(C.c_void_p), C.c_int, C.c_void_p]
+        L.kvc_decompress_timed.restype = C.c_int
+        L.kvc_decompress_timed.argtypes = [C.c_void_p, C.c_size_t, D, C.c_void_p, C.c_size_t,
+                                           C.POINTER(C.c_void_p), C.c_int, C.c_void_p]
         L.kvc_test_compress_stalled.restype = C.c_int
         L.kvc_test_compress_stalled.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p,
                                                 C.c_void_p, C.c_size_t, C.c_uint32, C.c_uint64,
@@ -141,6 +153,26 @@ def kvc_test_compress_stalled(desc, params, out_ptr, out_capacity, out_bytes_dev
                                            wait_ns, stream)
 
 
+def _event_array(events):
+    """torch.cuda.Event objects -> a C array of their cudaEvent_t handles."""
+    return (C.c_void_p * len(events))(*[e.cuda_event for e in events])
+
+
+def kvc_compress_timed(desc, params, out_ptr, out_capacity, out_bytes_dev_ptr, ws_ptr, ws_bytes,
+                       events, stream) -> int:
+    """kvc_compress recording `events` (5 torch.cuda.Event, created with
+    enable_timing=True and already created on the device) around its kernels."""
+    arr = _event_array(events)
+    return lib().kvc_compress_timed(C.byref(desc), C.byref(params), out_ptr, out_capacity,
+                                    out_bytes_dev_ptr, ws_ptr, ws_bytes, arr, len(events), stream)
+
+
+def kvc_decompress_timed(in_ptr, in_bytes, desc, ws_ptr, ws_bytes, events, stream) -> int:
+    arr = _event_array(events)
+    return lib().kvc_decompress_timed(in_ptr, in_bytes, C.byref(desc), ws_ptr, ws_bytes, arr,
+                                      len(events), stream)
+
+
 def kvc_decompress(in_ptr, in_bytes, desc, ws_ptr, ws_bytes, stream) -> int:
     return lib().kvc_decompress(in_ptr, in_bytes, C.byref(desc), ws_ptr, ws_bytes, stream)
 
@@ -154,8 +186,9 @@ def kvc_status_string(status: int) -> str:
 
 
 # ------------------------------------------------------- descriptor helpers --
-def params(bits: int, group: int, sign_seed: int = 0) -> kvc_params:
-    return kvc_params(bits, group, sign_seed)
+def params(bits: int, group: int, sign_seed: int = 0,
+           lossless: int = KVC_LOSSLESS_FIXED) -> kvc_params:
+    return kvc_params(bits, group, sign_seed, lossless, 0)
 
 
 def dense_desc(kv) -> kvc_kv_desc:
@@ -210,8 +243,9 @@ class Codec:
     Buffers come from PyTorch's caching allocator (plumbing only); every
     compute step runs in libkvc's kernels. Errors raise KvcError."""
 
-    def __init__(self, bits: int = 4, group: int = 128, sign_seed: int = 0):
-        self.params = params(bits, group, sign_seed)
+    def __init__(self, bits: int = 4, group: int = 128, sign_seed: int = 0,
+                 lossless: int = KVC_LOSSLESS_FIXED):
+        self.params = params(bits, group, sign_seed, lossless)
 
     def buffers(self, desc: kvc_kv_desc, device="cuda"):
         import torch

@@ -13,6 +13,13 @@
 
 using namespace kvc;
 
+namespace kvc {
+KernelTiming &kernel_timing() {
+  static thread_local KernelTiming t;
+  return t;
+}
+}  // namespace kvc
+
 namespace {
 
 struct Shape {
@@ -37,9 +44,17 @@ __global__ void __launch_bounds__(256) clear_words_kernel(uint4 *p, uint64_t n) 
 inline cudaError_t clear_words(void *p, uint64_t bytes, int sms, cudaStream_t st) {
   const uint64_t n = bytes / 16, want = (n + 255) / 256, cap = uint64_t(sms) * 4;
   const int grid = int(want == 0 ? 1 : (want < cap ? want : cap));
+  timing_mark(st);  // before a call's first kernel
   clear_words_kernel<<<grid, 256, 0, st>>>(static_cast<uint4 *>(p), n);
+  timing_mark(st);
   return cudaGetLastError();
 }
+
+// Sets this thread's kernel timing for the duration of one timed call.
+struct TimedCall {
+  explicit TimedCall(const cudaEvent_t *ev) { kernel_timing() = KernelTiming{ev, 0}; }
+  ~TimedCall() { kernel_timing() = KernelTiming{}; }
+};
 
 bool stride_ok(int64_t s) { return s % 8 == 0; }  // 16-byte vector starts
 
@@ -84,6 +99,8 @@ kvc_status describe(const kvc_kv_desc *kv, const kvc_params *p, Shape &s) {
   if (p->group_size != 32 && p->group_size != 64 && p->group_size != 128)
     return KVC_ERR_UNSUPPORTED;
   if (p->group_size > s.D) return KVC_ERR_UNSUPPORTED;
+  if (p->lossless < KVC_LOSSLESS_FIXED || p->lossless > KVC_LOSSLESS_NONE || p->reserved != 0)
+    return KVC_ERR_UNSUPPORTED;
   s.bits = p->bits;
   s.G = p->group_size;
   // Stream layout (readings R12/R13): codes and meta chunked separately into
@@ -186,7 +203,33 @@ void add_tensor_map(const kvc_kv_desc *kv, const Shape &s, DenseLayout &L) {
     L.tma = 1;
 }
 
+// Tensor map of a paged pool for the encoder's run loads: 5-D [layers]
+// [pages][2 * kv_heads][page_tokens][head_dim] with kv and head merged into
+// one dimension (needs stride_kv == kv_heads * stride_head), boxes of 8 slots
+// x 64 channels with 128-byte swizzle (needs page_tokens % 8 == 0).
+void add_tensor_map_paged(const kvc_kv_desc *kv, const Shape &s, PagedLayout &L) {
+  L.tma = 0;
+  if (s.V == 0 || kv->page_tokens % 8 != 0 || kv->stride_kv != kv->kv_heads * kv->stride_head)
+    return;
+  if (kv->stride_slot <= 0 || kv->stride_head <= 0 || kv->stride_page <= 0 || kv->stride_layer <= 0)
+    return;
+  const EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return;
+  const cuuint64_t dims[5] = {cuuint64_t(s.D), cuuint64_t(kv->page_tokens),
+                              cuuint64_t(2 * kv->kv_heads), cuuint64_t(kv->num_pages),
+                              cuuint64_t(kv->layers)};
+  const cuuint64_t strides[4] = {cuuint64_t(L.s_slot), cuuint64_t(L.s_h), cuuint64_t(L.s_p),
+                                 cuuint64_t(L.s_l)};
+  const cuuint32_t box[5] = {64, 8, 1, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  if (fn(&L.tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, kv->data, dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+    L.tma = 1;
+}
+
 void paged_layout(const kvc_kv_desc *kv, const Shape &s, PagedLayout &L) {
+  L.tma = 0;  // add_tensor_map_paged sets it for the encoder
   L.base = static_cast<uint8_t *>(kv->data);
   L.s_l = kv->stride_layer * 2;
   L.s_p = kv->stride_page * 2;
@@ -266,10 +309,11 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   a.first_inv = ctl + 4;
   a.saved = reinterpret_cast<unsigned long long *>(ctl + 6);
   a.code_nnz = reinterpret_cast<unsigned long long *>(ws + w.code_nnz);
-  a.meta_nnz = reinterpret_cast<uint32_t *>(ws + w.meta_nnz);
+  a.meta_nnz = reinterpret_cast<unsigned long long *>(ws + w.meta_nnz);
   a.ws_meta = ws + w.meta;
   a.ymid = unfused ? reinterpret_cast<float *>(ws + round256(s.ws_bytes)) : nullptr;
   a.one = 1.0f;
+  a.mode = uint32_t(params->lossless);
   sign_masks(params->sign_seed, s.D, a.sign_mask);
 
   FinArgs f{};
@@ -307,6 +351,7 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   f.n_req = s.n_req;
   f.tokens = s.T;
   f.seed = params->sign_seed;
+  f.mode = uint32_t(params->lossless);
   f.wait_ns = wait_ns;
   f.ticket_skip = ticket_skip;
 
@@ -321,17 +366,22 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
     } else if (s.n_code) {
       e = s.D == 128 ? launch_encode_dense_d128(s.bits, s.G, a, L, sms, cs)
                      : launch_encode_dense_d64(s.bits, s.G, a, L, sms, cs);
+    } else {
+      timing_mark(cs);  // no encode kernel: its interval is empty
     }
     if (e == cudaSuccess) e = launch_finish_dense(f, L, sms, cs);
   } else {
     static thread_local PagedLayout L;  // large (4 KB) parameter block
     paged_layout(kv, s, L);
+    add_tensor_map_paged(kv, s, L);
     if (s.n_code && unfused) {
       e = launch_transform_paged(s.D, a, L, sms, cs);
       if (e == cudaSuccess) e = launch_quantize(s.D, s.bits, s.G, a, sms, cs);
     } else if (s.n_code) {
       e = s.D == 128 ? launch_encode_paged_d128(s.bits, s.G, a, L, sms, cs)
                      : launch_encode_paged_d64(s.bits, s.G, a, L, sms, cs);
+    } else {
+      timing_mark(cs);  // no encode kernel: its interval is empty
     }
     if (e == cudaSuccess) e = launch_finish_paged(f, L, sms, cs);
   }
@@ -362,6 +412,28 @@ kvc_status kvc_test_compress_stalled(const kvc_kv_desc *kv, const kvc_params *pa
   if (skip_chunks == 0 || wait_ns == 0 || wait_ns > kWaitNs) return KVC_ERR_INVALID_ARG;
   return compress_impl(kv, params, out, out_capacity, out_bytes_dev, workspace, workspace_bytes,
                        stream, false, skip_chunks, wait_ns);
+}
+
+kvc_status kvc_compress_timed(const kvc_kv_desc *kv, const kvc_params *params, void *out,
+                              size_t out_capacity, uint64_t *out_bytes_dev, void *workspace,
+                              size_t workspace_bytes, void *const *events, int n_events,
+                              kvc_stream_t stream) {
+  if (!events || n_events != 5) return KVC_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return KVC_ERR_INVALID_ARG;
+  TimedCall timed(reinterpret_cast<const cudaEvent_t *>(events));
+  return compress_impl(kv, params, out, out_capacity, out_bytes_dev, workspace, workspace_bytes,
+                       stream, false);
+}
+
+kvc_status kvc_decompress_timed(const void *in, size_t in_bytes, const kvc_kv_desc *out,
+                                void *workspace, size_t workspace_bytes, void *const *events,
+                                int n_events, kvc_stream_t stream) {
+  if (!events || n_events != 5) return KVC_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return KVC_ERR_INVALID_ARG;
+  TimedCall timed(reinterpret_cast<const cudaEvent_t *>(events));
+  return kvc_decompress(in, in_bytes, out, workspace, workspace_bytes, stream);
 }
 
 kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *out,

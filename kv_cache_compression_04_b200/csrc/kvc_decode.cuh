@@ -237,17 +237,21 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   // seg0..seg1): each offset continues its predecessor, stays inside the
   // stream, and each size is the chunk's raw length or a valid eliminated
   // size (full chunks only); the last chunk ends the stream.
-  auto entry_ok = [&](uint64_t i, uint32_t len) {
+  // Pipeline ids (reading R17): 0 on a raw chunk; 0 or 2 on a code chunk;
+  // 0..3 on a meta chunk. Sizes: at least the bitmap of the chosen form.
+  auto entry_ok = [&](uint64_t i, uint32_t len, bool is_meta) {
     const uint64_t e = ld_u64(table + 8 * i);
-    const uint64_t off = (e >> 16) << 4;
-    const uint32_t size = uint32_t(e & 0xFFFFu);
+    const uint64_t off = entry_offset(e);
+    const uint32_t size = entry_size(e), pipe = entry_pipe(e);
     uint64_t expect = 0;
     if (i > 0) {
       const uint64_t p = ld_u64(table + 8 * (i - 1));
-      expect = ((p >> 16) << 4) + round16(p & 0xFFFFu);
+      expect = entry_offset(p) + round16(entry_size(p));
     }
-    bool ok = off == expect && base + off + round16(size) <= limit &&
-              (size == len || (len == uint32_t(kChunk) && size >= kBitmap && size < len));
+    const bool pipe_ok = size == len ? pipe == 0 : (pipe <= 3 && (is_meta || !(pipe & 1u)));
+    const uint32_t min_size = (pipe & 2u) ? uint32_t(kBitmap2) : uint32_t(kBitmap);
+    bool ok = off == expect && base + off + round16(size) <= limit && pipe_ok &&
+              (size == len || (len == uint32_t(kChunk) && size >= min_size && size < len));
     if (i + 1 == ctl->n_chunks) ok = ok && base + off + round16(size) == ctl->stream_bytes;
     return ok;
   };
@@ -258,11 +262,11 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     uint32_t bad = 0, elim = 0;
     for (uint32_t t = t0 + tid; t < t1; t += kDecThreads) {
       const uint32_t len = min(uint32_t(C::VC), V - t * C::VC) * C::CB;
-      bad |= !entry_ok(t, len);
-      elim |= uint32_t(ld_u64(table + 8 * uint64_t(t)) & 0xFFFFu) != len;
+      bad |= !entry_ok(t, len, false);
+      elim |= entry_size(ld_u64(table + 8 * uint64_t(t))) != len;
     }
     for (uint32_t s = seg0 + tid; s <= seg1; s += kDecThreads)
-      bad |= !entry_ok(uint64_t(n_tiles) + s, min(uint32_t(C::VM), V - s * C::VM) * C::MB);
+      bad |= !entry_ok(uint64_t(n_tiles) + s, min(uint32_t(C::VM), V - s * C::VM) * C::MB, true);
     const uint32_t sum = block_sum<kDecThreads>(bad | (elim << 16), ctl->red);
     any_elim = sum != 0;
     // such chunks must be announced by the header (elim_decode_kernel
@@ -279,8 +283,8 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     const uint32_t s = v0 / C::VM;
     const uint64_t me = ld_u64(table + 8 * (uint64_t(n_tiles) + s));
     const uint32_t mlen = min(uint32_t(C::VM), V - s * C::VM) * C::MB;
-    const uint8_t *chunk = uint32_t(me & 0xFFFFu) == mlen ? in + base + ((me >> 16) << 4)
-                                                          : a.ws_meta + uint64_t(s) * kChunk;
+    const uint8_t *chunk = entry_size(me) == mlen ? in + base + entry_offset(me)
+                                                  : a.ws_meta + uint64_t(s) * kChunk;
     return chunk + uint64_t(v0 - s * C::VM) * C::MB;
   };
   // Lane 0 starts the loads of a block's meta bytes and, unless they are
@@ -348,7 +352,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   auto raw_block = [&](uint32_t b) {  // block b lies in a raw code chunk
     const uint32_t t = (vs0 + b * 32) / C::VC;
     const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
-    return uint32_t(ce & 0xFFFFu) == min(uint32_t(C::VC), V - t * C::VC) * C::CB;
+    return entry_size(ce) == min(uint32_t(C::VC), V - t * C::VC) * C::CB;
   };
   auto next_raw = [&](uint32_t b) {
     while (any_elim && b < nblk && !raw_block(b)) b += kDecWarps;
@@ -358,7 +362,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     const uint32_t v0 = vs0 + b * 32, t = v0 / C::VC;
     const uint64_t ce = ld_u64(table + 8 * uint64_t(t));
     issue(v0, min(32u, vs1 - v0),
-          in + base + ((ce >> 16) << 4) + uint64_t(v0 - t * C::VC) * C::CB, k);
+          in + base + entry_offset(ce) + uint64_t(v0 - t * C::VC) * C::CB, k);
   };
   uint32_t b = next_raw(warp), k = 0;
   __syncwarp();
@@ -472,15 +476,17 @@ struct MetaCtl {
   uint64_t base, limit;
 };
 constexpr int kMetaCtas = 6;  // per SM: one chunk buffer each, so latency hides across CTAs
-constexpr size_t meta_smem_bytes() { return 2 * size_t(kChunk) + sizeof(MetaCtl); }
+// Shared memory: chunk buffer | plane-word scratch | 2 KB bitmap of the
+// two-level form | MetaCtl.
+constexpr size_t meta_smem_bytes() { return 2 * size_t(kChunk) + kBitmap + sizeof(MetaCtl); }
 
 template <int D>
 __global__ void __launch_bounds__(kMetaThreads, kMetaCtas)
     meta_expand_kernel(const __grid_constant__ DecArgs a) {
   grid_dependency_wait();  // the status clear
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t *buf = smem, *scr = smem + kChunk;
-  MetaCtl *ctl = reinterpret_cast<MetaCtl *>(smem + 2 * kChunk);
+  uint8_t *buf = smem, *scr = smem + kChunk, *bm = smem + 2 * kChunk;
+  MetaCtl *ctl = reinterpret_cast<MetaCtl *>(smem + 2 * kChunk + kBitmap);
   const int tid = threadIdx.x;
   if (tid == 0) {
     mbar_init(&ctl->full[0], 1);
@@ -505,11 +511,12 @@ __global__ void __launch_bounds__(kMetaThreads, kMetaCtas)
   // this CTA's chunks s = blockIdx.x + i * gridDim.x that used elimination
 #pragma unroll 1
   for (uint32_t s = blockIdx.x; s < n_meta; s += gridDim.x) {
-    const uint64_t e = ld_u64(table + 8 * (uint64_t(n_code) + s)), off = (e >> 16) << 4;
-    const uint32_t size = uint32_t(e & 0xFFFFu), len = min(vm, a.V - s * vm) * mb;
-    if (size == len) continue;  // raw: read in place by the decode kernel
-    const bool ok = len == uint32_t(kChunk) && size >= kBitmap && size < len &&
-                    base + off + round16(size) <= limit;
+    const uint64_t e = ld_u64(table + 8 * (uint64_t(n_code) + s)), off = entry_offset(e);
+    const uint32_t size = entry_size(e), pipe = entry_pipe(e), len = min(vm, a.V - s * vm) * mb;
+    if (size == len) continue;  // raw: read in place by the decode kernel (which checks it)
+    const bool ok = len == uint32_t(kChunk) && pipe <= 3 &&
+                    size >= ((pipe & 2u) ? uint32_t(kBitmap2) : uint32_t(kBitmap)) &&
+                    size < len && base + off + round16(size) <= limit;
     if (!ok) {
       if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
       continue;
@@ -522,7 +529,7 @@ __global__ void __launch_bounds__(kMetaThreads, kMetaCtas)
     }
     if (!mbar_wait(&ctl->full[0], phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
     phase ^= 1;
-    if (ze_decode<kMetaThreads>(buf, scr, ctl->red, size)) {
+    if (lossless_decode<kMetaThreads>(buf, scr, bm, ctl->red, size, pipe, 8 * mb)) {
       fence_proxy_async_smem();
       named_bar_sync(1, kMetaThreads);
       if (tid == 0) {
@@ -566,7 +573,8 @@ struct ElimSmem {
   static constexpr size_t meta = kElimWarps * WBUF;
   static constexpr size_t chunk = meta + kElimWarps * MBLK;
   static constexpr size_t scr = chunk + kChunk;
-  static constexpr size_t ctl = scr + kChunk;
+  static constexpr size_t bm = scr + kChunk;  // bitmap of the two-level form
+  static constexpr size_t ctl = bm + kBitmap;
   static constexpr size_t cum = ctl + ((sizeof(ElimCtl) + 15) & ~size_t(15));
   static constexpr size_t bytes(bool paged) {
     return cum + (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
@@ -587,6 +595,7 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
   uint8_t *mbuf = smem + S::meta + warp * S::MBLK;
   uint8_t *chunk = smem + S::chunk;
   uint8_t *scr = smem + S::scr;
+  uint8_t *bmp = smem + S::bm;
   bool use_tma = false;
   if constexpr (!kIsPaged<Layout>) use_tma = lay.tma != 0;
   bool stage_busy = false;
@@ -598,8 +607,8 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
     const uint32_t s = v0 / C::VM;
     const uint64_t e = ld_u64(table + 8 * (uint64_t(n_code) + s));
     const uint32_t mlen = min(uint32_t(C::VM), V - s * C::VM) * C::MB;
-    const uint64_t off = (e >> 16) << 4;
-    if (uint32_t(e & 0xFFFFu) != mlen) return a.ws_meta + uint64_t(s) * kChunk + (v0 - s * C::VM) * C::MB;
+    const uint64_t off = entry_offset(e);
+    if (entry_size(e) != mlen) return a.ws_meta + uint64_t(s) * kChunk + (v0 - s * C::VM) * C::MB;
     const uint64_t at = off + uint64_t(v0 - s * C::VM) * C::MB;
     return base + at + round16(nv * C::MB) <= limit ? a.in + base + at : nullptr;
   };
@@ -608,16 +617,17 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
     if (tid == 0) ctl->nlist = 0;
     __syncthreads();
     const uint64_t cc = uint64_t(blockIdx.x) + (j0 + tid) * gridDim.x;
-    if (cc < n_code && uint32_t(ld_u64(table + 8 * cc) & 0xFFFFu) != len_of(uint32_t(cc)))
+    if (cc < n_code && entry_size(ld_u64(table + 8 * cc)) != len_of(uint32_t(cc)))
       ctl->list[atomicAdd(&ctl->nlist, 1u)] = uint32_t(cc);
     __syncthreads();
     const uint32_t nl = ctl->nlist;
 #pragma unroll 1
     for (uint32_t i = 0; i < nl; ++i) {
       const uint32_t c = ctl->list[i];
-      const uint64_t e = ld_u64(table + 8 * uint64_t(c)), off = (e >> 16) << 4;
-      const uint32_t size = uint32_t(e & 0xFFFFu), len = len_of(c);
-      const bool good = len == uint32_t(kChunk) && size >= kBitmap && size < len &&
+      const uint64_t e = ld_u64(table + 8 * uint64_t(c)), off = entry_offset(e);
+      const uint32_t size = entry_size(e), len = len_of(c), pipe = entry_pipe(e);
+      const bool good = len == uint32_t(kChunk) && (pipe == 0 || pipe == 2) &&
+                        size >= (pipe ? uint32_t(kBitmap2) : uint32_t(kBitmap)) && size < len &&
                         base + off + round16(size) <= limit;
       if (tid == 0) {
         if (good) {
@@ -631,7 +641,7 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
       if (!good) continue;  // uniform over the CTA
       if (!mbar_wait(&ctl->zbar, zphase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
       zphase ^= 1;
-      const bool ok = ze_decode<kElimThreads>(chunk, scr, ctl->red, size);
+      const bool ok = lossless_decode<kElimThreads>(chunk, scr, bmp, ctl->red, size, pipe, 32u);
       if (!ok) {
         if (tid == 0) set_status(a.status, KVC_ERR_CORRUPT);
         __syncthreads();

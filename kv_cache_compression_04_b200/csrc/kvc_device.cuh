@@ -482,7 +482,8 @@ __device__ __forceinline__ uint32_t compact_selector(uint32_t n) {
 // threads). The caller passes another barrier before red is reused.
 template <int NT>
 __device__ __forceinline__ void ze_positions(const uint32_t (&cnt)[4], uint32_t *red,
-                                             uint32_t (&q)[4], uint32_t &total) {
+                                             uint32_t (&q)[4], uint32_t &total,
+                                             uint32_t data_base = kBitmap) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t i01 = warp_incl_scan(cnt[0] | (cnt[1] << 16));
   const uint32_t i23 = warp_incl_scan(cnt[2] | (cnt[3] << 16));
@@ -490,7 +491,7 @@ __device__ __forceinline__ void ze_positions(const uint32_t (&cnt)[4], uint32_t 
   const uint32_t r0 = t01 & 0xFFFFu, r1 = t01 >> 16, r2 = t23 & 0xFFFFu, r3 = t23 >> 16;
   if (lane == 0) red[warp] = r0 + r1 + r2 + r3;
   named_bar_sync(1, NT);
-  uint32_t base = kBitmap, all = 0;
+  uint32_t base = data_base, all = 0;
 #pragma unroll
   for (int w = 0; w < NT / 32; ++w) {
     const uint32_t v = red[w];
@@ -507,9 +508,12 @@ __device__ __forceinline__ void ze_positions(const uint32_t (&cnt)[4], uint32_t 
 // buf holds a full chunk (first 256 threads); on return it holds bitmap + nonzero bytes (the
 // caller knows their count from chunk_nnz_part). scr: 16 KB scratch. Each
 // word's nonzero bytes are packed by one byte permute and stored at its
-// position; the lanes of a warp store next to one another.
+// position; the lanes of a warp store next to one another. The bitmap goes
+// to `bitmap` (buf itself for the one-level form) and the nonzero bytes to
+// buf from `data_base` on.
 template <int NT>
-__device__ __forceinline__ void ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *red) {
+__device__ __forceinline__ bool ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *red,
+                                          uint8_t *bitmap = nullptr, uint32_t data_base = kBitmap) {
   static_assert(NT == 256, "eight warps of 512 plane words");
   __shared__ uint32_t lut[16];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -526,10 +530,15 @@ __device__ __forceinline__ void ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *
 #pragma unroll
     for (int e = 0; e < 4; ++e) nib[k] |= nz_nibble(x[k][e]) << (4 * e);
     cnt[k] = __popc(nib[k]);
-    reinterpret_cast<uint16_t *>(buf)[128 * warp + 32 * k + lane] = uint16_t(nib[k]);
+    reinterpret_cast<uint16_t *>(bitmap ? bitmap : buf)[128 * warp + 32 * k + lane] =
+        uint16_t(nib[k]);
   }
   uint32_t q[4], total;
-  ze_positions<NT>(cnt, red, q, total);
+  ze_positions<NT>(cnt, red, q, total, data_base);
+  if (data_base + total > uint32_t(kChunk)) {  // counts and data disagree: write nothing
+    named_bar_sync(1, NT);
+    return false;
+  }
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
 #pragma unroll
@@ -543,6 +552,7 @@ __device__ __forceinline__ void ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *
     }
   }
   named_bar_sync(1, NT);
+  return true;
 }
 
 // Inverse: buf holds bitmap + nonzero bytes (`size` bytes); on return it
@@ -551,7 +561,9 @@ __device__ __forceinline__ void ze_encode(uint8_t *buf, uint8_t *scr, uint32_t *
 // takes the next popcount(n) source bytes (an unaligned 4-byte window) and
 // spreads them with one byte permute.
 template <int NT>
-__device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *red, uint32_t size) {
+__device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *red, uint32_t size,
+                                          const uint8_t *bitmap = nullptr,
+                                          uint32_t data_base = kBitmap) {
   static_assert(NT == 256, "eight warps of 512 plane words");
   __shared__ uint32_t lut[16];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -560,12 +572,12 @@ __device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *
   uint32_t nib[4], cnt[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    nib[k] = reinterpret_cast<const uint16_t *>(buf)[128 * warp + 32 * k + lane];
+    nib[k] = reinterpret_cast<const uint16_t *>(bitmap ? bitmap : buf)[128 * warp + 32 * k + lane];
     cnt[k] = __popc(nib[k]);
   }
   uint32_t q[4], total;
-  ze_positions<NT>(cnt, red, q, total);  // lut visible after its barrier
-  if (total != size - kBitmap) {
+  ze_positions<NT>(cnt, red, q, total, data_base);  // lut visible after its barrier
+  if (total != size - data_base) {
     named_bar_sync(1, NT);  // red read by all before anyone reuses it
     return false;
   }
@@ -591,14 +603,157 @@ __device__ __forceinline__ bool ze_decode(uint8_t *buf, uint8_t *scr, uint32_t *
   return true;
 }
 
+// ------------------------------------ composable pipelines (reading R17) --
+// A stored chunk's pipeline id: bit 0 = the XOR of each word with the
+// previous one, restarting every `run` words (32 vectors), before the
+// bit-plane shuffle; bit 1 = the two-level form of zero-byte elimination
+// (the 2048-byte bitmap reduced to a 256-byte map and its nonzero bytes).
+
+// Forward XOR over the 4096 words of buf: w'[j] = w[j] ^ w[j - 1] unless j
+// starts a run. Thread t (first 256) rewrites words 16t .. 16t+15.
+template <int NT>
+__device__ __forceinline__ void xor_runs_forward(uint8_t *buf, uint32_t run) {
+  static_assert(NT == 256, "16 words per thread");
+  uint32_t *w = reinterpret_cast<uint32_t *>(buf);
+  const uint32_t t = threadIdx.x;
+  uint32_t v[17];
+  v[0] = t ? w[16 * t - 1] : 0u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 x = reinterpret_cast<const uint4 *>(w + 16 * t)[q];
+    v[4 * q + 1] = x.x, v[4 * q + 2] = x.y, v[4 * q + 3] = x.z, v[4 * q + 4] = x.w;
+  }
+  named_bar_sync(1, NT);  // every thread has read its predecessor's last word
+  uint32_t o[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) o[i] = ((16 * t + i) % run) ? v[i + 1] ^ v[i] : v[i + 1];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    reinterpret_cast<uint4 *>(w + 16 * t)[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2],
+                                                          o[4 * q + 3]);
+  named_bar_sync(1, NT);
+}
+
+// Inverse: each word becomes the XOR of its run's words up to itself. A run
+// of 32, 64 or 128 words spans 2, 4 or 8 consecutive threads (aligned in the
+// warp), which exchange their partial XORs by shuffles.
+template <int NT>
+__device__ __forceinline__ void xor_runs_inverse(uint8_t *buf, uint32_t run) {
+  static_assert(NT == 256, "16 words per thread");
+  uint32_t *w = reinterpret_cast<uint32_t *>(buf);
+  const uint32_t t = threadIdx.x, gs = run / 16, gl = t % gs;
+  uint32_t p[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 x = reinterpret_cast<const uint4 *>(w + 16 * t)[q];
+    p[4 * q] = x.x, p[4 * q + 1] = x.y, p[4 * q + 2] = x.z, p[4 * q + 3] = x.w;
+  }
+#pragma unroll
+  for (int i = 1; i < 16; ++i) p[i] ^= p[i - 1];
+  uint32_t incl = p[15];
+#pragma unroll
+  for (uint32_t o = 1; o < 8; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (o < gs && gl >= o) incl ^= y;
+  }
+  const uint32_t ex = incl ^ p[15];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    reinterpret_cast<uint4 *>(w + 16 * t)[q] =
+        make_uint4(p[4 * q] ^ ex, p[4 * q + 1] ^ ex, p[4 * q + 2] ^ ex, p[4 * q + 3] ^ ex);
+  named_bar_sync(1, NT);
+}
+
+// Two-level form, encode side: the 2048-byte bitmap in bm becomes, at the
+// start of buf, a 256-byte map (bit i: bitmap byte i is nonzero) followed by
+// the nonzero bitmap bytes in order. Returns their count (every thread).
+template <int NT>
+__device__ __forceinline__ uint32_t ze2_pack_bitmap(const uint8_t *bm, uint8_t *buf,
+                                                    uint32_t *red) {
+  static_assert(NT == 256, "8 bitmap bytes per thread");
+  const uint32_t t = threadIdx.x;
+  const uint2 v = *reinterpret_cast<const uint2 *>(bm + 8 * t);
+  const uint32_t m = nz_nibble(v.x) | (nz_nibble(v.y) << 4);
+  uint32_t total;
+  const uint32_t ex = block_excl_scan<NT>(__popc(m), red, total);
+  buf[t] = uint8_t(m);
+  uint32_t pos = kBitmap2 + ex;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if ((m >> i) & 1u) buf[pos++] = uint8_t((i < 4 ? v.x : v.y) >> (8 * (i & 3)));
+  named_bar_sync(1, NT);
+  return total;
+}
+
+// Two-level form, decode side: expands the map and bitmap bytes at the start
+// of buf into the 2048-byte bitmap bm. Returns the number of bitmap bytes
+// (every thread); the caller checks it against the chunk's size.
+template <int NT>
+__device__ __forceinline__ uint32_t ze2_unpack_bitmap(const uint8_t *buf, uint8_t *bm,
+                                                      uint32_t *red) {
+  static_assert(NT == 256, "8 bitmap bytes per thread");
+  const uint32_t t = threadIdx.x, m = buf[t];
+  uint32_t total;
+  const uint32_t ex = block_excl_scan<NT>(__popc(m), red, total);
+  uint32_t pos = kBitmap2 + ex, lo = 0, hi = 0;  // pos < 256 + 2048 < 16384: inside buf
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if ((m >> i) & 1u) {
+      const uint32_t b = buf[pos++];
+      if (i < 4) lo |= b << (8 * i); else hi |= b << (8 * (i - 4));
+    }
+  }
+  *reinterpret_cast<uint2 *>(bm + 8 * t) = make_uint2(lo, hi);
+  named_bar_sync(1, NT);
+  return total;
+}
+
+// A full chunk in buf through pipeline `pipe` into buf[0, size). run: words
+// per 32 vectors; bnz: the nonzero bitmap bytes of the two-level form (from
+// the encoder's counts; a mismatch records KVC_ERR_CORRUPT). bm: 2 KB.
+template <int NT>
+__device__ __forceinline__ void lossless_encode(uint8_t *buf, uint8_t *scr, uint8_t *bm,
+                                                uint32_t *red, uint32_t pipe, uint32_t run,
+                                                uint32_t bnz, uint32_t *status) {
+  if (pipe & 1u) xor_runs_forward<NT>(buf, run);
+  bool ok;
+  if (pipe & 2u) {
+    ok = ze_encode<NT>(buf, scr, red, bm, kBitmap2 + bnz) &&
+         ze2_pack_bitmap<NT>(bm, buf, red) == bnz;
+  } else {
+    ok = ze_encode<NT>(buf, scr, red);
+  }
+  if (!ok && threadIdx.x == 0) set_status(status, KVC_ERR_CORRUPT);
+}
+
+// Inverse of any pipeline on a full chunk of `size` stored bytes in buf;
+// false (every thread) if the chunk is inconsistent.
+template <int NT>
+__device__ __forceinline__ bool lossless_decode(uint8_t *buf, uint8_t *scr, uint8_t *bm,
+                                                uint32_t *red, uint32_t size, uint32_t pipe,
+                                                uint32_t run) {
+  bool ok;
+  if (pipe & 2u) {
+    const uint32_t nb = ze2_unpack_bitmap<NT>(buf, bm, red);
+    ok = kBitmap2 + nb <= size && ze_decode<NT>(buf, scr, red, size, bm, kBitmap2 + nb);
+  } else {
+    ok = size >= kBitmap && ze_decode<NT>(buf, scr, red, size);
+  }
+  if (ok && (pipe & 1u)) xor_runs_inverse<NT>(buf, run);
+  return ok;
+}
+
 // ------------------------------------------- warp row blocks (32 rows) --
 // A per-warp buffer of 32 rows in column blocks of 32 x 128 bytes (64 bf16
 // channels, or 32 fp32), 16-byte piece c of row r at (c / 8) * 4096 +
 // r * 128 + ((c % 8) ^ (r % 8)) * 16: the tensor maps' 128-byte swizzle, in
 // which lane r reading its own row, or a group of lanes reading one row, hits
 // distinct bank groups.
+// HALF: bytes between column blocks (4096 for 32 rows; the paged encoder's
+// buffers hold 40 rows, 5120).
+template <int HALF = 4096>
 __device__ __forceinline__ uint32_t swz_offset(int r, int c) {
-  return uint32_t((c >> 3) * 4096 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+  return uint32_t((c >> 3) * HALF + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
 // Gathers the 32 rows whose global addresses the lanes hold (lane r: row r;
@@ -606,7 +761,7 @@ __device__ __forceinline__ uint32_t swz_offset(int r, int c) {
 // instruction covers D/8-lane groups, one whole row per group, so every
 // group reads 2*D contiguous bytes. `dummy` is any valid global address
 // (passed with zero-fill copies). Completion: cp_async_wait_all + __syncwarp.
-template <int P>  // 16-byte pieces per row: 8, 16 or 32
+template <int P, int HALF = 4096>  // 16-byte pieces per row: 8, 16 or 32
 __device__ __forceinline__ void gather_rows_p(uint8_t *wbuf, const uint8_t *row, const void *dummy) {
   constexpr int RPI = 32 / P;  // rows per instruction
   const int lane = threadIdx.x & 31, c = lane % P, rs = lane / P;
@@ -616,7 +771,7 @@ __device__ __forceinline__ void gather_rows_p(uint8_t *wbuf, const uint8_t *row,
     const int r = i * RPI + rs;
     const uint64_t s = __shfl_sync(0xFFFFFFFFu, me, r);
     const void *src = s ? reinterpret_cast<const void *>(s + 16u * c) : dummy;
-    cp_async16(wbuf + swz_offset(r, c), src, s ? 16u : 0u);
+    cp_async16(wbuf + swz_offset<HALF>(r, c), src, s ? 16u : 0u);
   }
   cp_async_commit();
 }
@@ -666,7 +821,7 @@ __device__ __forceinline__ uint4 lds128(uint32_t saddr) {
                : "r"(saddr));
   return v;
 }
-template <int P>
+template <int P, int HALF = 4096>
 struct RowPieces {
   static constexpr int RPI = 32 / P;              // rows per copy instruction
   static constexpr int NI = 32 / RPI;             // instructions per 32 rows
@@ -677,7 +832,7 @@ struct RowPieces {
     const int lane = threadIdx.x & 31;
     c = lane % P;
     rs = lane / P;
-    const uint32_t sb = smem_u32(wbuf) + uint32_t((c >> 3) * 4096 + rs * 128);
+    const uint32_t sb = smem_u32(wbuf) + uint32_t((c >> 3) * HALF + rs * 128);
     const uint32_t k = uint32_t((c & 7) ^ (rs & 7));
 #pragma unroll
     for (int j = 0; j < K; ++j) s[j] = sb + ((k ^ uint32_t((j * RPI) & 7)) << 4);
@@ -686,14 +841,14 @@ struct RowPieces {
 };
 // Lanes without a row pass offset 0 (their row reads base's first row,
 // which is not used).
-template <int P>
+template <int P, int HALF = 4096>
 __device__ __forceinline__ void gather_rows_narrow(uint8_t *wbuf, const uint8_t *base,
                                                    uint32_t off16) {
-  const RowPieces<P> rp(wbuf);
+  const RowPieces<P, HALF> rp(wbuf);
   const uint8_t *g = base + 16 * rp.c;
 #pragma unroll
-  for (int i = 0; i < RowPieces<P>::NI; ++i) {
-    const uint32_t o = __shfl_sync(0xFFFFFFFFu, off16, i * RowPieces<P>::RPI + rp.rs);
+  for (int i = 0; i < RowPieces<P, HALF>::NI; ++i) {
+    const uint32_t o = __shfl_sync(0xFFFFFFFFu, off16, i * RowPieces<P, HALF>::RPI + rp.rs);
     cp_async16_s(rp.at(i), g + uint64_t(o) * 16);
   }
   cp_async_commit();
@@ -721,9 +876,9 @@ __device__ __forceinline__ void scatter_rows_narrow(const uint8_t *wbuf, uint8_t
 }
 
 // Rows of D bf16 (2*D bytes, D/8 pieces).
-template <int D>
+template <int D, int HALF = 4096>
 __device__ __forceinline__ void gather_rows(uint8_t *wbuf, const uint8_t *row, const void *dummy) {
-  gather_rows_p<D / 8>(wbuf, row, dummy);
+  gather_rows_p<D / 8, HALF>(wbuf, row, dummy);
 }
 template <int D>
 __device__ __forceinline__ void scatter_rows(const uint8_t *wbuf, uint8_t *row) {

@@ -56,16 +56,22 @@ struct Cfg {
 
 // Shared memory: per-warp row buffers | per-warp mbarriers | request prefix
 // (paged).
-template <int D>
+// A row buffer holds 32 rows (dense input) or 40 (paged input: a block's 32
+// tokens start anywhere in an 8-slot run of their pages, and its runs come
+// in whole), per 64-channel half.
+template <int D, bool kPaged = false>
 struct EncSmem {
-  static constexpr size_t WBUF = size_t(D / 64) * 32 * 128;  // 32 rows, 128-byte swizzled halves
+  static constexpr int ROWS = kPaged ? 40 : 32;
+  static constexpr int HALF = ROWS * 128;                   // bytes per 64-channel half
+  static constexpr size_t WBUF = size_t(D / 64) * HALF;     // 128-byte swizzled halves
   static constexpr size_t wbars = kEncWarps * WBUF;
   static constexpr size_t cum = wbars + kEncWarps * 8;
   static_assert(WBUF % 1024 == 0, "swizzled buffers stay 1024-byte aligned");
 };
 template <int D>
 constexpr size_t enc_smem_bytes(bool paged) {
-  return EncSmem<D>::cum + (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
+  return paged ? EncSmem<D, true>::cum + sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1)
+               : EncSmem<D, false>::cum;
 }
 
 template <class L>
@@ -128,14 +134,16 @@ struct Enc : Cfg<D, BITS, G> {
     }
   }
 
-  // E1/E2 from a per-warp tensor-load buffer: lane r's row r of each 64-channel
-  // half, 16-byte chunk c stored at r * 128 + ((c ^ (r % 8)) * 16) (the
-  // tensor map's 128-byte swizzle, which keeps these reads conflict-free).
-  static __device__ __forceinline__ void unpack_swz(const uint8_t *wbuf, int lane,
+  // E1/E2 from a per-warp tensor-load buffer: this lane's row `row` of each
+  // 64-channel half (HALF bytes apart), 16-byte chunk c stored at
+  // row * 128 + ((c ^ (row % 8)) * 16) (the tensor maps' 128-byte swizzle,
+  // which keeps these reads conflict-free for consecutive rows).
+  template <int HALF = 4096>
+  static __device__ __forceinline__ void unpack_swz(const uint8_t *wbuf, int row,
                                                     const uint32_t *__restrict__ mask, Pairs<D> &y) {
-    const int sw = lane & 7;
+    const int sw = row & 7;
     auto chunk = [&](int q) {
-      return *reinterpret_cast<const uint4 *>(wbuf + (q >> 3) * 4096 + lane * 128 +
+      return *reinterpret_cast<const uint4 *>(wbuf + (q >> 3) * HALF + row * 128 +
                                               (((q & 7) ^ sw) << 4));
     };
 #pragma unroll
@@ -240,8 +248,13 @@ struct Enc : Cfg<D, BITS, G> {
 
 // E3..E7 (kFwht) or E4..E7 of this lane's vector v of block blk, its stores
 // (codes in place, meta to the workspace), and the block's shuffled-byte
-// nonzero counts, accumulated per code and meta chunk.
-template <int D, int BITS, int G, bool kFwht>
+// nonzero counts, accumulated per code and meta chunk. With kSearch (the
+// lossless search mode, reading R17) also the counts that size the other
+// candidate pipelines: nonzero bitmap bytes (a bitmap byte covers 64 words
+// of one bit plane, so it is nonzero iff that plane's bit is set in the OR
+// of the 64 words) and the meta counts after the XOR of each word with the
+// previous one, restarted at every run of 32 vectors (a block is one run).
+template <int D, int BITS, int G, bool kFwht, bool kSearch>
 __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t blk, uint32_t v,
                                                     bool valid, Pairs<D> &y, uint32_t &err) {
   using C = Cfg<D, BITS, G>;
@@ -289,43 +302,76 @@ __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t b
     o |= __shfl_xor_sync(0xFFFFFFFFu, o, 1);
     cn = (lane & 1) ? 0u : __popc(o);
   }
+  if constexpr (kSearch) {  // nonzero bitmap bytes of the code region
+    constexpr int L64 = 64 / C::CW;  // vectors per 64-word group
+    uint32_t ov = 0;
+#pragma unroll
+    for (int w = 0; w < C::CW; ++w) ov |= code[w];
+#pragma unroll
+    for (int o = 1; o < L64; o <<= 1) ov |= __shfl_xor_sync(0xFFFFFFFFu, ov, o);
+    cn |= ((lane % L64) ? 0u : uint32_t(__popc(ov))) << 16;
+  }
   uint32_t mo = 0;
 #pragma unroll
   for (int g = 0; g < C::NG; ++g) mo |= meta[g];
   constexpr int kVecPerGroup = 32 / C::MB;  // vectors per 8-word meta group
 #pragma unroll
   for (int o = 1; o < kVecPerGroup; o <<= 1) mo |= __shfl_xor_sync(0xFFFFFFFFu, mo, o);
-  const uint32_t mcnt = (lane % kVecPerGroup) ? 0u : __popc(mo);
+  uint32_t mcnt = (lane % kVecPerGroup) ? 0u : __popc(mo), mbits = 0;
+  if constexpr (kSearch) {
+    // the XOR of pipelines 1 and 3 on this run of 32 vectors
+    const uint32_t prev = __shfl_up_sync(0xFFFFFFFFu, meta[C::NG - 1], 1);
+    uint32_t xo = valid ? meta[0] ^ (lane ? prev : 0u) : 0u;
+#pragma unroll
+    for (int g = 1; g < C::NG; ++g) xo |= valid ? meta[g] ^ meta[g - 1] : 0u;
+#pragma unroll
+    for (int o = 1; o < kVecPerGroup; o <<= 1) xo |= __shfl_xor_sync(0xFFFFFFFFu, xo, o);
+    mcnt |= ((lane % kVecPerGroup) ? 0u : uint32_t(__popc(xo))) << 16;
+    if constexpr (C::NG >= 2) {  // 64-word groups lie inside the block
+      constexpr int L64 = 64 / C::NG;
+      uint32_t b0 = mo, b1 = xo;
+#pragma unroll
+      for (int o = kVecPerGroup; o < L64; o <<= 1) {
+        b0 |= __shfl_xor_sync(0xFFFFFFFFu, b0, o);
+        b1 |= __shfl_xor_sync(0xFFFFFFFFu, b1, o);
+      }
+      mbits = (lane % L64) ? 0u : uint32_t(__popc(b0)) | (uint32_t(__popc(b1)) << 16);
+    }
+  }
   const uint32_t cs = __reduce_add_sync(0xFFFFFFFFu, cn);
   const uint32_t ms = __reduce_add_sync(0xFFFFFFFFu, mcnt);
+  uint32_t mb = 0;
+  if constexpr (kSearch && C::NG >= 2) mb = __reduce_add_sync(0xFFFFFFFFu, mbits);
   if (lane == 0) {
-    // The block that completes a full code chunk sees its final count and
-    // flags the chunk if zero-byte elimination makes it shorter (reading
-    // R11), adding the padded bytes it would save (reading R16 weighs them).
+    // The block that completes a full code chunk sees its final counts and
+    // flags the chunk if a lossless pipeline makes it shorter (reading R11,
+    // R17), adding the padded bytes it would save (reading R16 weighs them).
     const uint32_t c = blk * 32 / C::VC;
     const unsigned long long old = atomicAdd(a.code_nnz + c, (1ull << 32) | cs);
     const uint32_t blocks = (min(uint32_t(C::VC), V - c * C::VC) + 31) / 32;
-    const uint32_t size = kBitmap + uint32_t(old) + cs;
+    const uint32_t nnz = (uint32_t(old) & 0xFFFFu) + (cs & 0xFFFFu);
+    uint32_t size = kBitmap + nnz;
+    if constexpr (kSearch) size = min(size, kBitmap2 + ((uint32_t(old) >> 16) + (cs >> 16)) + nnz);
     if (uint32_t(old >> 32) + 1 == blocks && blocks * 32 == uint32_t(C::VC) &&
-        size < uint32_t(kChunk)) {
+        size < uint32_t(kChunk) && a.mode != KVC_LOSSLESS_NONE) {
       atomicOr(a.flags, 1u);
       atomicMax(a.first_inv, ~c);
       atomicAdd(a.saved, (unsigned long long)(uint32_t(kChunk) - uint32_t(round16(size))));
     }
-    atomicAdd(a.meta_nnz + blk * 32 / C::VM, ms);
+    atomicAdd(a.meta_nnz + blk * 32 / C::VM, (unsigned long long)ms | ((unsigned long long)mb << 32));
   }
 }
 
 // ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
-template <int D, int BITS, int G, class Layout, bool kNarrow>
+template <int D, int BITS, int G, class Layout, bool kNarrow, bool kSearch>
 __global__ void __launch_bounds__(kEncThreads, 1)
     encode_kernel(const __grid_constant__ EncArgs a, const __grid_constant__ Layout lay) {
   using C = Cfg<D, BITS, G>;
   using E = Enc<D, BITS, G>;
   constexpr bool kPaged = kIsPaged<Layout>;
-  using S = EncSmem<D>;
+  using S = EncSmem<D, kPaged>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint8_t *wbuf = smem + warp * S::WBUF;
@@ -362,7 +408,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
 
   uint32_t phase = 0, err = 0;
   auto finish_block = [&](uint32_t blk, uint32_t v, bool valid, Pairs<D> &y) {
-    encode_finish_block<D, BITS, G, true>(a, blk, v, valid, y, err);
+    encode_finish_block<D, BITS, G, true, kSearch>(a, blk, v, valid, y, err);
   };
 
   bool use_tma = false;
@@ -375,7 +421,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
         if (lane == 0) {
           const uint32_t v0 = b * 32, lkh = fdiv(lay.T, v0), t0 = v0 - lkh * lay.T.d;
           const uint32_t lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
-          mbar_arrive_expect_tx(wbar, uint32_t(S::WBUF));
+          mbar_arrive_expect_tx(wbar, uint32_t(D / 64) * 4096u);  // two 32-row boxes
 #pragma unroll
           for (int hh = 0; hh < D / 64; ++hh)
             tma_load_5d(wbuf + hh * 4096, &lay.tmap, hh * 64, int(t0), int(h), int(lk & 1u),
@@ -400,17 +446,114 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       }
     }
   }
-  if (!use_tma) {
-    grid_dependency_wait();  // the workspace clear (src_of may record a status)
-    // Row addresses are looked up one block ahead of their gather, so the
-    // page-table read overlaps a block of arithmetic; a layout whose rows fit
-    // 32-bit offsets from its base (the common case) uses the narrow copies.
-    auto gather = [&](const uint8_t *rowp) {
-      if constexpr (kNarrow)
-        gather_rows_narrow<D / 8>(wbuf, lay.base, rowp ? uint32_t((rowp - lay.base) >> 4) : 0u);
-      else
-        gather_rows<D>(wbuf, rowp, a.out);
+  auto gather = [&](const uint8_t *rowp) {
+    if constexpr (kNarrow)
+      gather_rows_narrow<D / 8, S::HALF>(wbuf, lay.base,
+                                         rowp ? uint32_t((rowp - lay.base) >> 4) : 0u);
+    else
+      gather_rows<D, S::HALF>(wbuf, rowp, a.out);
+  };
+  if constexpr (kPaged) {
+    grid_dependency_wait();  // the workspace clear (a plan may record a status)
+    // Block plans. A block whose 32 tokens lie in one request (all
+    // but about one in a hundred of a batch of long requests) loads as the
+    // 8-slot runs of its pages: lane j < runs reads run j's page and issues
+    // one tensor box of 8 rows per 64-channel half into 1 KB slot j of the
+    // buffer, so lane i's row is row (t0 % 8) + i. Other blocks (a request
+    // boundary, a page outside the pool, no tensor map) are gathered row by
+    // row, lane i's row at row i. A plan is one word per lane: kind (bits
+    // 0-1: 0 past the end, 1 boxes, 2 gather), t0 % 8 (2-4), the lane's run
+    // starting at slot 8 (5), the head row lkh (6..); plus the lane's page or
+    // gather row.
+    // A plan is made one block ahead of its issue (the page-table reads and
+    // the request search overlap a block of arithmetic). Per lane it is one
+    // word (kind in bits 0-1: 0 past the end, 1 boxes, 2 gather; t0 % 8 in
+    // bits 2-4; the lane's run starting at slot 8 in bit 5; the head row lkh
+    // from bit 6) and one 64-bit value: the lane's run page (boxes) or row
+    // address (gather).
+    auto plan = [&](uint32_t b, uint64_t &arg) -> uint32_t {
+      const uint32_t v0 = b * 32;
+      arg = 0;
+      if (v0 >= V) return 0u;
+      uint32_t simple = 0, t0 = 0, r = 0, lkh = 0;
+      if (lay.tma && lane == 0) {
+        lkh = fdiv(lay.T, v0);
+        const uint32_t u0 = v0 - lkh * lay.T.d;
+        uint32_t lo = 0, hi = lay.n_req - 1;  // largest r with cum[r] <= u0
+        while (lo < hi) {
+          const uint32_t mid = (lo + hi + 1) >> 1;
+          if (s_cum[mid] <= u0)
+            lo = mid;
+          else
+            hi = mid - 1;
+        }
+        r = lo;
+        t0 = u0 - s_cum[r];
+        simple = v0 + 32 <= V && u0 + 32 <= s_cum[r + 1];
+      }
+      if (__shfl_sync(0xFFFFFFFFu, simple, 0)) {
+        t0 = __shfl_sync(0xFFFFFFFFu, t0, 0);
+        r = __shfl_sync(0xFFFFFFFFu, r, 0);
+        lkh = __shfl_sync(0xFFFFFFFFu, lkh, 0);
+        const uint32_t runs = ((t0 + 31) >> 3) - (t0 >> 3) + 1;  // 4 or 5
+        bool ok = true;
+        uint32_t hi8 = 0;
+        if (uint32_t(lane) < runs) {
+          const uint32_t hp = (t0 >> 3) + lane;  // the run's 8-slot half page
+          const int32_t pg = __ldg(lay.page_table + int64_t(r) * lay.pt_stride + (hp >> 1));
+          ok = pg >= 0 && int64_t(pg) < lay.num_pages;
+          hi8 = hp & 1u;
+          arg = uint32_t(pg);
+        }
+        if (__all_sync(0xFFFFFFFFu, ok)) return 1u | ((t0 & 7u) << 2) | (hi8 << 5) | (lkh << 6);
+      }
+      arg = reinterpret_cast<uint64_t>(src_of(v0 + lane));
+      return 2u;
     };
+    auto issue = [&](uint32_t p, uint64_t arg) {
+      if ((p & 3u) == 1u) {
+        const uint32_t runs = (((p >> 2) & 7u) + 31) / 8 + 1;
+        if (lane == 0) mbar_arrive_expect_tx(wbar, runs * uint32_t(D / 64) * 1024u);
+        __syncwarp();
+        if (uint32_t(lane) < runs) {
+          const uint32_t lkh = p >> 6, lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
+          const int kvh = int((lk & 1u) * lay.H.d + h), slot = int(((p >> 5) & 1u) * 8);
+#pragma unroll
+          for (int hh = 0; hh < D / 64; ++hh)
+            tma_load_5d(wbuf + hh * S::HALF + lane * 1024, &lay.tmap, hh * 64, slot, kvh,
+                        int(uint32_t(arg)), int(lk >> 1), wbar);
+        }
+      } else if ((p & 3u) == 2u) {
+        gather(reinterpret_cast<const uint8_t *>(arg));
+      }
+    };
+    uint64_t narg;
+    uint32_t cur = plan(blk, narg);
+    issue(cur, narg);
+    uint32_t next = plan(blk + stride, narg);
+#pragma unroll 1
+    for (; blk < n_blocks; blk += stride) {
+      const uint32_t v = blk * 32 + lane;
+      if ((cur & 3u) == 1u) {
+        if (!mbar_wait(wbar, phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
+        phase ^= 1;
+      } else {
+        cp_async_wait_all();
+        __syncwarp();  // every lane's copies have landed
+      }
+      Pairs<D> y;
+      E::template unpack_swz<S::HALF>(wbuf, lane + int((cur >> 2) & 7u), a.sign_mask, y);
+      // every lane has read the buffer; the next load may overwrite it
+      fence_proxy_async_smem();
+      __syncwarp();
+      issue(next, narg);
+      cur = next & 31u;
+      next = plan(blk + 2 * stride, narg);
+      finish_block(blk, v, v < V, y);
+    }
+  } else if (!use_tma) {
+    grid_dependency_wait();  // the workspace clear (src_of may record a status)
+    // Row addresses are looked up one block ahead of their gather.
     if (blk < n_blocks) gather(src_of(blk * 32 + lane));
     const uint8_t *next = src_of((blk + stride) * 32 + lane);
 #pragma unroll 1

@@ -17,7 +17,11 @@ cudaError_t launch_fin(const FinArgs &a, const Layout &lay, int sms, cudaStream_
   const uint32_t want = a.n_meta > 1 ? a.n_meta : 1u, cap = 4u * uint32_t(sms);
   const int grid = int(want < cap ? want : cap);
   e = launch_after(fk, grid, kFinThreads, fsmem, st, a, lay);
-  if (e != cudaSuccess || a.n_code == 0) return e;
+  if (e != cudaSuccess) return e;
+  if (a.n_code == 0) {
+    timing_mark(st);  // no compaction kernel: its interval is empty
+    return e;
+  }
   // Returns at once unless a code chunk shrank (flag set by the encode kernel).
   auto ck = compact_kernel;
   const size_t csmem = fin_smem_bytes(false);

@@ -33,9 +33,12 @@ struct FinCtl {
   uint32_t tick;
 };
 
+// Shared memory: two chunk buffers | plane-word scratch | 2 KB bitmap of the
+// two-level form | FinCtl | request prefix (paged).
+constexpr size_t kFinBm = 3 * size_t(kChunk);
+constexpr size_t kFinCtl = kFinBm + kBitmap;
 constexpr size_t fin_smem_bytes(bool paged) {
-  return 3 * size_t(kChunk) + sizeof(FinCtl) +
-         (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
+  return kFinCtl + sizeof(FinCtl) + (paged ? sizeof(uint32_t) * (KVC_MAX_REQUESTS + 1) : 0);
 }
 
 // 64-bit block sum over the first NT threads.
@@ -60,17 +63,47 @@ __device__ __forceinline__ void st_u64(uint8_t *p, uint64_t v) {
 __device__ __forceinline__ uint32_t code_len(const FinArgs &a, uint32_t c) {
   return min(a.vc, a.V - c * a.vc) * a.cb;
 }
+// How a chunk is stored (readings R11, R17): size, pipeline id and, for the
+// two-level form, its nonzero bitmap bytes. Only full chunks are coded, only
+// when strictly shorter; the search mode takes the shortest candidate (code:
+// pipelines 0, 2; meta: 0..3, or 0, 1 with one meta word per vector), ties
+// to the lower id; the NONE mode stores everything raw.
+struct Stored {
+  uint32_t size, pipe, bnz;
+};
+__device__ __forceinline__ Stored code_stored(const FinArgs &a, uint32_t c) {
+  const uint32_t len = code_len(a, c);
+  if (len != uint32_t(kChunk) || a.mode == KVC_LOSSLESS_NONE) return {len, 0u, 0u};
+  const unsigned long long n = a.code_nnz[c];
+  const uint32_t n0 = uint32_t(n) & 0xFFFFu, b0 = (uint32_t(n) >> 16) & 0xFFFFu;
+  Stored r{kBitmap + n0, 0u, 0u};
+  if (a.mode == KVC_LOSSLESS_SEARCH && kBitmap2 + b0 + n0 < r.size) r = {kBitmap2 + b0 + n0, 2u, b0};
+  return r.size < len ? r : Stored{len, 0u, 0u};
+}
 __device__ __forceinline__ uint32_t code_stored_size(const FinArgs &a, uint32_t c) {
-  const uint32_t len = code_len(a, c), n = uint32_t(a.code_nnz[c]);
-  return (len == uint32_t(kChunk) && kBitmap + n < uint32_t(kChunk)) ? kBitmap + n : len;
+  return code_stored(a, c).size;
 }
 __device__ __forceinline__ uint32_t meta_len(const FinArgs &a, uint32_t s) {
   return min(a.vm, a.V - s * a.vm) * a.mb;
 }
-// Reading R11: zero-byte elimination only when strictly shorter, full chunks only.
+__device__ __forceinline__ Stored meta_stored(const FinArgs &a, uint32_t s) {
+  const uint32_t len = meta_len(a, s);
+  if (len != uint32_t(kChunk) || a.mode == KVC_LOSSLESS_NONE) return {len, 0u, 0u};
+  const unsigned long long n = a.meta_nnz[s];
+  const uint32_t n0 = uint32_t(n) & 0xFFFFu, n1 = uint32_t(n) >> 16;
+  const uint32_t b0 = uint32_t(n >> 32) & 0xFFFFu, b1 = uint32_t(n >> 48);
+  Stored r{kBitmap + n0, 0u, 0u};
+  if (a.mode == KVC_LOSSLESS_SEARCH) {
+    if (kBitmap + n1 < r.size) r = {kBitmap + n1, 1u, 0u};
+    if (a.mb >= 8) {  // the two-level form needs at least two meta words per vector
+      if (kBitmap2 + b0 + n0 < r.size) r = {kBitmap2 + b0 + n0, 2u, b0};
+      if (kBitmap2 + b1 + n1 < r.size) r = {kBitmap2 + b1 + n1, 3u, b1};
+    }
+  }
+  return r.size < len ? r : Stored{len, 0u, 0u};
+}
 __device__ __forceinline__ uint32_t meta_stored_size(const FinArgs &a, uint32_t s) {
-  const uint32_t len = meta_len(a, s), n = a.meta_nnz[s];
-  return (len == uint32_t(kChunk) && kBitmap + n < uint32_t(kChunk)) ? kBitmap + n : len;
+  return meta_stored(a, s).size;
 }
 
 // Reading R16: some code chunk shrank (flag bit 0); keep zero-byte
@@ -132,7 +165,8 @@ __global__ void __launch_bounds__(kFinThreads, 4)
   constexpr int NT = kFinThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *scr = smem + 2 * kChunk;  // buffers 0 and 1 below it
-  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + 3 * kChunk);
+  uint8_t *bm = smem + kFinBm;
+  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + kFinCtl);
   uint32_t *s_cum = reinterpret_cast<uint32_t *>(ctl + 1);
   const int tid = threadIdx.x;
   const uint32_t nb = gridDim.x, b = blockIdx.x;
@@ -196,8 +230,10 @@ __global__ void __launch_bounds__(kFinThreads, 4)
     }
     if (!mbar_wait(&ctl->full[k], (phase >> k) & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
     phase ^= 1u << k;
-    const uint32_t len = meta_len(a, s), size = meta_stored_size(a, s);
-    if (size < len) ze_encode<NT>(buf, scr, ctl->red);
+    const uint32_t len = meta_len(a, s);
+    const Stored so = meta_stored(a, s);
+    const uint32_t size = so.size;
+    if (size < len) lossless_encode<NT>(buf, scr, bm, ctl->red, so.pipe, 8 * a.mb, so.bnz, a.status);
     for (uint32_t i = size + tid; i < round16(size); i += NT) buf[i] = 0;
     fence_proxy_async_smem();
     named_bar_sync(1, NT);
@@ -210,7 +246,7 @@ __global__ void __launch_bounds__(kFinThreads, 4)
         uint8_t *dst = shrank ? a.ws_meta + uint64_t(s) * kChunk : a.out + a.data_base + off;
         bulk_s2g(dst, buf, uint32_t(round16(size)));
         bulk_commit();
-        st_u64(a.out + kHeader + 8ull * (a.n_code + s), ((off >> 4) << 16) | size);
+        st_u64(a.out + kHeader + 8ull * (a.n_code + s), make_entry(off, size, so.pipe));
       } else {
         set_status(a.status, KVC_ERR_CAPACITY);
       }
@@ -224,21 +260,22 @@ __global__ void __launch_bounds__(kFinThreads, 4)
   const uint32_t c1 = uint32_t(uint64_t(b + 1) * a.n_code / nb);
   if (!shrank) {
     for (uint32_t c = c0 + tid; c < c1; c += NT)
-      st_u64(a.out + kHeader + 8ull * c, ((uint64_t(c) * kChunk >> 4) << 16) | code_len(a, c));
+      st_u64(a.out + kHeader + 8ull * c, make_entry(uint64_t(c) * kChunk, code_len(a, c), 0u));
   } else {
     uint64_t part = 0;
     for (uint32_t c = tid; c < c0; c += NT) part += round16(code_stored_size(a, c));
     uint64_t base = block_sum64<NT>(part, ctl->red);
     for (uint32_t c = c0; c < c1; c += NT) {  // block-wide scan, NT chunks at a time
       const uint32_t me = c + tid;
-      const uint32_t sz = me < c1 ? code_stored_size(a, me) : 0u;
+      const Stored so = me < c1 ? code_stored(a, me) : Stored{0u, 0u, 0u};
+      const uint32_t sz = so.size;
       if (me < c1) a.code_size[me] = sz;
       uint32_t total;
       const uint32_t ex = block_excl_scan<NT>(uint32_t(round16(sz)) >> 4, ctl->red, total);
       if (me < c1) {
         const uint64_t off = base + (uint64_t(ex) << 4);
         a.code_off[me] = off;
-        st_u64(a.out + kHeader + 8ull * me, ((off >> 4) << 16) | sz);
+        st_u64(a.out + kHeader + 8ull * me, make_entry(off, sz, so.pipe));
       }
       base += uint64_t(total) << 4;
     }
@@ -266,7 +303,8 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *buf = smem;
   uint8_t *scr = smem + kChunk;
-  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + 3 * kChunk);
+  uint8_t *bm = smem + kFinBm;
+  FinCtl *ctl = reinterpret_cast<FinCtl *>(smem + kFinCtl);
   const int tid = threadIdx.x;
   if (tid == 0) {
     mbar_init(&ctl->full[0], 1);
@@ -305,8 +343,9 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
         atomicExch(a.done + c, 1u);  // raw bytes read
         atomicAdd(a.ticket + 1, 1u);
       }
-      if (size != len) {  // shrinks: bit-plane shuffle + zero-byte elimination
-        ze_encode<NT>(buf, scr, ctl->red);
+      if (size != len) {  // shrinks: its lossless pipeline (0 or 2 for code chunks)
+        const Stored so = code_stored(a, c);
+        lossless_encode<NT>(buf, scr, bm, ctl->red, so.pipe, 0u, so.bnz, a.status);
         for (uint32_t i = size + tid; i < round16(size); i += NT) buf[i] = 0;
       }
       const uint32_t j0 = uint32_t(dst / kChunk);
@@ -357,7 +396,7 @@ __global__ void __launch_bounds__(kFinThreads, 4) compact_kernel(const __grid_co
       mbar_arrive_expect_tx(&ctl->full[0], uint32_t(round16(size)));
       bulk_g2s(buf, a.ws_meta + uint64_t(s) * kChunk, uint32_t(round16(size)), &ctl->full[0]);
       if (!mbar_wait(&ctl->full[0], phase & 1, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
-      bulk_s2g(a.out + a.data_base + ((e >> 16) << 4), buf, uint32_t(round16(size)));
+      bulk_s2g(a.out + a.data_base + entry_offset(e), buf, uint32_t(round16(size)));
       bulk_commit();
       bulk_wait_read<0>();
     }

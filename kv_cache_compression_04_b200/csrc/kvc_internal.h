@@ -24,6 +24,7 @@ namespace kvc {
 
 constexpr int kChunk = 16384;   // lossless chunk bytes
 constexpr int kBitmap = 2048;   // zero-byte-elimination bitmap bytes
+constexpr int kBitmap2 = 256;   // second-level bitmap bytes (pipelines 2 and 3)
 constexpr int kHeader = 64;     // stream header bytes
 constexpr uint32_t kMagic = 0x3143564Bu;  // "KVC1"
 constexpr int kThreads = 256;   // compute threads per CTA (one vector each)
@@ -42,9 +43,14 @@ constexpr uint32_t kWaitIters = 1u << 26;
 //             compaction ticket, compaction read count, ~(first shrinking
 //             code chunk), (u64 at byte 24) padded bytes the shrinking code
 //             chunks save
-//   meta_nnz  u32 per meta chunk: shuffled-byte nonzero count (accumulated)
-//   code_nnz  u64 per code chunk: the same count (low half) and the number
-//             of 32-vector blocks accumulated so far (high half)
+//   meta_nnz  u64 per meta chunk, accumulated 16-bit fields: shuffled-byte
+//             nonzero count (bits 0..15), the same after the XOR of
+//             pipelines 1 and 3 (16..31), nonzero bytes of the 2048-byte
+//             bitmap (32..47) and of the bitmap after the XOR (48..63); all
+//             but the first only in the search mode
+//   code_nnz  u64 per code chunk: shuffled-byte nonzero count (bits 0..15),
+//             nonzero bitmap bytes (16..31, search mode) and the number of
+//             32-vector blocks accumulated so far (32..63)
 //   done      u32 per code chunk: compaction read flags
 //   code_size u32 per code chunk: stored size
 //   meta_size u32 per meta chunk: stored size
@@ -58,12 +64,21 @@ struct WsLayout {
 };
 
 KVC_HD uint64_t round16(uint64_t x) { return (x + 15u) & ~uint64_t(15); }
+
+// Chunk table entry (readings R12, R17): bits 0..15 unpadded size, 16..59
+// offset from the data base in 16-byte units, 60..63 lossless pipeline id.
+KVC_HD uint32_t entry_size(uint64_t e) { return uint32_t(e & 0xFFFFu); }
+KVC_HD uint64_t entry_offset(uint64_t e) { return ((e >> 16) & 0xFFFFFFFFFFFull) << 4; }
+KVC_HD uint32_t entry_pipe(uint64_t e) { return uint32_t(e >> 60); }
+KVC_HD uint64_t make_entry(uint64_t off, uint32_t size, uint32_t pipe) {
+  return (uint64_t(pipe) << 60) | ((off >> 4) << 16) | size;
+}
 KVC_HD uint64_t round256(uint64_t x) { return (x + 255u) & ~uint64_t(255); }
 
 inline WsLayout ws_layout(uint64_t n_code, uint64_t n_meta) {
   WsLayout w{};
   w.meta_nnz = kWsCtl;
-  w.code_nnz = w.meta_nnz + round256(4 * n_meta);
+  w.code_nnz = w.meta_nnz + round256(8 * n_meta);
   w.done = w.code_nnz + round256(8 * n_code);
   w.code_size = w.done + round256(4 * n_code);
   w.meta_size = w.code_size + round256(4 * n_code);
@@ -130,6 +145,12 @@ struct DenseLayout {
 };
 
 struct PagedLayout {
+  // Tensor map of the pool as 5-D [layers][pages][2 * kv_heads][page_tokens]
+  // [head_dim] (boxes of 8 slots x 64 channels, 128-byte swizzle), valid iff
+  // tma != 0: set by the host when kv and head merge into one dimension
+  // (stride_kv == kv_heads * stride_head) and page_tokens % 8 == 0.
+  alignas(64) CUtensorMap tmap;
+  uint32_t tma;
   uint8_t *base;
   int64_t s_l, s_p, s_kv, s_h, s_slot;  // bytes
   const int32_t *page_table;
@@ -152,10 +173,11 @@ struct EncArgs {
   uint32_t *first_inv; // max over shrinking code chunks c of ~c (0: none)
   unsigned long long *saved;  // padded bytes the shrinking code chunks save
   unsigned long long *code_nnz;
-  uint32_t *meta_nnz;
+  unsigned long long *meta_nnz;
   uint8_t *ws_meta;
   float *ymid;         // unfused baseline only: transformed vectors, d fp32 each
   float one;           // 1.0: the quantizer's integer rounding multiplies by it
+  uint32_t mode;       // KVC_LOSSLESS_*
   uint32_t sign_mask[128];
 };
 
@@ -174,7 +196,7 @@ struct FinArgs {
   const unsigned long long *saved;  // padded bytes the shrinking code chunks save
   uint32_t *ticket;
   const unsigned long long *code_nnz;
-  const uint32_t *meta_nnz;
+  const unsigned long long *meta_nnz;
   uint32_t *code_size;
   uint32_t *done;
   uint32_t *meta_size;
@@ -188,6 +210,7 @@ struct FinArgs {
   // tickets that many chunks late, so those chunks' read flags are never set
   uint64_t wait_ns;
   uint32_t ticket_skip;
+  uint32_t mode;  // KVC_LOSSLESS_*
 };
 
 struct DecArgs {
@@ -201,6 +224,21 @@ struct DecArgs {
   uint8_t *ws_meta;          // expanded meta chunks, 16 KB each
   uint32_t ws_meta_chunks;   // slots in ws_meta
 };
+
+// Per-kernel timing of the measurement entry points (kvc_compress_timed,
+// kvc_decompress_timed): while such a call runs on this host thread, the
+// launchers record timing_events[i] after the i-th kernel of the call
+// (timing_events[0] before the first) and launch without programmatic
+// dependence, so that each pair of events brackets exactly one kernel.
+struct KernelTiming {
+  const cudaEvent_t *events = nullptr;  // null: an ordinary call
+  int next = 0;
+};
+KernelTiming &kernel_timing();  // this host thread's state
+inline void timing_mark(cudaStream_t st) {
+  KernelTiming &t = kernel_timing();
+  if (t.events) cudaEventRecord(t.events[t.next++], st);
+}
 
 // Launchers, one translation unit per (head_dim, layout).
 #define KVC_DECLARE_LAUNCHERS(D)                                                          \

@@ -23,8 +23,10 @@ inline cudaError_t launch_after(void (*k)(KArgs...), int grid, int threads, size
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+  cfg.numAttrs = kernel_timing().events ? 0 : 1;  // timed calls: plain stream order
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+  timing_mark(st);
+  return e;
 }
 
 // Opt each instantiation into large dynamic shared memory once per device.
@@ -42,9 +44,9 @@ inline cudaError_t prepare(Kernel k, size_t smem) {
   return e;
 }
 
-template <int D, int BITS, int G, class Layout, bool kNarrow>
+template <int D, int BITS, int G, class Layout, bool kNarrow, bool kSearch>
 cudaError_t launch_enc_k(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
-  auto k = encode_kernel<D, BITS, G, Layout, kNarrow>;
+  auto k = encode_kernel<D, BITS, G, Layout, kNarrow, kSearch>;
   const size_t smem = enc_smem_bytes<D>(kIsPaged<Layout>);
   struct Tag {};
   cudaError_t e = prepare<Tag>(k, smem);
@@ -59,12 +61,18 @@ cudaError_t launch_enc_k(const EncArgs &a, const Layout &lay, int sms, cudaStrea
 // Paged rows named by 32-bit offsets when the pool allows (narrow row
 // copies). Dense inputs keep the 64-bit gather next to their tensor-map
 // loads: both paths in one kernel would not fit its registers.
+// The search mode counts more per block (encode_finish_block's kSearch).
+template <int D, int BITS, int G, class Layout, bool kSearch>
+cudaError_t launch_enc_s(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
+  if constexpr (kIsPaged<Layout>) {
+    if (lay.narrow) return launch_enc_k<D, BITS, G, Layout, true, kSearch>(a, lay, sms, st);
+  }
+  return launch_enc_k<D, BITS, G, Layout, false, kSearch>(a, lay, sms, st);
+}
 template <int D, int BITS, int G, class Layout>
 cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
-  if constexpr (kIsPaged<Layout>) {
-    if (lay.narrow) return launch_enc_k<D, BITS, G, Layout, true>(a, lay, sms, st);
-  }
-  return launch_enc_k<D, BITS, G, Layout, false>(a, lay, sms, st);
+  return a.mode == KVC_LOSSLESS_SEARCH ? launch_enc_s<D, BITS, G, Layout, true>(a, lay, sms, st)
+                                       : launch_enc_s<D, BITS, G, Layout, false>(a, lay, sms, st);
 }
 
 template <int D, class Layout, bool kNarrow>
@@ -109,6 +117,7 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
   e = launch_after(ek, egrid, kElimThreads, esmem, st, a, lay);
   if (e != cudaSuccess) return e;
   k<<<grid, kDecThreads, smem, st>>>(a, lay);
+  timing_mark(st);
   return cudaGetLastError();
 }
 

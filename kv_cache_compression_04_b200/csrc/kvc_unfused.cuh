@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) quantize_kernel(const __grid_c
     }
     __syncwarp();
     if (blk + stride < n_blocks) gather_rows_p<D / 4>(wbuf, row((blk + stride) * 32 + lane), a.out);
-    encode_finish_block<D, BITS, G, false>(a, blk, v, v < V, y, err);
+    encode_finish_block<D, BITS, G, false, false>(a, blk, v, v < V, y, err);
   }
   err = __reduce_or_sync(0xFFFFFFFFu, err);
   if (lane == 0) {

@@ -14,9 +14,9 @@ def u16(t: torch.Tensor) -> np.ndarray:
     return synth.bf16_bits(t)
 
 
-def gpu_compress(desc, bits, group, seed=0, slack: int = 0):
+def gpu_compress(desc, bits, group, seed=0, slack: int = 0, lossless: int = 0):
     """-> (status, stream uint8 numpy, device buffers)."""
-    p = kvc.params(bits, group, seed)
+    p = kvc.params(bits, group, seed, lossless)
     cap = kvc.kvc_max_compressed_bytes(desc, p)
     wsb = kvc.kvc_workspace_bytes(desc, p)
     assert cap > 0 and wsb > 0
@@ -43,8 +43,8 @@ def gpu_decompress(stream: np.ndarray | torch.Tensor, desc, nbytes: int | None =
     return kvc.kvc_stream_status(ws.data_ptr(), kvc._stream_ptr(None))
 
 
-def oracle_desc(bits, group, d, layers, heads, token_lens, seed=0, origin=0):
-    return oracle.StreamDesc(bits, group, d, layers, heads, token_lens, seed, origin)
+def oracle_desc(bits, group, d, layers, heads, token_lens, seed=0, origin=0, lossless=0):
+    return oracle.StreamDesc(bits, group, d, layers, heads, token_lens, seed, origin, lossless)
 
 
 def first_diff(a: np.ndarray, b: np.ndarray, lay=None) -> str:
@@ -63,5 +63,11 @@ def first_diff(a: np.ndarray, b: np.ndarray, lay=None) -> str:
 
 
 def chunk_table(stream: np.ndarray, n_chunks: int):
+    """-> (sizes, offsets) of the chunk table (pipeline ids in pipelines())."""
     e = stream[64:64 + 8 * n_chunks].view("<u8").astype(np.uint64)
-    return (e & 0xFFFF).astype(np.int64), ((e >> 16) * 16).astype(np.int64)
+    return (e & 0xFFFF).astype(np.int64), (((e >> 16) & 0xFFFFFFFFFFF) * 16).astype(np.int64)
+
+
+def pipelines(stream: np.ndarray, n_chunks: int):
+    e = stream[64:64 + 8 * n_chunks].view("<u8").astype(np.uint64)
+    return (e >> 60).astype(np.int64)

@@ -244,3 +244,18 @@ def test_unfused_workspace_and_argument_checks(L):
     assert kvc.kvc_compress_unfused(d, kvc.params(3, 128, 0), FAKE, cap, nb, FAKE, wsb,
                                     None) == kvc.KVC_ERR_UNSUPPORTED
     assert kvc.kvc_unfused_workspace_bytes(dense(2, 2, 64, 96), p) == 0
+
+
+def test_timed_calls_refuse_bad_event_arrays(L):
+    import ctypes as C
+    d = dense(2, 2, 64, 128)
+    p = kvc.params(4, 128)
+    cap = kvc.kvc_max_compressed_bytes(d, p)
+    wsb = kvc.kvc_workspace_bytes(d, p)
+    four = (C.c_void_p * 4)(*([FAKE] * 4))
+    five_null = (C.c_void_p * 5)(FAKE, FAKE, None, FAKE, FAKE)
+    for arr, n in [(four, 4), (five_null, 5), (None, 5)]:
+        assert L.kvc_compress_timed(C.byref(d), C.byref(p), FAKE, cap, None, FAKE, wsb, arr, n,
+                                    None) == kvc.KVC_ERR_INVALID_ARG
+        assert L.kvc_decompress_timed(FAKE, 4096, C.byref(d), FAKE, 1 << 20, arr, n,
+                                      None) == kvc.KVC_ERR_INVALID_ARG
