@@ -140,6 +140,12 @@ def lib():
                                            C.c_uint64, u64p]),
                 "orc_decompress": (C.c_int, [u8p, C.c_uint64,
                                              C.POINTER(Desc), u16p]),
+                "orc_dequantize_vector_f64": (None, [u8p, u8p, C.c_int, C.c_int, C.c_int,
+                                                     u64p, C.POINTER(C.c_double)]),
+                "orc_decode_values_mt": (C.c_int, [u8p, C.c_uint64, C.POINTER(Desc),
+                                                   C.POINTER(C.c_double), C.c_int]),
+                "orc_attend": (C.c_int, [u8p, C.c_uint64, C.POINTER(Desc), u16p, C.c_int,
+                                         C.c_double, C.POINTER(C.c_double), C.c_int]),
                 "orc_compress_mt": (C.c_int, [C.POINTER(Desc), u16p, u8p,
                                               C.c_uint64, u64p, C.c_int]),
                 "orc_decompress_mt": (C.c_int, [u8p, C.c_uint64,
@@ -491,3 +497,29 @@ def gather_paged(pool: np.ndarray, layers, kv_heads, d, strides, page_tokens,
                            pt.shape[1] if pt.ndim == 2 else 0, v_begin, v_end,
                            _p(out, C.c_uint16))
     return out
+
+
+# --------------------------------------------------------------------------
+# attention over the compressed cache (reading R18)
+# --------------------------------------------------------------------------
+def decode_values(stream: np.ndarray, desc: StreamDesc, threads: int = 1):
+    """-> (status, float64 [V, d]): decoded vectors without the bf16 rounding."""
+    stream = np.ascontiguousarray(stream, np.uint8)
+    lay = desc.layout()
+    out = np.empty((lay.V, desc.head_dim), np.float64)
+    st = lib().orc_decode_values_mt(_p(stream, C.c_uint8), stream.size, C.byref(desc.c),
+                                    _p(out, C.c_double), int(max(1, threads)))
+    return st, out
+
+
+def attend(stream: np.ndarray, desc: StreamDesc, q: np.ndarray, q_per_kv: int,
+           scale: float, threads: int = 1):
+    """q: uint16 bf16 bits [layers, n_requests, kv_heads * q_per_kv, d] ->
+    (status, float64 output of the same shape)."""
+    stream = np.ascontiguousarray(stream, np.uint8)
+    q = np.ascontiguousarray(q, np.uint16)
+    out = np.zeros(q.shape, np.float64)
+    st = lib().orc_attend(_p(stream, C.c_uint8), stream.size, C.byref(desc.c),
+                          _p(q, C.c_uint16), int(q_per_kv), float(scale), _p(out, C.c_double),
+                          int(max(1, threads)))
+    return st, out

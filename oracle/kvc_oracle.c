@@ -295,6 +295,42 @@ void orc_dequantize_vector(const uint8_t *codes, const uint8_t *meta, int d,
   }
 }
 
+/* The same decode without the final bf16 rounding, in double: y^ as above
+ * (fp32, the decoder's value), then x^_c = sign_c * (H_d y^)_c / d evaluated in
+ * double (every fp32 input and product is exact there; the butterfly's sums
+ * round at 2^-53). Reading R18: these are the key and value vectors an
+ * attention step that consumes the compressed cache works with; the bf16
+ * rounding of the decoder moves each of them by at most half a bf16 ulp. */
+void orc_dequantize_vector_f64(const uint8_t *codes, const uint8_t *meta, int d,
+                               int bits, int g, const uint64_t *sign_words,
+                               double *xhat) {
+  float yf[ORC_MAX_D];
+  double y[ORC_MAX_D];
+  uint8_t q[ORC_MAX_D];
+  int k = orc_meta_shift(d), c, j, h, i;
+  float up = ldexpf(1.0f, k);
+  orc_unpack_codes(codes, d, bits, q);
+  for (j = 0; j < d / g; j++) {
+    uint16_t sh = (uint16_t)(meta[4 * j] | (meta[4 * j + 1] << 8));
+    uint16_t zh = (uint16_t)(meta[4 * j + 2] | (meta[4 * j + 3] << 8));
+    float sf = orc_f16_to_f32(sh) * up;
+    float zf = orc_f16_to_f32(zh) * up;
+    for (c = j * g; c < (j + 1) * g; c++) {
+      float p = (float)q[c] * sf;
+      yf[c] = zf + p;
+    }
+  }
+  for (c = 0; c < d; c++) y[c] = (double)yf[c];
+  for (h = 1; h < d; h *= 2)
+    for (i = 0; i < d; i++)
+      if ((i & h) == 0) {
+        double a = y[i], b = y[i + h];
+        y[i] = a + b;
+        y[i + h] = a - b;
+      }
+  for (c = 0; c < d; c++) xhat[c] = (sign_bit(sign_words, c) ? -y[c] : y[c]) / (double)d;
+}
+
 /* ========================================================================== */
 /* Lossless stage on one 16 KB chunk ([P2]: LC-style backend composed of      */
 /* primitives). The components are a bit-plane shuffle, zero-byte            */
@@ -721,7 +757,7 @@ int orc_encode_segment(const orc_desc *d, uint64_t s, const uint16_t *vectors,
 
 static int decode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t s,
                              const uint8_t *chunks, const uint32_t *sizes,
-                             const uint8_t *pipes, uint16_t *vectors) {
+                             const uint8_t *pipes, uint16_t *vectors, double *vals) {
   uint64_t vm, v0, nv, v, c0, c1, c, i = 0;
   uint8_t *codes, *meta;
   uint64_t sw[4];
@@ -750,10 +786,15 @@ static int decode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t 
     st = orc_chunk_decode_pipe(chunks + pos, sizes[i], (uint32_t)(nv * lay->meta_bytes),
                                pipes[i], (int)(lay->meta_bytes / 4), meta);
   if (st == ORC_OK)
-    for (v = 0; v < nv; v++)
-      orc_dequantize_vector(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
-                            d->head_dim, d->bits, d->group, sw,
-                            vectors + v * d->head_dim);
+    for (v = 0; v < nv; v++) {
+      if (vals)
+        orc_dequantize_vector_f64(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
+                                  d->head_dim, d->bits, d->group, sw, vals + v * d->head_dim);
+      else
+        orc_dequantize_vector(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
+                              d->head_dim, d->bits, d->group, sw,
+                              vectors + v * d->head_dim);
+    }
   free(codes);
   free(meta);
   return st;
@@ -765,7 +806,7 @@ int orc_decode_segment(const orc_desc *d, uint64_t s, const uint8_t *chunks,
   int st = orc_layout_of(d, &lay);
   if (st != ORC_OK) return st;
   if (s >= lay.n_seg) return ORC_ERR_INVALID_ARG;
-  return decode_segment_in(d, &lay, s, chunks, sizes, pipes, vectors);
+  return decode_segment_in(d, &lay, s, chunks, sizes, pipes, vectors, NULL);
 }
 
 /* Runs fn(job, s) for every segment s in [0, n_seg) on n_threads threads
@@ -989,6 +1030,7 @@ typedef struct {
   const orc_layout *lay;
   const uint8_t *stream;
   uint16_t *vectors;
+  double *vals; /* non-null: unrounded values instead of bf16 */
   int *seg_status;
 } dec_job;
 
@@ -1011,8 +1053,9 @@ static void dec_one_segment(void *arg, uint64_t s) {
     pipes[k] = (uint8_t)(e >> 60);
     pos += sz;
   }
-  j->seg_status[s] = decode_segment_in(j->d, lay, s, seg, sizes, pipes,
-                                       j->vectors + s * vm * j->d->head_dim);
+  j->seg_status[s] = decode_segment_in(
+      j->d, lay, s, seg, sizes, pipes, j->vectors ? j->vectors + s * vm * j->d->head_dim : NULL,
+      j->vals ? j->vals + s * vm * j->d->head_dim : NULL);
   free(seg);
 }
 
@@ -1021,8 +1064,23 @@ int orc_decompress(const uint8_t *stream, uint64_t stream_bytes,
   return orc_decompress_mt(stream, stream_bytes, expect, vectors, 1);
 }
 
+static int decompress_impl(const uint8_t *stream, uint64_t stream_bytes,
+                           const orc_desc *expect, uint16_t *vectors, double *vals,
+                           int n_threads);
+
 int orc_decompress_mt(const uint8_t *stream, uint64_t stream_bytes,
                       const orc_desc *expect, uint16_t *vectors, int n_threads) {
+  return decompress_impl(stream, stream_bytes, expect, vectors, NULL, n_threads);
+}
+
+int orc_decode_values_mt(const uint8_t *stream, uint64_t stream_bytes,
+                         const orc_desc *expect, double *vals, int n_threads) {
+  return decompress_impl(stream, stream_bytes, expect, NULL, vals, n_threads);
+}
+
+static int decompress_impl(const uint8_t *stream, uint64_t stream_bytes,
+                           const orc_desc *expect, uint16_t *vectors, double *vals,
+                           int n_threads) {
   orc_layout lay;
   uint64_t s, T = 0, expect_off = 0, total;
   int *seg_status;
@@ -1072,6 +1130,7 @@ int orc_decompress_mt(const uint8_t *stream, uint64_t stream_bytes,
   job.lay = &lay;
   job.stream = stream;
   job.vectors = vectors;
+  job.vals = vals;
   job.seg_status = seg_status;
   for_each_segment(lay.n_seg, n_threads, &job, dec_one_segment);
   /* the first error in segment order wins */
@@ -1079,6 +1138,63 @@ int orc_decompress_mt(const uint8_t *stream, uint64_t stream_bytes,
     if (seg_status[s] != ORC_OK && st == ORC_OK) st = seg_status[s];
   free(seg_status);
   if (st == ORC_OK && lay.data_base + expect_off != total) st = ORC_ERR_CORRUPT;
+  return st;
+}
+
+/* ========================================================================== */
+/* Attention over a compressed cache (reading R18; the ZipFusion abstract on  */
+/* the first page: decode attention that consumes the compressed KV cache).   */
+/* One decode step of grouped-query attention for every layer and request:   */
+/* query head j of layer l and request r reads kv head h = j / q_per_kv;     */
+/*   s_t = scale * (q . k^_t),  p = softmax_t(s),  o = sum_t p_t v^_t,       */
+/* t over the request's tokens, k^ and v^ the stream's decoded key and value */
+/* vectors without the bf16 rounding (orc_dequantize_vector_f64), all in     */
+/* double. q: bf16 [layers][n_requests][kv_heads * q_per_kv][d]; out: double  */
+/* of the same shape (zeros for a request without tokens).                   */
+/* ========================================================================== */
+int orc_attend(const uint8_t *stream, uint64_t stream_bytes, const orc_desc *expect,
+               const uint16_t *q, int q_per_kv, double scale, double *out, int n_threads) {
+  orc_layout lay;
+  double *vals, *s = NULL;
+  uint64_t T = 0, cum = 0, t;
+  int st = orc_layout_of(expect, &lay), l, r, j, c, H, d, Hq;
+  if (st != ORC_OK) return st;
+  if (q_per_kv < 1) return ORC_ERR_INVALID_ARG;
+  d = expect->head_dim;
+  H = expect->kv_heads;
+  Hq = H * q_per_kv;
+  for (r = 0; r < expect->n_requests; r++) T += expect->token_lens[r];
+  vals = (double *)malloc((size_t)(lay.V ? lay.V : 1) * (size_t)d * sizeof(double));
+  st = orc_decode_values_mt(stream, stream_bytes, expect, vals, n_threads);
+  if (st == ORC_OK) s = (double *)malloc((size_t)(T ? T : 1) * sizeof(double));
+  for (r = 0, cum = 0; st == ORC_OK && r < expect->n_requests; cum += expect->token_lens[r], r++) {
+    const uint64_t n = expect->token_lens[r];
+    for (l = 0; l < expect->layers; l++) {
+      for (j = 0; j < Hq; j++) {
+        const uint64_t qi = (((uint64_t)l * expect->n_requests + r) * Hq + j) * d;
+        const int h = j / q_per_kv;
+        const double *K = vals + ((((uint64_t)l * 2 + 0) * H + h) * T + cum) * d;
+        const double *Vv = vals + ((((uint64_t)l * 2 + 1) * H + h) * T + cum) * d;
+        double m = -INFINITY, den = 0.0;
+        for (c = 0; c < d; c++) out[qi + c] = 0.0;
+        if (n == 0) continue;
+        for (t = 0; t < n; t++) {
+          double acc = 0.0;
+          for (c = 0; c < d; c++) acc += (double)orc_bf16_to_f32(q[qi + c]) * K[t * d + c];
+          s[t] = scale * acc;
+          if (s[t] > m) m = s[t];
+        }
+        for (t = 0; t < n; t++) {
+          const double p = exp(s[t] - m);
+          den += p;
+          for (c = 0; c < d; c++) out[qi + c] += p * Vv[t * d + c];
+        }
+        for (c = 0; c < d; c++) out[qi + c] /= den;
+      }
+    }
+  }
+  free(s);
+  free(vals);
   return st;
 }
 

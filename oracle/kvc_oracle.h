@@ -68,6 +68,9 @@ int orc_quantize_vector(const uint16_t *x, int d, int bits, int g,
 void orc_dequantize_vector(const uint8_t *codes, const uint8_t *meta, int d,
                            int bits, int g, const uint64_t *sign_words,
                            uint16_t *xhat);
+void orc_dequantize_vector_f64(const uint8_t *codes, const uint8_t *meta, int d,
+                               int bits, int g, const uint64_t *sign_words,
+                               double *xhat);
 void orc_pack_codes(const uint8_t *q, int d, int bits, uint8_t *packed);
 void orc_unpack_codes(const uint8_t *packed, int d, int bits, uint8_t *q);
 
@@ -167,6 +170,16 @@ int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
                     uint64_t capacity, uint64_t *out_bytes, int n_threads);
 int orc_decompress_mt(const uint8_t *stream, uint64_t stream_bytes,
                       const orc_desc *expect, uint16_t *vectors, int n_threads);
+
+/* The stream's decoded vectors without the final bf16 rounding, in double
+ * ([V][d], orc_dequantize_vector_f64). */
+int orc_decode_values_mt(const uint8_t *stream, uint64_t stream_bytes,
+                         const orc_desc *expect, double *vals, int n_threads);
+
+/* Reading R18: one decode step of grouped-query attention over the stream's
+ * keys and values (all layers and requests), in double; see kvc_oracle.c. */
+int orc_attend(const uint8_t *stream, uint64_t stream_bytes, const orc_desc *expect,
+               const uint16_t *q, int q_per_kv, double scale, double *out, int n_threads);
 
 /* ---- layouts: logical vector order [layer][kv][head][request][token] ------ */
 void orc_gather_dense(const uint16_t *base, int layers, int kv_heads,
