@@ -288,6 +288,45 @@ kvc_status kvc_compress_unfused(const kvc_kv_desc *kv, const kvc_params *params,
                                 uint64_t *out_bytes_dev, void *workspace,
                                 size_t workspace_bytes, kvc_stream_t stream);
 
+/* ---- Attention over the compressed cache (the first page's ZipFusion
+ * abstract: decode attention that consumes the compressed KV cache in
+ * registers, without decompressing it to memory first).
+ *
+ * One decode step of grouped-query attention for every layer and request of
+ * a compressed cache: query head j of layer l and request r attends to kv
+ * head j / q_per_kv over the request's tokens,
+ *   out = sum_t softmax_t(scale * q . k_t) v_t,
+ * with k_t, v_t the stream's decoded vectors without the decoder's final
+ * bf16 rounding (its fp32 transformed values mapped back by the inverse
+ * transform). The kernels score and accumulate in the transformed domain
+ * (q . k = (H D q) . y / d) and invert the transform once per query head, so
+ * no decoded key or value is written to memory.
+ *
+ * The stream must describe a cache of this shape with these bits and group,
+ * head_dim 128, and store every code chunk raw (the header flag clear, the
+ * usual case; KVC_ERR_CORRUPT in the status word otherwise); its meta chunks
+ * may use any lossless pipeline. q: DEVICE bf16 [layers][n_requests]
+ * [kv_heads * q_per_kv][128], contiguous; out: DEVICE fp32 of the same shape
+ * (zeros for a request without tokens). seq_lens: HOST, the stream's
+ * per-request token counts. q_per_kv 1 to 8. The workspace holds the
+ * status word, the expanded meta chunks and the split partials. */
+typedef struct {
+  int32_t layers;
+  int32_t kv_heads;
+  int32_t head_dim;           /* 128 */
+  int32_t q_per_kv;           /* 1 .. 8 (e.g. 4 for 32 query / 8 kv heads) */
+  int32_t bits;               /* as compressed */
+  int32_t group_size;         /* as compressed */
+  int32_t n_requests;         /* 1 .. KVC_MAX_REQUESTS */
+  float scale;                /* e.g. 1 / sqrt(head_dim) */
+  const int32_t *seq_lens;    /* HOST [n_requests] */
+  const void *q;              /* DEVICE bf16 */
+  float *out;                 /* DEVICE fp32 */
+} kvc_attn_desc;
+size_t kvc_attend_workspace_bytes(const kvc_attn_desc *attn);
+kvc_status kvc_attend(const void *in, size_t in_bytes, const kvc_attn_desc *attn,
+                      void *workspace, size_t workspace_bytes, kvc_stream_t stream);
+
 /* Measurement only (no page defines these; they let a benchmark time each
  * kernel of a call with CUDA events on the call's own stream). The same work
  * and results as kvc_compress / kvc_decompress, with n_events == 5 caller-

@@ -29,7 +29,7 @@ EXPORTS = ["kvc_max_compressed_bytes", "kvc_workspace_bytes", "kvc_compress",
            "kvc_decompress", "kvc_stream_status", "kvc_status_string", "kvc_compress_noalloc",
            "kvc_decompress_workspace_bytes", "kvc_unfused_workspace_bytes",
            "kvc_compress_unfused", "kvc_test_compress_stalled", "kvc_compress_timed",
-           "kvc_decompress_timed"]
+           "kvc_decompress_timed", "kvc_attend_workspace_bytes", "kvc_attend"]
 
 
 class KvcError(RuntimeError):
@@ -45,6 +45,13 @@ class kvc_params(C.Structure):
 
 # Lossless-stage modes (kvc_params.lossless) and pipeline ids of a chunk.
 KVC_LOSSLESS_FIXED, KVC_LOSSLESS_SEARCH, KVC_LOSSLESS_NONE = range(3)
+
+
+class kvc_attn_desc(C.Structure):
+    _fields_ = [("layers", C.c_int32), ("kv_heads", C.c_int32), ("head_dim", C.c_int32),
+                ("q_per_kv", C.c_int32), ("bits", C.c_int32), ("group_size", C.c_int32),
+                ("n_requests", C.c_int32), ("scale", C.c_float),
+                ("seq_lens", C.POINTER(C.c_int32)), ("q", C.c_void_p), ("out", C.c_void_p)]
 
 
 class kvc_kv_desc(C.Structure):
@@ -101,6 +108,11 @@ def lib() -> C.CDLL:
         L.kvc_decompress_timed.restype = C.c_int
         L.kvc_decompress_timed.argtypes = [C.c_void_p, C.c_size_t, D, C.c_void_p, C.c_size_t,
                                            C.POINTER(C.c_void_p), C.c_int, C.c_void_p]
+        A = C.POINTER(kvc_attn_desc)
+        L.kvc_attend_workspace_bytes.restype = C.c_size_t
+        L.kvc_attend_workspace_bytes.argtypes = [A]
+        L.kvc_attend.restype = C.c_int
+        L.kvc_attend.argtypes = [C.c_void_p, C.c_size_t, A, C.c_void_p, C.c_size_t, C.c_void_p]
         L.kvc_test_compress_stalled.restype = C.c_int
         L.kvc_test_compress_stalled.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p,
                                                 C.c_void_p, C.c_size_t, C.c_uint32, C.c_uint64,
@@ -171,6 +183,26 @@ def kvc_decompress_timed(in_ptr, in_bytes, desc, ws_ptr, ws_bytes, events, strea
     arr = _event_array(events)
     return lib().kvc_decompress_timed(in_ptr, in_bytes, C.byref(desc), ws_ptr, ws_bytes, arr,
                                       len(events), stream)
+
+
+def attn_desc(layers, kv_heads, q_per_kv, bits, group, seq_lens, q, out, scale,
+              head_dim: int = 128) -> kvc_attn_desc:
+    """Descriptor of kvc_attend: q bf16 [layers, n_requests, kv_heads * q_per_kv,
+    head_dim] and out fp32 of the same shape (device tensors)."""
+    seq = (C.c_int32 * max(len(seq_lens), 1))(*[int(x) for x in seq_lens])
+    d = kvc_attn_desc(layers, kv_heads, head_dim, q_per_kv, bits, group, len(seq_lens),
+                      float(scale), C.cast(seq, C.POINTER(C.c_int32)), q.data_ptr(),
+                      out.data_ptr())
+    d._keep = (seq, q, out)
+    return d
+
+
+def kvc_attend_workspace_bytes(attn: kvc_attn_desc) -> int:
+    return lib().kvc_attend_workspace_bytes(C.byref(attn))
+
+
+def kvc_attend(in_ptr, in_bytes, attn, ws_ptr, ws_bytes, stream) -> int:
+    return lib().kvc_attend(in_ptr, in_bytes, C.byref(attn), ws_ptr, ws_bytes, stream)
 
 
 def kvc_decompress(in_ptr, in_bytes, desc, ws_ptr, ws_bytes, stream) -> int:

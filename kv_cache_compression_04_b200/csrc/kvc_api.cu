@@ -473,6 +473,110 @@ kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *ou
   return e == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
+namespace {
+constexpr int kAttTokHost = 256;  // tokens per attention CTA (kvc_attend.cuh: kAttTok)
+
+// Shape checks of kvc_attend and its workspace layout: status | expanded
+// meta chunks | split partials.
+struct AttnShape {
+  Shape s;
+  uint64_t meta_off, part_off, total;
+  uint32_t splits, units;
+};
+kvc_status attn_shape(const kvc_attn_desc *at, AttnShape &r) {
+  if (!at) return KVC_ERR_INVALID_ARG;
+  if (at->head_dim != 128) return KVC_ERR_UNSUPPORTED;
+  if (at->q_per_kv < 1 || at->q_per_kv > 8) return KVC_ERR_UNSUPPORTED;
+  if (at->n_requests < 1 || at->n_requests > KVC_MAX_REQUESTS || !at->seq_lens)
+    return KVC_ERR_INVALID_ARG;
+  // the stream's logical shape as a paged description without pages: the
+  // shape checks and layout arithmetic of the codec
+  kvc_kv_desc kv{};
+  kv.kind = KVC_DENSE;
+  kv.layers = at->layers;
+  kv.kv_heads = at->kv_heads;
+  kv.head_dim = at->head_dim;
+  int64_t T = 0, maxlen = 0;
+  for (int i = 0; i < at->n_requests; ++i) {
+    if (at->seq_lens[i] < 0) return KVC_ERR_INVALID_ARG;
+    T += at->seq_lens[i];
+    maxlen = at->seq_lens[i] > maxlen ? at->seq_lens[i] : maxlen;
+  }
+  kv.tokens = T;
+  kv.data = reinterpret_cast<void *>(uintptr_t(16));  // shape only: never read
+  kv.stride_token = at->head_dim;
+  kv.stride_head = T * at->head_dim;
+  kv.stride_kv = kv.stride_head * at->kv_heads;
+  kv.stride_layer = kv.stride_kv * 2;
+  kvc_params p{at->bits, at->group_size, 0, KVC_LOSSLESS_FIXED, 0};
+  const kvc_status st = describe(&kv, &p, r.s);
+  if (st != KVC_OK) return st;
+  r.s.n_req = uint32_t(at->n_requests);
+  r.splits = uint32_t(maxlen == 0 ? 1 : (maxlen + kAttTokHost - 1) / kAttTokHost);
+  r.units = uint32_t(at->layers) * uint32_t(at->n_requests) * uint32_t(at->kv_heads);
+  r.meta_off = kWsCtl;
+  r.part_off = round256(r.meta_off + max_meta_chunks(r.s) * kChunk);
+  r.total = r.part_off + uint64_t(r.units) * r.splits * uint64_t(at->q_per_kv) *
+                             (uint64_t(at->head_dim) + 4) * sizeof(float);
+  return KVC_OK;
+}
+}  // namespace
+
+size_t kvc_attend_workspace_bytes(const kvc_attn_desc *at) {
+  AttnShape r;
+  return attn_shape(at, r) == KVC_OK ? size_t(r.total) : 0;
+}
+
+kvc_status kvc_attend(const void *in, size_t in_bytes, const kvc_attn_desc *at, void *workspace,
+                      size_t workspace_bytes, kvc_stream_t stream) {
+  AttnShape r;
+  kvc_status st = attn_shape(at, r);
+  if (st != KVC_OK) return st;
+  if (!in || !aligned16(in) || !workspace || !aligned16(workspace) || !at->q || !at->out ||
+      (reinterpret_cast<uintptr_t>(at->q) & 1u) || (reinterpret_cast<uintptr_t>(at->out) & 3u))
+    return KVC_ERR_INVALID_ARG;
+  if (workspace_bytes < r.total) return KVC_ERR_CAPACITY;
+  const int sms = sm_count();
+  if (sms <= 0) return KVC_ERR_CUDA;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  DecArgs d{};
+  d.in = static_cast<const uint8_t *>(in);
+  d.in_bytes = in_bytes;
+  d.status = reinterpret_cast<uint32_t *>(ws);
+  d.layers = uint32_t(at->layers);
+  d.kv_heads = uint32_t(at->kv_heads);
+  d.head_dim = uint32_t(at->head_dim);
+  d.n_req = r.s.n_req;
+  d.tokens = r.s.T;
+  d.V = uint32_t(r.s.V);
+  d.paged_receiver = 0;
+  d.ws_meta = ws + r.meta_off;
+  d.ws_meta_chunks = uint32_t(max_meta_chunks(r.s));
+  static thread_local AttnArgs a;  // large (4 KB) parameter block
+  a.in = d.in;
+  a.in_bytes = in_bytes;
+  a.status = d.status;
+  a.layers = d.layers;
+  a.kv_heads = d.kv_heads;
+  a.n_req = d.n_req;
+  a.qpk = uint32_t(at->q_per_kv);
+  a.bits = uint32_t(at->bits);
+  a.group = uint32_t(at->group_size);
+  a.tokens = r.s.T;
+  a.V = d.V;
+  a.splits = r.splits;
+  a.q = static_cast<const uint16_t *>(at->q);
+  a.scale = at->scale;
+  a.out = at->out;
+  a.part = reinterpret_cast<float *>(ws + r.part_off);
+  a.ws_meta = d.ws_meta;
+  a.cum[0] = 0;
+  for (int i = 0; i < at->n_requests; ++i) a.cum[i + 1] = a.cum[i] + uint32_t(at->seq_lens[i]);
+  if (clear_words(workspace, kWsCtl, sms, cs) != cudaSuccess) return KVC_ERR_CUDA;
+  return launch_attend(a, d, sms, cs) == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
 kvc_status kvc_stream_status(const void *workspace, kvc_stream_t stream) {
   if (!workspace) return KVC_ERR_INVALID_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);

@@ -455,82 +455,72 @@ __global__ void __launch_bounds__(kEncThreads, 1)
   };
   if constexpr (kPaged) {
     grid_dependency_wait();  // the workspace clear (a plan may record a status)
-    // Block plans. A block whose 32 tokens lie in one request (all
-    // but about one in a hundred of a batch of long requests) loads as the
-    // 8-slot runs of its pages: lane j < runs reads run j's page and issues
-    // one tensor box of 8 rows per 64-channel half into 1 KB slot j of the
-    // buffer, so lane i's row is row (t0 % 8) + i. Other blocks (a request
-    // boundary, a page outside the pool, no tensor map) are gathered row by
-    // row, lane i's row at row i. A plan is one word per lane: kind (bits
-    // 0-1: 0 past the end, 1 boxes, 2 gather), t0 % 8 (2-4), the lane's run
-    // starting at slot 8 (5), the head row lkh (6..); plus the lane's page or
-    // gather row.
-    // A plan is made one block ahead of its issue (the page-table reads and
-    // the request search overlap a block of arithmetic). Per lane it is one
-    // word (kind in bits 0-1: 0 past the end, 1 boxes, 2 gather; t0 % 8 in
-    // bits 2-4; the lane's run starting at slot 8 in bit 5; the head row lkh
-    // from bit 6) and one 64-bit value: the lane's run page (boxes) or row
-    // address (gather).
-    auto plan = [&](uint32_t b, uint64_t &arg) -> uint32_t {
+    // A block whose 32 tokens lie in one request (all but about one in a
+    // hundred of a batch of long requests) loads as the 8-slot runs of its
+    // pages: lane j < runs reads run j's page and issues one tensor box of 8
+    // rows per 64-channel half into 1 KB slot j of the buffer, so lane i's
+    // row is row (t0 % 8) + i. Other blocks (a request boundary, a page
+    // outside the pool, no tensor map) are gathered row by row, lane i's row
+    // at row i. A plan is made one block ahead of its issue and reads nothing it
+    // needs at once: the block's request comes from one shared-memory load
+    // per lane and a ballot over the request prefix (no dependent search),
+    // and the lanes of its runs load their pages, which are checked only at
+    // issue, a block of arithmetic later. Per lane a plan is one word (kind
+    // in bits 0-1: 0 past the end, 1 runs of one request, 2 any other block;
+    // t0 % 8 in bits 2-4; the lane's run starting at slot 8 in bit 5; the
+    // head row lkh from bit 6) and the lane's run page.
+    auto plan = [&](uint32_t b, int32_t &pg) -> uint32_t {
       const uint32_t v0 = b * 32;
-      arg = 0;
+      pg = -1;
       if (v0 >= V) return 0u;
-      uint32_t simple = 0, t0 = 0, r = 0, lkh = 0;
-      if (lay.tma && lane == 0) {
-        lkh = fdiv(lay.T, v0);
-        const uint32_t u0 = v0 - lkh * lay.T.d;
-        uint32_t lo = 0, hi = lay.n_req - 1;  // largest r with cum[r] <= u0
-        while (lo < hi) {
-          const uint32_t mid = (lo + hi + 1) >> 1;
-          if (s_cum[mid] <= u0)
-            lo = mid;
-          else
-            hi = mid - 1;
-        }
-        r = lo;
-        t0 = u0 - s_cum[r];
-        simple = v0 + 32 <= V && u0 + 32 <= s_cum[r + 1];
+      if (!lay.tma) return 2u;
+      const uint32_t lkh = fdiv(lay.T, v0), u0 = v0 - lkh * lay.T.d;
+      uint32_t r = 0;  // the largest r with cum[r] <= u0 (cum is nondecreasing)
+      for (uint32_t g0 = 0; g0 <= lay.n_req; g0 += 32) {
+        const uint32_t i = g0 + lane;
+        const uint32_t below = __ballot_sync(0xFFFFFFFFu, i <= lay.n_req && s_cum[min(i, lay.n_req)] <= u0);
+        r = g0 + __popc(below) - 1;
+        if (below != 0xFFFFFFFFu) break;
       }
-      if (__shfl_sync(0xFFFFFFFFu, simple, 0)) {
-        t0 = __shfl_sync(0xFFFFFFFFu, t0, 0);
-        r = __shfl_sync(0xFFFFFFFFu, r, 0);
-        lkh = __shfl_sync(0xFFFFFFFFu, lkh, 0);
-        const uint32_t runs = ((t0 + 31) >> 3) - (t0 >> 3) + 1;  // 4 or 5
-        bool ok = true;
-        uint32_t hi8 = 0;
-        if (uint32_t(lane) < runs) {
-          const uint32_t hp = (t0 >> 3) + lane;  // the run's 8-slot half page
-          const int32_t pg = __ldg(lay.page_table + int64_t(r) * lay.pt_stride + (hp >> 1));
-          ok = pg >= 0 && int64_t(pg) < lay.num_pages;
-          hi8 = hp & 1u;
-          arg = uint32_t(pg);
-        }
-        if (__all_sync(0xFFFFFFFFu, ok)) return 1u | ((t0 & 7u) << 2) | (hi8 << 5) | (lkh << 6);
+      const uint32_t t0 = u0 - s_cum[r];
+      if (!(v0 + 32 <= V && u0 + 32 <= s_cum[r + 1])) return 2u;
+      const uint32_t runs = ((t0 + 31) >> 3) - (t0 >> 3) + 1;  // 4 or 5
+      uint32_t hi8 = 0;
+      if (uint32_t(lane) < runs) {
+        const uint32_t hp = (t0 >> 3) + lane;  // the run's 8-slot half page
+        pg = __ldg(lay.page_table + int64_t(r) * lay.pt_stride + (hp >> 1));
+        hi8 = hp & 1u;
       }
-      arg = reinterpret_cast<uint64_t>(src_of(v0 + lane));
-      return 2u;
+      return 1u | ((t0 & 7u) << 2) | (hi8 << 5) | (lkh << 6);
     };
-    auto issue = [&](uint32_t p, uint64_t arg) {
+    // Issues block b's loads; returns the kind used (runs need every page in
+    // the pool, else the block is gathered row by row, which records a bad
+    // page) and the row shift.
+    auto issue = [&](uint32_t b, uint32_t p, int32_t pg) -> uint32_t {
       if ((p & 3u) == 1u) {
         const uint32_t runs = (((p >> 2) & 7u) + 31) / 8 + 1;
-        if (lane == 0) mbar_arrive_expect_tx(wbar, runs * uint32_t(D / 64) * 1024u);
-        __syncwarp();
-        if (uint32_t(lane) < runs) {
-          const uint32_t lkh = p >> 6, lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
-          const int kvh = int((lk & 1u) * lay.H.d + h), slot = int(((p >> 5) & 1u) * 8);
+        const bool ok = uint32_t(lane) >= runs || (pg >= 0 && int64_t(pg) < lay.num_pages);
+        if (__all_sync(0xFFFFFFFFu, ok)) {
+          if (lane == 0) mbar_arrive_expect_tx(wbar, runs * uint32_t(D / 64) * 1024u);
+          __syncwarp();
+          if (uint32_t(lane) < runs) {
+            const uint32_t lkh = p >> 6, lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
+            const int kvh = int((lk & 1u) * lay.H.d + h), slot = int(((p >> 5) & 1u) * 8);
 #pragma unroll
-          for (int hh = 0; hh < D / 64; ++hh)
-            tma_load_5d(wbuf + hh * S::HALF + lane * 1024, &lay.tmap, hh * 64, slot, kvh,
-                        int(uint32_t(arg)), int(lk >> 1), wbar);
+            for (int hh = 0; hh < D / 64; ++hh)
+              tma_load_5d(wbuf + hh * S::HALF + lane * 1024, &lay.tmap, hh * 64, slot, kvh, pg,
+                          int(lk >> 1), wbar);
+          }
+          return p & 31u;
         }
-      } else if ((p & 3u) == 2u) {
-        gather(reinterpret_cast<const uint8_t *>(arg));
+        p = 2u;
       }
+      if ((p & 3u) == 2u) gather(src_of(b * 32 + lane));
+      return p & 3u;
     };
-    uint64_t narg;
-    uint32_t cur = plan(blk, narg);
-    issue(cur, narg);
-    uint32_t next = plan(blk + stride, narg);
+    int32_t npg;
+    uint32_t cur = issue(blk, plan(blk, npg), npg);
+    uint32_t next = plan(blk + stride, npg);
 #pragma unroll 1
     for (; blk < n_blocks; blk += stride) {
       const uint32_t v = blk * 32 + lane;
@@ -546,9 +536,8 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       // every lane has read the buffer; the next load may overwrite it
       fence_proxy_async_smem();
       __syncwarp();
-      issue(next, narg);
-      cur = next & 31u;
-      next = plan(blk + 2 * stride, narg);
+      cur = issue(blk + stride, next, npg);
+      next = plan(blk + 2 * stride, npg);
       finish_block(blk, v, v < V, y);
     }
   } else if (!use_tma) {

@@ -260,6 +260,23 @@ cudaError_t launch_transform_paged(int d, const EncArgs &a, const PagedLayout &l
                                    cudaStream_t st);
 cudaError_t launch_quantize(int d, int bits, int group, const EncArgs &a, int sms, cudaStream_t st);
 cudaError_t launch_finish_dense(const FinArgs &a, const DenseLayout &lay, int sms, cudaStream_t st);
+// Attention over the compressed cache (kvc_attend).
+struct AttnArgs {
+  const uint8_t *in;
+  uint64_t in_bytes;
+  uint32_t *status;
+  uint32_t layers, kv_heads, n_req, qpk;  // qpk: query heads per kv head
+  uint32_t bits, group;                   // as the caller states them (checked)
+  uint64_t tokens;                        // all requests
+  uint32_t V, splits;                     // vectors; CTAs per (layer, request, kv head)
+  const uint16_t *q;                      // bf16 [layers][n_req][kv_heads * qpk][D]
+  float scale;
+  float *out;                             // fp32, the shape of q
+  float *part;                            // per CTA and query head: m, l, o[D]
+  const uint8_t *ws_meta;                 // meta chunks expanded by meta_expand_kernel
+  uint32_t cum[KVC_MAX_REQUESTS + 1];     // token prefix per request
+};
+cudaError_t launch_attend(const AttnArgs &a, const DecArgs &d, int sms, cudaStream_t st);
 cudaError_t launch_finish_paged(const FinArgs &a, const PagedLayout &lay, int sms, cudaStream_t st);
 
 }  // namespace kvc
