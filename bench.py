@@ -577,6 +577,127 @@ def time_config(wname: str, dev, steps: int, warmup: int, hbm: float, flush=None
     return r
 
 
+# query heads per kv head of the model each workload is shaped after
+ATTN_QPK = {"llama8b": 4, "qwen7b": 7, "paged": 8}
+
+
+def time_attend(wname: str, dev, steps: int, warmup: int, hbm: float, qpk: int | None = None):
+    """One decode step of grouped-query attention over the compressed cache
+    of a workload (kvc_attend: every layer, request and query head), timed
+    like time_config, against (dense workloads) decompress-to-bf16 followed
+    by torch's scaled_dot_product_attention, and the same attention on the
+    uncompressed bf16 cache. Algorithmic bytes of the attention kernel: the
+    packed codes and scale/zero of every key and value it scores (the
+    payload), the bf16 queries and the fp32 outputs."""
+    import torch
+    import kv_cache_compression_04_b200 as kvc
+    qpk = qpk or ATTN_QPK.get(wname.split("-")[0], 4)
+    w, desc, out_desc_fn, keep = make_input(wname, dev, 0)
+    codec = kvc.Codec(w.bits, w.group, w.sign_seed)
+    out, ws, nb = codec.buffers(desc, dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = kvc._stream_ptr(stream)
+    assert kvc.kvc_compress(desc, codec.params, out.data_ptr(), out.numel(), nb.data_ptr(),
+                            ws.data_ptr(), ws.numel(), sp) == kvc.KVC_OK
+    assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+    n = int(nb.item())
+    lens = list(w.seq_lens) if w.paged else [w.tokens]
+    L, H, d = w.layers, w.kv_heads, w.head_dim
+    g = torch.Generator(device=dev).manual_seed(7)
+    q = torch.randn(L, len(lens), H * qpk, d, generator=g, device=dev).to(torch.bfloat16)
+    o = torch.empty(L, len(lens), H * qpk, d, device=dev)
+    scale = d ** -0.5
+    ad = kvc.attn_desc(L, H, qpk, w.bits, w.group, lens, q, o, scale)
+    aws = torch.empty(kvc.kvc_attend_workspace_bytes(ad), dtype=torch.uint8, device=dev)
+
+    def att():
+        assert kvc.kvc_attend(out.data_ptr(), n, ad, aws.data_ptr(), aws.numel(),
+                              sp) == kvc.KVC_OK
+
+    att()
+    assert kvc.kvc_stream_status(aws.data_ptr(), sp) == kvc.KVC_OK
+    evs = [new_events(2, stream) for _ in range(warmup + steps)]
+    tev = [new_events(5, stream) for _ in range(warmup + steps)]
+    torch.cuda.synchronize(dev)
+    for e in evs:
+        e[0].record(stream)
+        att()
+        e[1].record(stream)
+    for e in tev:
+        assert kvc.kvc_attend_timed(out.data_ptr(), n, ad, aws.data_ptr(), aws.numel(), e,
+                                    sp) == kvc.KVC_OK
+    torch.cuda.synchronize(dev)
+    assert kvc.kvc_stream_status(aws.data_ptr(), sp) == kvc.KVC_OK
+    call_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs[warmup:])
+    kt = [statistics.median(e[i].elapsed_time(e[i + 1]) for e in tev[warmup:]) for i in range(4)]
+    alg = payload_bytes(w) + q.numel() * 2 + o.numel() * 4
+    r = {"workload": describe(w), "q_per_kv": qpk, "query_heads": H * qpk,
+         "requests": len(lens), "call_ms": round(call_ms, 4),
+         "kernel_ms": {"clear": round(kt[0], 4), "meta_expand": round(kt[1], 4),
+                       "attend": round(kt[2], 4), "combine": round(kt[3], 4)},
+         "attend_kernel": {"bound": "hbm", "algorithmic_bytes": alg,
+                           "achieved": round(alg / (kt[2] * 1e-3) / 1e9, 1), "peak": hbm,
+                           "unit": "GB/s", "frac": round(alg / (kt[2] * 1e-3) / 1e9 / hbm, 4)},
+         "kv_positions_per_s": round(L * H * w.total_tokens / (call_ms * 1e-3), 1),
+         "steps": steps, "timing": "median of steps", "l2": "inputs larger than L2"}
+    if not w.paged:
+        # decompress to bf16, then torch's attention (flash or memory-efficient)
+        odesc, obuf = out_desc_fn()
+        dws = torch.empty(kvc.kvc_decompress_workspace_bytes(odesc), dtype=torch.uint8,
+                          device=dev)
+        qs = q.view(L, H * qpk, 1, d)
+        k4, v4 = obuf[:, 0], obuf[:, 1]
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        F = torch.nn.functional
+
+        def sdpa():
+            with sdpa_kernel([SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION,
+                              SDPBackend.CUDNN_ATTENTION]):
+                return F.scaled_dot_product_attention(qs, k4, v4, scale=scale, enable_gqa=True)
+
+        def unfused():
+            assert kvc.kvc_decompress(out.data_ptr(), n, odesc, dws.data_ptr(), dws.numel(),
+                                      sp) == kvc.KVC_OK
+            return sdpa()
+
+        try:
+            unfused()
+            ref = sdpa().float().view_as(o)
+            torch.cuda.synchronize(dev)
+            ue = [new_events(3, stream) for _ in range(warmup + steps)]
+            se = [new_events(2, stream) for _ in range(warmup + steps)]
+            for e in ue:
+                e[0].record(stream)
+                assert kvc.kvc_decompress(out.data_ptr(), n, odesc, dws.data_ptr(),
+                                          dws.numel(), sp) == kvc.KVC_OK
+                e[1].record(stream)
+                sdpa()
+                e[2].record(stream)
+            for e in se:
+                e[0].record(stream)
+                sdpa()
+                e[1].record(stream)
+            torch.cuda.synchronize(dev)
+            dms = statistics.median(e[0].elapsed_time(e[1]) for e in ue[warmup:])
+            ams = statistics.median(e[1].elapsed_time(e[2]) for e in ue[warmup:])
+            bms = statistics.median(e[0].elapsed_time(e[1]) for e in se[warmup:])
+            rel = float((o - ref).abs().max() / ref.abs().max())
+            r["unfused"] = {"decompress_ms": round(dms, 4), "sdpa_ms": round(ams, 4),
+                            "total_ms": round(dms + ams, 4),
+                            "fused_speedup": round((dms + ams) / call_ms, 3),
+                            "what": "kvc_decompress to bf16, then torch "
+                                    "scaled_dot_product_attention (GQA)"}
+            r["uncompressed_sdpa_ms"] = round(bms, 4)
+            r["vs_uncompressed_sdpa"] = round(bms / call_ms, 3)
+            r["max_rel_diff_vs_bf16_sdpa"] = round(rel, 6)
+        except RuntimeError as exc:  # no fused torch attention for this shape
+            r["unfused"] = {"unavailable": str(exc).splitlines()[0][:200]}
+        del obuf, dws
+    del keep, out, ws, nb, aws, q, o
+    torch.cuda.empty_cache()
+    return r
+
+
 def run_sweep(args):
     """Message-size sweep: [32, 2, 8, T, 128] with T = 8 * 2^i tokens (1 MiB ..
     4 GiB), 4-bit g128 and 2-bit g32. Each step times one compress and one
@@ -830,6 +951,8 @@ def main():
                     help="layer groups of the end-to-end timing (one call pair each)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--unfused-steps", type=int, default=20)
+    ap.add_argument("--attend", type=int, default=1,
+                    help="1: also time decode attention over each compressed cache")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--pipeline", action="store_true")
     args = ap.parse_args()
@@ -977,6 +1100,13 @@ def main():
         per_config = {}
         for wname in [x for x in args.per_config.split(",") if x and x != args.workload]:
             per_config[wname] = time_config(wname, dev, args.config_steps, args.warmup, hbm_)
+            if args.attend:
+                per_config[wname]["attend"] = time_attend(wname, dev, args.config_steps,
+                                                          args.warmup, hbm_)
+        if args.attend:
+            per_config["attend_" + args.workload] = time_attend(args.workload, dev,
+                                                                args.config_steps, args.warmup,
+                                                                hbm_)
         if args.sweep_points:
             flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
             per_config["sweep"] = [time_config(f"sweep-{i}-{b}", dev, args.config_steps,
@@ -998,7 +1128,8 @@ def main():
     # algorithmic bytes: a call reads the KV cache and writes the stream (or
     # the reverse); the fused encode kernel reads the KV cache and writes the
     # quantized payload (codes in place, raw meta to the workspace), the
-    # decode kernel the reverse (units: SURVEY 8(d) per-element figures)
+    # decode kernel the reverse (2 bytes per raw element, bits/8 per code,
+    # 4 bytes of scale and zero per group)
     pay = payload_bytes(w)
     enc_gbs = (raw + nbytes) / (enc_avg * 1e-3) / 1e9
     dec_gbs = (raw + nbytes) / (dec_avg * 1e-3) / 1e9

@@ -334,7 +334,8 @@ kvc_status kvc_attend(const void *in, size_t in_bytes, const kvc_attn_desc *attn
  * events[0] before the call's first kernel and events[i] after its i-th
  * kernel. Compress: workspace clear, encode, finishing (table, meta chunks,
  * header), compaction. Decompress: status clear, meta chunk expansion,
- * decode of eliminated code chunks, decode. A kernel that a call does not
+ * decode of eliminated code chunks, decode. Attend: status clear, meta chunk
+ * expansion, attention (split-K), combination. A kernel that a call does not
  * need gets an empty interval. The kernels of a timed call start in plain
  * stream order, without overlapping the previous kernel's tail, so a timed
  * call can take a few microseconds longer than an ordinary one. Other
@@ -346,6 +347,9 @@ kvc_status kvc_compress_timed(const kvc_kv_desc *kv, const kvc_params *params, v
 kvc_status kvc_decompress_timed(const void *in, size_t in_bytes, const kvc_kv_desc *out,
                                 void *workspace, size_t workspace_bytes, void *const *events,
                                 int n_events, kvc_stream_t stream);
+kvc_status kvc_attend_timed(const void *in, size_t in_bytes, const kvc_attn_desc *attn,
+                            void *workspace, size_t workspace_bytes, void *const *events,
+                            int n_events, kvc_stream_t stream);
 
 #ifdef __cplusplus
 }

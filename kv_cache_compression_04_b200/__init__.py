@@ -29,7 +29,8 @@ EXPORTS = ["kvc_max_compressed_bytes", "kvc_workspace_bytes", "kvc_compress",
            "kvc_decompress", "kvc_stream_status", "kvc_status_string", "kvc_compress_noalloc",
            "kvc_decompress_workspace_bytes", "kvc_unfused_workspace_bytes",
            "kvc_compress_unfused", "kvc_test_compress_stalled", "kvc_compress_timed",
-           "kvc_decompress_timed", "kvc_attend_workspace_bytes", "kvc_attend"]
+           "kvc_decompress_timed", "kvc_attend_workspace_bytes", "kvc_attend",
+           "kvc_attend_timed"]
 
 
 class KvcError(RuntimeError):
@@ -113,6 +114,9 @@ def lib() -> C.CDLL:
         L.kvc_attend_workspace_bytes.argtypes = [A]
         L.kvc_attend.restype = C.c_int
         L.kvc_attend.argtypes = [C.c_void_p, C.c_size_t, A, C.c_void_p, C.c_size_t, C.c_void_p]
+        L.kvc_attend_timed.restype = C.c_int
+        L.kvc_attend_timed.argtypes = [C.c_void_p, C.c_size_t, A, C.c_void_p, C.c_size_t,
+                                       C.POINTER(C.c_void_p), C.c_int, C.c_void_p]
         L.kvc_test_compress_stalled.restype = C.c_int
         L.kvc_test_compress_stalled.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p,
                                                 C.c_void_p, C.c_size_t, C.c_uint32, C.c_uint64,
@@ -203,6 +207,12 @@ def kvc_attend_workspace_bytes(attn: kvc_attn_desc) -> int:
 
 def kvc_attend(in_ptr, in_bytes, attn, ws_ptr, ws_bytes, stream) -> int:
     return lib().kvc_attend(in_ptr, in_bytes, C.byref(attn), ws_ptr, ws_bytes, stream)
+
+
+def kvc_attend_timed(in_ptr, in_bytes, attn, ws_ptr, ws_bytes, events, stream) -> int:
+    arr = _event_array(events)
+    return lib().kvc_attend_timed(in_ptr, in_bytes, C.byref(attn), ws_ptr, ws_bytes, arr,
+                                  len(events), stream)
 
 
 def kvc_decompress(in_ptr, in_bytes, desc, ws_ptr, ws_bytes, stream) -> int:

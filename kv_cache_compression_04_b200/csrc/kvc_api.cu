@@ -436,6 +436,16 @@ kvc_status kvc_decompress_timed(const void *in, size_t in_bytes, const kvc_kv_de
   return kvc_decompress(in, in_bytes, out, workspace, workspace_bytes, stream);
 }
 
+kvc_status kvc_attend_timed(const void *in, size_t in_bytes, const kvc_attn_desc *attn,
+                            void *workspace, size_t workspace_bytes, void *const *events,
+                            int n_events, kvc_stream_t stream) {
+  if (!events || n_events != 5) return KVC_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return KVC_ERR_INVALID_ARG;
+  TimedCall timed(reinterpret_cast<const cudaEvent_t *>(events));
+  return kvc_attend(in, in_bytes, attn, workspace, workspace_bytes, stream);
+}
+
 kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *out,
                           void *workspace, size_t workspace_bytes, kvc_stream_t stream) {
   Shape s;
@@ -480,7 +490,7 @@ constexpr int kAttTokHost = 256;  // tokens per attention CTA (kvc_attend.cuh: k
 // meta chunks | split partials.
 struct AttnShape {
   Shape s;
-  uint64_t meta_off, part_off, total;
+  uint64_t meta_off, meta_chunks, part_off, total;
   uint32_t splits, units;
 };
 kvc_status attn_shape(const kvc_attn_desc *at, AttnShape &r) {
@@ -515,7 +525,10 @@ kvc_status attn_shape(const kvc_attn_desc *at, AttnShape &r) {
   r.splits = uint32_t(maxlen == 0 ? 1 : (maxlen + kAttTokHost - 1) / kAttTokHost);
   r.units = uint32_t(at->layers) * uint32_t(at->n_requests) * uint32_t(at->kv_heads);
   r.meta_off = kWsCtl;
-  r.part_off = round256(r.meta_off + max_meta_chunks(r.s) * kChunk);
+  // the stated group fixes the meta chunk count (a stream with another
+  // group fails the header check; meta expansion never exceeds the slots)
+  r.meta_chunks = (r.s.V * uint64_t(at->head_dim / at->group_size) * 4 + kChunk - 1) / kChunk;
+  r.part_off = round256(r.meta_off + r.meta_chunks * kChunk);
   r.total = r.part_off + uint64_t(r.units) * r.splits * uint64_t(at->q_per_kv) *
                              (uint64_t(at->head_dim) + 4) * sizeof(float);
   return KVC_OK;
@@ -552,7 +565,7 @@ kvc_status kvc_attend(const void *in, size_t in_bytes, const kvc_attn_desc *at, 
   d.V = uint32_t(r.s.V);
   d.paged_receiver = 0;
   d.ws_meta = ws + r.meta_off;
-  d.ws_meta_chunks = uint32_t(max_meta_chunks(r.s));
+  d.ws_meta_chunks = uint32_t(r.meta_chunks);
   static thread_local AttnArgs a;  // large (4 KB) parameter block
   a.in = d.in;
   a.in_bytes = in_bytes;

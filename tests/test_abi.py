@@ -259,3 +259,47 @@ def test_timed_calls_refuse_bad_event_arrays(L):
                                     None) == kvc.KVC_ERR_INVALID_ARG
         assert L.kvc_decompress_timed(FAKE, 4096, C.byref(d), FAKE, 1 << 20, arr, n,
                                       None) == kvc.KVC_ERR_INVALID_ARG
+
+
+class _Ptr:
+    def __init__(self, p):
+        self.p = p
+
+    def data_ptr(self):
+        return self.p
+
+
+def test_attend_refuses_bad_arguments_and_sizes_its_workspace(L):
+    """kvc_attend / kvc_attend_workspace_bytes on the host side: shape and
+    pointer checks, and the workspace size (status words, one 16 KB slot per
+    meta chunk, one partial record of 4 + 128 floats per CTA and query head)."""
+    q, out = _Ptr(FAKE), _Ptr(FAKE)
+    lens = [1000, 0, 513]
+    ad = kvc.attn_desc(2, 8, 4, 4, 64, lens, q, out, 0.1)
+    wsb = kvc.kvc_attend_workspace_bytes(ad)
+    V = 2 * 2 * 8 * sum(lens)
+    n_meta = -(-V * 8 // 16384)            # 2 groups of 4 bytes per vector
+    splits = -(-1000 // 256)
+    parts = 2 * 3 * 8 * splits * 4 * 132 * 4
+    assert wsb >= n_meta * 16384 + parts
+    assert wsb <= n_meta * 16384 + parts + 4096
+    for bad, why in [(kvc.attn_desc(2, 8, 0, 4, 64, lens, q, out, 0.1), "q_per_kv 0"),
+                     (kvc.attn_desc(2, 8, 9, 4, 64, lens, q, out, 0.1), "q_per_kv 9"),
+                     (kvc.attn_desc(2, 8, 4, 3, 64, lens, q, out, 0.1), "bits 3"),
+                     (kvc.attn_desc(2, 8, 4, 4, 48, lens, q, out, 0.1), "group 48"),
+                     (kvc.attn_desc(2, 8, 4, 4, 64, lens, q, out, 0.1, head_dim=64), "d 64"),
+                     (kvc.attn_desc(2, 8, 4, 4, 64, [], q, out, 0.1), "no requests")]:
+        assert kvc.kvc_attend_workspace_bytes(bad) == 0, why
+        assert kvc.kvc_attend(FAKE, 1 << 20, bad, FAKE, wsb, None) != kvc.KVC_OK, why
+    assert kvc.kvc_attend(FAKE, 1 << 20, ad, FAKE, wsb - 1, None) == kvc.KVC_ERR_CAPACITY
+    assert kvc.kvc_attend(FAKE + 8, 1 << 20, ad, FAKE, wsb, None) == kvc.KVC_ERR_INVALID_ARG
+    assert kvc.kvc_attend(FAKE, 1 << 20, kvc.attn_desc(2, 8, 4, 4, 64, lens, _Ptr(FAKE + 1),
+                                                       out, 0.1), FAKE, wsb,
+                          None) == kvc.KVC_ERR_INVALID_ARG
+    assert kvc.kvc_attend(FAKE, 1 << 20, kvc.attn_desc(2, 8, 4, 4, 64, lens, q, _Ptr(FAKE + 2),
+                                                       0.1), FAKE, wsb,
+                          None) == kvc.KVC_ERR_INVALID_ARG
+    assert L.kvc_attend(FAKE, 1 << 20, None, FAKE, wsb, None) == kvc.KVC_ERR_INVALID_ARG
+    four = (C.c_void_p * 4)(*([FAKE] * 4))
+    assert L.kvc_attend_timed(FAKE, 1 << 20, C.byref(ad), FAKE, wsb, four, 4,
+                              None) == kvc.KVC_ERR_INVALID_ARG
