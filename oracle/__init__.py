@@ -60,13 +60,17 @@ class Desc(C.Structure):
                 ("head_dim", C.c_int32), ("layers", C.c_int32),
                 ("kv_heads", C.c_int32), ("origin", C.c_int32),
                 ("n_requests", C.c_int32), ("sign_seed", C.c_uint64),
-                ("token_lens", C.POINTER(C.c_uint32)), ("lossless", C.c_int32)]
+                ("token_lens", C.POINTER(C.c_uint32)), ("lossless", C.c_int32),
+                ("quant", C.c_int32), ("signs", C.c_int32)]
 
 
 # Lossless pipeline ids of a chunk and encoder modes (reading R17).
 PIPE_ZE, PIPE_XOR_ZE, PIPE_ZE2, PIPE_XOR_ZE2 = range(4)
 LOSSLESS_FIXED, LOSSLESS_SEARCH, LOSSLESS_NONE = range(3)
 BITMAP2 = 256
+# Quantizer (readings R5, R19) and sign diagonals (readings R3, R20).
+QUANT_ASYM, QUANT_SYM = 0, 1
+SIGNS_GLOBAL, SIGNS_PER_VECTOR = 0, 1
 
 
 class Layout(C.Structure):
@@ -102,6 +106,10 @@ def lib():
                 "orc_f32_to_f16_rd": (C.c_uint16, [C.c_float]),
                 "orc_f32_to_f16_ru": (C.c_uint16, [C.c_float]),
                 "orc_quantize_scalar": (C.c_int, [C.c_float, C.c_float, C.c_float, C.c_int]),
+                "orc_quantize_scalar_sym": (C.c_int, [C.c_float, C.c_float, C.c_int]),
+                "orc_quantize_vector_q": (C.c_int, [u16p, C.c_int, C.c_int, C.c_int,
+                                                    C.c_int, u64p, u8p, u8p]),
+                "orc_sign_words_at": (None, [C.c_uint64, C.c_int, C.c_uint64, u64p]),
                 "orc_quantize_vector": (C.c_int, [u16p, C.c_int, C.c_int,
                                                   C.c_int, u64p, u8p, u8p]),
                 "orc_dequantize_vector": (None, [u8p, u8p, C.c_int, C.c_int,
@@ -183,6 +191,13 @@ def sign_words(seed: int, d: int) -> np.ndarray:
     return w[: (d + 63) // 64]
 
 
+def sign_words_at(seed: int, d: int, index: int) -> np.ndarray:
+    """Sign words of the diagonal of (layer, kv, head) index `index` (R20)."""
+    w = np.zeros(4, np.uint64)
+    lib().orc_sign_words_at(seed, d, index, _p(w, C.c_uint64))
+    return w[: (d + 63) // 64]
+
+
 def fwht(y: np.ndarray) -> np.ndarray:
     y = np.ascontiguousarray(y, np.float32).copy()
     lib().orc_fwht(_p(y, C.c_float), y.shape[-1])
@@ -220,7 +235,11 @@ def quantize_scalar(y: float, zf: float, r: float, qmax: int) -> int:
     return lib().orc_quantize_scalar(y, zf, r, qmax)
 
 
-def quantize_vectors(x: np.ndarray, bits: int, group: int, seed: int):
+def quantize_scalar_sym(y: float, r: float, bits: int) -> int:
+    return lib().orc_quantize_scalar_sym(y, r, bits)
+
+
+def quantize_vectors(x: np.ndarray, bits: int, group: int, seed: int, quant: int = QUANT_ASYM):
     """x: uint16 [V, d] bf16 bits -> (status, codes [V, d*b/8], meta [V, d/g*4])."""
     x = np.ascontiguousarray(x, np.uint16)
     V, d = x.shape
@@ -230,9 +249,9 @@ def quantize_vectors(x: np.ndarray, bits: int, group: int, seed: int):
     meta = np.zeros((V, d // group * 4), np.uint8)
     status = OK
     for v in range(V):
-        st = lib().orc_quantize_vector(_p(x[v], C.c_uint16), d, bits, group,
-                                       _p(sw, C.c_uint64), _p(codes[v], C.c_uint8),
-                                       _p(meta[v], C.c_uint8))
+        st = lib().orc_quantize_vector_q(_p(x[v], C.c_uint16), d, bits, group, quant,
+                                         _p(sw, C.c_uint64), _p(codes[v], C.c_uint8),
+                                         _p(meta[v], C.c_uint8))
         if st != OK and status == OK:
             status = st
     return status, codes, meta
@@ -319,11 +338,12 @@ class StreamDesc:
     """Shape and parameters of one stream (the oracle's own description)."""
 
     def __init__(self, bits, group, head_dim, layers, kv_heads, token_lens,
-                 sign_seed=0, origin=0, lossless=LOSSLESS_FIXED):
+                 sign_seed=0, origin=0, lossless=LOSSLESS_FIXED, quant=QUANT_ASYM,
+                 signs=SIGNS_GLOBAL):
         self.token_lens = np.ascontiguousarray(np.asarray(token_lens, np.uint32))
         self.c = Desc(bits, group, head_dim, layers, kv_heads, origin,
                       len(self.token_lens), sign_seed,
-                      _p(self.token_lens, C.c_uint32), lossless)
+                      _p(self.token_lens, C.c_uint32), lossless, quant, signs)
 
     @property
     def head_dim(self):

@@ -50,6 +50,19 @@ void orc_sign_words(uint64_t seed, int d, uint64_t *words) {
   for (i = 0; i < (d + 63) / 64; i++) words[i] = orc_splitmix64_next(&state);
 }
 
+/* Reading R20 (per-(layer, kv, head) sign diagonals, the FP4Quant abstract's
+ * variant of the randomized transform): vector index i (= its position in
+ * the order [layer][kv][head]) takes the SplitMix64 outputs number
+ * i*W .. i*W + W - 1 (W = ceil(d / 64)) of the same generator from state =
+ * sign_seed. Output n comes from state seed + (n + 1) * gamma, so the
+ * generator is advanced by i*W increments first; index 0 is reading R3. */
+void orc_sign_words_at(uint64_t seed, int d, uint64_t index, uint64_t *words) {
+  const uint64_t W = (uint64_t)((d + 63) / 64);
+  uint64_t state = seed + index * W * 0x9E3779B97F4A7C15ull;
+  uint64_t i;
+  for (i = 0; i < W; i++) words[i] = orc_splitmix64_next(&state);
+}
+
 static int sign_bit(const uint64_t *words, int c) {
   return (int)((words[c / 64] >> (c % 64)) & 1u);
 }
@@ -160,7 +173,8 @@ static int f16_is_inf(uint16_t h) { return (h & 0x7FFFu) == 0x7C00u; }
 /* ========================================================================== */
 /* Code packing. Reading R6: codes of one vector in channel order, LSB first: */
 /* 4-bit: byte j = q[2j] | q[2j+1] << 4;                                      */
-/* 2-bit: byte j = q[4j] | q[4j+1] << 2 | q[4j+2] << 4 | q[4j+3] << 6.        */
+/* 2-bit: byte j = q[4j] | q[4j+1] << 2 | q[4j+2] << 4 | q[4j+3] << 6;        */
+/* 8-bit (reading R21): byte j = q[j].                                        */
 /* ========================================================================== */
 void orc_pack_codes(const uint8_t *q, int d, int bits, uint8_t *packed) {
   int per = 8 / bits, j, i;
@@ -192,6 +206,18 @@ int orc_quantize_scalar(float y, float zf, float r, int qmax) {
   return (int)n;
 }
 
+/* One code of reading R19 (symmetric absmax): p = fl(y * r) (one fp32
+ * rounding), then the nearest integer to p, ties to even, clamped to
+ * [-qh, qh], qh = 2^(b-1) - 1. The stored code is that integer + 2^(b-1). */
+int orc_quantize_scalar_sym(float y, float r, int bits) {
+  const int qh = (1 << (bits - 1)) - 1;
+  float p = y * r;
+  double n = nearbyint((double)p);
+  if (n < (double)-qh) n = (double)-qh;
+  if (n > (double)qh) n = (double)qh;
+  return (int)n + (1 << (bits - 1));
+}
+
 /* ========================================================================== */
 /* Quantization of one vector ([P2] Methodology: distribution transformation  */
 /* then low-bit quantization; [P3]: only this step loses information).        */
@@ -210,6 +236,21 @@ int orc_quantize_scalar(float y, float zf, float r, int qmax) {
 int orc_quantize_vector(const uint16_t *x, int d, int bits, int g,
                         const uint64_t *sign_words, uint8_t *codes,
                         uint8_t *meta) {
+  return orc_quantize_vector_q(x, d, bits, g, ORC_QUANT_ASYM, sign_words, codes, meta);
+}
+
+/* Reading R19 (symmetric absmax, one of the quantizer variants of the
+ * FP4Quant abstract), in the meta format of reading R5 so that the decoder
+ * of reading R9 is unchanged:
+ *   a = max |y| over the group (+0);  s32 = a / (2^(b-1) - 1);
+ *   s_h = RU16(s32 * 2^-k), sf = f32(s_h) * 2^k;  r = 0 if s_h == 0 else 1/sf;
+ *   code = clamp(nearest integer to fl(y * r), ties to even, -qh, qh) + 2^(b-1);
+ *   z_h = fp16 of -2^(b-1) * f32(s_h) (exact: a power-of-two multiple; +0
+ *   when s_h is 0), so zf + code * sf = (code - 2^(b-1)) * sf exactly.
+ * A non-finite y gives NONFINITE, an infinite s_h or z_h RANGE (R8). */
+int orc_quantize_vector_q(const uint16_t *x, int d, int bits, int g, int quant,
+                          const uint64_t *sign_words, uint8_t *codes,
+                          uint8_t *meta) {
   float y[ORC_MAX_D];
   uint8_t q[ORC_MAX_D];
   int k = orc_meta_shift(d);
@@ -242,17 +283,30 @@ int orc_quantize_vector(const uint16_t *x, int d, int bits, int g,
     }
     mn = mn + 0.0f;
     mx = mx + 0.0f;
-    zh = orc_f32_to_f16_rd(mn * down);
-    zf = orc_f16_to_f32(zh) * up;
-    s32 = (mx - zf) / (float)qmax;
-    sh = orc_f32_to_f16_ru(s32 * down);
+    if (quant == ORC_QUANT_SYM) {
+      const float a = fabsf(mn) > fabsf(mx) ? fabsf(mn) : fabsf(mx);
+      const int qh = (1 << (bits - 1)) - 1;
+      s32 = a / (float)qh;
+      sh = orc_f32_to_f16_ru(s32 * down);
+      zh = (sh & 0x7FFFu) == 0 ? 0
+                               : f32_to_f16_directed(-ldexpf(orc_f16_to_f32(sh), bits - 1), 1);
+    } else {
+      zh = orc_f32_to_f16_rd(mn * down);
+      zf = orc_f16_to_f32(zh) * up;
+      s32 = (mx - zf) / (float)qmax;
+      sh = orc_f32_to_f16_ru(s32 * down);
+    }
     sf = orc_f16_to_f32(sh) * up;
+    zf = orc_f16_to_f32(zh) * up;
     if (f16_is_inf(zh) || f16_is_inf(sh)) {
       if (status == ORC_OK) status = ORC_ERR_RANGE;
       for (c = 0; c < g; c++) q[j * g + c] = 0;
     } else {
       r = ((sh & 0x7FFFu) == 0) ? 0.0f : 1.0f / sf;
-      for (c = 0; c < g; c++) q[j * g + c] = (uint8_t)orc_quantize_scalar(yg[c], zf, r, qmax);
+      for (c = 0; c < g; c++)
+        q[j * g + c] = (uint8_t)(quant == ORC_QUANT_SYM
+                                     ? orc_quantize_scalar_sym(yg[c], r, bits)
+                                     : orc_quantize_scalar(yg[c], zf, r, qmax));
     }
     meta[4 * j + 0] = (uint8_t)(sh & 0xFF);
     meta[4 * j + 1] = (uint8_t)(sh >> 8);
@@ -619,7 +673,10 @@ static uint64_t round16(uint64_t x) { return (x + 15u) & ~(uint64_t)15u; }
 int orc_check_desc(const orc_desc *d) {
   int r;
   if (!d) return ORC_ERR_INVALID_ARG;
-  if (d->bits != 2 && d->bits != 4) return ORC_ERR_UNSUPPORTED;
+  if (d->bits != 2 && d->bits != 4 && d->bits != 8) return ORC_ERR_UNSUPPORTED;
+  if (d->quant != ORC_QUANT_ASYM && d->quant != ORC_QUANT_SYM) return ORC_ERR_UNSUPPORTED;
+  if (d->signs != ORC_SIGNS_GLOBAL && d->signs != ORC_SIGNS_PER_VECTOR)
+    return ORC_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256)
     return ORC_ERR_UNSUPPORTED;
   if (d->group != 32 && d->group != 64 && d->group != 128)
@@ -701,6 +758,13 @@ static uint64_t get64(const uint8_t *p) {
   return (uint64_t)get32(p) | ((uint64_t)get32(p + 4) << 32);
 }
 
+/* The (layer, kv, head) index of stream vector v (order [layer][kv][head]
+ * [request][token], requests concatenated): v / T, T the total tokens. */
+static uint64_t vector_index(const orc_desc *d, const orc_layout *lay, uint64_t v) {
+  uint64_t T = lay->V / (2u * (uint64_t)d->layers * (uint64_t)d->kv_heads);
+  return v / T;
+}
+
 /* Segment s's chunks from its vectors, for a layout computed once by the
  * caller (orc_encode_segment and the compressor below). */
 static int encode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t s,
@@ -719,9 +783,11 @@ static int encode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t 
   codes = (uint8_t *)malloc((size_t)(nv * lay->code_bytes));
   meta = (uint8_t *)malloc((size_t)(nv * lay->meta_bytes));
   for (v = 0; v < nv; v++) {
-    vst = orc_quantize_vector(vectors + v * d->head_dim, d->head_dim, d->bits,
-                              d->group, sw, codes + v * lay->code_bytes,
-                              meta + v * lay->meta_bytes);
+    if (d->signs == ORC_SIGNS_PER_VECTOR)
+      orc_sign_words_at(d->sign_seed, d->head_dim, vector_index(d, lay, v0 + v), sw);
+    vst = orc_quantize_vector_q(vectors + v * d->head_dim, d->head_dim, d->bits,
+                                d->group, d->quant, sw, codes + v * lay->code_bytes,
+                                meta + v * lay->meta_bytes);
     if (vst != ORC_OK && st == ORC_OK) st = vst;
   }
   c0 = s * lay->code_per_seg;
@@ -787,6 +853,8 @@ static int decode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t 
                                pipes[i], (int)(lay->meta_bytes / 4), meta);
   if (st == ORC_OK)
     for (v = 0; v < nv; v++) {
+      if (d->signs == ORC_SIGNS_PER_VECTOR)
+        orc_sign_words_at(d->sign_seed, d->head_dim, vector_index(d, lay, v0 + v), sw);
       if (vals)
         orc_dequantize_vector_f64(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
                                   d->head_dim, d->bits, d->group, sw, vals + v * d->head_dim);
@@ -935,7 +1003,9 @@ int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
   out[8] = (uint8_t)d->bits;
   out[9] = (uint8_t)orc_meta_shift(d->head_dim);
   out[10] = (uint8_t)d->origin;
-  out[11] = 0;
+  /* header flags: bit 0 set below; bits 1..2 the quantizer (R19), bit 3
+     the sign diagonals (R20) */
+  out[11] = (uint8_t)((d->quant << 1) | (d->signs << 3));
   put32(out + 12, (uint32_t)d->group);
   put32(out + 16, (uint32_t)d->layers);
   put32(out + 20, 2);
@@ -1010,7 +1080,7 @@ int orc_compress_mt(const orc_desc *d, const uint16_t *vectors, uint8_t *out,
     uint64_t nv = lay.V - i * lay.vec_per_code;
     if (nv > lay.vec_per_code) nv = lay.vec_per_code;
     if (all_sizes[orc_code_chunk_index(&lay, i)] != nv * lay.code_bytes) {
-      out[11] = 1;
+      out[11] |= 1;
       break;
     }
   }
@@ -1115,10 +1185,13 @@ static int decompress_impl(const uint8_t *stream, uint64_t stream_bytes,
       return ORC_ERR_CORRUPT;
     expect_off = off + round16(sz);
   }
-  /* header flags: only bit 0, which must be set if a code chunk uses
-     zero-byte elimination */
-  if (stream[11] > 1) return ORC_ERR_CORRUPT;
-  for (s = 0; s < lay.n_code && !stream[11]; s++) {
+  /* header flags: bit 0 must be set if a code chunk uses zero-byte
+     elimination; bits 1..3 name the quantizer and the sign diagonals, which
+     must be the expected ones; the other bits are zero */
+  if ((stream[11] & 0xF0u) || ((stream[11] >> 1) & 3u) != (unsigned)expect->quant ||
+      ((stream[11] >> 3) & 1u) != (unsigned)expect->signs)
+    return ORC_ERR_CORRUPT;
+  for (s = 0; s < lay.n_code && !(stream[11] & 1u); s++) {
     uint64_t nv = lay.V - s * lay.vec_per_code;
     if (nv > lay.vec_per_code) nv = lay.vec_per_code;
     if ((get64(stream + ORC_HEADER + 8 * orc_code_chunk_index(&lay, s)) & 0xFFFFu) !=

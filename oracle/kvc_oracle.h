@@ -48,10 +48,15 @@ enum {
 #define ORC_HEADER 64        /* stream header bytes                       */
 #define ORC_MAGIC 0x3143564Bu /* "KVC1" little-endian                    */
 #define ORC_MAX_D 256
+#define ORC_QUANT_ASYM 0      /* reading R5: min/max, zero and scale        */
+#define ORC_QUANT_SYM 1       /* reading R19: symmetric absmax              */
+#define ORC_SIGNS_GLOBAL 0    /* reading R3: one diagonal for the tensor    */
+#define ORC_SIGNS_PER_VECTOR 1 /* reading R20: one per (layer, kv, head)   */
 
 /* ---- scalar building blocks (each pinned by its own test) ---------------- */
 uint64_t orc_splitmix64_next(uint64_t *state);
 void orc_sign_words(uint64_t seed, int d, uint64_t *words);
+void orc_sign_words_at(uint64_t seed, int d, uint64_t index, uint64_t *words);
 void orc_fwht(float *y, int d);
 int orc_meta_shift(int d);
 float orc_bf16_to_f32(uint16_t b);
@@ -62,6 +67,10 @@ uint16_t orc_f32_to_f16_ru(float x);
 
 /* ---- one vector ----------------------------------------------------------- */
 int orc_quantize_scalar(float y, float zf, float r, int qmax);
+int orc_quantize_scalar_sym(float y, float r, int bits);
+int orc_quantize_vector_q(const uint16_t *x, int d, int bits, int g, int quant,
+                          const uint64_t *sign_words, uint8_t *codes,
+                          uint8_t *meta);
 int orc_quantize_vector(const uint16_t *x, int d, int bits, int g,
                         const uint64_t *sign_words, uint8_t *codes,
                         uint8_t *meta);
@@ -120,6 +129,8 @@ typedef struct {
   uint64_t sign_seed;
   const uint32_t *token_lens; /* [n_requests] tokens per request          */
   int32_t lossless;           /* ORC_LOSSLESS_* (encoder only)            */
+  int32_t quant;              /* ORC_QUANT_* (header flags bits 1..2)     */
+  int32_t signs;              /* ORC_SIGNS_* (header flags bit 3)         */
 } orc_desc;
 
 typedef struct {
