@@ -961,8 +961,8 @@ static void enc_one_segment(void *arg, uint64_t s) {
   const orc_layout *lay = j->lay;
   uint64_t vm = (uint64_t)lay->vec_per_code * lay->code_per_seg;
   uint8_t *seg = (uint8_t *)malloc((size_t)(lay->code_per_seg + 1) * ORC_CHUNK);
-  uint32_t sizes[17], n, k, pos = 0;
-  uint8_t pipes[17];
+  uint32_t sizes[ORC_MAX_SEG + 1], n, k, pos = 0;
+  uint8_t pipes[ORC_MAX_SEG + 1];
   j->seg_status[s] = encode_segment_in(j->d, lay, s, j->vectors + s * vm * j->d->head_dim,
                                        seg, sizes, pipes, &n);
   for (k = 0; k < n; k++) {
@@ -1111,8 +1111,8 @@ static void dec_one_segment(void *arg, uint64_t s) {
   uint64_t c0 = s * lay->code_per_seg;
   uint64_t c1 = c0 + lay->code_per_seg < lay->n_code ? c0 + lay->code_per_seg : lay->n_code;
   uint64_t i, k = 0;
-  uint32_t pos = 0, sizes[17];
-  uint8_t pipes[17];
+  uint32_t pos = 0, sizes[ORC_MAX_SEG + 1];
+  uint8_t pipes[ORC_MAX_SEG + 1];
   uint8_t *seg = (uint8_t *)malloc((size_t)(lay->code_per_seg + 1) * ORC_CHUNK);
   for (i = c0; i <= c1; i++, k++) { /* code chunks c0..c1-1, then the meta chunk */
     uint64_t idx = i < c1 ? orc_code_chunk_index(lay, i) : orc_meta_chunk_index(lay, s);

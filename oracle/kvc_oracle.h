@@ -48,6 +48,7 @@ enum {
 #define ORC_HEADER 64        /* stream header bytes                       */
 #define ORC_MAGIC 0x3143564Bu /* "KVC1" little-endian                    */
 #define ORC_MAX_D 256
+#define ORC_MAX_SEG 32       /* code chunks per segment: g * b / 32 <= 128 * 8 / 32 */
 #define ORC_QUANT_ASYM 0      /* reading R5: min/max, zero and scale        */
 #define ORC_QUANT_SYM 1       /* reading R19: symmetric absmax              */
 #define ORC_SIGNS_GLOBAL 0    /* reading R3: one diagonal for the tensor    */

@@ -300,3 +300,25 @@ def test_eight_bit_stream_roundtrip_error_bound():
     # bf16 decode: the unrounded decode rounded to nearest even
     back = synth.bf16_bits(torch.from_numpy(xh).to(torch.bfloat16))
     assert (back == xb).mean() > 0.999
+
+
+def test_eight_bit_group_128_full_segment():
+    """8-bit codes with group 128: a meta chunk covers 32 code chunks (the
+    largest segment); 8400 vectors (1 layer x 2 x 2 heads x 2100 tokens)
+    fill two segments and start a third. Round trip on the grid, in one and
+    in several threads."""
+    d, g = 128, 128
+    desc, s, x, codes, meta = _raw_stream(8, g, 1, 2, [2100])
+    lay = desc.layout()
+    assert lay.code_per_seg == 32 and lay.n_code == 66 and lay.n_seg == 3
+    st, xh = oracle.decode_values(s, desc)
+    assert st == oracle.OK
+    grid = _grid_values(codes, meta, d, 8, g)
+    Hm = sylvester(d)
+    D = signs_of(oracle.sign_words(11, d), d)
+    for v in (0, 1, 4095, 4096, 8191, 8192, 8399):
+        np.testing.assert_allclose(Hm @ (D * xh[v]), grid[v], rtol=0,
+                                   atol=1e-9 * abs(grid[v]).max())
+    st2, s2 = oracle.compress(desc, x, threads=3)
+    assert st2 == oracle.OK and np.array_equal(s, s2)
+    assert (oracle.decompress(s, desc, threads=3)[1] == oracle.decompress(s, desc)[1]).all()
