@@ -83,21 +83,43 @@ typedef enum {
  * kvc_compress. A decoder handles every mode. */
 enum { KVC_LOSSLESS_FIXED = 0, KVC_LOSSLESS_SEARCH = 1, KVC_LOSSLESS_NONE = 2 };
 
+/* Quantizer variants and sign diagonals (the FP4Quant abstract on the first
+ * page lists quantizer variants of the transform + low-bit step; these are
+ * the ones with an exact oracle):
+ *   KVC_QUANT_ASYM  asymmetric min/max per group: zero = RD16(min), scale =
+ *                   RU16((max - zero) / (2^b - 1)), code = RNE((y - zero) / scale)
+ *   KVC_QUANT_SYM   symmetric absmax per group: scale = RU16(max|y| /
+ *                   (2^(b-1) - 1)), code = RNE(y / scale) + 2^(b-1) in
+ *                   [1, 2^b - 1]; the stored zero is -2^(b-1) * scale, so
+ *                   every decoder reads both alike (zero + code * scale)
+ *   KVC_SIGNS_GLOBAL      one +-1 diagonal for every vector
+ *   KVC_SIGNS_PER_VECTOR  one per (layer, kv, head): vector index i (its
+ *                   position in the order [layer][kv][head]) takes the
+ *                   SplitMix64 outputs i*W .. i*W + W - 1 (W = head_dim / 64)
+ * The stream's header flags record both (bits 1..2 and 3); a decoder needs
+ * no parameter for them. */
+enum { KVC_QUANT_ASYM = 0, KVC_QUANT_SYM = 1 };
+enum { KVC_SIGNS_GLOBAL = 0, KVC_SIGNS_PER_VECTOR = 1 };
+
 /* Quantization and lossless parameters.
- *  bits       2 or 4 bits per code.
+ *  bits       2, 4 or 8 bits per code.
  *  group_size 32, 64 or 128 consecutive channels of the transformed vector
  *             share one fp16 zero and scale; must divide head_dim.
  *  sign_seed  seeds the +-1 diagonal: channel c is negated iff bit (c mod 64)
  *             of SplitMix64 output number floor(c/64), counted from state =
- *             sign_seed, is 1.
- *  lossless   KVC_LOSSLESS_* (encoder only); other values are refused with
- *             KVC_ERR_UNSUPPORTED.
- *  reserved   must be 0. */
+ *             sign_seed, is 1 (per-vector diagonals: see above).
+ *  lossless   KVC_LOSSLESS_* (encoder only).
+ *  quant      KVC_QUANT_*.
+ *  signs      KVC_SIGNS_* (kvc_compress_unfused: KVC_SIGNS_GLOBAL only).
+ *  reserved   must be 0.
+ * Other values are refused with KVC_ERR_UNSUPPORTED. */
 typedef struct {
   int32_t bits;
   int32_t group_size;
   uint64_t sign_seed;
   int32_t lossless;
+  int32_t quant;
+  int32_t signs;
   int32_t reserved;
 } kvc_params;
 

@@ -41,7 +41,13 @@ class KvcError(RuntimeError):
 
 class kvc_params(C.Structure):
     _fields_ = [("bits", C.c_int32), ("group_size", C.c_int32), ("sign_seed", C.c_uint64),
-                ("lossless", C.c_int32), ("reserved", C.c_int32)]
+                ("lossless", C.c_int32), ("quant", C.c_int32), ("signs", C.c_int32),
+                ("reserved", C.c_int32)]
+
+
+# Quantizers (kvc_params.quant) and sign diagonals (kvc_params.signs).
+KVC_QUANT_ASYM, KVC_QUANT_SYM = 0, 1
+KVC_SIGNS_GLOBAL, KVC_SIGNS_PER_VECTOR = 0, 1
 
 
 # Lossless-stage modes (kvc_params.lossless) and pipeline ids of a chunk.
@@ -228,9 +234,9 @@ def kvc_status_string(status: int) -> str:
 
 
 # ------------------------------------------------------- descriptor helpers --
-def params(bits: int, group: int, sign_seed: int = 0,
-           lossless: int = KVC_LOSSLESS_FIXED) -> kvc_params:
-    return kvc_params(bits, group, sign_seed, lossless, 0)
+def params(bits: int, group: int, sign_seed: int = 0, lossless: int = KVC_LOSSLESS_FIXED,
+           quant: int = KVC_QUANT_ASYM, signs: int = KVC_SIGNS_GLOBAL) -> kvc_params:
+    return kvc_params(bits, group, sign_seed, lossless, quant, signs, 0)
 
 
 def dense_desc(kv) -> kvc_kv_desc:
@@ -286,8 +292,9 @@ class Codec:
     compute step runs in libkvc's kernels. Errors raise KvcError."""
 
     def __init__(self, bits: int = 4, group: int = 128, sign_seed: int = 0,
-                 lossless: int = KVC_LOSSLESS_FIXED):
-        self.params = params(bits, group, sign_seed, lossless)
+                 lossless: int = KVC_LOSSLESS_FIXED, quant: int = KVC_QUANT_ASYM,
+                 signs: int = KVC_SIGNS_GLOBAL):
+        self.params = params(bits, group, sign_seed, lossless, quant, signs)
 
     def buffers(self, desc: kvc_kv_desc, device="cuda"):
         import torch

@@ -95,7 +95,10 @@ kvc_status describe(const kvc_kv_desc *kv, const kvc_params *p, Shape &s) {
   if (s.V >= (uint64_t(1) << 31)) return KVC_ERR_UNSUPPORTED;
   if (s.V > 0 && (!kv->data || !aligned16(kv->data))) return KVC_ERR_INVALID_ARG;
   if (!p) return KVC_OK;
-  if (p->bits != 2 && p->bits != 4) return KVC_ERR_UNSUPPORTED;
+  if (p->bits != 2 && p->bits != 4 && p->bits != 8) return KVC_ERR_UNSUPPORTED;
+  if ((p->quant != KVC_QUANT_ASYM && p->quant != KVC_QUANT_SYM) ||
+      (p->signs != KVC_SIGNS_GLOBAL && p->signs != KVC_SIGNS_PER_VECTOR))
+    return KVC_ERR_UNSUPPORTED;
   if (p->group_size != 32 && p->group_size != 64 && p->group_size != 128)
     return KVC_ERR_UNSUPPORTED;
   if (p->group_size > s.D) return KVC_ERR_UNSUPPORTED;
@@ -290,6 +293,8 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   if (!params) return KVC_ERR_INVALID_ARG;
   kvc_status st = describe(kv, params, s);
   if (st != KVC_OK) return st;
+  // the unfused baseline's transform kernel applies the global diagonal only
+  if (unfused && params->signs != KVC_SIGNS_GLOBAL) return KVC_ERR_UNSUPPORTED;
   if (!out || !aligned16(out) || !workspace || !aligned16(workspace)) return KVC_ERR_INVALID_ARG;
   const uint64_t need = unfused ? round256(s.ws_bytes) + s.V * uint64_t(s.D) * 4 : s.ws_bytes;
   if (out_capacity < s.max_bytes || workspace_bytes < need) return KVC_ERR_CAPACITY;
@@ -314,6 +319,10 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   a.ymid = unfused ? reinterpret_cast<float *>(ws + round256(s.ws_bytes)) : nullptr;
   a.one = 1.0f;
   a.mode = uint32_t(params->lossless);
+  a.sym = params->quant == KVC_QUANT_SYM ? 1u : 0u;
+  a.vec_signs = params->signs == KVC_SIGNS_PER_VECTOR ? 1u : 0u;
+  a.seed = params->sign_seed;
+  a.tdiv = make_fastdiv(uint32_t(s.T ? s.T : 1));
   sign_masks(params->sign_seed, s.D, a.sign_mask);
 
   FinArgs f{};
@@ -352,6 +361,8 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   f.tokens = s.T;
   f.seed = params->sign_seed;
   f.mode = uint32_t(params->lossless);
+  f.quant = uint32_t(params->quant);
+  f.signs = uint32_t(params->signs);
   f.wait_ns = wait_ns;
   f.ticket_skip = ticket_skip;
 
@@ -467,6 +478,7 @@ kvc_status kvc_decompress(const void *in, size_t in_bytes, const kvc_kv_desc *ou
   a.tokens = s.T;
   a.V = uint32_t(s.V);
   a.paged_receiver = out->kind == KVC_PAGED ? 1u : 0u;
+  a.tdiv = make_fastdiv(uint32_t(s.T ? s.T : 1));
   a.ws_meta = static_cast<uint8_t *>(workspace) + kWsCtl;
   a.ws_meta_chunks = uint32_t(max_meta_chunks(s));
   if (clear_words(workspace, kWsCtl, sms, cs) != cudaSuccess) return KVC_ERR_CUDA;
@@ -518,7 +530,8 @@ kvc_status attn_shape(const kvc_attn_desc *at, AttnShape &r) {
   kv.stride_head = T * at->head_dim;
   kv.stride_kv = kv.stride_head * at->kv_heads;
   kv.stride_layer = kv.stride_kv * 2;
-  kvc_params p{at->bits, at->group_size, 0, KVC_LOSSLESS_FIXED, 0};
+  kvc_params p{at->bits, at->group_size, 0, KVC_LOSSLESS_FIXED, KVC_QUANT_ASYM, KVC_SIGNS_GLOBAL,
+               0};
   const kvc_status st = describe(&kv, &p, r.s);
   if (st != KVC_OK) return st;
   r.s.n_req = uint32_t(at->n_requests);

@@ -38,7 +38,10 @@ cudaError_t launch_attend(const AttnArgs &a, const DecArgs &d, int sms, cudaStre
   e = launch_after(mk, mgrid, kMetaThreads, meta_smem_bytes(), st, d);
   if (e != cudaSuccess) return e;
   const int units = int(a.layers * a.n_req * a.kv_heads);
-  if (a.bits == 4 && a.group == 128) e = launch_att_q<4, 128>(a, units, st);
+  if (a.bits == 8 && a.group == 128) e = launch_att_q<8, 128>(a, units, st);
+  else if (a.bits == 8 && a.group == 64) e = launch_att_q<8, 64>(a, units, st);
+  else if (a.bits == 8 && a.group == 32) e = launch_att_q<8, 32>(a, units, st);
+  else if (a.bits == 4 && a.group == 128) e = launch_att_q<4, 128>(a, units, st);
   else if (a.bits == 4 && a.group == 64) e = launch_att_q<4, 64>(a, units, st);
   else if (a.bits == 4 && a.group == 32) e = launch_att_q<4, 32>(a, units, st);
   else if (a.bits == 2 && a.group == 128) e = launch_att_q<2, 128>(a, units, st);

@@ -28,7 +28,9 @@ constexpr int kAttMaxG = 8;    // query heads per kv head
 
 // Header checks shared by the attention kernels: the stream describes this
 // cache with the stated bits and group, and stores every code chunk raw (the
-// code region is then the plain array of per-vector codes).
+// code region is then the plain array of per-vector codes). Flags: bit 0
+// (eliminated code chunks) clear; either quantizer (both decode as zero +
+// code * scale); either sign mode (bit 3: per-vector diagonals).
 template <int D>
 __device__ __forceinline__ bool attn_header_ok(const AttnArgs &a, uint64_t &base, uint32_t &n_code,
                                                uint64_t &seed) {
@@ -44,7 +46,7 @@ __device__ __forceinline__ bool attn_header_ok(const AttnArgs &a, uint64_t &base
   seed = ld_u64(h + 40);
   return ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 &&
          (ld_u32(h + 4) >> 16) == kHeader && h[8] == a.bits && h[9] == kLog2D / 2 &&
-         h[11] == 0 && ld_u32(h + 12) == a.group && ld_u32(h + 16) == a.layers &&
+         (h[11] & 0xF5u) == 0 && ld_u32(h + 12) == a.group && ld_u32(h + 16) == a.layers &&
          ld_u32(h + 20) == 2 && ld_u32(h + 24) == a.kv_heads && ld_u32(h + 28) == D &&
          ld_u64(h + 32) == a.tokens && n_req == a.n_req && n_chunks == nc + nm &&
          ld_u64(h + 56) <= a.in_bytes && base + uint64_t(a.V) * cb <= ld_u64(h + 56);
@@ -140,8 +142,15 @@ __global__ void __launch_bounds__(kAttThreads) attend_kernel(const __grid_consta
     }
     sm.ok = ok;
     sm.base = base;
-    if (!ok) set_status(a.status, KVC_ERR_CORRUPT);
-    else sign_masks(seed, D, sm.mask);
+    if (!ok) {
+      set_status(a.status, KVC_ERR_CORRUPT);
+    } else if (in[11] & 8u) {  // the keys' own diagonal: index (l, 0, h)
+      uint32_t S[D / 32];
+      vec_sign_words<D>(seed, (l * 2 + 0) * H + h, S);
+      for (int k = 0; k < D / 2; ++k) sm.mask[k] = pair_mask<D>(S, 2 * k);
+    } else {
+      sign_masks(seed, D, sm.mask);
+    }
   }
   __syncthreads();
   if (!sm.ok) return;
@@ -259,7 +268,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_kernel(const __grid_consta
 
   // ---- values: lane = (token of the step, 8 consecutive channels, which
   // lie in one group and one code word)
-  constexpr int CPL = 8;              // channels per lane
+  constexpr int CPL = BITS == 8 ? 4 : 8;  // channels per lane (one code word at most)
   constexpr int LPT = D / CPL;        // lanes per token
   constexpr int TPS = 32 / LPT;       // tokens per step
   const int wi = lane % LPT, tp = lane / LPT;
@@ -360,7 +369,9 @@ __global__ void __launch_bounds__(kCombWarps * 32) attend_combine_kernel(const _
   }
   warp_fwht128(y, lane);
   // sign of channel c: bit c % 64 of the (c / 64 + 1)-th SplitMix64 output
+  // of the diagonal (the global one, or the values' own: index (l, 1, h))
   uint64_t st = ld_u64(a.in + 40);
+  if (a.in[11] & 8u) st += uint64_t((l * 2 + 1) * H + h) * 2u * 0x9E3779B97F4A7C15ull;
   const uint64_t w0 = splitmix64(st), w1 = splitmix64(st);
   const float f = 1.f / (L * float(D));
 #pragma unroll

@@ -35,7 +35,7 @@ struct DecCtl {
   uint64_t cbar[kDecWarps][2];  // per-warp code + meta blocks loaded (two buffers)
   uint32_t red[kDecThreads / 32];
   uint32_t hdr_ok;
-  uint32_t bits, group, n_req_stream, n_chunks, code_elim;
+  uint32_t bits, group, n_req_stream, n_chunks, code_elim, vec_signs;
   uint64_t data_base, stream_bytes, seed;
   alignas(16) uint32_t mask[128];  // read as uint4
 };
@@ -45,7 +45,9 @@ struct DecCtl {
 template <int D>
 struct DecSmem {
   static constexpr size_t WBUF = size_t(D / 64) * 4096;    // 32 rows, 128-byte swizzled halves
-  static constexpr size_t BLK = 32 * size_t(D) / 2;       // widest code block (4-bit)
+  // code block of 32 vectors at up to 4 bits (an 8-bit block fills both of a
+  // warp's buffers and is loaded single-buffered)
+  static constexpr size_t BLK = 32 * size_t(D) / 2;
   static constexpr size_t MBLK = 32 * (size_t(D) / 32) * 4;  // widest meta block (group 32)
   static constexpr size_t rows = 0;
   static constexpr size_t code = rows + kDecWarps * WBUF;
@@ -66,7 +68,7 @@ __device__ __forceinline__ uint64_t ld_u64(const uint8_t *p) {
 
 // D1: the header (reading R12) against the receiver's description.
 struct StreamHdr {
-  uint32_t ok, bits, group, n_req, n_chunks, code_elim;
+  uint32_t ok, bits, group, n_req, n_chunks, code_elim, vec_signs;
   uint64_t data_base, stream_bytes, seed;
 };
 template <int D>
@@ -76,8 +78,12 @@ __device__ __forceinline__ StreamHdr parse_header(const DecArgs &a) {
   const uint8_t *h = a.in;
   if (a.in_bytes < kHeader) return r;
   const uint32_t bits = h[8], k = h[9], group = ld_u32(h + 12);
-  bool ok = ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 && h[11] <= 1 &&
-            (ld_u32(h + 4) >> 16) == kHeader && (bits == 2 || bits == 4) && k == kLog2D / 2 &&
+  // flags: bit 0 code chunks eliminated, bits 1..2 the quantizer (0 or 1;
+  // both decode alike), bit 3 per-vector sign diagonals, the rest zero
+  const uint32_t flags = h[11];
+  bool ok = ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 && (flags & 0xF4u) == 0 &&
+            (ld_u32(h + 4) >> 16) == kHeader && (bits == 2 || bits == 4 || bits == 8) &&
+            k == kLog2D / 2 &&
             (group == 32 || group == 64 || group == 128) && group <= D &&
             ld_u32(h + 16) == a.layers && ld_u32(h + 20) == 2 && ld_u32(h + 24) == a.kv_heads &&
             ld_u32(h + 28) == a.head_dim && ld_u64(h + 32) == a.tokens;
@@ -98,7 +104,8 @@ __device__ __forceinline__ StreamHdr parse_header(const DecArgs &a) {
   r.data_base = base;
   r.stream_bytes = stream_bytes;
   r.seed = ld_u64(h + 40);
-  r.code_elim = h[11];
+  r.code_elim = flags & 1u;
+  r.vec_signs = (flags >> 3) & 1u;
   return r;
 }
 
@@ -115,8 +122,9 @@ struct Dec : Cfg<D, BITS, G> {
   // rounding. q*sf is exact (q < 16 times an fp16 value needs at most 15
   // significant bits), so one fused multiply-add equals fl(zf + fl(q*sf)).
   // The vector is held as pairs (c, c + d/2) like the encoder's.
+  template <class SG>
   static __device__ __forceinline__ void vector(const uint8_t *codes, const uint8_t *meta,
-                                                const uint32_t *mask, uint32_t (&out)[D / 2]) {
+                                                const SG &sg, uint32_t (&out)[D / 2]) {
     float zf[C::NG], sf[C::NG];
     const float up = float(1 << C::K) / float(D);
 #pragma unroll
@@ -154,7 +162,8 @@ struct Dec : Cfg<D, BITS, G> {
       }
       auto code_float = [&](const uint32_t (&w)[PW], int c) -> float {
         const int W = c / per_word, r = c % per_word, k = r / per_byte, e = r % per_byte;
-        const uint32_t part = (w[W] >> (e * BITS)) & (BITS == 4 ? 0x0F0F0F0Fu : 0x03030303u);
+        const uint32_t part =
+            (w[W] >> (e * BITS)) & (BITS == 8 ? 0xFFFFFFFFu : BITS == 4 ? 0x0F0F0F0Fu : 0x03030303u);
         return __uint_as_float(__byte_perm(part, kMagicBits, 0x7640 | k));
       };
 #pragma unroll
@@ -168,7 +177,7 @@ struct Dec : Cfg<D, BITS, G> {
     fwht_pairs<D>(y);
 #pragma unroll
     for (int q = 0; q < D / 8; ++q) {
-      const uint4 m4 = reinterpret_cast<const uint4 *>(mask)[q];
+      const uint4 m4 = sg.quad(q);
       const uint32_t m[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -179,6 +188,23 @@ struct Dec : Cfg<D, BITS, G> {
     }
   }
 };
+
+// D5..D8 of vector v with the stream's sign diagonals: the global one (masks
+// in shared memory) or, with per-vector diagonals, v's own (derived from
+// the seed and v's (layer, kv, head) index).
+template <int D, int BITS, int G>
+__device__ __forceinline__ void decode_vector(const DecArgs &a, uint32_t vec_signs, uint64_t seed,
+                                              const uint32_t *mask, uint32_t v,
+                                              const uint8_t *codes, const uint8_t *meta,
+                                              uint32_t (&out)[D / 2]) {
+  if (vec_signs) {
+    VectorSigns<D> sg;
+    vec_sign_words<D>(seed, fdiv(a.tdiv, v), sg.S);
+    Dec<D, BITS, G>::vector(codes, meta, sg, out);
+  } else {
+    Dec<D, BITS, G>::vector(codes, meta, GlobalSigns{mask}, out);
+  }
+}
 
 // Writes this lane's decoded row (bf16 words `out`) into the warp's staging
 // buffer as row `lane` of the 128-byte swizzle (conflict-free).
@@ -318,7 +344,8 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   auto emit = [&](const uint8_t *codes, const uint8_t *meta, uint32_t v0, uint32_t nv) {
     uint32_t out[D / 2];
     const bool act = uint32_t(lane) < nv;
-    if (act) Dec<D, BITS, G>::vector(codes + lane * C::CB, meta + lane * C::MB, ctl->mask, out);
+    if (act) decode_vector<D, BITS, G>(a, ctl->vec_signs, ctl->seed, ctl->mask, v0 + lane,
+                                       codes + lane * C::CB, meta + lane * C::MB, out);
     if constexpr (!kIsPaged<Layout>) {
       if (use_tma) {
         store_block_tma<D>(lay, out, v0, stage, stage_busy);
@@ -366,6 +393,19 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   };
   uint32_t b = next_raw(warp), k = 0;
   __syncwarp();
+  if constexpr (32 * C::CB > S::BLK) {  // 8-bit: one block in both buffers
+#pragma unroll 1
+    while (b < nblk) {
+      issue_raw(b, 0);
+      wait(0);
+      const uint32_t v0 = vs0 + b * 32;
+      emit(cbuf, mbuf, v0, min(32u, vs1 - v0));
+      b = next_raw(b + kDecWarps);
+      __syncwarp();  // every lane is done with the buffers
+    }
+    bulk_wait_all<0>();
+    return;
+  }
   if (b < nblk) issue_raw(b, 0);
 #pragma unroll 1
   while (b < nblk) {
@@ -407,6 +447,7 @@ __global__ void __launch_bounds__(kDecThreads)
     ctl->n_req_stream = h.n_req;
     ctl->n_chunks = h.n_chunks;
     ctl->code_elim = h.code_elim;
+    ctl->vec_signs = h.vec_signs;
     ctl->data_base = h.data_base;
     ctl->stream_bytes = h.stream_bytes;
     ctl->seed = h.seed;
@@ -437,7 +478,13 @@ __global__ void __launch_bounds__(kDecThreads)
   }
   const uint32_t bits = ctl->bits, group = ctl->group;
   if constexpr (D == 128) {
-    if (bits == 4 && group == 128)
+    if (bits == 8 && group == 128)
+      decode_body<128, 8, 128, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
+    else if (bits == 8 && group == 64)
+      decode_body<128, 8, 64, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
+    else if (bits == 8 && group == 32)
+      decode_body<128, 8, 32, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
+    else if (bits == 4 && group == 128)
       decode_body<128, 4, 128, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 64)
       decode_body<128, 4, 64, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
@@ -450,7 +497,11 @@ __global__ void __launch_bounds__(kDecThreads)
     else
       decode_body<128, 2, 32, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
   } else {
-    if (bits == 4 && group == 64)
+    if (bits == 8 && group == 64)
+      decode_body<64, 8, 64, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
+    else if (bits == 8 && group == 32)
+      decode_body<64, 8, 32, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
+    else if (bits == 4 && group == 64)
       decode_body<64, 4, 64, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 32)
       decode_body<64, 4, 32, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
@@ -559,8 +610,8 @@ struct ElimCtl {
   uint64_t zbar;
   uint64_t mbar[kElimWarps];
   uint32_t red[kElimThreads / 32];
-  uint32_t ok, bits, group, nlist;
-  uint64_t base, limit;
+  uint32_t ok, bits, group, nlist, vec_signs;
+  uint64_t base, limit, seed;
   alignas(16) uint32_t mask[128];
   uint32_t list[kElimThreads];
 };
@@ -668,7 +719,8 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
         uint32_t out[D / 2];
         const bool act = uint32_t(lane) < nv;
         if (act)
-          Dec<D, BITS, G>::vector(chunk + (b * 32 + lane) * C::CB, mbuf + lane * C::MB, ctl->mask, out);
+          decode_vector<D, BITS, G>(a, ctl->vec_signs, ctl->seed, ctl->mask, v0 + lane,
+                                    chunk + (b * 32 + lane) * C::CB, mbuf + lane * C::MB, out);
         if constexpr (!kIsPaged<Layout>) {
           if (use_tma) {
             store_block_tma<D>(lay, out, v0, stage, stage_busy);
@@ -719,6 +771,8 @@ __global__ void __launch_bounds__(kElimThreads, 1)
     ctl->group = h.group;
     ctl->base = h.data_base;
     ctl->limit = min(a.in_bytes, h.stream_bytes);
+    ctl->vec_signs = h.vec_signs;
+    ctl->seed = h.seed;
     if (h.ok) sign_masks(h.seed, D, ctl->mask);
   }
   if constexpr (kIsPaged<Layout>) {
@@ -728,7 +782,13 @@ __global__ void __launch_bounds__(kElimThreads, 1)
   if (!ctl->ok) return;  // decode_kernel reports the header
   const uint32_t bits = ctl->bits, group = ctl->group;
   if constexpr (D == 128) {
-    if (bits == 4 && group == 128)
+    if (bits == 8 && group == 128)
+      elim_body<128, 8, 128>(a, lay, ctl, smem, s_cum);
+    else if (bits == 8 && group == 64)
+      elim_body<128, 8, 64>(a, lay, ctl, smem, s_cum);
+    else if (bits == 8 && group == 32)
+      elim_body<128, 8, 32>(a, lay, ctl, smem, s_cum);
+    else if (bits == 4 && group == 128)
       elim_body<128, 4, 128>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 64)
       elim_body<128, 4, 64>(a, lay, ctl, smem, s_cum);
@@ -741,7 +801,11 @@ __global__ void __launch_bounds__(kElimThreads, 1)
     else
       elim_body<128, 2, 32>(a, lay, ctl, smem, s_cum);
   } else {
-    if (bits == 4 && group == 64)
+    if (bits == 8 && group == 64)
+      elim_body<64, 8, 64>(a, lay, ctl, smem, s_cum);
+    else if (bits == 8 && group == 32)
+      elim_body<64, 8, 32>(a, lay, ctl, smem, s_cum);
+    else if (bits == 4 && group == 64)
       elim_body<64, 4, 64>(a, lay, ctl, smem, s_cum);
     else if (bits == 4 && group == 32)
       elim_body<64, 4, 32>(a, lay, ctl, smem, s_cum);

@@ -49,8 +49,9 @@ struct Cfg {
   static constexpr int LOG2D = D == 64 ? 6 : D == 128 ? 7 : 8;
   static constexpr int K = LOG2D / 2;            // meta stored x 2^-K
   static constexpr int QMAX = (1 << BITS) - 1;
+  static constexpr int QH = (1 << (BITS - 1)) - 1;  // symmetric: codes -QH .. QH
   static_assert(VC % 32 == 0 && VM % 32 == 0, "a block of 32 vectors lies in one chunk");
-  static_assert(R >= 2 && R <= 16, "segment size");
+  static_assert(R >= 2 && R <= 32, "segment size");
   static_assert(SLICE % 32 == 0, "meta slices hold whole 8-word groups");
 };
 
@@ -116,8 +117,8 @@ struct Enc : Cfg<D, BITS, G> {
 
   // E1/E2: widen bf16 exactly and flip the sign bit of negative channels.
   // Word k of the row holds channels 2k (low half) and 2k+1 (high half).
-  static __device__ __forceinline__ void unpack(const uint8_t *row, const uint32_t *__restrict__ mask,
-                                                Pairs<D> &y) {
+  template <class SG>
+  static __device__ __forceinline__ void unpack(const uint8_t *row, const SG &sg, Pairs<D> &y) {
     const uint4 *r4 = reinterpret_cast<const uint4 *>(row);
 #pragma unroll
     for (int q = 0; q < D / 16; ++q) {
@@ -126,7 +127,7 @@ struct Enc : Cfg<D, BITS, G> {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int k = 4 * q + e;
-        const uint32_t x0 = wa[e] ^ mask[k], x1 = wb[e] ^ mask[k + D / 4];
+        const uint32_t x0 = wa[e] ^ sg.word(k), x1 = wb[e] ^ sg.word(k + D / 4);
         y.p[2 * k] = make_float2(__uint_as_float(x0 << 16), __uint_as_float(x1 << 16));
         y.p[2 * k + 1] =
             make_float2(__uint_as_float(x0 & 0xFFFF0000u), __uint_as_float(x1 & 0xFFFF0000u));
@@ -138,9 +139,9 @@ struct Enc : Cfg<D, BITS, G> {
   // 64-channel half (HALF bytes apart), 16-byte chunk c stored at
   // row * 128 + ((c ^ (row % 8)) * 16) (the tensor maps' 128-byte swizzle,
   // which keeps these reads conflict-free for consecutive rows).
-  template <int HALF = 4096>
-  static __device__ __forceinline__ void unpack_swz(const uint8_t *wbuf, int row,
-                                                    const uint32_t *__restrict__ mask, Pairs<D> &y) {
+  template <int HALF = 4096, class SG>
+  static __device__ __forceinline__ void unpack_swz(const uint8_t *wbuf, int row, const SG &sg,
+                                                    Pairs<D> &y) {
     const int sw = row & 7;
     auto chunk = [&](int q) {
       return *reinterpret_cast<const uint4 *>(wbuf + (q >> 3) * HALF + row * 128 +
@@ -153,7 +154,7 @@ struct Enc : Cfg<D, BITS, G> {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int k = 4 * q + e;
-        const uint32_t x0 = wa[e] ^ mask[k], x1 = wb[e] ^ mask[k + D / 4];
+        const uint32_t x0 = wa[e] ^ sg.word(k), x1 = wb[e] ^ sg.word(k + D / 4);
         y.p[2 * k] = make_float2(__uint_as_float(x0 << 16), __uint_as_float(x1 << 16));
         y.p[2 * k + 1] =
             make_float2(__uint_as_float(x0 & 0xFFFF0000u), __uint_as_float(x1 & 0xFFFF0000u));
@@ -192,15 +193,23 @@ struct Enc : Cfg<D, BITS, G> {
   // sf >= (max - zf) / (2^b - 1) keeps p below 2^b - 1 + 2^-18. Codes pack
   // LSB first (reading R6).
   static __device__ __forceinline__ uint32_t vector(Pairs<D> &y, uint32_t (&code)[C::CW],
-                                                    uint32_t (&meta)[C::NG], float one) {
+                                                    uint32_t (&meta)[C::NG], float one,
+                                                    uint32_t sym) {
     fwht_pairs<D>(y);
-    return quantize(y, code, meta, one);
+    return quantize(y, code, meta, one, sym);
   }
-  // E4..E7 on the transformed vector.
+  // E4..E7 on the transformed vector. With `sym` (reading R19, symmetric
+  // absmax): scale s_h = RU16(fl(max|y| / (2^(b-1) - 1)) * 2^-K), stored zero
+  // -2^(b-1) * s_h (exact, so the decoder's zf + q * sf is (q - 2^(b-1)) * sf),
+  // p = fl(y * r) and code = nearest integer to p + 2^(b-1): the offset is
+  // folded into the rounding constant (1.5 * 2^23 + 2^(b-1) is even, so ties
+  // still go to even p) and the clamp to [-(2^(b-1) - 1), 2^(b-1) - 1] never
+  // acts for a finite group (|p| <= max|y| / s32 * (1 + 2^-22)).
   static __device__ __forceinline__ uint32_t quantize(Pairs<D> &y, uint32_t (&code)[C::CW],
-                                                      uint32_t (&meta)[C::NG], float one) {
+                                                      uint32_t (&meta)[C::NG], float one,
+                                                      uint32_t sym) {
     uint32_t err = 0;
-    float zf[C::NG], rr[C::NG];
+    float zf[C::NG], rr[C::NG];  // zf: subtracted before the product (0 when symmetric)
 #pragma unroll
     for (int g = 0; g < C::NG; ++g) {
       float mn, mx;
@@ -209,17 +218,27 @@ struct Enc : Cfg<D, BITS, G> {
       mx = __fadd_rn(mx, 0.0f);
       if (!(isfinite(mn) && isfinite(mx))) err |= 1u;
       const float down = 1.0f / float(1 << C::K), up = float(1 << C::K);
-      const __half zh = __float2half_rd(__fmul_rn(mn, down));
-      zf[g] = __fmul_rn(__half2float(zh), up);
-      const float s32 = __fdiv_rn(__fsub_rn(mx, zf[g]), float(C::QMAX));
-      const __half sh = __float2half_ru(__fmul_rn(s32, down));
+      __half zh, sh;
+      if (sym) {
+        const float am = fmaxf(fabsf(mn), fabsf(mx));
+        sh = __float2half_ru(__fmul_rn(__fdiv_rn(am, float(C::QH)), down));
+        zh = (__half_as_ushort(sh) & 0x7FFFu) == 0
+                 ? __ushort_as_half(0)
+                 : __float2half_rd(__fmul_rn(__half2float(sh), -float(1 << (BITS - 1))));
+        zf[g] = 0.0f;
+      } else {
+        zh = __float2half_rd(__fmul_rn(mn, down));
+        zf[g] = __fmul_rn(__half2float(zh), up);
+        const float s32 = __fdiv_rn(__fsub_rn(mx, zf[g]), float(C::QMAX));
+        sh = __float2half_ru(__fmul_rn(s32, down));
+      }
       const float sf = __fmul_rn(__half2float(sh), up);
       const uint16_t zb = __half_as_ushort(zh), sb = __half_as_ushort(sh);
       if ((zb & 0x7FFFu) == 0x7C00u || (sb & 0x7FFFu) == 0x7C00u) err |= 2u;
       rr[g] = ((sb & 0x7FFFu) == 0) ? 0.0f : __frcp_rn(sf);
       meta[g] = uint32_t(sb) | (uint32_t(zb) << 16);
     }
-    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const float kMagic = sym ? 12582912.0f + float(1 << (BITS - 1)) : 12582912.0f;  // 1.5 * 2^23
     const float2 mag = make_float2(kMagic, kMagic), one2 = make_float2(one, one);
 #pragma unroll
     for (int j = 0; j < D / 2; ++j) {
@@ -264,9 +283,9 @@ __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t b
   uint32_t code[C::CW], meta[C::NG];
   if (valid) {
     if constexpr (kFwht)
-      err |= E::vector(y, code, meta, a.one);
+      err |= E::vector(y, code, meta, a.one, a.sym);
     else
-      err |= E::quantize(y, code, meta, a.one);
+      err |= E::quantize(y, code, meta, a.one, a.sym);
     uint4 *cd = reinterpret_cast<uint4 *>(a.out + a.data_base + uint64_t(v) * C::CB);
 #pragma unroll
     for (int q = 0; q < C::CW / 4; ++q)
@@ -365,7 +384,9 @@ __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t b
 // ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
-template <int D, int BITS, int G, class Layout, bool kNarrow, bool kSearch>
+// kVec: per-(layer, kv, head) sign diagonals (each lane derives its vector's
+// diagonal from the seed) instead of the one in the kernel's parameters.
+template <int D, int BITS, int G, class Layout, bool kNarrow, bool kSearch, bool kVec>
 __global__ void __launch_bounds__(kEncThreads, 1)
     encode_kernel(const __grid_constant__ EncArgs a, const __grid_constant__ Layout lay) {
   using C = Cfg<D, BITS, G>;
@@ -410,6 +431,16 @@ __global__ void __launch_bounds__(kEncThreads, 1)
   auto finish_block = [&](uint32_t blk, uint32_t v, bool valid, Pairs<D> &y) {
     encode_finish_block<D, BITS, G, true, kSearch>(a, blk, v, valid, y, err);
   };
+  // E1/E2 of vector v from row `row` of the warp's buffer.
+  auto unpack = [&](int row, uint32_t v, Pairs<D> &y) {
+    if constexpr (kVec) {
+      VectorSigns<D> sg;
+      vec_sign_words<D>(a.seed, fdiv(a.tdiv, v), sg.S);
+      E::template unpack_swz<S::HALF>(wbuf, row, sg, y);
+    } else {
+      E::template unpack_swz<S::HALF>(wbuf, row, GlobalSigns{a.sign_mask}, y);
+    }
+  };
 
   bool use_tma = false;
   if constexpr (!kPaged) use_tma = lay.tma != 0;
@@ -437,7 +468,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
         if (!mbar_wait(wbar, phase, a.status)) set_status(a.status, KVC_ERR_TIMEOUT);
         phase ^= 1;
         Pairs<D> y;
-        E::unpack_swz(wbuf, lane, a.sign_mask, y);
+        unpack(lane, blk * 32 + lane, y);
         // every lane has read the buffer; the next load may overwrite it
         fence_proxy_async_smem();
         __syncwarp();
@@ -532,7 +563,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
         __syncwarp();  // every lane's copies have landed
       }
       Pairs<D> y;
-      E::template unpack_swz<S::HALF>(wbuf, lane + int((cur >> 2) & 7u), a.sign_mask, y);
+      unpack(lane + int((cur >> 2) & 7u), v, y);
       // every lane has read the buffer; the next load may overwrite it
       fence_proxy_async_smem();
       __syncwarp();
@@ -551,7 +582,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       cp_async_wait_all();
       __syncwarp();  // every lane's copies have landed
       Pairs<D> y;
-      E::unpack_swz(wbuf, lane, a.sign_mask, y);
+      unpack(lane, v, y);
       __syncwarp();  // every lane has read the buffer; the next gather may overwrite it
       if (blk + stride < n_blocks) gather(next);
       next = src_of((blk + 2 * stride) * 32 + lane);

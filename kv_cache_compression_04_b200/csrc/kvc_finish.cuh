@@ -134,7 +134,9 @@ __device__ void fin_header(const FinArgs &a, const uint32_t *cum, uint64_t strea
   st_u32(o + 0, kMagic);
   st_u16(o + 4, 1);
   st_u16(o + 6, kHeader);
-  st_u32(o + 8, a.bits | (a.k << 8) | (a.origin << 16) | (code_elim << 24));
+  // flags: bit 0 code chunks eliminated, bits 1..2 quantizer, bit 3 signs
+  const uint32_t flags = code_elim | (a.quant << 1) | (a.signs << 3);
+  st_u32(o + 8, a.bits | (a.k << 8) | (a.origin << 16) | (flags << 24));
   st_u32(o + 12, a.group);
   st_u32(o + 16, a.layers);
   st_u32(o + 20, 2);

@@ -109,6 +109,49 @@ KVC_HD void sign_masks(uint64_t seed, int d, uint32_t *mask) {
   }
 }
 
+// Per-(layer, kv, head) diagonals (the FP4Quant abstract's variant of the
+// randomized transform): vector index i takes SplitMix64 outputs number
+// i*W .. i*W + W - 1 (W = d / 64) from state = seed, i.e. the generator
+// advanced by i*W steps; index 0 is the global diagonal. S receives them as
+// 32-bit words, S[j] holding channels 32j .. 32j + 31.
+template <int D>
+KVC_HD void vec_sign_words(uint64_t seed, uint32_t index, uint32_t (&S)[D / 32]) {
+  uint64_t st = seed + uint64_t(index) * uint64_t(D / 64) * 0x9E3779B97F4A7C15ull;
+#pragma unroll
+  for (int j = 0; j < D / 64; ++j) {
+    const uint64_t w = splitmix64(st);
+    S[2 * j] = uint32_t(w);
+    S[2 * j + 1] = uint32_t(w >> 32);
+  }
+}
+
+// The XOR mask of channel pair (c, c + 1) (c even) from such words: bit 15
+// flips channel c's bf16 sign, bit 31 channel c + 1's.
+template <int D>
+KVC_HD uint32_t pair_mask(const uint32_t (&S)[D / 32], int c) {
+  const uint32_t w = S[c / 32] >> (c % 32);
+  return ((w & 1u) << 15) | ((w & 2u) << 30);
+}
+
+// Sign sources of the transform kernels: the diagonal shared by every vector
+// (masks in the kernel's parameters) or the vector's own (its words in
+// registers). word(k) is the mask of channel pair (2k, 2k + 1).
+struct GlobalSigns {
+  const uint32_t *mask;
+  __device__ __forceinline__ uint32_t word(int k) const { return mask[k]; }
+  __device__ __forceinline__ uint4 quad(int q) const {  // words 4q .. 4q + 3
+    return reinterpret_cast<const uint4 *>(mask)[q];
+  }
+};
+template <int D>
+struct VectorSigns {
+  uint32_t S[D / 32];
+  __device__ __forceinline__ uint32_t word(int k) const { return pair_mask<D>(S, 2 * k); }
+  __device__ __forceinline__ uint4 quad(int q) const {
+    return make_uint4(word(4 * q), word(4 * q + 1), word(4 * q + 2), word(4 * q + 3));
+  }
+};
+
 // Unsigned 32-bit division by a run-time constant (Granlund and Montgomery,
 // "Division by invariant integers using multiplication", PLDI 1994, the
 // round-up variant): q = (umulhi(n, m) + n) >> s, exact for every n < 2^32.
@@ -178,6 +221,10 @@ struct EncArgs {
   float *ymid;         // unfused baseline only: transformed vectors, d fp32 each
   float one;           // 1.0: the quantizer's integer rounding multiplies by it
   uint32_t mode;       // KVC_LOSSLESS_*
+  uint32_t sym;        // 1: symmetric absmax quantizer (KVC_QUANT_SYM)
+  uint32_t vec_signs;  // 1: per-(layer, kv, head) sign diagonals
+  uint64_t seed;       // sign seed (per-vector diagonals)
+  FastDiv tdiv;        // tokens per (layer, kv, head): vector index = v / tokens
   uint32_t sign_mask[128];
 };
 
@@ -211,6 +258,7 @@ struct FinArgs {
   uint64_t wait_ns;
   uint32_t ticket_skip;
   uint32_t mode;  // KVC_LOSSLESS_*
+  uint32_t quant, signs;  // KVC_QUANT_*, KVC_SIGNS_* (header flags bits 1..3)
 };
 
 struct DecArgs {
@@ -221,6 +269,7 @@ struct DecArgs {
   uint64_t tokens;
   uint32_t V;
   uint32_t paged_receiver;   // 1: request count and lengths must match
+  FastDiv tdiv;              // tokens: a vector's (layer, kv, head) index = v / tokens
   uint8_t *ws_meta;          // expanded meta chunks, 16 KB each
   uint32_t ws_meta_chunks;   // slots in ws_meta
 };
@@ -246,6 +295,12 @@ inline void timing_mark(cudaStream_t st) {
                                        const DenseLayout &lay, int sms, cudaStream_t st); \
   cudaError_t launch_encode_paged_d##D(int bits, int group, const EncArgs &a,             \
                                        const PagedLayout &lay, int sms, cudaStream_t st); \
+  cudaError_t launch_encode_dense_d##D##_var(int bits, int group, const EncArgs &a,       \
+                                             const DenseLayout &lay, int sms,             \
+                                             cudaStream_t st);                            \
+  cudaError_t launch_encode_paged_d##D##_var(int bits, int group, const EncArgs &a,       \
+                                             const PagedLayout &lay, int sms,             \
+                                             cudaStream_t st);                            \
   cudaError_t launch_decode_dense_d##D(const DecArgs &a, const DenseLayout &lay, int sms, \
                                        cudaStream_t st);                                  \
   cudaError_t launch_decode_paged_d##D(const DecArgs &a, const PagedLayout &lay, int sms, \

@@ -46,6 +46,9 @@ cudaError_t launch_transform_paged(int d, const EncArgs &a, const PagedLayout &l
 }
 cudaError_t launch_quantize(int d, int bits, int group, const EncArgs &a, int sms, cudaStream_t st) {
   if (d == 128) {
+    if (bits == 8 && group == 128) return launch_q<128, 8, 128>(a, sms, st);
+    if (bits == 8 && group == 64) return launch_q<128, 8, 64>(a, sms, st);
+    if (bits == 8 && group == 32) return launch_q<128, 8, 32>(a, sms, st);
     if (bits == 4 && group == 128) return launch_q<128, 4, 128>(a, sms, st);
     if (bits == 4 && group == 64) return launch_q<128, 4, 64>(a, sms, st);
     if (bits == 4 && group == 32) return launch_q<128, 4, 32>(a, sms, st);
@@ -53,6 +56,8 @@ cudaError_t launch_quantize(int d, int bits, int group, const EncArgs &a, int sm
     if (bits == 2 && group == 64) return launch_q<128, 2, 64>(a, sms, st);
     if (bits == 2 && group == 32) return launch_q<128, 2, 32>(a, sms, st);
   } else {
+    if (bits == 8 && group == 64) return launch_q<64, 8, 64>(a, sms, st);
+    if (bits == 8 && group == 32) return launch_q<64, 8, 32>(a, sms, st);
     if (bits == 4 && group == 64) return launch_q<64, 4, 64>(a, sms, st);
     if (bits == 4 && group == 32) return launch_q<64, 4, 32>(a, sms, st);
     if (bits == 2 && group == 64) return launch_q<64, 2, 64>(a, sms, st);

@@ -14,9 +14,10 @@ def u16(t: torch.Tensor) -> np.ndarray:
     return synth.bf16_bits(t)
 
 
-def gpu_compress(desc, bits, group, seed=0, slack: int = 0, lossless: int = 0):
+def gpu_compress(desc, bits, group, seed=0, slack: int = 0, lossless: int = 0, quant: int = 0,
+                 signs: int = 0):
     """-> (status, stream uint8 numpy, device buffers)."""
-    p = kvc.params(bits, group, seed, lossless)
+    p = kvc.params(bits, group, seed, lossless, quant, signs)
     cap = kvc.kvc_max_compressed_bytes(desc, p)
     wsb = kvc.kvc_workspace_bytes(desc, p)
     assert cap > 0 and wsb > 0
@@ -43,8 +44,10 @@ def gpu_decompress(stream: np.ndarray | torch.Tensor, desc, nbytes: int | None =
     return kvc.kvc_stream_status(ws.data_ptr(), kvc._stream_ptr(None))
 
 
-def oracle_desc(bits, group, d, layers, heads, token_lens, seed=0, origin=0, lossless=0):
-    return oracle.StreamDesc(bits, group, d, layers, heads, token_lens, seed, origin, lossless)
+def oracle_desc(bits, group, d, layers, heads, token_lens, seed=0, origin=0, lossless=0, quant=0,
+                signs=0):
+    return oracle.StreamDesc(bits, group, d, layers, heads, token_lens, seed, origin, lossless,
+                             quant, signs)
 
 
 def first_diff(a: np.ndarray, b: np.ndarray, lay=None) -> str:

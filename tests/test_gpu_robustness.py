@@ -80,7 +80,8 @@ def test_good_stream_decodes():
 @pytest.mark.parametrize("field,offset,value", [
     ("magic", 0, 0x4A), ("version", 4, 2), ("bits", 8, 3), ("k", 9, 4), ("group", 12, 48),
     ("layers", 16, 3), ("kv", 20, 3), ("heads", 24, 5), ("head_dim", 28, 64),
-    ("tokens", 32, 0x11), ("n_chunks", 52, 0x77), ("stream_bytes", 61, 0x7F), ("flags", 11, 2)])
+    ("tokens", 32, 0x11), ("n_chunks", 52, 0x77), ("stream_bytes", 61, 0x7F),
+    ("flags: an undefined bit", 11, 0x10), ("flags: quantizer id 3", 11, 6)])
 def test_corrupt_header(field, offset, value):
     _, s = _good_stream()
     bad = s.copy()

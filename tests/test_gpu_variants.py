@@ -1,0 +1,165 @@
+"""The quantizer variants on the GPU against the oracle (readings R19-R21:
+symmetric absmax, 8-bit codes, per-(layer, kv, head) sign diagonals): every
+stream byte equal, the oracle's stream decoded on the GPU to the oracle's
+bf16 values bit for bit, attention over such streams within the attention
+tolerance, for dense and paged inputs, every group size, both lossless
+modes, and the full-size Llama-3-8B-shaped cache for each variant."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_compression_04_b200 as kvc
+import oracle
+from kv_cache_compression_04_b200 import synth
+from kvc_testutil import first_diff, gpu_compress, gpu_decompress, oracle_desc, u16
+
+pytestmark = pytest.mark.gpu
+
+SYM, VEC = kvc.KVC_QUANT_SYM, kvc.KVC_SIGNS_PER_VECTOR
+THREADS = max(1, min(os.cpu_count() or 1, 64))
+
+
+def _dense(d, bits, g, L, H, T, quant=0, signs=0, lossless=0, seed=5, kind="lognormal"):
+    w = synth.Workload("v", L, H, d, bits, g, seed=L * 31 + T, kind=kind, scale_sigma=1.5,
+                       tokens=T)
+    kv = synth.dense_kv(w).cuda()
+    x = u16(kv).reshape(-1, d)
+    od = oracle_desc(bits, g, d, L, H, [T], seed, 0, lossless, quant, signs)
+    ost, ostream = oracle.compress(od, x, threads=THREADS)
+    assert ost == oracle.OK
+    st, gstream, _, _ = gpu_compress(kvc.dense_desc(kv), bits, g, seed, lossless=lossless,
+                                     quant=quant, signs=signs)
+    assert st == kvc.KVC_OK, kvc.STATUS[st]
+    assert np.array_equal(gstream, ostream), first_diff(gstream, ostream, od.layout())
+    out = torch.zeros_like(kv)
+    assert gpu_decompress(ostream, kvc.dense_desc(out)) == kvc.KVC_OK
+    _, ox = oracle.decompress(ostream, od, threads=THREADS)
+    got = u16(out).reshape(-1, d)
+    assert np.array_equal(got, ox), f"{np.count_nonzero(got != ox)} decoded values differ"
+    return ostream
+
+
+@pytest.mark.parametrize("d,bits,g,L,H,T", [
+    (128, 2, 32, 2, 3, 1000), (128, 4, 64, 2, 3, 777), (128, 4, 128, 1, 4, 1111),
+    (128, 8, 32, 2, 2, 900), (128, 8, 64, 1, 3, 1500), (128, 8, 128, 2, 2, 2100),
+    (64, 4, 32, 2, 3, 999), (64, 8, 64, 2, 2, 1300), (64, 2, 64, 1, 3, 1777)])
+def test_symmetric_dense(d, bits, g, L, H, T):
+    s = _dense(d, bits, g, L, H, T, quant=SYM)
+    assert s[11] & 6 == 2
+
+
+@pytest.mark.parametrize("d,bits,g,L,H,T", [
+    (128, 8, 32, 2, 3, 1000), (128, 8, 64, 2, 2, 2049), (128, 8, 128, 1, 4, 4200),
+    (64, 8, 32, 3, 2, 999), (64, 8, 64, 2, 2, 2500)])
+def test_eight_bit_dense(d, bits, g, L, H, T):
+    _dense(d, bits, g, L, H, T)
+
+
+@pytest.mark.parametrize("d,bits,g,L,H,T", [
+    (128, 4, 128, 2, 3, 1000), (128, 2, 32, 2, 2, 777), (128, 8, 64, 1, 3, 640),
+    (64, 4, 64, 3, 2, 555), (128, 4, 32, 2, 2, 17)])
+def test_per_vector_signs_dense(d, bits, g, L, H, T):
+    s = _dense(d, bits, g, L, H, T, signs=VEC)
+    assert s[11] & 8
+
+
+def test_variants_combined_search_mode():
+    """Symmetric 2-bit codes with per-vector signs and the lossless search
+    (meta chunks through the XOR pipelines) on heavy-tailed input."""
+    _dense(128, 2, 32, 2, 4, 3000, quant=SYM, signs=VEC, lossless=kvc.KVC_LOSSLESS_SEARCH,
+           kind="outlier_t")
+    _dense(128, 8, 32, 2, 2, 2100, quant=SYM, lossless=kvc.KVC_LOSSLESS_SEARCH)
+
+
+@pytest.mark.parametrize("bits,g,quant,signs", [(4, 64, SYM, VEC), (8, 32, 0, VEC),
+                                                (8, 128, SYM, 0)])
+def test_variants_paged(bits, g, quant, signs):
+    seq = [20, 0, 33, 700, 16, 257]
+    w = synth.Workload("p", 2, 3, 128, bits, g, seed=3, kind="lognormal", scale_sigma=1.5,
+                       seq_lens=seq)
+    pk = synth.paged_kv(w, device="cuda")
+    x = oracle.gather_paged(u16(pk.pool).reshape(-1), 2, 3, 128, pk.strides(), 16, seq,
+                            pk.page_table.cpu().numpy(), 0, w.vectors)
+    od = oracle_desc(bits, g, 128, 2, 3, seq, 0, 1, 0, quant, signs)
+    ost, ostream = oracle.compress(od, x)
+    assert ost == oracle.OK
+    st, gstream, _, _ = gpu_compress(kvc.paged_desc(pk.pool, pk.page_table, seq), bits, g,
+                                     quant=quant, signs=signs)
+    assert st == kvc.KVC_OK
+    assert np.array_equal(gstream, ostream), first_diff(gstream, ostream, od.layout())
+    pool2 = torch.full_like(pk.pool, 1.5)
+    assert gpu_decompress(ostream, kvc.paged_desc(pool2, pk.page_table, seq)) == kvc.KVC_OK
+    got = oracle.gather_paged(u16(pool2).reshape(-1), 2, 3, 128, pk.strides(), 16, seq,
+                              pk.page_table.cpu().numpy(), 0, w.vectors)
+    _, ox = oracle.decompress(ostream, od)
+    assert np.array_equal(got, ox)
+
+
+def test_unfused_variants():
+    """The unfused baseline writes the fused path's stream for the symmetric
+    quantizer and 8-bit codes, and refuses per-vector diagonals."""
+    w = synth.Workload("u", 2, 2, 128, 8, 64, seed=4, kind="lognormal", tokens=700)
+    kv = synth.dense_kv(w).cuda()
+    desc = kvc.dense_desc(kv)
+    for bits, g, quant in [(8, 64, 0), (4, 32, SYM), (8, 128, SYM)]:
+        p = kvc.params(bits, g, 3, 0, quant)
+        cap = kvc.kvc_max_compressed_bytes(desc, p)
+        outs = []
+        for unfused in (False, True):
+            wsb = (kvc.kvc_unfused_workspace_bytes if unfused else kvc.kvc_workspace_bytes)(desc, p)
+            ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+            out = torch.zeros(cap, dtype=torch.uint8, device="cuda")
+            nb = torch.zeros(1, dtype=torch.int64, device="cuda")
+            fn = kvc.kvc_compress_unfused if unfused else kvc.kvc_compress
+            assert fn(desc, p, out.data_ptr(), cap, nb.data_ptr(), ws.data_ptr(), wsb,
+                      kvc._stream_ptr(None)) == kvc.KVC_OK
+            assert kvc.kvc_stream_status(ws.data_ptr(), kvc._stream_ptr(None)) == kvc.KVC_OK
+            outs.append(out[:int(nb.item())].cpu().numpy())
+        assert np.array_equal(outs[0], outs[1]), (bits, g, quant)
+    p = kvc.params(4, 64, 3, 0, 0, VEC)
+    wsb = kvc.kvc_unfused_workspace_bytes(desc, p)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    out = torch.zeros(kvc.kvc_max_compressed_bytes(desc, p), dtype=torch.uint8, device="cuda")
+    assert kvc.kvc_compress_unfused(desc, p, out.data_ptr(), out.numel(), None, ws.data_ptr(),
+                                    wsb, kvc._stream_ptr(None)) == kvc.KVC_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("bits,g,quant,signs,qpk", [(4, 128, SYM, 0, 4), (2, 32, 0, VEC, 7),
+                                                    (8, 64, SYM, VEC, 2), (8, 32, 0, 0, 8)])
+def test_attend_over_variant_streams(bits, g, quant, signs, qpk):
+    L, H, T, d = 2, 2, 900, 128
+    w = synth.Workload("a", L, H, d, bits, g, seed=12, kind="lognormal", scale_sigma=1.5,
+                       tokens=T)
+    kv = synth.dense_kv(w).cuda()
+    st, s, gbuf, n = gpu_compress(kvc.dense_desc(kv), bits, g, 9, quant=quant, signs=signs)
+    assert st == kvc.KVC_OK and s[11] & 1 == 0
+    q = torch.randn(L, 1, H * qpk, d, generator=torch.Generator(device="cuda").manual_seed(1),
+                    device="cuda").to(torch.bfloat16)
+    out = torch.full((L, 1, H * qpk, d), float("nan"), device="cuda")
+    ad = kvc.attn_desc(L, H, qpk, bits, g, [T], q, out, d ** -0.5)
+    ws = torch.empty(kvc.kvc_attend_workspace_bytes(ad), dtype=torch.uint8, device="cuda")
+    sp = kvc._stream_ptr(None)
+    assert kvc.kvc_attend(gbuf.data_ptr(), n, ad, ws.data_ptr(), ws.numel(), sp) == kvc.KVC_OK
+    assert kvc.kvc_stream_status(ws.data_ptr(), sp) == kvc.KVC_OK
+    od = oracle_desc(bits, g, d, L, H, [T], 9, 0, 0, quant, signs)
+    ost, ref = oracle.attend(s, od, u16(q.cpu()), qpk, d ** -0.5, threads=THREADS)
+    assert ost == oracle.OK
+    _, vals = oracle.decode_values(s, od, threads=THREADS)
+    V = vals.reshape(L, 2, H, T, d)[:, 1]
+    got = out.cpu().numpy().astype(np.float64)
+    for h in range(H):
+        vmax = np.abs(V[:, h]).max()
+        sl = slice(h * qpk, (h + 1) * qpk)
+        err = np.abs(got[:, 0, sl] - ref[:, 0, sl]).max()
+        assert err <= 2e-4 * vmax + 1e-6, (h, err, vmax)
+
+
+@pytest.mark.parametrize("bits,g,quant,signs", [(4, 128, SYM, 0), (4, 128, 0, VEC),
+                                                (8, 128, 0, 0)])
+def test_full_llama8b_variant(bits, g, quant, signs):
+    """The Llama-3-8B-shaped cache (32 x 2 x 8 x 4096 x 128) in each variant,
+    compared whole: stream bytes and decoded values."""
+    w = synth.workload("llama8b")
+    _dense(128, bits, g, w.layers, w.kv_heads, w.tokens, quant=quant, signs=signs)
