@@ -189,20 +189,34 @@ struct Dec : Cfg<D, BITS, G> {
   }
 };
 
-// D5..D8 of vector v with the stream's sign diagonals: the global one (masks
-// in shared memory) or, with per-vector diagonals, v's own (derived from
-// the seed and v's (layer, kv, head) index).
+// D5..D8 of vector v with the global sign diagonal (masks in shared
+// memory). A stream with per-vector diagonals (reading R20) is corrected in
+// the staging buffer by fix_row_signs.
 template <int D, int BITS, int G>
-__device__ __forceinline__ void decode_vector(const DecArgs &a, uint32_t vec_signs, uint64_t seed,
-                                              const uint32_t *mask, uint32_t v,
-                                              const uint8_t *codes, const uint8_t *meta,
-                                              uint32_t (&out)[D / 2]) {
-  if (vec_signs) {
-    VectorSigns<D> sg;
-    vec_sign_words<D>(seed, fdiv(a.tdiv, v), sg.S);
-    Dec<D, BITS, G>::vector(codes, meta, sg, out);
-  } else {
-    Dec<D, BITS, G>::vector(codes, meta, GlobalSigns{mask}, out);
+__device__ __forceinline__ void decode_vector(const uint32_t *mask, const uint8_t *codes,
+                                              const uint8_t *meta, uint32_t (&out)[D / 2]) {
+  Dec<D, BITS, G>::vector(codes, meta, GlobalSigns{mask}, out);
+}
+
+// This lane's staged row XOR the global masks XOR the masks of its vector's
+// own diagonal ((layer, kv, head) index `index`). Not inlined: inlined, the
+// untaken branch alone measured 7% on the default decode (register and
+// schedule changes of the surrounding loop).
+template <int D>
+__device__ __noinline__ void fix_row_signs(uint8_t *stage, const uint32_t *mask, uint64_t seed,
+                                           uint32_t index) {
+  const int lane = threadIdx.x & 31;
+  VectorSigns<D> sg;
+  vec_sign_words<D>(seed, index, sg.S);
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    uint4 *p = reinterpret_cast<uint4 *>(stage + swz_offset(lane, c));
+    uint4 w = *p;
+    w.x ^= mask[4 * c] ^ sg.word(4 * c);
+    w.y ^= mask[4 * c + 1] ^ sg.word(4 * c + 1);
+    w.z ^= mask[4 * c + 2] ^ sg.word(4 * c + 2);
+    w.w ^= mask[4 * c + 3] ^ sg.word(4 * c + 3);
+    *p = w;
   }
 }
 
@@ -222,11 +236,14 @@ __device__ __forceinline__ void stage_row(const uint32_t (&out)[D / 2], uint8_t 
 // copy per 64-channel half.
 template <int D>
 __device__ __forceinline__ void store_block_tma(const DenseLayout &lay, const uint32_t (&out)[D / 2],
-                                                uint32_t v0, uint8_t *stage, bool &stage_busy) {
+                                                uint32_t v0, uint8_t *stage, bool &stage_busy,
+                                                const DecArgs &a, uint32_t vec_signs,
+                                                const uint32_t *mask, uint64_t seed) {
   const int lane = threadIdx.x & 31;
   if (stage_busy && lane == 0) bulk_wait_read<0>();  // the previous block's stores have read it
   __syncwarp();
   stage_row<D>(out, stage);
+  if (vec_signs) fix_row_signs<D>(stage, mask, seed, fdiv(a.tdiv, v0 + lane));
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
@@ -344,11 +361,11 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   auto emit = [&](const uint8_t *codes, const uint8_t *meta, uint32_t v0, uint32_t nv) {
     uint32_t out[D / 2];
     const bool act = uint32_t(lane) < nv;
-    if (act) decode_vector<D, BITS, G>(a, ctl->vec_signs, ctl->seed, ctl->mask, v0 + lane,
-                                       codes + lane * C::CB, meta + lane * C::MB, out);
+    if (act) decode_vector<D, BITS, G>(ctl->mask, codes + lane * C::CB, meta + lane * C::MB, out);
     if constexpr (!kIsPaged<Layout>) {
       if (use_tma) {
-        store_block_tma<D>(lay, out, v0, stage, stage_busy);
+        store_block_tma<D>(lay, out, v0, stage, stage_busy, a, ctl->vec_signs, ctl->mask,
+                           ctl->seed);
         return;
       }
     }
@@ -363,6 +380,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
     }
     __syncwarp();  // the previous block's scatter has read the buffer
     stage_row<D>(out, stage);
+    if (ctl->vec_signs) fix_row_signs<D>(stage, ctl->mask, ctl->seed, fdiv(a.tdiv, v0 + lane));
     __syncwarp();
     if constexpr (kNarrow)
       scatter_rows_narrow<D / 8>(stage, lay.base, dst ? uint32_t((dst - lay.base) >> 4) : ~0u);
@@ -719,11 +737,12 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
         uint32_t out[D / 2];
         const bool act = uint32_t(lane) < nv;
         if (act)
-          decode_vector<D, BITS, G>(a, ctl->vec_signs, ctl->seed, ctl->mask, v0 + lane,
-                                    chunk + (b * 32 + lane) * C::CB, mbuf + lane * C::MB, out);
+          decode_vector<D, BITS, G>(ctl->mask, chunk + (b * 32 + lane) * C::CB,
+                                    mbuf + lane * C::MB, out);
         if constexpr (!kIsPaged<Layout>) {
           if (use_tma) {
-            store_block_tma<D>(lay, out, v0, stage, stage_busy);
+            store_block_tma<D>(lay, out, v0, stage, stage_busy, a, ctl->vec_signs, ctl->mask,
+                               ctl->seed);
             continue;
           }
         }
@@ -738,6 +757,7 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
         }
         __syncwarp();  // the previous block's scatter has read the buffer
         stage_row<D>(out, stage);
+        if (ctl->vec_signs) fix_row_signs<D>(stage, ctl->mask, ctl->seed, fdiv(a.tdiv, v0 + lane));
         __syncwarp();
         scatter_rows<D>(stage, dst);
       }
