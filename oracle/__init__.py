@@ -69,7 +69,7 @@ PIPE_ZE, PIPE_XOR_ZE, PIPE_ZE2, PIPE_XOR_ZE2 = range(4)
 LOSSLESS_FIXED, LOSSLESS_SEARCH, LOSSLESS_NONE = range(3)
 BITMAP2 = 256
 # Quantizer (readings R5, R19) and sign diagonals (readings R3, R20).
-QUANT_ASYM, QUANT_SYM = 0, 1
+QUANT_ASYM, QUANT_SYM, QUANT_FP4 = 0, 1, 2
 SIGNS_GLOBAL, SIGNS_PER_VECTOR = 0, 1
 
 
@@ -110,6 +110,12 @@ def lib():
                 "orc_quantize_vector_q": (C.c_int, [u16p, C.c_int, C.c_int, C.c_int,
                                                     C.c_int, u64p, u8p, u8p]),
                 "orc_sign_words_at": (None, [C.c_uint64, C.c_int, C.c_uint64, u64p]),
+                "orc_dequantize_vector_q": (None, [u8p, u8p, C.c_int, C.c_int, C.c_int,
+                                                   C.c_int, u64p, u16p]),
+                "orc_e2m1_to_f32": (C.c_float, [C.c_int]),
+                "orc_f32_to_e2m1_rne": (C.c_int, [C.c_float]),
+                "orc_e4m3_to_f32": (C.c_float, [C.c_int]),
+                "orc_f32_to_e4m3_ru": (C.c_int, [C.c_float]),
                 "orc_quantize_vector": (C.c_int, [u16p, C.c_int, C.c_int,
                                                   C.c_int, u64p, u8p, u8p]),
                 "orc_dequantize_vector": (None, [u8p, u8p, C.c_int, C.c_int,
@@ -235,6 +241,22 @@ def quantize_scalar(y: float, zf: float, r: float, qmax: int) -> int:
     return lib().orc_quantize_scalar(y, zf, r, qmax)
 
 
+def e2m1_to_f32(code: int) -> float:
+    return lib().orc_e2m1_to_f32(code)
+
+
+def f32_to_e2m1_rne(p: float) -> int:
+    return lib().orc_f32_to_e2m1_rne(float(np.float32(p)))
+
+
+def e4m3_to_f32(b: int) -> float:
+    return lib().orc_e4m3_to_f32(b)
+
+
+def f32_to_e4m3_ru(x: float) -> int:
+    return lib().orc_f32_to_e4m3_ru(float(np.float32(x)))
+
+
 def quantize_scalar_sym(y: float, r: float, bits: int) -> int:
     return lib().orc_quantize_scalar_sym(y, r, bits)
 
@@ -258,7 +280,7 @@ def quantize_vectors(x: np.ndarray, bits: int, group: int, seed: int, quant: int
 
 
 def dequantize_vectors(codes: np.ndarray, meta: np.ndarray, d: int, bits: int,
-                       group: int, seed: int) -> np.ndarray:
+                       group: int, seed: int, quant: int = QUANT_ASYM) -> np.ndarray:
     codes = np.ascontiguousarray(codes, np.uint8)
     meta = np.ascontiguousarray(meta, np.uint8)
     V = codes.shape[0]
@@ -266,9 +288,9 @@ def dequantize_vectors(codes: np.ndarray, meta: np.ndarray, d: int, bits: int,
     lib().orc_sign_words(seed, d, _p(sw, C.c_uint64))
     out = np.zeros((V, d), np.uint16)
     for v in range(V):
-        lib().orc_dequantize_vector(_p(codes[v], C.c_uint8), _p(meta[v], C.c_uint8),
-                                    d, bits, group, _p(sw, C.c_uint64),
-                                    _p(out[v], C.c_uint16))
+        lib().orc_dequantize_vector_q(_p(codes[v], C.c_uint8), _p(meta[v], C.c_uint8),
+                                      d, bits, group, quant, _p(sw, C.c_uint64),
+                                      _p(out[v], C.c_uint16))
     return out
 
 

@@ -206,6 +206,51 @@ int orc_quantize_scalar(float y, float zf, float r, int qmax) {
   return (int)n;
 }
 
+/* ---- FP4 (reading R22) ---------------------------------------------------- */
+/* e2m1 (1 sign, 2 exponent, 1 mantissa bit, no inf/NaN): magnitude index   */
+/* i = 0..7 has the values 0, 0.5, 1, 1.5, 2, 3, 4, 6; code = i | 8 for a    */
+/* negative value (never for magnitude 0).                                    */
+float orc_e2m1_to_f32(int code) {
+  static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  return (code & 8) ? -mag[code & 7] : mag[code & 7];
+}
+
+/* The e2m1 code nearest to p, ties to the even magnitude index (even
+ * mantissa bit); magnitudes above 6 give 6; zero is always code 0. The
+ * nearest value is found by scanning the eight magnitudes in double. */
+int orc_f32_to_e2m1_rne(float p) {
+  double a = fabs((double)p), best = 1e300;
+  int i, bi = 0;
+  for (i = 0; i < 8; i++) {
+    double e = fabs(a - (double)orc_e2m1_to_f32(i));
+    if (e < best || (e == best && (i & 1) == 0)) {
+      best = e;
+      bi = i;
+    }
+  }
+  return (bi != 0 && p < 0.0f) ? (bi | 8) : bi;
+}
+
+/* e4m3 (the fn variant: 1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits, no inf, 0x7F/0xFF NaN; largest finite 448; subnormals m * 2^-9). */
+float orc_e4m3_to_f32(int b) {
+  int e = (b >> 3) & 15, m = b & 7;
+  float v;
+  if ((b & 0x7F) == 0x7F) return NAN;
+  v = e ? ldexpf(1.0f + (float)m / 8.0f, e - 7) : ldexpf((float)m, -9);
+  return (b & 0x80) ? -v : v;
+}
+
+/* The smallest non-negative finite e4m3 value >= x (x >= 0, finite), 448
+ * (0x7E) if x exceeds it: a scan over the 127 non-negative finite codes,
+ * which are increasing in their bit patterns. */
+int orc_f32_to_e4m3_ru(float x) {
+  int b;
+  for (b = 0; b < 0x7F; b++)
+    if ((double)orc_e4m3_to_f32(b) >= (double)x) return b;
+  return 0x7E;
+}
+
 /* One code of reading R19 (symmetric absmax): p = fl(y * r) (one fp32
  * rounding), then the nearest integer to p, ties to even, clamped to
  * [-qh, qh], qh = 2^(b-1) - 1. The stored code is that integer + 2^(b-1). */
@@ -248,6 +293,48 @@ int orc_quantize_vector(const uint16_t *x, int d, int bits, int g,
  *   z_h = fp16 of -2^(b-1) * f32(s_h) (exact: a power-of-two multiple; +0
  *   when s_h is 0), so zf + code * sf = (code - 2^(b-1)) * sf exactly.
  * A non-finite y gives NONFINITE, an infinite s_h or z_h RANGE (R8). */
+/* Reading R22 (the FP4Quant abstract: micro-grouped dual-scale FP4), bits
+ * 4, in the 4-byte-per-group meta of reading R6:
+ *   a = max |y| over the group (+0);
+ *   s2_h = RU16(fl(a / 2688) * 2^-k), s2 = f32(s2_h) * 2^k   (2688 = 6 * 448);
+ *   per half-group j (g/2 channels): a_j = max |y| over it,
+ *     s1_j = e4m3 RU(fl(a_j / (6 * s2))), at most 448 (0 when s2 is 0);
+ *     S_j = s1_j * s2 (exact in fp32), r_j = 0 if S_j == 0 else fl(1 / S_j);
+ *   code = e2m1 nearest to fl(y * r_j), ties to even, |.| <= 6;
+ *   meta bytes: s2_h (little-endian), s1_0, s1_1.
+ * The decoded value e2m1(code) * S_j is exact in fp32. A non-finite y gives
+ * NONFINITE, an infinite s2_h RANGE. */
+static int quantize_group_fp4(const float *yg, int g, int k, uint8_t *q, uint8_t *m) {
+  float a = 0.0f, up = ldexpf(1.0f, k), down = ldexpf(1.0f, -k), s2;
+  uint16_t s2h;
+  int c, j;
+  for (c = 0; c < g; c++)
+    if (fabsf(yg[c]) > a) a = fabsf(yg[c]);
+  a = a + 0.0f;
+  s2h = orc_f32_to_f16_ru((a / 2688.0f) * down);
+  s2 = orc_f16_to_f32(s2h) * up;
+  m[0] = (uint8_t)(s2h & 0xFF);
+  m[1] = (uint8_t)(s2h >> 8);
+  if (f16_is_inf(s2h)) {
+    for (c = 0; c < g; c++) q[c] = 0;
+    m[2] = m[3] = 0;
+    return ORC_ERR_RANGE;
+  }
+  for (j = 0; j < 2; j++) {
+    const float *yh = yg + j * (g / 2);
+    float aj = 0.0f, S, r;
+    int s1;
+    for (c = 0; c < g / 2; c++)
+      if (fabsf(yh[c]) > aj) aj = fabsf(yh[c]);
+    s1 = s2 == 0.0f ? 0 : orc_f32_to_e4m3_ru(aj / (6.0f * s2));
+    S = orc_e4m3_to_f32(s1) * s2;
+    r = S == 0.0f ? 0.0f : 1.0f / S;
+    for (c = 0; c < g / 2; c++) q[j * (g / 2) + c] = (uint8_t)orc_f32_to_e2m1_rne(yh[c] * r);
+    m[2 + j] = (uint8_t)s1;
+  }
+  return ORC_OK;
+}
+
 int orc_quantize_vector_q(const uint16_t *x, int d, int bits, int g, int quant,
                           const uint64_t *sign_words, uint8_t *codes,
                           uint8_t *meta) {
@@ -283,6 +370,11 @@ int orc_quantize_vector_q(const uint16_t *x, int d, int bits, int g, int quant,
     }
     mn = mn + 0.0f;
     mx = mx + 0.0f;
+    if (quant == ORC_QUANT_FP4) {
+      const int st = quantize_group_fp4(yg, g, k, q + j * g, meta + 4 * j);
+      if (st != ORC_OK && status == ORC_OK) status = st;
+      continue;
+    }
     if (quant == ORC_QUANT_SYM) {
       const float a = fabsf(mn) > fabsf(mx) ? fabsf(mn) : fabsf(mx);
       const int qh = (1 << (bits - 1)) - 1;
@@ -317,19 +409,15 @@ int orc_quantize_vector_q(const uint16_t *x, int d, int bits, int g, int quant,
   return status;
 }
 
-/* Decode of one vector, the inverse path of [P3]. Reading R9:
- *   y^ = zf + q*sf (the product rounded, then the sum rounded);
- *   the same butterfly as the encoder (H_d H_d = d I);
- *   x^ = bf16_RNE(sign_c * (u * 2^-log2(d))). */
-void orc_dequantize_vector(const uint8_t *codes, const uint8_t *meta, int d,
-                           int bits, int g, const uint64_t *sign_words,
-                           uint16_t *xhat) {
-  float y[ORC_MAX_D];
+/* The decoder's transformed values y^ of one vector (fp32):
+ *   readings R5 / R19 (reading R9): y^ = zf + q*sf, the product rounded,
+ *   then the sum rounded;
+ *   reading R22 (FP4): y^ = e2m1(q) * (s1_j * s2), exact. */
+static void grid_values(const uint8_t *codes, const uint8_t *meta, int d, int bits, int g,
+                        int quant, float *y) {
   uint8_t q[ORC_MAX_D];
-  int k = orc_meta_shift(d), l2d = 0, c, j;
-  float up = ldexpf(1.0f, k), inv_d;
-  while ((1 << l2d) < d) l2d++;
-  inv_d = ldexpf(1.0f, -l2d);
+  int k = orc_meta_shift(d), c, j;
+  float up = ldexpf(1.0f, k);
   orc_unpack_codes(codes, d, bits, q);
   for (j = 0; j < d / g; j++) {
     uint16_t sh = (uint16_t)(meta[4 * j] | (meta[4 * j + 1] << 8));
@@ -337,10 +425,35 @@ void orc_dequantize_vector(const uint8_t *codes, const uint8_t *meta, int d,
     float sf = orc_f16_to_f32(sh) * up;
     float zf = orc_f16_to_f32(zh) * up;
     for (c = j * g; c < (j + 1) * g; c++) {
-      float p = (float)q[c] * sf;
-      y[c] = zf + p;
+      if (quant == ORC_QUANT_FP4) {
+        const float S = orc_e4m3_to_f32(meta[4 * j + 2 + (c - j * g) / (g / 2)]) * sf;
+        y[c] = orc_e2m1_to_f32(q[c]) * S;
+      } else {
+        float p = (float)q[c] * sf;
+        y[c] = zf + p;
+      }
     }
   }
+}
+
+/* Decode of one vector, the inverse path of [P3]. Reading R9:
+ *   y^ as grid_values;
+ *   the same butterfly as the encoder (H_d H_d = d I);
+ *   x^ = bf16_RNE(sign_c * (u * 2^-log2(d))). */
+void orc_dequantize_vector(const uint8_t *codes, const uint8_t *meta, int d,
+                           int bits, int g, const uint64_t *sign_words,
+                           uint16_t *xhat) {
+  orc_dequantize_vector_q(codes, meta, d, bits, g, ORC_QUANT_ASYM, sign_words, xhat);
+}
+
+void orc_dequantize_vector_q(const uint8_t *codes, const uint8_t *meta, int d, int bits, int g,
+                             int quant, const uint64_t *sign_words, uint16_t *xhat) {
+  float y[ORC_MAX_D];
+  int l2d = 0, c;
+  float inv_d;
+  while ((1 << l2d) < d) l2d++;
+  inv_d = ldexpf(1.0f, -l2d);
+  grid_values(codes, meta, d, bits, g, quant, y);
   orc_fwht(y, d);
   for (c = 0; c < d; c++) {
     float u = y[c] * inv_d;
@@ -358,22 +471,15 @@ void orc_dequantize_vector(const uint8_t *codes, const uint8_t *meta, int d,
 void orc_dequantize_vector_f64(const uint8_t *codes, const uint8_t *meta, int d,
                                int bits, int g, const uint64_t *sign_words,
                                double *xhat) {
+  orc_dequantize_vector_f64_q(codes, meta, d, bits, g, ORC_QUANT_ASYM, sign_words, xhat);
+}
+
+void orc_dequantize_vector_f64_q(const uint8_t *codes, const uint8_t *meta, int d, int bits,
+                                 int g, int quant, const uint64_t *sign_words, double *xhat) {
   float yf[ORC_MAX_D];
   double y[ORC_MAX_D];
-  uint8_t q[ORC_MAX_D];
-  int k = orc_meta_shift(d), c, j, h, i;
-  float up = ldexpf(1.0f, k);
-  orc_unpack_codes(codes, d, bits, q);
-  for (j = 0; j < d / g; j++) {
-    uint16_t sh = (uint16_t)(meta[4 * j] | (meta[4 * j + 1] << 8));
-    uint16_t zh = (uint16_t)(meta[4 * j + 2] | (meta[4 * j + 3] << 8));
-    float sf = orc_f16_to_f32(sh) * up;
-    float zf = orc_f16_to_f32(zh) * up;
-    for (c = j * g; c < (j + 1) * g; c++) {
-      float p = (float)q[c] * sf;
-      yf[c] = zf + p;
-    }
-  }
+  int c, h, i;
+  grid_values(codes, meta, d, bits, g, quant, yf);
   for (c = 0; c < d; c++) y[c] = (double)yf[c];
   for (h = 1; h < d; h *= 2)
     for (i = 0; i < d; i++)
@@ -674,7 +780,9 @@ int orc_check_desc(const orc_desc *d) {
   int r;
   if (!d) return ORC_ERR_INVALID_ARG;
   if (d->bits != 2 && d->bits != 4 && d->bits != 8) return ORC_ERR_UNSUPPORTED;
-  if (d->quant != ORC_QUANT_ASYM && d->quant != ORC_QUANT_SYM) return ORC_ERR_UNSUPPORTED;
+  if (d->quant != ORC_QUANT_ASYM && d->quant != ORC_QUANT_SYM && d->quant != ORC_QUANT_FP4)
+    return ORC_ERR_UNSUPPORTED;
+  if (d->quant == ORC_QUANT_FP4 && d->bits != 4) return ORC_ERR_UNSUPPORTED;
   if (d->signs != ORC_SIGNS_GLOBAL && d->signs != ORC_SIGNS_PER_VECTOR)
     return ORC_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256)
@@ -856,12 +964,13 @@ static int decode_segment_in(const orc_desc *d, const orc_layout *lay, uint64_t 
       if (d->signs == ORC_SIGNS_PER_VECTOR)
         orc_sign_words_at(d->sign_seed, d->head_dim, vector_index(d, lay, v0 + v), sw);
       if (vals)
-        orc_dequantize_vector_f64(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
-                                  d->head_dim, d->bits, d->group, sw, vals + v * d->head_dim);
+        orc_dequantize_vector_f64_q(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
+                                    d->head_dim, d->bits, d->group, d->quant, sw,
+                                    vals + v * d->head_dim);
       else
-        orc_dequantize_vector(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
-                              d->head_dim, d->bits, d->group, sw,
-                              vectors + v * d->head_dim);
+        orc_dequantize_vector_q(codes + v * lay->code_bytes, meta + v * lay->meta_bytes,
+                                d->head_dim, d->bits, d->group, d->quant, sw,
+                                vectors + v * d->head_dim);
     }
   free(codes);
   free(meta);

@@ -51,6 +51,7 @@ enum {
 #define ORC_MAX_SEG 32       /* code chunks per segment: g * b / 32 <= 128 * 8 / 32 */
 #define ORC_QUANT_ASYM 0      /* reading R5: min/max, zero and scale        */
 #define ORC_QUANT_SYM 1       /* reading R19: symmetric absmax              */
+#define ORC_QUANT_FP4 2       /* reading R22: e2m1 codes, dual scales (4 bit) */
 #define ORC_SIGNS_GLOBAL 0    /* reading R3: one diagonal for the tensor    */
 #define ORC_SIGNS_PER_VECTOR 1 /* reading R20: one per (layer, kv, head)   */
 
@@ -81,6 +82,14 @@ void orc_dequantize_vector(const uint8_t *codes, const uint8_t *meta, int d,
 void orc_dequantize_vector_f64(const uint8_t *codes, const uint8_t *meta, int d,
                                int bits, int g, const uint64_t *sign_words,
                                double *xhat);
+void orc_dequantize_vector_q(const uint8_t *codes, const uint8_t *meta, int d, int bits, int g,
+                             int quant, const uint64_t *sign_words, uint16_t *xhat);
+void orc_dequantize_vector_f64_q(const uint8_t *codes, const uint8_t *meta, int d, int bits,
+                                 int g, int quant, const uint64_t *sign_words, double *xhat);
+float orc_e2m1_to_f32(int code);
+int orc_f32_to_e2m1_rne(float p);
+float orc_e4m3_to_f32(int b);
+int orc_f32_to_e4m3_ru(float x);
 void orc_pack_codes(const uint8_t *q, int d, int bits, uint8_t *packed);
 void orc_unpack_codes(const uint8_t *packed, int d, int bits, uint8_t *q);
 

@@ -258,7 +258,7 @@ def test_eight_bit_packing_and_layout():
         with pytest.raises(ValueError):
             oracle.StreamDesc(bad, 32, 128, 1, 1, [10]).layout()
     with pytest.raises(ValueError):
-        oracle.StreamDesc(4, 32, 128, 1, 1, [10], quant=2).layout()
+        oracle.StreamDesc(4, 32, 128, 1, 1, [10], quant=3).layout()
     with pytest.raises(ValueError):
         oracle.StreamDesc(4, 32, 128, 1, 1, [10], signs=2).layout()
 
@@ -322,3 +322,129 @@ def test_eight_bit_group_128_full_segment():
     st2, s2 = oracle.compress(desc, x, threads=3)
     assert st2 == oracle.OK and np.array_equal(s, s2)
     assert (oracle.decompress(s, desc, threads=3)[1] == oracle.decompress(s, desc)[1]).all()
+
+
+# --------------------------------------------------------------- R22 --
+E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]   # OCP e2m1 magnitudes (exponent bias 1)
+
+
+def test_e2m1_table_and_nearest_even():
+    assert [oracle.e2m1_to_f32(c) for c in range(8)] == E2M1
+    assert [oracle.e2m1_to_f32(c | 8) for c in range(1, 8)] == [-v for v in E2M1[1:]]
+    # every p on a fine grid (all midpoints included), against a scan written
+    # here: nearest magnitude, ties to the even index, zero is code 0
+    grid = np.concatenate([np.arange(-8, 8.0001, 1 / 64), [0.25, 0.75, 1.25, 1.75, 2.5, 3.5,
+                                                           5.0, -0.25, -5.0, 1e9, -1e9]])
+    for p in grid.astype(np.float32):
+        a = abs(float(p))
+        d = [abs(a - v) for v in E2M1]
+        best = min(d)
+        i = min(j for j in range(8) if d[j] == best and (j % 2 == 0 or d.count(best) == 1))
+        want = i | (8 if (i and p < 0) else 0)
+        assert oracle.f32_to_e2m1_rne(p) == want, p
+    assert oracle.f32_to_e2m1_rne(0.25) == 0 and oracle.f32_to_e2m1_rne(0.75) == 2
+    assert oracle.f32_to_e2m1_rne(1.25) == 2 and oracle.f32_to_e2m1_rne(1.75) == 4
+    assert oracle.f32_to_e2m1_rne(2.5) == 4 and oracle.f32_to_e2m1_rne(3.5) == 6
+    assert oracle.f32_to_e2m1_rne(5.0) == 6 and oracle.f32_to_e2m1_rne(-0.1) == 0
+
+
+def test_e4m3_against_torch_and_round_up():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    for b in range(256):
+        got = oracle.e4m3_to_f32(b)
+        assert (np.isnan(got) and np.isnan(ref[b])) or got == ref[b], b
+    finite = sorted(set(float(v) for v in ref[:0x7F]))      # non-negative finite values
+    rng = np.random.default_rng(0)
+    xs = np.concatenate([rng.uniform(0, 450, 2000), np.exp(rng.uniform(-12, 6, 2000)), finite,
+                         np.nextafter(np.array(finite, np.float32), np.float32(1e9))])
+    for x in xs.astype(np.float32):
+        b = oracle.f32_to_e4m3_ru(x)
+        above = [v for v in finite if v >= float(x)]
+        want = above[0] if above else 448.0
+        assert oracle.e4m3_to_f32(b) == want, x
+
+
+@pytest.mark.parametrize("g", [32, 64, 128])
+def test_fp4_groups_are_dual_scale_e2m1_grids(g):
+    d = 128
+    rng = np.random.default_rng(g + 7)
+    x = rng.standard_normal((50, d)).astype(np.float32) * np.exp(rng.standard_normal((50, 1)) * 2)
+    x[4] = 0.0
+    x[6, :8] *= 100.0                                   # one dominant half-group
+    xb = bf16(x)
+    st, codes, meta = oracle.quantize_vectors(xb, 4, g, 2, quant=oracle.QUANT_FP4)
+    assert st == oracle.OK
+    up = 2.0 ** oracle.meta_shift(d)
+    e4 = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for v in range(x.shape[0]):
+        y = transformed(xb[v], 2)
+        q = codes_of(codes[v], d, 4)
+        m = meta[v].reshape(d // g, 4)
+        for j in range(d // g):
+            yg = y[j * g:(j + 1) * g]
+            s2h = int(m[j, 0]) | (int(m[j, 1]) << 8)
+            s2 = f16(s2h) * up
+            a = np.abs(yg).max()
+            target = float(np.float32(np.float32(a) / np.float32(2688.0)))
+            assert s2 >= target and (s2h == 0 or f16(np.uint16(s2h - 1)) * up < target)
+            for h in range(2):
+                yh = yg[h * g // 2:(h + 1) * g // 2]
+                qh = q[j * g + h * g // 2: j * g + (h + 1) * g // 2]
+                s1 = e4[m[j, 2 + h]]
+                assert 0 <= s1 <= 448
+                S = s1 * s2
+                if s2 == 0:
+                    assert s1 == 0 and (qh == 0).all()
+                    continue
+                u = float(np.float32(np.float32(np.abs(yh).max()) / np.float32(6 * s2)))
+                assert s1 == min(min(v2 for v2 in e4[:0x7F] if v2 >= u), 448.0)
+                vals = np.array([E2M1[c & 7] * (-1 if c & 8 else 1) for c in qh]) * S
+                # nearest point of the grid e2m1 x S (ties either way), and
+                # within it: |y| <= 6 S up to the fp32 roundings of u and 1/S
+                grid = np.array(E2M1 + [-v for v in E2M1[1:]]) * S
+                err = np.abs(yh - vals)
+                alt = np.abs(yh[:, None] - grid[None, :]).min(axis=1)
+                assert (err <= alt + 1e-6 * S).all()
+                assert np.abs(yh).max() <= 6 * S * (1 + 1e-6)
+
+
+def test_fp4_stream_decodes_to_the_grid_and_flags():
+    d, g = 128, 32
+    desc, s, x, codes, meta = _raw_stream(4, g, 2, 2, [60], quant=oracle.QUANT_FP4,
+                                          signs=oracle.SIGNS_PER_VECTOR, kind="outlier_t")
+    assert s[11] == 4 | 8                                 # quantizer 2, per-vector signs
+    st, xh = oracle.decode_values(s, desc)
+    assert st == oracle.OK
+    e4 = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    up = 2.0 ** oracle.meta_shift(d)
+    Hm = sylvester(d)
+    T = 60
+    for v in range(codes.shape[0]):
+        q = codes_of(codes[v], d, 4)
+        m = meta[v].reshape(d // g, 4)
+        want = np.empty(d)
+        for c in range(d):
+            j, h = c // g, (c % g) // (g // 2)
+            s2 = f16(int(m[j, 0]) | (int(m[j, 1]) << 8)) * up
+            want[c] = E2M1[q[c] & 7] * (-1 if q[c] & 8 else 1) * e4[m[j, 2 + h]] * s2
+        D = signs_of(oracle.sign_words_at(11, d, v // T), d)
+        np.testing.assert_allclose(Hm @ (D * xh[v]), want, rtol=0, atol=1e-9 * abs(want).max())
+    st, xb = oracle.decompress(s, desc)
+    assert st == oracle.OK
+    back = synth.bf16_bits(torch.from_numpy(xh).to(torch.bfloat16))
+    assert (back == xb).mean() > 0.999
+    other = oracle.StreamDesc(4, g, d, 2, 2, [60], 11, 0, oracle.LOSSLESS_NONE, oracle.QUANT_SYM,
+                              oracle.SIGNS_PER_VECTOR)
+    assert oracle.decompress(s, other)[0] == oracle.CORRUPT
+
+
+def test_fp4_errors():
+    d = 128
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 3.0e38                                    # y ~ 3e38: the fp16 scale overflows
+    assert oracle.quantize_vectors(bf16(x), 4, 64, 0, quant=oracle.QUANT_FP4)[0] == oracle.RANGE
+    x[0, 0] = np.inf
+    assert oracle.quantize_vectors(bf16(x), 4, 64, 0, quant=oracle.QUANT_FP4)[0] == oracle.NONFINITE
+    with pytest.raises(ValueError):                      # FP4 codes are 4-bit
+        oracle.StreamDesc(2, 32, 128, 1, 1, [10], quant=oracle.QUANT_FP4).layout()
