@@ -92,13 +92,22 @@ enum { KVC_LOSSLESS_FIXED = 0, KVC_LOSSLESS_SEARCH = 1, KVC_LOSSLESS_NONE = 2 };
  *                   (2^(b-1) - 1)), code = RNE(y / scale) + 2^(b-1) in
  *                   [1, 2^b - 1]; the stored zero is -2^(b-1) * scale, so
  *                   every decoder reads both alike (zero + code * scale)
+ *   KVC_QUANT_FP4   4-bit e2m1 codes (0, +-0.5, +-1, +-1.5, +-2, +-3, +-4,
+ *                   +-6) with two scales (the FP4Quant abstract's
+ *                   micro-grouped dual-scale FP4): per group an fp16 scale
+ *                   s2 = RU16(max|y| / 2688), per half-group an e4m3
+ *                   micro-scale s1 = RU(max_half|y| / (6 s2)) (at most 448);
+ *                   code = e2m1 nearest to y / (s1 s2), ties to even; meta
+ *                   bytes s2 (LE), s1 of each half. bits must be 4.
  *   KVC_SIGNS_GLOBAL      one +-1 diagonal for every vector
  *   KVC_SIGNS_PER_VECTOR  one per (layer, kv, head): vector index i (its
  *                   position in the order [layer][kv][head]) takes the
  *                   SplitMix64 outputs i*W .. i*W + W - 1 (W = head_dim / 64)
  * The stream's header flags record both (bits 1..2 and 3); a decoder needs
- * no parameter for them. */
-enum { KVC_QUANT_ASYM = 0, KVC_QUANT_SYM = 1 };
+ * no parameter for them. Decoded values: zero + code * scale (ASYM, SYM),
+ * e2m1(code) * s1 * s2 (FP4), each exact in fp32 before the inverse
+ * transform. */
+enum { KVC_QUANT_ASYM = 0, KVC_QUANT_SYM = 1, KVC_QUANT_FP4 = 2 };
 enum { KVC_SIGNS_GLOBAL = 0, KVC_SIGNS_PER_VECTOR = 1 };
 
 /* Quantization and lossless parameters.
@@ -110,7 +119,8 @@ enum { KVC_SIGNS_GLOBAL = 0, KVC_SIGNS_PER_VECTOR = 1 };
  *             sign_seed, is 1 (per-vector diagonals: see above).
  *  lossless   KVC_LOSSLESS_* (encoder only).
  *  quant      KVC_QUANT_*.
- *  signs      KVC_SIGNS_* (kvc_compress_unfused: KVC_SIGNS_GLOBAL only).
+ *  signs      KVC_SIGNS_* (kvc_compress_unfused: KVC_SIGNS_GLOBAL and the
+ *             min/max or absmax quantizer only).
  *  reserved   must be 0.
  * Other values are refused with KVC_ERR_UNSUPPORTED. */
 typedef struct {
@@ -324,8 +334,9 @@ kvc_status kvc_compress_unfused(const kvc_kv_desc *kv, const kvc_params *params,
  * (q . k = (H D q) . y / d) and invert the transform once per query head, so
  * no decoded key or value is written to memory.
  *
- * The stream must describe a cache of this shape with these bits and group,
- * head_dim 128, and store every code chunk raw (the header flag clear, the
+ * The stream must describe a cache of this shape with these bits, group and
+ * quantizer (ASYM and SYM decode alike, either matches the other), head_dim
+ * 128, either sign mode, and store every code chunk raw (the header flag clear, the
  * usual case; KVC_ERR_CORRUPT in the status word otherwise); its meta chunks
  * may use any lossless pipeline. q: DEVICE bf16 [layers][n_requests]
  * [kv_heads * q_per_kv][128], contiguous; out: DEVICE fp32 of the same shape
@@ -339,6 +350,7 @@ typedef struct {
   int32_t q_per_kv;           /* 1 .. 8 (e.g. 4 for 32 query / 8 kv heads) */
   int32_t bits;               /* as compressed */
   int32_t group_size;         /* as compressed */
+  int32_t quant;              /* as compressed (KVC_QUANT_*; ASYM and SYM alike) */
   int32_t n_requests;         /* 1 .. KVC_MAX_REQUESTS */
   float scale;                /* e.g. 1 / sqrt(head_dim) */
   const int32_t *seq_lens;    /* HOST [n_requests] */

@@ -96,9 +96,10 @@ kvc_status describe(const kvc_kv_desc *kv, const kvc_params *p, Shape &s) {
   if (s.V > 0 && (!kv->data || !aligned16(kv->data))) return KVC_ERR_INVALID_ARG;
   if (!p) return KVC_OK;
   if (p->bits != 2 && p->bits != 4 && p->bits != 8) return KVC_ERR_UNSUPPORTED;
-  if ((p->quant != KVC_QUANT_ASYM && p->quant != KVC_QUANT_SYM) ||
+  if ((p->quant != KVC_QUANT_ASYM && p->quant != KVC_QUANT_SYM && p->quant != KVC_QUANT_FP4) ||
       (p->signs != KVC_SIGNS_GLOBAL && p->signs != KVC_SIGNS_PER_VECTOR))
     return KVC_ERR_UNSUPPORTED;
+  if (p->quant == KVC_QUANT_FP4 && p->bits != 4) return KVC_ERR_UNSUPPORTED;
   if (p->group_size != 32 && p->group_size != 64 && p->group_size != 128)
     return KVC_ERR_UNSUPPORTED;
   if (p->group_size > s.D) return KVC_ERR_UNSUPPORTED;
@@ -293,8 +294,9 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   if (!params) return KVC_ERR_INVALID_ARG;
   kvc_status st = describe(kv, params, s);
   if (st != KVC_OK) return st;
-  // the unfused baseline's transform kernel applies the global diagonal only
-  if (unfused && params->signs != KVC_SIGNS_GLOBAL) return KVC_ERR_UNSUPPORTED;
+  // the unfused baseline: the global diagonal and the affine quantizers only
+  if (unfused && (params->signs != KVC_SIGNS_GLOBAL || params->quant == KVC_QUANT_FP4))
+    return KVC_ERR_UNSUPPORTED;
   if (!out || !aligned16(out) || !workspace || !aligned16(workspace)) return KVC_ERR_INVALID_ARG;
   const uint64_t need = unfused ? round256(s.ws_bytes) + s.V * uint64_t(s.D) * 4 : s.ws_bytes;
   if (out_capacity < s.max_bytes || workspace_bytes < need) return KVC_ERR_CAPACITY;
@@ -321,6 +323,7 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   a.mode = uint32_t(params->lossless);
   a.sym = params->quant == KVC_QUANT_SYM ? 1u : 0u;
   a.vec_signs = params->signs == KVC_SIGNS_PER_VECTOR ? 1u : 0u;
+  a.fp4 = params->quant == KVC_QUANT_FP4 ? 1u : 0u;
   a.seed = params->sign_seed;
   a.tdiv = make_fastdiv(uint32_t(s.T ? s.T : 1));
   sign_masks(params->sign_seed, s.D, a.sign_mask);
@@ -530,8 +533,7 @@ kvc_status attn_shape(const kvc_attn_desc *at, AttnShape &r) {
   kv.stride_head = T * at->head_dim;
   kv.stride_kv = kv.stride_head * at->kv_heads;
   kv.stride_layer = kv.stride_kv * 2;
-  kvc_params p{at->bits, at->group_size, 0, KVC_LOSSLESS_FIXED, KVC_QUANT_ASYM, KVC_SIGNS_GLOBAL,
-               0};
+  kvc_params p{at->bits, at->group_size, 0, KVC_LOSSLESS_FIXED, at->quant, KVC_SIGNS_GLOBAL, 0};
   const kvc_status st = describe(&kv, &p, r.s);
   if (st != KVC_OK) return st;
   r.s.n_req = uint32_t(at->n_requests);
@@ -589,6 +591,7 @@ kvc_status kvc_attend(const void *in, size_t in_bytes, const kvc_attn_desc *at, 
   a.qpk = uint32_t(at->q_per_kv);
   a.bits = uint32_t(at->bits);
   a.group = uint32_t(at->group_size);
+  a.fp4 = at->quant == KVC_QUANT_FP4 ? 1u : 0u;
   a.tokens = r.s.T;
   a.V = d.V;
   a.splits = r.splits;

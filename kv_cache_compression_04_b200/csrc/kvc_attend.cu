@@ -9,7 +9,14 @@ namespace {
 
 template <int BITS, int G, int QPK>
 cudaError_t launch_att_k(const AttnArgs &a, int units, cudaStream_t st) {
-  attend_kernel<128, BITS, G, QPK><<<units * a.splits, kAttThreads, 0, st>>>(a);
+  if constexpr (BITS == 4) {
+    if (a.fp4)
+      attend_kernel<128, 4, G, QPK, true><<<units * a.splits, kAttThreads, 0, st>>>(a);
+    else
+      attend_kernel<128, 4, G, QPK><<<units * a.splits, kAttThreads, 0, st>>>(a);
+  } else {
+    attend_kernel<128, BITS, G, QPK><<<units * a.splits, kAttThreads, 0, st>>>(a);
+  }
   const cudaError_t e = cudaGetLastError();
   timing_mark(st);
   return e;

@@ -29,8 +29,9 @@ constexpr int kAttMaxG = 8;    // query heads per kv head
 // Header checks shared by the attention kernels: the stream describes this
 // cache with the stated bits and group, and stores every code chunk raw (the
 // code region is then the plain array of per-vector codes). Flags: bit 0
-// (eliminated code chunks) clear; either quantizer (both decode as zero +
-// code * scale); either sign mode (bit 3: per-vector diagonals).
+// (eliminated code chunks) clear; the min/max or absmax quantizer (both
+// decode as zero + code * scale) or, as the caller states, FP4 (e2m1(code) *
+// s1 * s2); either sign mode (bit 3: per-vector diagonals).
 template <int D>
 __device__ __forceinline__ bool attn_header_ok(const AttnArgs &a, uint64_t &base, uint32_t &n_code,
                                                uint64_t &seed) {
@@ -46,7 +47,9 @@ __device__ __forceinline__ bool attn_header_ok(const AttnArgs &a, uint64_t &base
   seed = ld_u64(h + 40);
   return ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 &&
          (ld_u32(h + 4) >> 16) == kHeader && h[8] == a.bits && h[9] == kLog2D / 2 &&
-         (h[11] & 0xF5u) == 0 && ld_u32(h + 12) == a.group && ld_u32(h + 16) == a.layers &&
+         (h[11] & 0xF1u) == 0 && ((h[11] >> 1) & 3u) <= 2 &&
+         (((h[11] >> 1) & 3u) == 2) == (a.fp4 != 0) && ld_u32(h + 12) == a.group &&
+         ld_u32(h + 16) == a.layers &&
          ld_u32(h + 20) == 2 && ld_u32(h + 24) == a.kv_heads && ld_u32(h + 28) == D &&
          ld_u64(h + 32) == a.tokens && n_req == a.n_req && n_chunks == nc + nm &&
          ld_u64(h + 56) <= a.in_bytes && base + uint64_t(a.V) * cb <= ld_u64(h + 56);
@@ -97,7 +100,8 @@ constexpr int kAttRec = 128 + 4;
 // QPK: query heads per kv head rounded up to 1, 2, 4 or 8 (a.qpk of them
 // are real; the others score a zero query and are not written); G: the
 // quantization group.
-template <int D, int BITS, int G, int QPK>
+// kFp4: the stream's FP4 quantizer (reading R22).
+template <int D, int BITS, int G, int QPK, bool kFp4 = false>
 __global__ void __launch_bounds__(kAttThreads) attend_kernel(const __grid_constant__ AttnArgs a) {
   using C = Cfg<D, BITS, G>;
   static_assert(D == 128, "attention kernel: head_dim 128");
@@ -215,11 +219,16 @@ __global__ void __launch_bounds__(kAttThreads) attend_kernel(const __grid_consta
         const uint32_t m = reinterpret_cast<const uint32_t *>(mp)[c0 / G];
         const float sf = __half2float(__ushort_as_half(uint16_t(m))) * float(1 << C::K);
         const float zf = __half2float(__ushort_as_half(uint16_t(m >> 16))) * float(1 << C::K);
+        // FP4: the word's channels lie in one half-group (8 of >= 16)
+        const float S = kFp4 ? e4m3_value((m >> (16 + 8 * ((c0 % G) / (G / 2)))) & 0xFFu) * sf : 0.f;
 #pragma unroll
         for (int k = 0; k < per; k += 4) {
           float y[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) y[i] = fmaf(float((ws[e] >> ((k + i) * BITS)) & qmask), sf, zf);
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t code = (ws[e] >> ((k + i) * BITS)) & qmask;
+            y[i] = kFp4 ? e2m1_value(code) * S : fmaf(float(code), sf, zf);
+          }
 #pragma unroll
           for (int g = 0; g < QPK; ++g) {
             // read per token (a volatile load): kept in registers across
@@ -288,12 +297,15 @@ __global__ void __launch_bounds__(kAttThreads) attend_kernel(const __grid_consta
       const uint32_t m = reinterpret_cast<const uint32_t *>(meta_of(v, 1))[(wi * CPL) / G];
       const float sf = __half2float(__ushort_as_half(uint16_t(m))) * float(1 << C::K);
       const float zf = __half2float(__ushort_as_half(uint16_t(m >> 16))) * float(1 << C::K);
+      const float S =
+          kFp4 ? e4m3_value((m >> (16 + 8 * (((wi * CPL) % G) / (G / 2)))) & 0xFFu) * sf : 0.f;
       float p[QPK];
 #pragma unroll
       for (int g = 0; g < QPK; ++g) p[g] = sm.s[t - t_a][g];
 #pragma unroll
       for (int k = 0; k < CPL; ++k) {
-        const float y = fmaf(float((bits >> (k * BITS)) & qmask), sf, zf);
+        const uint32_t code = (bits >> (k * BITS)) & qmask;
+        const float y = kFp4 ? e2m1_value(code) * S : fmaf(float(code), sf, zf);
 #pragma unroll
         for (int g = 0; g < QPK; ++g) o[g][k] = fmaf(p[g], y, o[g][k]);
       }

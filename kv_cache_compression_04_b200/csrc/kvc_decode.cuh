@@ -35,9 +35,10 @@ struct DecCtl {
   uint64_t cbar[kDecWarps][2];  // per-warp code + meta blocks loaded (two buffers)
   uint32_t red[kDecThreads / 32];
   uint32_t hdr_ok;
-  uint32_t bits, group, n_req_stream, n_chunks, code_elim, vec_signs;
+  uint32_t bits, group, n_req_stream, n_chunks, code_elim, vec_signs, quant;
   uint64_t data_base, stream_bytes, seed;
   alignas(16) uint32_t mask[128];  // read as uint4
+  float e2m1[16];                  // FP4 code values
 };
 
 // Shared memory: per-warp output staging | per-warp code blocks | per-warp
@@ -68,7 +69,7 @@ __device__ __forceinline__ uint64_t ld_u64(const uint8_t *p) {
 
 // D1: the header (reading R12) against the receiver's description.
 struct StreamHdr {
-  uint32_t ok, bits, group, n_req, n_chunks, code_elim, vec_signs;
+  uint32_t ok, bits, group, n_req, n_chunks, code_elim, vec_signs, quant;
   uint64_t data_base, stream_bytes, seed;
 };
 template <int D>
@@ -80,8 +81,9 @@ __device__ __forceinline__ StreamHdr parse_header(const DecArgs &a) {
   const uint32_t bits = h[8], k = h[9], group = ld_u32(h + 12);
   // flags: bit 0 code chunks eliminated, bits 1..2 the quantizer (0 or 1;
   // both decode alike), bit 3 per-vector sign diagonals, the rest zero
-  const uint32_t flags = h[11];
-  bool ok = ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 && (flags & 0xF4u) == 0 &&
+  const uint32_t flags = h[11], quant = (flags >> 1) & 3u;
+  bool ok = ld_u32(h) == kMagic && (ld_u32(h + 4) & 0xFFFFu) == 1 && (flags & 0xF0u) == 0 &&
+            quant <= 2 && (quant != 2 || bits == 4) &&
             (ld_u32(h + 4) >> 16) == kHeader && (bits == 2 || bits == 4 || bits == 8) &&
             k == kLog2D / 2 &&
             (group == 32 || group == 64 || group == 128) && group <= D &&
@@ -106,10 +108,11 @@ __device__ __forceinline__ StreamHdr parse_header(const DecArgs &a) {
   r.seed = ld_u64(h + 40);
   r.code_elim = flags & 1u;
   r.vec_signs = (flags >> 3) & 1u;
+  r.quant = quant;
   return r;
 }
 
-template <int D, int BITS, int G>
+template <int D, int BITS, int G, bool kFp4 = false>
 struct Dec : Cfg<D, BITS, G> {
   using C = Cfg<D, BITS, G>;
 
@@ -122,16 +125,25 @@ struct Dec : Cfg<D, BITS, G> {
   // rounding. q*sf is exact (q < 16 times an fp16 value needs at most 15
   // significant bits), so one fused multiply-add equals fl(zf + fl(q*sf)).
   // The vector is held as pairs (c, c + d/2) like the encoder's.
+  // e2m1 (FP4 only): the 16 code values, a table in shared memory.
   template <class SG>
   static __device__ __forceinline__ void vector(const uint8_t *codes, const uint8_t *meta,
-                                                const SG &sg, uint32_t (&out)[D / 2]) {
-    float zf[C::NG], sf[C::NG];
+                                                const SG &sg, uint32_t (&out)[D / 2],
+                                                const float *e2m1 = nullptr) {
+    float zf[kFp4 ? 1 : C::NG], sf[kFp4 ? 1 : C::NG];
+    float S[kFp4 ? 2 * C::NG : 1];  // FP4 (reading R22): s1 * s2 per half-group, x 2^-log2 d
     const float up = float(1 << C::K) / float(D);
 #pragma unroll
     for (int g = 0; g < C::NG; ++g) {
       const uint32_t m = reinterpret_cast<const uint32_t *>(meta)[g];
-      sf[g] = __fmul_rn(__half2float(__ushort_as_half(uint16_t(m & 0xFFFFu))), up);
-      zf[g] = __fmul_rn(__half2float(__ushort_as_half(uint16_t(m >> 16))), up);
+      const float s = __fmul_rn(__half2float(__ushort_as_half(uint16_t(m & 0xFFFFu))), up);
+      if constexpr (kFp4) {
+        S[2 * g] = __fmul_rn(e4m3_value((m >> 16) & 0xFFu), s);
+        S[2 * g + 1] = __fmul_rn(e4m3_value(m >> 24), s);
+      } else {
+        sf[g] = s;
+        zf[g] = __fmul_rn(__half2float(__ushort_as_half(uint16_t(m >> 16))), up);
+      }
     }
     // Code -> float: a byte permute puts the code in the low byte of the bit
     // pattern 0x4B4000qq = 1.5*2^23 + q; subtracting 1.5*2^23 gives q exactly.
@@ -169,9 +181,16 @@ struct Dec : Cfg<D, BITS, G> {
 #pragma unroll
       for (int i = 0; i < JP; ++i) {
         const int j = piece * JP + i;
-        const int ga = j / G, gb = (j + D / 2) / G;
-        const float2 q = sub2(make_float2(code_float(lo, i), code_float(hi, i)), mag);
-        y.p[j] = fma2(q, make_float2(sf[ga], sf[gb]), make_float2(zf[ga], zf[gb]));
+        if constexpr (kFp4) {  // e2m1(code) * S, exact
+          const int ha = j / (G / 2), hb = (j + D / 2) / (G / 2);
+          const uint32_t ca = __float_as_uint(code_float(lo, i)) & 15u;
+          const uint32_t cb = __float_as_uint(code_float(hi, i)) & 15u;
+          y.p[j] = mul2(make_float2(e2m1[ca], e2m1[cb]), make_float2(S[ha], S[hb]));
+        } else {
+          const int ga = j / G, gb = (j + D / 2) / G;
+          const float2 q = sub2(make_float2(code_float(lo, i), code_float(hi, i)), mag);
+          y.p[j] = fma2(q, make_float2(sf[ga], sf[gb]), make_float2(zf[ga], zf[gb]));
+        }
       }
     }
     fwht_pairs<D>(y);
@@ -192,10 +211,11 @@ struct Dec : Cfg<D, BITS, G> {
 // D5..D8 of vector v with the global sign diagonal (masks in shared
 // memory). A stream with per-vector diagonals (reading R20) is corrected in
 // the staging buffer by fix_row_signs.
-template <int D, int BITS, int G>
-__device__ __forceinline__ void decode_vector(const uint32_t *mask, const uint8_t *codes,
-                                              const uint8_t *meta, uint32_t (&out)[D / 2]) {
-  Dec<D, BITS, G>::vector(codes, meta, GlobalSigns{mask}, out);
+template <int D, int BITS, int G, bool kFp4>
+__device__ __forceinline__ void decode_vector(const uint32_t *mask, const float *e2m1,
+                                              const uint8_t *codes, const uint8_t *meta,
+                                              uint32_t (&out)[D / 2]) {
+  Dec<D, BITS, G, kFp4>::vector(codes, meta, GlobalSigns{mask}, out, e2m1);
 }
 
 // This lane's staged row XOR the global masks XOR the masks of its vector's
@@ -257,7 +277,7 @@ __device__ __forceinline__ void store_block_tma(const DenseLayout &lay, const ui
   stage_busy = true;
 }
 
-template <int D, int BITS, int G, class Layout, bool kNarrow>
+template <int D, int BITS, int G, class Layout, bool kNarrow, bool kFp4 = false>
 __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, uint8_t *smem,
                             const uint32_t *cum) {
   using C = Cfg<D, BITS, G>;
@@ -361,7 +381,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   auto emit = [&](const uint8_t *codes, const uint8_t *meta, uint32_t v0, uint32_t nv) {
     uint32_t out[D / 2];
     const bool act = uint32_t(lane) < nv;
-    if (act) decode_vector<D, BITS, G>(ctl->mask, codes + lane * C::CB, meta + lane * C::MB, out);
+    if (act) decode_vector<D, BITS, G, kFp4>(ctl->mask, ctl->e2m1, codes + lane * C::CB, meta + lane * C::MB, out);
     if constexpr (!kIsPaged<Layout>) {
       if (use_tma) {
         store_block_tma<D>(lay, out, v0, stage, stage_busy, a, ctl->vec_signs, ctl->mask,
@@ -457,6 +477,7 @@ __global__ void __launch_bounds__(kDecThreads)
     mbar_init(&ctl->cbar[tid][1], 1);
     mbar_fence_init();
   }
+  if (tid < 16) ctl->e2m1[tid] = e2m1_value(uint32_t(tid));  // FP4 code values
   if (tid == 0) {
     const StreamHdr h = parse_header<D>(a);
     ctl->hdr_ok = h.ok;
@@ -466,6 +487,7 @@ __global__ void __launch_bounds__(kDecThreads)
     ctl->n_chunks = h.n_chunks;
     ctl->code_elim = h.code_elim;
     ctl->vec_signs = h.vec_signs;
+    ctl->quant = h.quant;
     ctl->data_base = h.data_base;
     ctl->stream_bytes = h.stream_bytes;
     ctl->seed = h.seed;
@@ -495,6 +517,22 @@ __global__ void __launch_bounds__(kDecThreads)
     return;
   }
   const uint32_t bits = ctl->bits, group = ctl->group;
+  if (ctl->quant == 2) {  // FP4 (4-bit; the header check guarantees it)
+    if constexpr (D == 128) {
+      if (group == 128)
+        decode_body<128, 4, 128, Layout, kNarrow, true>(a, lay, ctl, smem, s_cum);
+      else if (group == 64)
+        decode_body<128, 4, 64, Layout, kNarrow, true>(a, lay, ctl, smem, s_cum);
+      else
+        decode_body<128, 4, 32, Layout, kNarrow, true>(a, lay, ctl, smem, s_cum);
+    } else {
+      if (group == 64)
+        decode_body<64, 4, 64, Layout, kNarrow, true>(a, lay, ctl, smem, s_cum);
+      else
+        decode_body<64, 4, 32, Layout, kNarrow, true>(a, lay, ctl, smem, s_cum);
+    }
+    return;
+  }
   if constexpr (D == 128) {
     if (bits == 8 && group == 128)
       decode_body<128, 8, 128, Layout, kNarrow>(a, lay, ctl, smem, s_cum);
@@ -628,9 +666,10 @@ struct ElimCtl {
   uint64_t zbar;
   uint64_t mbar[kElimWarps];
   uint32_t red[kElimThreads / 32];
-  uint32_t ok, bits, group, nlist, vec_signs;
+  uint32_t ok, bits, group, nlist, vec_signs, quant;
   uint64_t base, limit, seed;
   alignas(16) uint32_t mask[128];
+  float e2m1[16];  // FP4 code values
   uint32_t list[kElimThreads];
 };
 // Shared memory: per-warp staging | per-warp meta blocks | chunk | scratch |
@@ -650,7 +689,7 @@ struct ElimSmem {
   }
 };
 
-template <int D, int BITS, int G, class Layout>
+template <int D, int BITS, int G, class Layout, bool kFp4 = false>
 __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uint8_t *smem,
                           const uint32_t *cum) {
   using C = Cfg<D, BITS, G>;
@@ -737,7 +776,7 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
         uint32_t out[D / 2];
         const bool act = uint32_t(lane) < nv;
         if (act)
-          decode_vector<D, BITS, G>(ctl->mask, chunk + (b * 32 + lane) * C::CB,
+          decode_vector<D, BITS, G, kFp4>(ctl->mask, ctl->e2m1, chunk + (b * 32 + lane) * C::CB,
                                     mbuf + lane * C::MB, out);
         if constexpr (!kIsPaged<Layout>) {
           if (use_tma) {
@@ -777,11 +816,12 @@ __global__ void __launch_bounds__(kElimThreads, 1)
   ElimCtl *ctl = reinterpret_cast<ElimCtl *>(smem + S::ctl);
   uint32_t *s_cum = reinterpret_cast<uint32_t *>(smem + S::cum);
   const int tid = threadIdx.x;
-  if (a.in_bytes < kHeader || a.in[11] != 1) return;  // no code chunk uses elimination
+  if (a.in_bytes < kHeader || (a.in[11] & 1u) == 0) return;  // no code chunk uses elimination
   if (tid < kElimWarps) {
     mbar_init(&ctl->mbar[tid], 1);
     mbar_fence_init();
   }
+  if (tid < 16) ctl->e2m1[tid] = e2m1_value(uint32_t(tid));  // FP4 code values
   if (tid == 0) {
     mbar_init(&ctl->zbar, 1);
     mbar_fence_init();
@@ -792,6 +832,7 @@ __global__ void __launch_bounds__(kElimThreads, 1)
     ctl->base = h.data_base;
     ctl->limit = min(a.in_bytes, h.stream_bytes);
     ctl->vec_signs = h.vec_signs;
+    ctl->quant = h.quant;
     ctl->seed = h.seed;
     if (h.ok) sign_masks(h.seed, D, ctl->mask);
   }
@@ -801,6 +842,22 @@ __global__ void __launch_bounds__(kElimThreads, 1)
   __syncthreads();
   if (!ctl->ok) return;  // decode_kernel reports the header
   const uint32_t bits = ctl->bits, group = ctl->group;
+  if (ctl->quant == 2) {  // FP4
+    if constexpr (D == 128) {
+      if (group == 128)
+        elim_body<128, 4, 128, Layout, true>(a, lay, ctl, smem, s_cum);
+      else if (group == 64)
+        elim_body<128, 4, 64, Layout, true>(a, lay, ctl, smem, s_cum);
+      else
+        elim_body<128, 4, 32, Layout, true>(a, lay, ctl, smem, s_cum);
+    } else {
+      if (group == 64)
+        elim_body<64, 4, 64, Layout, true>(a, lay, ctl, smem, s_cum);
+      else
+        elim_body<64, 4, 32, Layout, true>(a, lay, ctl, smem, s_cum);
+    }
+    return;
+  }
   if constexpr (D == 128) {
     if (bits == 8 && group == 128)
       elim_body<128, 8, 128>(a, lay, ctl, smem, s_cum);

@@ -166,17 +166,63 @@ struct Enc : Cfg<D, BITS, G> {
   // group is always seen: four independent running minima and maxima keep
   // few values live next to the vector.
   static __device__ __forceinline__ void minmax(Pairs<D> &y, int g, float &mn, float &mx) {
+    minmax_at<G>(y, g * G, mn, mx);
+  }
+  // The same over channels c0 .. c0 + N - 1.
+  template <int N>
+  static __device__ __forceinline__ void minmax_at(Pairs<D> &y, int c0, float &mn, float &mx) {
     float lo[4], hi[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) lo[i] = hi[i] = y.at(g * G + i);
+    for (int i = 0; i < 4; ++i) lo[i] = hi[i] = y.at(c0 + i);
 #pragma unroll
-    for (int c = 4; c < G; ++c) {
-      const float u = y.at(g * G + c);
+    for (int c = 4; c < N; ++c) {
+      const float u = y.at(c0 + c);
       lo[c & 3] = min2n(lo[c & 3], u);
       hi[c & 3] = max2n(hi[c & 3], u);
     }
     mn = min2n(min2n(lo[0], lo[1]), min2n(lo[2], lo[3]));
     mx = max2n(max2n(hi[0], hi[1]), max2n(hi[2], hi[3]));
+  }
+
+  // E4..E7 of the FP4 quantizer (reading R22, 4-bit only): per group an fp16
+  // scale s2_h = RU16(fl(max|y| / 2688) * 2^-K) (2688 = 6 * 448), per
+  // half-group an e4m3 micro-scale s1 = RU(fl(max_half|y| / (6 * s2))), at
+  // most 448; S = s1 * s2 (exact), r = fl(1 / S) (0 for S = 0), code = e2m1
+  // nearest to fl(y * r), ties to even. Meta word: s2_h | s1_0 << 16 |
+  // s1_1 << 24. Each code leaves in the low bits of a float for the packer.
+  static __device__ __forceinline__ uint32_t quantize_fp4(Pairs<D> &y, uint32_t (&meta)[C::NG]) {
+    static_assert(BITS == 4, "FP4 codes are 4-bit");
+    uint32_t err = 0;
+    float rr[2 * C::NG];  // 1 / S per half-group
+    const float down = 1.0f / float(1 << C::K), up = float(1 << C::K);
+#pragma unroll
+    for (int g = 0; g < C::NG; ++g) {
+      float lo[2], hi[2];
+      minmax_at<G / 2>(y, g * G, lo[0], hi[0]);
+      minmax_at<G / 2>(y, g * G + G / 2, lo[1], hi[1]);
+      if (!(isfinite(lo[0]) && isfinite(hi[0]) && isfinite(lo[1]) && isfinite(hi[1]))) err |= 1u;
+      const float a0 = fmaxf(fabsf(lo[0]), fabsf(hi[0])), a1 = fmaxf(fabsf(lo[1]), fabsf(hi[1]));
+      const __half sh = __float2half_ru(__fmul_rn(__fdiv_rn(fmaxf(a0, a1), 2688.0f), down));
+      const uint16_t sb = __half_as_ushort(sh);
+      if ((sb & 0x7FFFu) == 0x7C00u) err |= 2u;
+      const float s2 = __fmul_rn(__half2float(sh), up);
+      uint32_t s1[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        s1[h] = s2 == 0.0f ? 0u : e4m3_ru(__fdiv_rn(h ? a1 : a0, __fmul_rn(6.0f, s2)));
+        const float S = __fmul_rn(e4m3_value(s1[h]), s2);
+        rr[2 * g + h] = S == 0.0f ? 0.0f : __frcp_rn(S);
+      }
+      meta[g] = uint32_t(sb) | (s1[0] << 16) | (s1[1] << 24);
+    }
+#pragma unroll
+    for (int j = 0; j < D / 2; ++j) {
+      const int ha = j / (G / 2), hb = (j + D / 2) / (G / 2);
+      const float2 p = mul2(y.p[j], make_float2(rr[ha], rr[hb]));
+      y.p[j] = make_float2(__uint_as_float(0x4B400000u | e2m1_rne(p.x)),
+                           __uint_as_float(0x4B400000u | e2m1_rne(p.y)));
+    }
+    return err;
   }
 
   // E3..E7. Reading R5: asymmetric min/max group quantization, fp16 zero
@@ -192,11 +238,12 @@ struct Enc : Cfg<D, BITS, G> {
   // [0, 2^b - 1] never acts for a finite group: t >= 0 since zf <= min, and
   // sf >= (max - zf) / (2^b - 1) keeps p below 2^b - 1 + 2^-18. Codes pack
   // LSB first (reading R6).
+  template <bool kFp4 = false>
   static __device__ __forceinline__ uint32_t vector(Pairs<D> &y, uint32_t (&code)[C::CW],
                                                     uint32_t (&meta)[C::NG], float one,
                                                     uint32_t sym) {
     fwht_pairs<D>(y);
-    return quantize(y, code, meta, one, sym);
+    return quantize<kFp4>(y, code, meta, one, sym);
   }
   // E4..E7 on the transformed vector. With `sym` (reading R19, symmetric
   // absmax): scale s_h = RU16(fl(max|y| / (2^(b-1) - 1)) * 2^-K), stored zero
@@ -205,10 +252,16 @@ struct Enc : Cfg<D, BITS, G> {
   // folded into the rounding constant (1.5 * 2^23 + 2^(b-1) is even, so ties
   // still go to even p) and the clamp to [-(2^(b-1) - 1), 2^(b-1) - 1] never
   // acts for a finite group (|p| <= max|y| / s32 * (1 + 2^-22)).
+  template <bool kFp4 = false>
   static __device__ __forceinline__ uint32_t quantize(Pairs<D> &y, uint32_t (&code)[C::CW],
                                                       uint32_t (&meta)[C::NG], float one,
                                                       uint32_t sym) {
     uint32_t err = 0;
+    if constexpr (kFp4) {
+      err = quantize_fp4(y, meta);
+      pack(y, code);
+      return err;
+    }
     float zf[C::NG], rr[C::NG];  // zf: subtracted before the product (0 when symmetric)
 #pragma unroll
     for (int g = 0; g < C::NG; ++g) {
@@ -247,6 +300,11 @@ struct Enc : Cfg<D, BITS, G> {
       const float2 p = mul2(t, make_float2(rr[ga], rr[gb]));
       y.p[j] = fma2(p, one2, mag);
     }
+    pack(y, code);
+    return err;
+  }
+  // E7: each code in the low bits of its float, packed LSB first (reading R6).
+  static __device__ __forceinline__ void pack(Pairs<D> &y, uint32_t (&code)[C::CW]) {
     constexpr int per = 8 / BITS;  // codes per byte
 #pragma unroll
     for (int W = 0; W < C::CW; ++W) {
@@ -261,7 +319,6 @@ struct Enc : Cfg<D, BITS, G> {
       }
       code[W] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     }
-    return err;
   }
 };
 
@@ -273,7 +330,7 @@ struct Enc : Cfg<D, BITS, G> {
 // of one bit plane, so it is nonzero iff that plane's bit is set in the OR
 // of the 64 words) and the meta counts after the XOR of each word with the
 // previous one, restarted at every run of 32 vectors (a block is one run).
-template <int D, int BITS, int G, bool kFwht, bool kSearch>
+template <int D, int BITS, int G, bool kFwht, bool kSearch, bool kFp4 = false>
 __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t blk, uint32_t v,
                                                     bool valid, Pairs<D> &y, uint32_t &err) {
   using C = Cfg<D, BITS, G>;
@@ -283,9 +340,9 @@ __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t b
   uint32_t code[C::CW], meta[C::NG];
   if (valid) {
     if constexpr (kFwht)
-      err |= E::vector(y, code, meta, a.one, a.sym);
+      err |= E::template vector<kFp4>(y, code, meta, a.one, a.sym);
     else
-      err |= E::quantize(y, code, meta, a.one, a.sym);
+      err |= E::template quantize<kFp4>(y, code, meta, a.one, a.sym);
     uint4 *cd = reinterpret_cast<uint4 *>(a.out + a.data_base + uint64_t(v) * C::CB);
 #pragma unroll
     for (int q = 0; q < C::CW / 4; ++q)
@@ -384,14 +441,16 @@ __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t b
 // ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
-// kVec: per-(layer, kv, head) sign diagonals (each lane derives its vector's
-// diagonal from the seed) instead of the one in the kernel's parameters.
-template <int D, int BITS, int G, class Layout, bool kNarrow, bool kSearch, bool kVec>
+// kVar bit 0: per-(layer, kv, head) sign diagonals (each lane derives its
+// vector's diagonal from the seed) instead of the one in the kernel's
+// parameters; bit 1: the FP4 quantizer (reading R22).
+template <int D, int BITS, int G, class Layout, bool kNarrow, bool kSearch, int kVar>
 __global__ void __launch_bounds__(kEncThreads, 1)
     encode_kernel(const __grid_constant__ EncArgs a, const __grid_constant__ Layout lay) {
   using C = Cfg<D, BITS, G>;
   using E = Enc<D, BITS, G>;
   constexpr bool kPaged = kIsPaged<Layout>;
+  constexpr bool kVec = (kVar & 1) != 0, kFp4 = (kVar & 2) != 0;
   using S = EncSmem<D, kPaged>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -429,7 +488,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
 
   uint32_t phase = 0, err = 0;
   auto finish_block = [&](uint32_t blk, uint32_t v, bool valid, Pairs<D> &y) {
-    encode_finish_block<D, BITS, G, true, kSearch>(a, blk, v, valid, y, err);
+    encode_finish_block<D, BITS, G, true, kSearch, kFp4>(a, blk, v, valid, y, err);
   };
   // E1/E2 of vector v from row `row` of the warp's buffer.
   auto unpack = [&](int row, uint32_t v, Pairs<D> &y) {

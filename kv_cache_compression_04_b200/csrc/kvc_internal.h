@@ -152,6 +152,43 @@ struct VectorSigns {
   }
 };
 
+#ifdef __CUDACC__
+// FP4 helpers (the dual-scale e2m1 quantizer). e4m3 (fn variant: bias 7,
+// 3 mantissa bits, largest finite 448, no inf) and e2m1 (bias 1, 1 mantissa
+// bit: 0, 0.5, 1, 1.5, 2, 3, 4, 6) from their bit patterns.
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  const float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : float(m) * (1.0f / 512.0f);
+  return (b & 0x80u) ? -v : v;
+}
+// The smallest e4m3 value >= x (0 <= x, finite), at most 448: normals round
+// the fp32 mantissa up to 3 bits (an integer add on the bit pattern),
+// subnormals (x < 2^-6) to a multiple of 2^-9; the byte is returned.
+__device__ __forceinline__ uint32_t e4m3_ru(float x) {
+  if (x < 0.015625f) return uint32_t(ceilf(x * 512.0f));  // 0..8 (8 = 2^-6, code 0x08)
+  const uint32_t u = (__float_as_uint(x) + 0xFFFFFu) & ~0xFFFFFu;
+  if (__uint_as_float(u) > 448.0f) return 0x7Eu;
+  return ((((u >> 23) & 255u) - 120u) << 3) | ((u >> 20) & 7u);
+}
+// e2m1 code -> fp32: magnitude index i = 2e + m, value 2^(e-1) (1 + m/2) for
+// e > 0, m/2 for e = 0; bit 3 is the sign.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t i = c & 7u, e = i >> 1, m = i & 1u;
+  const uint32_t mag = e ? (((e + 126u) << 23) | (m << 22)) : (m ? 0x3F000000u : 0u);
+  return __uint_as_float(mag | ((c & 8u) << 28));
+}
+// The e2m1 code nearest to p, ties to the even magnitude index, |p| > 6 to
+// 6; magnitude 0 is always code 0. Each comparison is one boundary of the
+// grid: ties at 0.25, 1.25, 2.5, 5 go down, at 0.75, 1.75, 3.5 up.
+__device__ __forceinline__ uint32_t e2m1_rne(float p) {
+  const float a = fabsf(p);
+  const uint32_t i = uint32_t(a > 0.25f) + uint32_t(a >= 0.75f) + uint32_t(a > 1.25f) +
+                     uint32_t(a >= 1.75f) + uint32_t(a > 2.5f) + uint32_t(a >= 3.5f) +
+                     uint32_t(a > 5.0f);
+  return i | ((i != 0u && p < 0.0f) ? 8u : 0u);
+}
+#endif
+
 // Unsigned 32-bit division by a run-time constant (Granlund and Montgomery,
 // "Division by invariant integers using multiplication", PLDI 1994, the
 // round-up variant): q = (umulhi(n, m) + n) >> s, exact for every n < 2^32.
@@ -223,6 +260,7 @@ struct EncArgs {
   uint32_t mode;       // KVC_LOSSLESS_*
   uint32_t sym;        // 1: symmetric absmax quantizer (KVC_QUANT_SYM)
   uint32_t vec_signs;  // 1: per-(layer, kv, head) sign diagonals
+  uint32_t fp4;        // 1: the FP4 quantizer (KVC_QUANT_FP4, 4-bit codes)
   uint64_t seed;       // sign seed (per-vector diagonals)
   FastDiv tdiv;        // tokens per (layer, kv, head): vector index = v / tokens
   uint32_t sign_mask[128];
@@ -322,6 +360,7 @@ struct AttnArgs {
   uint32_t *status;
   uint32_t layers, kv_heads, n_req, qpk;  // qpk: query heads per kv head
   uint32_t bits, group;                   // as the caller states them (checked)
+  uint32_t fp4;                           // 1: the FP4 quantizer (checked)
   uint64_t tokens;                        // all requests
   uint32_t V, splits;                     // vectors; CTAs per (layer, request, kv head)
   const uint16_t *q;                      // bf16 [layers][n_req][kv_heads * qpk][D]

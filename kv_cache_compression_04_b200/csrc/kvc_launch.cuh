@@ -44,9 +44,9 @@ inline cudaError_t prepare(Kernel k, size_t smem) {
   return e;
 }
 
-template <int D, int BITS, int G, class Layout, bool kNarrow, bool kSearch, bool kVec>
+template <int D, int BITS, int G, class Layout, bool kNarrow, bool kSearch, int kVar>
 cudaError_t launch_enc_k(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
-  auto k = encode_kernel<D, BITS, G, Layout, kNarrow, kSearch, kVec>;
+  auto k = encode_kernel<D, BITS, G, Layout, kNarrow, kSearch, kVar>;
   const size_t smem = enc_smem_bytes<D>(kIsPaged<Layout>);
   struct Tag {};
   cudaError_t e = prepare<Tag>(k, smem);
@@ -62,18 +62,18 @@ cudaError_t launch_enc_k(const EncArgs &a, const Layout &lay, int sms, cudaStrea
 // copies). Dense inputs keep the 64-bit gather next to their tensor-map
 // loads: both paths in one kernel would not fit its registers.
 // The search mode counts more per block (encode_finish_block's kSearch).
-template <int D, int BITS, int G, class Layout, bool kSearch, bool kVec>
+template <int D, int BITS, int G, class Layout, bool kSearch, int kVar>
 cudaError_t launch_enc_s(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
   if constexpr (kIsPaged<Layout>) {
-    if (lay.narrow) return launch_enc_k<D, BITS, G, Layout, true, kSearch, kVec>(a, lay, sms, st);
+    if (lay.narrow) return launch_enc_k<D, BITS, G, Layout, true, kSearch, kVar>(a, lay, sms, st);
   }
-  return launch_enc_k<D, BITS, G, Layout, false, kSearch, kVec>(a, lay, sms, st);
+  return launch_enc_k<D, BITS, G, Layout, false, kSearch, kVar>(a, lay, sms, st);
 }
-template <int D, int BITS, int G, class Layout, bool kVec>
+template <int D, int BITS, int G, class Layout, int kVar>
 cudaError_t launch_enc(const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
   return a.mode == KVC_LOSSLESS_SEARCH
-             ? launch_enc_s<D, BITS, G, Layout, true, kVec>(a, lay, sms, st)
-             : launch_enc_s<D, BITS, G, Layout, false, kVec>(a, lay, sms, st);
+             ? launch_enc_s<D, BITS, G, Layout, true, kVar>(a, lay, sms, st)
+             : launch_enc_s<D, BITS, G, Layout, false, kVar>(a, lay, sms, st);
 }
 
 template <int D, class Layout, bool kNarrow>
@@ -123,34 +123,40 @@ cudaError_t launch_dec(const DecArgs &a, const Layout &lay, int sms, cudaStream_
 }
 
 // The encode kernel for `group` at fixed head_dim and bits.
-template <int D, int BITS, bool kVec, class Layout>
+template <int D, int BITS, int kVar, class Layout>
 cudaError_t launch_enc_g(int group, const EncArgs &a, const Layout &lay, int sms, cudaStream_t st) {
   if constexpr (D == 128) {
-    if (group == 128) return launch_enc<D, BITS, 128, Layout, kVec>(a, lay, sms, st);
+    if (group == 128) return launch_enc<D, BITS, 128, Layout, kVar>(a, lay, sms, st);
   }
-  if (group == 64) return launch_enc<D, BITS, 64, Layout, kVec>(a, lay, sms, st);
-  if (group == 32) return launch_enc<D, BITS, 32, Layout, kVec>(a, lay, sms, st);
+  if (group == 64) return launch_enc<D, BITS, 64, Layout, kVar>(a, lay, sms, st);
+  if (group == 32) return launch_enc<D, BITS, 32, Layout, kVar>(a, lay, sms, st);
   return cudaErrorInvalidValue;
 }
 
-// 2- and 4-bit codes with the global sign diagonal here; 8-bit codes and
-// per-vector diagonals in the `_var` launchers (their own translation units).
+// 2- and 4-bit codes of the min/max and absmax quantizers with the global
+// sign diagonal here; 8-bit codes, per-vector diagonals and the FP4
+// quantizer in the `_var` launchers (their own translation units).
 template <int D, class Layout, class Var>
 cudaError_t launch_enc_dispatch(int bits, int group, const EncArgs &a, const Layout &lay, int sms,
                                 cudaStream_t st, Var var) {
-  if (a.vec_signs || bits == 8) return var(bits, group, a, lay, sms, st);
-  if (bits == 4) return launch_enc_g<D, 4, false>(group, a, lay, sms, st);
-  if (bits == 2) return launch_enc_g<D, 2, false>(group, a, lay, sms, st);
+  if (a.vec_signs || a.fp4 || bits == 8) return var(bits, group, a, lay, sms, st);
+  if (bits == 4) return launch_enc_g<D, 4, 0>(group, a, lay, sms, st);
+  if (bits == 2) return launch_enc_g<D, 2, 0>(group, a, lay, sms, st);
   return cudaErrorInvalidValue;
 }
 template <int D, class Layout>
 cudaError_t launch_enc_dispatch_var(int bits, int group, const EncArgs &a, const Layout &lay,
                                     int sms, cudaStream_t st) {
+  if (a.fp4) {
+    if (bits != 4) return cudaErrorInvalidValue;
+    return a.vec_signs ? launch_enc_g<D, 4, 3>(group, a, lay, sms, st)
+                       : launch_enc_g<D, 4, 2>(group, a, lay, sms, st);
+  }
   if (!a.vec_signs)
-    return bits == 8 ? launch_enc_g<D, 8, false>(group, a, lay, sms, st) : cudaErrorInvalidValue;
-  if (bits == 8) return launch_enc_g<D, 8, true>(group, a, lay, sms, st);
-  if (bits == 4) return launch_enc_g<D, 4, true>(group, a, lay, sms, st);
-  if (bits == 2) return launch_enc_g<D, 2, true>(group, a, lay, sms, st);
+    return bits == 8 ? launch_enc_g<D, 8, 0>(group, a, lay, sms, st) : cudaErrorInvalidValue;
+  if (bits == 8) return launch_enc_g<D, 8, 1>(group, a, lay, sms, st);
+  if (bits == 4) return launch_enc_g<D, 4, 1>(group, a, lay, sms, st);
+  if (bits == 2) return launch_enc_g<D, 2, 1>(group, a, lay, sms, st);
   return cudaErrorInvalidValue;
 }
 

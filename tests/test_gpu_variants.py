@@ -1,5 +1,6 @@
-"""The quantizer variants on the GPU against the oracle (readings R19-R21:
-symmetric absmax, 8-bit codes, per-(layer, kv, head) sign diagonals): every
+"""The quantizer variants on the GPU against the oracle (readings R19-R22:
+symmetric absmax, 8-bit codes, per-(layer, kv, head) sign diagonals, FP4
+e2m1 codes with dual scales): every
 stream byte equal, the oracle's stream decoded on the GPU to the oracle's
 bf16 values bit for bit, attention over such streams within the attention
 tolerance, for dense and paged inputs, every group size, both lossless
@@ -17,14 +18,15 @@ from kvc_testutil import first_diff, gpu_compress, gpu_decompress, oracle_desc, 
 
 pytestmark = pytest.mark.gpu
 
-SYM, VEC = kvc.KVC_QUANT_SYM, kvc.KVC_SIGNS_PER_VECTOR
+SYM, FP4, VEC = kvc.KVC_QUANT_SYM, kvc.KVC_QUANT_FP4, kvc.KVC_SIGNS_PER_VECTOR
 THREADS = max(1, min(os.cpu_count() or 1, 64))
 
 
-def _dense(d, bits, g, L, H, T, quant=0, signs=0, lossless=0, seed=5, kind="lognormal"):
-    w = synth.Workload("v", L, H, d, bits, g, seed=L * 31 + T, kind=kind, scale_sigma=1.5,
-                       tokens=T)
-    kv = synth.dense_kv(w).cuda()
+def _dense(d, bits, g, L, H, T, quant=0, signs=0, lossless=0, seed=5, kind="lognormal", kv=None):
+    if kv is None:
+        w = synth.Workload("v", L, H, d, bits, g, seed=L * 31 + T, kind=kind, scale_sigma=1.5,
+                           tokens=T)
+        kv = synth.dense_kv(w).cuda()
     x = u16(kv).reshape(-1, d)
     od = oracle_desc(bits, g, d, L, H, [T], seed, 0, lossless, quant, signs)
     ost, ostream = oracle.compress(od, x, threads=THREADS)
@@ -48,6 +50,14 @@ def _dense(d, bits, g, L, H, T, quant=0, signs=0, lossless=0, seed=5, kind="logn
 def test_symmetric_dense(d, bits, g, L, H, T):
     s = _dense(d, bits, g, L, H, T, quant=SYM)
     assert s[11] & 6 == 2
+
+
+@pytest.mark.parametrize("d,g,L,H,T,signs", [
+    (128, 32, 2, 3, 1000, 0), (128, 64, 2, 2, 777, VEC), (128, 128, 1, 4, 1111, 0),
+    (64, 32, 2, 3, 999, VEC), (64, 64, 2, 2, 1300, 0)])
+def test_fp4_dense(d, g, L, H, T, signs):
+    s = _dense(d, 4, g, L, H, T, quant=FP4, signs=signs, kind="outlier_t")
+    assert s[11] & 6 == 4
 
 
 @pytest.mark.parametrize("d,bits,g,L,H,T", [
@@ -74,7 +84,7 @@ def test_variants_combined_search_mode():
 
 
 @pytest.mark.parametrize("bits,g,quant,signs", [(4, 64, SYM, VEC), (8, 32, 0, VEC),
-                                                (8, 128, SYM, 0)])
+                                                (8, 128, SYM, 0), (4, 32, FP4, VEC)])
 def test_variants_paged(bits, g, quant, signs):
     seq = [20, 0, 33, 700, 16, 257]
     w = synth.Workload("p", 2, 3, 128, bits, g, seed=3, kind="lognormal", scale_sigma=1.5,
@@ -103,7 +113,7 @@ def test_unfused_variants():
     w = synth.Workload("u", 2, 2, 128, 8, 64, seed=4, kind="lognormal", tokens=700)
     kv = synth.dense_kv(w).cuda()
     desc = kvc.dense_desc(kv)
-    for bits, g, quant in [(8, 64, 0), (4, 32, SYM), (8, 128, SYM)]:
+    for bits, g, quant in [(8, 64, 0), (4, 32, SYM), (8, 128, SYM)]:  # FP4: refused below
         p = kvc.params(bits, g, 3, 0, quant)
         cap = kvc.kvc_max_compressed_bytes(desc, p)
         outs = []
@@ -124,10 +134,29 @@ def test_unfused_variants():
     out = torch.zeros(kvc.kvc_max_compressed_bytes(desc, p), dtype=torch.uint8, device="cuda")
     assert kvc.kvc_compress_unfused(desc, p, out.data_ptr(), out.numel(), None, ws.data_ptr(),
                                     wsb, kvc._stream_ptr(None)) == kvc.KVC_ERR_UNSUPPORTED
+    p = kvc.params(4, 64, 3, 0, FP4)
+    assert kvc.kvc_compress_unfused(desc, p, out.data_ptr(), out.numel(), None, ws.data_ptr(),
+                                    wsb, kvc._stream_ptr(None)) == kvc.KVC_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("bits,g,quant,signs", [(4, 128, SYM, VEC), (4, 64, FP4, VEC),
+                                                (8, 32, 0, VEC), (4, 32, FP4, 0)])
+def test_variants_with_eliminated_code_chunks(bits, g, quant, signs):
+    """Half of the 256-token blocks all zero: code chunks stored eliminated
+    (header flag bit 0 next to the variant's bits), compacted by the encoder
+    and expanded by the eliminated-chunk decoder."""
+    L, H, T, D = 2, 8, 4096, 128
+    gen = torch.Generator().manual_seed(21)
+    x = torch.randn(L, 2, H, T, D, generator=gen)
+    blocks = x.view(L, 2, H, T // 256, 256, D)
+    blocks[torch.rand(L, 2, H, T // 256, generator=gen) < 0.5] = 0
+    s = _dense(D, bits, g, L, H, T, quant=quant, signs=signs, kv=x.to(torch.bfloat16).cuda())
+    assert s[11] & 1, "some code chunk stored eliminated"
 
 
 @pytest.mark.parametrize("bits,g,quant,signs,qpk", [(4, 128, SYM, 0, 4), (2, 32, 0, VEC, 7),
-                                                    (8, 64, SYM, VEC, 2), (8, 32, 0, 0, 8)])
+                                                    (8, 64, SYM, VEC, 2), (8, 32, 0, 0, 8),
+                                                    (4, 64, FP4, VEC, 4), (4, 32, FP4, 0, 1)])
 def test_attend_over_variant_streams(bits, g, quant, signs, qpk):
     L, H, T, d = 2, 2, 900, 128
     w = synth.Workload("a", L, H, d, bits, g, seed=12, kind="lognormal", scale_sigma=1.5,
@@ -138,7 +167,7 @@ def test_attend_over_variant_streams(bits, g, quant, signs, qpk):
     q = torch.randn(L, 1, H * qpk, d, generator=torch.Generator(device="cuda").manual_seed(1),
                     device="cuda").to(torch.bfloat16)
     out = torch.full((L, 1, H * qpk, d), float("nan"), device="cuda")
-    ad = kvc.attn_desc(L, H, qpk, bits, g, [T], q, out, d ** -0.5)
+    ad = kvc.attn_desc(L, H, qpk, bits, g, [T], q, out, d ** -0.5, quant=quant)
     ws = torch.empty(kvc.kvc_attend_workspace_bytes(ad), dtype=torch.uint8, device="cuda")
     sp = kvc._stream_ptr(None)
     assert kvc.kvc_attend(gbuf.data_ptr(), n, ad, ws.data_ptr(), ws.numel(), sp) == kvc.KVC_OK
@@ -157,7 +186,7 @@ def test_attend_over_variant_streams(bits, g, quant, signs, qpk):
 
 
 @pytest.mark.parametrize("bits,g,quant,signs", [(4, 128, SYM, 0), (4, 128, 0, VEC),
-                                                (8, 128, 0, 0)])
+                                                (8, 128, 0, 0), (4, 128, FP4, 0)])
 def test_full_llama8b_variant(bits, g, quant, signs):
     """The Llama-3-8B-shaped cache (32 x 2 x 8 x 4096 x 128) in each variant,
     compared whole: stream bytes and decoded values."""
