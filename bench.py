@@ -478,7 +478,7 @@ def job_gbs(raw_bytes_per_rank: int, world: int, ms: float) -> float:
 
 # ------------------------------------------------------------------ main --
 def time_config(wname: str, dev, steps: int, warmup: int, hbm: float, flush=None,
-                brief: bool = False):
+                brief: bool = False, variant: dict | None = None):
     """kvc_compress and kvc_decompress of one workload resident in HBM, timed
     like the headline step (CUDA events on the launching stream around each
     call, after `warmup` untimed steps; with `flush`, a write of it before
@@ -488,7 +488,10 @@ def time_config(wname: str, dev, steps: int, warmup: int, hbm: float, flush=None
     import torch
     import kv_cache_compression_04_b200 as kvc
     w, desc, out_desc_fn, keep = make_input(wname, dev, 0)
-    codec = kvc.Codec(w.bits, w.group, w.sign_seed)
+    v = variant or {}
+    w.bits, w.group = v.get("bits", w.bits), v.get("group", w.group)
+    codec = kvc.Codec(w.bits, w.group, w.sign_seed, quant=v.get("quant", 0),
+                      signs=v.get("signs", 0))
     out, ws, nb = codec.buffers(desc, dev)
     odesc, obuf = out_desc_fn()
     dws = torch.empty(kvc.kvc_decompress_workspace_bytes(odesc), dtype=torch.uint8, device=dev)
@@ -575,6 +578,14 @@ def time_config(wname: str, dev, steps: int, warmup: int, hbm: float, flush=None
     del keep, out, ws, nb, obuf, dws
     torch.cuda.empty_cache()
     return r
+
+
+# Quantizer variants timed on the Llama-3-8B-shaped cache (same call, same
+# timing as the per-config lines).
+VARIANTS = {"symmetric_4bit_g128": {"quant": 1},
+            "fp4_e2m1_g128": {"quant": 2},
+            "8bit_g128": {"bits": 8},
+            "per_vector_signs_4bit_g128": {"signs": 1}}
 
 
 # query heads per kv head of the model each workload is shaped after
@@ -953,6 +964,8 @@ def main():
     ap.add_argument("--unfused-steps", type=int, default=20)
     ap.add_argument("--attend", type=int, default=1,
                     help="1: also time decode attention over each compressed cache")
+    ap.add_argument("--variants", type=int, default=1,
+                    help="1: also time the quantizer variants on the llama8b cache")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--pipeline", action="store_true")
     args = ap.parse_args()
@@ -1107,6 +1120,10 @@ def main():
             per_config["attend_" + args.workload] = time_attend(args.workload, dev,
                                                                 args.config_steps, args.warmup,
                                                                 hbm_)
+        if args.variants:
+            per_config["variants_llama8b"] = {
+                name: time_config("llama8b", dev, args.config_steps, args.warmup, hbm_,
+                                  brief=True, variant=v) for name, v in VARIANTS.items()}
         if args.sweep_points:
             flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
             per_config["sweep"] = [time_config(f"sweep-{i}-{b}", dev, args.config_steps,
