@@ -351,6 +351,9 @@ typedef struct {
   int32_t bits;               /* as compressed */
   int32_t group_size;         /* as compressed */
   int32_t quant;              /* as compressed (KVC_QUANT_*; ASYM and SYM alike) */
+  int32_t kernel;             /* 0: tensor cores (2- and 4-bit ASYM / SYM codes, 2..8
+                                 query heads per kv head), CUDA cores otherwise;
+                                 1: CUDA cores always (for comparison) */
   int32_t n_requests;         /* 1 .. KVC_MAX_REQUESTS */
   float scale;                /* e.g. 1 / sqrt(head_dim) */
   const int32_t *seq_lens;    /* HOST [n_requests] */

@@ -57,7 +57,8 @@ KVC_LOSSLESS_FIXED, KVC_LOSSLESS_SEARCH, KVC_LOSSLESS_NONE = range(3)
 class kvc_attn_desc(C.Structure):
     _fields_ = [("layers", C.c_int32), ("kv_heads", C.c_int32), ("head_dim", C.c_int32),
                 ("q_per_kv", C.c_int32), ("bits", C.c_int32), ("group_size", C.c_int32),
-                ("quant", C.c_int32), ("n_requests", C.c_int32), ("scale", C.c_float),
+                ("quant", C.c_int32), ("kernel", C.c_int32), ("n_requests", C.c_int32),
+                ("scale", C.c_float),
                 ("seq_lens", C.POINTER(C.c_int32)), ("q", C.c_void_p), ("out", C.c_void_p)]
 
 
@@ -196,12 +197,12 @@ def kvc_decompress_timed(in_ptr, in_bytes, desc, ws_ptr, ws_bytes, events, strea
 
 
 def attn_desc(layers, kv_heads, q_per_kv, bits, group, seq_lens, q, out, scale,
-              head_dim: int = 128, quant: int = 0) -> kvc_attn_desc:
+              head_dim: int = 128, quant: int = 0, kernel: int = 0) -> kvc_attn_desc:
     """Descriptor of kvc_attend: q bf16 [layers, n_requests, kv_heads * q_per_kv,
     head_dim] and out fp32 of the same shape (device tensors)."""
     seq = (C.c_int32 * max(len(seq_lens), 1))(*[int(x) for x in seq_lens])
-    d = kvc_attn_desc(layers, kv_heads, head_dim, q_per_kv, bits, group, quant, len(seq_lens),
-                      float(scale), C.cast(seq, C.POINTER(C.c_int32)), q.data_ptr(),
+    d = kvc_attn_desc(layers, kv_heads, head_dim, q_per_kv, bits, group, quant, kernel,
+                      len(seq_lens), float(scale), C.cast(seq, C.POINTER(C.c_int32)), q.data_ptr(),
                       out.data_ptr())
     d._keep = (seq, q, out)
     return d

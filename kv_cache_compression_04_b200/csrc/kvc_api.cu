@@ -512,6 +512,7 @@ kvc_status attn_shape(const kvc_attn_desc *at, AttnShape &r) {
   if (!at) return KVC_ERR_INVALID_ARG;
   if (at->head_dim != 128) return KVC_ERR_UNSUPPORTED;
   if (at->q_per_kv < 1 || at->q_per_kv > 8) return KVC_ERR_UNSUPPORTED;
+  if (at->kernel != 0 && at->kernel != 1) return KVC_ERR_INVALID_ARG;
   if (at->n_requests < 1 || at->n_requests > KVC_MAX_REQUESTS || !at->seq_lens)
     return KVC_ERR_INVALID_ARG;
   // the stream's logical shape as a paged description without pages: the
@@ -592,6 +593,7 @@ kvc_status kvc_attend(const void *in, size_t in_bytes, const kvc_attn_desc *at, 
   a.bits = uint32_t(at->bits);
   a.group = uint32_t(at->group_size);
   a.fp4 = at->quant == KVC_QUANT_FP4 ? 1u : 0u;
+  a.cuda_cores = at->kernel == 1 ? 1u : 0u;
   a.tokens = r.s.T;
   a.V = d.V;
   a.splits = r.splits;

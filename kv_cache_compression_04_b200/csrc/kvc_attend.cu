@@ -1,6 +1,7 @@
 // Launches of kvc_attend: meta chunk expansion (shared with the decoder),
 // the split-K attention kernel, the combining kernel.
 #include "kvc_attend.cuh"
+#include "kvc_attend_mma.cuh"
 #include "kvc_launch.cuh"
 
 namespace kvc {
@@ -9,6 +10,16 @@ namespace {
 
 template <int BITS, int G, int QPK>
 cudaError_t launch_att_k(const AttnArgs &a, int units, cudaStream_t st) {
+  // 2- and 4-bit codes of the affine quantizers: tensor cores (query heads
+  // in tiles of 4); 8-bit and FP4 codes: CUDA cores
+  if constexpr (BITS != 8 && QPK >= 2) {
+    if (!a.fp4 && !a.cuda_cores) {
+      attend_mma_kernel<BITS, G, QPK < 4 ? 4 : QPK><<<units * a.splits, kAttThreads, 0, st>>>(a);
+      const cudaError_t e = cudaGetLastError();
+      timing_mark(st);
+      return e;
+    }
+  }
   if constexpr (BITS == 4) {
     if (a.fp4)
       attend_kernel<128, 4, G, QPK, true><<<units * a.splits, kAttThreads, 0, st>>>(a);

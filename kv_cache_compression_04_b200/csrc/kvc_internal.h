@@ -361,6 +361,7 @@ struct AttnArgs {
   uint32_t layers, kv_heads, n_req, qpk;  // qpk: query heads per kv head
   uint32_t bits, group;                   // as the caller states them (checked)
   uint32_t fp4;                           // 1: the FP4 quantizer (checked)
+  uint32_t cuda_cores;                    // 1: the CUDA-core kernel (measurement)
   uint64_t tokens;                        // all requests
   uint32_t V, splits;                     // vectors; CTAs per (layer, request, kv head)
   const uint16_t *q;                      // bf16 [layers][n_req][kv_heads * qpk][D]

@@ -38,7 +38,7 @@ def _stream(w, lossless):
     return st, s, gbuf, n, od
 
 
-def _check(w, qpk, lossless=0, seed=3):
+def _check(w, qpk, lossless=0, seed=3, kernel=0):
     L, H, d = w.layers, w.kv_heads, 128
     lens = list(w.seq_lens) if w.paged else [w.tokens]
     dev = torch.device("cuda", 0)
@@ -50,7 +50,7 @@ def _check(w, qpk, lossless=0, seed=3):
     q = torch.randn(L, n_req, H * qpk, d, generator=g, device=dev).to(torch.bfloat16)
     out = torch.full((L, n_req, H * qpk, d), float("nan"), device=dev)
     scale = 1.0 / np.sqrt(d)
-    ad = kvc.attn_desc(L, H, qpk, w.bits, w.group, lens, q, out, scale)
+    ad = kvc.attn_desc(L, H, qpk, w.bits, w.group, lens, q, out, scale, kernel=kernel)
     wsb = kvc.kvc_attend_workspace_bytes(ad)
     assert wsb > 0
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
@@ -78,23 +78,25 @@ def _check(w, qpk, lossless=0, seed=3):
     return worst
 
 
+@pytest.mark.parametrize("kernel", [0, 1])   # tensor cores where supported / CUDA cores
 @pytest.mark.parametrize("bits,g", [(4, 128), (4, 64), (4, 32), (2, 128), (2, 64), (2, 32)])
-@pytest.mark.parametrize("qpk", [1, 4, 8])
-def test_attend_dense_one_request(bits, g, qpk):
+@pytest.mark.parametrize("qpk", [1, 2, 4, 8])
+def test_attend_dense_one_request(bits, g, qpk, kernel):
     w = synth.Workload("a", 2, 2, 128, bits, g, seed=bits * 7 + g, kind="lognormal",
                        scale_sigma=1.5, tokens=1000)
-    _check(w, qpk)
+    _check(w, qpk, kernel=kernel)
 
 
+@pytest.mark.parametrize("kernel", [0, 1])
 @pytest.mark.parametrize("qpk", [3, 7])
-def test_attend_several_requests_and_search_mode(qpk):
+def test_attend_several_requests_and_search_mode(qpk, kernel):
     """A paged cache with requests of 0, 1, 255, 256, 257 and 700 tokens
     (split boundaries), meta chunks through the search mode's XOR pipelines,
     and a query-head count per kv head that is not a power of two (7: the
     28 query / 4 kv heads of a Qwen2-7B-shaped model)."""
     w = synth.Workload("a", 2, 2, 128, 2, 32, seed=9, kind="outlier_t",
                        seq_lens=[0, 1, 255, 256, 257, 700])
-    _check(w, qpk, lossless=kvc.KVC_LOSSLESS_SEARCH)
+    _check(w, qpk, lossless=kvc.KVC_LOSSLESS_SEARCH, kernel=kernel)
 
 
 def test_attend_rejects_eliminated_code_chunks_and_bad_arguments():
@@ -120,9 +122,18 @@ def test_attend_rejects_eliminated_code_chunks_and_bad_arguments():
     assert kvc.kvc_stream_status(ws2.data_ptr(), sp) == kvc.KVC_ERR_CORRUPT
 
 
-def test_attend_full_llama8b():
+@pytest.mark.parametrize("kernel", [0, 1])
+def test_attend_full_llama8b(kernel):
     """The Llama-3-8B-shaped cache (32 layers, 8 kv heads, 4096 tokens) with
     32 query heads (4 per kv head)."""
     w = synth.workload("llama8b")
-    worst = _check(w, 4)
+    worst = _check(w, 4, kernel=kernel)
+    print(f"worst error / max|v|: {worst:.3g}")
+
+
+def test_attend_full_qwen7b():
+    """The Qwen-7B-shaped cache (28 layers, 4 kv heads, 32768 tokens, 2-bit
+    group 32) with 28 query heads (7 per kv head): 128 splits per head."""
+    w = synth.workload("qwen7b")
+    worst = _check(w, 7)
     print(f"worst error / max|v|: {worst:.3g}")
