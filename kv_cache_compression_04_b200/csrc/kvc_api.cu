@@ -505,7 +505,7 @@ constexpr int kAttTokHost = 256;  // tokens per attention CTA (kvc_attend.cuh: k
 // meta chunks | split partials.
 struct AttnShape {
   Shape s;
-  uint64_t meta_off, meta_chunks, part_off, total;
+  uint64_t meta_off, meta_chunks, part_off, prep_off, total;
   uint32_t splits, units;
 };
 kvc_status attn_shape(const kvc_attn_desc *at, AttnShape &r) {
@@ -545,8 +545,9 @@ kvc_status attn_shape(const kvc_attn_desc *at, AttnShape &r) {
   // group fails the header check; meta expansion never exceeds the slots)
   r.meta_chunks = (r.s.V * uint64_t(at->head_dim / at->group_size) * 4 + kChunk - 1) / kChunk;
   r.part_off = round256(r.meta_off + r.meta_chunks * kChunk);
-  r.total = r.part_off + uint64_t(r.units) * r.splits * uint64_t(at->q_per_kv) *
-                             (uint64_t(at->head_dim) + 4) * sizeof(float);
+  r.prep_off = round256(r.part_off + uint64_t(r.units) * r.splits * uint64_t(at->q_per_kv) *
+                                         (uint64_t(at->head_dim) + 4) * sizeof(float));
+  r.total = r.prep_off + prep_bytes(uint32_t(r.meta_chunks), r.units);
   return KVC_OK;
 }
 }  // namespace
@@ -602,6 +603,8 @@ kvc_status kvc_attend(const void *in, size_t in_bytes, const kvc_attn_desc *at, 
   a.out = at->out;
   a.part = reinterpret_cast<float *>(ws + r.part_off);
   a.ws_meta = d.ws_meta;
+  a.prep = ws + r.prep_off;
+  a.n_meta = uint32_t(r.meta_chunks);
   a.cum[0] = 0;
   for (int i = 0; i < at->n_requests; ++i) a.cum[i + 1] = a.cum[i] + uint32_t(at->seq_lens[i]);
   if (clear_words(workspace, kWsCtl, sms, cs) != cudaSuccess) return KVC_ERR_CUDA;

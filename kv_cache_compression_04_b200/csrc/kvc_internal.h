@@ -369,9 +369,22 @@ struct AttnArgs {
   float *out;                             // fp32, the shape of q
   float *part;                            // per CTA and query head: m, l, o[D]
   const uint8_t *ws_meta;                 // meta chunks expanded by meta_expand_kernel
+  uint8_t *prep;                          // tensor-core path: attend_prep_kernel's results
+  uint32_t n_meta;                        // meta chunks
   uint32_t cum[KVC_MAX_REQUESTS + 1];     // token prefix per request
 };
 cudaError_t launch_attend(const AttnArgs &a, const DecArgs &d, int sms, cudaStream_t st);
+// The tensor-core attention's preparation area (kvc_attend_mma.cuh).
+struct PrepCtl {
+  uint64_t base;
+  uint32_t n_code;
+};
+KVC_HD uint64_t prep_qfrag_off(uint32_t n_meta) {
+  return (64 + 8 * uint64_t(n_meta) + 255) & ~uint64_t(255);
+}
+KVC_HD uint64_t prep_bytes(uint32_t n_meta, uint32_t units) {
+  return prep_qfrag_off(n_meta) + uint64_t(units) * (4096 + 256);
+}
 cudaError_t launch_finish_paged(const FinArgs &a, const PagedLayout &lay, int sms, cudaStream_t st);
 
 }  // namespace kvc

@@ -29,6 +29,24 @@ inline cudaError_t launch_after(void (*k)(KArgs...), int grid, int threads, size
   return e;
 }
 
+// launch_after without the timing mark: the kernel's time is counted in the
+// interval of the launch that follows it.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_after_unmarked(void (*k)(KArgs...), int grid, int threads, size_t smem,
+                                         cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(unsigned(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kernel_timing().events ? 0 : 1;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
+
 // Opt each instantiation into large dynamic shared memory once per device.
 // `Tag` makes the flag per kernel instantiation (kernels share a pointer type).
 template <class Tag, class Kernel>
