@@ -342,7 +342,8 @@ kvc_status kvc_compress_unfused(const kvc_kv_desc *kv, const kvc_params *params,
  * [kv_heads * q_per_kv][128], contiguous; out: DEVICE fp32 of the same shape
  * (zeros for a request without tokens). seq_lens: HOST, the stream's
  * per-request token counts. q_per_kv 1 to 8. The workspace holds the
- * status word, the expanded meta chunks and the split partials. */
+ * status word, the expanded meta chunks, the split partials and (tensor-core
+ * path) each (layer, request, kv head)'s prepared query fragments. */
 typedef struct {
   int32_t layers;
   int32_t kv_heads;

@@ -272,7 +272,9 @@ class _Ptr:
 def test_attend_refuses_bad_arguments_and_sizes_its_workspace(L):
     """kvc_attend / kvc_attend_workspace_bytes on the host side: shape and
     pointer checks, and the workspace size (status words, one 16 KB slot per
-    meta chunk, one partial record of 4 + 128 floats per CTA and query head)."""
+    meta chunk, one partial record of 4 + 128 floats per CTA and query head,
+    the tensor-core path's 4 KB of query fragments and 256 bytes of sums per
+    (layer, request, kv head) and one address per meta chunk)."""
     q, out = _Ptr(FAKE), _Ptr(FAKE)
     lens = [1000, 0, 513]
     ad = kvc.attn_desc(2, 8, 4, 4, 64, lens, q, out, 0.1)
@@ -281,8 +283,9 @@ def test_attend_refuses_bad_arguments_and_sizes_its_workspace(L):
     n_meta = -(-V * 8 // 16384)            # 2 groups of 4 bytes per vector
     splits = -(-1000 // 256)
     parts = 2 * 3 * 8 * splits * 4 * 132 * 4
-    assert wsb >= n_meta * 16384 + parts
-    assert wsb <= n_meta * 16384 + parts + 4096
+    prep = 2 * 3 * 8 * (4096 + 256) + 64 + 8 * n_meta   # query fragments and sums per unit
+    assert wsb >= n_meta * 16384 + parts + prep
+    assert wsb <= n_meta * 16384 + parts + prep + 4096
     for bad, why in [(kvc.attn_desc(2, 8, 0, 4, 64, lens, q, out, 0.1), "q_per_kv 0"),
                      (kvc.attn_desc(2, 8, 9, 4, 64, lens, q, out, 0.1), "q_per_kv 9"),
                      (kvc.attn_desc(2, 8, 4, 3, 64, lens, q, out, 0.1), "bits 3"),
