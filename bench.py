@@ -23,6 +23,9 @@ the only collectives are a barrier and a max over ranks of the timings.
 of 1 MiB .. 4 GiB, 4-bit g128 and 2-bit g32, one JSON line per point.
 `--pipeline` times a layer-pipelined transfer of the llama8b cache over a
 simulated 100 and 400 Gbit/s link instead (1 GPU), one JSON line per speed.
+After the timed region (1 GPU), `per_config` also holds decode attention over
+each compressed cache (kvc_attend against decompress + torch attention) and
+the quantizer variants on the llama8b cache.
 """
 from __future__ import annotations
 
@@ -1106,7 +1109,7 @@ def main():
     # -------------------------- the other workloads, timed the same way --
     # (after the timed region, with the headline workload's buffers freed)
     per_config = None
-    if world == 1 and args.per_config:
+    if world == 1 and (args.per_config or args.attend or args.variants or args.sweep_points):
         del out, ws, nb, obuf, dws, keep
         torch.cuda.empty_cache()
         hbm_, _ = peaks()
