@@ -16,8 +16,8 @@ cudaError_t launch_att_k(const AttnArgs &a, int units, cudaStream_t st) {
     if (!a.fp4 && !a.cuda_cores) {
       // the per-call and per-unit preparation, then the attention (dependent
       // launches; the preparation's time counts in the attention's interval)
-      cudaError_t e = launch_after_unmarked(attend_prep_kernel<BITS, G>, units + 1, kAttThreads,
-                                            0, st, a);
+      cudaError_t e = launch_after_unmarked(attend_prep_kernel<BITS, G, (QPK <= 4)>, units + 1,
+                                            kAttThreads, 0, st, a);
       if (e != cudaSuccess) return e;
       return launch_after(attend_mma_kernel<BITS, G, QPK < 4 ? 4 : QPK>, units * int(a.splits),
                           kAttThreads, 0, st, a);

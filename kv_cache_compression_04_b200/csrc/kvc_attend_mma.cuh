@@ -90,7 +90,11 @@ struct AttnMmaSmem {
 // group sums, the power-of-two scale 2^eq of the fp16 split and the lanes'
 // B fragments of the score products. The attention CTAs of a unit (one per
 // 256-token split) then start from these.
-template <int BITS, int G>
+// kPairs (4 query heads per kv head): the score product's 8 columns are
+// (head, hi / lo) pairs, column n = 2 * head + part, so one product per
+// k-block carries both parts; otherwise the columns are 8 heads and the hi
+// and lo parts are two products.
+template <int BITS, int G, bool kPairs>
 __global__ void __launch_bounds__(kAttThreads) attend_prep_kernel(const __grid_constant__ AttnArgs a) {
   constexpr int D = 128;
   using C = Cfg<D, BITS, G>;
@@ -212,10 +216,16 @@ __global__ void __launch_bounds__(kAttThreads) attend_prep_kernel(const __grid_c
     const int kb = 2 * warp + i;
     float hi[4], lo[4];
     const int ks[4] = {2 * tq, 2 * tq + 1, 2 * tq + 8, 2 * tq + 9};
+    const int head = kPairs ? gq >> 1 : gq;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) split_f16(qt[gq][score_ch(kb, ks[k])] * es, hi[k], lo[k]);
-    qf[kb * 32 + lane] = make_uint4(f16x2(hi[0], hi[1]), f16x2(hi[2], hi[3]), f16x2(lo[0], lo[1]),
-                                    f16x2(lo[2], lo[3]));
+    for (int k = 0; k < 4; ++k) split_f16(qt[head][score_ch(kb, ks[k])] * es, hi[k], lo[k]);
+    if constexpr (kPairs) {  // column gq = (head gq / 2, part gq % 2)
+      const float *v = (gq & 1) ? lo : hi;
+      qf[kb * 32 + lane] = make_uint4(f16x2(v[0], v[1]), f16x2(v[2], v[3]), 0u, 0u);
+    } else {
+      qf[kb * 32 + lane] = make_uint4(f16x2(hi[0], hi[1]), f16x2(hi[2], hi[3]), f16x2(lo[0], lo[1]),
+                                      f16x2(lo[2], lo[3]));
+    }
   }
 }
 
@@ -227,6 +237,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const __grid_co
   using C = Cfg<D, BITS, G>;
   static_assert(BITS == 2 || BITS == 4, "2- and 4-bit codes");
   static_assert(QPK == 4 || QPK == 8, "query-head tiles of 4");
+  constexpr bool kPairs = QPK == 4;  // columns (head, hi / lo): see attend_prep_kernel
   constexpr int NG = D / G;
   __shared__ AttnMmaSmem sm;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -335,7 +346,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const __grid_co
       }
       constexpr int kPerG = G / 16;  // k-blocks per group
       mma16816(acc[kb / kPerG], af, qh[kb][0], qh[kb][1]);
-      mma16816(acc[kb / kPerG], af, ql[kb][0], ql[kb][1]);
+      if constexpr (!kPairs) mma16816(acc[kb / kPerG], af, ql[kb][0], ql[kb][1]);
     }
     // scores: c0, c1 = token tA, heads 2tq, 2tq + 1; c2, c3 = token tB
     const uint32_t *mA = reinterpret_cast<const uint32_t *>(meta_of(kv0 + (okA ? tA : 0), 0));
@@ -348,30 +359,47 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const __grid_co
       const float zfa = __half2float(__ushort_as_half(uint16_t(ma >> 16))) * kup;
       const float sfb = __half2float(__ushort_as_half(uint16_t(mb))) * kup;
       const float zfb = __half2float(__ushort_as_half(uint16_t(mb >> 16))) * kup;
-      const float q0 = sm.qs[2 * tq][gg], q1 = sm.qs[2 * tq + 1][gg];
-      sc[0] = fmaf(sfa, acc[gg][0] * inv_eq, fmaf(zfa, q0, sc[0]));
-      sc[1] = fmaf(sfa, acc[gg][1] * inv_eq, fmaf(zfa, q1, sc[1]));
-      sc[2] = fmaf(sfb, acc[gg][2] * inv_eq, fmaf(zfb, q0, sc[2]));
-      sc[3] = fmaf(sfb, acc[gg][3] * inv_eq, fmaf(zfb, q1, sc[3]));
+      if constexpr (kPairs) {  // c0 + c1: token tA, head tq; c2 + c3: token tB
+        const float q0 = sm.qs[tq][gg];
+        sc[0] = fmaf(sfa, (acc[gg][0] + acc[gg][1]) * inv_eq, fmaf(zfa, q0, sc[0]));
+        sc[2] = fmaf(sfb, (acc[gg][2] + acc[gg][3]) * inv_eq, fmaf(zfb, q0, sc[2]));
+      } else {
+        const float q0 = sm.qs[2 * tq][gg], q1 = sm.qs[2 * tq + 1][gg];
+        sc[0] = fmaf(sfa, acc[gg][0] * inv_eq, fmaf(zfa, q0, sc[0]));
+        sc[1] = fmaf(sfa, acc[gg][1] * inv_eq, fmaf(zfa, q1, sc[1]));
+        sc[2] = fmaf(sfb, acc[gg][2] * inv_eq, fmaf(zfb, q0, sc[2]));
+        sc[3] = fmaf(sfb, acc[gg][3] * inv_eq, fmaf(zfb, q1, sc[3]));
+      }
     }
-    if (okA) {
-      *reinterpret_cast<float2 *>(&sm.s[tA][2 * tq]) = make_float2(sc[0], sc[1]);
-      mx[0] = fmaxf(mx[0], sc[0]);
-      mx[1] = fmaxf(mx[1], sc[1]);
-    }
-    if (okB) {
-      *reinterpret_cast<float2 *>(&sm.s[tB][2 * tq]) = make_float2(sc[2], sc[3]);
-      mx[0] = fmaxf(mx[0], sc[2]);
-      mx[1] = fmaxf(mx[1], sc[3]);
+    if constexpr (kPairs) {
+      if (okA) {
+        sm.s[tA][tq] = sc[0];
+        mx[0] = fmaxf(mx[0], sc[0]);
+      }
+      if (okB) {
+        sm.s[tB][tq] = sc[2];
+        mx[0] = fmaxf(mx[0], sc[2]);
+      }
+    } else {
+      if (okA) {
+        *reinterpret_cast<float2 *>(&sm.s[tA][2 * tq]) = make_float2(sc[0], sc[1]);
+        mx[0] = fmaxf(mx[0], sc[0]);
+        mx[1] = fmaxf(mx[1], sc[1]);
+      }
+      if (okB) {
+        *reinterpret_cast<float2 *>(&sm.s[tB][2 * tq]) = make_float2(sc[2], sc[3]);
+        mx[0] = fmaxf(mx[0], sc[2]);
+        mx[1] = fmaxf(mx[1], sc[3]);
+      }
     }
   }
-  // per-head maxima: lanes of equal tq hold the same heads
+  // per-head maxima: lanes of equal tq hold the same heads (kPairs: head tq)
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
+  for (int e = 0; e < (kPairs ? 1 : 2); ++e) {
     float x = mx[e];
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) x = fmaxf(x, __shfl_xor_sync(0xFFFFFFFFu, x, o));
-    if (gq == 0) sm.wmax[warp][2 * tq + e] = x;
+    if (gq == 0) sm.wmax[warp][kPairs ? tq : 2 * tq + e] = x;
   }
   __syncthreads();
   if (tid < QPK) {
@@ -461,7 +489,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const __grid_co
       const uint32_t t = t0 + i;
       const bool ok = t < n;
       const uint8_t *row = in + base + uint64_t(vv0 + (ok ? t : 0)) * C::CB;
-      const float p = ok ? sm.s[t][gq] * ew : 0.f;
+      const float p = ok ? sm.s[t][kPairs ? gq >> 1 : gq] * ew : 0.f;
 #pragma unroll
       for (int gg = 0; gg < NG; ++gg) {
         const uint8_t *src = row + gg * (G * BITS / 8) + gq * NB;
@@ -487,9 +515,14 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const __grid_co
       for (int k = 0; k < 2; ++k) {
         const float x0 = x[2 * k][gg], x1 = x[2 * k + 1][gg];
         const uint32_t hv = f16x2(x0, x1);
-        wh[gg][k] = hv;
-        wl[gg][k] = f16x2(x0 - __half2float(__ushort_as_half(uint16_t(hv))),
-                          x1 - __half2float(__ushort_as_half(uint16_t(hv >> 16))));
+        const uint32_t lv = f16x2(x0 - __half2float(__ushort_as_half(uint16_t(hv))),
+                                  x1 - __half2float(__ushort_as_half(uint16_t(hv >> 16))));
+        if constexpr (kPairs) {  // column gq = (head gq / 2, part gq % 2)
+          wh[gg][k] = (gq & 1) ? lv : hv;
+        } else {
+          wh[gg][k] = hv;
+          wl[gg][k] = lv;
+        }
       }
     // A fragments (codes, rows = channels) and the products
 #pragma unroll
@@ -507,7 +540,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const __grid_co
           af[2] = codes_f16x2<0x000F000Fu>(x23);
           af[3] = codes_f16x2<0x000F000Fu>(x23 >> 4);
           mma16816(oacc[mt], af, wh[gg][0], wh[gg][1]);
-          mma16816(oacc[mt], af, wl[gg][0], wl[gg][1]);
+          if constexpr (!kPairs) mma16816(oacc[mt], af, wl[gg][0], wl[gg][1]);
         } else {
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
@@ -518,7 +551,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const __grid_co
             af[2] = codes_f16x2<0x00030003u>(x23 >> (4 * hf));
             af[3] = codes_f16x2<0x00030003u>(x23 >> (4 * hf + 2));
             mma16816(oacc[mt], af, wh[gg][0], wh[gg][1]);
-            mma16816(oacc[mt], af, wl[gg][0], wl[gg][1]);
+            if constexpr (!kPairs) mma16816(oacc[mt], af, wl[gg][0], wl[gg][1]);
           }
         }
       }
@@ -533,10 +566,15 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const __grid_co
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
     const int c0 = row_channel(mt, 0), c1 = row_channel(mt, 1);
-    sm.o[warp][2 * tq][c0] = oacc[mt][0] * inv_ew;
-    sm.o[warp][2 * tq + 1][c0] = oacc[mt][1] * inv_ew;
-    sm.o[warp][2 * tq][c1] = oacc[mt][2] * inv_ew;
-    sm.o[warp][2 * tq + 1][c1] = oacc[mt][3] * inv_ew;
+    if constexpr (kPairs) {  // columns 2tq, 2tq + 1: head tq's hi and lo parts
+      sm.o[warp][tq][c0] = (oacc[mt][0] + oacc[mt][1]) * inv_ew;
+      sm.o[warp][tq][c1] = (oacc[mt][2] + oacc[mt][3]) * inv_ew;
+    } else {
+      sm.o[warp][2 * tq][c0] = oacc[mt][0] * inv_ew;
+      sm.o[warp][2 * tq + 1][c0] = oacc[mt][1] * inv_ew;
+      sm.o[warp][2 * tq][c1] = oacc[mt][2] * inv_ew;
+      sm.o[warp][2 * tq + 1][c1] = oacc[mt][3] * inv_ew;
+    }
   }
   __syncthreads();
   for (uint32_t i = tid; i < qpk * D; i += kAttThreads) {
