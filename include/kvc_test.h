@@ -1,8 +1,10 @@
 /*
- * kvc_test.h — test-only entry point of libkvc.so. Not part of the codec's
- * interface: it exists so that a test can make one of the codec's bounded
+ * kvc_test.h — test-only entry points of libkvc.so. Not part of the codec's
+ * interface: one exists so that a test can make one of the codec's bounded
  * device waits run out, on purpose and harmlessly, and check that the call
- * ends with KVC_ERR_TIMEOUT while the CUDA context stays usable.
+ * ends with KVC_ERR_TIMEOUT while the CUDA context stays usable; the other
+ * runs the FP4 quantizer's device rounding on given values so that a test
+ * can compare it with the rule it implements at every tie.
  *
  * Every wait of the codec's kernels is bounded (one second of the GPU's
  * global timer, or an iteration cap); when one runs out the kernel records
@@ -37,6 +39,13 @@ kvc_status kvc_test_compress_stalled(const kvc_kv_desc *kv, const kvc_params *pa
                                      void *workspace, size_t workspace_bytes,
                                      uint32_t skip_chunks, uint64_t wait_ns,
                                      kvc_stream_t stream);
+
+/* The FP4 quantizer's e2m1 rounding (the same device function its encoder
+ * uses) on n DEVICE fp32 values: out[i] = the e2m1 code nearest to in[i],
+ * ties to the even magnitude index, magnitudes above 6 to 6, magnitude 0
+ * always code 0 (no negative zero). in, out: device pointers; n < 2^31,
+ * else KVC_ERR_INVALID_ARG. Asynchronous on `stream`. */
+kvc_status kvc_test_e2m1(const float *in, uint8_t *out, uint64_t n, kvc_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -450,6 +450,21 @@ kvc_status kvc_decompress_timed(const void *in, size_t in_bytes, const kvc_kv_de
   return kvc_decompress(in, in_bytes, out, workspace, workspace_bytes, stream);
 }
 
+namespace kvc {
+__global__ void e2m1_test_kernel(const float *in, uint8_t *out, uint32_t n) {
+  const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = uint8_t(e2m1_rne(in[i]));
+}
+}  // namespace kvc
+
+kvc_status kvc_test_e2m1(const float *in, uint8_t *out, uint64_t n, kvc_stream_t stream) {
+  if (!in || !out || n >= (uint64_t(1) << 31)) return KVC_ERR_INVALID_ARG;
+  if (n == 0) return KVC_OK;
+  kvc::e2m1_test_kernel<<<unsigned((n + 255) / 256), 256, 0,
+                          reinterpret_cast<cudaStream_t>(stream)>>>(in, out, uint32_t(n));
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
 kvc_status kvc_attend_timed(const void *in, size_t in_bytes, const kvc_attn_desc *attn,
                             void *workspace, size_t workspace_bytes, void *const *events,
                             int n_events, kvc_stream_t stream) {

@@ -219,8 +219,9 @@ struct Enc : Cfg<D, BITS, G> {
     for (int j = 0; j < D / 2; ++j) {
       const int ha = j / (G / 2), hb = (j + D / 2) / (G / 2);
       const float2 p = mul2(y.p[j], make_float2(rr[ha], rr[hb]));
-      y.p[j] = make_float2(__uint_as_float(0x4B400000u | e2m1_rne(p.x)),
-                           __uint_as_float(0x4B400000u | e2m1_rne(p.y)));
+      const uint32_t c2 = e2m1x2_rne(p.x, p.y);
+      y.p[j] = make_float2(__uint_as_float(0x4B400000u | (c2 & 0xFu)),
+                           __uint_as_float(0x4B400000u | (c2 >> 4)));
     }
     return err;
   }

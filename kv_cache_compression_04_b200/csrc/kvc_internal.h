@@ -177,16 +177,20 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
   const uint32_t mag = e ? (((e + 126u) << 23) | (m << 22)) : (m ? 0x3F000000u : 0u);
   return __uint_as_float(mag | ((c & 8u) << 28));
 }
-// The e2m1 code nearest to p, ties to the even magnitude index, |p| > 6 to
-// 6; magnitude 0 is always code 0. Each comparison is one boundary of the
-// grid: ties at 0.25, 1.25, 2.5, 5 go down, at 0.75, 1.75, 3.5 up.
-__device__ __forceinline__ uint32_t e2m1_rne(float p) {
-  const float a = fabsf(p);
-  const uint32_t i = uint32_t(a > 0.25f) + uint32_t(a >= 0.75f) + uint32_t(a > 1.25f) +
-                     uint32_t(a >= 1.75f) + uint32_t(a > 2.5f) + uint32_t(a >= 3.5f) +
-                     uint32_t(a > 5.0f);
-  return i | ((i != 0u && p < 0.0f) ? 8u : 0u);
+// The e2m1 codes nearest to lo and hi (bits 0-3 and 4-7), ties to the even
+// magnitude index, magnitudes above 6 to 6: the sm_100a conversion
+// cvt.rn.satfinite.e2m1x2.f32, whose rounding is the rule of the FP4
+// quantizer (a test compares it with the rule at every tie); a magnitude-0
+// code loses its sign bit (no negative zero).
+__device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
+  uint32_t d;
+  asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u32.u8 %0, t;\n}"
+      : "=r"(d) : "f"(hi), "f"(lo));
+  const uint32_t m = d & 0x77u;                      // magnitudes
+  const uint32_t nz = (m | (m >> 1) | (m >> 2)) & 0x11u;  // a nonzero magnitude per nibble
+  return m | (d & (nz << 3));
 }
+__device__ __forceinline__ uint32_t e2m1_rne(float p) { return e2m1x2_rne(p, 0.f) & 0xFu; }
 #endif
 
 // Unsigned 32-bit division by a run-time constant (Granlund and Montgomery,

@@ -221,6 +221,8 @@ float orc_e2m1_to_f32(int code) {
 int orc_f32_to_e2m1_rne(float p) {
   double a = fabs((double)p), best = 1e300;
   int i, bi = 0;
+  if (a >= 6.0) /* the largest magnitude (the scan's differences lose 4 vs 6 far above it) */
+    return p < 0.0f ? (7 | 8) : 7;
   for (i = 0; i < 8; i++) {
     double e = fabs(a - (double)orc_e2m1_to_f32(i));
     if (e < best || (e == best && (i & 1) == 0)) {

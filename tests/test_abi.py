@@ -29,7 +29,7 @@ def test_exports_every_declared_symbol(L):
     for path in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))):
         with open(path) as f:
             hdr += f.read()
-    declared = set(re.findall(r"\b(kvc_[a-z_]+)\s*\(", hdr))
+    declared = set(re.findall(r"\b(kvc_[a-z0-9_]+)\s*\(", hdr))
     assert declared == set(kvc.EXPORTS)
     for name in declared:
         assert hasattr(L, name), name

@@ -192,3 +192,30 @@ def test_full_llama8b_variant(bits, g, quant, signs):
     compared whole: stream bytes and decoded values."""
     w = synth.workload("llama8b")
     _dense(128, bits, g, w.layers, w.kv_heads, w.tokens, quant=quant, signs=signs)
+
+
+def test_device_e2m1_rounding_is_the_oracles_rule():
+    """The FP4 encoder's e2m1 rounding (the sm_100a conversion it uses) against
+    the oracle's rule: every multiple of 1/256 in [-8, 8] (every tie of the
+    e2m1 grid included: 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5), the fp32
+    neighbours of each tie, signed zeros, values far above 6, tiny and
+    subnormal values, and random values over several binades."""
+    grid = np.arange(-8 * 256, 8 * 256 + 1, dtype=np.float64) / 256
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0])
+    ties = np.concatenate([ties, -ties])
+    t32 = ties.astype(np.float32)
+    near = np.concatenate([np.nextafter(t32, np.float32(np.inf)),
+                           np.nextafter(t32, np.float32(-np.inf))])
+    rng = np.random.default_rng(5)
+    rnd = (rng.standard_normal(20000) * np.exp2(rng.integers(-12, 6, 20000))).astype(np.float32)
+    special = np.array([0.0, -0.0, 7.0, -7.0, 1e30, -1e30, 1e-40, -1e-40, 6.25, -6.25],
+                       np.float32)
+    x = np.concatenate([grid.astype(np.float32), t32, near, rnd, special]).astype(np.float32)
+    din = torch.from_numpy(x).cuda()
+    dout = torch.zeros(x.size, dtype=torch.uint8, device="cuda")
+    assert kvc.lib().kvc_test_e2m1(din.data_ptr(), dout.data_ptr(), x.size,
+                                   kvc._stream_ptr(None)) == kvc.KVC_OK
+    got = dout.cpu().numpy()
+    want = np.array([oracle.f32_to_e2m1_rne(float(v)) for v in x], np.uint8)
+    bad = np.flatnonzero(got != want)
+    assert bad.size == 0, [(float(x[i]), int(got[i]), int(want[i])) for i in bad[:10]]

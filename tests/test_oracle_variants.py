@@ -346,6 +346,10 @@ def test_e2m1_table_and_nearest_even():
     assert oracle.f32_to_e2m1_rne(1.25) == 2 and oracle.f32_to_e2m1_rne(1.75) == 4
     assert oracle.f32_to_e2m1_rne(2.5) == 4 and oracle.f32_to_e2m1_rne(3.5) == 6
     assert oracle.f32_to_e2m1_rne(5.0) == 6 and oracle.f32_to_e2m1_rne(-0.1) == 0
+    # magnitudes above 6 give 6 however large (a double scan alone would see
+    # 1e30 - 4 and 1e30 - 6 as equal)
+    for big in (6.0, 7.0, 1e9, 1e30, 3.4e38):
+        assert oracle.f32_to_e2m1_rne(big) == 7 and oracle.f32_to_e2m1_rne(-big) == 15
 
 
 def test_e4m3_against_torch_and_round_up():
