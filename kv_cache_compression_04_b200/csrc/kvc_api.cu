@@ -209,11 +209,17 @@ void add_tensor_map(const kvc_kv_desc *kv, const Shape &s, DenseLayout &L) {
 
 // Tensor map of a paged pool for the encoder's run loads: 5-D [layers]
 // [pages][2 * kv_heads][page_tokens][head_dim] with kv and head merged into
-// one dimension (needs stride_kv == kv_heads * stride_head), boxes of 8 slots
-// x 64 channels with 128-byte swizzle (needs page_tokens % 8 == 0).
+// one dimension (needs stride_kv == kv_heads * stride_head), boxes of one run
+// of slots x 64 channels with 128-byte swizzle. A run is 16 slots, 8 for
+// pages of 8; page_tokens must be a power of two from 8 to 512 (a block's
+// plan word holds a run's position in its page in 5 bits) and the head rows
+// fewer than 2^21 (the plan word's head-row field).
 void add_tensor_map_paged(const kvc_kv_desc *kv, const Shape &s, PagedLayout &L) {
   L.tma = 0;
-  if (s.V == 0 || kv->page_tokens % 8 != 0 || kv->stride_kv != kv->kv_heads * kv->stride_head)
+  const int64_t pt = kv->page_tokens;
+  if (s.V == 0 || pt < 8 || pt > 512 || (pt & (pt - 1)) != 0 ||
+      kv->stride_kv != kv->kv_heads * kv->stride_head ||
+      int64_t(kv->layers) * 2 * kv->kv_heads >= (int64_t(1) << 21))
     return;
   if (kv->stride_slot <= 0 || kv->stride_head <= 0 || kv->stride_page <= 0 || kv->stride_layer <= 0)
     return;
@@ -224,16 +230,23 @@ void add_tensor_map_paged(const kvc_kv_desc *kv, const Shape &s, PagedLayout &L)
                               cuuint64_t(kv->layers)};
   const cuuint64_t strides[4] = {cuuint64_t(L.s_slot), cuuint64_t(L.s_h), cuuint64_t(L.s_p),
                                  cuuint64_t(L.s_l)};
-  const cuuint32_t box[5] = {64, 8, 1, 1, 1};
+  uint32_t page_lg = 3;
+  while ((int64_t(1) << page_lg) < pt) ++page_lg;
+  const uint32_t run_lg = page_lg < 4 ? page_lg : 4;
+  const cuuint32_t box[5] = {64, cuuint32_t(1u << run_lg), 1, 1, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   if (fn(&L.tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, kv->data, dims, strides, box, estr,
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS) {
     L.tma = 1;
+    L.run_lg = run_lg;
+    L.page_lg = page_lg;
+  }
 }
 
 void paged_layout(const kvc_kv_desc *kv, const Shape &s, PagedLayout &L) {
   L.tma = 0;  // add_tensor_map_paged sets it for the encoder
+  L.run_lg = L.page_lg = 0;
   L.base = static_cast<uint8_t *>(kv->data);
   L.s_l = kv->stride_layer * 2;
   L.s_p = kv->stride_page * 2;
@@ -327,6 +340,7 @@ kvc_status compress_impl(const kvc_kv_desc *kv, const kvc_params *params, void *
   a.seed = params->sign_seed;
   a.tdiv = make_fastdiv(uint32_t(s.T ? s.T : 1));
   sign_masks(params->sign_seed, s.D, a.sign_mask);
+  for (int k = 0; k < s.D / 2; ++k) a.sign_lo[k] = a.sign_mask[k] << 16;
 
   FinArgs f{};
   f.V = uint32_t(s.V);

@@ -57,12 +57,12 @@ struct Cfg {
 
 // Shared memory: per-warp row buffers | per-warp mbarriers | request prefix
 // (paged).
-// A row buffer holds 32 rows (dense input) or 40 (paged input: a block's 32
-// tokens start anywhere in an 8-slot run of their pages, and its runs come
-// in whole), per 64-channel half.
+// A row buffer holds 32 rows (dense input) or 48 (paged input: a block's 32
+// tokens start anywhere in a run of at most 16 slots of their pages, and its
+// runs come in whole), per 64-channel half.
 template <int D, bool kPaged = false>
 struct EncSmem {
-  static constexpr int ROWS = kPaged ? 40 : 32;
+  static constexpr int ROWS = kPaged ? 48 : 32;
   static constexpr int HALF = ROWS * 128;                   // bytes per 64-channel half
   static constexpr size_t WBUF = size_t(D / 64) * HALF;     // 128-byte swizzled halves
   static constexpr size_t wbars = kEncWarps * WBUF;
@@ -116,7 +116,9 @@ struct Enc : Cfg<D, BITS, G> {
   using C = Cfg<D, BITS, G>;
 
   // E1/E2: widen bf16 exactly and flip the sign bit of negative channels.
-  // Word k of the row holds channels 2k (low half) and 2k+1 (high half).
+  // Word k of the row holds channels 2k (low half) and 2k+1 (high half): one
+  // shift-and-add (the flip at bit 31 added) widens the low channel, one
+  // three-input logic op the high one.
   template <class SG>
   static __device__ __forceinline__ void unpack(const uint8_t *row, const SG &sg, Pairs<D> &y) {
     const uint4 *r4 = reinterpret_cast<const uint4 *>(row);
@@ -127,10 +129,10 @@ struct Enc : Cfg<D, BITS, G> {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int k = 4 * q + e;
-        const uint32_t x0 = wa[e] ^ sg.word(k), x1 = wb[e] ^ sg.word(k + D / 4);
-        y.p[2 * k] = make_float2(__uint_as_float(x0 << 16), __uint_as_float(x1 << 16));
-        y.p[2 * k + 1] =
-            make_float2(__uint_as_float(x0 & 0xFFFF0000u), __uint_as_float(x1 & 0xFFFF0000u));
+        y.p[2 * k] = make_float2(__uint_as_float((wa[e] << 16) + sg.lo(k)),
+                                 __uint_as_float((wb[e] << 16) + sg.lo(k + D / 4)));
+        y.p[2 * k + 1] = make_float2(__uint_as_float((wa[e] ^ sg.word(k)) & 0xFFFF0000u),
+                                     __uint_as_float((wb[e] ^ sg.word(k + D / 4)) & 0xFFFF0000u));
       }
     }
   }
@@ -154,10 +156,10 @@ struct Enc : Cfg<D, BITS, G> {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int k = 4 * q + e;
-        const uint32_t x0 = wa[e] ^ sg.word(k), x1 = wb[e] ^ sg.word(k + D / 4);
-        y.p[2 * k] = make_float2(__uint_as_float(x0 << 16), __uint_as_float(x1 << 16));
-        y.p[2 * k + 1] =
-            make_float2(__uint_as_float(x0 & 0xFFFF0000u), __uint_as_float(x1 & 0xFFFF0000u));
+        y.p[2 * k] = make_float2(__uint_as_float((wa[e] << 16) + sg.lo(k)),
+                                 __uint_as_float((wb[e] << 16) + sg.lo(k + D / 4)));
+        y.p[2 * k + 1] = make_float2(__uint_as_float((wa[e] ^ sg.word(k)) & 0xFFFF0000u),
+                                     __uint_as_float((wb[e] ^ sg.word(k + D / 4)) & 0xFFFF0000u));
       }
     }
   }
@@ -498,7 +500,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       vec_sign_words<D>(a.seed, fdiv(a.tdiv, v), sg.S);
       E::template unpack_swz<S::HALF>(wbuf, row, sg, y);
     } else {
-      E::template unpack_swz<S::HALF>(wbuf, row, GlobalSigns{a.sign_mask}, y);
+      E::template unpack_swz<S::HALF>(wbuf, row, GlobalSigns{a.sign_mask, a.sign_lo}, y);
     }
   };
 
@@ -547,19 +549,22 @@ __global__ void __launch_bounds__(kEncThreads, 1)
   if constexpr (kPaged) {
     grid_dependency_wait();  // the workspace clear (a plan may record a status)
     // A block whose 32 tokens lie in one request (all but about one in a
-    // hundred of a batch of long requests) loads as the 8-slot runs of its
-    // pages: lane j < runs reads run j's page and issues one tensor box of 8
-    // rows per 64-channel half into 1 KB slot j of the buffer, so lane i's
-    // row is row (t0 % 8) + i. Other blocks (a request boundary, a page
-    // outside the pool, no tensor map) are gathered row by row, lane i's row
-    // at row i. A plan is made one block ahead of its issue and reads nothing it
-    // needs at once: the block's request comes from one shared-memory load
-    // per lane and a ballot over the request prefix (no dependent search),
-    // and the lanes of its runs load their pages, which are checked only at
-    // issue, a block of arithmetic later. Per lane a plan is one word (kind
-    // in bits 0-1: 0 past the end, 1 runs of one request, 2 any other block;
-    // t0 % 8 in bits 2-4; the lane's run starting at slot 8 in bit 5; the
-    // head row lkh from bit 6) and the lane's run page.
+    // hundred of a batch of long requests) loads as the runs of its pages (a
+    // run: 2^run_lg slots, 16 or, for pages of 8, 8): lane j < runs reads run
+    // j's page and issues one tensor box of a run per 64-channel half into
+    // slot j of the buffer, so lane i's row is row (t0 % run) + i. Other
+    // blocks (a request boundary, a page outside the pool, no tensor map) are
+    // gathered row by row, lane i's row at row i. A plan is made one block
+    // ahead of its issue and reads nothing it needs at once: the block's
+    // request comes from one shared-memory load per lane and a ballot over the
+    // request prefix (no dependent search), and the lanes of its runs load
+    // their pages, which are checked only at issue, a block of arithmetic
+    // later. Per lane a plan is one word (kind in bits 0-1: 0 past the end, 1
+    // runs of one request, 2 any other block; t0 % run in bits 2-5; the first
+    // run's position in its page, (t0 / run) % (runs per page), in bits 6-10;
+    // the head row lkh from bit 11) and the lane's run page.
+    const uint32_t rlg = lay.run_lg, plg = lay.page_lg;
+    const uint32_t rmask = (1u << rlg) - 1u, qmask = (1u << (plg - rlg)) - 1u;
     auto plan = [&](uint32_t b, int32_t &pg) -> uint32_t {
       const uint32_t v0 = b * 32;
       pg = -1;
@@ -575,34 +580,33 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       }
       const uint32_t t0 = u0 - s_cum[r];
       if (!(v0 + 32 <= V && u0 + 32 <= s_cum[r + 1])) return 2u;
-      const uint32_t runs = ((t0 + 31) >> 3) - (t0 >> 3) + 1;  // 4 or 5
-      uint32_t hi8 = 0;
+      const uint32_t runs = ((t0 + 31) >> rlg) - (t0 >> rlg) + 1;  // 2 or 3 (runs of 16)
       if (uint32_t(lane) < runs) {
-        const uint32_t hp = (t0 >> 3) + lane;  // the run's 8-slot half page
-        pg = __ldg(lay.page_table + int64_t(r) * lay.pt_stride + (hp >> 1));
-        hi8 = hp & 1u;
+        const uint32_t hp = (t0 >> rlg) + lane;  // the run's index in the request
+        pg = __ldg(lay.page_table + int64_t(r) * lay.pt_stride + (hp >> (plg - rlg)));
       }
-      return 1u | ((t0 & 7u) << 2) | (hi8 << 5) | (lkh << 6);
+      return 1u | ((t0 & rmask) << 2) | (((t0 >> rlg) & qmask) << 6) | (lkh << 11);
     };
     // Issues block b's loads; returns the kind used (runs need every page in
     // the pool, else the block is gathered row by row, which records a bad
     // page) and the row shift.
     auto issue = [&](uint32_t b, uint32_t p, int32_t pg) -> uint32_t {
       if ((p & 3u) == 1u) {
-        const uint32_t runs = (((p >> 2) & 7u) + 31) / 8 + 1;
+        const uint32_t runs = ((((p >> 2) & 15u) + 31) >> rlg) + 1;
         const bool ok = uint32_t(lane) >= runs || (pg >= 0 && int64_t(pg) < lay.num_pages);
         if (__all_sync(0xFFFFFFFFu, ok)) {
-          if (lane == 0) mbar_arrive_expect_tx(wbar, runs * uint32_t(D / 64) * 1024u);
+          if (lane == 0) mbar_arrive_expect_tx(wbar, (runs << rlg) * uint32_t(D / 64) * 128u);
           __syncwarp();
           if (uint32_t(lane) < runs) {
-            const uint32_t lkh = p >> 6, lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
-            const int kvh = int((lk & 1u) * lay.H.d + h), slot = int(((p >> 5) & 1u) * 8);
+            const uint32_t lkh = p >> 11, lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
+            const int kvh = int((lk & 1u) * lay.H.d + h);
+            const int slot = int(((((p >> 6) & 31u) + lane) & qmask) << rlg);
 #pragma unroll
             for (int hh = 0; hh < D / 64; ++hh)
-              tma_load_5d(wbuf + hh * S::HALF + lane * 1024, &lay.tmap, hh * 64, slot, kvh, pg,
-                          int(lk >> 1), wbar);
+              tma_load_5d(wbuf + hh * S::HALF + (lane << (rlg + 7)), &lay.tmap, hh * 64, slot, kvh,
+                          pg, int(lk >> 1), wbar);
           }
-          return p & 31u;
+          return p & 63u;
         }
         p = 2u;
       }
@@ -623,7 +627,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
         __syncwarp();  // every lane's copies have landed
       }
       Pairs<D> y;
-      unpack(lane + int((cur >> 2) & 7u), v, y);
+      unpack(lane + int((cur >> 2) & 15u), v, y);
       // every lane has read the buffer; the next load may overwrite it
       fence_proxy_async_smem();
       __syncwarp();

@@ -136,9 +136,13 @@ KVC_HD uint32_t pair_mask(const uint32_t (&S)[D / 32], int c) {
 // Sign sources of the transform kernels: the diagonal shared by every vector
 // (masks in the kernel's parameters) or the vector's own (its words in
 // registers). word(k) is the mask of channel pair (2k, 2k + 1).
+// lo(k) is word(k) << 16: channel 2k's flip moved to bit 31, where adding it
+// to the widened channel (an integer add) is the same as XOR-ing it in.
 struct GlobalSigns {
   const uint32_t *mask;
+  const uint32_t *lo_mask = nullptr;  // words << 16 (the encoder's widening)
   __device__ __forceinline__ uint32_t word(int k) const { return mask[k]; }
+  __device__ __forceinline__ uint32_t lo(int k) const { return lo_mask[k]; }
   __device__ __forceinline__ uint4 quad(int q) const {  // words 4q .. 4q + 3
     return reinterpret_cast<const uint4 *>(mask)[q];
   }
@@ -147,6 +151,7 @@ template <int D>
 struct VectorSigns {
   uint32_t S[D / 32];
   __device__ __forceinline__ uint32_t word(int k) const { return pair_mask<D>(S, 2 * k); }
+  __device__ __forceinline__ uint32_t lo(int k) const { return ((S[k / 16] >> (2 * k % 32)) & 1u) << 31; }
   __device__ __forceinline__ uint4 quad(int q) const {
     return make_uint4(word(4 * q), word(4 * q + 1), word(4 * q + 2), word(4 * q + 3));
   }
@@ -230,11 +235,14 @@ struct DenseLayout {
 
 struct PagedLayout {
   // Tensor map of the pool as 5-D [layers][pages][2 * kv_heads][page_tokens]
-  // [head_dim] (boxes of 8 slots x 64 channels, 128-byte swizzle), valid iff
-  // tma != 0: set by the host when kv and head merge into one dimension
-  // (stride_kv == kv_heads * stride_head) and page_tokens % 8 == 0.
+  // [head_dim] (boxes of one run of 2^run_lg slots x 64 channels, 128-byte
+  // swizzle), valid iff tma != 0: set by the host when kv and head merge into
+  // one dimension (stride_kv == kv_heads * stride_head) and page_tokens is a
+  // power of two 2^page_lg from 8 to 512 (runs of 16 slots, of 8 for pages
+  // of 8).
   alignas(64) CUtensorMap tmap;
   uint32_t tma;
+  uint32_t run_lg, page_lg;
   uint8_t *base;
   int64_t s_l, s_p, s_kv, s_h, s_slot;  // bytes
   const int32_t *page_table;
@@ -268,6 +276,7 @@ struct EncArgs {
   uint64_t seed;       // sign seed (per-vector diagonals)
   FastDiv tdiv;        // tokens per (layer, kv, head): vector index = v / tokens
   uint32_t sign_mask[128];
+  uint32_t sign_lo[128];  // sign_mask[k] << 16
 };
 
 // Finishing kernels: sizes and offsets of every chunk, meta chunks,

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       __syncwarp();
     }
     Pairs<D> y;
-    E::unpack_swz(wbuf, lane, GlobalSigns{a.sign_mask}, y);
+    E::unpack_swz(wbuf, lane, GlobalSigns{a.sign_mask, a.sign_lo}, y);
     fwht_pairs<D>(y);
     __syncwarp();  // every lane has read its input row
 #pragma unroll

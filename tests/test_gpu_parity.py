@@ -177,12 +177,12 @@ def test_compaction_many_chunks_mixed():
 
 
 # -------------------------------------------------------------------- paged --
-def _paged_setup(seq, L=2, H=3, D=128, bits=4, g=64, seed=3):
+def _paged_setup(seq, L=2, H=3, D=128, bits=4, g=64, seed=3, page_tokens=16):
     w = synth.Workload("p", L, H, D, bits, g, seed=seed, kind="lognormal", scale_sigma=1.5,
-                       seq_lens=seq)
+                       seq_lens=seq, page_tokens=page_tokens)
     pk = synth.paged_kv(w, device="cuda")
     pool = u16(pk.pool)
-    x = oracle.gather_paged(pool.reshape(-1), L, H, D, pk.strides(), 16, seq,
+    x = oracle.gather_paged(pool.reshape(-1), L, H, D, pk.strides(), page_tokens, seq,
                             pk.page_table.cpu().numpy(), 0, w.vectors)
     return w, pk, x
 
@@ -224,6 +224,33 @@ def test_paged_parity_and_cross_layout_decode(seq, bits, g):
                         device="cuda")
     assert gpu_decompress(ostream, kvc.dense_desc(dense)) == kvc.KVC_OK
     assert np.array_equal(u16(dense).reshape(-1, 128), ox)
+
+
+@pytest.mark.parametrize("page_tokens", [8, 32, 64, 24])
+def test_paged_page_sizes(page_tokens):
+    """Pages of 8, 32 and 64 slots (tensor-map runs of 8 or 16 slots, a run's
+    page and slot taken from its index in the request) and of 24 (not a power
+    of two: every block gathered row by row), with requests that start and end
+    inside pages; decode scatters through another page table."""
+    seq = [300, 1025, 77, 2000, 33]
+    w, pk, x = _paged_setup(seq, L=2, H=2, page_tokens=page_tokens)
+    od = oracle_desc(4, 64, 128, w.layers, w.kv_heads, seq, origin=1)
+    ost, ostream = oracle.compress(od, x)
+    assert ost == oracle.OK
+    st, gstream, _, _ = gpu_compress(kvc.paged_desc(pk.pool, pk.page_table, seq), 4, 64)
+    assert st == kvc.KVC_OK
+    assert np.array_equal(gstream, ostream), first_diff(gstream, ostream, od.layout())
+    _, ox = oracle.decompress(ostream, od)
+    pt2 = synth.page_table_for(seq, page_tokens, pk.pool.shape[1], 5, device="cuda")
+    pool2 = torch.full_like(pk.pool, 1.5)
+    assert gpu_decompress(ostream, kvc.paged_desc(pool2, pt2, seq)) == kvc.KVC_OK
+    got = oracle.gather_paged(u16(pool2).reshape(-1), w.layers, w.kv_heads, 128,
+                              [s for s in pool2.stride()][:5], page_tokens, seq,
+                              pt2.cpu().numpy(), 0, w.vectors)
+    assert np.array_equal(got, ox)
+    unused = ~_used_slots(synth.PagedKV(pool2, pt2, seq), seq, page_tokens)
+    canary = pool2.cpu().float().permute(1, 4, 0, 2, 3, 5)[unused]
+    assert torch.all(canary == 1.5), "decode wrote outside the described slots"
 
 
 @pytest.mark.parametrize("bits,g", [(4, 64), (2, 32)])
