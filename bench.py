@@ -1189,7 +1189,8 @@ def main():
                       "decompress": {"clear": round(kd[0], 4), "meta_expand": round(kd[1], 4),
                                      "elim_decode": round(kd[2], 4),
                                      "decode": round(kd[3], 4)}},
-        "gpu_launches": 8 * K,  # per step: workspace clear, encode, finish, compaction
+        "gpu_launches": (9 if w.paged else 8) * K,  # per step: workspace clear, load plans
+        # (paged pools), encode, finish, compaction
         # (returns at once unless code chunks are stored eliminated); status clear, meta
         # expansion, eliminated-chunk decode (returns at once unless the header flags such
         # chunks), decode

@@ -211,15 +211,15 @@ void add_tensor_map(const kvc_kv_desc *kv, const Shape &s, DenseLayout &L) {
 // [pages][2 * kv_heads][page_tokens][head_dim] with kv and head merged into
 // one dimension (needs stride_kv == kv_heads * stride_head), boxes of one run
 // of slots x 64 channels with 128-byte swizzle. A run is 16 slots, 8 for
-// pages of 8; page_tokens must be a power of two from 8 to 512 (a block's
-// plan word holds a run's position in its page in 5 bits) and the head rows
-// fewer than 2^21 (the plan word's head-row field).
+// pages of 8; page_tokens must be a power of two from 8 to 512, and the
+// pool fit the load plans' fields (paged_plan_kernel): 2 * kv_heads <= 2048,
+// layers <= 4096, num_pages < 2^27.
 void add_tensor_map_paged(const kvc_kv_desc *kv, const Shape &s, PagedLayout &L) {
   L.tma = 0;
   const int64_t pt = kv->page_tokens;
   if (s.V == 0 || pt < 8 || pt > 512 || (pt & (pt - 1)) != 0 ||
-      kv->stride_kv != kv->kv_heads * kv->stride_head ||
-      int64_t(kv->layers) * 2 * kv->kv_heads >= (int64_t(1) << 21))
+      kv->stride_kv != kv->kv_heads * kv->stride_head || 2 * int64_t(kv->kv_heads) > 2048 ||
+      kv->layers > 4096 || kv->num_pages >= (int64_t(1) << 27))
     return;
   if (kv->stride_slot <= 0 || kv->stride_head <= 0 || kv->stride_page <= 0 || kv->stride_layer <= 0)
     return;

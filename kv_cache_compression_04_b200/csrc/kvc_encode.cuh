@@ -442,6 +442,67 @@ __device__ __forceinline__ void encode_finish_block(const EncArgs &a, uint32_t b
 }
 
 // ------------------------------------------------------------------------
+// Load plans of a paged pool's blocks (before the encoder, in the encode
+// step's interval). Block b (32 vectors, every full block but the last) gets
+// 8 words at ws_meta + b * 32 * MB, the start of its own meta slot:
+//   word 0: kind (bits 0-1: 1 = tensor-map runs, 2 = row gather), t0 % run
+//           (bits 2-5), runs (6-8), kv * kv_heads + head (9-19), layer (20-31)
+//   word 1 + j: run j's page << 5 | the run's position in its page.
+// Runs need the block inside one request and every page inside the pool.
+// Host conditions (add_tensor_map_paged): 2 * kv_heads <= 2048,
+// layers <= 4096, num_pages < 2^27.
+// ------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+    paged_plan_kernel(const __grid_constant__ EncArgs a, const __grid_constant__ PagedLayout lay,
+                      uint32_t slot_bytes) {
+  __shared__ uint32_t cum[KVC_MAX_REQUESTS + 1];
+  for (uint32_t r = threadIdx.x; r <= lay.n_req; r += blockDim.x) cum[r] = lay.cum[r];
+  __syncthreads();
+  // the meta slots' previous users (the last call's finishing kernels) are
+  // done: the clear before this waited for them
+  grid_dependency_wait();
+  const uint32_t n_blocks = (a.V + 31) / 32;
+  const uint32_t rlg = lay.run_lg, plg = lay.page_lg;
+  const uint32_t rmask = (1u << rlg) - 1u, qmask = (1u << (plg - rlg)) - 1u;
+  for (uint32_t b = blockIdx.x * blockDim.x + threadIdx.x; b + 1 < n_blocks;
+       b += gridDim.x * blockDim.x) {
+    const uint32_t v0 = b * 32, lkh = fdiv(lay.T, v0), u0 = v0 - lkh * lay.T.d;
+    uint32_t w[8] = {2u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (u0 + 32 <= lay.T.d) {
+      uint32_t lo = 0, hi = lay.n_req;  // cum[lo] <= u0 < cum[hi]
+      while (hi - lo > 1) {
+        const uint32_t mid = (lo + hi) / 2;
+        if (cum[mid] <= u0) lo = mid; else hi = mid;
+      }
+      const uint32_t t0 = u0 - cum[lo];
+      if (u0 + 32 <= cum[lo + 1]) {
+        const uint32_t runs = ((t0 + 31) >> rlg) - (t0 >> rlg) + 1;  // 2 or 3 (runs of 16)
+        const int32_t *row = lay.page_table + int64_t(lo) * lay.pt_stride;
+        bool ok = true;
+#pragma unroll
+        for (uint32_t j = 0; j < 5; ++j) {  // (at most 5 runs: runs of 8)
+          if (j < runs) {
+            const uint32_t hp = (t0 >> rlg) + j;  // the run's index in the request
+            const int32_t pg = __ldg(row + (hp >> (plg - rlg)));
+            ok &= pg >= 0 && int64_t(pg) < lay.num_pages;
+            w[1 + j] = (uint32_t(pg) << 5) | (hp & qmask);
+          }
+        }
+        if (ok) {
+          const uint32_t lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
+          w[0] = 1u | ((t0 & rmask) << 2) | (runs << 6) | (((lk & 1u) * lay.H.d + h) << 9) |
+                 ((lk >> 1) << 20);
+        }
+      }
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(a.ws_meta + uint64_t(b) * slot_bytes);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+// ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
 // kVar bit 0: per-(layer, kv, head) sign diagonals (each lane derives its
@@ -547,73 +608,47 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       gather_rows<D, S::HALF>(wbuf, rowp, a.out);
   };
   if constexpr (kPaged) {
-    grid_dependency_wait();  // the workspace clear (a plan may record a status)
+    grid_dependency_wait();  // the plans (paged_plan_kernel)
     // A block whose 32 tokens lie in one request (all but about one in a
     // hundred of a batch of long requests) loads as the runs of its pages (a
-    // run: 2^run_lg slots, 16 or, for pages of 8, 8): lane j < runs reads run
-    // j's page and issues one tensor box of a run per 64-channel half into
-    // slot j of the buffer, so lane i's row is row (t0 % run) + i. Other
-    // blocks (a request boundary, a page outside the pool, no tensor map) are
-    // gathered row by row, lane i's row at row i. A plan is made one block
-    // ahead of its issue and reads nothing it needs at once: the block's
-    // request comes from one shared-memory load per lane and a ballot over the
-    // request prefix (no dependent search), and the lanes of its runs load
-    // their pages, which are checked only at issue, a block of arithmetic
-    // later. Per lane a plan is one word (kind in bits 0-1: 0 past the end, 1
-    // runs of one request, 2 any other block; t0 % run in bits 2-5; the first
-    // run's position in its page, (t0 / run) % (runs per page), in bits 6-10;
-    // the head row lkh from bit 11) and the lane's run page.
-    const uint32_t rlg = lay.run_lg, plg = lay.page_lg;
-    const uint32_t rmask = (1u << rlg) - 1u, qmask = (1u << (plg - rlg)) - 1u;
-    auto plan = [&](uint32_t b, int32_t &pg) -> uint32_t {
-      const uint32_t v0 = b * 32;
-      pg = -1;
-      if (v0 >= V) return 0u;
-      if (!lay.tma) return 2u;
-      const uint32_t lkh = fdiv(lay.T, v0), u0 = v0 - lkh * lay.T.d;
-      uint32_t r = 0;  // the largest r with cum[r] <= u0 (cum is nondecreasing)
-      for (uint32_t g0 = 0; g0 <= lay.n_req; g0 += 32) {
-        const uint32_t i = g0 + lane;
-        const uint32_t below = __ballot_sync(0xFFFFFFFFu, i <= lay.n_req && s_cum[min(i, lay.n_req)] <= u0);
-        r = g0 + __popc(below) - 1;
-        if (below != 0xFFFFFFFFu) break;
-      }
-      const uint32_t t0 = u0 - s_cum[r];
-      if (!(v0 + 32 <= V && u0 + 32 <= s_cum[r + 1])) return 2u;
-      const uint32_t runs = ((t0 + 31) >> rlg) - (t0 >> rlg) + 1;  // 2 or 3 (runs of 16)
-      if (uint32_t(lane) < runs) {
-        const uint32_t hp = (t0 >> rlg) + lane;  // the run's index in the request
-        pg = __ldg(lay.page_table + int64_t(r) * lay.pt_stride + (hp >> (plg - rlg)));
-      }
-      return 1u | ((t0 & rmask) << 2) | (((t0 >> rlg) & qmask) << 6) | (lkh << 11);
+    // run: 2^run_lg slots, 16 or, for pages of 8, 8): lane j < runs issues
+    // one tensor box of run j per 64-channel half into slot j of the buffer,
+    // so lane i's row is row (t0 % run) + i. Other blocks (a request
+    // boundary, a page outside the pool, no tensor map, the last block) are
+    // gathered row by row, lane i's row at row i, which records a bad page.
+    // paged_plan_kernel wrote each full block's plan into the first 32 bytes
+    // of the block's own meta slot, which only this warp writes, and only
+    // after reading the plan (two blocks ahead of its use).
+    const uint32_t rlg = lay.run_lg;
+    const uint8_t *plans = a.ws_meta;
+    auto plan = [&](uint32_t b, uint32_t &own) -> uint32_t {
+      own = 0;
+      if (b >= n_blocks) return 0u;
+      if (!lay.tma || b + 1 == n_blocks) return 2u;
+      const uint32_t *pw = reinterpret_cast<const uint32_t *>(plans + uint64_t(b) * (32 * C::MB));
+      own = __ldcg(pw + 1 + min(lane, 4));
+      return __ldcg(pw);
     };
-    // Issues block b's loads; returns the kind used (runs need every page in
-    // the pool, else the block is gathered row by row, which records a bad
-    // page) and the row shift.
-    auto issue = [&](uint32_t b, uint32_t p, int32_t pg) -> uint32_t {
+    // Issues block b's loads; returns the kind and the row shift.
+    auto issue = [&](uint32_t b, uint32_t p, uint32_t own) -> uint32_t {
       if ((p & 3u) == 1u) {
-        const uint32_t runs = ((((p >> 2) & 15u) + 31) >> rlg) + 1;
-        const bool ok = uint32_t(lane) >= runs || (pg >= 0 && int64_t(pg) < lay.num_pages);
-        if (__all_sync(0xFFFFFFFFu, ok)) {
-          if (lane == 0) mbar_arrive_expect_tx(wbar, (runs << rlg) * uint32_t(D / 64) * 128u);
-          __syncwarp();
-          if (uint32_t(lane) < runs) {
-            const uint32_t lkh = p >> 11, lk = fdiv(lay.H, lkh), h = lkh - lk * lay.H.d;
-            const int kvh = int((lk & 1u) * lay.H.d + h);
-            const int slot = int(((((p >> 6) & 31u) + lane) & qmask) << rlg);
+        const uint32_t runs = (p >> 6) & 7u;
+        if (lane == 0) mbar_arrive_expect_tx(wbar, (runs << rlg) * uint32_t(D / 64) * 128u);
+        __syncwarp();
+        if (uint32_t(lane) < runs) {
+          const int kvh = int((p >> 9) & 2047u), layer = int(p >> 20);
+          const int slot = int((own & 31u) << rlg), pg = int(own >> 5);
 #pragma unroll
-            for (int hh = 0; hh < D / 64; ++hh)
-              tma_load_5d(wbuf + hh * S::HALF + (lane << (rlg + 7)), &lay.tmap, hh * 64, slot, kvh,
-                          pg, int(lk >> 1), wbar);
-          }
-          return p & 63u;
+          for (int hh = 0; hh < D / 64; ++hh)
+            tma_load_5d(wbuf + hh * S::HALF + (lane << (rlg + 7)), &lay.tmap, hh * 64, slot, kvh,
+                        pg, layer, wbar);
         }
-        p = 2u;
+        return p & 63u;
       }
       if ((p & 3u) == 2u) gather(src_of(b * 32 + lane));
       return p & 3u;
     };
-    int32_t npg;
+    uint32_t npg;
     uint32_t cur = issue(blk, plan(blk, npg), npg);
     uint32_t next = plan(blk + stride, npg);
 #pragma unroll 1

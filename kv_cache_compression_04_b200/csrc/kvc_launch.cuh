@@ -73,7 +73,18 @@ cudaError_t launch_enc_k(const EncArgs &a, const Layout &lay, int sms, cudaStrea
   const uint32_t n_blocks = (a.V + 31) / 32;
   const uint32_t want = (n_blocks + kEncWarps - 1) / kEncWarps;
   const int grid = int(want < uint32_t(sms) ? want : uint32_t(sms));
-  // a dependent launch after the workspace clear: see encode_kernel
+  if constexpr (kIsPaged<Layout>) {
+    // the blocks' load plans, a dependent launch after the workspace clear
+    // whose time counts in the encode interval
+    if (lay.tma && n_blocks > 1) {
+      const uint32_t pw = (n_blocks - 1 + 255) / 256, pcap = uint32_t(sms) * 16;
+      e = launch_after_unmarked(paged_plan_kernel<D>, int(pw < pcap ? pw : pcap), 256, 0, st, a,
+                                lay, uint32_t(32 * Cfg<D, BITS, G>::MB));
+      if (e != cudaSuccess) return e;
+    }
+  }
+  // a dependent launch after the workspace clear (or the plans): see
+  // encode_kernel
   return launch_after(k, grid, kEncThreads, smem, st, a, lay);
 }
 // Paged rows named by 32-bit offsets when the pool allows (narrow row
