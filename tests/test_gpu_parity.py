@@ -253,6 +253,47 @@ def test_paged_page_sizes(page_tokens):
     assert torch.all(canary == 1.5), "decode wrote outside the described slots"
 
 
+# permutation from a slot-major pool's storage order to the logical
+# [layers, pages, kv, heads, slots, d] view the descriptor takes
+_SLOT_MAJOR = {
+    # [layers][pages][slot][kv][head][d]: kv and head still merge (tensor-map runs)
+    "slot_kv_head": ((0, 1, 4, 2, 3, 5), (0, 1, 3, 4, 2, 5)),
+    # [layers][pages][kv][slot][head][d]: they do not (row gathers)
+    "kv_slot_head": ((0, 1, 2, 4, 3, 5), (0, 1, 2, 4, 3, 5)),
+}
+
+
+@pytest.mark.parametrize("order", sorted(_SLOT_MAJOR))
+def test_paged_slot_major_pools(order):
+    """Pools stored slot-major (the layouts of serving engines that keep a
+    page's heads together per token) through strided views: parity with the
+    oracle's gather of the same strides, decode into another such pool."""
+    seq = [300, 1025, 77]
+    to_store, to_view = _SLOT_MAJOR[order]
+    w, pk, _ = _paged_setup(seq, L=2, H=2)
+    store = pk.pool.permute(*to_store).contiguous()
+    view = store.permute(*to_view)
+    assert view.shape == pk.pool.shape and torch.equal(view, pk.pool)
+    x = oracle.gather_paged(u16(store).reshape(-1), w.layers, w.kv_heads, 128,
+                            [st for st in view.stride()][:5], 16, seq,
+                            pk.page_table.cpu().numpy(), 0, w.vectors)
+    od = oracle_desc(4, 64, 128, w.layers, w.kv_heads, seq, origin=1)
+    ost, ostream = oracle.compress(od, x)
+    assert ost == oracle.OK
+    st, gstream, _, _ = gpu_compress(kvc.paged_desc(view, pk.page_table, seq), 4, 64)
+    assert st == kvc.KVC_OK
+    assert np.array_equal(gstream, ostream), first_diff(gstream, ostream, od.layout())
+    _, ox = oracle.decompress(ostream, od)
+    pt2 = synth.page_table_for(seq, 16, pk.pool.shape[1], 8, device="cuda")
+    store2 = torch.full_like(store, 1.5)
+    view2 = store2.permute(*to_view)
+    assert gpu_decompress(ostream, kvc.paged_desc(view2, pt2, seq)) == kvc.KVC_OK
+    got = oracle.gather_paged(u16(store2).reshape(-1), w.layers, w.kv_heads, 128,
+                              [st for st in view2.stride()][:5], 16, seq, pt2.cpu().numpy(), 0,
+                              w.vectors)
+    assert np.array_equal(got, ox)
+
+
 @pytest.mark.parametrize("bits,g", [(4, 64), (2, 32)])
 def test_paged_parity_eliminated_code_chunks(bits, g):
     """A paged batch whose middle request is all zeros: the code chunks inside

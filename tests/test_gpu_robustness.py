@@ -159,6 +159,27 @@ def test_page_index_outside_pool():
     assert st == kvc.KVC_ERR_CORRUPT
 
 
+@pytest.mark.parametrize("page_tokens", [16, 32])
+@pytest.mark.parametrize("bad", ["past_pool", "negative"])
+def test_page_index_outside_pool_inside_a_long_request(page_tokens, bad):
+    """A bad page in the middle of a long request: the blocks over it lie in
+    one request, so their load plan (not a row gather) meets the page first;
+    the plan falls back to the row gather, which records the bad page. The
+    decoder's scatter through such a page table fails the same way."""
+    seq = [300, 200]
+    w = synth.Workload("p", 2, 2, 128, 4, 64, seed=1, kind="lognormal", seq_lens=seq,
+                       page_tokens=page_tokens)
+    pk = synth.paged_kv(w, device="cuda")
+    st, s, _, _ = gpu_compress(kvc.paged_desc(pk.pool, pk.page_table, seq), 4, 64)
+    assert st == kvc.KVC_OK
+    pt = pk.page_table.clone()
+    pt[0, 96 // page_tokens] = pk.pool.shape[1] if bad == "past_pool" else -1
+    st, _, _, _ = gpu_compress(kvc.paged_desc(pk.pool, pt, seq), 4, 64)
+    assert st == kvc.KVC_ERR_CORRUPT
+    pool2 = torch.zeros_like(pk.pool)
+    assert gpu_decompress(s, kvc.paged_desc(pool2, pt, seq)) == kvc.KVC_ERR_CORRUPT
+
+
 def test_paged_receiver_request_mismatch():
     seq = [40, 17]
     w = synth.Workload("p", 2, 2, 128, 4, 64, seed=1, kind="lognormal", seq_lens=seq)
