@@ -47,6 +47,14 @@ kvc_status kvc_test_compress_stalled(const kvc_kv_desc *kv, const kvc_params *pa
  * else KVC_ERR_INVALID_ARG. Asynchronous on `stream`. */
 kvc_status kvc_test_e2m1(const float *in, uint8_t *out, uint64_t n, kvc_stream_t stream);
 
+/* The quantizers' division by their constant (the same device function the
+ * encoder uses for fl(x / (2^b - 1)) and fl(x / (2^(b-1) - 1))) on n DEVICE
+ * fp32 values x >= 0: out[i] = in[i] / q rounded to nearest even, for q in
+ * {1, 3, 7, 15, 127, 255} (else KVC_ERR_INVALID_ARG; n < 2^31).
+ * Asynchronous on `stream`. */
+kvc_status kvc_test_div_const(const float *in, float *out, uint64_t n, int q,
+                              kvc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -30,7 +30,7 @@ EXPORTS = ["kvc_max_compressed_bytes", "kvc_workspace_bytes", "kvc_compress",
            "kvc_decompress_workspace_bytes", "kvc_unfused_workspace_bytes",
            "kvc_compress_unfused", "kvc_test_compress_stalled", "kvc_compress_timed",
            "kvc_decompress_timed", "kvc_attend_workspace_bytes", "kvc_attend",
-           "kvc_attend_timed", "kvc_test_e2m1"]
+           "kvc_attend_timed", "kvc_test_e2m1", "kvc_test_div_const"]
 
 
 class KvcError(RuntimeError):
@@ -126,6 +126,8 @@ def lib() -> C.CDLL:
                                        C.POINTER(C.c_void_p), C.c_int, C.c_void_p]
         L.kvc_test_e2m1.restype = C.c_int
         L.kvc_test_e2m1.argtypes = [C.c_void_p, C.c_void_p, C.c_uint64, C.c_void_p]
+        L.kvc_test_div_const.restype = C.c_int
+        L.kvc_test_div_const.argtypes = [C.c_void_p, C.c_void_p, C.c_uint64, C.c_int, C.c_void_p]
         L.kvc_test_compress_stalled.restype = C.c_int
         L.kvc_test_compress_stalled.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p,
                                                 C.c_void_p, C.c_size_t, C.c_uint32, C.c_uint64,

@@ -464,12 +464,38 @@ kvc_status kvc_decompress_timed(const void *in, size_t in_bytes, const kvc_kv_de
   return kvc_decompress(in, in_bytes, out, workspace, workspace_bytes, stream);
 }
 
+extern "C++" {  // (the test kernels, inside the C-linkage block)
 namespace kvc {
 __global__ void e2m1_test_kernel(const float *in, uint8_t *out, uint32_t n) {
   const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = uint8_t(e2m1_rne(in[i]));
 }
+template <int Q>
+__global__ void div_const_test_kernel(const float *in, float *out, uint32_t n) {
+  const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = div_const<Q>(in[i]);
+}
 }  // namespace kvc
+}
+
+kvc_status kvc_test_div_const(const float *in, float *out, uint64_t n, int q,
+                              kvc_stream_t stream) {
+  if (!in || !out || n >= (uint64_t(1) << 31)) return KVC_ERR_INVALID_ARG;
+  void (*k)(const float *, float *, uint32_t) = nullptr;
+  switch (q) {
+    case 1: k = kvc::div_const_test_kernel<1>; break;
+    case 3: k = kvc::div_const_test_kernel<3>; break;
+    case 7: k = kvc::div_const_test_kernel<7>; break;
+    case 15: k = kvc::div_const_test_kernel<15>; break;
+    case 127: k = kvc::div_const_test_kernel<127>; break;
+    case 255: k = kvc::div_const_test_kernel<255>; break;
+    default: return KVC_ERR_INVALID_ARG;
+  }
+  if (n == 0) return KVC_OK;
+  k<<<unsigned((n + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(in, out,
+                                                                                 uint32_t(n));
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
 
 kvc_status kvc_test_e2m1(const float *in, uint8_t *out, uint64_t n, kvc_stream_t stream) {
   if (!in || !out || n >= (uint64_t(1) << 31)) return KVC_ERR_INVALID_ARG;

@@ -266,18 +266,22 @@ struct Enc : Cfg<D, BITS, G> {
       return err;
     }
     float zf[C::NG], rr[C::NG];  // zf: subtracted before the product (0 when symmetric)
+    // x * 0 is 0 for finite x and NaN for an infinite or NaN x: nf turns NaN
+    // once a group's min or max is not finite, rg once a stored zero or
+    // scale overflows fp16
+    float nf = 0.0f, rg = 0.0f;
 #pragma unroll
     for (int g = 0; g < C::NG; ++g) {
       float mn, mx;
       minmax(y, g, mn, mx);
       mn = __fadd_rn(mn, 0.0f);  // -0 -> +0
       mx = __fadd_rn(mx, 0.0f);
-      if (!(isfinite(mn) && isfinite(mx))) err |= 1u;
+      nf = __fmaf_rn(mn, 0.0f, __fmaf_rn(mx, 0.0f, nf));
       const float down = 1.0f / float(1 << C::K), up = float(1 << C::K);
       __half zh, sh;
       if (sym) {
         const float am = fmaxf(fabsf(mn), fabsf(mx));
-        sh = __float2half_ru(__fmul_rn(__fdiv_rn(am, float(C::QH)), down));
+        sh = __float2half_ru(__fmul_rn(div_const<C::QH>(am), down));
         zh = (__half_as_ushort(sh) & 0x7FFFu) == 0
                  ? __ushort_as_half(0)
                  : __float2half_rd(__fmul_rn(__half2float(sh), -float(1 << (BITS - 1))));
@@ -285,15 +289,17 @@ struct Enc : Cfg<D, BITS, G> {
       } else {
         zh = __float2half_rd(__fmul_rn(mn, down));
         zf[g] = __fmul_rn(__half2float(zh), up);
-        const float s32 = __fdiv_rn(__fsub_rn(mx, zf[g]), float(C::QMAX));
+        const float s32 = div_const<C::QMAX>(__fsub_rn(mx, zf[g]));
         sh = __float2half_ru(__fmul_rn(s32, down));
       }
       const float sf = __fmul_rn(__half2float(sh), up);
       const uint16_t zb = __half_as_ushort(zh), sb = __half_as_ushort(sh);
-      if ((zb & 0x7FFFu) == 0x7C00u || (sb & 0x7FFFu) == 0x7C00u) err |= 2u;
-      rr[g] = ((sb & 0x7FFFu) == 0) ? 0.0f : __frcp_rn(sf);
+      rg = __fmaf_rn(__half2float(zh), 0.0f, __fmaf_rn(sf, 0.0f, rg));
+      rr[g] = sf == 0.0f ? 0.0f : __frcp_rn(sf);
       meta[g] = uint32_t(sb) | (uint32_t(zb) << 16);
     }
+    if (nf != 0.0f) err |= 1u;       // (NaN compares unequal)
+    else if (rg != 0.0f) err |= 2u;
     const float kMagic = sym ? 12582912.0f + float(1 << (BITS - 1)) : 12582912.0f;  // 1.5 * 2^23
     const float2 mag = make_float2(kMagic, kMagic), one2 = make_float2(one, one);
 #pragma unroll

@@ -12,6 +12,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <cmath>
+
 #include "../../include/kvc.h"
 
 #if defined(__CUDACC__)
@@ -131,6 +133,32 @@ template <int D>
 KVC_HD uint32_t pair_mask(const uint32_t (&S)[D / 32], int c) {
   const uint32_t w = S[c / 32] >> (c % 32);
   return ((w & 1u) << 15) | ((w & 2u) << 30);
+}
+
+// x / Q, correctly rounded, for a constant Q and x >= 0 (the quantizers'
+// 2^b - 1 and 2^(b-1) - 1): Markstein's correction of the product with the
+// rounded reciprocal (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990):
+// q = RN(x * RN(1/Q)), the remainder x - q * Q exactly by one fused
+// multiply-add, then RN(q + remainder * RN(1/Q)). The result equals the
+// correctly rounded quotient for every finite x >= 0 and Q in {3, 7, 15, 127,
+// 255}: checked over all of them on the host (this function compiled for
+// the host), and on the GPU over samples of every binade through
+// kvc_test_div_const.
+template <int Q>
+KVC_HD float div_const(float x) {
+  if constexpr (Q == 1) {
+    return x;
+  } else {
+    constexpr float c = 1.0f / float(Q);
+#ifdef __CUDA_ARCH__
+    const float q = __fmul_rn(x, c);
+    return __fmaf_rn(__fmaf_rn(-q, float(Q), x), c, q);
+#else
+    const float q = x * c;
+    return std::fmaf(std::fmaf(-q, float(Q), x), c, q);
+#endif
+  }
 }
 
 // Sign sources of the transform kernels: the diagonal shared by every vector

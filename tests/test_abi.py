@@ -171,7 +171,25 @@ def host_logic():
     lib.hl_nz_nibble_mismatches.restype = C.c_uint64
     lib.hl_nz_nibble_mismatches.argtypes = [C.c_uint64, C.c_uint64]
     lib.hl_sign_masks.argtypes = [C.c_uint64, C.c_int, C.c_void_p]
+    lib.hl_div_const_mismatches.restype = C.c_uint64
+    lib.hl_div_const_mismatches.argtypes = [C.c_int, C.c_uint32, C.c_uint32]
     return lib
+
+
+@pytest.mark.parametrize("q", [3, 7, 15, 127, 255])
+def test_division_by_quantizer_constant_sampled(host_logic, q):
+    """The encoder's x / q (Markstein's correction of x * RN(1/q), compiled
+    for the host) is the correctly rounded quotient: every 9973rd fp32
+    pattern, i.e. samples of every binade, subnormals included."""
+    assert host_logic.hl_div_const_mismatches(q, 0, 9973) == 0
+    assert host_logic.hl_div_const_mismatches(q, 1, 104729) == 0
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("q", [3, 7, 15, 127, 255])
+def test_division_by_quantizer_constant_exhaustive(host_logic, q):
+    """The same over every finite x >= 0."""
+    assert host_logic.hl_div_const_mismatches(q, 0, 1) == 0
 
 
 def test_fast_division_exact(host_logic):

@@ -219,3 +219,26 @@ def test_device_e2m1_rounding_is_the_oracles_rule():
     want = np.array([oracle.f32_to_e2m1_rne(float(v)) for v in x], np.uint8)
     bad = np.flatnonzero(got != want)
     assert bad.size == 0, [(float(x[i]), int(got[i]), int(want[i])) for i in bad[:10]]
+
+
+@pytest.mark.parametrize("q", [1, 3, 7, 15, 127, 255])
+def test_device_division_by_quantizer_constant(q):
+    """The encoder's division by its quantizer's constant, on the GPU, against
+    numpy's correctly rounded fp32 division: 2048 random significands in
+    every binade (subnormals included), each binade's first and last value,
+    and zero."""
+    rng = np.random.default_rng(q)
+    exps = np.repeat(np.arange(0, 255, dtype=np.uint32), 2048)
+    sig = rng.integers(0, 1 << 23, exps.size, dtype=np.uint32)
+    bits = np.concatenate([(exps << 23) | sig, (np.arange(0, 255, dtype=np.uint32) << 23),
+                           (np.arange(0, 255, dtype=np.uint32) << 23) | 0x7FFFFF,
+                           np.array([0], np.uint32)])
+    x = bits.view(np.float32)
+    din = torch.from_numpy(x.copy()).cuda()
+    dout = torch.zeros_like(din)
+    assert kvc.lib().kvc_test_div_const(din.data_ptr(), dout.data_ptr(), x.size, q,
+                                        kvc._stream_ptr(None)) == kvc.KVC_OK
+    got = dout.cpu().numpy()
+    want = x / np.float32(q)
+    bad = np.flatnonzero(got.view(np.uint32) != want.view(np.uint32))
+    assert bad.size == 0, [(float(x[i]), float(got[i]), float(want[i])) for i in bad[:10]]
