@@ -55,6 +55,13 @@ kvc_status kvc_test_e2m1(const float *in, uint8_t *out, uint64_t n, kvc_stream_t
 kvc_status kvc_test_div_const(const float *in, float *out, uint64_t n, int q,
                               kvc_stream_t stream);
 
+/* The encoder's reciprocal of its stored scales (the same device function it
+ * uses for 1 / s, s = an fp16 scale times 2^K) on n DEVICE fp32 values:
+ * out[i] = 1 / in[i] rounded to nearest even, for in[i] a positive finite
+ * fp16 value times 8 or 16 (other inputs: the result is not specified);
+ * n < 2^31, else KVC_ERR_INVALID_ARG. Asynchronous on `stream`. */
+kvc_status kvc_test_rcp_scale(const float *in, float *out, uint64_t n, kvc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

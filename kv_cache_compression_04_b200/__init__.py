@@ -30,7 +30,8 @@ EXPORTS = ["kvc_max_compressed_bytes", "kvc_workspace_bytes", "kvc_compress",
            "kvc_decompress_workspace_bytes", "kvc_unfused_workspace_bytes",
            "kvc_compress_unfused", "kvc_test_compress_stalled", "kvc_compress_timed",
            "kvc_decompress_timed", "kvc_attend_workspace_bytes", "kvc_attend",
-           "kvc_attend_timed", "kvc_test_e2m1", "kvc_test_div_const"]
+           "kvc_attend_timed", "kvc_test_e2m1", "kvc_test_div_const",
+           "kvc_test_rcp_scale"]
 
 
 class KvcError(RuntimeError):
@@ -128,6 +129,8 @@ def lib() -> C.CDLL:
         L.kvc_test_e2m1.argtypes = [C.c_void_p, C.c_void_p, C.c_uint64, C.c_void_p]
         L.kvc_test_div_const.restype = C.c_int
         L.kvc_test_div_const.argtypes = [C.c_void_p, C.c_void_p, C.c_uint64, C.c_int, C.c_void_p]
+        L.kvc_test_rcp_scale.restype = C.c_int
+        L.kvc_test_rcp_scale.argtypes = [C.c_void_p, C.c_void_p, C.c_uint64, C.c_void_p]
         L.kvc_test_compress_stalled.restype = C.c_int
         L.kvc_test_compress_stalled.argtypes = [D, P, C.c_void_p, C.c_size_t, C.c_void_p,
                                                 C.c_void_p, C.c_size_t, C.c_uint32, C.c_uint64,

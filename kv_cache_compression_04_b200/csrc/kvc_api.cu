@@ -475,7 +475,19 @@ __global__ void div_const_test_kernel(const float *in, float *out, uint32_t n) {
   const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = div_const<Q>(in[i]);
 }
+__global__ void rcp_scale_test_kernel(const float *in, float *out, uint32_t n) {
+  const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = rcp_scale(in[i]);
+}
 }  // namespace kvc
+}
+
+kvc_status kvc_test_rcp_scale(const float *in, float *out, uint64_t n, kvc_stream_t stream) {
+  if (!in || !out || n >= (uint64_t(1) << 31)) return KVC_ERR_INVALID_ARG;
+  if (n == 0) return KVC_OK;
+  kvc::rcp_scale_test_kernel<<<unsigned((n + 255) / 256), 256, 0,
+                               reinterpret_cast<cudaStream_t>(stream)>>>(in, out, uint32_t(n));
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
 kvc_status kvc_test_div_const(const float *in, float *out, uint64_t n, int q,

@@ -295,7 +295,7 @@ struct Enc : Cfg<D, BITS, G> {
       const float sf = __fmul_rn(__half2float(sh), up);
       const uint16_t zb = __half_as_ushort(zh), sb = __half_as_ushort(sh);
       rg = __fmaf_rn(__half2float(zh), 0.0f, __fmaf_rn(sf, 0.0f, rg));
-      rr[g] = sf == 0.0f ? 0.0f : __frcp_rn(sf);
+      rr[g] = sf == 0.0f ? 0.0f : rcp_scale(sf);
       meta[g] = uint32_t(sb) | (uint32_t(zb) << 16);
     }
     if (nf != 0.0f) err |= 1u;       // (NaN compares unequal)

@@ -161,6 +161,21 @@ KVC_HD float div_const(float x) {
   }
 }
 
+#ifdef __CUDACC__
+// 1 / s for the encoder's scales s = h * 2^K (h a positive finite fp16
+// value, K = 3 or 4): the hardware's approximate reciprocal y, then one
+// Newton step with its residual fused, y + y * (1 - s * y) (Markstein's
+// method, P. Markstein, IBM J. Res. Develop. 34(1), 1990). It equals the
+// correctly rounded 1 / s for every such s: checked on the GPU over all of
+// them through kvc_test_rcp_scale. (s is normal and so is 1 / s, so the
+// approximation's flush of subnormals never acts.)
+__device__ __forceinline__ float rcp_scale(float s) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(s));
+  return __fmaf_rn(__fmaf_rn(-s, y, 1.0f), y, y);
+}
+#endif
+
 // Sign sources of the transform kernels: the diagonal shared by every vector
 // (masks in the kernel's parameters) or the vector's own (its words in
 // registers). word(k) is the mask of channel pair (2k, 2k + 1).

@@ -242,3 +242,19 @@ def test_device_division_by_quantizer_constant(q):
     want = x / np.float32(q)
     bad = np.flatnonzero(got.view(np.uint32) != want.view(np.uint32))
     assert bad.size == 0, [(float(x[i]), float(got[i]), float(want[i])) for i in bad[:10]]
+
+
+def test_device_reciprocal_of_every_scale():
+    """The encoder's 1 / s for every scale it can hold (each positive finite
+    fp16 value times 2^3 and 2^4) against numpy's correctly rounded fp32
+    division."""
+    h = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)
+    s = np.concatenate([h * np.float32(8), h * np.float32(16)]).astype(np.float32)
+    din = torch.from_numpy(s.copy()).cuda()
+    dout = torch.zeros_like(din)
+    assert kvc.lib().kvc_test_rcp_scale(din.data_ptr(), dout.data_ptr(), s.size,
+                                        kvc._stream_ptr(None)) == kvc.KVC_OK
+    got = dout.cpu().numpy()
+    want = np.float32(1) / s
+    bad = np.flatnonzero(got.view(np.uint32) != want.view(np.uint32))
+    assert bad.size == 0, [(float(s[i]), float(got[i]), float(want[i])) for i in bad[:10]]
