@@ -230,7 +230,9 @@ size_t kvc_decompress_workspace_bytes(const kvc_kv_desc *out);
  * (the bytes that shift), else every code chunk is stored raw. The call
  * launches four kernels on `stream` (workspace clear; encode; table, meta
  * chunks and header; compaction, which returns at once unless code chunks
- * are stored eliminated). */
+ * are stored eliminated), five for a paged pool whose page size is a power
+ * of two from 8 to 512 (the blocks' load plans, written into the
+ * workspace's meta region, before the encode). */
 kvc_status kvc_compress(const kvc_kv_desc *kv, const kvc_params *params,
                         void *out, size_t out_capacity, uint64_t *out_bytes_dev,
                         void *workspace, size_t workspace_bytes,
