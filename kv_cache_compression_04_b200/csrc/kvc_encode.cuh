@@ -191,8 +191,11 @@ struct Enc : Cfg<D, BITS, G> {
   // half-group an e4m3 micro-scale s1 = RU(fl(max_half|y| / (6 * s2))), at
   // most 448; S = s1 * s2 (exact), r = fl(1 / S) (0 for S = 0), code = e2m1
   // nearest to fl(y * r), ties to even. Meta word: s2_h | s1_0 << 16 |
-  // s1_1 << 24. Each code leaves in the low bits of a float for the packer.
-  static __device__ __forceinline__ uint32_t quantize_fp4(Pairs<D> &y, uint32_t (&meta)[C::NG]) {
+  // s1_1 << 24. The codes are packed here: the conversion turns channels
+  // (2k, 2k + 1) into byte k of the vector's codes (LSB first, reading R6),
+  // and the -0 codes of a word's eight nibbles become 0 in one step.
+  static __device__ __forceinline__ uint32_t quantize_fp4(Pairs<D> &y, uint32_t (&meta)[C::NG],
+                                                          uint32_t (&code)[C::CW]) {
     static_assert(BITS == 4, "FP4 codes are 4-bit");
     uint32_t err = 0;
     float rr[2 * C::NG];  // 1 / S per half-group
@@ -220,10 +223,15 @@ struct Enc : Cfg<D, BITS, G> {
 #pragma unroll
     for (int j = 0; j < D / 2; ++j) {
       const int ha = j / (G / 2), hb = (j + D / 2) / (G / 2);
-      const float2 p = mul2(y.p[j], make_float2(rr[ha], rr[hb]));
-      const uint32_t c2 = e2m1x2_rne(p.x, p.y);
-      y.p[j] = make_float2(__uint_as_float(0x4B400000u | (c2 & 0xFu)),
-                           __uint_as_float(0x4B400000u | (c2 >> 4)));
+      y.p[j] = mul2(y.p[j], make_float2(rr[ha], rr[hb]));
+    }
+#pragma unroll
+    for (int W = 0; W < C::CW; ++W) {  // channels 8W .. 8W + 7
+      uint32_t b[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) b[k] = e2m1x2_raw(y.at(8 * W + 2 * k), y.at(8 * W + 2 * k + 1));
+      code[W] = e2m1_zero_signs(
+          __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410));
     }
     return err;
   }
@@ -260,11 +268,7 @@ struct Enc : Cfg<D, BITS, G> {
                                                       uint32_t (&meta)[C::NG], float one,
                                                       uint32_t sym) {
     uint32_t err = 0;
-    if constexpr (kFp4) {
-      err = quantize_fp4(y, meta);
-      pack(y, code);
-      return err;
-    }
+    if constexpr (kFp4) return quantize_fp4(y, meta, code);
     float zf[C::NG], rr[C::NG];  // zf: subtracted before the product (0 when symmetric)
     // x * 0 is 0 for finite x and NaN for an infinite or NaN x: nf turns NaN
     // once a group's min or max is not finite, rg once a stored zero or

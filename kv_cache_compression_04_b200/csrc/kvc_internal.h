@@ -230,13 +230,21 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
 // cvt.rn.satfinite.e2m1x2.f32, whose rounding is the rule of the FP4
 // quantizer (a test compares it with the rule at every tie); a magnitude-0
 // code loses its sign bit (no negative zero).
-__device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
+// The conversion's byte (lo in the low nibble) as it comes, -0 codes included.
+__device__ __forceinline__ uint32_t e2m1x2_raw(float lo, float hi) {
   uint32_t d;
   asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u32.u8 %0, t;\n}"
       : "=r"(d) : "f"(hi), "f"(lo));
-  const uint32_t m = d & 0x77u;                      // magnitudes
-  const uint32_t nz = (m | (m >> 1) | (m >> 2)) & 0x11u;  // a nonzero magnitude per nibble
-  return m | (d & (nz << 3));
+  return d;
+}
+// Every nibble of w whose magnitude is 0 loses its sign bit (-0 -> code 0).
+__device__ __forceinline__ uint32_t e2m1_zero_signs(uint32_t w) {
+  const uint32_t m = w & 0x77777777u;                            // magnitudes
+  const uint32_t nz = (m | (m >> 1) | (m >> 2)) & 0x11111111u;   // a nonzero magnitude per nibble
+  return m | (w & (nz << 3));
+}
+__device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
+  return e2m1_zero_signs(e2m1x2_raw(lo, hi));
 }
 __device__ __forceinline__ uint32_t e2m1_rne(float p) { return e2m1x2_rne(p, 0.f) & 0xFu; }
 #endif
