@@ -38,7 +38,6 @@ struct DecCtl {
   uint32_t bits, group, n_req_stream, n_chunks, code_elim, vec_signs, quant;
   uint64_t data_base, stream_bytes, seed;
   alignas(16) uint32_t mask[128];  // read as uint4
-  float e2m1[16];                  // FP4 code values
 };
 
 // Shared memory: per-warp output staging | per-warp code blocks | per-warp
@@ -125,11 +124,11 @@ struct Dec : Cfg<D, BITS, G> {
   // rounding. q*sf is exact (q < 16 times an fp16 value needs at most 15
   // significant bits), so one fused multiply-add equals fl(zf + fl(q*sf)).
   // The vector is held as pairs (c, c + d/2) like the encoder's.
-  // e2m1 (FP4 only): the 16 code values, a table in shared memory.
+  // FP4: the hardware's e2m1 -> f16 conversion turns each code byte (two
+  // adjacent channels) into their values, exact in f16 and in fp32.
   template <class SG>
   static __device__ __forceinline__ void vector(const uint8_t *codes, const uint8_t *meta,
-                                                const SG &sg, uint32_t (&out)[D / 2],
-                                                const float *e2m1 = nullptr) {
+                                                const SG &sg, uint32_t (&out)[D / 2]) {
     float zf[kFp4 ? 1 : C::NG], sf[kFp4 ? 1 : C::NG];
     float S[kFp4 ? 2 * C::NG : 1];  // FP4 (reading R22): s1 * s2 per half-group, x 2^-log2 d
     const float up = float(1 << C::K) / float(D);
@@ -145,48 +144,64 @@ struct Dec : Cfg<D, BITS, G> {
         zf[g] = __fmul_rn(__half2float(__ushort_as_half(uint16_t(m >> 16))), up);
       }
     }
-    // Code -> float: a byte permute puts the code in the low byte of the bit
-    // pattern 0x4B4000qq = 1.5*2^23 + q; subtracting 1.5*2^23 gives q exactly.
-    // Pair j takes channel j from the first half of the code words and
-    // channel j + d/2 from the second; each 16-byte piece of either half is
-    // loaded when the pairs reach it.
-    constexpr int per_word = 32 / BITS;          // codes per word
-    constexpr int per_byte = 8 / BITS;
-    constexpr int HW = C::CW / 2;                // words per half
-    constexpr int PW = HW < 4 ? HW : 4;          // words per piece
-    constexpr int NP = HW / PW;                  // pieces per half
-    constexpr int JP = PW * per_word;            // pairs per piece
-    constexpr uint32_t kMagicBits = 0x4B400000u;
-    constexpr float kMagic = 12582912.0f;
-    const float2 mag = make_float2(kMagic, kMagic);
     Pairs<D> y;
+    if constexpr (kFp4) {  // e2m1(code) * S, exact
+      static_assert(BITS == 4, "FP4 codes are 4-bit");
 #pragma unroll
-    for (int piece = 0; piece < NP; ++piece) {
-      uint32_t lo[PW], hi[PW];
-      if constexpr (PW == 4) {
-        const uint4 a = reinterpret_cast<const uint4 *>(codes)[piece];
-        const uint4 b = reinterpret_cast<const uint4 *>(codes)[NP + piece];
-        lo[0] = a.x, lo[1] = a.y, lo[2] = a.z, lo[3] = a.w;
-        hi[0] = b.x, hi[1] = b.y, hi[2] = b.z, hi[3] = b.w;
-      } else {
-        const uint4 a = reinterpret_cast<const uint4 *>(codes)[0];
-        lo[0] = a.x, lo[1] = a.y, hi[0] = a.z, hi[1] = a.w;
+      for (int q4 = 0; q4 < C::CW / 4; ++q4) {
+        const uint4 v = reinterpret_cast<const uint4 *>(codes)[q4];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // byte k of word 4 q4 + e: channels c, c + 1
+            const int c = 8 * (4 * q4 + e) + 2 * k;
+            const float2 f = e2m1x2_to_float2(w[e] >> (8 * k));
+            y.at(c) = f.x;
+            y.at(c + 1) = f.y;
+          }
       }
-      auto code_float = [&](const uint32_t (&w)[PW], int c) -> float {
-        const int W = c / per_word, r = c % per_word, k = r / per_byte, e = r % per_byte;
-        const uint32_t part =
-            (w[W] >> (e * BITS)) & (BITS == 8 ? 0xFFFFFFFFu : BITS == 4 ? 0x0F0F0F0Fu : 0x03030303u);
-        return __uint_as_float(__byte_perm(part, kMagicBits, 0x7640 | k));
-      };
 #pragma unroll
-      for (int i = 0; i < JP; ++i) {
-        const int j = piece * JP + i;
-        if constexpr (kFp4) {  // e2m1(code) * S, exact
-          const int ha = j / (G / 2), hb = (j + D / 2) / (G / 2);
-          const uint32_t ca = __float_as_uint(code_float(lo, i)) & 15u;
-          const uint32_t cb = __float_as_uint(code_float(hi, i)) & 15u;
-          y.p[j] = mul2(make_float2(e2m1[ca], e2m1[cb]), make_float2(S[ha], S[hb]));
+      for (int j = 0; j < D / 2; ++j) {
+        const int ha = j / (G / 2), hb = (j + D / 2) / (G / 2);
+        y.p[j] = mul2(y.p[j], make_float2(S[ha], S[hb]));
+      }
+    } else {
+      // Code -> float: a byte permute puts the code in the low byte of the bit
+      // pattern 0x4B4000qq = 1.5*2^23 + q; subtracting 1.5*2^23 gives q exactly.
+      // Pair j takes channel j from the first half of the code words and
+      // channel j + d/2 from the second; each 16-byte piece of either half is
+      // loaded when the pairs reach it.
+      constexpr int per_word = 32 / BITS;          // codes per word
+      constexpr int per_byte = 8 / BITS;
+      constexpr int HW = C::CW / 2;                // words per half
+      constexpr int PW = HW < 4 ? HW : 4;          // words per piece
+      constexpr int NP = HW / PW;                  // pieces per half
+      constexpr int JP = PW * per_word;            // pairs per piece
+      constexpr uint32_t kMagicBits = 0x4B400000u;
+      constexpr float kMagic = 12582912.0f;
+      const float2 mag = make_float2(kMagic, kMagic);
+#pragma unroll
+      for (int piece = 0; piece < NP; ++piece) {
+        uint32_t lo[PW], hi[PW];
+        if constexpr (PW == 4) {
+          const uint4 a = reinterpret_cast<const uint4 *>(codes)[piece];
+          const uint4 b = reinterpret_cast<const uint4 *>(codes)[NP + piece];
+          lo[0] = a.x, lo[1] = a.y, lo[2] = a.z, lo[3] = a.w;
+          hi[0] = b.x, hi[1] = b.y, hi[2] = b.z, hi[3] = b.w;
         } else {
+          const uint4 a = reinterpret_cast<const uint4 *>(codes)[0];
+          lo[0] = a.x, lo[1] = a.y, hi[0] = a.z, hi[1] = a.w;
+        }
+        auto code_float = [&](const uint32_t (&w)[PW], int c) -> float {
+          const int W = c / per_word, r = c % per_word, k = r / per_byte, e = r % per_byte;
+          const uint32_t part =
+              (w[W] >> (e * BITS)) & (BITS == 8 ? 0xFFFFFFFFu : BITS == 4 ? 0x0F0F0F0Fu : 0x03030303u);
+          return __uint_as_float(__byte_perm(part, kMagicBits, 0x7640 | k));
+        };
+#pragma unroll
+        for (int i = 0; i < JP; ++i) {
+          const int j = piece * JP + i;
           const int ga = j / G, gb = (j + D / 2) / G;
           const float2 q = sub2(make_float2(code_float(lo, i), code_float(hi, i)), mag);
           y.p[j] = fma2(q, make_float2(sf[ga], sf[gb]), make_float2(zf[ga], zf[gb]));
@@ -212,10 +227,10 @@ struct Dec : Cfg<D, BITS, G> {
 // memory). A stream with per-vector diagonals (reading R20) is corrected in
 // the staging buffer by fix_row_signs.
 template <int D, int BITS, int G, bool kFp4>
-__device__ __forceinline__ void decode_vector(const uint32_t *mask, const float *e2m1,
+__device__ __forceinline__ void decode_vector(const uint32_t *mask,
                                               const uint8_t *codes, const uint8_t *meta,
                                               uint32_t (&out)[D / 2]) {
-  Dec<D, BITS, G, kFp4>::vector(codes, meta, GlobalSigns{mask}, out, e2m1);
+  Dec<D, BITS, G, kFp4>::vector(codes, meta, GlobalSigns{mask}, out);
 }
 
 // This lane's staged row XOR the global masks XOR the masks of its vector's
@@ -381,7 +396,7 @@ __device__ void decode_body(const DecArgs &a, const Layout &lay, DecCtl *ctl, ui
   auto emit = [&](const uint8_t *codes, const uint8_t *meta, uint32_t v0, uint32_t nv) {
     uint32_t out[D / 2];
     const bool act = uint32_t(lane) < nv;
-    if (act) decode_vector<D, BITS, G, kFp4>(ctl->mask, ctl->e2m1, codes + lane * C::CB, meta + lane * C::MB, out);
+    if (act) decode_vector<D, BITS, G, kFp4>(ctl->mask, codes + lane * C::CB, meta + lane * C::MB, out);
     if constexpr (!kIsPaged<Layout>) {
       if (use_tma) {
         store_block_tma<D>(lay, out, v0, stage, stage_busy, a, ctl->vec_signs, ctl->mask,
@@ -477,7 +492,6 @@ __global__ void __launch_bounds__(kDecThreads)
     mbar_init(&ctl->cbar[tid][1], 1);
     mbar_fence_init();
   }
-  if (tid < 16) ctl->e2m1[tid] = e2m1_value(uint32_t(tid));  // FP4 code values
   if (tid == 0) {
     const StreamHdr h = parse_header<D>(a);
     ctl->hdr_ok = h.ok;
@@ -669,7 +683,6 @@ struct ElimCtl {
   uint32_t ok, bits, group, nlist, vec_signs, quant;
   uint64_t base, limit, seed;
   alignas(16) uint32_t mask[128];
-  float e2m1[16];  // FP4 code values
   uint32_t list[kElimThreads];
 };
 // Shared memory: per-warp staging | per-warp meta blocks | chunk | scratch |
@@ -776,7 +789,7 @@ __device__ void elim_body(const DecArgs &a, const Layout &lay, ElimCtl *ctl, uin
         uint32_t out[D / 2];
         const bool act = uint32_t(lane) < nv;
         if (act)
-          decode_vector<D, BITS, G, kFp4>(ctl->mask, ctl->e2m1, chunk + (b * 32 + lane) * C::CB,
+          decode_vector<D, BITS, G, kFp4>(ctl->mask, chunk + (b * 32 + lane) * C::CB,
                                     mbuf + lane * C::MB, out);
         if constexpr (!kIsPaged<Layout>) {
           if (use_tma) {
@@ -821,7 +834,6 @@ __global__ void __launch_bounds__(kElimThreads, 1)
     mbar_init(&ctl->mbar[tid], 1);
     mbar_fence_init();
   }
-  if (tid < 16) ctl->e2m1[tid] = e2m1_value(uint32_t(tid));  // FP4 code values
   if (tid == 0) {
     mbar_init(&ctl->zbar, 1);
     mbar_fence_init();

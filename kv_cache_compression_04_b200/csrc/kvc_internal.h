@@ -247,6 +247,16 @@ __device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
   return e2m1_zero_signs(e2m1x2_raw(lo, hi));
 }
 __device__ __forceinline__ uint32_t e2m1_rne(float p) { return e2m1x2_rne(p, 0.f) & 0xFu; }
+// Two e2m1 codes (the low byte of b: the low nibble first) as their values,
+// by the hardware conversion to f16 (exact: every e2m1 value is an f16).
+__device__ __forceinline__ float2 e2m1x2_to_float2(uint32_t b) {
+  float lo, hi;
+  asm("{\n .reg .b8 t;\n .reg .b16 a, c;\n .reg .b32 h;\n cvt.u8.u32 t, %2;\n"
+      " cvt.rn.f16x2.e2m1x2 h, t;\n mov.b32 {a, c}, h;\n cvt.f32.f16 %0, a;\n"
+      " cvt.f32.f16 %1, c;\n}"
+      : "=f"(lo), "=f"(hi) : "r"(b));
+  return make_float2(lo, hi);
+}
 #endif
 
 // Unsigned 32-bit division by a run-time constant (Granlund and Montgomery,
